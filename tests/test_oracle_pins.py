@@ -1,0 +1,314 @@
+"""Pins of the CPU oracle to things other than itself (CPU only).
+
+Each test ties one oracle function to an independent fact: a library routine
+(numpy's binary16 decoder, numpy.packbits, a numpy matmul of the explicitly
+reconstructed weight), exact rational arithmetic, a closed form, or an
+invariant of the method (linearity across the two paths, rank additivity).
+Shapes are non-square (N != K) so that a transposed operand cannot pass.
+"""
+
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from sub_bit_weight_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- formats
+
+def test_half_decoder_matches_numpy_on_all_codes():
+    codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = codes.view(np.float16).astype(np.float64)
+    got = np.array([oracle.half_to_double(int(c)) for c in codes])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_bf16_decoder_matches_binary32_upper_half_on_all_codes():
+    codes = np.arange(65536, dtype=np.uint32)
+    ref = (codes << np.uint32(16)).view(np.float32).astype(np.float64)
+    got = np.array([oracle.bf16_to_double(int(c)) for c in codes])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_generator_bf16_rounding_matches_torch():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(5)
+    a = np.concatenate([rng.standard_normal(10000).astype(np.float32),
+                        np.float32([0.0, -0.0, 1.0, 1.00390625, 1.01171875, 3.0e38, -1e-40])])
+    ref = torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(synth.f32_to_bf16_bits(a), ref)
+
+
+# ---------------------------------------------------------------- packing
+
+def _golden_pack_cases():
+    cases = []
+    with open(os.path.join(GOLDEN, "pack_vectors.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            head, vals, words = (s.strip() for s in line.split("|"))
+            rows, r = (int(t) for t in head.split())
+            F = np.array([float(v) for v in vals.split()], dtype=np.float32).reshape(rows, r)
+            W = np.array([int(w, 16) for w in words.split()], dtype=np.uint32).reshape(rows, -1)
+            cases.append((F, W))
+    return cases
+
+
+@pytest.mark.parametrize("case", range(len(_golden_pack_cases())))
+def test_pack_golden_vectors(case):
+    F, W = _golden_pack_cases()[case]
+    assert np.array_equal(oracle.pack_signs(F), W)
+
+
+def _special_factor(rng, rows, r):
+    F = rng.standard_normal((rows, r)).astype(np.float32)
+    flat = F.reshape(-1)
+    idx = rng.choice(flat.size, size=min(flat.size, 40), replace=False)
+    specials = np.float32([0.0, -0.0, np.nan, -np.inf, np.inf, -1e-45, 1e-45, -3e-8])
+    flat[idx] = specials[np.arange(idx.size) % specials.size]
+    return F
+
+
+@pytest.mark.parametrize("rows,r", [(1, 1), (7, 31), (5, 32), (9, 33), (64, 80), (3, 184), (2, 800)])
+def test_pack_layout_matches_numpy_packbits(rows, r):
+    rng = np.random.default_rng(rows * 1000 + r)
+    F = _special_factor(rng, rows, r)
+    wpr = (r + 31) // 32
+    neg = np.zeros((rows, wpr * 32), dtype=np.uint8)
+    neg[:, :r] = F < 0
+    ref = np.packbits(neg, axis=1, bitorder="little").view("<u4").reshape(rows, wpr)
+    got = oracle.pack_signs(F)
+    assert got.shape == (rows, wpr) and oracle.packed_words(rows, r) == rows * wpr
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("rows,r", [(4, 1), (6, 45), (3, 96)])
+def test_unpack_inverts_pack(rows, r):
+    rng = np.random.default_rng(r)
+    F = _special_factor(rng, rows, r)
+    s = oracle.unpack_signs(oracle.pack_signs(F), r)
+    assert set(np.unique(s)) <= {-1, 1}
+    assert np.array_equal(s == -1, F < 0)
+
+
+def test_negating_a_factor_complements_its_bits():
+    rng = np.random.default_rng(3)
+    F = rng.standard_normal((11, 70)).astype(np.float32)
+    F[F == 0] = 1.0
+    a, b = oracle.pack_signs(F), oracle.pack_signs(-F)
+    valid = oracle.pack_signs(-np.ones_like(F))
+    assert np.array_equal(a ^ b, valid)
+
+
+# ---------------------------------------------------------------- BPW
+
+def test_bpw_golden():
+    with open(os.path.join(GOLDEN, "bpw.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            if "|" in line:
+                head, frac = line.split("|")
+                N, K, r, P = (int(t) for t in head.split())
+                num, den = (int(t) for t in frac.split())
+                assert oracle.bpw(N, K, r, P) == num / den
+            else:
+                head, claim = line.split("~")
+                N, K, r, P = (int(t) for t in head.split())
+                target, tol = (float(t) for t in claim.split())
+                assert abs(oracle.bpw(N, K, r, P) - target) <= tol * target, (N, K, r)
+
+
+def test_storage_claims_are_consistent_with_bpw():
+    # Llama-2-70B: 138.04 GB of FP16 weights -> 69.02e9 parameters; at 0.1 BPW
+    # the factored weights take under 2 GB (news page, summary table).
+    params = 138.04e9 / 2
+    assert params * 0.1 / 8 < 2e9
+    # Llama-2-13B at 0.1 BPW is under 0.9 GB (notes page, key findings).
+    assert 13e9 * 0.1 / 8 < 0.9e9
+
+
+# ---------------------------------------------------------------- forward
+
+def _layer(seed, N, K, r, npaths=2, tie=False, ones=False, all_plus=False):
+    L = synth.layer_inputs(seed, 0, synth.LayerShape("t", N, K, r), npaths)
+    if tie:
+        L["h"] = [L["h"][0]] * npaths
+        L["g"] = [L["g"][0]] * npaths
+    if ones:
+        one = np.uint16(0x3C00)
+        L["h"] = [np.full(N, one) for _ in range(npaths)]
+        L["g"] = [np.full(K, one) for _ in range(npaths)]
+        L["l"] = [np.full(r, one) for _ in range(npaths)]
+    if all_plus:
+        L["F_U"] = [np.abs(a) for a in L["F_U"]]
+        L["F_V"] = [np.abs(a) for a in L["F_V"]]
+    L["U"] = [oracle.pack_signs(a) for a in L["F_U"]]
+    L["V"] = [oracle.pack_signs(a) for a in L["F_V"]]
+    return L
+
+
+def _f16(b):
+    return np.asarray(b, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def _sign(F):
+    return np.where(F < 0, -1.0, 1.0)
+
+
+def _dense_numpy(L):
+    """W = sum_p diag(h) U diag(l) V^T diag(g), from the generator's factors."""
+    W = np.zeros((L["N"], L["K"]))
+    for p in range(len(L["F_U"])):
+        W += (_f16(L["h"][p])[:, None] * _sign(L["F_U"][p])) @ \
+             (_f16(L["l"][p])[:, None] * _sign(L["F_V"][p]).T) * _f16(L["g"][p])[None, :]
+    return W
+
+
+def _x(seed, M, K):
+    return synth.activations(seed, 99, M, K)
+
+
+def _xf(xb):
+    return synth.bf16_bits_to_f32(xb).astype(np.float64)
+
+
+def _rel(a, b):
+    return np.max(np.abs(a - b)) / np.max(np.abs(b))
+
+
+@pytest.mark.parametrize("N,K,r,M,P", [(48, 80, 5, 3, 2), (96, 40, 33, 2, 2), (33, 70, 16, 1, 1),
+                                       (20, 64, 64, 4, 2)])
+def test_forward_matches_dense_reconstruction(N, K, r, M, P):
+    L = _layer(N + K + r, N, K, r, P)
+    xb = _x(r, M, K)
+    W = _dense_numpy(L)
+    assert _rel(oracle.dense_weight(L), W) <= 1e-13
+    y_ref = _xf(xb) @ W.T
+    assert _rel(oracle.forward(xb, L), y_ref) <= 1e-12
+
+
+def test_forward_exact_rational_single_512():
+    """The 512x512, r=16 workload (M = 1 and 8) against exact rationals."""
+    w = synth.WORKLOADS["single_512"]
+    shape = w.block[0]
+    L = _layer(w.seed, shape.N, shape.K, shape.r)
+    fr = lambda a: [Fraction(float(v)) for v in a]
+    for M in w.Ms:
+        xb = synth.activations(w.seed, 0, M, shape.K)
+        y = oracle.forward(xb, L)
+        sU = [oracle.unpack_signs(u, shape.r) for u in L["U"]]
+        sV = [oracle.unpack_signs(v, shape.r) for v in L["V"]]
+        assert np.array_equal(sU[0] == -1, L["F_U"][0] < 0)
+        h = [fr(_f16(a)) for a in L["h"]]
+        g = [fr(_f16(a)) for a in L["g"]]
+        l = [fr(_f16(a)) for a in L["l"]]
+        worst = 0.0
+        for m in range(M):
+            x = fr(_xf(xb[m]))
+            exact = [Fraction(0)] * shape.N
+            for p in range(2):
+                t = [x[k] * g[p][k] for k in range(shape.K)]
+                zl = []
+                for j in range(shape.r):
+                    col = sV[p][:, j]
+                    z = sum((t[k] if col[k] > 0 else -t[k]) for k in range(shape.K))
+                    zl.append(z * l[p][j])
+                for n in range(shape.N):
+                    row = sU[p][n]
+                    s = sum((zl[j] if row[j] > 0 else -zl[j]) for j in range(shape.r))
+                    exact[n] += h[p][n] * s
+            ex = np.array([float(v) for v in exact])
+            worst = max(worst, np.max(np.abs(y[m] - ex)) / np.max(np.abs(ex)))
+        assert worst <= 1e-13
+
+
+def test_special_case_unit_scales_is_integer_matmul():
+    N, K, r, M = 40, 72, 24, 3
+    L = _layer(11, N, K, r, npaths=2, ones=True)
+    rng = np.random.default_rng(2)
+    xi = rng.integers(-8, 9, size=(M, K))
+    xb = synth.f32_to_bf16_bits(xi.astype(np.float32))
+    ref = np.zeros((M, N), dtype=np.int64)
+    for p in range(2):
+        sV = _sign(L["F_V"][p]).astype(np.int64)
+        sU = _sign(L["F_U"][p]).astype(np.int64)
+        ref += xi @ sV @ sU.T
+    assert np.array_equal(oracle.forward(xb, L), ref.astype(np.float64))
+
+
+def test_special_case_all_plus_signs_closed_form():
+    N, K, r, M = 24, 56, 9, 2
+    L = _layer(12, N, K, r, all_plus=True)
+    xb = _x(3, M, K)
+    x = _xf(xb)
+    ref = sum(_f16(L["h"][p])[None, :] * _f16(L["l"][p]).sum() * (x @ _f16(L["g"][p]))[:, None]
+              for p in range(2))
+    assert _rel(oracle.forward(xb, L), ref) <= 1e-13
+
+
+def test_special_case_rank_one_outer_product():
+    N, K, M = 30, 50, 2
+    L = _layer(13, N, K, 1, npaths=1)
+    xb = _x(4, M, K)
+    x = _xf(xb)
+    u = _sign(L["F_U"][0][:, 0]) * _f16(L["h"][0])
+    v = _sign(L["F_V"][0][:, 0]) * _f16(L["g"][0])
+    ref = _f16(L["l"][0])[0] * np.outer(x @ v, u)
+    assert _rel(oracle.forward(xb, L), ref) <= 1e-13
+
+
+def _one_path(L, p):
+    return {"N": L["N"], "K": L["K"], "r": L["r"], **{k: [L[k][p]] for k in ("U", "V", "h", "g", "l")}}
+
+
+def test_linearity_across_paths():
+    L = _layer(14, 36, 44, 12)
+    xb = _x(5, 3, 44)
+    y = oracle.forward(xb, L)
+    y0 = oracle.forward(xb, _one_path(L, 0))
+    y1 = oracle.forward(xb, _one_path(L, 1))
+    assert _rel(y, y0 + y1) <= 1e-14
+
+
+def test_rank_additivity_with_tied_scales():
+    N, K, r = 28, 52, 7
+    L = _layer(15, N, K, r, tie=True)
+    xb = _x(6, 2, K)
+    cat = {"N": N, "K": K, "r": 2 * r,
+           "U": [oracle.pack_signs(np.concatenate(L["F_U"], axis=1))],
+           "V": [oracle.pack_signs(np.concatenate(L["F_V"], axis=1))],
+           "h": [L["h"][0]], "g": [L["g"][0]], "l": [np.concatenate(L["l"])]}
+    assert _rel(oracle.forward(xb, L), oracle.forward(xb, cat)) <= 1e-13
+
+
+def test_sampled_forward_equals_full_forward():
+    L = _layer(16, 64, 96, 20)
+    xb = _x(7, 5, 96)
+    y = oracle.forward(xb, L)
+    ms, ns = [4, 0, 2], [63, 0, 17, 17]
+    assert np.array_equal(oracle.forward_sampled(xb, L, ms, ns), y[np.ix_(ms, ns)])
+
+
+def test_zero_activations_give_zero_output():
+    L = _layer(17, 16, 24, 3)
+    assert not np.any(oracle.forward(np.zeros((2, 24), dtype=np.uint16), L))
+
+
+def test_generator_sign_blocks_are_consistent():
+    full = synth.sign_factor(1, 2, 0, synth.MAT_U, 50, 70)
+    part = synth.sign_factor(1, 2, 0, synth.MAT_U, 50, 70, row0=13, row1=29)
+    assert np.array_equal(full[13:29], part)
+    assert 0.4 < np.mean(full < 0) < 0.6
