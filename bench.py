@@ -1,0 +1,380 @@
+#!/usr/bin/env python3
+"""Benchmark of the LittleBit compressed-linear forward on B200.
+
+One step = one forward pass of every layer of a synthetic Llama-2-shaped
+stack (both binary contractions, all scalings, both paths) through the C ABI.
+Default workload: the Llama-2-70B-shaped decode stack at ~0.1 BPW (560
+layers, M = 1, 857 MB of packed signs and scales: larger than L2, so every
+step streams from HBM).  The same JSON line carries the Llama-2-13B-shaped
+prefill stack (M = 2048, tensor-core bound) as "prefill".
+
+Metric: algorithmic bytes (packed signs + binary16 scales + x + y) per second
+for decode, algorithmic FLOPs (2*M*2r*(K+N) per layer) per second for prefill.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+        python bench.py --impl reference ...   (the CPU oracle, timed as is)
+Multi-GPU: one process per GPU (torchrun); every rank runs the whole stack
+(independent replicas, weak scaling); time = max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sub_bit_weight_b200 import synth  # noqa: E402
+
+METRIC = "LittleBit linear decode GB/s & prefill TFLOP/s, % of B200 roofline"
+DECODE_DEFAULT = "llama2_70b_0.1"
+PREFILL_DEFAULT = "llama2_13b_0.3_prefill"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+# ----------------------------------------------------------------- algorithmic work
+
+def layer_bytes(s: synth.LayerShape, M: int, npaths: int = 2):
+    """(contraction-1 bytes, contraction-2 bytes) of one layer: signs, scales, x, y."""
+    k1 = npaths * (s.K * s.r / 8 + 2 * s.K + 2 * s.r) + 2 * M * s.K
+    k2 = npaths * (s.N * s.r / 8 + 2 * s.N) + 4 * M * s.N
+    return k1, k2
+
+
+def layer_flops(s: synth.LayerShape, M: int, npaths: int = 2):
+    return 2.0 * M * npaths * s.r * (s.K + s.N)
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.period = period
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report that
+            self.nv = None
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.nv:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------- CPU oracle baseline
+
+def oracle_sample(w: synth.Workload, M: int, budget_s: float, max_layers: int | None = None):
+    """Time the oracle (as it stands) on the first layers of the stack until the budget is used."""
+    import oracle
+    shapes = [s for _, s in w.layers()]
+    done_bytes = done_flops = 0.0
+    n = 0
+    elapsed = 0.0
+    pools = {}
+    for idx, s in enumerate(shapes):
+        inp = synth.layer_inputs(w.seed, idx, s)
+        inp["U"] = [oracle.pack_signs(F) for F in inp.pop("F_U")]
+        inp["V"] = [oracle.pack_signs(F) for F in inp.pop("F_V")]
+        xb = synth.layer_activations(w, idx, M, s.K, pools)
+        rows = M
+        if w.pool_rows:             # prefill: a bounded number of activation rows
+            rows = max(1, min(M, 4))
+            xb = xb[:rows]
+        t0 = time.perf_counter()
+        oracle.forward(np.ascontiguousarray(xb), inp)
+        elapsed += time.perf_counter() - t0
+        b1, b2 = layer_bytes(s, rows)
+        done_bytes += b1 + b2
+        done_flops += layer_flops(s, rows)
+        n += 1
+        if elapsed >= budget_s or (max_layers and n >= max_layers):
+            break
+    return {"seconds": elapsed, "layers": n, "bytes": done_bytes, "flops": done_flops,
+            "rows": rows if w.pool_rows else M}
+
+
+# ----------------------------------------------------------------- GPU runs
+
+def run_gpu(w: synth.Workload, M: int, steps: int, warmup: int, dist, dev, want_e2e=True):
+    import torch
+    from sub_bit_weight_b200 import lib, stacks
+
+    layers, shapes = stacks.build_workload(w, device=dev)
+    S = lib.lb_stack_create(layers)
+    # contiguous x / y so that the end-to-end run moves them with one copy each way
+    xsz = [M * s.K for s in shapes]
+    ysz = [M * s.N for s in shapes]
+    x_all = torch.empty(sum(xsz), dtype=torch.bfloat16, device=dev)
+    y_all = torch.empty(sum(ysz), dtype=torch.float32, device=dev)
+    xs_src, _ = stacks.workload_activations(w, shapes, M, device=dev)
+    xs, ys = [], []
+    ox = oy = 0
+    for s, a, b, src in zip(shapes, xsz, ysz, xs_src):
+        xs.append(x_all[ox:ox + a].view(M, s.K))
+        xs[-1].copy_(src)
+        ys.append(y_all[oy:oy + b].view(M, s.N))
+        ox += a
+        oy += b
+    del xs_src
+    io = lib.StackIO(S, xs, ys)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(warmup):
+        lib.lb_stack_forward(S, io=io)
+    torch.cuda.synchronize()
+
+    nlaunch_per_step = None
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for trio in ev:          # torch creates the CUDA event on first record
+        for e in trio:
+            e.record(stream)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        start.record(stream)
+        for k in range(steps):
+            lib.lb_profile_events(ev[k])
+            lib.lb_stack_forward(S, io=io)
+            if nlaunch_per_step is None:
+                nlaunch_per_step = lib.lb_last_launch_count()
+        stop.record(stream)
+        torch.cuda.synchronize()
+    lib.lb_profile_events([])
+    if dist:
+        dist.barrier()
+    total_ms = start.elapsed_time(stop)
+    per_launch = None
+    if nlaunch_per_step == 2:
+        k1 = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+        k2 = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+        per_launch = (k1, k2)
+
+    e2e = None
+    if want_e2e:
+        hx = torch.empty(x_all.numel(), dtype=torch.bfloat16, pin_memory=True)
+        hx.copy_(x_all)
+        hy = torch.empty(y_all.numel(), dtype=torch.float32, pin_memory=True)
+        e_steps = max(3, min(steps, 200))
+        for _ in range(2):
+            x_all.copy_(hx, non_blocking=True)
+            lib.lb_stack_forward(S, io=io)
+            hy.copy_(y_all, non_blocking=True)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e_steps):
+            x_all.copy_(hx, non_blocking=True)
+            lib.lb_stack_forward(S, io=io)
+            hy.copy_(y_all, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e = {"ms": a.elapsed_time(b) / e_steps, "h2d": x_all.numel() * 2, "d2h": y_all.numel() * 4,
+               "steps": e_steps}
+    out = {"total_ms": total_ms, "per_launch": per_launch, "launches": nlaunch_per_step * steps,
+           "clocks": clk.summary(), "e2e": e2e, "shapes": shapes}
+    del S, layers, io
+    torch.cuda.synchronize()
+    return out
+
+
+def max_over_ranks(v: float, dist):
+    if not dist:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DECODE_DEFAULT, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--M", type=int, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--prefill", default=PREFILL_DEFAULT, help="prefill workload for the 'prefill' object ('' = skip)")
+    ap.add_argument("--prefill-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    w = synth.WORKLOADS[args.workload]
+    M = args.M if args.M is not None else w.Ms[0]
+    pk = peaks()
+
+    if args.impl == "reference":
+        return reference_arm(args, w, M, world, rank, pk)
+
+    import torch
+    dist = None
+    if world > 1:
+        import torch.distributed as tdist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        import datetime
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    res = run_gpu(w, M, args.steps, args.warmup, dist, dev)
+    total_ms = max_over_ranks(res["total_ms"], dist)
+    shapes = res["shapes"]
+    k1b = sum(layer_bytes(s, M)[0] for s in shapes)
+    k2b = sum(layer_bytes(s, M)[1] for s in shapes)
+    step_bytes = k1b + k2b
+    ms_step = total_ms / args.steps
+    value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
+
+    roof = None
+    if res["per_launch"]:
+        k1ms, k2ms = res["per_launch"]
+        dom = 1 if k2ms >= k1ms else 0
+        dom_bytes, dom_ms = (k2b, k2ms) if dom else (k1b, k1ms)
+        ach = dom_bytes / (dom_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": "contraction2_kernel" if dom else "contraction1_kernel",
+                "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / pk["hbm_gbs"], 4), "peak_src": pk["src"],
+                "traffic": None,
+                "per_kernel_ms": {"contraction1_kernel": round(k1ms, 5), "contraction2_kernel": round(k2ms, 5)},
+                "per_kernel_bytes": {"contraction1_kernel": k1b, "contraction2_kernel": k2b}}
+    e2e = None
+    if res["e2e"]:
+        e_ms = max_over_ranks(res["e2e"]["ms"], dist)
+        e2e = {"value": round(world * step_bytes / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": res["e2e"]["h2d"], "d2h_bytes_per_step": res["e2e"]["d2h"],
+               "ms_per_step": round(e_ms, 4)}
+
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 in, int8 tensor-core MMA (u8 signs x s8 fixed-point digits, s32 acc), fp32 out",
+            "data": "synthetic (seeded; signs Bernoulli(0.5), scales lognormal(-3,0.5) fp16, x N(0,1) bf16)",
+            "config": {"workload": f"{w.key}: {w.title}", "layers": len(shapes), "M": M,
+                       "bytes_per_step": step_bytes,
+                       "l2": "inputs larger than L2 (stack streams from HBM every step)"
+                             if step_bytes > 126e6 else "stack fits in L2 (effective GB/s)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roof, "gpu_launches": res["launches"], "clocks": res["clocks"], "e2e": e2e}
+
+    if args.prefill and world == 1:
+        pw = synth.WORKLOADS[args.prefill]
+        pM = pw.Ms[0]
+        pres = run_gpu(pw, pM, args.prefill_steps, 3, dist, dev, want_e2e=False)
+        pflops = sum(layer_flops(s, pM) for s in pres["shapes"])
+        pms = pres["total_ms"] / args.prefill_steps
+        tf = pflops / (pms * 1e-3) / 1e12
+        line["prefill"] = {"workload": f"{pw.key}: {pw.title}", "M": pM, "layers": len(pres["shapes"]),
+                           "value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(pms, 3),
+                           "steps": args.prefill_steps, "gpu_launches": pres["launches"],
+                           "roofline": {"bound": "tensor", "achieved": round(tf, 2),
+                                        "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                                        "frac": round(tf / pk["bf16_tflops_sustained"], 4),
+                                        "peak_src": pk["src"] + " bf16 sustained (dense 16-bit tensor peak)",
+                                        "traffic": None},
+                           "clocks": pres["clocks"]}
+
+    if rank == 0 and args.cpu_seconds > 0:
+        cs = oracle_sample(w, M, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(cs["bytes"] / cs["seconds"] / 1e9, 5), "unit": "GB/s",
+                                "cores": 1, "kind": "oracle",
+                                "sample": f"first {cs['layers']} layers of the stack, M={M}, "
+                                          f"{cs['seconds']:.1f} s single-threaded float64 C"}
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+
+
+def reference_arm(args, w, M, world, rank, pk):
+    """The CPU oracle timed as it stands, on the same workload/metric (rank 0 only)."""
+    if rank != 0:
+        return
+    per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, M, per_step / 4, max_layers=1)
+    t_bytes = t_sec = 0.0
+    layers = 0
+    for _ in range(args.steps):
+        cs = oracle_sample(w, M, per_step)
+        t_bytes += cs["bytes"]
+        t_sec += cs["seconds"]
+        layers += cs["layers"]
+    v = t_bytes / t_sec / 1e9
+    line = {"metric": METRIC, "value": round(v, 5), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * t_sec / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"{w.key}: {w.title}", "M": M},
+            "cpu_baseline": {"value": round(v, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{layers} layers over {args.steps} steps (first layers of the stack), "
+                                       f"single-threaded float64 C"},
+            "e2e": {"value": round(v, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

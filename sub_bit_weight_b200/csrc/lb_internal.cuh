@@ -1,0 +1,153 @@
+// Internal declarations of the LittleBit CUDA library (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+#include <vector>
+
+#include "littlebit.h"
+
+namespace lb {
+
+// ---------------------------------------------------------------------------
+// Decode-path tiling (the fused small-batch kernels).
+//
+// Both binary contractions run on integer tensor cores (mma.sync m16n8k32,
+// A = unsigned 8-bit, B = signed 8-bit, s32 accumulate).  The weight is the A
+// operand ("row" = an output of the contraction, "k" = the contracted index),
+// the activations are the B operand as two balanced base-256 digits of a
+// 16-bit fixed-point value (column = 2*m + digit).
+//
+// A "unit" is 64 rows x 32 k of one weight matrix, stored as 256 contiguous
+// bytes: lane L (g = L >> 2, t = L & 3) owns the uint2 {w0, w1}.  Bit i of
+// byte b of word q is the sign bit (1 = -1) of
+//     row = 16 * (i & 3) + g + 8 * (i >> 2),   k = 4 * t + b + 16 * q.
+// Masking a word with (0x01010101 << i) gives four u8 A elements equal to
+// 2^i times the bit, in exactly the register slots mma.sync expects, so a
+// row-block's MMA costs four LOP3s and no shifts:
+//     row-block rb:  a0 = w0 & m(rb)   a1 = w0 & m(rb + 4)
+//                    a2 = w1 & m(rb)   a3 = w1 & m(rb + 4)
+// Rows g of row-block rb then carry the factor 2^rb and rows g + 8 the factor
+// 2^(rb+4); both are divided out exactly after accumulation.
+// ---------------------------------------------------------------------------
+constexpr int kRowsPerBlock = 16;
+constexpr int kRowsPerGroup = 64;
+constexpr int kKPerBlock = 32;
+constexpr int kP1ChunkKB = 32;          // k-blocks per contraction-1 work item (1024 inputs)
+constexpr int kP2ItemGroups = 8;        // row groups per contraction-2 work item (512 outputs)
+constexpr int kDecodeThreads = 128;     // 4 warps
+constexpr int kMaxDecodeM = LB_DECODE_MAX_M;
+constexpr int kMaxNT = (kMaxDecodeM + 3) / 4;   // n-tiles of 4 activation rows
+constexpr int kIoBatch = 1024;          // layers per launch (pointer tables ride in kernel params)
+
+static inline int round_up(int a, int b) { return (a + b - 1) / b * b; }
+static inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Per-layer descriptor read by the kernels (device copy lives in a plan).
+struct LayerDev {
+    int N, K, r, npaths;
+    int r16, r32;       // rank rounded up to 16 (contraction-1 rows) / 32 (contraction-2 k)
+    int R1, RG1;        // contraction-1 rows (both paths, padded to 64) and row groups
+    int K32, KB1;       // inputs rounded to 32, contraction-1 k-blocks
+    int N64, RG2;       // outputs rounded to 64, contraction-2 row groups
+    int KB2;            // contraction-2 k-blocks (npaths * r32 / 32)
+    int nkc;            // contraction-1 work items (k chunks)
+    const uint2 *vt;    // V tiles  [RG1][KB1][32]
+    const uint2 *ut;    // U tiles  [RG2][KB2][32]
+    const __half *g;    // [npaths][K32], zero padded
+    const __half *h;    // [npaths][N64], zero padded
+    const __half *l;    // [npaths][r16], zero padded
+    // scratch (owned by the plan that holds this descriptor)
+    int *partT;         // [nkc][R1][16]   integer partial sums of contraction 1
+    int2 *pmeta;        // [nkc][2][16]    (exponent, digit sum) of each chunk
+    float *zl;          // [R1][16]        latent vector after l
+    uint2 *zfrag;       // [KB2][kMaxNT][32] B fragments of contraction 2
+    int2 *zmeta;        // [2][16]         (exponent, digit sum) of zl
+    unsigned *counter;  // chunks of contraction 1 finished (self-resetting)
+};
+
+struct P1Item { int layer, kc; };
+struct P2Item { int layer, rg0, rg1, pad; };
+
+struct IoPtrs {
+    const uint16_t *x[kIoBatch];
+    float *y[kIoBatch];
+};
+
+// Sentinel exponent marking a non-finite activation block.
+constexpr int kNanExp = -0x40000000;
+
+// Host-side record of a layer (what lb_layer points to).
+}  // namespace lb
+
+struct lb_layer {
+    lb::LayerDev d;            // descriptor with pointers into `weights`
+    void *weights = nullptr;   // one allocation: tiles + scales
+    size_t weight_bytes = 0;
+    struct lb_stack *self = nullptr;   // single-layer plan (owns scratch)
+};
+
+namespace lb {
+
+// A plan: descriptors + work items + scratch for a list of layers.
+struct Plan {
+    int n = 0;
+    std::vector<LayerDev> host;     // descriptors (scratch pointers filled in)
+    LayerDev *dev = nullptr;        // device copy of `host`
+    P1Item *p1 = nullptr;           // device work items
+    P2Item *p2 = nullptr;
+    std::vector<int> p1_start, p2_start;   // per IO batch: first item index
+    int n_p1 = 0, n_p2 = 0;
+    void *scratch = nullptr;
+    size_t scratch_bytes = 0;
+};
+
+cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream_t s);
+void plan_free(Plan &P);
+
+lb_status decode_forward(const Plan &P, const uint16_t *const *xs, float *const *ys, int M,
+                         cudaStream_t s, int *launches);
+
+lb_status status_from(cudaError_t e);
+void set_launch_count(int n);
+// Timing hook: record the registered event `i` (if any) on stream s.
+void profile_mark(int i, cudaStream_t s);
+
+}  // namespace lb
+
+struct lb_stack {
+    lb::Plan plan;
+    std::vector<const lb_layer *> layers;
+};
+
+// ---------------------------------------------------------------------------
+// Small device helpers
+// ---------------------------------------------------------------------------
+namespace lb {
+
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Streamed once: read-only path, no L1 allocation.
+__device__ __forceinline__ uint2 ld_stream_u2(const uint2 *p)
+{
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];\n"
+                 : "=r"(v.x), "=r"(v.y)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b)
+{
+    return __uint_as_float(((uint32_t)b) << 16);
+}
+
+}  // namespace lb

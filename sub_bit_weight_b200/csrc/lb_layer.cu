@@ -1,0 +1,369 @@
+// Layer objects, their private weight layouts, execution plans and stacks.
+//
+// A layer is built from the canonical packed signs (one bit per sign, sign(0)
+// = +1) and binary16 scales of its two paths (LittleBit notes page,
+// "Multi-scale compensation" and "Residual compensation").  It re-tiles the
+// signs into the layouts its kernels stream (see lb_internal.cuh) and keeps
+// the scales zero-padded, so padded rank slots and rows contribute nothing.
+
+#include <algorithm>
+#include <cstring>
+#include <new>
+
+#include "lb_internal.cuh"
+
+namespace lb {
+
+__device__ __forceinline__ uint32_t canon_bit(const uint32_t *P, int wpr, int64_t row, int col)
+{
+    return (__ldg(P + row * wpr + (col >> 5)) >> (col & 31)) & 1u;
+}
+
+// Contraction-1 tiles: rows are latent indices of both paths (path p owns
+// rows [p*r16, p*r16 + r16)), k runs over the K inputs.  Bit = V_sign[k][j] < 0.
+__global__ void build_vtiles_kernel(uint2 *__restrict__ vt, int RG1, int KB1, int r, int r16, int K,
+                                    int npaths, const uint32_t *__restrict__ V0,
+                                    const uint32_t *__restrict__ V1)
+{
+    const int wpr = (r + 31) / 32;
+    const int64_t total = (int64_t)RG1 * KB1 * 32;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int lane = (int)(idx & 31);
+        const int64_t u = idx >> 5;
+        const int kb = (int)(u % KB1);
+        const int rg = (int)(u / KB1);
+        const int g = lane >> 2, t = lane & 3;
+        uint32_t w[2] = {0u, 0u};
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int row = rg * kRowsPerGroup + 16 * (i & 3) + g + 8 * (i >> 2);
+                    const int k = kb * kKPerBlock + 4 * t + b + 16 * q;
+                    const int p = row / r16;
+                    const int j = row - p * r16;
+                    if (p < npaths && j < r && k < K)
+                        w[q] |= canon_bit(p ? V1 : V0, wpr, k, j) << (8 * b + i);
+                }
+        vt[idx] = make_uint2(w[0], w[1]);
+    }
+}
+
+// Contraction-2 tiles: rows are the N outputs, k runs over the latent indices
+// of both paths (path p owns k in [p*r32, p*r32 + r32)).  Bit = U_sign[n][j] < 0.
+__global__ void build_utiles_kernel(uint2 *__restrict__ ut, int RG2, int KB2, int r, int r32, int N,
+                                    int npaths, const uint32_t *__restrict__ U0,
+                                    const uint32_t *__restrict__ U1)
+{
+    const int wpr = (r + 31) / 32;
+    const int64_t total = (int64_t)RG2 * KB2 * 32;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int lane = (int)(idx & 31);
+        const int64_t u = idx >> 5;
+        const int kb = (int)(u % KB2);
+        const int rg = (int)(u / KB2);
+        const int g = lane >> 2, t = lane & 3;
+        uint32_t w[2] = {0u, 0u};
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int n = rg * kRowsPerGroup + 16 * (i & 3) + g + 8 * (i >> 2);
+                    const int jj = kb * kKPerBlock + 4 * t + b + 16 * q;
+                    const int p = jj / r32;
+                    const int j = jj - p * r32;
+                    if (p < npaths && j < r && n < N)
+                        w[q] |= canon_bit(p ? U1 : U0, wpr, n, j) << (8 * b + i);
+                }
+        ut[idx] = make_uint2(w[0], w[1]);
+    }
+}
+
+// dst[p][0..npad) = src_p[0..n) followed by zeros.
+__global__ void pad_copy_kernel(uint16_t *__restrict__ dst, const uint16_t *__restrict__ s0,
+                                const uint16_t *__restrict__ s1, int npaths, int n, int npad)
+{
+    const int64_t total = (int64_t)npaths * npad;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int p = (int)(idx / npad);
+        const int i = (int)(idx - (int64_t)p * npad);
+        dst[idx] = (i < n) ? (p ? s1 : s0)[i] : (uint16_t)0;
+    }
+}
+
+static size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+static int grid_for(int64_t work, int threads)
+{
+    int64_t b = (work + threads - 1) / threads;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(b, 148 * 32));
+}
+
+// ---------------------------------------------------------------- plans
+
+void plan_free(Plan &P)
+{
+    if (P.dev) cudaFree(P.dev);
+    if (P.p1) cudaFree(P.p1);
+    if (P.p2) cudaFree(P.p2);
+    if (P.scratch) cudaFree(P.scratch);
+    P = Plan();
+}
+
+cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream_t s)
+{
+    P.n = n;
+    P.host.resize(n);
+    // scratch layout
+    std::vector<size_t> off(n);
+    size_t total = 0;
+    for (int i = 0; i < n; ++i) {
+        const LayerDev &d = layers[i]->d;
+        off[i] = total;
+        total += align256((size_t)d.nkc * d.R1 * 16 * sizeof(int));
+        total += align256((size_t)d.nkc * 2 * 16 * sizeof(int2));
+        total += align256((size_t)d.R1 * 16 * sizeof(float));
+        total += align256((size_t)d.KB2 * kMaxNT * 32 * sizeof(uint2));
+        total += align256((size_t)2 * 16 * sizeof(int2));
+        total += align256(sizeof(unsigned));
+    }
+    cudaError_t e = cudaMalloc(&P.scratch, std::max<size_t>(total, 256));
+    if (e != cudaSuccess) return e;
+    P.scratch_bytes = total;
+    e = cudaMemsetAsync(P.scratch, 0, total, s);
+    if (e != cudaSuccess) return e;
+    char *base = (char *)P.scratch;
+    for (int i = 0; i < n; ++i) {
+        LayerDev d = layers[i]->d;
+        char *c = base + off[i];
+        d.partT = (int *)c;      c += align256((size_t)d.nkc * d.R1 * 16 * sizeof(int));
+        d.pmeta = (int2 *)c;     c += align256((size_t)d.nkc * 2 * 16 * sizeof(int2));
+        d.zl = (float *)c;       c += align256((size_t)d.R1 * 16 * sizeof(float));
+        d.zfrag = (uint2 *)c;    c += align256((size_t)d.KB2 * kMaxNT * 32 * sizeof(uint2));
+        d.zmeta = (int2 *)c;     c += align256((size_t)2 * 16 * sizeof(int2));
+        d.counter = (unsigned *)c;
+        P.host[i] = d;
+    }
+    // work items, layer-major; one IO batch per kIoBatch layers
+    std::vector<P1Item> p1;
+    std::vector<P2Item> p2;
+    for (int i = 0; i < n; ++i) {
+        if (i % kIoBatch == 0) {
+            P.p1_start.push_back((int)p1.size());
+            P.p2_start.push_back((int)p2.size());
+        }
+        const LayerDev &d = P.host[i];
+        for (int kc = 0; kc < d.nkc; ++kc) p1.push_back({i, kc});
+        for (int rg = 0; rg < d.RG2; rg += kP2ItemGroups)
+            p2.push_back({i, rg, std::min(rg + kP2ItemGroups, d.RG2), 0});
+    }
+    P.p1_start.push_back((int)p1.size());
+    P.p2_start.push_back((int)p2.size());
+    P.n_p1 = (int)p1.size();
+    P.n_p2 = (int)p2.size();
+    if ((e = cudaMalloc(&P.dev, sizeof(LayerDev) * n)) != cudaSuccess) return e;
+    if ((e = cudaMalloc(&P.p1, sizeof(P1Item) * std::max(1, P.n_p1))) != cudaSuccess) return e;
+    if ((e = cudaMalloc(&P.p2, sizeof(P2Item) * std::max(1, P.n_p2))) != cudaSuccess) return e;
+    // synchronous copies from pageable memory: the host vectors die with this call
+    if ((e = cudaMemcpy(P.dev, P.host.data(), sizeof(LayerDev) * n, cudaMemcpyHostToDevice)) != cudaSuccess)
+        return e;
+    if ((e = cudaMemcpy(P.p1, p1.data(), sizeof(P1Item) * P.n_p1, cudaMemcpyHostToDevice)) != cudaSuccess)
+        return e;
+    if ((e = cudaMemcpy(P.p2, p2.data(), sizeof(P2Item) * P.n_p2, cudaMemcpyHostToDevice)) != cudaSuccess)
+        return e;
+    return cudaSuccess;
+}
+
+}  // namespace lb
+
+using namespace lb;
+
+extern "C" {
+
+lb_status lb_layer_create(lb_layer **out, int N, int K, int r, int npaths, const uint32_t *const *U,
+                          const uint32_t *const *V, const uint16_t *const *h,
+                          const uint16_t *const *g, const uint16_t *const *l, void *stream)
+{
+    set_launch_count(0);
+    if (!out) return LB_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (N < 1 || K < 1 || r < 1 || r > LB_MAX_RANK) return LB_ERR_INVALID_ARG;
+    if (npaths != 1 && npaths != 2) return LB_ERR_UNSUPPORTED;
+    if (!U || !V || !h || !g || !l) return LB_ERR_INVALID_ARG;
+    for (int p = 0; p < npaths; ++p)
+        if (!U[p] || !V[p] || !h[p] || !g[p] || !l[p]) return LB_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+
+    lb_layer *L = new (std::nothrow) lb_layer();
+    if (!L) return LB_ERR_OOM;
+    LayerDev &d = L->d;
+    std::memset(&d, 0, sizeof(d));
+    d.N = N; d.K = K; d.r = r; d.npaths = npaths;
+    d.r16 = round_up(r, 16);
+    d.r32 = round_up(r, 32);
+    d.R1 = round_up(npaths * d.r16, kRowsPerGroup);
+    d.RG1 = d.R1 / kRowsPerGroup;
+    d.K32 = round_up(K, kKPerBlock);
+    d.KB1 = d.K32 / kKPerBlock;
+    d.N64 = round_up(N, kRowsPerGroup);
+    d.RG2 = d.N64 / kRowsPerGroup;
+    d.KB2 = npaths * d.r32 / kKPerBlock;
+    d.nkc = ceil_div(d.KB1, kP1ChunkKB);
+
+    const size_t b_vt = align256((size_t)d.RG1 * d.KB1 * 32 * sizeof(uint2));
+    const size_t b_ut = align256((size_t)d.RG2 * d.KB2 * 32 * sizeof(uint2));
+    const size_t b_g = align256((size_t)npaths * d.K32 * 2);
+    const size_t b_h = align256((size_t)npaths * d.N64 * 2);
+    const size_t b_l = align256((size_t)npaths * d.r16 * 2);
+    L->weight_bytes = b_vt + b_ut + b_g + b_h + b_l;
+    cudaError_t e = cudaMalloc(&L->weights, L->weight_bytes);
+    if (e != cudaSuccess) {
+        delete L;
+        return status_from(e);
+    }
+    char *c = (char *)L->weights;
+    d.vt = (const uint2 *)c;   c += b_vt;
+    d.ut = (const uint2 *)c;   c += b_ut;
+    d.g = (const __half *)c;   c += b_g;
+    d.h = (const __half *)c;   c += b_h;
+    d.l = (const __half *)c;
+
+    const int T = 256;
+    const uint32_t *V1 = npaths > 1 ? V[1] : V[0];
+    const uint32_t *U1 = npaths > 1 ? U[1] : U[0];
+    int launches = 0;
+    build_vtiles_kernel<<<grid_for((int64_t)d.RG1 * d.KB1 * 32, T), T, 0, s>>>(
+        (uint2 *)d.vt, d.RG1, d.KB1, r, d.r16, K, npaths, V[0], V1);
+    build_utiles_kernel<<<grid_for((int64_t)d.RG2 * d.KB2 * 32, T), T, 0, s>>>(
+        (uint2 *)d.ut, d.RG2, d.KB2, r, d.r32, N, npaths, U[0], U1);
+    pad_copy_kernel<<<grid_for((int64_t)npaths * d.K32, T), T, 0, s>>>(
+        (uint16_t *)d.g, g[0], npaths > 1 ? g[1] : g[0], npaths, K, d.K32);
+    pad_copy_kernel<<<grid_for((int64_t)npaths * d.N64, T), T, 0, s>>>(
+        (uint16_t *)d.h, h[0], npaths > 1 ? h[1] : h[0], npaths, N, d.N64);
+    pad_copy_kernel<<<grid_for((int64_t)npaths * d.r16, T), T, 0, s>>>(
+        (uint16_t *)d.l, l[0], npaths > 1 ? l[1] : l[0], npaths, r, d.r16);
+    launches = 5;
+    e = cudaGetLastError();
+    if (e == cudaSuccess) {
+        lb_stack *S = new (std::nothrow) lb_stack();
+        if (!S) {
+            e = cudaErrorMemoryAllocation;
+        } else {
+            S->layers.push_back(L);
+            const lb_layer *one = L;
+            e = plan_build(S->plan, &one, 1, s);
+            L->self = S;
+        }
+    }
+    if (e != cudaSuccess) {
+        lb_layer_destroy(L);
+        return status_from(e);
+    }
+    set_launch_count(launches);
+    *out = L;
+    return LB_OK;
+}
+
+void lb_layer_destroy(lb_layer *L)
+{
+    if (!L) return;
+    cudaDeviceSynchronize();
+    if (L->self) {
+        plan_free(L->self->plan);
+        delete L->self;
+    }
+    if (L->weights) cudaFree(L->weights);
+    delete L;
+}
+
+lb_status lb_layer_shape(const lb_layer *L, int *N, int *K, int *r, int *npaths)
+{
+    if (!L) return LB_ERR_INVALID_ARG;
+    if (N) *N = L->d.N;
+    if (K) *K = L->d.K;
+    if (r) *r = L->d.r;
+    if (npaths) *npaths = L->d.npaths;
+    return LB_OK;
+}
+
+double lb_layer_bpw(const lb_layer *L)
+{
+    if (!L) return 0.0;
+    const double N = L->d.N, K = L->d.K, r = L->d.r;
+    return L->d.npaths * (r * (N + K) + 16.0 * (N + K + r)) / (N * K);
+}
+
+size_t lb_layer_device_bytes(const lb_layer *L)
+{
+    if (!L) return 0;
+    size_t b = L->weight_bytes;
+    if (L->self) b += L->self->plan.scratch_bytes;
+    return b;
+}
+
+lb_status lb_linear_forward(const uint16_t *x, int M, const lb_layer *L, float *y, void *stream)
+{
+    set_launch_count(0);
+    if (!L || M < 0) return LB_ERR_INVALID_ARG;
+    if (M == 0) return LB_OK;
+    if (!x || !y || ((uintptr_t)x & 15) || ((uintptr_t)y & 15)) return LB_ERR_INVALID_ARG;
+    const uint16_t *xs[1] = {x};
+    float *ys[1] = {y};
+    int launches = 0;
+    lb_status st = decode_forward(L->self->plan, xs, ys, M, (cudaStream_t)stream, &launches);
+    set_launch_count(launches);
+    return st;
+}
+
+lb_status lb_stack_create(lb_stack **out, const lb_layer *const *layers, int n, void *stream)
+{
+    set_launch_count(0);
+    if (!out) return LB_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!layers || n < 1 || n > LB_STACK_MAX_LAYERS) return LB_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i)
+        if (!layers[i]) return LB_ERR_INVALID_ARG;
+    lb_stack *S = new (std::nothrow) lb_stack();
+    if (!S) return LB_ERR_OOM;
+    S->layers.assign(layers, layers + n);
+    cudaError_t e = plan_build(S->plan, layers, n, (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        plan_free(S->plan);
+        delete S;
+        return status_from(e);
+    }
+    *out = S;
+    return LB_OK;
+}
+
+void lb_stack_destroy(lb_stack *S)
+{
+    if (!S) return;
+    cudaDeviceSynchronize();
+    plan_free(S->plan);
+    delete S;
+}
+
+lb_status lb_stack_forward(lb_stack *S, const uint16_t *const *xs, float *const *ys, int M, void *stream)
+{
+    set_launch_count(0);
+    if (!S || M < 0) return LB_ERR_INVALID_ARG;
+    if (M == 0) return LB_OK;
+    if (!xs || !ys) return LB_ERR_INVALID_ARG;
+    for (int i = 0; i < S->plan.n; ++i)
+        if (!xs[i] || !ys[i] || ((uintptr_t)xs[i] & 15) || ((uintptr_t)ys[i] & 15))
+            return LB_ERR_INVALID_ARG;
+    int launches = 0;
+    lb_status st = decode_forward(S->plan, xs, ys, M, (cudaStream_t)stream, &launches);
+    set_launch_count(launches);
+    return st;
+}
+
+}  // extern "C"

@@ -1,0 +1,233 @@
+"""Thin Python binding of the C ABI in ``include/littlebit.h``.
+
+Argument marshalling only: every step of the forward pass runs in the CUDA
+kernels of ``liblittlebit.so``.  PyTorch supplies device memory and streams.
+Importing this module loads the library and raises ImportError when it has not
+been built (``python -m sub_bit_weight_b200.build``); there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblittlebit.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sub_bit_weight_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+LB_OK, LB_ERR_INVALID_ARG, LB_ERR_UNSUPPORTED, LB_ERR_OOM, LB_ERR_CUDA, LB_ERR_TIMEOUT = range(6)
+LB_DECODE_MAX_M = 16
+LB_MAX_RANK = 2048
+LB_STACK_MAX_LAYERS = 4096
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_i64 = ctypes.c_int64
+_st = ctypes.c_int
+
+
+def _sig(name, res, args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = args
+    return f
+
+
+_sig("lb_status_string", ctypes.c_char_p, [_st])
+_sig("lb_packed_words", ctypes.c_size_t, [_i64, _i])
+_sig("lb_pack_signs", _st, [_vp, _i64, _i, _vp, _vp])
+_sig("lb_layer_create", _st, [ctypes.POINTER(_vp), _i, _i, _i, _i] + [ctypes.POINTER(_vp)] * 5 + [_vp])
+_sig("lb_layer_destroy", None, [_vp])
+_sig("lb_layer_shape", _st, [_vp] + [ctypes.POINTER(_i)] * 4)
+_sig("lb_layer_bpw", ctypes.c_double, [_vp])
+_sig("lb_layer_device_bytes", ctypes.c_size_t, [_vp])
+_sig("lb_linear_forward", _st, [_vp, _i, _vp, _vp, _vp])
+_sig("lb_stack_create", _st, [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp])
+_sig("lb_stack_destroy", None, [_vp])
+_sig("lb_stack_forward", _st, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp])
+_sig("lb_last_launch_count", _i, [])
+_sig("lb_profile_events", _st, [ctypes.POINTER(_vp), _i])
+
+
+class LittleBitError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lb_status_string(status)}")
+
+
+def lb_status_string(status: int) -> str:
+    return _lib.lb_status_string(status).decode()
+
+
+def _check(status: int, where: str):
+    if status != LB_OK:
+        raise LittleBitError(status, where)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def lb_packed_words(rows: int, r: int) -> int:
+    return int(_lib.lb_packed_words(rows, r))
+
+
+def lb_last_launch_count() -> int:
+    return int(_lib.lb_last_launch_count())
+
+
+def lb_profile_events(events) -> None:
+    """Register torch.cuda.Event objects (timing enabled) for the next forward calls; [] clears."""
+    n = len(events)
+    arr = (_vp * max(1, n))(*[e.cuda_event for e in events]) if n else None
+    _check(_lib.lb_profile_events(arr, n), "lb_profile_events")
+
+
+def lb_pack_signs(F: torch.Tensor, packed: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """fp32 factor [rows, r] (CUDA) -> canonical packed signs, int32 [rows, ceil(r/32)] (bit patterns)."""
+    if F.dim() != 2:
+        raise ValueError("F must be 2-D [rows, r]")
+    rows, r = F.shape
+    if packed is None:
+        packed = torch.empty((rows, (r + 31) // 32), dtype=torch.int32, device=F.device)
+    _check(_lib.lb_pack_signs(_dev(F, torch.float32, "F"), rows, r, _dev(packed, torch.int32, "packed"),
+                              _stream(stream)), "lb_pack_signs")
+    return packed
+
+
+def _u16(t: torch.Tensor, name: str) -> int:
+    if t.dtype in (torch.float16, torch.bfloat16, torch.int16, torch.uint16):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+        return t.data_ptr()
+    raise TypeError(f"{name} must be a 16-bit tensor, got {t.dtype}")
+
+
+class Layer:
+    """Owns an ``lb_layer`` handle (see ``lb_layer_create``)."""
+
+    def __init__(self, handle: int, N: int, K: int, r: int, npaths: int):
+        self.handle = handle
+        self.N, self.K, self.r, self.npaths = N, K, r, npaths
+
+    @property
+    def bpw(self) -> float:
+        return float(_lib.lb_layer_bpw(self.handle))
+
+    @property
+    def device_bytes(self) -> int:
+        return int(_lib.lb_layer_device_bytes(self.handle))
+
+    def close(self):
+        if self.handle:
+            _lib.lb_layer_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def lb_layer_create(N: int, K: int, r: int, U, V, h, g, l, stream=None) -> Layer:
+    """Per-path lists: U[p] int32 [N, ceil(r/32)], V[p] int32 [K, ceil(r/32)] (canonical packed),
+    h[p] [N], g[p] [K], l[p] [r] binary16 (float16 or int16/uint16 bit patterns), all CUDA."""
+    npaths = len(U)
+    arrs = []
+    for name, lst in (("U", U), ("V", V), ("h", h), ("g", g), ("l", l)):
+        if len(lst) != npaths:
+            raise ValueError(f"{name} must have one entry per path")
+        if name in ("U", "V"):
+            ptrs = [_dev(t, torch.int32, f"{name}[{p}]") for p, t in enumerate(lst)]
+        else:
+            ptrs = [_u16(t, f"{name}[{p}]") for p, t in enumerate(lst)]
+        arrs.append((_vp * max(1, npaths))(*ptrs))
+    out = _vp()
+    _check(_lib.lb_layer_create(ctypes.byref(out), N, K, r, npaths, *arrs, _stream(stream)), "lb_layer_create")
+    return Layer(out.value, N, K, r, npaths)
+
+
+def lb_linear_forward(x: torch.Tensor, layer: Layer, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[M, N] float32 = x[M, K] (bfloat16) . W_hat^T."""
+    if x.dim() != 2 or x.shape[1] != layer.K:
+        raise ValueError(f"x must be [M, {layer.K}]")
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty((M, layer.N), dtype=torch.float32, device=x.device)
+    elif tuple(y.shape) != (M, layer.N):
+        raise ValueError(f"y must be [{M}, {layer.N}]")
+    _check(_lib.lb_linear_forward(_dev(x, torch.bfloat16, "x") if M else None, M, layer.handle,
+                                  _dev(y, torch.float32, "y") if M else None, _stream(stream)),
+           "lb_linear_forward")
+    return y
+
+
+class Stack:
+    """Owns an ``lb_stack`` handle; keeps its layers alive."""
+
+    def __init__(self, handle: int, layers):
+        self.handle = handle
+        self.layers = list(layers)
+
+    def close(self):
+        if self.handle:
+            _lib.lb_stack_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def lb_stack_create(layers, stream=None) -> Stack:
+    arr = (_vp * len(layers))(*[L.handle for L in layers])
+    out = _vp()
+    _check(_lib.lb_stack_create(ctypes.byref(out), arr, len(layers), _stream(stream)), "lb_stack_create")
+    return Stack(out.value, layers)
+
+
+class StackIO:
+    """Pointer tables of a stack call, marshalled once and reused."""
+
+    def __init__(self, stack: Stack, xs, ys):
+        if len(xs) != len(stack.layers) or len(ys) != len(stack.layers):
+            raise ValueError("one x and one y per layer")
+        M = xs[0].shape[0]
+        for L, x, y in zip(stack.layers, xs, ys):
+            if tuple(x.shape) != (M, L.K) or tuple(y.shape) != (M, L.N):
+                raise ValueError("x/y shapes do not match the layers")
+        self.M = M
+        self.xs, self.ys = list(xs), list(ys)
+        self.xp = (_vp * len(xs))(*[_dev(x, torch.bfloat16, "x") for x in xs])
+        self.yp = (_vp * len(ys))(*[_dev(y, torch.float32, "y") for y in ys])
+
+
+def lb_stack_forward(stack: Stack, xs=None, ys=None, stream=None, io: StackIO | None = None) -> StackIO:
+    """Run every layer i: ys[i] = xs[i] . W_hat_i^T.  Pass ``io`` to reuse marshalled pointer tables."""
+    if io is None:
+        io = StackIO(stack, xs, ys)
+    _check(_lib.lb_stack_forward(stack.handle, io.xp, io.yp, io.M, _stream(stream)), "lb_stack_forward")
+    return io

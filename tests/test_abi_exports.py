@@ -1,0 +1,76 @@
+"""The C-ABI library builds, loads and exports every symbol its header declares.
+
+CPU only: no call here reaches the GPU.  Argument validation runs before any
+CUDA call, so the error paths are checked on the host as well.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "littlebit.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sub_bit_weight_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lb_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("lb_pack_signs", "lb_layer_create", "lb_linear_forward", "lb_layer_destroy",
+                     "lb_stack_create", "lb_stack_forward", "lb_stack_destroy", "lb_layer_bpw"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_host_side_argument_checks(lib):
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    lib.lb_status_string.restype = ctypes.c_char_p
+    assert lib.lb_status_string(0) == b"LB_OK"
+    assert b"INVALID" in lib.lb_status_string(1)
+    lib.lb_packed_words.restype = ctypes.c_size_t
+    lib.lb_packed_words.argtypes = [i64, ctypes.c_int]
+    assert lib.lb_packed_words(10, 33) == 20
+    assert lib.lb_packed_words(-1, 3) == 0
+    lib.lb_pack_signs.argtypes = [vp, i64, ctypes.c_int, vp, vp]
+    assert lib.lb_pack_signs(None, -1, 4, None, None) == 1
+    assert lib.lb_pack_signs(None, 3, 0, None, None) == 1
+    assert lib.lb_pack_signs(None, 0, 4, None, None) == 0          # empty: nothing to do
+    assert lib.lb_pack_signs(None, 5, 4, None, None) == 1
+    assert lib.lb_pack_signs(vp(2), 5, 4, vp(64), None) == 1       # misaligned F
+    out = vp()
+    lib.lb_layer_create.argtypes = [ctypes.POINTER(vp)] + [ctypes.c_int] * 4 + [vp] * 6
+    assert lib.lb_layer_create(ctypes.byref(out), 8, 8, 4, 3, None, None, None, None, None, None) == 2
+    assert lib.lb_layer_create(ctypes.byref(out), 0, 8, 4, 2, None, None, None, None, None, None) == 1
+    assert lib.lb_layer_create(ctypes.byref(out), 8, 8, 4096, 2, None, None, None, None, None, None) == 1
+    assert lib.lb_layer_create(ctypes.byref(out), 8, 8, 4, 2, None, None, None, None, None, None) == 1
+    assert lib.lb_layer_create(None, 8, 8, 4, 2, None, None, None, None, None, None) == 1
+    lib.lb_linear_forward.argtypes = [vp, ctypes.c_int, vp, vp, vp]
+    assert lib.lb_linear_forward(None, 1, None, None, None) == 1
+    lib.lb_stack_create.argtypes = [ctypes.POINTER(vp), vp, ctypes.c_int, vp]
+    assert lib.lb_stack_create(ctypes.byref(out), None, 0, None) == 1
+    lib.lb_stack_forward.argtypes = [vp, vp, vp, ctypes.c_int, vp]
+    assert lib.lb_stack_forward(None, None, None, 1, None) == 1
+    lib.lb_layer_bpw.restype = ctypes.c_double
+    lib.lb_layer_bpw.argtypes = [vp]
+    assert lib.lb_layer_bpw(None) == 0.0
+    lib.lb_layer_destroy.argtypes = [vp]
+    lib.lb_layer_destroy(None)
+    lib.lb_stack_destroy.argtypes = [vp]
+    lib.lb_stack_destroy(None)
