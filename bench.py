@@ -150,11 +150,11 @@ def oracle_sample(w: synth.Workload, M: int, budget_s: float, max_layers: int | 
 
 # ----------------------------------------------------------------- GPU runs
 
-def run_gpu(w: synth.Workload, M: int, steps: int, warmup: int, dist, dev, want_e2e=True):
+def run_gpu(w: synth.Workload, M: int, steps: int, warmup: int, dist, dev, want_e2e=True, nblocks=None):
     import torch
     from sub_bit_weight_b200 import lib, stacks
 
-    layers, shapes = stacks.build_workload(w, device=dev)
+    layers, shapes = stacks.build_workload(w, device=dev, nblocks=nblocks)
     S = lib.lb_stack_create(layers)
     # contiguous x / y so that the end-to-end run moves them with one copy each way
     xsz = [M * s.K for s in shapes]
@@ -256,6 +256,7 @@ def main():
     ap.add_argument("--prefill", default=PREFILL_DEFAULT, help="prefill workload for the 'prefill' object ('' = skip)")
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--blocks", type=int, default=None, help="only the first N blocks of the stack (profiling)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -279,7 +280,7 @@ def main():
         dist = tdist
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    res = run_gpu(w, M, args.steps, args.warmup, dist, dev)
+    res = run_gpu(w, M, args.steps, args.warmup, dist, dev, nblocks=args.blocks)
     total_ms = max_over_ranks(res["total_ms"], dist)
     shapes = res["shapes"]
     k1b = sum(layer_bytes(s, M)[0] for s in shapes)

@@ -85,6 +85,9 @@ __device__ __forceinline__ int warp_sum(int v)
     return v;
 }
 
+// Per-thread contribution (no shuffles: callers may be divergent).
+__device__ __forceinline__ int warp_sum_partial(int v, int) { return v; }
+
 __device__ __forceinline__ int warp_or(int v)
 {
 #pragma unroll
@@ -93,87 +96,108 @@ __device__ __forceinline__ int warp_or(int v)
 }
 
 // ---------------------------------------------------------------------------
-// Finish contraction 1 of one layer (run by the last of its items):
-// z = sum over chunks, zl = z (.) l, then zl as B fragments for contraction 2.
+// Shared helpers of both kernels
 // ---------------------------------------------------------------------------
-__device__ void finish_latent(const LayerDev &d, int M, int *sE, int *sQs, float *sMax, int *sBad)
+__device__ __forceinline__ void copy_desc(LayerDev &dst, const LayerDev *src)
 {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nw = blockDim.x >> 5;
-    const int rows = d.npaths * d.r16;
+    static_assert(sizeof(LayerDev) % 4 == 0, "descriptor is copied as words");
+    for (int i = threadIdx.x; i < (int)(sizeof(LayerDev) / 4); i += blockDim.x)
+        reinterpret_cast<int *>(&dst)[i] = reinterpret_cast<const int *>(src)[i];
+}
+
+// non-negative floats order like their bit patterns
+__device__ __forceinline__ void smem_max(float *a, float v) { atomicMax((int *)a, __float_as_int(v)); }
+
+// ---------------------------------------------------------------------------
+// Finish contraction 1 of one layer (run by the last of its items):
+// z = sum over chunks (fixed order), zl = z (.) l, zl as B fragments for
+// contraction 2.  Also returns the integer partials to zero for the next call.
+// ---------------------------------------------------------------------------
+__device__ void finish_latent(const LayerDev &d, int M, int NT, int *sE, int *sQs, float *sMax, int *sBad)
+{
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int T = blockDim.x;
     if (tid < 32) {
         sMax[tid] = 0.0f;
         sBad[tid] = 0;
         sQs[tid] = 0;
     }
     __syncthreads();
-    // one warp per (path, row m): contiguous rows j of that path
-    for (int seg = warp; seg < d.npaths * M; seg += nw) {
-        const int p = seg / M, m = seg - p * M;
-        float amax = 0.0f;
-        int bad = 0;
-        for (int j = lane; j < d.r16; j += 32) {
-            const int jr = p * d.r16 + j;
-            float z = 0.0f;
-            for (int kc = 0; kc < d.nkc; ++kc) {
-                const int2 meta = __ldcg(&d.pmeta[(kc * 2 + p) * 16 + m]);
-                const int T = __ldcg(&d.partT[((size_t)kc * d.R1 + jr) * 16 + m]);
-                z += (meta.x == kNanExp) ? __int_as_float(0x7fc00000)
-                                         : ldexpf((float)(meta.y - 2 * T), -meta.x);
+    const int rows = d.npaths * d.r16;
+    for (int e = tid; e < rows * M; e += T) {
+        const int jr = e / M, m = e - jr * M;
+        const int p = jr / d.r16, j = jr - p * d.r16;
+        float z = 0.0f;
+        int kc = 0;
+        for (; kc + 4 <= d.nkc; kc += 4) {
+            int2 mt[4];
+            int tv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                mt[u] = __ldcg(&d.pmeta[((kc + u) * 2 + p) * 16 + m]);
+                tv[u] = __ldcg(&d.partT[((size_t)(kc + u) * d.R1 + jr) * 16 + m]);
             }
-            const float zl = (j < d.r) ? z * __half2float(d.l[p * d.r16 + j]) : 0.0f;
-            d.zl[(size_t)jr * 16 + m] = zl;
-            if (!(fabsf(zl) <= FLT_MAX)) bad = 1;
-            else amax = fmaxf(amax, fabsf(zl));
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                z += (mt[u].x == kNanExp) ? __int_as_float(0x7fc00000)
+                                          : ldexpf((float)(mt[u].y - 2 * tv[u]), -mt[u].x);
         }
-        amax = warp_max(amax);
-        bad = warp_or(bad);
-        if (lane == 0) {
-            sMax[p * 16 + m] = amax;
-            sBad[p * 16 + m] = bad;
+        for (; kc < d.nkc; ++kc) {
+            const int2 mt = __ldcg(&d.pmeta[(kc * 2 + p) * 16 + m]);
+            const int tv = __ldcg(&d.partT[((size_t)kc * d.R1 + jr) * 16 + m]);
+            z += (mt.x == kNanExp) ? __int_as_float(0x7fc00000) : ldexpf((float)(mt.y - 2 * tv), -mt.x);
         }
-    }
-    // zero the fragment buffer (columns of rows >= M must read as zero)
-    {
-        uint4 *zf = (uint4 *)d.zfrag;
-        const int n16 = d.KB2 * kMaxNT * 32 * (int)sizeof(uint2) / 16;
-        for (int i = tid; i < n16; i += blockDim.x) zf[i] = make_uint4(0, 0, 0, 0);
+        const float zl = (j < d.r) ? z * __half2float(d.l[p * d.r16 + j]) : 0.0f;
+        d.zl[(size_t)jr * 16 + m] = zl;
+        if (!(fabsf(zl) <= FLT_MAX)) atomicOr(&sBad[p * 16 + m], 1);
+        else smem_max(&sMax[p * 16 + m], fabsf(zl));
     }
     __syncthreads();
+    // integer partials back to zero (every row, including padding rows)
+    for (size_t e = tid; e < (size_t)d.nkc * d.R1 * 16; e += T) d.partT[e] = 0;
     if (tid < d.npaths * M) {
         const int p = tid / M, m = tid - p * M;
         sE[p * 16 + m] = exponent_for(sMax[p * 16 + m], sBad[p * 16 + m] != 0);
     }
     __syncthreads();
-    (void)rows;
-    // digits into fragments: one warp per (path, m), lanes over groups of 4 latent indices
-    for (int seg = warp; seg < d.npaths * M; seg += nw) {
-        const int p = seg / M, m = seg - p * M;
-        const int E = sE[p * 16 + m];
+    // digits into fragments; rows m in [M, 4*NT) get zero digits
+    const int MT = 4 * NT;
+    const int ngrp = d.r32 / 4;
+    for (int e = tid; e < d.npaths * MT * ngrp; e += T) {
+        const int c = e % ngrp;
+        const int pm = e / ngrp;
+        const int p = pm / MT, m = pm - p * MT;
+        uint32_t wlo = 0, whi = 0;
         int qs = 0;
-        for (int c = lane; c < d.r32 / 4; c += 32) {
-            uint32_t wlo = 0, whi = 0;
+        if (m < M) {
+            const int E = sE[p * 16 + m];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = 4 * c + e;
-                const float zl = (j < d.r16) ? d.zl[(size_t)(p * d.r16 + j) * 16 + m] : 0.0f;
+            for (int u = 0; u < 4; ++u) {
+                const int j = 4 * c + u;
+                const float zl = (j < d.r) ? d.zl[(size_t)(p * d.r16 + j) * 16 + m] : 0.0f;
                 const int q = (j < d.r) ? quantize(zl, E) : 0;
                 int lo, hi;
                 digits(q, lo, hi);
-                wlo |= (uint32_t)(lo & 255) << (8 * e);
-                whi |= (uint32_t)(hi & 255) << (8 * e);
+                wlo |= (uint32_t)(lo & 255) << (8 * u);
+                whi |= (uint32_t)(hi & 255) << (8 * u);
                 qs += q;
             }
-            const int jj = p * d.r32 + 4 * c;
-            const int kb = jj >> 5;
-            int llo, lhi, word;
-            frag_slot(m, jj & 31, llo, lhi, word);
-            uint2 *base = d.zfrag + ((size_t)kb * kMaxNT + (m >> 2)) * 32;
-            set_word(base[llo], word, wlo);
-            set_word(base[lhi], word, whi);
         }
-        qs = warp_sum(qs);
-        if (lane == 0) d.zmeta[p * 16 + m] = make_int2(E, qs);
+        const int jj = p * d.r32 + 4 * c;
+        int llo, lhi, word;
+        frag_slot(m, jj & 31, llo, lhi, word);
+        uint2 *fb = d.zfrag + ((size_t)(m >> 2) * d.KB2 + (jj >> 5)) * 32;
+        set_word(fb[llo], word, wlo);
+        set_word(fb[lhi], word, whi);
+        if (m < M) {
+            qs = warp_sum_partial(qs, lane);
+            if (qs) atomicAdd(&sQs[p * 16 + m], qs);
+        }
+    }
+    __syncthreads();
+    if (tid < d.npaths * M) {
+        const int p = tid / M, m = tid - p * M;
+        d.zmeta[p * 16 + m] = make_int2(sE[p * 16 + m], sQs[p * 16 + m]);
     }
 }
 
@@ -187,17 +211,31 @@ __global__ void __launch_bounds__(kDecodeThreads)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint2 *sB = (uint2 *)smem_raw;              // [2][kP1ChunkKB][NT][32]
+    __shared__ LayerDev sd;
     __shared__ float sMax[32];
     __shared__ int sBad[32], sE[32], sQs[32];
     __shared__ int sLast;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nw = kDecodeThreads / 32;
+    constexpr int NW = kDecodeThreads / 32;
     const int g = lane >> 2, t4 = lane & 3;
 
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
         const P1Item item = items[it];
-        const LayerDev &d = layers[item.layer];
+        __syncthreads();                    // previous item fully done with shared state
+        copy_desc(sd, layers + item.layer);
+        {
+            uint4 *z4 = (uint4 *)sB;
+            const int n16 = 2 * kP1ChunkKB * NT * 32 * (int)sizeof(uint2) / 16;
+            for (int i = tid; i < n16; i += kDecodeThreads) z4[i] = make_uint4(0, 0, 0, 0);
+        }
+        if (tid < 32) {
+            sMax[tid] = 0.0f;
+            sBad[tid] = 0;
+            sQs[tid] = 0;
+        }
+        __syncthreads();
+        const LayerDev &d = sd;
         const uint16_t *__restrict__ x = io.x[item.layer - base];
         const int kc = item.kc;
         const int kb0 = kc * kP1ChunkKB;
@@ -205,110 +243,130 @@ __global__ void __launch_bounds__(kDecodeThreads)
         const int k0 = kb0 * kKPerBlock;
         const int klen = nkb * kKPerBlock;
 
-        // zero the fragments (rows >= M and absent paths read as zero)
-        {
-            uint4 *z4 = (uint4 *)sB;
-            const int n16 = 2 * kP1ChunkKB * NT * 32 * (int)sizeof(uint2) / 16;
-            for (int i = tid; i < n16; i += kDecodeThreads) z4[i] = make_uint4(0, 0, 0, 0);
-        }
-        // pass 1: largest |x * g| per (path, m) over this chunk
-        for (int seg = warp; seg < d.npaths * M; seg += nw) {
-            const int p = seg / M, m = seg - p * M;
-            float amax = 0.0f;
-            int bad = 0;
-            for (int kk = lane; kk < klen; kk += 32) {
-                const int k = k0 + kk;
-                if (k < d.K) {
-                    const float tv = bf16_bits_to_float(x[(size_t)m * d.K + k]) *
-                                     __half2float(d.g[p * d.K32 + k]);
-                    if (!(fabsf(tv) <= FLT_MAX)) bad = 1;
-                    else amax = fmaxf(amax, fabsf(tv));
-                }
-            }
-            amax = warp_max(amax);
-            bad = warp_or(bad);
-            if (lane == 0) {
-                sE[p * 16 + m] = exponent_for(amax, bad != 0);
+        // ---- t = x (.) g for 8 consecutive inputs per thread: largest magnitude per (path, m)
+        const int kk0 = 8 * tid;
+        const bool act = kk0 < klen;
+        const int kg = k0 + kk0;
+        float gv[2][8];
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            if (act && p < d.npaths) {
+                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(d.g + (size_t)p * d.K32 + kg));
+                const __half *hv = reinterpret_cast<const __half *>(&raw);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) gv[p][e] = __half2float(hv[e]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) gv[p][e] = 0.0f;
             }
         }
-        __syncthreads();
-        // pass 2: digits into B fragments; digit sums per (path, m)
-        for (int seg = warp; seg < d.npaths * M; seg += nw) {
-            const int p = seg / M, m = seg - p * M;
-            const int E = sE[p * 16 + m];
-            int qs = 0;
-            for (int c = lane; c < klen / 4; c += 32) {
-                uint32_t wlo = 0, whi = 0;
+        const bool vec = ((d.K & 7) == 0) && (kg + 8 <= d.K);
+        auto load_x = [&](int m, float (&xv)[8]) {
+            if (!act) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) xv[e] = 0.0f;
+            } else if (vec) {
+                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * d.K + kg));
+                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int k = k0 + 4 * c + e;
-                    int q = 0;
-                    if (k < d.K) {
-                        const float tv = bf16_bits_to_float(x[(size_t)m * d.K + k]) *
-                                         __half2float(d.g[p * d.K32 + k]);
-                        q = quantize(tv, E);
-                    }
-                    int lo, hi;
-                    digits(q, lo, hi);
-                    wlo |= (uint32_t)(lo & 255) << (8 * e);
-                    whi |= (uint32_t)(hi & 255) << (8 * e);
-                    qs += q;
+                    xv[2 * e] = __uint_as_float(w4[e] << 16);
+                    xv[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
                 }
-                const int kk = 4 * c;
-                const int kbc = kk >> 5;
-                int llo, lhi, word;
-                frag_slot(m, kk & 31, llo, lhi, word);
-                uint2 *fb = sB + (((size_t)p * kP1ChunkKB + kbc) * NT + (m >> 2)) * 32;
-                set_word(fb[llo], word, wlo);
-                set_word(fb[lhi], word, whi);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    xv[e] = (kg + e < d.K) ? bf16_bits_to_float(__ldg(x + (size_t)m * d.K + kg + e)) : 0.0f;
             }
-            qs = warp_sum(qs);
-            if (lane == 0) {
-                sQs[p * 16 + m] = qs;
-                d.pmeta[(kc * 2 + p) * 16 + m] = make_int2(E, qs);
+        };
+        for (int m = 0; m < M; ++m) {
+            float xv[8];
+            load_x(m, xv);
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                float amax = 0.0f;
+                int bad = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float tv = fabsf(xv[e] * gv[p][e]);
+                    if (!(tv <= FLT_MAX)) bad = 1;
+                    else amax = fmaxf(amax, tv);
+                }
+                amax = warp_max(amax);
+                bad = warp_or(bad);
+                if (lane == 0 && p < d.npaths) {
+                    smem_max(&sMax[p * 16 + m], amax);
+                    if (bad) atomicOr(&sBad[p * 16 + m], 1);
+                }
             }
         }
         __syncthreads();
+        if (tid < d.npaths * M) {
+            const int p = tid / M, m = tid - p * M;
+            sE[p * 16 + m] = exponent_for(sMax[p * 16 + m], sBad[p * 16 + m] != 0);
+        }
+        __syncthreads();
+        // ---- digits into B fragments, digit sums per (path, m)
+        for (int m = 0; m < M; ++m) {
+            float xv[8];
+            load_x(m, xv);
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                if (p >= d.npaths) continue;
+                const int E = sE[p * 16 + m];
+                int qs = 0;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t wlo = 0, whi = 0;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int q = quantize(xv[4 * h + e] * gv[p][4 * h + e], E);
+                        int lo, hi;
+                        digits(q, lo, hi);
+                        wlo |= (uint32_t)(lo & 255) << (8 * e);
+                        whi |= (uint32_t)(hi & 255) << (8 * e);
+                        qs += q;
+                    }
+                    if (act) {
+                        const int kk = kk0 + 4 * h;
+                        int llo, lhi, word;
+                        frag_slot(m, kk & 31, llo, lhi, word);
+                        uint2 *fb = sB + (((size_t)p * kP1ChunkKB + (kk >> 5)) * NT + (m >> 2)) * 32;
+                        set_word(fb[llo], word, wlo);
+                        set_word(fb[lhi], word, whi);
+                    }
+                }
+                qs = warp_sum(qs);
+                if (lane == 0 && qs) atomicAdd(&sQs[p * 16 + m], qs);
+            }
+        }
+        __syncthreads();
+        if (tid < d.npaths * M) {
+            const int p = tid / M, m = tid - p * M;
+            d.pmeta[(kc * 2 + p) * 16 + m] = make_int2(sE[p * 16 + m], sQs[p * 16 + m]);
+        }
 
-        // main loop: one warp per row group of 64 latent rows
-        for (int rg = warp; rg < d.RG1; rg += nw) {
-            int acc[4][NT][4];
+        // ---- main stream: units (row group, k-block) of this chunk, split evenly over the warps
+        const int U1 = d.RG1 * nkb;
+        const int ub = (int)((long long)U1 * warp / NW), ue = (int)((long long)U1 * (warp + 1) / NW);
+        int acc[4][NT][4];
 #pragma unroll
-            for (int rb = 0; rb < 4; ++rb)
+        for (int rb = 0; rb < 4; ++rb)
 #pragma unroll
-                for (int n = 0; n < NT; ++n)
+            for (int n = 0; n < NT; ++n)
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) acc[rb][n][c] = 0;
-            int prb[4];
+                for (int c = 0; c < 4; ++c) acc[rb][n][c] = 0;
+        int lrg = ub / nkb, lkb = ub - lrg * nkb;     // load cursor
+        int prg = lrg, pkb = lkb;                     // process cursor
+        int nload = ue - ub, nproc = ue - ub;
+        int prb[4];
+        auto set_paths = [&](int rg) {
 #pragma unroll
             for (int rb = 0; rb < 4; ++rb)
                 prb[rb] = min((rg * kRowsPerGroup + rb * kRowsPerBlock) / d.r16, d.npaths - 1);
-            const uint2 *src = d.vt + ((size_t)rg * d.KB1 + kb0) * 32 + lane;
-            constexpr int UNR = 8;
-            for (int kb = 0; kb < nkb; kb += UNR) {
-                uint2 w[UNR];
-#pragma unroll
-                for (int u = 0; u < UNR; ++u)
-                    if (kb + u < nkb) w[u] = ld_stream_u2(src + (size_t)(kb + u) * 32);
-#pragma unroll
-                for (int u = 0; u < UNR; ++u) {
-                    if (kb + u < nkb) {
-#pragma unroll
-                        for (int rb = 0; rb < 4; ++rb) {
-                            const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                            const uint32_t a0 = w[u].x & mlo, a1 = w[u].x & mhi;
-                            const uint32_t a2 = w[u].y & mlo, a3 = w[u].y & mhi;
-                            const uint2 *fb = sB + ((size_t)prb[rb] * kP1ChunkKB + kb + u) * NT * 32 + lane;
-#pragma unroll
-                            for (int n = 0; n < NT; ++n) {
-                                const uint2 b = fb[n * 32];
-                                mma_u8s8(acc[rb][n], a0, a1, a2, a3, b.x, b.y);
-                            }
-                        }
-                    }
-                }
-            }
-            // integer partials: rows g (scale 2^rb) and g + 8 (scale 2^(rb+4))
+        };
+        set_paths(prg);
+        auto flush = [&](int rg) {
 #pragma unroll
             for (int rb = 0; rb < 4; ++rb)
 #pragma unroll
@@ -318,24 +376,77 @@ __global__ void __launch_bounds__(kDecodeThreads)
                         const int Tlo = (acc[rb][n][0] >> rb) + 256 * (acc[rb][n][1] >> rb);
                         const int Thi = (acc[rb][n][2] >> (rb + 4)) + 256 * (acc[rb][n][3] >> (rb + 4));
                         const int row = rg * kRowsPerGroup + rb * kRowsPerBlock + g;
-                        d.partT[((size_t)kc * d.R1 + row) * 16 + m] = Tlo;
-                        d.partT[((size_t)kc * d.R1 + row + 8) * 16 + m] = Thi;
+                        if (Tlo) atomicAdd(&d.partT[((size_t)kc * d.R1 + row) * 16 + m], Tlo);
+                        if (Thi) atomicAdd(&d.partT[((size_t)kc * d.R1 + row + 8) * 16 + m], Thi);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) acc[rb][n][c] = 0;
+                }
+        };
+        constexpr int B = 8;
+        uint2 bufA[B], bufB[B];
+        auto load_batch = [&](uint2 (&buf)[B]) {
+#pragma unroll
+            for (int i = 0; i < B; ++i) {
+                if (nload > 0) {
+                    buf[i] = ld_stream_u2(d.vt + ((size_t)lrg * d.KB1 + kb0 + lkb) * 32 + lane);
+                    if (++lkb == nkb) { lkb = 0; ++lrg; }
+                    --nload;
+                }
+            }
+        };
+        auto proc_batch = [&](const uint2 (&buf)[B]) {
+#pragma unroll
+            for (int i = 0; i < B; ++i) {
+                if (nproc > 0) {
+                    const uint2 w = buf[i];
+                    uint2 bp[2][NT];
+#pragma unroll
+                    for (int p = 0; p < 2; ++p)
+#pragma unroll
+                        for (int n = 0; n < NT; ++n)
+                            bp[p][n] = sB[(((size_t)p * kP1ChunkKB + pkb) * NT + n) * 32 + lane];
+#pragma unroll
+                    for (int rb = 0; rb < 4; ++rb) {
+                        const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                        const uint32_t a0 = w.x & mlo, a1 = w.x & mhi, a2 = w.y & mlo, a3 = w.y & mhi;
+#pragma unroll
+                        for (int n = 0; n < NT; ++n) {
+                            const uint2 b = prb[rb] ? bp[1][n] : bp[0][n];
+                            mma_u8s8(acc[rb][n], a0, a1, a2, a3, b.x, b.y);
+                        }
+                    }
+                    --nproc;
+                    if (++pkb == nkb) {
+                        flush(prg);
+                        pkb = 0;
+                        ++prg;
+                        set_paths(prg);
                     }
                 }
+            }
+        };
+        load_batch(bufA);
+        load_batch(bufB);
+        while (nproc > 0) {
+            proc_batch(bufA);
+            load_batch(bufA);
+            proc_batch(bufB);
+            load_batch(bufB);
         }
+        if (pkb != 0) flush(prg);
 
-        // completion count; the last item of the layer finishes the latent vector
+        // ---- completion count; the last item of the layer finishes the latent vector
         __threadfence();
         __syncthreads();
         if (tid == 0) sLast = (atomicAdd(d.counter, 1u) == (unsigned)(d.nkc - 1));
         __syncthreads();
         if (sLast) {
             __threadfence();
-            finish_latent(d, M, sE, sQs, sMax, sBad);
+            finish_latent(d, M, NT, sE, sQs, sMax, sBad);
             __syncthreads();
             if (tid == 0) atomicExch(d.counter, 0u);
         }
-        __syncthreads();
     }
 }
 
@@ -348,102 +459,143 @@ __global__ void __launch_bounds__(kDecodeThreads)
                         int nitems, const __grid_constant__ IoPtrs io, int base, int M)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    uint2 *sB = (uint2 *)smem_raw;              // [KB2][NT][32]
+    uint2 *sB = (uint2 *)smem_raw;              // [NT][KB2][32]
+    __shared__ LayerDev sd;
     __shared__ int2 sMeta[32];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nw = kDecodeThreads / 32;
+    constexpr int NW = kDecodeThreads / 32;
     const int g = lane >> 2, t4 = lane & 3;
 
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
         const P2Item item = items[it];
-        const LayerDev &d = layers[item.layer];
+        __syncthreads();   // previous item's readers of shared state are done
+        copy_desc(sd, layers + item.layer);
+        __syncthreads();
+        const LayerDev &d = sd;
         float *__restrict__ y = io.y[item.layer - base];
-        __syncthreads();   // previous item's readers of sB are done
-        for (int i = tid; i < d.KB2 * NT * 32; i += kDecodeThreads) {
-            const int l = i & 31, rest = i >> 5;
-            const int n = rest % NT, kb = rest / NT;
-            sB[i] = __ldcg(&d.zfrag[((size_t)kb * kMaxNT + n) * 32 + l]);
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(d.zfrag);
+            uint4 *dst = reinterpret_cast<uint4 *>(sB);
+            const int n16 = NT * d.KB2 * 32 * (int)sizeof(uint2) / 16;
+            for (int i = tid; i < n16; i += kDecodeThreads) dst[i] = __ldcg(src + i);
         }
         if (tid < 32) sMeta[tid] = __ldcg(&d.zmeta[tid]);
         __syncthreads();
 
         const int kbp = d.r32 / kKPerBlock;   // k-blocks per path
-        for (int rg = item.rg0 + warp; rg < item.rg1; rg += nw) {
-            float yv[4][NT][2];
+        const int KB2 = d.KB2;
+        const int nrg = (item.rg1 - item.rg0 - warp + NW - 1) / NW;   // this warp's row groups
+        int nload = max(0, nrg) * KB2, nproc = nload;
+        int lrg = item.rg0 + warp, lkb = 0;
+        int prg = lrg, pkb = 0;
+        int acc[4][NT][4];
+        float yv[4][NT][2];
+        float hv[2][4][2];
 #pragma unroll
-            for (int rb = 0; rb < 4; ++rb)
+        for (int rb = 0; rb < 4; ++rb)
 #pragma unroll
-                for (int n = 0; n < NT; ++n) yv[rb][n][0] = yv[rb][n][1] = 0.0f;
-            const uint2 *src = d.ut + (size_t)rg * d.KB2 * 32 + lane;
-            for (int p = 0; p < d.npaths; ++p) {
-                int acc[4][NT][4];
+            for (int n = 0; n < NT; ++n) {
+                yv[rb][n][0] = yv[rb][n][1] = 0.0f;
 #pragma unroll
-                for (int rb = 0; rb < 4; ++rb)
-#pragma unroll
-                    for (int n = 0; n < NT; ++n)
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) acc[rb][n][c] = 0;
-                const int kbA = p * kbp, kbB = kbA + kbp;
-                constexpr int UNR = 8;
-                for (int kb = kbA; kb < kbB; kb += UNR) {
-                    uint2 w[UNR];
-#pragma unroll
-                    for (int u = 0; u < UNR; ++u)
-                        if (kb + u < kbB) w[u] = ld_stream_u2(src + (size_t)(kb + u) * 32);
-#pragma unroll
-                    for (int u = 0; u < UNR; ++u) {
-                        if (kb + u < kbB) {
-                            const uint2 *fb = sB + (size_t)(kb + u) * NT * 32 + lane;
-                            uint2 b[NT];
-#pragma unroll
-                            for (int n = 0; n < NT; ++n) b[n] = fb[n * 32];
-#pragma unroll
-                            for (int rb = 0; rb < 4; ++rb) {
-                                const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                                const uint32_t a0 = w[u].x & mlo, a1 = w[u].x & mhi;
-                                const uint32_t a2 = w[u].y & mlo, a3 = w[u].y & mhi;
-#pragma unroll
-                                for (int n = 0; n < NT; ++n) mma_u8s8(acc[rb][n], a0, a1, a2, a3, b[n].x, b[n].y);
-                            }
-                        }
-                    }
-                }
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    const int m = 4 * n + t4;
-                    const int2 meta = (m < M) ? sMeta[p * 16 + m] : make_int2(0, 0);
-#pragma unroll
-                    for (int rb = 0; rb < 4; ++rb) {
-                        const int Tlo = (acc[rb][n][0] >> rb) + 256 * (acc[rb][n][1] >> rb);
-                        const int Thi = (acc[rb][n][2] >> (rb + 4)) + 256 * (acc[rb][n][3] >> (rb + 4));
-                        const int nlo = rg * kRowsPerGroup + rb * kRowsPerBlock + g;
-                        const float hlo = __half2float(d.h[p * d.N64 + nlo]);
-                        const float hhi = __half2float(d.h[p * d.N64 + nlo + 8]);
-                        float slo, shi;
-                        if (meta.x == kNanExp) {
-                            slo = shi = __int_as_float(0x7fc00000);
-                        } else {
-                            slo = ldexpf((float)(meta.y - 2 * Tlo), -meta.x);
-                            shi = ldexpf((float)(meta.y - 2 * Thi), -meta.x);
-                        }
-                        yv[rb][n][0] += hlo * slo;
-                        yv[rb][n][1] += hhi * shi;
-                    }
-                }
+                for (int c = 0; c < 4; ++c) acc[rb][n][c] = 0;
             }
+        auto load_h = [&](int rg) {
+#pragma unroll
+            for (int p = 0; p < 2; ++p)
+#pragma unroll
+                for (int rb = 0; rb < 4; ++rb) {
+                    const int n = rg * kRowsPerGroup + rb * kRowsPerBlock + g;
+                    const bool ok = p < d.npaths && rg < item.rg1;
+                    hv[p][rb][0] = ok ? __half2float(d.h[p * d.N64 + n]) : 0.0f;
+                    hv[p][rb][1] = ok ? __half2float(d.h[p * d.N64 + n + 8]) : 0.0f;
+                }
+        };
+        load_h(prg);
+        auto fold = [&](int p) {
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
                 const int m = 4 * n + t4;
-                if (m < M) {
+                const int2 meta = (m < M) ? sMeta[p * 16 + m] : make_int2(0, 0);
 #pragma unroll
-                    for (int rb = 0; rb < 4; ++rb) {
-                        const int nlo = rg * kRowsPerGroup + rb * kRowsPerBlock + g;
+                for (int rb = 0; rb < 4; ++rb) {
+                    const int Tlo = (acc[rb][n][0] >> rb) + 256 * (acc[rb][n][1] >> rb);
+                    const int Thi = (acc[rb][n][2] >> (rb + 4)) + 256 * (acc[rb][n][3] >> (rb + 4));
+                    float slo, shi;
+                    if (meta.x == kNanExp) {
+                        slo = shi = __int_as_float(0x7fc00000);
+                    } else {
+                        slo = ldexpf((float)(meta.y - 2 * Tlo), -meta.x);
+                        shi = ldexpf((float)(meta.y - 2 * Thi), -meta.x);
+                    }
+                    yv[rb][n][0] += (p ? hv[1][rb][0] : hv[0][rb][0]) * slo;
+                    yv[rb][n][1] += (p ? hv[1][rb][1] : hv[0][rb][1]) * shi;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) acc[rb][n][c] = 0;
+                }
+            }
+        };
+        auto store = [&](int rg) {
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const int m = 4 * n + t4;
+#pragma unroll
+                for (int rb = 0; rb < 4; ++rb) {
+                    const int nlo = rg * kRowsPerGroup + rb * kRowsPerBlock + g;
+                    if (m < M) {
                         if (nlo < d.N) y[(size_t)m * d.N + nlo] = yv[rb][n][0];
                         if (nlo + 8 < d.N) y[(size_t)m * d.N + nlo + 8] = yv[rb][n][1];
                     }
+                    yv[rb][n][0] = yv[rb][n][1] = 0.0f;
                 }
             }
+        };
+        constexpr int B = 8;
+        uint2 bufA[B], bufB[B];
+        auto load_batch = [&](uint2 (&buf)[B]) {
+#pragma unroll
+            for (int i = 0; i < B; ++i) {
+                if (nload > 0) {
+                    buf[i] = ld_stream_u2(d.ut + ((size_t)lrg * KB2 + lkb) * 32 + lane);
+                    if (++lkb == KB2) { lkb = 0; lrg += NW; }
+                    --nload;
+                }
+            }
+        };
+        auto proc_batch = [&](const uint2 (&buf)[B]) {
+#pragma unroll
+            for (int i = 0; i < B; ++i) {
+                if (nproc > 0) {
+                    const uint2 w = buf[i];
+                    uint2 b[NT];
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) b[n] = sB[((size_t)n * KB2 + pkb) * 32 + lane];
+#pragma unroll
+                    for (int rb = 0; rb < 4; ++rb) {
+                        const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                        const uint32_t a0 = w.x & mlo, a1 = w.x & mhi, a2 = w.y & mlo, a3 = w.y & mhi;
+#pragma unroll
+                        for (int n = 0; n < NT; ++n) mma_u8s8(acc[rb][n], a0, a1, a2, a3, b[n].x, b[n].y);
+                    }
+                    --nproc;
+                    ++pkb;
+                    if (pkb % kbp == 0) fold(pkb / kbp - 1);
+                    if (pkb == KB2) {
+                        store(prg);
+                        pkb = 0;
+                        prg += NW;
+                        load_h(prg);
+                    }
+                }
+            }
+        };
+        load_batch(bufA);
+        load_batch(bufB);
+        while (nproc > 0) {
+            proc_batch(bufA);
+            load_batch(bufA);
+            proc_batch(bufB);
+            load_batch(bufB);
         }
     }
 }

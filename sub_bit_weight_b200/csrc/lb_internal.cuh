@@ -62,7 +62,7 @@ struct LayerDev {
     int *partT;         // [nkc][R1][16]   integer partial sums of contraction 1
     int2 *pmeta;        // [nkc][2][16]    (exponent, digit sum) of each chunk
     float *zl;          // [R1][16]        latent vector after l
-    uint2 *zfrag;       // [KB2][kMaxNT][32] B fragments of contraction 2
+    uint2 *zfrag;       // [kMaxNT][KB2][32] B fragments of contraction 2
     int2 *zmeta;        // [2][16]         (exponent, digit sum) of zl
     unsigned *counter;  // chunks of contraction 1 finished (self-resetting)
 };
