@@ -3,24 +3,27 @@
 // The notes page of LittleBit (section "Multi-scale compensation") evaluates
 // a path as  x (.) g -> . V_sign -> (.) l -> . U_sign^T -> (.) h  and
 // "Residual compensation" sums the primary and residual paths.  Two kernels
-// cover every layer of a plan:
+// cover every layer of a plan (a stack) in one launch each:
 //
-//   contraction 1 (one work item = one layer x 1024 inputs):
-//     t = x (.) g_p for both paths, written as 16-bit fixed point with one
-//     power-of-two exponent per (item, path, row) and split into two signed
-//     base-256 digits; z-partials = t . V_sign on integer tensor cores, exact
-//     in int32.  The last item of a layer to finish (a completion counter,
-//     no waiting) sums the partials in a fixed order, applies l, and writes
-//     the latent vector as 16-bit fixed-point B fragments for contraction 2.
-//   contraction 2 (one work item = one layer x 512 outputs):
-//     s_p = zl_p . U_sign,p^T on integer tensor cores, y = sum_p h_p (.) s_p.
+//   contraction 1 (work item = one layer x 1024 inputs):
+//     t = x (.) g_p for both paths in 16-bit fixed point (one power-of-two
+//     exponent E per item, path and activation row; two signed base-256
+//     digits), then sum_k b[k][j] * t[k] on integer tensor cores (exact in
+//     int32, b = stored sign bit).  Each item adds 2^-E times its integer
+//     results into float64 accumulators: sum_k b*t per latent row and sum_k t
+//     per path.  Those terms are integers times powers of two a few dozen bits
+//     wide, so the float64 sums are exact and independent of arrival order.
+//   contraction 2 (work item = one layer x 512 outputs):
+//     z = sum_k t - 2 * sum_k b*t (a sign s = 1 - 2b), zl = z (.) l, zl in
+//     16-bit fixed point as B fragments (rebuilt by every item from the
+//     accumulators), then s = zl . U_sign^T on integer tensor cores and
+//     y = sum_p h_p (.) s_p.
 //
-// A sign s = 1 - 2b (b = stored bit) turns sum_k s_k q_k into
-// Qsum - 2 * sum_k b_k q_k, so the tensor cores only ever see {0, 2^i} bytes
-// (see the unit layout in lb_internal.cuh).  Rounding happens only when the
-// activations enter fixed point (16 significant bits relative to the largest
-// magnitude of their block) and in float32 sums; the tolerance budget is in
-// the design notes.
+// Weights stream through a small ring of shared-memory buffers per warp,
+// filled by bulk asynchronous copies (cp.async.bulk) that complete on an
+// mbarrier; every wait is bounded and reports a timeout instead of hanging.
+// The accumulators come in two parities that alternate between calls: the
+// contraction-2 kernel of call c zeroes the parity that call c+1 will use.
 
 #include <cfloat>
 
@@ -28,6 +31,9 @@
 
 namespace lb {
 
+// ---------------------------------------------------------------------------
+// Fixed point
+// ---------------------------------------------------------------------------
 __device__ __forceinline__ int exponent_for(float amax, bool nonfinite)
 {
     // Largest E with amax * 2^E <= 32639, so that q = rint(t * 2^E) splits into
@@ -53,10 +59,10 @@ __device__ __forceinline__ void digits(int q, int &lo, int &hi)
     hi = (q - lo) >> 8;
 }
 
-// Where the two digit words of activation row m, k-group (4 consecutive k
-// starting at kk within a 32-wide k-block) live among the 32 lanes' B
-// fragments of m16n8k32: column g = 2 * (m % 4) + digit, lane = 4 * g + t,
-// word (kk / 16), with t = (kk % 16) / 4.
+// Where the two digit words of activation row m and 4 consecutive k starting
+// at kk (within a 32-wide k-block) live among the lanes' m16n8k32 B
+// fragments: column g = 2 * (m % 4) + digit, lane = 4 * g + t, word kk / 16,
+// with t = (kk % 16) / 4.
 __device__ __forceinline__ void frag_slot(int m, int kk, int &lane_lo, int &lane_hi, int &word)
 {
     const int mm = m & 3;
@@ -85,9 +91,6 @@ __device__ __forceinline__ int warp_sum(int v)
     return v;
 }
 
-// Per-thread contribution (no shuffles: callers may be divergent).
-__device__ __forceinline__ int warp_sum_partial(int v, int) { return v; }
-
 __device__ __forceinline__ int warp_or(int v)
 {
 #pragma unroll
@@ -95,110 +98,54 @@ __device__ __forceinline__ int warp_or(int v)
     return v;
 }
 
-// ---------------------------------------------------------------------------
-// Shared helpers of both kernels
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void copy_desc(LayerDev &dst, const LayerDev *src)
-{
-    static_assert(sizeof(LayerDev) % 4 == 0, "descriptor is copied as words");
-    for (int i = threadIdx.x; i < (int)(sizeof(LayerDev) / 4); i += blockDim.x)
-        reinterpret_cast<int *>(&dst)[i] = reinterpret_cast<const int *>(src)[i];
-}
-
 // non-negative floats order like their bit patterns
 __device__ __forceinline__ void smem_max(float *a, float v) { atomicMax((int *)a, __float_as_int(v)); }
 
 // ---------------------------------------------------------------------------
-// Finish contraction 1 of one layer (run by the last of its items):
-// z = sum over chunks (fixed order), zl = z (.) l, zl as B fragments for
-// contraction 2.  Also returns the integer partials to zero for the next call.
+// mbarrier + bulk copy (one ring of buffers per warp)
 // ---------------------------------------------------------------------------
-__device__ void finish_latent(const LayerDev &d, int M, int NT, int *sE, int *sQs, float *sMax, int *sBad)
+__device__ __forceinline__ uint32_t sm_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void bar_init(uint64_t *b)
 {
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int T = blockDim.x;
-    if (tid < 32) {
-        sMax[tid] = 0.0f;
-        sBad[tid] = 0;
-        sQs[tid] = 0;
-    }
-    __syncthreads();
-    const int rows = d.npaths * d.r16;
-    for (int e = tid; e < rows * M; e += T) {
-        const int jr = e / M, m = e - jr * M;
-        const int p = jr / d.r16, j = jr - p * d.r16;
-        float z = 0.0f;
-        int kc = 0;
-        for (; kc + 4 <= d.nkc; kc += 4) {
-            int2 mt[4];
-            int tv[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                mt[u] = __ldcg(&d.pmeta[((kc + u) * 2 + p) * 16 + m]);
-                tv[u] = __ldcg(&d.partT[((size_t)(kc + u) * d.R1 + jr) * 16 + m]);
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                z += (mt[u].x == kNanExp) ? __int_as_float(0x7fc00000)
-                                          : ldexpf((float)(mt[u].y - 2 * tv[u]), -mt[u].x);
-        }
-        for (; kc < d.nkc; ++kc) {
-            const int2 mt = __ldcg(&d.pmeta[(kc * 2 + p) * 16 + m]);
-            const int tv = __ldcg(&d.partT[((size_t)kc * d.R1 + jr) * 16 + m]);
-            z += (mt.x == kNanExp) ? __int_as_float(0x7fc00000) : ldexpf((float)(mt.y - 2 * tv), -mt.x);
-        }
-        const float zl = (j < d.r) ? z * __half2float(d.l[p * d.r16 + j]) : 0.0f;
-        d.zl[(size_t)jr * 16 + m] = zl;
-        if (!(fabsf(zl) <= FLT_MAX)) atomicOr(&sBad[p * 16 + m], 1);
-        else smem_max(&sMax[p * 16 + m], fabsf(zl));
-    }
-    __syncthreads();
-    // integer partials back to zero (every row, including padding rows)
-    for (size_t e = tid; e < (size_t)d.nkc * d.R1 * 16; e += T) d.partT[e] = 0;
-    if (tid < d.npaths * M) {
-        const int p = tid / M, m = tid - p * M;
-        sE[p * 16 + m] = exponent_for(sMax[p * 16 + m], sBad[p * 16 + m] != 0);
-    }
-    __syncthreads();
-    // digits into fragments; rows m in [M, 4*NT) get zero digits
-    const int MT = 4 * NT;
-    const int ngrp = d.r32 / 4;
-    for (int e = tid; e < d.npaths * MT * ngrp; e += T) {
-        const int c = e % ngrp;
-        const int pm = e / ngrp;
-        const int p = pm / MT, m = pm - p * MT;
-        uint32_t wlo = 0, whi = 0;
-        int qs = 0;
-        if (m < M) {
-            const int E = sE[p * 16 + m];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int j = 4 * c + u;
-                const float zl = (j < d.r) ? d.zl[(size_t)(p * d.r16 + j) * 16 + m] : 0.0f;
-                const int q = (j < d.r) ? quantize(zl, E) : 0;
-                int lo, hi;
-                digits(q, lo, hi);
-                wlo |= (uint32_t)(lo & 255) << (8 * u);
-                whi |= (uint32_t)(hi & 255) << (8 * u);
-                qs += q;
-            }
-        }
-        const int jj = p * d.r32 + 4 * c;
-        int llo, lhi, word;
-        frag_slot(m, jj & 31, llo, lhi, word);
-        uint2 *fb = d.zfrag + ((size_t)(m >> 2) * d.KB2 + (jj >> 5)) * 32;
-        set_word(fb[llo], word, wlo);
-        set_word(fb[lhi], word, whi);
-        if (m < M) {
-            qs = warp_sum_partial(qs, lane);
-            if (qs) atomicAdd(&sQs[p * 16 + m], qs);
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(sm_addr(b)));
+}
+
+__device__ __forceinline__ void ring_fill(void *dst, const void *src, unsigned bytes, uint64_t *bar)
+{
+    asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(sm_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                     sm_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(sm_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ bool bar_try(uint64_t *b, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+                 : "=r"(ok)
+                 : "r"(sm_addr(b)), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+constexpr long long kDecWaitCycles = 4000000000LL;   // ~2 s
+
+// Bounded wait for a ring buffer; false (and an error code) on timeout.
+__device__ __forceinline__ bool ring_wait(uint64_t *b, uint32_t parity, int *err)
+{
+    if (bar_try(b, parity)) return true;
+    const long long t0 = clock64();
+    while (!bar_try(b, parity)) {
+        if (clock64() - t0 > kDecWaitCycles) {
+            atomicCAS(err, 0, 16);
+            return false;
         }
     }
-    __syncthreads();
-    if (tid < d.npaths * M) {
-        const int p = tid / M, m = tid - p * M;
-        d.zmeta[p * 16 + m] = make_int2(sE[p * 16 + m], sQs[p * 16 + m]);
-    }
+    return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -206,24 +153,53 @@ __device__ void finish_latent(const LayerDev &d, int M, int NT, int *sE, int *sQ
 // ---------------------------------------------------------------------------
 template <int NT>
 __global__ void __launch_bounds__(kDecodeThreads)
-    contraction1_kernel(const LayerDev *__restrict__ layers, const P1Item *__restrict__ items,
-                        int nitems, const __grid_constant__ IoPtrs io, int base, int M)
+    contraction1_kernel(const LayerDev *__restrict__ layers, const P1Item *__restrict__ items, int nitems,
+                        const __grid_constant__ IoPtrs io, int base, int M, int parity, int *err)
 {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    uint2 *sB = (uint2 *)smem_raw;              // [2][kP1ChunkKB][NT][32]
-    __shared__ LayerDev sd;
+    constexpr int NW = kDecodeThreads / 32;
+    constexpr int kStage = kP1ChunkKB * 256;                 // one row group x one chunk of k
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char *ring = smem_raw;                          // [NW][kP1Stages][kStage]
+    uint2 *sB = (uint2 *)(smem_raw + NW * kP1Stages * kStage);   // [2][kP1ChunkKB][NT][32]
+    __shared__ uint64_t bars[NW][kP1Stages];
     __shared__ float sMax[32];
     __shared__ int sBad[32], sE[32], sQs[32];
-    __shared__ int sLast;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr int NW = kDecodeThreads / 32;
     const int g = lane >> 2, t4 = lane & 3;
+    if (lane == 0)
+        for (int s = 0; s < kP1Stages; ++s) bar_init(&bars[warp][s]);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    __syncwarp();
+    uint32_t issued = 0, consumed = 0;   // this warp's ring sequence numbers
+    unsigned char *my_ring = ring + warp * kP1Stages * kStage;
 
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
         const P1Item item = items[it];
-        __syncthreads();                    // previous item fully done with shared state
-        copy_desc(sd, layers + item.layer);
+        const LayerDev *dp = layers + item.layer;
+        const int K = dp->K, K32 = dp->K32, KB1 = dp->KB1, RG1 = dp->RG1, r16 = dp->r16, npaths = dp->npaths;
+        const uint2 *__restrict__ vt = dp->vt;
+        const __half *__restrict__ gsc = dp->g;
+        double *__restrict__ acc = dp->acc[parity];
+        const uint16_t *__restrict__ x = io.x[item.layer - base];
+        const int kc = item.kc;
+        const int kb0 = kc * kP1ChunkKB;
+        const int nkb = min(kP1ChunkKB, KB1 - kb0);
+        const int k0 = kb0 * kKPerBlock;
+        const int klen = nkb * kKPerBlock;
+        const unsigned stage_bytes = (unsigned)nkb * 256u;
+
+        // start streaming this warp's first row groups while the activations are prepared
+        if (lane == 0)
+            for (int s = 0; s < kP1Stages; ++s) {
+                const int rg = warp + NW * s;
+                if (rg < RG1) {
+                    const int st = issued % kP1Stages;
+                    ring_fill(my_ring + st * kStage, vt + ((size_t)rg * KB1 + kb0) * 32, stage_bytes, &bars[warp][st]);
+                    ++issued;
+                }
+            }
+
         {
             uint4 *z4 = (uint4 *)sB;
             const int n16 = 2 * kP1ChunkKB * NT * 32 * (int)sizeof(uint2) / 16;
@@ -235,23 +211,16 @@ __global__ void __launch_bounds__(kDecodeThreads)
             sQs[tid] = 0;
         }
         __syncthreads();
-        const LayerDev &d = sd;
-        const uint16_t *__restrict__ x = io.x[item.layer - base];
-        const int kc = item.kc;
-        const int kb0 = kc * kP1ChunkKB;
-        const int nkb = min(kP1ChunkKB, d.KB1 - kb0);
-        const int k0 = kb0 * kKPerBlock;
-        const int klen = nkb * kKPerBlock;
 
-        // ---- t = x (.) g for 8 consecutive inputs per thread: largest magnitude per (path, m)
+        // ---- t = x (.) g for 8 consecutive inputs per thread; largest magnitude per (path, m)
         const int kk0 = 8 * tid;
         const bool act = kk0 < klen;
         const int kg = k0 + kk0;
         float gv[2][8];
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
-            if (act && p < d.npaths) {
-                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(d.g + (size_t)p * d.K32 + kg));
+            if (act && p < npaths) {
+                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(gsc + (size_t)p * K32 + kg));
                 const __half *hv = reinterpret_cast<const __half *>(&raw);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) gv[p][e] = __half2float(hv[e]);
@@ -260,13 +229,13 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 for (int e = 0; e < 8; ++e) gv[p][e] = 0.0f;
             }
         }
-        const bool vec = ((d.K & 7) == 0) && (kg + 8 <= d.K);
+        const bool vec = ((K & 7) == 0) && (kg + 8 <= K);
         auto load_x = [&](int m, float (&xv)[8]) {
             if (!act) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) xv[e] = 0.0f;
             } else if (vec) {
-                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * d.K + kg));
+                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + kg));
                 const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -276,7 +245,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
             } else {
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    xv[e] = (kg + e < d.K) ? bf16_bits_to_float(__ldg(x + (size_t)m * d.K + kg + e)) : 0.0f;
+                    xv[e] = (kg + e < K) ? bf16_bits_to_float(__ldg(x + (size_t)m * K + kg + e)) : 0.0f;
             }
         };
         for (int m = 0; m < M; ++m) {
@@ -294,14 +263,14 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 }
                 amax = warp_max(amax);
                 bad = warp_or(bad);
-                if (lane == 0 && p < d.npaths) {
+                if (lane == 0 && p < npaths) {
                     smem_max(&sMax[p * 16 + m], amax);
                     if (bad) atomicOr(&sBad[p * 16 + m], 1);
                 }
             }
         }
         __syncthreads();
-        if (tid < d.npaths * M) {
+        if (tid < npaths * M) {
             const int p = tid / M, m = tid - p * M;
             sE[p * 16 + m] = exponent_for(sMax[p * 16 + m], sBad[p * 16 + m] != 0);
         }
@@ -312,7 +281,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
             load_x(m, xv);
 #pragma unroll
             for (int p = 0; p < 2; ++p) {
-                if (p >= d.npaths) continue;
+                if (p >= npaths) continue;
                 const int E = sE[p * 16 + m];
                 int qs = 0;
 #pragma unroll
@@ -341,302 +310,307 @@ __global__ void __launch_bounds__(kDecodeThreads)
             }
         }
         __syncthreads();
-        if (tid < d.npaths * M) {
+        // sum over this chunk of t (per path, row m), and non-finite flags
+        if (tid < npaths * M) {
             const int p = tid / M, m = tid - p * M;
-            d.pmeta[(kc * 2 + p) * 16 + m] = make_int2(sE[p * 16 + m], sQs[p * 16 + m]);
+            const int E = sE[p * 16 + m];
+            if (E == kNanExp) atomicOr(reinterpret_cast<int *>(acc + (size_t)dp->R1 * 16 + 32) + p * 16 + m, 1);
+            else if (sQs[p * 16 + m]) atomicAdd(acc + (size_t)dp->R1 * 16 + p * 16 + m, ldexp((double)sQs[p * 16 + m], -E));
         }
 
-        // ---- main stream: units (row group, k-block) of this chunk, split evenly over the warps
-        const int U1 = d.RG1 * nkb;
-        const int ub = (int)((long long)U1 * warp / NW), ue = (int)((long long)U1 * (warp + 1) / NW);
-        int acc[4][NT][4];
-#pragma unroll
-        for (int rb = 0; rb < 4; ++rb)
-#pragma unroll
-            for (int n = 0; n < NT; ++n)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc[rb][n][c] = 0;
-        int lrg = ub / nkb, lkb = ub - lrg * nkb;     // load cursor
-        int prg = lrg, pkb = lkb;                     // process cursor
-        int nload = ue - ub, nproc = ue - ub;
-        int prb[4];
-        auto set_paths = [&](int rg) {
+        // ---- main stream: this warp's row groups of 64 latent rows
+        for (int rg = warp; rg < RG1; rg += NW) {
+            const int st = consumed % kP1Stages;
+            const uint32_t ph = (consumed / kP1Stages) & 1;
+            if (!ring_wait(&bars[warp][st], ph, err)) return;
+            ++consumed;
+            const uint2 *src = reinterpret_cast<const uint2 *>(my_ring + st * kStage) + lane;
+            int prb[4];
 #pragma unroll
             for (int rb = 0; rb < 4; ++rb)
-                prb[rb] = min((rg * kRowsPerGroup + rb * kRowsPerBlock) / d.r16, d.npaths - 1);
-        };
-        set_paths(prg);
-        auto flush = [&](int rg) {
+                prb[rb] = min((rg * kRowsPerGroup + rb * kRowsPerBlock) / r16, npaths - 1);
+            int a4[4][NT][4];
+#pragma unroll
+            for (int rb = 0; rb < 4; ++rb)
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) a4[rb][n][c] = 0;
+#pragma unroll 4
+            for (int kb = 0; kb < nkb; ++kb) {
+                const uint2 w = src[kb * 32];
+                uint2 bp[2][NT];
+#pragma unroll
+                for (int p = 0; p < 2; ++p)
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) bp[p][n] = sB[(((size_t)p * kP1ChunkKB + kb) * NT + n) * 32 + lane];
+#pragma unroll
+                for (int rb = 0; rb < 4; ++rb) {
+                    const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                    const uint32_t a0 = w.x & mlo, a1 = w.x & mhi, a2 = w.y & mlo, a3 = w.y & mhi;
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+                        const uint2 b = prb[rb] ? bp[1][n] : bp[0][n];
+                        mma_u8s8(a4[rb][n], a0, a1, a2, a3, b.x, b.y);
+                    }
+                }
+            }
+            // buffer consumed: refill it with this warp's row group kP1Stages ahead
+            __syncwarp();
+            if (lane == 0) {
+                const int rgn = rg + NW * kP1Stages;
+                if (rgn < RG1) {
+                    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                    const int sn = issued % kP1Stages;
+                    ring_fill(my_ring + sn * kStage, vt + ((size_t)rgn * KB1 + kb0) * 32, stage_bytes, &bars[warp][sn]);
+                    ++issued;
+                }
+            }
+            // sum_k b * t for rows g (scale 2^rb) and g + 8 (scale 2^(rb+4)), times 2^-E
 #pragma unroll
             for (int rb = 0; rb < 4; ++rb)
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
                     const int m = 4 * n + t4;
                     if (m < M) {
-                        const int Tlo = (acc[rb][n][0] >> rb) + 256 * (acc[rb][n][1] >> rb);
-                        const int Thi = (acc[rb][n][2] >> (rb + 4)) + 256 * (acc[rb][n][3] >> (rb + 4));
+                        const int E = sE[prb[rb] * 16 + m];
+                        if (E == kNanExp) continue;
+                        const int Tlo = (a4[rb][n][0] >> rb) + 256 * (a4[rb][n][1] >> rb);
+                        const int Thi = (a4[rb][n][2] >> (rb + 4)) + 256 * (a4[rb][n][3] >> (rb + 4));
                         const int row = rg * kRowsPerGroup + rb * kRowsPerBlock + g;
-                        if (Tlo) atomicAdd(&d.partT[((size_t)kc * d.R1 + row) * 16 + m], Tlo);
-                        if (Thi) atomicAdd(&d.partT[((size_t)kc * d.R1 + row + 8) * 16 + m], Thi);
-                    }
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) acc[rb][n][c] = 0;
-                }
-        };
-        constexpr int B = 8;
-        uint2 bufA[B], bufB[B];
-        auto load_batch = [&](uint2 (&buf)[B]) {
-#pragma unroll
-            for (int i = 0; i < B; ++i) {
-                if (nload > 0) {
-                    buf[i] = ld_stream_u2(d.vt + ((size_t)lrg * d.KB1 + kb0 + lkb) * 32 + lane);
-                    if (++lkb == nkb) { lkb = 0; ++lrg; }
-                    --nload;
-                }
-            }
-        };
-        auto proc_batch = [&](const uint2 (&buf)[B]) {
-#pragma unroll
-            for (int i = 0; i < B; ++i) {
-                if (nproc > 0) {
-                    const uint2 w = buf[i];
-                    uint2 bp[2][NT];
-#pragma unroll
-                    for (int p = 0; p < 2; ++p)
-#pragma unroll
-                        for (int n = 0; n < NT; ++n)
-                            bp[p][n] = sB[(((size_t)p * kP1ChunkKB + pkb) * NT + n) * 32 + lane];
-#pragma unroll
-                    for (int rb = 0; rb < 4; ++rb) {
-                        const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                        const uint32_t a0 = w.x & mlo, a1 = w.x & mhi, a2 = w.y & mlo, a3 = w.y & mhi;
-#pragma unroll
-                        for (int n = 0; n < NT; ++n) {
-                            const uint2 b = prb[rb] ? bp[1][n] : bp[0][n];
-                            mma_u8s8(acc[rb][n], a0, a1, a2, a3, b.x, b.y);
-                        }
-                    }
-                    --nproc;
-                    if (++pkb == nkb) {
-                        flush(prg);
-                        pkb = 0;
-                        ++prg;
-                        set_paths(prg);
+                        if (Tlo) atomicAdd(acc + (size_t)row * 16 + m, ldexp((double)Tlo, -E));
+                        if (Thi) atomicAdd(acc + (size_t)(row + 8) * 16 + m, ldexp((double)Thi, -E));
                     }
                 }
-            }
-        };
-        load_batch(bufA);
-        load_batch(bufB);
-        while (nproc > 0) {
-            proc_batch(bufA);
-            load_batch(bufA);
-            proc_batch(bufB);
-            load_batch(bufB);
         }
-        if (pkb != 0) flush(prg);
-
-        // ---- completion count; the last item of the layer finishes the latent vector
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) sLast = (atomicAdd(d.counter, 1u) == (unsigned)(d.nkc - 1));
-        __syncthreads();
-        if (sLast) {
-            __threadfence();
-            finish_latent(d, M, NT, sE, sQs, sMax, sBad);
-            __syncthreads();
-            if (tid == 0) atomicExch(d.counter, 0u);
-        }
+        __syncthreads();   // shared fragments are rebuilt by the next item
     }
 }
 
 // ---------------------------------------------------------------------------
-// Contraction 2 (+ h, + path sum)
+// Contraction 2 (+ l, + h, + path sum)
 // ---------------------------------------------------------------------------
 template <int NT>
 __global__ void __launch_bounds__(kDecodeThreads)
-    contraction2_kernel(const LayerDev *__restrict__ layers, const P2Item *__restrict__ items,
-                        int nitems, const __grid_constant__ IoPtrs io, int base, int M)
+    contraction2_kernel(const LayerDev *__restrict__ layers, const P2Item *__restrict__ items, int nitems,
+                        const __grid_constant__ IoPtrs io, int base, int M, int parity, int kb2max, int *err)
 {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    uint2 *sB = (uint2 *)smem_raw;              // [NT][KB2][32]
-    __shared__ LayerDev sd;
-    __shared__ int2 sMeta[32];
+    constexpr int NW = kDecodeThreads / 32;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const int kStage = kb2max * 256;
+    unsigned char *ring = smem_raw;                                          // [NW][kP2Stages][kStage]
+    uint2 *sB = (uint2 *)(smem_raw + (size_t)NW * kP2Stages * kStage);      // [NT][KB2][32]
+    __shared__ uint64_t bars[NW][kP2Stages];
+    __shared__ float sMax[32];
+    __shared__ int sBad[32], sE[32], sQs[32];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr int NW = kDecodeThreads / 32;
     const int g = lane >> 2, t4 = lane & 3;
+    if (lane == 0)
+        for (int s = 0; s < kP2Stages; ++s) bar_init(&bars[warp][s]);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    __syncwarp();
+    uint32_t issued = 0, consumed = 0;
+    unsigned char *my_ring = ring + (size_t)warp * kP2Stages * kStage;
 
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
         const P2Item item = items[it];
-        __syncthreads();   // previous item's readers of shared state are done
-        copy_desc(sd, layers + item.layer);
-        __syncthreads();
-        const LayerDev &d = sd;
+        const LayerDev *dp = layers + item.layer;
+        const int N = dp->N, N64 = dp->N64, KB2 = dp->KB2, r = dp->r, r16 = dp->r16, r32 = dp->r32;
+        const int npaths = dp->npaths, R1 = dp->R1;
+        const uint2 *__restrict__ ut = dp->ut;
+        const __half *__restrict__ hsc = dp->h;
+        const __half *__restrict__ lsc = dp->l;
+        const double *__restrict__ acc = dp->acc[parity];
         float *__restrict__ y = io.y[item.layer - base];
-        {
-            const uint4 *src = reinterpret_cast<const uint4 *>(d.zfrag);
-            uint4 *dst = reinterpret_cast<uint4 *>(sB);
-            const int n16 = NT * d.KB2 * 32 * (int)sizeof(uint2) / 16;
-            for (int i = tid; i < n16; i += kDecodeThreads) dst[i] = __ldcg(src + i);
+        const unsigned stage_bytes = (unsigned)KB2 * 256u;
+
+        if (lane == 0)
+            for (int s = 0; s < kP2Stages; ++s) {
+                const int rg = item.rg0 + warp + NW * s;
+                if (rg < item.rg1) {
+                    const int st = issued % kP2Stages;
+                    ring_fill(my_ring + (size_t)st * kStage, ut + (size_t)rg * KB2 * 32, stage_bytes, &bars[warp][st]);
+                    ++issued;
+                }
+            }
+        if (tid < 32) {
+            sMax[tid] = 0.0f;
+            sBad[tid] = 0;
+            sQs[tid] = 0;
         }
-        if (tid < 32) sMeta[tid] = __ldcg(&d.zmeta[tid]);
         __syncthreads();
 
-        const int kbp = d.r32 / kKPerBlock;   // k-blocks per path
-        const int KB2 = d.KB2;
-        const int nrg = (item.rg1 - item.rg0 - warp + NW - 1) / NW;   // this warp's row groups
-        int nload = max(0, nrg) * KB2, nproc = nload;
-        int lrg = item.rg0 + warp, lkb = 0;
-        int prg = lrg, pkb = 0;
-        int acc[4][NT][4];
-        float yv[4][NT][2];
-        float hv[2][4][2];
+        // ---- zl = (sum t - 2 sum b t) (.) l per (path, row m), its largest magnitude
+        const double *S = acc + (size_t)R1 * 16;
+        const int *badf = reinterpret_cast<const int *>(acc + (size_t)R1 * 16 + 32);
+        auto zl_at = [&](int p, int j, int m) -> float {
+            const double z = __ldcg(S + p * 16 + m) - 2.0 * __ldcg(acc + (size_t)(p * r16 + j) * 16 + m);
+            return (float)z * __half2float(lsc[p * r16 + j]);
+        };
+        for (int e = tid; e < npaths * r * M; e += kDecodeThreads) {
+            const int m = e % M, pj = e / M;
+            const int p = pj / r, j = pj - p * r;
+            const float zl = zl_at(p, j, m);
+            if (!(fabsf(zl) <= FLT_MAX)) atomicOr(&sBad[p * 16 + m], 1);
+            else smem_max(&sMax[p * 16 + m], fabsf(zl));
+        }
+        __syncthreads();
+        if (tid < npaths * M) {
+            const int p = tid / M, m = tid - p * M;
+            sE[p * 16 + m] = exponent_for(sMax[p * 16 + m], sBad[p * 16 + m] != 0 || __ldcg(badf + p * 16 + m) != 0);
+        }
+        __syncthreads();
+        // ---- digits into B fragments (rows m in [M, 4*NT) get zeros)
+        {
+            const int MT = 4 * NT, ngrp = r32 / 4;
+            for (int e = tid; e < npaths * MT * ngrp; e += kDecodeThreads) {
+                const int c = e % ngrp, pm = e / ngrp;
+                const int p = pm / MT, m = pm - p * MT;
+                uint32_t wlo = 0, whi = 0;
+                int qs = 0;
+                if (m < M) {
+                    const int E = sE[p * 16 + m];
 #pragma unroll
-        for (int rb = 0; rb < 4; ++rb)
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                yv[rb][n][0] = yv[rb][n][1] = 0.0f;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc[rb][n][c] = 0;
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = 4 * c + u;
+                        const int q = (j < r) ? quantize(zl_at(p, j, m), E) : 0;
+                        int lo, hi;
+                        digits(q, lo, hi);
+                        wlo |= (uint32_t)(lo & 255) << (8 * u);
+                        whi |= (uint32_t)(hi & 255) << (8 * u);
+                        qs += q;
+                    }
+                    if (qs) atomicAdd(&sQs[p * 16 + m], qs);
+                }
+                const int jj = p * r32 + 4 * c;
+                int llo, lhi, word;
+                frag_slot(m, jj & 31, llo, lhi, word);
+                uint2 *fb = sB + ((size_t)(m >> 2) * KB2 + (jj >> 5)) * 32;
+                set_word(fb[llo], word, wlo);
+                set_word(fb[lhi], word, whi);
             }
-        auto load_h = [&](int rg) {
+        }
+        // the first item of a layer clears the other parity for the next call
+        if (item.rg0 == 0) {
+            double *o = dp->acc[parity ^ 1];
+            const int n = (int)acc_doubles(R1);
+            for (int i = tid; i < n; i += kDecodeThreads) o[i] = 0.0;
+        }
+        __syncthreads();
+
+        // ---- main stream: this warp's row groups of 64 outputs
+        const int kbp = r32 / kKPerBlock;
+        for (int rg = item.rg0 + warp; rg < item.rg1; rg += NW) {
+            const int st = consumed % kP2Stages;
+            const uint32_t ph = (consumed / kP2Stages) & 1;
+            float hv[2][4][2];
 #pragma unroll
             for (int p = 0; p < 2; ++p)
 #pragma unroll
                 for (int rb = 0; rb < 4; ++rb) {
                     const int n = rg * kRowsPerGroup + rb * kRowsPerBlock + g;
-                    const bool ok = p < d.npaths && rg < item.rg1;
-                    hv[p][rb][0] = ok ? __half2float(d.h[p * d.N64 + n]) : 0.0f;
-                    hv[p][rb][1] = ok ? __half2float(d.h[p * d.N64 + n + 8]) : 0.0f;
+                    hv[p][rb][0] = (p < npaths) ? __half2float(hsc[p * N64 + n]) : 0.0f;
+                    hv[p][rb][1] = (p < npaths) ? __half2float(hsc[p * N64 + n + 8]) : 0.0f;
                 }
-        };
-        load_h(prg);
-        auto fold = [&](int p) {
+            if (!ring_wait(&bars[warp][st], ph, err)) return;
+            ++consumed;
+            const uint2 *src = reinterpret_cast<const uint2 *>(my_ring + (size_t)st * kStage) + lane;
+            float yv[4][NT][2];
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                const int m = 4 * n + t4;
-                const int2 meta = (m < M) ? sMeta[p * 16 + m] : make_int2(0, 0);
+            for (int rb = 0; rb < 4; ++rb)
 #pragma unroll
-                for (int rb = 0; rb < 4; ++rb) {
-                    const int Tlo = (acc[rb][n][0] >> rb) + 256 * (acc[rb][n][1] >> rb);
-                    const int Thi = (acc[rb][n][2] >> (rb + 4)) + 256 * (acc[rb][n][3] >> (rb + 4));
-                    float slo, shi;
-                    if (meta.x == kNanExp) {
-                        slo = shi = __int_as_float(0x7fc00000);
-                    } else {
-                        slo = ldexpf((float)(meta.y - 2 * Tlo), -meta.x);
-                        shi = ldexpf((float)(meta.y - 2 * Thi), -meta.x);
-                    }
-                    yv[rb][n][0] += (p ? hv[1][rb][0] : hv[0][rb][0]) * slo;
-                    yv[rb][n][1] += (p ? hv[1][rb][1] : hv[0][rb][1]) * shi;
+                for (int n = 0; n < NT; ++n) yv[rb][n][0] = yv[rb][n][1] = 0.0f;
+            for (int p = 0; p < npaths; ++p) {
+                int a4[4][NT][4];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) acc[rb][n][c] = 0;
-                }
-            }
-        };
-        auto store = [&](int rg) {
+                for (int rb = 0; rb < 4; ++rb)
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                const int m = 4 * n + t4;
+                    for (int n = 0; n < NT; ++n)
 #pragma unroll
-                for (int rb = 0; rb < 4; ++rb) {
-                    const int nlo = rg * kRowsPerGroup + rb * kRowsPerBlock + g;
-                    if (m < M) {
-                        if (nlo < d.N) y[(size_t)m * d.N + nlo] = yv[rb][n][0];
-                        if (nlo + 8 < d.N) y[(size_t)m * d.N + nlo + 8] = yv[rb][n][1];
-                    }
-                    yv[rb][n][0] = yv[rb][n][1] = 0.0f;
-                }
-            }
-        };
-        constexpr int B = 8;
-        uint2 bufA[B], bufB[B];
-        auto load_batch = [&](uint2 (&buf)[B]) {
-#pragma unroll
-            for (int i = 0; i < B; ++i) {
-                if (nload > 0) {
-                    buf[i] = ld_stream_u2(d.ut + ((size_t)lrg * KB2 + lkb) * 32 + lane);
-                    if (++lkb == KB2) { lkb = 0; lrg += NW; }
-                    --nload;
-                }
-            }
-        };
-        auto proc_batch = [&](const uint2 (&buf)[B]) {
-#pragma unroll
-            for (int i = 0; i < B; ++i) {
-                if (nproc > 0) {
-                    const uint2 w = buf[i];
+                        for (int c = 0; c < 4; ++c) a4[rb][n][c] = 0;
+#pragma unroll 4
+                for (int kb = p * kbp; kb < (p + 1) * kbp; ++kb) {
+                    const uint2 w = src[kb * 32];
                     uint2 b[NT];
 #pragma unroll
-                    for (int n = 0; n < NT; ++n) b[n] = sB[((size_t)n * KB2 + pkb) * 32 + lane];
+                    for (int n = 0; n < NT; ++n) b[n] = sB[((size_t)n * KB2 + kb) * 32 + lane];
 #pragma unroll
                     for (int rb = 0; rb < 4; ++rb) {
                         const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
                         const uint32_t a0 = w.x & mlo, a1 = w.x & mhi, a2 = w.y & mlo, a3 = w.y & mhi;
 #pragma unroll
-                        for (int n = 0; n < NT; ++n) mma_u8s8(acc[rb][n], a0, a1, a2, a3, b[n].x, b[n].y);
+                        for (int n = 0; n < NT; ++n) mma_u8s8(a4[rb][n], a0, a1, a2, a3, b[n].x, b[n].y);
                     }
-                    --nproc;
-                    ++pkb;
-                    if (pkb % kbp == 0) fold(pkb / kbp - 1);
-                    if (pkb == KB2) {
-                        store(prg);
-                        pkb = 0;
-                        prg += NW;
-                        load_h(prg);
+                }
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    const int m = 4 * n + t4;
+                    const int E = (m < M) ? sE[p * 16 + m] : 0;
+                    const int Q = (m < M) ? sQs[p * 16 + m] : 0;
+#pragma unroll
+                    for (int rb = 0; rb < 4; ++rb) {
+                        const int Tlo = (a4[rb][n][0] >> rb) + 256 * (a4[rb][n][1] >> rb);
+                        const int Thi = (a4[rb][n][2] >> (rb + 4)) + 256 * (a4[rb][n][3] >> (rb + 4));
+                        float slo, shi;
+                        if (E == kNanExp) {
+                            slo = shi = __int_as_float(0x7fc00000);
+                        } else {
+                            slo = ldexpf((float)(Q - 2 * Tlo), -E);
+                            shi = ldexpf((float)(Q - 2 * Thi), -E);
+                        }
+                        yv[rb][n][0] += (p ? hv[1][rb][0] : hv[0][rb][0]) * slo;
+                        yv[rb][n][1] += (p ? hv[1][rb][1] : hv[0][rb][1]) * shi;
                     }
                 }
             }
-        };
-        load_batch(bufA);
-        load_batch(bufB);
-        while (nproc > 0) {
-            proc_batch(bufA);
-            load_batch(bufA);
-            proc_batch(bufB);
-            load_batch(bufB);
+            __syncwarp();
+            if (lane == 0) {
+                const int rgn = rg + NW * kP2Stages;
+                if (rgn < item.rg1) {
+                    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                    const int sn = issued % kP2Stages;
+                    ring_fill(my_ring + (size_t)sn * kStage, ut + (size_t)rgn * KB2 * 32, stage_bytes, &bars[warp][sn]);
+                    ++issued;
+                }
+            }
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const int m = 4 * n + t4;
+                if (m < M) {
+#pragma unroll
+                    for (int rb = 0; rb < 4; ++rb) {
+                        const int nlo = rg * kRowsPerGroup + rb * kRowsPerBlock + g;
+                        if (nlo < N) y[(size_t)m * N + nlo] = yv[rb][n][0];
+                        if (nlo + 8 < N) y[(size_t)m * N + nlo + 8] = yv[rb][n][1];
+                    }
+                }
+            }
         }
+        __syncthreads();   // shared fragments are rebuilt by the next item
     }
 }
 
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-struct DecodeLaunch {
-    void (*k1)(const LayerDev *, const P1Item *, int, const IoPtrs, int, int);
-    void (*k2)(const LayerDev *, const P2Item *, int, const IoPtrs, int, int);
-    int occ1 = 0, occ2 = 0;
-    size_t smem1 = 0, smem2_cap = 0;
-    bool ready = false;
-};
-
-static DecodeLaunch g_launch[kMaxNT + 1];
-static int g_sms = 0;
+typedef void (*K1Fn)(const LayerDev *, const P1Item *, int, const IoPtrs, int, int, int, int *);
+typedef void (*K2Fn)(const LayerDev *, const P2Item *, int, const IoPtrs, int, int, int, int, int *);
 
 template <int NT>
-static cudaError_t prepare(DecodeLaunch &L)
+static void kernels_for(K1Fn &k1, K2Fn &k2)
 {
-    if (L.ready) return cudaSuccess;
-    L.k1 = contraction1_kernel<NT>;
-    L.k2 = contraction2_kernel<NT>;
-    L.smem1 = (size_t)2 * kP1ChunkKB * NT * 32 * sizeof(uint2);
-    // contraction-2 fragments: up to LB_MAX_RANK latent indices per path
-    L.smem2_cap = (size_t)(2 * LB_MAX_RANK / kKPerBlock) * NT * 32 * sizeof(uint2);
-    cudaError_t e = cudaFuncSetAttribute(L.k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem1);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(L.k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem2_cap);
-    if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&L.occ1, L.k1, kDecodeThreads, L.smem1);
-    if (e != cudaSuccess) return e;
-    L.ready = true;
-    return cudaSuccess;
+    k1 = contraction1_kernel<NT>;
+    k2 = contraction2_kernel<NT>;
 }
 
-lb_status decode_forward(const Plan &P, const uint16_t *const *xs, float *const *ys, int M,
-                         cudaStream_t s, int *launches)
+static int g_sms = 0;
+static int g_smem_set1[kMaxNT + 1] = {0}, g_smem_set2[kMaxNT + 1] = {0};
+
+lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const *ys, int M, cudaStream_t s,
+                         int *launches)
 {
-    *launches = 0;
+    Plan &P = const_cast<Plan &>(Pc);
     if (M > kMaxDecodeM) {
         // Rows beyond the decode limit run as consecutive blocks of 16 rows.
         std::vector<const uint16_t *> xc(P.n);
@@ -646,9 +620,7 @@ lb_status decode_forward(const Plan &P, const uint16_t *const *xs, float *const 
                 xc[i] = xs[i] + (size_t)m0 * P.host[i].K;
                 yc[i] = ys[i] + (size_t)m0 * P.host[i].N;
             }
-            int l = 0;
-            lb_status st = decode_forward(P, xc.data(), yc.data(), std::min(kMaxDecodeM, M - m0), s, &l);
-            *launches += l;
+            lb_status st = decode_forward(P, xc.data(), yc.data(), std::min(kMaxDecodeM, M - m0), s, launches);
             if (st != LB_OK) return st;
         }
         return LB_OK;
@@ -661,24 +633,40 @@ lb_status decode_forward(const Plan &P, const uint16_t *const *xs, float *const 
         if ((e = cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
             return status_from(e);
     }
-    DecodeLaunch &L = g_launch[NT];
+    K1Fn k1;
+    K2Fn k2;
     switch (NT) {
-    case 1: e = prepare<1>(L); break;
-    case 2: e = prepare<2>(L); break;
-    case 3: e = prepare<3>(L); break;
-    default: e = prepare<4>(L); break;
+    case 1: kernels_for<1>(k1, k2); break;
+    case 2: kernels_for<2>(k1, k2); break;
+    case 3: kernels_for<3>(k1, k2); break;
+    default: kernels_for<4>(k1, k2); break;
     }
-    if (e != cudaSuccess) return status_from(e);
-
-    int maxKB2 = 0;
-    for (const LayerDev &d : P.host) maxKB2 = std::max(maxKB2, d.KB2);
-    const size_t smem2 = (size_t)maxKB2 * NT * 32 * sizeof(uint2);
-    int occ2 = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ2, L.k2, kDecodeThreads, smem2)) != cudaSuccess)
+    int kb2max = 0;
+    for (const LayerDev &d : P.host) kb2max = std::max(kb2max, d.KB2);
+    const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * kP1ChunkKB * 256 +
+                         (size_t)2 * kP1ChunkKB * NT * 32 * sizeof(uint2);
+    const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * kb2max * 256 +
+                         (size_t)NT * kb2max * 32 * sizeof(uint2);
+    if (smem2 > 227 * 1024) return LB_ERR_UNSUPPORTED;
+    if ((int)smem1 > g_smem_set1[NT]) {
+        if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) != cudaSuccess)
+            return status_from(e);
+        g_smem_set1[NT] = (int)smem1;
+    }
+    if ((int)smem2 > g_smem_set2[NT]) {
+        if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)) != cudaSuccess)
+            return status_from(e);
+        g_smem_set2[NT] = (int)smem2;
+    }
+    int occ1 = 0, occ2 = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, k1, kDecodeThreads, smem1)) != cudaSuccess)
         return status_from(e);
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ2, k2, kDecodeThreads, smem2)) != cudaSuccess)
+        return status_from(e);
+    occ1 = std::max(1, occ1);
     occ2 = std::max(1, occ2);
-    const int occ1 = std::max(1, L.occ1);
 
+    const int parity = (int)(P.calls & 1);
     static thread_local IoPtrs io;
     profile_mark(0, s);
     const int nb = (int)P.p1_start.size() - 1;
@@ -693,11 +681,12 @@ lb_status decode_forward(const Plan &P, const uint16_t *const *xs, float *const 
         const int n2 = P.p2_start[b + 1] - P.p2_start[b];
         const int grid1 = std::max(1, std::min(n1, g_sms * occ1));
         const int grid2 = std::max(1, std::min(n2, g_sms * occ2));
-        L.k1<<<grid1, kDecodeThreads, L.smem1, s>>>(P.dev, P.p1 + P.p1_start[b], n1, io, base, M);
+        k1<<<grid1, kDecodeThreads, smem1, s>>>(P.dev, P.p1 + P.p1_start[b], n1, io, base, M, parity, P.err);
         profile_mark(++*launches, s);
-        L.k2<<<grid2, kDecodeThreads, smem2, s>>>(P.dev, P.p2 + P.p2_start[b], n2, io, base, M);
+        k2<<<grid2, kDecodeThreads, smem2, s>>>(P.dev, P.p2 + P.p2_start[b], n2, io, base, M, parity, kb2max, P.err);
         profile_mark(++*launches, s);
     }
+    ++P.calls;
     e = cudaGetLastError();
     return status_from(e);
 }

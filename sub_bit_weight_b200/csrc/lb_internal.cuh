@@ -40,6 +40,11 @@ constexpr int kDecodeThreads = 128;     // 4 warps
 constexpr int kMaxDecodeM = LB_DECODE_MAX_M;
 constexpr int kMaxNT = (kMaxDecodeM + 3) / 4;   // n-tiles of 4 activation rows
 constexpr int kIoBatch = 1024;          // layers per launch (pointer tables ride in kernel params)
+constexpr int kP1Stages = 2;            // per-warp bulk-copy ring depth, contraction 1
+constexpr int kP2Stages = 3;            // per-warp bulk-copy ring depth, contraction 2
+
+// doubles in one parity block of a layer's scratch
+__host__ __device__ inline size_t acc_doubles(int R1) { return (size_t)R1 * 16 + 32 + 16; }
 
 static inline int round_up(int a, int b) { return (a + b - 1) / b * b; }
 static inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -58,13 +63,11 @@ struct LayerDev {
     const __half *g;    // [npaths][K32], zero padded
     const __half *h;    // [npaths][N64], zero padded
     const __half *l;    // [npaths][r16], zero padded
-    // scratch (owned by the plan that holds this descriptor)
-    int *partT;         // [nkc][R1][16]   integer partial sums of contraction 1
-    int2 *pmeta;        // [nkc][2][16]    (exponent, digit sum) of each chunk
-    float *zl;          // [R1][16]        latent vector after l
-    uint2 *zfrag;       // [kMaxNT][KB2][32] B fragments of contraction 2
-    int2 *zmeta;        // [2][16]         (exponent, digit sum) of zl
-    unsigned *counter;  // chunks of contraction 1 finished (self-resetting)
+    // scratch (owned by the plan that holds this descriptor), one block per call parity:
+    //   [R1][16] double  sum over k of b * t (contraction-1 rows x activation rows)
+    //   [2][16]  double  sum over k of t (per path x activation row)
+    //   [2][16]  int     non-finite flags (per path x activation row)
+    double *acc[2];
 };
 
 struct P1Item { int layer, kc; };
@@ -78,26 +81,35 @@ struct IoPtrs {
 // Sentinel exponent marking a non-finite activation block.
 constexpr int kNanExp = -0x40000000;
 
-// Host-side record of a layer (what lb_layer points to).
 }  // namespace lb
 
+#include "lb_prefill_types.cuh"
+
+// Host-side record of a layer (what lb_layer points to).
 struct lb_layer {
-    lb::LayerDev d;            // descriptor with pointers into `weights`
-    void *weights = nullptr;   // one allocation: tiles + scales
+    lb::LayerDev d;            // decode descriptor with pointers into `weights`
+    lb::PfWeights pf;          // tensor-core (prefill) layouts, pointers into `weights`
+    void *weights = nullptr;   // one allocation: all layouts + scales
     size_t weight_bytes = 0;
     struct lb_stack *self = nullptr;   // single-layer plan (owns scratch)
 };
 
 namespace lb {
 
+struct PrefillState;
+
 // A plan: descriptors + work items + scratch for a list of layers.
 struct Plan {
     int n = 0;
+    std::vector<const lb_layer *> layers;
+    PrefillState *pf = nullptr;     // tensor-core path state, created on first use
     std::vector<LayerDev> host;     // descriptors (scratch pointers filled in)
     LayerDev *dev = nullptr;        // device copy of `host`
     P1Item *p1 = nullptr;           // device work items
     P2Item *p2 = nullptr;
     std::vector<int> p1_start, p2_start;   // per IO batch: first item index
+    unsigned long long calls = 0;   // decode calls so far (selects the scratch parity)
+    int *err = nullptr;             // device error code (bounded waits that gave up)
     int n_p1 = 0, n_p2 = 0;
     void *scratch = nullptr;
     size_t scratch_bytes = 0;

@@ -10,7 +10,7 @@
 #include <cstring>
 #include <new>
 
-#include "lb_internal.cuh"
+#include "lb_prefill.cuh"
 
 namespace lb {
 
@@ -110,6 +110,7 @@ static int grid_for(int64_t work, int threads)
 
 void plan_free(Plan &P)
 {
+    prefill_free(P.pf);
     if (P.dev) cudaFree(P.dev);
     if (P.p1) cudaFree(P.p1);
     if (P.p2) cudaFree(P.p2);
@@ -120,6 +121,7 @@ void plan_free(Plan &P)
 cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream_t s)
 {
     P.n = n;
+    P.layers.assign(layers, layers + n);
     P.host.resize(n);
     // scratch layout
     std::vector<size_t> off(n);
@@ -127,13 +129,9 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
     for (int i = 0; i < n; ++i) {
         const LayerDev &d = layers[i]->d;
         off[i] = total;
-        total += align256((size_t)d.nkc * d.R1 * 16 * sizeof(int));
-        total += align256((size_t)d.nkc * 2 * 16 * sizeof(int2));
-        total += align256((size_t)d.R1 * 16 * sizeof(float));
-        total += align256((size_t)d.KB2 * kMaxNT * 32 * sizeof(uint2));
-        total += align256((size_t)2 * 16 * sizeof(int2));
-        total += align256(sizeof(unsigned));
+        total += 2 * align256(acc_doubles(d.R1) * sizeof(double));
     }
+    total += 256;   // error code
     cudaError_t e = cudaMalloc(&P.scratch, std::max<size_t>(total, 256));
     if (e != cudaSuccess) return e;
     P.scratch_bytes = total;
@@ -143,14 +141,13 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
     for (int i = 0; i < n; ++i) {
         LayerDev d = layers[i]->d;
         char *c = base + off[i];
-        d.partT = (int *)c;      c += align256((size_t)d.nkc * d.R1 * 16 * sizeof(int));
-        d.pmeta = (int2 *)c;     c += align256((size_t)d.nkc * 2 * 16 * sizeof(int2));
-        d.zl = (float *)c;       c += align256((size_t)d.R1 * 16 * sizeof(float));
-        d.zfrag = (uint2 *)c;    c += align256((size_t)d.KB2 * kMaxNT * 32 * sizeof(uint2));
-        d.zmeta = (int2 *)c;     c += align256((size_t)2 * 16 * sizeof(int2));
-        d.counter = (unsigned *)c;
+        for (int b = 0; b < 2; ++b) {
+            d.acc[b] = (double *)c;
+            c += align256(acc_doubles(d.R1) * sizeof(double));
+        }
         P.host[i] = d;
     }
+    P.err = (int *)(base + total - 256);
     // work items, layer-major; one IO batch per kIoBatch layers
     std::vector<P1Item> p1;
     std::vector<P2Item> p2;
@@ -184,6 +181,18 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
 }  // namespace lb
 
 using namespace lb;
+
+// M <= LB_DECODE_MAX_M: fused decode kernels.  Larger M: tensor-core kernels;
+// shapes those cannot take (K not a multiple of 8) run as 16-row decode blocks.
+static lb_status forward_any(const Plan &P, const uint16_t *const *xs, float *const *ys, int M, cudaStream_t s,
+                             int *launches)
+{
+    if (M > kMaxDecodeM) {
+        lb_status st = prefill_forward(P, P.layers.data(), xs, ys, M, s, launches);
+        if (st != LB_ERR_UNSUPPORTED) return st;
+    }
+    return decode_forward(P, xs, ys, M, s, launches);
+}
 
 extern "C" {
 
@@ -222,7 +231,8 @@ lb_status lb_layer_create(lb_layer **out, int N, int K, int r, int npaths, const
     const size_t b_g = align256((size_t)npaths * d.K32 * 2);
     const size_t b_h = align256((size_t)npaths * d.N64 * 2);
     const size_t b_l = align256((size_t)npaths * d.r16 * 2);
-    L->weight_bytes = b_vt + b_ut + b_g + b_h + b_l;
+    const size_t b_pf = prefill_weight_bytes(d);
+    L->weight_bytes = b_vt + b_ut + b_g + b_h + b_l + b_pf;
     cudaError_t e = cudaMalloc(&L->weights, L->weight_bytes);
     if (e != cudaSuccess) {
         delete L;
@@ -233,7 +243,8 @@ lb_status lb_layer_create(lb_layer **out, int N, int K, int r, int npaths, const
     d.ut = (const uint2 *)c;   c += b_ut;
     d.g = (const __half *)c;   c += b_g;
     d.h = (const __half *)c;   c += b_h;
-    d.l = (const __half *)c;
+    d.l = (const __half *)c;   c += b_l;
+    L->pf.b1 = (uint32_t *)c;  // prefill layouts are carved from here
 
     const int T = 256;
     const uint32_t *V1 = npaths > 1 ? V[1] : V[0];
@@ -251,6 +262,10 @@ lb_status lb_layer_create(lb_layer **out, int N, int K, int r, int npaths, const
         (uint16_t *)d.l, l[0], npaths > 1 ? l[1] : l[0], npaths, r, d.r16);
     launches = 5;
     e = cudaGetLastError();
+    if (e == cudaSuccess) {
+        e = prefill_build_weights(L->pf, d, U, V, h, g, l, s);
+        launches += 5;
+    }
     if (e == cudaSuccess) {
         lb_stack *S = new (std::nothrow) lb_stack();
         if (!S) {
@@ -317,7 +332,7 @@ lb_status lb_linear_forward(const uint16_t *x, int M, const lb_layer *L, float *
     const uint16_t *xs[1] = {x};
     float *ys[1] = {y};
     int launches = 0;
-    lb_status st = decode_forward(L->self->plan, xs, ys, M, (cudaStream_t)stream, &launches);
+    lb_status st = forward_any(L->self->plan, xs, ys, M, (cudaStream_t)stream, &launches);
     set_launch_count(launches);
     return st;
 }
@@ -361,7 +376,7 @@ lb_status lb_stack_forward(lb_stack *S, const uint16_t *const *xs, float *const 
         if (!xs[i] || !ys[i] || ((uintptr_t)xs[i] & 15) || ((uintptr_t)ys[i] & 15))
             return LB_ERR_INVALID_ARG;
     int launches = 0;
-    lb_status st = decode_forward(S->plan, xs, ys, M, (cudaStream_t)stream, &launches);
+    lb_status st = forward_any(S->plan, xs, ys, M, (cudaStream_t)stream, &launches);
     set_launch_count(launches);
     return st;
 }

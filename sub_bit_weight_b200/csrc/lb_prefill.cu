@@ -1,0 +1,791 @@
+// Large-batch (prefill) forward of LittleBit layers on 5th-generation tensor
+// cores (tcgen05, accumulators in tensor memory).
+//
+// With many activation rows the two binary contractions of a path
+// (LittleBit notes page, "Multi-scale compensation": x (.) g . V_sign (.) l
+// . U_sign^T (.) h) are dense skinny GEMMs, so they run as two fp16 x fp16 ->
+// fp32 tensor-core GEMMs whose weight operand is generated in shared memory
+// from the packed signs:
+//
+//   latent:  z[m][j'] = sum_k fp16(x[m][k]) * (+-g_p[k])     (+-g exact in fp16)
+//            zl = fp16(z * l_p[j])                            (both paths: j' = p*r8 + j)
+//   output:  y[m][n]  = sum_j' zl[m][j'] * (+-h_p(j')[n])    (both paths in one GEMM)
+//
+// Folding g and h into the generated operand keeps every product exact and
+// lets one accumulator carry both paths ("Residual compensation" sums them).
+//
+// Kernel structure (one persistent CTA per SM, 16 warps):
+//   warp 0      TMA producer: A tile (128 x 64, 128-byte swizzle) + the 4 KB
+//               block of packed signs of the B tile, one mbarrier per stage
+//   warp 1      tcgen05.mma issuer (one thread) and tensor-memory owner
+//   warps 4-7   epilogue: tcgen05.ld of the fp32 accumulator, scaling, stores
+//   warps 8-15  generators: B tile (256 x 64 fp16, 128-byte swizzle) from
+//               signs and scales; the latent GEMM also converts the bf16 A
+//               tile to fp16 in place
+// Two accumulators of 256 columns in tensor memory let the epilogue of one
+// tile overlap the main loop of the next.  Every wait is bounded: on timeout
+// the kernel records an error code and returns.
+
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "lb_prefill.cuh"
+
+namespace lb {
+
+// ---------------------------------------------------------------------------
+// Weight layouts (built once per layer)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t canon_bit_pf(const uint32_t *P, int wpr, int64_t row, int col)
+{
+    return (__ldg(P + row * wpr + (col >> 5)) >> (col & 31)) & 1u;
+}
+
+// Spread words of the latent-contraction operand: rows j' (path p = j'/r8),
+// k = inputs.  Bit = V_sign_p[k][j] < 0.
+__global__ void build_b1_kernel(uint32_t *__restrict__ out, int RT1, int KB1, int r, int r8, int K,
+                                int npaths, const uint32_t *__restrict__ V0, const uint32_t *__restrict__ V1)
+{
+    const int wpr = (r + 31) / 32;
+    const int64_t total = (int64_t)RT1 * KB1 * 256 * 4;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int q = (int)(idx & 3);
+        const int row = (int)((idx >> 2) & 255);
+        const int64_t blk = idx >> 10;
+        const int kb = (int)(blk % KB1), rt = (int)(blk / KB1);
+        const int jr = rt * 256 + row;
+        const int p = jr / r8, j = jr - p * r8;
+        uint32_t w = 0;
+        if (p < npaths && j < r) {
+            const uint32_t *V = p ? V1 : V0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int k0 = kb * 64 + 16 * q + 2 * i;
+                if (k0 < K) w |= canon_bit_pf(V, wpr, k0, j) << (15 - i);
+                if (k0 + 1 < K) w |= canon_bit_pf(V, wpr, k0 + 1, j) << (31 - i);
+            }
+        }
+        out[idx] = w;
+    }
+}
+
+// Spread words of the output-contraction operand: rows n, k = j' (path p = j'/r8).
+// Bit = U_sign_p[n][j] < 0.
+__global__ void build_b2_kernel(uint32_t *__restrict__ out, int RT2, int KB2, int r, int r8, int N,
+                                int npaths, const uint32_t *__restrict__ U0, const uint32_t *__restrict__ U1)
+{
+    const int wpr = (r + 31) / 32;
+    const int64_t total = (int64_t)RT2 * KB2 * 256 * 4;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int q = (int)(idx & 3);
+        const int row = (int)((idx >> 2) & 255);
+        const int64_t blk = idx >> 10;
+        const int kb = (int)(blk % KB2), rt = (int)(blk / KB2);
+        const int n = rt * 256 + row;
+        uint32_t w = 0;
+        if (n < N) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int jr = kb * 64 + 16 * q + 2 * i + h;
+                    const int p = jr / r8, j = jr - p * r8;
+                    if (p < npaths && j < r)
+                        w |= canon_bit_pf(p ? U1 : U0, wpr, n, j) << (h ? 31 - i : 15 - i);
+                }
+            }
+        }
+        out[idx] = w;
+    }
+}
+
+__global__ void pad_half_kernel(__half *__restrict__ dst, const uint16_t *__restrict__ s0,
+                                const uint16_t *__restrict__ s1, int npaths, int n, int npad)
+{
+    const int64_t total = (int64_t)npaths * npad;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int p = (int)(idx / npad), i = (int)(idx - (int64_t)p * npad);
+        dst[idx] = __ushort_as_half((i < n) ? (p ? s1 : s0)[i] : (uint16_t)0);
+    }
+}
+
+__global__ void lcat_kernel(float *__restrict__ dst, const uint16_t *__restrict__ l0,
+                            const uint16_t *__restrict__ l1, int npaths, int r, int r8, int n)
+{
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const int p = i / r8, j = i - p * r8;
+        float v = 0.0f;
+        if (p < npaths && j < r) v = __half2float(__ushort_as_half((p ? l1 : l0)[j]));
+        dst[i] = v;
+    }
+}
+
+static void pf_dims(PfWeights &W, const LayerDev &d)
+{
+    W.r8 = round_up(d.r, 8);
+    W.N1 = d.npaths * W.r8;
+    W.N1p = round_up(W.N1, 16);
+    W.K64 = round_up(d.K, 64);
+    W.KB1 = W.K64 / 64;
+    W.RT1 = ceil_div(W.N1p, 256);
+    W.K2 = round_up(W.N1p, 64);
+    W.KB2 = W.K2 / 64;
+    W.RT2 = ceil_div(d.N, 256);
+    W.N256 = W.RT2 * 256;
+}
+
+static size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+size_t prefill_weight_bytes(const LayerDev &d)
+{
+    PfWeights W;
+    pf_dims(W, d);
+    return al256((size_t)W.RT1 * W.KB1 * 4096) + al256((size_t)d.npaths * W.K64 * 2) +
+           al256((size_t)W.N1p * 4) + al256((size_t)W.RT2 * W.KB2 * 4096) + al256((size_t)d.npaths * W.N256 * 2);
+}
+
+cudaError_t prefill_build_weights(PfWeights &W, const LayerDev &d, const uint32_t *const *U,
+                                  const uint32_t *const *V, const uint16_t *const *h,
+                                  const uint16_t *const *g, const uint16_t *const *l, cudaStream_t s)
+{
+    // memory was carved by the caller: W.b1 points at the start of prefill_weight_bytes(d) bytes
+    pf_dims(W, d);
+    char *c = (char *)W.b1;
+    W.b1 = (uint32_t *)c;      c += al256((size_t)W.RT1 * W.KB1 * 4096);
+    W.g64 = (__half *)c;       c += al256((size_t)d.npaths * W.K64 * 2);
+    W.lcat = (float *)c;       c += al256((size_t)W.N1p * 4);
+    W.b2 = (uint32_t *)c;      c += al256((size_t)W.RT2 * W.KB2 * 4096);
+    W.h256 = (__half *)c;
+    const int P = d.npaths;
+    const int T = 256;
+    auto grid = [](int64_t n) { return (int)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 148 * 32)); };
+    build_b1_kernel<<<grid((int64_t)W.RT1 * W.KB1 * 1024), T, 0, s>>>(W.b1, W.RT1, W.KB1, d.r, W.r8, d.K, P, V[0],
+                                                                      P > 1 ? V[1] : V[0]);
+    build_b2_kernel<<<grid((int64_t)W.RT2 * W.KB2 * 1024), T, 0, s>>>(W.b2, W.RT2, W.KB2, d.r, W.r8, d.N, P, U[0],
+                                                                      P > 1 ? U[1] : U[0]);
+    pad_half_kernel<<<grid((int64_t)P * W.K64), T, 0, s>>>(W.g64, g[0], P > 1 ? g[1] : g[0], P, d.K, W.K64);
+    pad_half_kernel<<<grid((int64_t)P * W.N256), T, 0, s>>>(W.h256, h[0], P > 1 ? h[1] : h[0], P, d.N, W.N256);
+    lcat_kernel<<<grid(W.N1p), T, 0, s>>>(W.lcat, l[0], P > 1 ? l[1] : l[0], P, d.r, W.r8, W.N1p);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// PTX helpers: mbarrier, TMA, tcgen05
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *b, unsigned count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(b)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *b)
+{
+    asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(smem_u32(b)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, unsigned bytes)
+{
+    asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(smem_u32(b)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *b, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+                 : "=r"(ok)
+                 : "r"(smem_u32(b)), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+constexpr long long kWaitCycles = 4000000000LL;   // ~2 s at 2 GHz
+
+// Bounded wait.  Returns false (and raises the CTA's abort flag) on timeout
+// or when another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile int *abort, int *err, int code)
+{
+    if (mbar_try_wait(b, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(b, parity)) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > kWaitCycles) {
+            *abort = 1;
+            atomicCAS(err, 0, code);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
+            smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, unsigned bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate)
+{
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns per warp
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void *p)
+{
+    const uint64_t a = (uint64_t)(smem_u32(p) >> 4) & 0x3fff;
+    return a | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor: fp16 A and B (K-major), fp32 accumulator, M = 128.
+__device__ __forceinline__ uint32_t idesc_f16(int n)
+{
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kPfBM >> 4) << 24);
+}
+
+// Byte offset of 16-byte chunk c of row `row` in a 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t sw128(int row, int c)
+{
+    return (uint32_t)row * 128u + ((uint32_t)(c ^ (row & 7)) << 4);
+}
+
+// bf16x2 -> fp16x2 (exact for |x| in the normal fp16 range)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v)
+{
+    const float lo = __uint_as_float(v << 16);
+    const float hi = __uint_as_float(v & 0xffff0000u);
+    const __half2 hh = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&hh);
+}
+
+// ---------------------------------------------------------------------------
+// The tensor-core contraction kernel
+// ---------------------------------------------------------------------------
+struct PfSmem {
+    alignas(1024) unsigned char A[kPfStages][kPfBM * kPfBK * 2];
+    alignas(1024) unsigned char B[kPfStages][kPfBN * kPfBK * 2];
+    alignas(16) uint32_t bits[kPfStages][256 * 4];
+    uint64_t full[kPfStages], ready[kPfStages], empty[kPfStages];
+    uint64_t accf[2], acce[2];
+    uint32_t tmem_base;
+    int abort;
+    int tile_start[1];   // flexible: [nlayers + 1]
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kPfThreads, 1)
+    prefill_kernel(const PfLayer *__restrict__ layers, const int *__restrict__ tile_start, int nlayers, int M,
+                   int *err)
+{
+    extern __shared__ __align__(1024) unsigned char pf_raw[];
+    PfSmem &S = *reinterpret_cast<PfSmem *>((reinterpret_cast<uintptr_t>(pf_raw) + 1023) & ~(uintptr_t)1023);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    volatile int *abort = &S.abort;
+
+    for (int i = tid; i <= nlayers; i += blockDim.x) S.tile_start[i] = tile_start[i];
+    if (tid == 0) {
+        for (int s = 0; s < kPfStages; ++s) {
+            mbar_init(&S.full[s], 1);
+            mbar_init(&S.ready[s], 8);
+            mbar_init(&S.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&S.accf[b], 1);
+            mbar_init(&S.acce[b], 4);
+        }
+        S.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;\n" ::"r"(smem_u32(&S.tmem_base)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    const int total = S.tile_start[nlayers];
+
+    auto locate = [&](int t, int &L, int &mt, int &nt) {
+        int lo = 0, hi = nlayers - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (S.tile_start[mid] <= t) lo = mid; else hi = mid - 1;
+        }
+        L = lo;
+        const int local = t - S.tile_start[lo];
+        const int ntn = layers[lo].ntn;
+        mt = local / ntn;
+        nt = local - mt * ntn;
+    };
+
+    if (warp == 0) {
+        // ---------------- producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            uint32_t pend = 0, pend_ph = 0;   // stages with a copy issued, and its phase parity
+            for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
+                int L, mt, nt;
+                locate(t, L, mt, nt);
+                const PfLayer &ly = layers[L];
+                const uint32_t *bits = ly.bits + (size_t)nt * ly.nk * 1024;
+                for (int kb = 0; kb < ly.nk; ++kb, ++it) {
+                    const int s = it % kPfStages;
+                    const uint32_t ph = (it / kPfStages) & 1;
+                    if (!mbar_wait(&S.empty[s], ph ^ 1, abort, err, 1)) break;
+                    mbar_expect_tx(&S.full[s], kPfBM * kPfBK * 2 + 4096);
+                    tma_load_2d(S.A[s], ly.tmA, kb * kPfBK, mt * kPfBM, &S.full[s]);
+                    bulk_load(S.bits[s], bits + (size_t)kb * 1024, 4096, &S.full[s]);
+                    pend |= 1u << s;
+                    pend_ph = (pend_ph & ~(1u << s)) | (ph << s);
+                }
+            }
+            if (*abort) {
+                // let the copies already issued land before the CTA leaves (bounded)
+                for (int s = 0; s < kPfStages; ++s) {
+                    if (!(pend >> s & 1)) continue;
+                    const long long t0 = clock64();
+                    while (!mbar_try_wait(&S.full[s], (pend_ph >> s) & 1) && clock64() - t0 < kWaitCycles / 20) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0, tcount = 0;
+            for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x, ++tcount) {
+                int L, mt, nt;
+                locate(t, L, mt, nt);
+                const PfLayer &ly = layers[L];
+                const int nw = min(kPfBN, ly.ncols - nt * kPfBN);
+                const int ab = tcount & 1;
+                const uint32_t aph = (tcount >> 1) & 1;
+                if (!mbar_wait(&S.acce[ab], aph ^ 1, abort, err, 2)) break;
+                tc_fence_after();
+                const uint32_t idesc = idesc_f16((nw + 15) & ~15);
+                const uint32_t dacc = tmem + (uint32_t)(ab * kPfBN);
+                bool ok = true;
+                for (int kb = 0; kb < ly.nk; ++kb, ++it) {
+                    const int s = it % kPfStages;
+                    const uint32_t ph = (it / kPfStages) & 1;
+                    if (!mbar_wait(&S.full[s], ph, abort, err, 3) || !mbar_wait(&S.ready[s], ph, abort, err, 4)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = smem_desc_sw128(S.A[s]);
+                    const uint64_t bd = smem_desc_sw128(S.B[s]);
+#pragma unroll
+                    for (int kk = 0; kk < kPfBK / 16; ++kk)
+                        tc_mma_f16(dacc, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+                    tc_commit(&S.empty[s]);
+                }
+                if (!ok) break;
+                tc_commit(&S.accf[ab]);
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ---------------- epilogue
+        const int q = warp - 4;
+        uint32_t tcount = 0;
+        for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x, ++tcount) {
+            int L, mt, nt;
+            locate(t, L, mt, nt);
+            const PfLayer &ly = layers[L];
+            const int nw = min(kPfBN, ly.ncols - nt * kPfBN);
+            const int ab = tcount & 1;
+            const uint32_t aph = (tcount >> 1) & 1;
+            if (!mbar_wait(&S.accf[ab], aph, abort, err, 5)) break;
+            tc_fence_after();
+            const int m = mt * kPfBM + q * 32 + lane;
+            for (int ch = 0; ch < nw; ch += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * kPfBN + ch), v);
+                const int c0 = nt * kPfBN + ch;
+                if (m < M) {
+                    if (MODE == 0) {
+                        __half *out = reinterpret_cast<__half *>(ly.out) + (size_t)m * ly.ld_out + c0;
+                        uint32_t hw[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int c = c0 + 2 * i;
+                            const float a = (c < ly.ncols) ? __uint_as_float(v[2 * i]) * __ldg(ly.lcat + c) : 0.0f;
+                            const float b =
+                                (c + 1 < ly.ncols) ? __uint_as_float(v[2 * i + 1]) * __ldg(ly.lcat + c + 1) : 0.0f;
+                            const __half2 hh = __floats2half2_rn(a, b);
+                            hw[i] = *reinterpret_cast<const uint32_t *>(&hh);
+                        }
+                        if (c0 + 32 <= ly.ncols) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                reinterpret_cast<uint4 *>(out)[i] = make_uint4(hw[4 * i], hw[4 * i + 1], hw[4 * i + 2], hw[4 * i + 3]);
+                        } else {
+                            for (int i = 0; i < 16 && c0 + 2 * i < ly.ncols; ++i)
+                                reinterpret_cast<uint32_t *>(out)[i] = hw[i];
+                        }
+                    } else {
+                        float *out = reinterpret_cast<float *>(ly.out) + (size_t)m * ly.ld_out + c0;
+                        if (c0 + 32 <= ly.ncols && (ly.ld_out & 3) == 0) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                reinterpret_cast<uint4 *>(out)[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                        } else {
+                            for (int i = 0; i < 32 && c0 + i < ly.ncols; ++i) out[i] = __uint_as_float(v[i]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.acce[ab]);
+        }
+    } else if (warp >= 8) {
+        // ---------------- generators (256 threads)
+        const int gt = tid - 256;
+        const int gw = warp - 8;
+        uint32_t it = 0;
+        for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
+            int L, mt, nt;
+            locate(t, L, mt, nt);
+            const PfLayer &ly = layers[L];
+            const int nw = min(kPfBN, ly.ncols - nt * kPfBN);
+            // output contraction: this thread's row n and its two path scales
+            uint32_t hh[2] = {0u, 0u};
+            if (MODE == 1) {
+                const int n = nt * kPfBN + gt;
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    if (p < ly.npaths) {
+                        const uint16_t hb = __half_as_ushort(ly.base[(size_t)p * ly.base_ld + n]);
+                        hh[p] = (uint32_t)hb | ((uint32_t)hb << 16);
+                    }
+                }
+            }
+            bool ok = true;
+            for (int kb = 0; kb < ly.nk; ++kb, ++it) {
+                const int s = it % kPfStages;
+                const uint32_t ph = (it / kPfStages) & 1;
+                if (!mbar_wait(&S.full[s], ph, abort, err, 6)) {
+                    ok = false;
+                    break;
+                }
+                unsigned char *Bt = S.B[s];
+                const uint32_t *bits = S.bits[s];
+                if (MODE == 0) {
+                    // thread -> chunk c (8 inputs), rows gt/8 + 32 i
+                    const int c = gt & 7;
+                    const int k = kb * kPfBK + 8 * c;
+                    uint4 gb[2];
+#pragma unroll
+                    for (int p = 0; p < 2; ++p)
+                        gb[p] = (p < ly.npaths) ? __ldg(reinterpret_cast<const uint4 *>(ly.base + (size_t)p * ly.base_ld + k))
+                                                : make_uint4(0, 0, 0, 0);
+                    const int sh0 = 4 * (c & 1);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int row = (gt >> 3) + 32 * i;
+                        if (row < nw) {
+                            const int jr = nt * kPfBN + row;
+                            const uint4 base = (jr >= ly.r8 && ly.npaths > 1) ? gb[1] : gb[0];
+                            const uint32_t R = bits[row * 4 + (c >> 1)];
+                            uint4 o;
+                            o.x = ((R << (sh0 + 0)) & 0x80008000u) ^ base.x;
+                            o.y = ((R << (sh0 + 1)) & 0x80008000u) ^ base.y;
+                            o.z = ((R << (sh0 + 2)) & 0x80008000u) ^ base.z;
+                            o.w = ((R << (sh0 + 3)) & 0x80008000u) ^ base.w;
+                            *reinterpret_cast<uint4 *>(Bt + sw128(row, c)) = o;
+                        }
+                    }
+                    // A tile: bf16 -> fp16 in place (element positions are unchanged)
+                    unsigned char *At = S.A[s];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint4 *p4 = reinterpret_cast<uint4 *>(At) + gt + 256 * i;
+                        uint4 v = *p4;
+                        v.x = bf16x2_to_f16x2(v.x);
+                        v.y = bf16x2_to_f16x2(v.y);
+                        v.z = bf16x2_to_f16x2(v.z);
+                        v.w = bf16x2_to_f16x2(v.w);
+                        *p4 = v;
+                    }
+                } else {
+                    // thread -> row gt, all 8 chunks
+                    const int row = gt;
+                    if (row < nw) {
+                        const uint4 Rw = *reinterpret_cast<const uint4 *>(bits + row * 4);
+                        const uint32_t Rs[4] = {Rw.x, Rw.y, Rw.z, Rw.w};
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const int jr = kb * kPfBK + 8 * c;
+                            const uint32_t base = (jr >= ly.r8 && ly.npaths > 1) ? hh[1] : hh[0];
+                            const uint32_t R = Rs[c >> 1];
+                            const int sh0 = 4 * (c & 1);
+                            uint4 o;
+                            o.x = ((R << (sh0 + 0)) & 0x80008000u) ^ base;
+                            o.y = ((R << (sh0 + 1)) & 0x80008000u) ^ base;
+                            o.z = ((R << (sh0 + 2)) & 0x80008000u) ^ base;
+                            o.w = ((R << (sh0 + 3)) & 0x80008000u) ^ base;
+                            *reinterpret_cast<uint4 *>(Bt + sw128(row, c)) = o;
+                        }
+                    }
+                }
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.ready[s]);
+            }
+            if (!ok) break;
+            (void)gw;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;\n" ::"r"(tmem));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+static std::once_flag g_encode_once;
+
+static cudaError_t get_encoder()
+{
+    std::call_once(g_encode_once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *fn = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+    });
+    return g_encode ? cudaSuccess : cudaErrorNotSupported;
+}
+
+static bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, int cols, int rows)
+{
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {kPfBK, kPfBM};
+    cuuint32_t estr[2] = {1, 1};
+    return g_encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct PrefillState {
+    int M = 0;                       // rows the scratch was sized for
+    int lastM = -1;
+    std::vector<const void *> lastX, lastY;
+    void *zl = nullptr;              // latent activations of every layer, fp16 [M][K2]
+    std::vector<size_t> zl_off;
+    CUtensorMap *maps = nullptr;     // device: [2 * n] (x maps, zl maps), 64-byte aligned
+    PfLayer *rec = nullptr;          // device: [2 * n] (latent records, output records)
+    int *starts = nullptr;           // device: [2 * (n + 1)]
+    int *err = nullptr;              // device error code
+    int tiles[2] = {0, 0};
+};
+
+void prefill_free(PrefillState *st)
+{
+    if (!st) return;
+    cudaFree(st->zl);
+    cudaFree(st->maps);
+    cudaFree(st->rec);
+    cudaFree(st->starts);
+    cudaFree(st->err);
+    delete st;
+}
+
+static size_t smem_bytes(int nlayers) { return sizeof(PfSmem) + 1024 + sizeof(int) * (size_t)(nlayers + 1); }
+
+lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const uint16_t *const *xs,
+                          float *const *ys, int M, cudaStream_t s, int *launches)
+{
+    Plan &P = const_cast<Plan &>(Pc);
+    const int n = P.n;
+    cudaError_t e = get_encoder();
+    if (e != cudaSuccess) return LB_ERR_UNSUPPORTED;
+    for (int i = 0; i < n; ++i) {
+        const LayerDev &d = layers[i]->d;
+        if (d.K % 8) return LB_ERR_UNSUPPORTED;   // TMA row stride must be a multiple of 16 bytes
+    }
+    if (!P.pf) {
+        P.pf = new (std::nothrow) PrefillState();
+        if (!P.pf) return LB_ERR_OOM;
+        PrefillState &st = *P.pf;
+        if ((e = cudaMalloc(&st.maps, sizeof(CUtensorMap) * 2 * n)) != cudaSuccess) return status_from(e);
+        if ((e = cudaMalloc(&st.rec, sizeof(PfLayer) * 2 * n)) != cudaSuccess) return status_from(e);
+        if ((e = cudaMalloc(&st.starts, sizeof(int) * 2 * (n + 1))) != cudaSuccess) return status_from(e);
+        if ((e = cudaMalloc(&st.err, sizeof(int))) != cudaSuccess) return status_from(e);
+        if ((e = cudaMemsetAsync(st.err, 0, sizeof(int), s)) != cudaSuccess) return status_from(e);
+    }
+    PrefillState &st = *P.pf;
+    bool dirty = false;
+    if (M > st.M) {
+        // grow the latent scratch; padding columns stay zero
+        if (st.zl) {
+            cudaStreamSynchronize(s);
+            cudaFree(st.zl);
+            st.zl = nullptr;
+        }
+        size_t tot = 0;
+        st.zl_off.resize(n);
+        for (int i = 0; i < n; ++i) {
+            st.zl_off[i] = tot;
+            tot += ((size_t)M * layers[i]->pf.K2 * 2 + 255) & ~(size_t)255;
+        }
+        if ((e = cudaMalloc(&st.zl, tot)) != cudaSuccess) return status_from(e);
+        if ((e = cudaMemsetAsync(st.zl, 0, tot, s)) != cudaSuccess) return status_from(e);
+        st.M = M;
+        dirty = true;
+    }
+    if (M != st.lastM) dirty = true;
+    if ((int)st.lastX.size() != n) {
+        st.lastX.assign(n, nullptr);
+        st.lastY.assign(n, nullptr);
+        dirty = true;
+    }
+    for (int i = 0; i < n && !dirty; ++i)
+        if (st.lastX[i] != xs[i] || st.lastY[i] != ys[i]) dirty = true;
+    if (dirty) {
+        std::vector<CUtensorMap> maps(2 * n);
+        std::vector<PfLayer> rec(2 * n);
+        std::vector<int> starts(2 * (n + 1));
+        starts[0] = starts[n + 1] = 0;
+        for (int i = 0; i < n; ++i) {
+            const LayerDev &d = layers[i]->d;
+            const PfWeights &W = layers[i]->pf;
+            __half *zl = (__half *)((char *)st.zl + st.zl_off[i]);
+            if (!encode_2d(&maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xs[i], d.K, M) ||
+                !encode_2d(&maps[n + i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, zl, W.K2, M))
+                return LB_ERR_UNSUPPORTED;
+            const int mtiles = ceil_div(M, kPfBM);
+            PfLayer &a = rec[i];
+            a.tmA = st.maps + i;
+            a.bits = W.b1;
+            a.base = W.g64;
+            a.lcat = W.lcat;
+            a.out = zl;
+            a.nk = W.KB1;
+            a.ncols = W.N1p;
+            a.ld_out = W.K2;
+            a.ntn = ceil_div(W.N1p, kPfBN);
+            a.r8 = W.r8;
+            a.base_ld = W.K64;
+            a.npaths = d.npaths;
+            PfLayer &b = rec[n + i];
+            b.tmA = st.maps + n + i;
+            b.bits = W.b2;
+            b.base = W.h256;
+            b.lcat = nullptr;
+            b.out = ys[i];
+            b.nk = W.KB2;
+            b.ncols = d.N;
+            b.ld_out = d.N;
+            b.ntn = ceil_div(d.N, kPfBN);
+            b.r8 = W.r8;
+            b.base_ld = W.N256;
+            b.npaths = d.npaths;
+            starts[i + 1] = starts[i] + mtiles * a.ntn;
+            starts[n + 1 + i + 1] = starts[n + 1 + i] + mtiles * b.ntn;
+            st.lastX[i] = xs[i];
+            st.lastY[i] = ys[i];
+        }
+        st.tiles[0] = starts[n];
+        st.tiles[1] = starts[2 * n + 1];
+        st.lastM = M;
+        // pageable sources: the copies are staged before these calls return
+        if ((e = cudaMemcpyAsync(st.maps, maps.data(), sizeof(CUtensorMap) * 2 * n, cudaMemcpyHostToDevice, s)) !=
+            cudaSuccess)
+            return status_from(e);
+        if ((e = cudaMemcpyAsync(st.rec, rec.data(), sizeof(PfLayer) * 2 * n, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+            return status_from(e);
+        if ((e = cudaMemcpyAsync(st.starts, starts.data(), sizeof(int) * 2 * (n + 1), cudaMemcpyHostToDevice, s)) !=
+            cudaSuccess)
+            return status_from(e);
+        if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return status_from(e);
+    }
+
+    static int sms = 0;
+    static size_t smem_set = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    const size_t smem = smem_bytes(n);
+    if (smem > 232448) return LB_ERR_UNSUPPORTED;
+    if (smem > smem_set) {
+        if ((e = cudaFuncSetAttribute(prefill_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return status_from(e);
+        if ((e = cudaFuncSetAttribute(prefill_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return status_from(e);
+        smem_set = smem;
+    }
+    const int g0 = std::max(1, std::min(st.tiles[0], sms));
+    const int g1 = std::max(1, std::min(st.tiles[1], sms));
+    prefill_kernel<0><<<g0, kPfThreads, smem, s>>>(st.rec, st.starts, n, M, st.err);
+    profile_mark(++*launches, s);
+    prefill_kernel<1><<<g1, kPfThreads, smem, s>>>(st.rec + n, st.starts + n + 1, n, M, st.err);
+    profile_mark(++*launches, s);
+    return status_from(cudaGetLastError());
+}
+
+}  // namespace lb

@@ -1,0 +1,26 @@
+// Prefill (large-M) path: declarations shared by the layer builder and the
+// tensor-core kernels.
+#pragma once
+
+#include "lb_internal.cuh"
+
+namespace lb {
+
+// Tiles of the two tensor-core contractions.
+constexpr int kPfBM = 128;          // activation rows per tile (UMMA M)
+constexpr int kPfBN = 256;          // output columns per tile (UMMA N, at most)
+constexpr int kPfBK = 64;           // contraction depth per pipeline stage (one 128-byte swizzle atom of fp16)
+constexpr int kPfStages = 4;
+constexpr int kPfThreads = 512;     // 16 warps: producer, MMA, 4 epilogue, 8 generator warps
+
+cudaError_t prefill_build_weights(PfWeights &W, const LayerDev &d, const uint32_t *const *U,
+                                  const uint32_t *const *V, const uint16_t *const *h,
+                                  const uint16_t *const *g, const uint16_t *const *l, cudaStream_t s);
+size_t prefill_weight_bytes(const LayerDev &d);
+
+struct PrefillState;   // per plan (owned by Plan)
+lb_status prefill_forward(const Plan &P, const lb_layer *const *layers, const uint16_t *const *xs,
+                          float *const *ys, int M, cudaStream_t s, int *launches);
+void prefill_free(PrefillState *st);
+
+}  // namespace lb
