@@ -159,6 +159,38 @@ LB_API void lb_stack_destroy(lb_stack *S);
  */
 LB_API lb_status lb_stack_forward(lb_stack *S, const uint16_t *const *xs, float *const *ys, int M, void *stream);
 
+/*
+ * Forward pass of one layer, M <= LB_DECODE_MAX_M, that allocates no memory.
+ *
+ * The paper has no counterpart to this call; it exists for callers that must
+ * not allocate device memory while they run: a serving loop whose device
+ * memory is planned once at start-up and must not touch the CUDA allocator
+ * again (cudaMalloc/cudaFree may synchronise the device, stall every stream
+ * and fragment a memory plan), or an embedding runtime that owns all device
+ * memory itself.  The layer itself still comes from lb_layer_create (which
+ * allocates); this call does not.
+ *
+ * Same arguments, layouts and result as lb_linear_forward for M <= 16.  The
+ * scratch of the two decode kernels (float64 accumulators, latent fragments,
+ * completion counter, error code) lives in one fixed array of
+ * LB_NOALLOC_SCRATCH_BYTES bytes of static device memory inside this library,
+ * which every GPU that loads the library holds until the process exits.  The
+ * call issues no cudaMalloc, cudaFree or allocating library routine: it
+ * launches one small kernel that writes the layer descriptor into that array
+ * and clears the accumulators and counter, then the two decode kernels.
+ * The first call on each device looks the array's device address up once
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture begins.
+ * Every call shares the one array and leaves its contents behind, so calls
+ * that overlap on the GPU (different streams, or other host threads) race:
+ * order them on one stream.
+ * Errors: LB_ERR_INVALID_ARG (NULL, M < 0, misalignment), LB_ERR_UNSUPPORTED
+ * (M > LB_DECODE_MAX_M, or the layer needs more than LB_NOALLOC_SCRATCH_BYTES
+ * of scratch), LB_ERR_CUDA.  M = 0 is a valid empty call.
+ */
+#define LB_NOALLOC_SCRATCH_BYTES (1u << 20)
+LB_API lb_status lb_linear_forward_noalloc(const uint16_t *x, int M, const lb_layer *L, float *y, void *stream);
+
 /* Timing hook.  Registers n CUDA events (cudaEvent_t passed as void*) for the
  * calling thread: the following forward calls record events[0] on their
  * stream before their first kernel launch and events[i] right after their

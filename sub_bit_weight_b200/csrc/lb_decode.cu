@@ -727,4 +727,51 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
     return status_from(e);
 }
 
+// One layer whose descriptor (and scratch) the caller placed in device
+// memory: the two decode kernels over the given work items.  Used by the
+// entry point that must not allocate.
+lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc, const P1Item *p1, int n1,
+                            const P2Item *p2, int n2, const uint16_t *x, float *y, int M, int *err, cudaStream_t s,
+                            int *launches)
+{
+    const int NT = (M + 3) / 4;
+    cudaError_t e = cudaSuccess;
+    int sms = 0, dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return status_from(e);
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return status_from(e);
+    K1Fn k1;
+    K2Fn k2;
+    switch (NT) {
+    case 1: kernels_for<1>(k1, k2); break;
+    case 2: kernels_for<2>(k1, k2); break;
+    case 3: kernels_for<3>(k1, k2); break;
+    default: kernels_for<4>(k1, k2); break;
+    }
+    const int kb2max = host_desc.KB2;
+    const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * (kP1ChunkKB / 2) * 256 +
+                         (size_t)2 * kP1ChunkKB * NT * 32 * sizeof(uint2);
+    const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * kb2max * 256 +
+                         (size_t)NT * kb2max * 32 * sizeof(uint2);
+    if (smem2 > 227 * 1024) return LB_ERR_UNSUPPORTED;
+    if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) != cudaSuccess)
+        return status_from(e);
+    if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)) != cudaSuccess)
+        return status_from(e);
+    int occ1 = 0, occ2 = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, k1, kDecodeThreads, smem1)) != cudaSuccess)
+        return status_from(e);
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ2, k2, kDecodeThreads, smem2)) != cudaSuccess)
+        return status_from(e);
+    static thread_local IoPtrs io;
+    io.x[0] = x;
+    io.y[0] = y;
+    const int grid1 = std::max(1, std::min(n1, sms * std::max(1, occ1)));
+    const int grid2 = std::max(1, std::min(n2, sms * std::max(1, occ2)));
+    k1<<<grid1, kDecodeThreads, smem1, s>>>(dev_desc, p1, n1, io, 0, M, err);
+    ++*launches;
+    k2<<<grid2, kDecodeThreads, smem2, s>>>(dev_desc, p2, n2, io, 0, M, kb2max, err);
+    ++*launches;
+    return status_from(cudaGetLastError());
+}
+
 }  // namespace lb

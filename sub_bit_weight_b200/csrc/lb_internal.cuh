@@ -125,6 +125,10 @@ void plan_free(Plan &P);
 lb_status decode_forward(const Plan &P, const uint16_t *const *xs, float *const *ys, int M,
                          cudaStream_t s, int *launches);
 
+lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc, const P1Item *p1, int n1,
+                            const P2Item *p2, int n2, const uint16_t *x, float *y, int M, int *err, cudaStream_t s,
+                            int *launches);
+
 lb_status status_from(cudaError_t e);
 void set_launch_count(int n);
 // Timing hook: record the registered event `i` (if any) on stream s.

@@ -48,6 +48,7 @@ _sig("lb_layer_shape", _st, [_vp] + [ctypes.POINTER(_i)] * 4)
 _sig("lb_layer_bpw", ctypes.c_double, [_vp])
 _sig("lb_layer_device_bytes", ctypes.c_size_t, [_vp])
 _sig("lb_linear_forward", _st, [_vp, _i, _vp, _vp, _vp])
+_sig("lb_linear_forward_noalloc", _st, [_vp, _i, _vp, _vp, _vp])
 _sig("lb_stack_create", _st, [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp])
 _sig("lb_stack_destroy", None, [_vp])
 _sig("lb_stack_forward", _st, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp])
@@ -180,6 +181,20 @@ def lb_linear_forward(x: torch.Tensor, layer: Layer, y: torch.Tensor | None = No
     _check(_lib.lb_linear_forward(_dev(x, torch.bfloat16, "x") if M else None, M, layer.handle,
                                   _dev(y, torch.float32, "y") if M else None, _stream(stream)),
            "lb_linear_forward")
+    return y
+
+
+def lb_linear_forward_noalloc(x: torch.Tensor, layer: Layer, y: torch.Tensor, stream=None) -> torch.Tensor:
+    """Same result as lb_linear_forward for M <= 16, without allocating: scratch is a static
+    device array inside the library and ``y`` must be supplied (see the C header)."""
+    if x.dim() != 2 or x.shape[1] != layer.K:
+        raise ValueError(f"x must be [M, {layer.K}]")
+    M = x.shape[0]
+    if tuple(y.shape) != (M, layer.N):
+        raise ValueError(f"y must be [{M}, {layer.N}]")
+    _check(_lib.lb_linear_forward_noalloc(_dev(x, torch.bfloat16, "x") if M else None, M, layer.handle,
+                                          _dev(y, torch.float32, "y") if M else None, _stream(stream)),
+           "lb_linear_forward_noalloc")
     return y
 
 

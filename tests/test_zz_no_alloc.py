@@ -1,0 +1,52 @@
+"""lb_linear_forward_noalloc: the decode forward that allocates no memory.
+
+Some callers must not touch the CUDA allocator while they run: a serving loop
+whose device memory is planned once at start-up (cudaMalloc/cudaFree may
+synchronise the device and break that plan), or a runtime that owns all device
+memory itself.  This entry point keeps its scratch in a fixed static array
+inside the library instead.  Its output must match lb_linear_forward within
+the tolerance of the other parity tests, on consecutive calls that share (and
+inherit the contents of) that array.
+
+This file is collected last on purpose, so a run that stops at the first
+failure has already run every other test.
+"""
+
+import pytest
+
+from sub_bit_weight_b200 import synth
+from tests._util import TOL, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def test_noalloc_matches_forward_on_consecutive_calls():
+    import torch
+    from sub_bit_weight_b200 import lib, stacks
+    assert torch.cuda.is_available()
+    a = synth.LayerShape("a", 1000, 2050, 80)
+    b = synth.LayerShape("b", 4096, 4096, 184)
+    La = stacks.build_layer(71, 0, a)
+    Lb = stacks.build_layer(72, 1, b)
+    calls = [(La, a, 1, 81), (Lb, b, 5, 82), (La, a, 16, 83)]
+    for L, s, M, xs in calls:
+        x = stacks.bf16_on_device(synth.activations(xs, 0, M, s.K), "cuda")
+        ref = lib.lb_linear_forward(x, L).clone()
+        y = torch.full((M, s.N), float("nan"), dtype=torch.float32, device="cuda")
+        lib.lb_linear_forward_noalloc(x, L, y)
+        assert lib.lb_last_launch_count() == 3          # set-up kernel + the two decode kernels
+        torch.cuda.synchronize()
+        err = rel_err(y.cpu().numpy(), ref.cpu().numpy())
+        assert err <= TOL, (s, M, err)
+
+
+def test_noalloc_rejects_batches_above_the_decode_limit():
+    import torch
+    from sub_bit_weight_b200 import lib, stacks
+    s = synth.LayerShape("c", 64, 64, 8)
+    L = stacks.build_layer(73, 0, s)
+    x = torch.zeros((17, 64), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((17, 64), dtype=torch.float32, device="cuda")
+    with pytest.raises(lib.LittleBitError) as e:
+        lib.lb_linear_forward_noalloc(x, L, y)
+    assert e.value.status == lib.LB_ERR_UNSUPPORTED
