@@ -280,27 +280,46 @@ def main():
         dist = tdist
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    res = run_gpu(w, M, args.steps, args.warmup, dist, dev, nblocks=args.blocks)
+    res = run_gpu(w, M, args.steps, args.warmup, dist, dev, nblocks=args.blocks, want_e2e=not w.pool_rows)
     total_ms = max_over_ranks(res["total_ms"], dist)
     shapes = res["shapes"]
-    k1b = sum(layer_bytes(s, M)[0] for s in shapes)
-    k2b = sum(layer_bytes(s, M)[1] for s in shapes)
-    step_bytes = k1b + k2b
     ms_step = total_ms / args.steps
-    value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
+    prefill_main = bool(w.pool_rows)
+    if prefill_main:
+        flops = sum(layer_flops(s, M) for s in shapes)
+        value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+    else:
+        k1b = sum(layer_bytes(s, M)[0] for s in shapes)
+        k2b = sum(layer_bytes(s, M)[1] for s in shapes)
+        step_bytes = k1b + k2b
+        value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
+        unit = "GB/s"
 
     roof = None
     if res["per_launch"]:
         k1ms, k2ms = res["per_launch"]
         dom = 1 if k2ms >= k1ms else 0
-        dom_bytes, dom_ms = (k2b, k2ms) if dom else (k1b, k1ms)
-        ach = dom_bytes / (dom_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "kernel": "contraction2_kernel" if dom else "contraction1_kernel",
-                "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": round(ach / pk["hbm_gbs"], 4), "peak_src": pk["src"],
-                "traffic": None,
-                "per_kernel_ms": {"contraction1_kernel": round(k1ms, 5), "contraction2_kernel": round(k2ms, 5)},
-                "per_kernel_bytes": {"contraction1_kernel": k1b, "contraction2_kernel": k2b}}
+        if prefill_main:
+            f1 = sum(2.0 * M * 2 * s.r * s.K for s in shapes)
+            f2 = sum(2.0 * M * 2 * s.r * s.N for s in shapes)
+            dom_w, dom_ms = (f2, k2ms) if dom else (f1, k1ms)
+            ach = dom_w / (dom_ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "kernel": "prefill_kernel<1> (output GEMM)" if dom else "prefill_kernel<0> (latent GEMM)",
+                    "achieved": round(ach, 1), "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                    "frac": round(ach / pk["bf16_tflops_sustained"], 4),
+                    "peak_src": pk["src"] + " bf16 sustained (dense 16-bit tensor peak)", "traffic": None,
+                    "per_kernel_ms": {"latent": round(k1ms, 4), "output": round(k2ms, 4)},
+                    "per_kernel_flops": {"latent": f1, "output": f2}}
+        else:
+            dom_bytes, dom_ms = (k2b, k2ms) if dom else (k1b, k1ms)
+            ach = dom_bytes / (dom_ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "kernel": "contraction2_kernel" if dom else "contraction1_kernel",
+                    "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(ach / pk["hbm_gbs"], 4), "peak_src": pk["src"],
+                    "traffic": None,
+                    "per_kernel_ms": {"contraction1_kernel": round(k1ms, 5), "contraction2_kernel": round(k2ms, 5)},
+                    "per_kernel_bytes": {"contraction1_kernel": k1b, "contraction2_kernel": k2b}}
     e2e = None
     if res["e2e"]:
         e_ms = max_over_ranks(res["e2e"]["ms"], dist)
@@ -308,19 +327,21 @@ def main():
                "h2d_bytes_per_step": res["e2e"]["h2d"], "d2h_bytes_per_step": res["e2e"]["d2h"],
                "ms_per_step": round(e_ms, 4)}
 
-    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+    line = {"metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16 in, int8 tensor-core MMA (u8 signs x s8 fixed-point digits, s32 acc), fp32 out",
+            "dtype": ("bf16 in, fp16 tcgen05 MMA (fp32 accumulate in TMEM), fp32 out" if prefill_main else
+                      "bf16 in, int8 tensor-core MMA (u8 signs x s8 fixed-point digits, s32 acc), fp32 out"),
             "data": "synthetic (seeded; signs Bernoulli(0.5), scales lognormal(-3,0.5) fp16, x N(0,1) bf16)",
             "config": {"workload": f"{w.key}: {w.title}", "layers": len(shapes), "M": M,
-                       "bytes_per_step": step_bytes,
-                       "l2": "inputs larger than L2 (stack streams from HBM every step)"
-                             if step_bytes > 126e6 else "stack fits in L2 (effective GB/s)",
+                       "l2": ("inputs larger than L2 (stack streams from HBM every step)"
+                              if prefill_main or step_bytes > 126e6 else "stack fits in L2 (effective GB/s)"),
                        "parallelism": f"replicas x{world}"},
             "roofline": roof, "gpu_launches": res["launches"], "clocks": res["clocks"], "e2e": e2e}
+    if not prefill_main:
+        line["config"]["bytes_per_step"] = step_bytes
 
-    if args.prefill and world == 1:
+    if args.prefill and world == 1 and not prefill_main:
         pw = synth.WORKLOADS[args.prefill]
         pM = pw.Ms[0]
         pres = run_gpu(pw, pM, args.prefill_steps, 3, dist, dev, want_e2e=False)
@@ -339,9 +360,10 @@ def main():
 
     if rank == 0 and args.cpu_seconds > 0:
         cs = oracle_sample(w, M, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": round(cs["bytes"] / cs["seconds"] / 1e9, 5), "unit": "GB/s",
+        cv = (cs["flops"] / cs["seconds"] / 1e12) if prefill_main else (cs["bytes"] / cs["seconds"] / 1e9)
+        line["cpu_baseline"] = {"value": round(cv, 7), "unit": unit,
                                 "cores": 1, "kind": "oracle",
-                                "sample": f"first {cs['layers']} layers of the stack, M={M}, "
+                                "sample": f"first {cs['layers']} layers of the stack, {cs['rows']} of M={M} rows, "
                                           f"{cs['seconds']:.1f} s single-threaded float64 C"}
     if dist:
         dist.barrier()
@@ -357,23 +379,25 @@ def reference_arm(args, w, M, world, rank, pk):
     per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample(w, M, per_step / 4, max_layers=1)
-    t_bytes = t_sec = 0.0
+    t_work = t_sec = 0.0
     layers = 0
+    prefill = bool(w.pool_rows)
     for _ in range(args.steps):
         cs = oracle_sample(w, M, per_step)
-        t_bytes += cs["bytes"]
+        t_work += cs["flops"] if prefill else cs["bytes"]
         t_sec += cs["seconds"]
         layers += cs["layers"]
-    v = t_bytes / t_sec / 1e9
-    line = {"metric": METRIC, "value": round(v, 5), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+    v = t_work / t_sec / (1e12 if prefill else 1e9)
+    unit = "TFLOP/s" if prefill else "GB/s"
+    line = {"metric": METRIC, "value": round(v, 7), "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * t_sec / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
             "config": {"workload": f"{w.key}: {w.title}", "M": M},
-            "cpu_baseline": {"value": round(v, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": round(v, 7), "unit": unit, "cores": 1, "kind": "oracle",
                              "sample": f"{layers} layers over {args.steps} steps (first layers of the stack), "
                                        f"single-threaded float64 C"},
-            "e2e": {"value": round(v, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": round(v, 7), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 
 
