@@ -44,13 +44,14 @@ __device__ __forceinline__ int exponent_for(float amax, bool nonfinite)
     frexpf(amax, &e);                    // amax = f * 2^e, f in [0.5, 1)
     int E = 15 - e;                      // amax * 2^E in [2^14, 2^15)
     if (ldexpf(amax, E) > 32639.0f) E -= 1;
-    return E;
+    return min(E, 126);                  // 2^E and 2^-E stay normal floats (inputs below 2^-111 lose bits)
 }
 
-__device__ __forceinline__ int quantize(float t, int E)
-{
-    return (E == kNanExp) ? 0 : __float2int_rn(ldexpf(t, E));
-}
+// 2^E as a float (exact: |E| <= 126); quantize(t) = rint(t * 2^E)
+__device__ __forceinline__ float pow2f(int E) { return __int_as_float((127 + E) << 23); }
+__device__ __forceinline__ double pow2d(int E) { return __longlong_as_double((long long)(1023 + E) << 52); }
+
+__device__ __forceinline__ int quantize_s(float t, float scale) { return __float2int_rn(t * scale); }
 
 // low digit in [-128, 127] and high digit, q = 256 * hi + lo
 __device__ __forceinline__ void digits(int q, int &lo, int &hi)
@@ -192,10 +193,11 @@ __device__ void finish_latent(const LayerDev *dp, int M, float *sMax, int *sBad,
         int qs = 0;
         if (m < M) {
             const int E = sE[p * 16 + m];
+            const float sc = (E == kNanExp) ? 0.0f : pow2f(E);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int j = 4 * c + u;
-                const int q = (j < r) ? quantize(zl_at(p, j, m), E) : 0;
+                const int q = (j < r) ? quantize_s(zl_at(p, j, m), sc) : 0;
                 int lo, hi;
                 digits(q, lo, hi);
                 wlo |= (uint32_t)(lo & 255) << (8 * u);
@@ -229,7 +231,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
                         const __grid_constant__ IoPtrs io, int base, int M, int *err)
 {
     constexpr int NW = kDecodeThreads / 32;
-    constexpr int kHalf = kP1ChunkKB / 2;                    // k-blocks per ring stage
+    constexpr int kHalf = kP1StageKB;                        // k-blocks per ring stage
     constexpr int kStage = kHalf * 256;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *ring = smem_raw;                          // [NW][kP1Stages][kStage]
@@ -360,13 +362,14 @@ __global__ void __launch_bounds__(kDecodeThreads)
             for (int p = 0; p < 2; ++p) {
                 if (p >= npaths) continue;
                 const int E = sE[p * 16 + m];
+                const float sc = (E == kNanExp) ? 0.0f : pow2f(E);
                 int qs = 0;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     uint32_t wlo = 0, whi = 0;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int q = quantize(xv[4 * h + e] * gv[p][4 * h + e], E);
+                        const int q = quantize_s(xv[4 * h + e] * gv[p][4 * h + e], sc);
                         int lo, hi;
                         digits(q, lo, hi);
                         wlo |= (uint32_t)(lo & 255) << (8 * e);
@@ -392,7 +395,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
             const int p = tid / M, m = tid - p * M;
             const int E = sE[p * 16 + m];
             if (E == kNanExp) atomicOr(reinterpret_cast<int *>(acc + (size_t)dp->R1 * 16 + 32) + p * 16 + m, 1);
-            else if (sQs[p * 16 + m]) atomicAdd(acc + (size_t)dp->R1 * 16 + p * 16 + m, ldexp((double)sQs[p * 16 + m], -E));
+            else if (sQs[p * 16 + m]) atomicAdd(acc + (size_t)dp->R1 * 16 + p * 16 + m, (double)sQs[p * 16 + m] * pow2d(-E));
         }
 
         // ---- main stream: this warp's row groups of 64 latent rows, half a chunk per stage
@@ -456,11 +459,12 @@ __global__ void __launch_bounds__(kDecodeThreads)
                     if (m < M) {
                         const int E = sE[prb[rb] * 16 + m];
                         if (E == kNanExp) continue;
+                        const double sc = pow2d(-E);
                         const int Tlo = (a4[rb][n][0] >> rb) + 256 * (a4[rb][n][1] >> rb);
                         const int Thi = (a4[rb][n][2] >> (rb + 4)) + 256 * (a4[rb][n][3] >> (rb + 4));
                         const int row = rg * kRowsPerGroup + rb * kRowsPerBlock + g;
-                        if (Tlo) atomicAdd(acc + (size_t)row * 16 + m, ldexp((double)Tlo, -E));
-                        if (Thi) atomicAdd(acc + (size_t)(row + 8) * 16 + m, ldexp((double)Thi, -E));
+                        if (Tlo) atomicAdd(acc + (size_t)row * 16 + m, (double)Tlo * sc);
+                        if (Thi) atomicAdd(acc + (size_t)(row + 8) * 16 + m, (double)Thi * sc);
                     }
                 }
         }
@@ -586,17 +590,13 @@ __global__ void __launch_bounds__(kDecodeThreads)
                     const int m = 4 * n + t4;
                     const int E = (m < M) ? sE[p * 16 + m] : 0;
                     const int Q = (m < M) ? sQs[p * 16 + m] : 0;
+                    const float sc = (E == kNanExp) ? __int_as_float(0x7fc00000) : pow2f(-E);
 #pragma unroll
                     for (int rb = 0; rb < 4; ++rb) {
                         const int Tlo = (a4[rb][n][0] >> rb) + 256 * (a4[rb][n][1] >> rb);
                         const int Thi = (a4[rb][n][2] >> (rb + 4)) + 256 * (a4[rb][n][3] >> (rb + 4));
-                        float slo, shi;
-                        if (E == kNanExp) {
-                            slo = shi = __int_as_float(0x7fc00000);
-                        } else {
-                            slo = ldexpf((float)(Q - 2 * Tlo), -E);
-                            shi = ldexpf((float)(Q - 2 * Thi), -E);
-                        }
+                        const float slo = (float)(Q - 2 * Tlo) * sc;
+                        const float shi = (float)(Q - 2 * Thi) * sc;
                         yv[rb][n][0] += (p ? hv[1][rb][0] : hv[0][rb][0]) * slo;
                         yv[rb][n][1] += (p ? hv[1][rb][1] : hv[0][rb][1]) * shi;
                     }
@@ -681,7 +681,7 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
     }
     int kb2max = 0;
     for (const LayerDev &d : P.host) kb2max = std::max(kb2max, d.KB2);
-    const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * (kP1ChunkKB / 2) * 256 +
+    const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * kP1StageKB * 256 +
                          (size_t)2 * kP1ChunkKB * NT * 32 * sizeof(uint2);
     const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * kb2max * 256 +
                          (size_t)NT * kb2max * 32 * sizeof(uint2);
@@ -748,7 +748,7 @@ lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc,
     default: kernels_for<4>(k1, k2); break;
     }
     const int kb2max = host_desc.KB2;
-    const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * (kP1ChunkKB / 2) * 256 +
+    const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * kP1StageKB * 256 +
                          (size_t)2 * kP1ChunkKB * NT * 32 * sizeof(uint2);
     const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * kb2max * 256 +
                          (size_t)NT * kb2max * 32 * sizeof(uint2);

@@ -40,8 +40,9 @@ constexpr int kDecodeThreads = 128;     // 4 warps
 constexpr int kMaxDecodeM = LB_DECODE_MAX_M;
 constexpr int kMaxNT = (kMaxDecodeM + 3) / 4;   // n-tiles of 4 activation rows
 constexpr int kIoBatch = 1024;          // layers per launch (pointer tables ride in kernel params)
-constexpr int kP1Stages = 2;            // per-warp bulk-copy ring depth, contraction 1 (half chunks)
-constexpr int kP2Stages = 3;            // per-warp bulk-copy ring depth, contraction 2
+constexpr int kP1StageKB = 8;           // k-blocks per ring stage, contraction 1 (2 KB)
+constexpr int kP1Stages = 3;            // per-warp bulk-copy ring depth, contraction 1
+constexpr int kP2Stages = 2;            // per-warp bulk-copy ring depth, contraction 2 (one row group per stage)
 
 // doubles in the accumulator block of a layer's scratch
 __host__ __device__ inline size_t acc_doubles(int R1) { return (size_t)R1 * 16 + 32 + 16; }

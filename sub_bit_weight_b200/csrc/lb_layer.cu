@@ -166,6 +166,19 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
     }
     P.p1_start.push_back((int)p1.size());
     P.p2_start.push_back((int)p2.size());
+    // Within a launch, hand out the largest items first: static round-robin over a
+    // largest-first list keeps the tail of the grid short.
+    auto w1 = [&](const P1Item &a) {
+        const LayerDev &d = P.host[a.layer];
+        return (long long)d.RG1 * std::min(kP1ChunkKB, d.KB1 - a.kc * kP1ChunkKB);
+    };
+    auto w2 = [&](const P2Item &a) { return (long long)(a.rg1 - a.rg0) * P.host[a.layer].KB2; };
+    for (size_t b = 0; b + 1 < P.p1_start.size(); ++b) {
+        std::stable_sort(p1.begin() + P.p1_start[b], p1.begin() + P.p1_start[b + 1],
+                         [&](const P1Item &a, const P1Item &c) { return w1(a) > w1(c); });
+        std::stable_sort(p2.begin() + P.p2_start[b], p2.begin() + P.p2_start[b + 1],
+                         [&](const P2Item &a, const P2Item &c) { return w2(a) > w2(c); });
+    }
     P.n_p1 = (int)p1.size();
     P.n_p2 = (int)p2.size();
     if ((e = cudaMalloc(&P.dev, sizeof(LayerDev) * n)) != cudaSuccess) return e;

@@ -105,6 +105,21 @@ __global__ void build_b2_kernel(uint32_t *__restrict__ out, int RT2, int KB2, in
     }
 }
 
+// g of both paths per 64-wide k-block: dst[kb][p][0..64), zero beyond K and for an absent path.
+__global__ void g_blocks_kernel(__half *__restrict__ dst, const uint16_t *__restrict__ g0,
+                                const uint16_t *__restrict__ g1, int npaths, int K, int KB1)
+{
+    const int64_t total = (int64_t)KB1 * 128;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int kb = (int)(idx >> 7), p = (int)((idx >> 6) & 1), i = (int)(idx & 63);
+        const int k = kb * 64 + i;
+        uint16_t v = 0;
+        if (p < npaths && k < K) v = (p ? g1 : g0)[k];
+        dst[idx] = __ushort_as_half(v);
+    }
+}
+
 __global__ void pad_half_kernel(__half *__restrict__ dst, const uint16_t *__restrict__ s0,
                                 const uint16_t *__restrict__ s1, int npaths, int n, int npad)
 {
@@ -147,7 +162,7 @@ size_t prefill_weight_bytes(const LayerDev &d)
 {
     PfWeights W;
     pf_dims(W, d);
-    return al256((size_t)W.RT1 * W.KB1 * 4096) + al256((size_t)d.npaths * W.K64 * 2) +
+    return al256((size_t)W.RT1 * W.KB1 * 4096) + al256((size_t)W.KB1 * 128 * 2) +
            al256((size_t)W.N1p * 4) + al256((size_t)W.RT2 * W.KB2 * 4096) + al256((size_t)d.npaths * W.N256 * 2);
 }
 
@@ -159,7 +174,7 @@ cudaError_t prefill_build_weights(PfWeights &W, const LayerDev &d, const uint32_
     pf_dims(W, d);
     char *c = (char *)W.b1;
     W.b1 = (uint32_t *)c;      c += al256((size_t)W.RT1 * W.KB1 * 4096);
-    W.g64 = (__half *)c;       c += al256((size_t)d.npaths * W.K64 * 2);
+    W.g64 = (__half *)c;       c += al256((size_t)W.KB1 * 128 * 2);
     W.lcat = (float *)c;       c += al256((size_t)W.N1p * 4);
     W.b2 = (uint32_t *)c;      c += al256((size_t)W.RT2 * W.KB2 * 4096);
     W.h256 = (__half *)c;
@@ -170,7 +185,7 @@ cudaError_t prefill_build_weights(PfWeights &W, const LayerDev &d, const uint32_
                                                                       P > 1 ? V[1] : V[0]);
     build_b2_kernel<<<grid((int64_t)W.RT2 * W.KB2 * 1024), T, 0, s>>>(W.b2, W.RT2, W.KB2, d.r, W.r8, d.N, P, U[0],
                                                                       P > 1 ? U[1] : U[0]);
-    pad_half_kernel<<<grid((int64_t)P * W.K64), T, 0, s>>>(W.g64, g[0], P > 1 ? g[1] : g[0], P, d.K, W.K64);
+    g_blocks_kernel<<<grid((int64_t)W.KB1 * 128), T, 0, s>>>(W.g64, g[0], P > 1 ? g[1] : g[0], P, d.K, W.KB1);
     pad_half_kernel<<<grid((int64_t)P * W.N256), T, 0, s>>>(W.h256, h[0], P > 1 ? h[1] : h[0], P, d.N, W.N256);
     lcat_kernel<<<grid(W.N1p), T, 0, s>>>(W.lcat, l[0], P > 1 ? l[1] : l[0], P, d.r, W.r8, W.N1p);
     return cudaGetLastError();
@@ -318,6 +333,8 @@ struct PfSmem {
     alignas(1024) unsigned char A[kPfStages][kPfBM * kPfBK * 2];
     alignas(1024) unsigned char B[kPfStages][kPfBN * kPfBK * 2];
     alignas(16) uint32_t bits[kPfStages][256 * 4];
+    alignas(16) __half gst[kPfStages][128];     // latent GEMM: g of both paths for the stage's k-block
+    alignas(16) float lsc[kPfBN];               // latent GEMM epilogue: l of the tile's columns
     uint64_t full[kPfStages], ready[kPfStages], empty[kPfStages];
     uint64_t accf[2], acce[2];
     uint32_t tmem_base;
@@ -380,15 +397,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
                 int L, mt, nt;
                 locate(t, L, mt, nt);
-                const PfLayer &ly = layers[L];
+                const PfLayer ly = layers[L];   // register copy: waits below clobber memory
                 const uint32_t *bits = ly.bits + (size_t)nt * ly.nk * 1024;
                 for (int kb = 0; kb < ly.nk; ++kb, ++it) {
                     const int s = it % kPfStages;
                     const uint32_t ph = (it / kPfStages) & 1;
                     if (!mbar_wait(&S.empty[s], ph ^ 1, abort, err, 1)) break;
-                    mbar_expect_tx(&S.full[s], kPfBM * kPfBK * 2 + 4096);
+                    mbar_expect_tx(&S.full[s], kPfBM * kPfBK * 2 + 4096 + (MODE == 0 ? 256 : 0));
                     tma_load_2d(S.A[s], ly.tmA, kb * kPfBK, mt * kPfBM, &S.full[s]);
                     bulk_load(S.bits[s], bits + (size_t)kb * 1024, 4096, &S.full[s]);
+                    if (MODE == 0) bulk_load(S.gst[s], ly.base + (size_t)kb * 128, 256, &S.full[s]);
                     pend |= 1u << s;
                     pend_ph = (pend_ph & ~(1u << s)) | (ph << s);
                 }
@@ -410,7 +428,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x, ++tcount) {
                 int L, mt, nt;
                 locate(t, L, mt, nt);
-                const PfLayer &ly = layers[L];
+                const PfLayer ly = layers[L];   // register copy: waits below clobber memory
                 const int nw = min(kPfBN, ly.ncols - nt * kPfBN);
                 const int ab = tcount & 1;
                 const uint32_t aph = (tcount >> 1) & 1;
@@ -445,12 +463,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x, ++tcount) {
             int L, mt, nt;
             locate(t, L, mt, nt);
-            const PfLayer &ly = layers[L];
+            const PfLayer ly = layers[L];   // register copy: waits below clobber memory
             const int nw = min(kPfBN, ly.ncols - nt * kPfBN);
             const int ab = tcount & 1;
             const uint32_t aph = (tcount >> 1) & 1;
             if (!mbar_wait(&S.accf[ab], aph, abort, err, 5)) break;
             tc_fence_after();
+            if (MODE == 0) {
+                // l of this tile's columns into shared memory (the 4 epilogue warps, named barrier 1)
+                asm volatile("bar.sync 1, 128;\n" ::: "memory");   // previous tile done with S.lsc
+                for (int i = tid - 128; i < kPfBN; i += 128) {
+                    const int c = nt * kPfBN + i;
+                    S.lsc[i] = (c < ly.ncols) ? __ldg(ly.lcat + c) : 0.0f;
+                }
+                asm volatile("bar.sync 1, 128;\n" ::: "memory");
+            }
             const int m = mt * kPfBM + q * 32 + lane;
             for (int ch = 0; ch < nw; ch += 32) {
                 uint32_t v[32];
@@ -463,9 +490,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int c = c0 + 2 * i;
-                            const float a = (c < ly.ncols) ? __uint_as_float(v[2 * i]) * __ldg(ly.lcat + c) : 0.0f;
-                            const float b =
-                                (c + 1 < ly.ncols) ? __uint_as_float(v[2 * i + 1]) * __ldg(ly.lcat + c + 1) : 0.0f;
+                            const float a = __uint_as_float(v[2 * i]) * S.lsc[ch + 2 * i];
+                            const float b = __uint_as_float(v[2 * i + 1]) * S.lsc[ch + 2 * i + 1];
+                            (void)c;
                             const __half2 hh = __floats2half2_rn(a, b);
                             hw[i] = *reinterpret_cast<const uint32_t *>(&hh);
                         }
@@ -474,8 +501,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                             for (int i = 0; i < 4; ++i)
                                 reinterpret_cast<uint4 *>(out)[i] = make_uint4(hw[4 * i], hw[4 * i + 1], hw[4 * i + 2], hw[4 * i + 3]);
                         } else {
-                            for (int i = 0; i < 16 && c0 + 2 * i < ly.ncols; ++i)
-                                reinterpret_cast<uint32_t *>(out)[i] = hw[i];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                if (c0 + 2 * i < ly.ncols) reinterpret_cast<uint32_t *>(out)[i] = hw[i];
                         }
                     } else {
                         float *out = reinterpret_cast<float *>(ly.out) + (size_t)m * ly.ld_out + c0;
@@ -484,7 +512,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                             for (int i = 0; i < 8; ++i)
                                 reinterpret_cast<uint4 *>(out)[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                         } else {
-                            for (int i = 0; i < 32 && c0 + i < ly.ncols; ++i) out[i] = __uint_as_float(v[i]);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (c0 + i < ly.ncols) out[i] = __uint_as_float(v[i]);
                         }
                     }
                 }
@@ -501,7 +531,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
             int L, mt, nt;
             locate(t, L, mt, nt);
-            const PfLayer &ly = layers[L];
+            const PfLayer ly = layers[L];   // register copy: waits below clobber memory
             const int nw = min(kPfBN, ly.ncols - nt * kPfBN);
             // output contraction: this thread's row n and its two path scales
             uint32_t hh[2] = {0u, 0u};
@@ -531,9 +561,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     const int k = kb * kPfBK + 8 * c;
                     uint4 gb[2];
 #pragma unroll
-                    for (int p = 0; p < 2; ++p)
-                        gb[p] = (p < ly.npaths) ? __ldg(reinterpret_cast<const uint4 *>(ly.base + (size_t)p * ly.base_ld + k))
-                                                : make_uint4(0, 0, 0, 0);
+                    for (int p = 0; p < 2; ++p) gb[p] = *reinterpret_cast<const uint4 *>(S.gst[s] + p * 64 + 8 * c);
+                    (void)k;
                     const int sh0 = 4 * (c & 1);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
