@@ -1,0 +1,128 @@
+// Device helpers shared by the decode (small-batch) kernels.
+#pragma once
+
+#include <cfloat>
+
+#include "lb_internal.cuh"
+
+namespace lb {
+
+// ---------------------------------------------------------------------------
+// Fixed point
+// ---------------------------------------------------------------------------
+static __device__ __forceinline__ int exponent_for(float amax, bool nonfinite)
+{
+    // Largest E with amax * 2^E <= 32639, so that q = rint(t * 2^E) splits into
+    // two balanced digits in [-128, 127].
+    if (nonfinite) return kNanExp;
+    if (!(amax > 0.0f)) return 0;
+    int e;
+    frexpf(amax, &e);                    // amax = f * 2^e, f in [0.5, 1)
+    int E = 15 - e;                      // amax * 2^E in [2^14, 2^15)
+    if (ldexpf(amax, E) > 32639.0f) E -= 1;
+    return min(E, 126);                  // 2^E and 2^-E stay normal floats (inputs below 2^-111 lose bits)
+}
+
+// 2^E as a float (exact: |E| <= 126); quantize(t) = rint(t * 2^E)
+static __device__ __forceinline__ float pow2f(int E) { return __int_as_float((127 + E) << 23); }
+static __device__ __forceinline__ double pow2d(int E) { return __longlong_as_double((long long)(1023 + E) << 52); }
+
+static __device__ __forceinline__ int quantize_s(float t, float scale) { return __float2int_rn(t * scale); }
+
+// low digit in [-128, 127] and high digit, q = 256 * hi + lo
+static __device__ __forceinline__ void digits(int q, int &lo, int &hi)
+{
+    lo = ((q + 128) & 255) - 128;
+    hi = (q - lo) >> 8;
+}
+
+// Where the two digit words of activation row m and 4 consecutive k starting
+// at kk (within a 32-wide k-block) live among the lanes' m16n8k32 B
+// fragments: column g = 2 * (m % 4) + digit, lane = 4 * g + t, word kk / 16,
+// with t = (kk % 16) / 4.
+static __device__ __forceinline__ void frag_slot(int m, int kk, int &lane_lo, int &lane_hi, int &word)
+{
+    const int mm = m & 3;
+    const int t = (kk & 15) >> 2;
+    word = kk >> 4;
+    lane_lo = (2 * mm) * 4 + t;
+    lane_hi = (2 * mm + 1) * 4 + t;
+}
+
+static __device__ __forceinline__ void set_word(uint2 &u, int word, uint32_t v)
+{
+    if (word) u.y = v; else u.x = v;
+}
+
+static __device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+static __device__ __forceinline__ int warp_sum(int v)
+{
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+static __device__ __forceinline__ int warp_or(int v)
+{
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// non-negative floats order like their bit patterns
+static __device__ __forceinline__ void smem_max(float *a, float v) { atomicMax((int *)a, __float_as_int(v)); }
+
+// ---------------------------------------------------------------------------
+// mbarrier + bulk copy (one ring of buffers per warp)
+// ---------------------------------------------------------------------------
+static __device__ __forceinline__ uint32_t sm_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+static __device__ __forceinline__ void bar_init(uint64_t *b)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(sm_addr(b)));
+}
+
+static __device__ __forceinline__ void ring_fill(void *dst, const void *src, unsigned bytes, uint64_t *bar)
+{
+    asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(sm_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                     sm_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(sm_addr(bar))
+                 : "memory");
+}
+
+static __device__ __forceinline__ bool bar_try(uint64_t *b, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+                 : "=r"(ok)
+                 : "r"(sm_addr(b)), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+constexpr long long kDecWaitCycles = 4000000000LL;   // ~2 s
+
+// Bounded wait for a ring buffer; false (and an error code) on timeout.
+static __device__ __forceinline__ bool ring_wait(uint64_t *b, uint32_t parity, int *err)
+{
+    if (bar_try(b, parity)) return true;
+    const long long t0 = clock64();
+    while (!bar_try(b, parity)) {
+        if (clock64() - t0 > kDecWaitCycles) {
+            atomicCAS(err, 0, 16);
+            return false;
+        }
+    }
+    return true;
+}
+
+}  // namespace lb

@@ -1,0 +1,533 @@
+// Decode kernels for one or two activation rows (M <= 2), both paths merged.
+//
+// Same method as lb_decode.cu (LittleBit notes page, "Multi-scale
+// compensation": x (.) g . V_sign (.) l . U_sign^T (.) h; "Residual
+// compensation": the two paths summed), specialised for the batch sizes of
+// token-by-token decoding.  With M <= 2 the 8 columns of one m16n8k32 B
+// fragment hold every activation operand at once:
+//
+//     column = 4 * m + 2 * path + digit        (m < 2, path < 2, digit < 2)
+//
+// so one MMA per (row block, k-block) serves both paths.  In contraction 1
+// (rows = latent indices of one path) the accumulator columns of the row
+// block's own path are kept; in contraction 2 (k = latent indices, the other
+// path's columns of a k-block are zero) lane pairs (path 0, path 1) hold the
+// two path results of one output and add them with one shuffle.  No
+// per-path loop, no operand selects, one fold per row group.
+
+#include "lb_decode_common.cuh"
+
+namespace lb {
+
+// Lane of column (m, path, digit) holding activation index kk of a k-block,
+// and which of its two fragment words.
+static __device__ __forceinline__ int pair_lane(int m, int p, int d, int kk)
+{
+    return ((4 * m + 2 * p + d) << 2) + ((kk & 15) >> 2);
+}
+
+// ---------------------------------------------------------------------------
+// Finish of contraction 1 (last item of a layer): zl fragments, merged layout
+// ---------------------------------------------------------------------------
+static __device__ void finish_pair(const LayerDev *dp, int M, float *sMax, int *sBad, int *sE, int *sQs)
+{
+    const int tid = threadIdx.x;
+    const int R1 = dp->R1, r = dp->r, r16 = dp->r16, r32 = dp->r32, npaths = dp->npaths, KB2 = dp->KB2;
+    double *acc = dp->acc;
+    const __half *lsc = dp->l;
+    const double *S = acc + (size_t)R1 * 16;
+    const int *badf = reinterpret_cast<const int *>(acc + (size_t)R1 * 16 + 32);
+    if (tid < 32) {
+        sMax[tid] = 0.0f;
+        sBad[tid] = 0;
+        sQs[tid] = 0;
+    }
+    {
+        uint4 *z = reinterpret_cast<uint4 *>(dp->zfrag);
+        for (int i = tid; i < KB2 * 32 * (int)sizeof(uint2) / 16; i += kDecodeThreads) z[i] = make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+    auto zl_at = [&](int p, int j, int m) -> float {
+        const double z = __ldcg(S + p * 16 + m) - 2.0 * __ldcg(acc + (size_t)(p * r16 + j) * 16 + m);
+        return (float)z * __half2float(lsc[p * r16 + j]);
+    };
+    for (int e = tid; e < npaths * r * M; e += kDecodeThreads) {
+        const int m = e % M, pj = e / M;
+        const int p = pj / r, j = pj - p * r;
+        const float zl = zl_at(p, j, m);
+        if (!(fabsf(zl) <= FLT_MAX)) atomicOr(&sBad[p * 16 + m], 1);
+        else smem_max(&sMax[p * 16 + m], fabsf(zl));
+    }
+    __syncthreads();
+    if (tid < npaths * M) {
+        const int p = tid / M, m = tid - p * M;
+        sE[p * 16 + m] = exponent_for(sMax[p * 16 + m], sBad[p * 16 + m] != 0 || __ldcg(badf + p * 16 + m) != 0);
+    }
+    __syncthreads();
+    const int ngrp = r32 / 4;
+    for (int e = tid; e < npaths * M * ngrp; e += kDecodeThreads) {
+        const int c = e % ngrp, pm = e / ngrp;
+        const int p = pm / M, m = pm - p * M;
+        const int E = sE[p * 16 + m];
+        const float sc = (E == kNanExp) ? 0.0f : pow2f(E);
+        uint32_t wlo = 0, whi = 0;
+        int qs = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = 4 * c + u;
+            const int q = (j < r) ? quantize_s(zl_at(p, j, m), sc) : 0;
+            int lo, hi;
+            digits(q, lo, hi);
+            wlo |= (uint32_t)(lo & 255) << (8 * u);
+            whi |= (uint32_t)(hi & 255) << (8 * u);
+            qs += q;
+        }
+        if (qs) atomicAdd(&sQs[p * 16 + m], qs);
+        const int jj = p * r32 + 4 * c;
+        uint2 *fb = dp->zfrag + (size_t)(jj >> 5) * 32;
+        const int word = (jj & 31) >> 4;
+        set_word(fb[pair_lane(m, p, 0, jj & 31)], word, wlo);
+        set_word(fb[pair_lane(m, p, 1, jj & 31)], word, whi);
+    }
+    __syncthreads();
+    if (tid < npaths * M) {
+        const int p = tid / M, m = tid - p * M;
+        dp->zmeta[p * 16 + m] = make_int2(sE[p * 16 + m], sQs[p * 16 + m]);
+    }
+    for (int i = tid; i < (int)acc_doubles(R1); i += kDecodeThreads) acc[i] = 0.0;
+}
+
+// ---------------------------------------------------------------------------
+// Contraction 1, M <= 2
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kDecodeThreads)
+    contraction1_pair_kernel(const LayerDev *__restrict__ layers, const P1Item *__restrict__ items, int nitems,
+                             const __grid_constant__ IoPtrs io, int base, int M, int *err)
+{
+    constexpr int NW = kDecodeThreads / 32;
+    constexpr int kHalf = kP1StageKB;
+    constexpr int kStage = kHalf * 256;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char *ring = smem_raw;                                      // [NW][kP1Stages][kStage]
+    uint2 *sB = (uint2 *)(smem_raw + NW * kP1Stages * kStage);          // [kP1ChunkKB][32]
+    __shared__ uint64_t bars[NW][kP1Stages];
+    __shared__ float sMax[32];
+    __shared__ int sBad[32], sE[32], sQs[32];
+    __shared__ int sLast;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int lane_m = t4 >> 1, lane_p = t4 & 1;       // accumulator columns of this lane
+    if (lane == 0)
+        for (int s = 0; s < kP1Stages; ++s) bar_init(&bars[warp][s]);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    __syncwarp();
+    uint32_t issued = 0, consumed = 0;
+    unsigned char *my_ring = ring + warp * kP1Stages * kStage;
+
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
+        const P1Item item = items[it];
+        const LayerDev *dp = layers + item.layer;
+        const int K = dp->K, K32 = dp->K32, KB1 = dp->KB1, RG1 = dp->RG1, r16 = dp->r16, npaths = dp->npaths;
+        const int R1 = dp->R1;
+        const uint2 *__restrict__ vt = dp->vt;
+        const __half *__restrict__ gsc = dp->g;
+        double *__restrict__ acc = dp->acc;
+        const uint16_t *__restrict__ x = io.x[item.layer - base];
+        const int kb0 = item.kc * kP1ChunkKB;
+        const int nkb = min(kP1ChunkKB, KB1 - kb0);
+        const int k0 = kb0 * kKPerBlock;
+        const int klen = nkb * kKPerBlock;
+        const int hp = (nkb + kHalf - 1) / kHalf;
+        const int nmine = (RG1 - warp + NW - 1) / NW;
+        const int nseq = max(0, nmine) * hp;
+        auto fill = [&](int q) {
+            const int rg = warp + NW * (q / hp), h = q % hp;
+            const int n = min(kHalf, nkb - h * kHalf);
+            const int st = issued % kP1Stages;
+            ring_fill(my_ring + st * kStage, vt + ((size_t)rg * KB1 + kb0 + h * kHalf) * 32, (unsigned)n * 256u,
+                      &bars[warp][st]);
+            ++issued;
+        };
+        if (lane == 0)
+            for (int q = 0; q < min(kP1Stages, nseq); ++q) fill(q);
+
+        {
+            uint4 *z4 = (uint4 *)sB;
+            for (int i = tid; i < kP1ChunkKB * 32 * (int)sizeof(uint2) / 16; i += kDecodeThreads)
+                z4[i] = make_uint4(0, 0, 0, 0);
+        }
+        if (tid < 32) {
+            sMax[tid] = 0.0f;
+            sBad[tid] = 0;
+            sQs[tid] = 0;
+        }
+        __syncthreads();
+
+        // ---- t = x (.) g_p for 8 consecutive inputs per thread
+        const int kk0 = 8 * tid;
+        const bool act = kk0 < klen;
+        const int kg = k0 + kk0;
+        float gv[2][8];
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            if (act && p < npaths) {
+                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(gsc + (size_t)p * K32 + kg));
+                const __half *hv = reinterpret_cast<const __half *>(&raw);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) gv[p][e] = __half2float(hv[e]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) gv[p][e] = 0.0f;
+            }
+        }
+        float xv[2][8];
+        const bool vec = ((K & 7) == 0) && (kg + 8 <= K);
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            if (!act || m >= M) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) xv[m][e] = 0.0f;
+            } else if (vec) {
+                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + kg));
+                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    xv[m][2 * e] = __uint_as_float(w4[e] << 16);
+                    xv[m][2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    xv[m][e] = (kg + e < K) ? bf16_bits_to_float(__ldg(x + (size_t)m * K + kg + e)) : 0.0f;
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                float amax = 0.0f;
+                int bad = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float tv = fabsf(xv[m][e] * gv[p][e]);
+                    if (!(tv <= FLT_MAX)) bad = 1;
+                    else amax = fmaxf(amax, tv);
+                }
+                amax = warp_max(amax);
+                bad = warp_or(bad);
+                if (lane == 0 && p < npaths && m < M) {
+                    smem_max(&sMax[p * 16 + m], amax);
+                    if (bad) atomicOr(&sBad[p * 16 + m], 1);
+                }
+            }
+        __syncthreads();
+        if (tid < npaths * M) {
+            const int p = tid / M, m = tid - p * M;
+            sE[p * 16 + m] = exponent_for(sMax[p * 16 + m], sBad[p * 16 + m] != 0);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                if (m >= M || p >= npaths) continue;
+                const int E = sE[p * 16 + m];
+                const float sc = (E == kNanExp) ? 0.0f : pow2f(E);
+                int qs = 0;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t wlo = 0, whi = 0;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int q = quantize_s(xv[m][4 * h + e] * gv[p][4 * h + e], sc);
+                        int lo, hi;
+                        digits(q, lo, hi);
+                        wlo |= (uint32_t)(lo & 255) << (8 * e);
+                        whi |= (uint32_t)(hi & 255) << (8 * e);
+                        qs += q;
+                    }
+                    if (act) {
+                        const int kk = kk0 + 4 * h;
+                        uint2 *fb = sB + (size_t)(kk >> 5) * 32;
+                        const int word = (kk & 31) >> 4;
+                        set_word(fb[pair_lane(m, p, 0, kk & 31)], word, wlo);
+                        set_word(fb[pair_lane(m, p, 1, kk & 31)], word, whi);
+                    }
+                }
+                qs = warp_sum(qs);
+                if (lane == 0 && qs) atomicAdd(&sQs[p * 16 + m], qs);
+            }
+        __syncthreads();
+        if (tid < npaths * M) {
+            const int p = tid / M, m = tid - p * M;
+            const int E = sE[p * 16 + m];
+            if (E == kNanExp) atomicOr(reinterpret_cast<int *>(acc + (size_t)R1 * 16 + 32) + p * 16 + m, 1);
+            else if (sQs[p * 16 + m]) atomicAdd(acc + (size_t)R1 * 16 + p * 16 + m, (double)sQs[p * 16 + m] * pow2d(-E));
+        }
+        // this lane's dequantisation scale for its (m, path) columns
+        const int lane_E = (lane_m < M && lane_p < npaths) ? sE[lane_p * 16 + lane_m] : kNanExp;
+        const double lane_sc = (lane_E == kNanExp) ? 0.0 : pow2d(-lane_E);
+
+        // ---- main stream
+        for (int rgi = 0; rgi < nmine; ++rgi) {
+            const int rg = warp + NW * rgi;
+            int a4[4][4];
+#pragma unroll
+            for (int rb = 0; rb < 4; ++rb)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) a4[rb][c] = 0;
+            for (int h = 0; h < hp; ++h) {
+                const int st = consumed % kP1Stages;
+                const uint32_t ph = (consumed / kP1Stages) & 1;
+                if (!ring_wait(&bars[warp][st], ph, err)) return;
+                ++consumed;
+                const uint2 *src = reinterpret_cast<const uint2 *>(my_ring + st * kStage) + lane;
+                const uint2 *bsrc = sB + (size_t)(h * kHalf) * 32 + lane;
+                const int n = min(kHalf, nkb - h * kHalf);
+                if (n == kHalf) {
+#pragma unroll
+                    for (int u = 0; u < kHalf; ++u) {
+                        const uint2 w = src[u * 32];
+                        const uint2 b = bsrc[u * 32];
+#pragma unroll
+                        for (int rb = 0; rb < 4; ++rb) {
+                            const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                            mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+                        }
+                    }
+                } else {
+                    for (int u = 0; u < n; ++u) {
+                        const uint2 w = src[u * 32];
+                        const uint2 b = bsrc[u * 32];
+#pragma unroll
+                        for (int rb = 0; rb < 4; ++rb) {
+                            const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                            mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    const int q = rgi * hp + h + kP1Stages;
+                    if (q < nseq) {
+                        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                        fill(q);
+                    }
+                }
+            }
+            // keep the columns of each row block's own path
+#pragma unroll
+            for (int rb = 0; rb < 4; ++rb) {
+                const int row0 = rg * kRowsPerGroup + rb * kRowsPerBlock;
+                const int prb = min(row0 / r16, npaths - 1);
+                if (prb != lane_p || lane_E == kNanExp) continue;
+                const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
+                const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
+                if (Tlo) atomicAdd(acc + (size_t)(row0 + g) * 16 + lane_m, (double)Tlo * lane_sc);
+                if (Thi) atomicAdd(acc + (size_t)(row0 + g + 8) * 16 + lane_m, (double)Thi * lane_sc);
+            }
+        }
+
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) sLast = (atomicAdd(dp->counter, 1u) == (unsigned)(dp->nkc - 1));
+        __syncthreads();
+        if (sLast) {
+            __threadfence();
+            finish_pair(dp, M, sMax, sBad, sE, sQs);
+            __syncthreads();
+            if (tid == 0) atomicExch(dp->counter, 0u);
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Contraction 2 (+ h, + path sum), M <= 2
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kDecodeThreads)
+    contraction2_pair_kernel(const LayerDev *__restrict__ layers, const P2Item *__restrict__ items, int nitems,
+                             const __grid_constant__ IoPtrs io, int base, int M, int kb2max, int *err)
+{
+    constexpr int NW = kDecodeThreads / 32;
+    constexpr int kRows = kP2ItemGroups * kRowsPerGroup;   // outputs per item
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const int kStage = kb2max * 256;
+    unsigned char *ring = smem_raw;                                         // [NW][kP2Stages][kStage]
+    uint2 *sB = (uint2 *)(smem_raw + (size_t)NW * kP2Stages * kStage);     // [KB2][32]
+    float *sH = (float *)(sB + (size_t)kb2max * 32);                       // [2][kRows]
+    __shared__ uint64_t bars[NW][kP2Stages];
+    __shared__ float sScale[4], sQsc[4];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int lane_m = t4 >> 1, lane_p = t4 & 1;
+    if (lane == 0)
+        for (int s = 0; s < kP2Stages; ++s) bar_init(&bars[warp][s]);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    __syncwarp();
+    uint32_t issued = 0, consumed = 0;
+    unsigned char *my_ring = ring + (size_t)warp * kP2Stages * kStage;
+
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
+        const P2Item item = items[it];
+        const LayerDev *dp = layers + item.layer;
+        const int N = dp->N, N64 = dp->N64, KB2 = dp->KB2, npaths = dp->npaths;
+        const uint2 *__restrict__ ut = dp->ut;
+        const __half *__restrict__ hsc = dp->h;
+        float *__restrict__ y = io.y[item.layer - base];
+        const unsigned stage_bytes = (unsigned)KB2 * 256u;
+
+        if (lane == 0)
+            for (int s = 0; s < kP2Stages; ++s) {
+                const int rg = item.rg0 + warp + NW * s;
+                if (rg < item.rg1) {
+                    const int st = issued % kP2Stages;
+                    ring_fill(my_ring + (size_t)st * kStage, ut + (size_t)rg * KB2 * 32, stage_bytes, &bars[warp][st]);
+                    ++issued;
+                }
+            }
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(dp->zfrag);
+            uint4 *dst = reinterpret_cast<uint4 *>(sB);
+            for (int i = tid; i < KB2 * 32 * (int)sizeof(uint2) / 16; i += kDecodeThreads) dst[i] = __ldcg(src + i);
+        }
+        const int n0 = item.rg0 * kRowsPerGroup;
+        for (int i = tid; i < 2 * kRows; i += kDecodeThreads) {
+            const int p = i / kRows, n = n0 + (i - p * kRows);
+            sH[i] = (p < npaths && n < N64) ? __half2float(hsc[p * N64 + n]) : 0.0f;
+        }
+        if (tid < 4) {
+            const int m = tid >> 1, p = tid & 1;
+            float sc = 0.0f, qsc = 0.0f;
+            if (m < M && p < npaths) {
+                const int2 mt = __ldcg(&dp->zmeta[p * 16 + m]);
+                if (mt.x == kNanExp) {
+                    sc = qsc = __int_as_float(0x7fc00000);
+                } else {
+                    sc = -2.0f * pow2f(-mt.x);                  // s = Q 2^-E - 2 T 2^-E
+                    qsc = (float)mt.y * pow2f(-mt.x);
+                }
+            }
+            sScale[tid] = sc;
+            sQsc[tid] = qsc;
+        }
+        __syncthreads();
+        const float my_sc = sScale[t4], my_q = sQsc[t4];
+
+        for (int rg = item.rg0 + warp; rg < item.rg1; rg += NW) {
+            const int st = consumed % kP2Stages;
+            const uint32_t ph = (consumed / kP2Stages) & 1;
+            if (!ring_wait(&bars[warp][st], ph, err)) return;
+            ++consumed;
+            const uint2 *src = reinterpret_cast<const uint2 *>(my_ring + (size_t)st * kStage) + lane;
+            const uint2 *bsrc = sB + lane;
+            int a4[4][4];
+#pragma unroll
+            for (int rb = 0; rb < 4; ++rb)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) a4[rb][c] = 0;
+            int kb = 0;
+            for (; kb + 4 <= KB2; kb += 4) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint2 w = src[(kb + u) * 32];
+                    const uint2 b = bsrc[(kb + u) * 32];
+#pragma unroll
+                    for (int rb = 0; rb < 4; ++rb) {
+                        const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                        mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+                    }
+                }
+            }
+            for (; kb < KB2; ++kb) {
+                const uint2 w = src[kb * 32];
+                const uint2 b = bsrc[kb * 32];
+#pragma unroll
+                for (int rb = 0; rb < 4; ++rb) {
+                    const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                    mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                const int rgn = rg + NW * kP2Stages;
+                if (rgn < item.rg1) {
+                    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                    const int sn = issued % kP2Stages;
+                    ring_fill(my_ring + (size_t)sn * kStage, ut + (size_t)rgn * KB2 * 32, stage_bytes, &bars[warp][sn]);
+                    ++issued;
+                }
+            }
+            // lane (m, path): its path's share of rows g and g + 8, then the pair sum
+            const float *hrow = sH + lane_p * kRows + (rg * kRowsPerGroup - n0) + g;
+#pragma unroll
+            for (int rb = 0; rb < 4; ++rb) {
+                const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
+                const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
+                float vlo = hrow[rb * kRowsPerBlock] * fmaf((float)Tlo, my_sc, my_q);
+                float vhi = hrow[rb * kRowsPerBlock + 8] * fmaf((float)Thi, my_sc, my_q);
+                vlo += __shfl_xor_sync(0xffffffffu, vlo, 1);
+                vhi += __shfl_xor_sync(0xffffffffu, vhi, 1);
+                const int nlo = rg * kRowsPerGroup + rb * kRowsPerBlock + g;
+                if (lane_p == 0 && lane_m < M) {
+                    if (nlo < N) y[(size_t)lane_m * N + nlo] = vlo;
+                    if (nlo + 8 < N) y[(size_t)lane_m * N + nlo + 8] = vhi;
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+lb_status decode_pair_launch(const LayerDev *dev_layers, const P1Item *p1, int n1, const P2Item *p2, int n2,
+                             const IoPtrs &io, int base, int M, int kb2max, int *err, cudaStream_t s, int *launches,
+                             bool mark)
+{
+    static int sms = 0, set1 = 0, set2 = 0;
+    cudaError_t e;
+    if (!sms) {
+        int dev = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return status_from(e);
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return status_from(e);
+    }
+    const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * kP1StageKB * 256 +
+                         (size_t)kP1ChunkKB * 32 * sizeof(uint2);
+    const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * kb2max * 256 + (size_t)kb2max * 32 * sizeof(uint2) +
+                         (size_t)2 * kP2ItemGroups * kRowsPerGroup * sizeof(float);
+    if (smem2 > 227 * 1024) return LB_ERR_UNSUPPORTED;
+    if ((int)smem1 > set1) {
+        if ((e = cudaFuncSetAttribute(contraction1_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) !=
+            cudaSuccess)
+            return status_from(e);
+        set1 = (int)smem1;
+    }
+    if ((int)smem2 > set2) {
+        if ((e = cudaFuncSetAttribute(contraction2_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)) !=
+            cudaSuccess)
+            return status_from(e);
+        set2 = (int)smem2;
+    }
+    int occ1 = 0, occ2 = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, contraction1_pair_kernel, kDecodeThreads, smem1)) !=
+        cudaSuccess)
+        return status_from(e);
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ2, contraction2_pair_kernel, kDecodeThreads, smem2)) !=
+        cudaSuccess)
+        return status_from(e);
+    const int grid1 = std::max(1, std::min(n1, sms * std::max(1, occ1)));
+    const int grid2 = std::max(1, std::min(n2, sms * std::max(1, occ2)));
+    contraction1_pair_kernel<<<grid1, kDecodeThreads, smem1, s>>>(dev_layers, p1, n1, io, base, M, err);
+    ++*launches;
+    if (mark) profile_mark(*launches, s);
+    contraction2_pair_kernel<<<grid2, kDecodeThreads, smem2, s>>>(dev_layers, p2, n2, io, base, M, kb2max, err);
+    ++*launches;
+    if (mark) profile_mark(*launches, s);
+    return status_from(cudaGetLastError());
+}
+
+}  // namespace lb

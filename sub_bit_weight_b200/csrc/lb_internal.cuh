@@ -126,6 +126,9 @@ void plan_free(Plan &P);
 lb_status decode_forward(const Plan &P, const uint16_t *const *xs, float *const *ys, int M,
                          cudaStream_t s, int *launches);
 
+lb_status decode_pair_launch(const LayerDev *dev_layers, const P1Item *p1, int n1, const P2Item *p2, int n2,
+                             const IoPtrs &io, int base, int M, int kb2max, int *err, cudaStream_t s, int *launches,
+                             bool mark);
 lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc, const P1Item *p1, int n1,
                             const P2Item *p2, int n2, const uint16_t *x, float *y, int M, int *err, cudaStream_t s,
                             int *launches);
