@@ -525,6 +525,16 @@ static void kernels_for(K1Fn &k1, K2Fn &k2)
 static int g_sms = 0;
 static int g_smem_set1[kMaxNT + 1] = {0}, g_smem_set2[kMaxNT + 1] = {0};
 
+// Raise a kernel's dynamic shared-memory limit to at least `bytes`, never lower it:
+// every launch path of that kernel shares the cached value.
+static cudaError_t ensure_smem(const void *fn, size_t bytes, int &cached)
+{
+    if ((int)bytes <= cached) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) cached = (int)bytes;
+    return e;
+}
+
 lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const *ys, int M, cudaStream_t s,
                          int *launches)
 {
@@ -566,16 +576,8 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
     const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * kb2max * 256 +
                          (size_t)NT * kb2max * 32 * sizeof(uint2);
     if (smem2 > 227 * 1024) return LB_ERR_UNSUPPORTED;
-    if ((int)smem1 > g_smem_set1[NT]) {
-        if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) != cudaSuccess)
-            return status_from(e);
-        g_smem_set1[NT] = (int)smem1;
-    }
-    if ((int)smem2 > g_smem_set2[NT]) {
-        if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)) != cudaSuccess)
-            return status_from(e);
-        g_smem_set2[NT] = (int)smem2;
-    }
+    if ((e = ensure_smem((const void *)k1, smem1, g_smem_set1[NT])) != cudaSuccess) return status_from(e);
+    if ((e = ensure_smem((const void *)k2, smem2, g_smem_set2[NT])) != cudaSuccess) return status_from(e);
     int occ1 = 0, occ2 = 0;
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, k1, kDecodeThreads, smem1)) != cudaSuccess)
         return status_from(e);
@@ -645,10 +647,8 @@ lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc,
     const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * kb2max * 256 +
                          (size_t)NT * kb2max * 32 * sizeof(uint2);
     if (smem2 > 227 * 1024) return LB_ERR_UNSUPPORTED;
-    if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) != cudaSuccess)
-        return status_from(e);
-    if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)) != cudaSuccess)
-        return status_from(e);
+    if ((e = ensure_smem((const void *)k1, smem1, g_smem_set1[NT])) != cudaSuccess) return status_from(e);
+    if ((e = ensure_smem((const void *)k2, smem2, g_smem_set2[NT])) != cudaSuccess) return status_from(e);
     int occ1 = 0, occ2 = 0;
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, k1, kDecodeThreads, smem1)) != cudaSuccess)
         return status_from(e);

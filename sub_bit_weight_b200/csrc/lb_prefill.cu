@@ -331,11 +331,11 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v)
 // ---------------------------------------------------------------------------
 struct PfSmem {
     alignas(1024) unsigned char A[kPfStages][kPfBM * kPfBK * 2];
-    alignas(1024) unsigned char B[kPfStages][kPfBN * kPfBK * 2];
-    alignas(16) uint32_t bits[kPfStages][256 * 4];
+    alignas(1024) unsigned char B[kPfStages][kPfBN * kPfBK * 2];   // the stage's sign bits land in its first 4 KB
+    alignas(1024) unsigned char ST[4][32 * 128];  // output GEMM epilogue: 32x32 fp32 block per warp (128B swizzle)
     alignas(16) __half gst[kPfStages][128];     // latent GEMM: g of both paths for the stage's k-block
     alignas(16) float lsc[kPfBN];               // latent GEMM epilogue: l of the tile's columns
-    uint64_t full[kPfStages], ready[kPfStages], empty[kPfStages];
+    uint64_t full[kPfStages], ready[kPfStages], empty[kPfStages], bread[kPfStages];
     uint64_t accf[2], acce[2];
     uint32_t tmem_base;
     int abort;
@@ -356,7 +356,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < kPfStages; ++s) {
             mbar_init(&S.full[s], 1);
-            mbar_init(&S.ready[s], 8);
+            mbar_init(&S.ready[s], MODE == 0 ? 10 : 8);   // generator warps (+ converter warps)
+            mbar_init(&S.bread[s], 8);                    // generator warps have read the stage's sign bits
             mbar_init(&S.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -405,7 +406,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     if (!mbar_wait(&S.empty[s], ph ^ 1, abort, err, 1)) break;
                     mbar_expect_tx(&S.full[s], kPfBM * kPfBK * 2 + 4096 + (MODE == 0 ? 256 : 0));
                     tma_load_2d(S.A[s], ly.tmA, kb * kPfBK, mt * kPfBM, &S.full[s]);
-                    bulk_load(S.bits[s], bits + (size_t)kb * 1024, 4096, &S.full[s]);
+                    bulk_load(S.B[s], bits + (size_t)kb * 1024, 4096, &S.full[s]);
                     if (MODE == 0) bulk_load(S.gst[s], ly.base + (size_t)kb * 128, 256, &S.full[s]);
                     pend |= 1u << s;
                     pend_ph = (pend_ph & ~(1u << s)) | (ph << s);
@@ -456,6 +457,40 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 tc_commit(&S.accf[ab]);
             }
         }
+    } else if (warp == 2 || warp == 3) {
+        // ---------------- converters (latent GEMM): bf16 -> fp16 A tile in place
+        if (MODE == 0) {
+            const int ct = tid - 64;   // 0..63
+            uint32_t it = 0;
+            for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
+                int L, mt, nt;
+                locate(t, L, mt, nt);
+                const int nk = layers[L].nk;
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kPfStages;
+                    const uint32_t ph = (it / kPfStages) & 1;
+                    if (!mbar_wait(&S.full[s], ph, abort, err, 7)) {
+                        ok = false;
+                        break;
+                    }
+                    uint4 *A4 = reinterpret_cast<uint4 *>(S.A[s]);
+#pragma unroll 4
+                    for (int i = 0; i < kPfBM * kPfBK * 2 / 16 / 64; ++i) {
+                        uint4 v = A4[ct + 64 * i];
+                        v.x = bf16x2_to_f16x2(v.x);
+                        v.y = bf16x2_to_f16x2(v.y);
+                        v.z = bf16x2_to_f16x2(v.z);
+                        v.w = bf16x2_to_f16x2(v.w);
+                        A4[ct + 64 * i] = v;
+                    }
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.ready[s]);
+                }
+                if (!ok) break;
+            }
+        }
     } else if (warp >= 4 && warp < 8) {
         // ---------------- epilogue
         const int q = warp - 4;
@@ -483,8 +518,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 uint32_t v[32];
                 tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * kPfBN + ch), v);
                 const int c0 = nt * kPfBN + ch;
-                if (m < M) {
-                    if (MODE == 0) {
+                if (MODE == 0) {
+                    if (m < M) {
                         __half *out = reinterpret_cast<__half *>(ly.out) + (size_t)m * ly.ld_out + c0;
                         uint32_t hw[16];
 #pragma unroll
@@ -505,17 +540,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                             for (int i = 0; i < 16; ++i)
                                 if (c0 + 2 * i < ly.ncols) reinterpret_cast<uint32_t *>(out)[i] = hw[i];
                         }
-                    } else {
-                        float *out = reinterpret_cast<float *>(ly.out) + (size_t)m * ly.ld_out + c0;
-                        if (c0 + 32 <= ly.ncols && (ly.ld_out & 3) == 0) {
+                    }
+                }
+                if (MODE == 1) {
+                    // 32 rows x 32 columns of y through a 128B-swizzled block and one TMA store
+                    if (ch > 0 || tcount > 0) {
+                        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+                        __syncwarp();
+                    }
+                    unsigned char *st = S.ST[q];
 #pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                reinterpret_cast<uint4 *>(out)[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (c0 + i < ly.ncols) out[i] = __uint_as_float(v[i]);
-                        }
+                    for (int i = 0; i < 8; ++i)
+                        *reinterpret_cast<uint4 *>(st + sw128(lane, i)) = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0 && mt * kPfBM + q * 32 < M) {
+                        asm volatile(
+                            "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(ly.tmY),
+                            "r"(c0), "r"(mt * kPfBM + q * 32), "r"(smem_u32(st))
+                            : "memory");
+                        asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
                     }
                 }
             }
@@ -554,15 +598,22 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     break;
                 }
                 unsigned char *Bt = S.B[s];
-                const uint32_t *bits = S.bits[s];
+                const uint32_t *bits = reinterpret_cast<const uint32_t *>(Bt);   // [256 rows][4 words]
                 if (MODE == 0) {
                     // thread -> chunk c (8 inputs), rows gt/8 + 32 i
                     const int c = gt & 7;
-                    const int k = kb * kPfBK + 8 * c;
+                    uint32_t R[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) R[i] = bits[((gt >> 3) + 32 * i) * 4 + (c >> 1)];
                     uint4 gb[2];
 #pragma unroll
                     for (int p = 0; p < 2; ++p) gb[p] = *reinterpret_cast<const uint4 *>(S.gst[s] + p * 64 + 8 * c);
-                    (void)k;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.bread[s]);
+                    if (!mbar_wait(&S.bread[s], ph, abort, err, 8)) {   // every generator has its bits
+                        ok = false;
+                        break;
+                    }
                     const int sh0 = 4 * (c & 1);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
@@ -570,32 +621,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         if (row < nw) {
                             const int jr = nt * kPfBN + row;
                             const uint4 base = (jr >= ly.r8 && ly.npaths > 1) ? gb[1] : gb[0];
-                            const uint32_t R = bits[row * 4 + (c >> 1)];
                             uint4 o;
-                            o.x = ((R << (sh0 + 0)) & 0x80008000u) ^ base.x;
-                            o.y = ((R << (sh0 + 1)) & 0x80008000u) ^ base.y;
-                            o.z = ((R << (sh0 + 2)) & 0x80008000u) ^ base.z;
-                            o.w = ((R << (sh0 + 3)) & 0x80008000u) ^ base.w;
+                            o.x = ((R[i] << (sh0 + 0)) & 0x80008000u) ^ base.x;
+                            o.y = ((R[i] << (sh0 + 1)) & 0x80008000u) ^ base.y;
+                            o.z = ((R[i] << (sh0 + 2)) & 0x80008000u) ^ base.z;
+                            o.w = ((R[i] << (sh0 + 3)) & 0x80008000u) ^ base.w;
                             *reinterpret_cast<uint4 *>(Bt + sw128(row, c)) = o;
                         }
-                    }
-                    // A tile: bf16 -> fp16 in place (element positions are unchanged)
-                    unsigned char *At = S.A[s];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        uint4 *p4 = reinterpret_cast<uint4 *>(At) + gt + 256 * i;
-                        uint4 v = *p4;
-                        v.x = bf16x2_to_f16x2(v.x);
-                        v.y = bf16x2_to_f16x2(v.y);
-                        v.z = bf16x2_to_f16x2(v.z);
-                        v.w = bf16x2_to_f16x2(v.w);
-                        *p4 = v;
                     }
                 } else {
                     // thread -> row gt, all 8 chunks
                     const int row = gt;
+                    const uint4 Rw = *reinterpret_cast<const uint4 *>(bits + row * 4);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.bread[s]);
+                    if (!mbar_wait(&S.bread[s], ph, abort, err, 8)) {   // every generator has its bits
+                        ok = false;
+                        break;
+                    }
                     if (row < nw) {
-                        const uint4 Rw = *reinterpret_cast<const uint4 *>(bits + row * 4);
                         const uint32_t Rs[4] = {Rw.x, Rw.y, Rw.z, Rw.w};
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
@@ -621,6 +665,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
     }
 
+    if (MODE == 1 && warp >= 4 && warp < 8 && lane == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -647,11 +692,12 @@ static cudaError_t get_encoder()
     return g_encode ? cudaSuccess : cudaErrorNotSupported;
 }
 
-static bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, int cols, int rows)
+static bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, int cols, int rows,
+                      int esize = 2, int box_cols = kPfBK, int box_rows = kPfBM)
 {
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {kPfBK, kPfBM};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * esize};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     return g_encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -693,13 +739,13 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
     if (e != cudaSuccess) return LB_ERR_UNSUPPORTED;
     for (int i = 0; i < n; ++i) {
         const LayerDev &d = layers[i]->d;
-        if (d.K % 8) return LB_ERR_UNSUPPORTED;   // TMA row stride must be a multiple of 16 bytes
+        if (d.K % 8 || d.N % 4) return LB_ERR_UNSUPPORTED;   // TMA row strides must be multiples of 16 bytes
     }
     if (!P.pf) {
         P.pf = new (std::nothrow) PrefillState();
         if (!P.pf) return LB_ERR_OOM;
         PrefillState &st = *P.pf;
-        if ((e = cudaMalloc(&st.maps, sizeof(CUtensorMap) * 2 * n)) != cudaSuccess) return status_from(e);
+        if ((e = cudaMalloc(&st.maps, sizeof(CUtensorMap) * 3 * n)) != cudaSuccess) return status_from(e);
         if ((e = cudaMalloc(&st.rec, sizeof(PfLayer) * 2 * n)) != cudaSuccess) return status_from(e);
         if ((e = cudaMalloc(&st.starts, sizeof(int) * 2 * (n + 1))) != cudaSuccess) return status_from(e);
         if ((e = cudaMalloc(&st.err, sizeof(int))) != cudaSuccess) return status_from(e);
@@ -734,7 +780,7 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
     for (int i = 0; i < n && !dirty; ++i)
         if (st.lastX[i] != xs[i] || st.lastY[i] != ys[i]) dirty = true;
     if (dirty) {
-        std::vector<CUtensorMap> maps(2 * n);
+        std::vector<CUtensorMap> maps(3 * n);
         std::vector<PfLayer> rec(2 * n);
         std::vector<int> starts(2 * (n + 1));
         starts[0] = starts[n + 1] = 0;
@@ -743,11 +789,13 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
             const PfWeights &W = layers[i]->pf;
             __half *zl = (__half *)((char *)st.zl + st.zl_off[i]);
             if (!encode_2d(&maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xs[i], d.K, M) ||
-                !encode_2d(&maps[n + i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, zl, W.K2, M))
+                !encode_2d(&maps[n + i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, zl, W.K2, M) ||
+                !encode_2d(&maps[2 * n + i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ys[i], d.N, M, 4, 32, 32))
                 return LB_ERR_UNSUPPORTED;
             const int mtiles = ceil_div(M, kPfBM);
             PfLayer &a = rec[i];
             a.tmA = st.maps + i;
+            a.tmY = nullptr;
             a.bits = W.b1;
             a.base = W.g64;
             a.lcat = W.lcat;
@@ -761,6 +809,7 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
             a.npaths = d.npaths;
             PfLayer &b = rec[n + i];
             b.tmA = st.maps + n + i;
+            b.tmY = st.maps + 2 * n + i;
             b.bits = W.b2;
             b.base = W.h256;
             b.lcat = nullptr;
@@ -781,7 +830,7 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
         st.tiles[1] = starts[2 * n + 1];
         st.lastM = M;
         // pageable sources: the copies are staged before these calls return
-        if ((e = cudaMemcpyAsync(st.maps, maps.data(), sizeof(CUtensorMap) * 2 * n, cudaMemcpyHostToDevice, s)) !=
+        if ((e = cudaMemcpyAsync(st.maps, maps.data(), sizeof(CUtensorMap) * 3 * n, cudaMemcpyHostToDevice, s)) !=
             cudaSuccess)
             return status_from(e);
         if ((e = cudaMemcpyAsync(st.rec, rec.data(), sizeof(PfLayer) * 2 * n, cudaMemcpyHostToDevice, s)) != cudaSuccess)

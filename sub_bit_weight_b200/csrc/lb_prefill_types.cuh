@@ -27,6 +27,7 @@ struct PfWeights {
 // Per-layer launch record of a tensor-core contraction.
 struct PfLayer {
     const CUtensorMap *tmA;   // A operand (activations) tensor map
+    const CUtensorMap *tmY;   // output GEMM: y tensor map (32 x 32 fp32 boxes)
     const uint32_t *bits;     // generated operand, spread layout
     const __half *base;       // g64 (latent) or h256 (output)
     const float *lcat;        // latent scales per output column (latent contraction only)

@@ -40,6 +40,23 @@ def test_noalloc_matches_forward_on_consecutive_calls():
         assert err <= TOL, (s, M, err)
 
 
+def test_regular_calls_still_work_after_noalloc_calls():
+    # the two entry points share kernel launch settings; a larger layer afterwards must still launch
+    import torch
+    from sub_bit_weight_b200 import lib, stacks
+    small = synth.LayerShape("s", 256, 512, 32)
+    big = synth.LayerShape("b", 1024, 4096, 800)
+    Ls, Lb = stacks.build_layer(74, 0, small), stacks.build_layer(75, 1, big)
+    for M in (1, 16):
+        xs = stacks.bf16_on_device(synth.activations(84, 0, M, small.K), "cuda")
+        lib.lb_linear_forward_noalloc(xs, Ls, torch.empty((M, small.N), dtype=torch.float32, device="cuda"))
+        xb = stacks.bf16_on_device(synth.activations(85, 0, M, big.K), "cuda")
+        y1 = lib.lb_linear_forward(xb, Lb)
+        y2 = lib.lb_linear_forward_noalloc(xb, Lb, torch.empty_like(y1))
+        torch.cuda.synchronize()
+        assert rel_err(y2.cpu().numpy(), y1.cpu().numpy()) <= TOL
+
+
 def test_noalloc_rejects_batches_above_the_decode_limit():
     import torch
     from sub_bit_weight_b200 import lib, stacks
