@@ -191,6 +191,27 @@ LB_API lb_status lb_stack_forward(lb_stack *S, const uint16_t *const *xs, float 
 #define LB_NOALLOC_SCRATCH_BYTES (1u << 20)
 LB_API lb_status lb_linear_forward_noalloc(const uint16_t *x, int M, const lb_layer *L, float *y, void *stream);
 
+/*
+ * Device-side failure reporting.  Every wait inside the library's kernels is
+ * bounded (about two seconds of clock ticks); a wait that gives up records an
+ * error code in the plan's device memory and its kernel returns instead of
+ * hanging.  These calls synchronise `stream`, read that code, clear it, and
+ * return LB_ERR_TIMEOUT if a wait gave up since the last check (LB_OK if not).
+ * A timed-out call leaves its outputs unspecified.
+ * Errors: LB_ERR_INVALID_ARG (NULL), LB_ERR_CUDA.
+ */
+LB_API lb_status lb_stack_status(lb_stack *S, void *stream);
+LB_API lb_status lb_layer_status(const lb_layer *L, void *stream);
+
+/*
+ * Self-test of the bounded-wait mechanism: launches one thread that waits, with
+ * the same helper the kernels use, on an mbarrier that nothing completes,
+ * giving up after `cycles` clock ticks.  Synchronises `stream`; returns
+ * LB_ERR_TIMEOUT when the wait gave up and reported it (the expected result),
+ * LB_OK if it did not.  No GPU fault or hang is involved.
+ */
+LB_API lb_status lb_selftest_wait_timeout(long long cycles, void *stream);
+
 /* Timing hook.  Registers n CUDA events (cudaEvent_t passed as void*) for the
  * calling thread: the following forward calls record events[0] on their
  * stream before their first kernel launch and events[i] right after their

@@ -112,12 +112,13 @@ static __device__ __forceinline__ bool bar_try(uint64_t *b, uint32_t parity)
 constexpr long long kDecWaitCycles = 4000000000LL;   // ~2 s
 
 // Bounded wait for a ring buffer; false (and an error code) on timeout.
-static __device__ __forceinline__ bool ring_wait(uint64_t *b, uint32_t parity, int *err)
+static __device__ __forceinline__ bool ring_wait(uint64_t *b, uint32_t parity, int *err,
+                                                 long long limit = kDecWaitCycles)
 {
     if (bar_try(b, parity)) return true;
     const long long t0 = clock64();
     while (!bar_try(b, parity)) {
-        if (clock64() - t0 > kDecWaitCycles) {
+        if (clock64() - t0 > limit) {
             atomicCAS(err, 0, 16);
             return false;
         }

@@ -5,7 +5,8 @@
 // sign(0) = +1: a bit is set iff the float compares below zero, so -0.0 and
 // NaN give +1.  Word i*ceil(r/32) + j/32, bit j%32 holds element (i, j).
 
-#include "lb_internal.cuh"
+#include "lb_decode_common.cuh"
+#include "lb_prefill.cuh"
 
 namespace lb {
 
@@ -47,6 +48,21 @@ __global__ void __launch_bounds__(256) pack_signs_kernel(const float *__restrict
     }
 }
 
+// Self-test of the bounded waits: one thread waits on an mbarrier that nothing
+// completes, gives up after `cycles` clock ticks and records the error code,
+// exactly as the decode kernels do when a bulk copy never lands.
+__global__ void wait_selftest_kernel(int *err, long long cycles)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        bar_init(&bar);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+        ring_wait(&bar, 0, err, cycles);   // phase 0 never completes
+    }
+}
+
+static int *g_selftest_err = nullptr;
+
 }  // namespace lb
 
 extern "C" {
@@ -71,6 +87,46 @@ size_t lb_packed_words(int64_t rows, int r)
 }
 
 int lb_last_launch_count(void) { return lb::g_last_launches; }
+
+static lb_status read_and_clear(int *dev_err, cudaStream_t s)
+{
+    int h = 0;
+    cudaError_t e = cudaMemcpyAsync(&h, dev_err, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess && h) e = cudaMemsetAsync(dev_err, 0, sizeof(int), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return lb::status_from(e);
+    return h ? LB_ERR_TIMEOUT : LB_OK;
+}
+
+lb_status lb_stack_status(lb_stack *S, void *stream)
+{
+    if (!S) return LB_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    lb_status st = read_and_clear(S->plan.err, s);
+    if (st == LB_OK && S->plan.pf) st = read_and_clear(lb::prefill_err_ptr(S->plan.pf), s);
+    return st;
+}
+
+lb_status lb_layer_status(const lb_layer *L, void *stream)
+{
+    if (!L) return LB_ERR_INVALID_ARG;
+    return lb_stack_status(L->self, stream);
+}
+
+lb_status lb_selftest_wait_timeout(long long cycles, void *stream)
+{
+    if (cycles < 0) return LB_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    if (!lb::g_selftest_err) {
+        if ((e = cudaMalloc(&lb::g_selftest_err, sizeof(int))) != cudaSuccess) return lb::status_from(e);
+    }
+    if ((e = cudaMemsetAsync(lb::g_selftest_err, 0, sizeof(int), s)) != cudaSuccess) return lb::status_from(e);
+    lb::wait_selftest_kernel<<<1, 32, 0, s>>>(lb::g_selftest_err, cycles);
+    if ((e = cudaGetLastError()) != cudaSuccess) return lb::status_from(e);
+    return read_and_clear(lb::g_selftest_err, s);
+}
 
 lb_status lb_profile_events(void *const *events, int n)
 {

@@ -717,6 +717,8 @@ struct PrefillState {
     int tiles[2] = {0, 0};
 };
 
+int *prefill_err_ptr(PrefillState *st) { return st->err; }
+
 void prefill_free(PrefillState *st)
 {
     if (!st) return;

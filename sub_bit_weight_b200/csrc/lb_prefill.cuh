@@ -22,5 +22,6 @@ struct PrefillState;   // per plan (owned by Plan)
 lb_status prefill_forward(const Plan &P, const lb_layer *const *layers, const uint16_t *const *xs,
                           float *const *ys, int M, cudaStream_t s, int *launches);
 void prefill_free(PrefillState *st);
+int *prefill_err_ptr(PrefillState *st);
 
 }  // namespace lb

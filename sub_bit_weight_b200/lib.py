@@ -54,6 +54,9 @@ _sig("lb_stack_destroy", None, [_vp])
 _sig("lb_stack_forward", _st, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp])
 _sig("lb_last_launch_count", _i, [])
 _sig("lb_profile_events", _st, [ctypes.POINTER(_vp), _i])
+_sig("lb_stack_status", _st, [_vp, _vp])
+_sig("lb_layer_status", _st, [_vp, _vp])
+_sig("lb_selftest_wait_timeout", _st, [ctypes.c_longlong, _vp])
 
 
 class LittleBitError(RuntimeError):
@@ -87,6 +90,19 @@ def _dev(t: torch.Tensor, dtype, name: str) -> int:
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return t.data_ptr()
+
+
+def lb_layer_status(layer, stream=None) -> int:
+    """Synchronise and return (and clear) the layer's device-side status: LB_OK or LB_ERR_TIMEOUT."""
+    return int(_lib.lb_layer_status(layer.handle, _stream(stream)))
+
+
+def lb_stack_status(stack, stream=None) -> int:
+    return int(_lib.lb_stack_status(stack.handle, _stream(stream)))
+
+
+def lb_selftest_wait_timeout(cycles: int, stream=None) -> int:
+    return int(_lib.lb_selftest_wait_timeout(int(cycles), _stream(stream)))
 
 
 def lb_packed_words(rows: int, r: int) -> int:
