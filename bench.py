@@ -49,6 +49,42 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
 
 
+# ----------------------------------------------------------------- measured DRAM traffic
+
+CSRC = os.path.join(ROOT, "sub_bit_weight_b200", "csrc")
+KERNEL_SOURCES = {
+    "contraction1_pair_kernel": ["lb_decode_pair.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
+    "contraction2_pair_kernel": ["lb_decode_pair.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
+    "contraction1_kernel": ["lb_decode.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
+    "contraction2_kernel": ["lb_decode.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
+    "prefill_kernel<0>": ["lb_prefill.cu", "lb_prefill.cuh", "lb_prefill_types.cuh", "lb_internal.cuh"],
+    "prefill_kernel<1>": ["lb_prefill.cu", "lb_prefill.cuh", "lb_prefill_types.cuh", "lb_internal.cuh"],
+}
+
+
+def source_hash(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kernel, []):
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from profiles/traffic.txt, only while the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = source_hash(kernel)
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload:
+                return float(parts[3]) if parts[2] == want else None
+    return None
+
+
 # ----------------------------------------------------------------- algorithmic work
 
 def layer_bytes(s: synth.LayerShape, M: int, npaths: int = 2):
@@ -305,19 +341,23 @@ def main():
             f2 = sum(2.0 * M * 2 * s.r * s.N for s in shapes)
             dom_w, dom_ms = (f2, k2ms) if dom else (f1, k1ms)
             ach = dom_w / (dom_ms * 1e-3) / 1e12
-            roof = {"bound": "tensor", "kernel": "prefill_kernel<1> (output GEMM)" if dom else "prefill_kernel<0> (latent GEMM)",
+            kname = "prefill_kernel<1>" if dom else "prefill_kernel<0>"
+            roof = {"bound": "tensor", "kernel": kname + (" (output GEMM)" if dom else " (latent GEMM)"),
                     "achieved": round(ach, 1), "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                     "frac": round(ach / pk["bf16_tflops_sustained"], 4),
-                    "peak_src": pk["src"] + " bf16 sustained (dense 16-bit tensor peak)", "traffic": None,
+                    "peak_src": pk["src"] + " bf16 sustained (dense 16-bit tensor peak)",
+                    "traffic": measured_traffic(kname, w.key),
                     "per_kernel_ms": {"latent": round(k1ms, 4), "output": round(k2ms, 4)},
                     "per_kernel_flops": {"latent": f1, "output": f2}}
         else:
             dom_bytes, dom_ms = (k2b, k2ms) if dom else (k1b, k1ms)
             ach = dom_bytes / (dom_ms * 1e-3) / 1e9
-            roof = {"bound": "hbm", "kernel": "contraction2_kernel" if dom else "contraction1_kernel",
+            suffix = "_pair_kernel" if M <= 2 else "_kernel"
+            kname = ("contraction2" if dom else "contraction1") + suffix
+            roof = {"bound": "hbm", "kernel": kname,
                     "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                     "frac": round(ach / pk["hbm_gbs"], 4), "peak_src": pk["src"],
-                    "traffic": None,
+                    "traffic": measured_traffic(kname, w.key), "algorithmic_bytes_per_launch": dom_bytes,
                     "per_kernel_ms": {"contraction1_kernel": round(k1ms, 5), "contraction2_kernel": round(k2ms, 5)},
                     "per_kernel_bytes": {"contraction1_kernel": k1b, "contraction2_kernel": k2b}}
     e2e = None

@@ -297,18 +297,19 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 const uint32_t ph = (consumed / kP1Stages) & 1;
                 if (!ring_wait(&bars[warp][st], ph, err)) return;
                 ++consumed;
-                const uint2 *src = reinterpret_cast<const uint2 *>(my_ring + st * kStage) + lane;
+                const uint32_t src = sm_addr(my_ring + st * kStage) + lane * 8;
+                const uint32_t bbase = sm_addr(sB) + lane * 8;
                 const int kbA = h * kHalf, n = min(kHalf, nkb - kbA);
 #pragma unroll 4
                 for (int u = 0; u < n; ++u) {
                     const int kb = kbA + u;
-                    const uint2 w = src[u * 32];
+                    const uint2 w = lds64(src + u * 256);
                     uint2 bp[2][NT];
 #pragma unroll
                     for (int p = 0; p < 2; ++p)
 #pragma unroll
                         for (int nn = 0; nn < NT; ++nn)
-                            bp[p][nn] = sB[(((size_t)p * kP1ChunkKB + kb) * NT + nn) * 32 + lane];
+                            bp[p][nn] = lds64(bbase + (uint32_t)(((p * kP1ChunkKB + kb) * NT + nn) * 256));
 #pragma unroll
                     for (int rb = 0; rb < 4; ++rb) {
                         const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
@@ -437,7 +438,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 }
             if (!ring_wait(&bars[warp][st], ph, err)) return;
             ++consumed;
-            const uint2 *src = reinterpret_cast<const uint2 *>(my_ring + (size_t)st * kStage) + lane;
+            const uint32_t src = sm_addr(my_ring + (size_t)st * kStage) + lane * 8;
+            const uint32_t bbase = sm_addr(sB) + lane * 8;
             float yv[4][NT][2];
 #pragma unroll
             for (int rb = 0; rb < 4; ++rb)
@@ -453,10 +455,10 @@ __global__ void __launch_bounds__(kDecodeThreads)
                         for (int c = 0; c < 4; ++c) a4[rb][n][c] = 0;
 #pragma unroll 4
                 for (int kb = p * kbp; kb < (p + 1) * kbp; ++kb) {
-                    const uint2 w = src[kb * 32];
+                    const uint2 w = lds64(src + kb * 256);
                     uint2 b[NT];
 #pragma unroll
-                    for (int n = 0; n < NT; ++n) b[n] = sB[((size_t)n * KB2 + kb) * 32 + lane];
+                    for (int n = 0; n < NT; ++n) b[n] = lds64(bbase + (uint32_t)((n * KB2 + kb) * 256));
 #pragma unroll
                     for (int rb = 0; rb < 4; ++rb) {
                         const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);

@@ -75,6 +75,22 @@ static __device__ __forceinline__ int warp_or(int v)
     return v;
 }
 
+// Explicit shared-memory loads on 32-bit shared-window addresses (a generic
+// pointer into dynamic shared memory may compile to a generic load).
+static __device__ __forceinline__ uint2 lds64(uint32_t addr)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
+static __device__ __forceinline__ float lds_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(v) : "r"(addr));
+    return v;
+}
+
 // non-negative floats order like their bit patterns
 static __device__ __forceinline__ void smem_max(float *a, float v) { atomicMax((int *)a, __float_as_int(v)); }
 

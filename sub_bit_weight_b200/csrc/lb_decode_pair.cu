@@ -282,14 +282,14 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 const uint32_t ph = (consumed / kP1Stages) & 1;
                 if (!ring_wait(&bars[warp][st], ph, err)) return;
                 ++consumed;
-                const uint2 *src = reinterpret_cast<const uint2 *>(my_ring + st * kStage) + lane;
-                const uint2 *bsrc = sB + (size_t)(h * kHalf) * 32 + lane;
+                const uint32_t src = sm_addr(my_ring + st * kStage) + lane * 8;
+                const uint32_t bsrc = sm_addr(sB + (size_t)(h * kHalf) * 32) + lane * 8;
                 const int n = min(kHalf, nkb - h * kHalf);
                 if (n == kHalf) {
 #pragma unroll
                     for (int u = 0; u < kHalf; ++u) {
-                        const uint2 w = src[u * 32];
-                        const uint2 b = bsrc[u * 32];
+                        const uint2 w = lds64(src + u * 256);
+                        const uint2 b = lds64(bsrc + u * 256);
 #pragma unroll
                         for (int rb = 0; rb < 4; ++rb) {
                             const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
@@ -298,8 +298,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
                     }
                 } else {
                     for (int u = 0; u < n; ++u) {
-                        const uint2 w = src[u * 32];
-                        const uint2 b = bsrc[u * 32];
+                        const uint2 w = lds64(src + u * 256);
+                        const uint2 b = lds64(bsrc + u * 256);
 #pragma unroll
                         for (int rb = 0; rb < 4; ++rb) {
                             const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
@@ -421,8 +421,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
             const uint32_t ph = (consumed / kP2Stages) & 1;
             if (!ring_wait(&bars[warp][st], ph, err)) return;
             ++consumed;
-            const uint2 *src = reinterpret_cast<const uint2 *>(my_ring + (size_t)st * kStage) + lane;
-            const uint2 *bsrc = sB + lane;
+            const uint32_t src = sm_addr(my_ring + (size_t)st * kStage) + lane * 8;
+            const uint32_t bsrc = sm_addr(sB) + lane * 8;
             int a4[4][4];
 #pragma unroll
             for (int rb = 0; rb < 4; ++rb)
@@ -432,8 +432,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
             for (; kb + 4 <= KB2; kb += 4) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const uint2 w = src[(kb + u) * 32];
-                    const uint2 b = bsrc[(kb + u) * 32];
+                    const uint2 w = lds64(src + (kb + u) * 256);
+                    const uint2 b = lds64(bsrc + (kb + u) * 256);
 #pragma unroll
                     for (int rb = 0; rb < 4; ++rb) {
                         const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
@@ -442,8 +442,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 }
             }
             for (; kb < KB2; ++kb) {
-                const uint2 w = src[kb * 32];
-                const uint2 b = bsrc[kb * 32];
+                const uint2 w = lds64(src + kb * 256);
+                const uint2 b = lds64(bsrc + kb * 256);
 #pragma unroll
                 for (int rb = 0; rb < 4; ++rb) {
                     const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
@@ -461,13 +461,13 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 }
             }
             // lane (m, path): its path's share of rows g and g + 8, then the pair sum
-            const float *hrow = sH + lane_p * kRows + (rg * kRowsPerGroup - n0) + g;
+            const uint32_t hrow = sm_addr(sH + lane_p * kRows + (rg * kRowsPerGroup - n0) + g);
 #pragma unroll
             for (int rb = 0; rb < 4; ++rb) {
                 const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
                 const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
-                float vlo = hrow[rb * kRowsPerBlock] * fmaf((float)Tlo, my_sc, my_q);
-                float vhi = hrow[rb * kRowsPerBlock + 8] * fmaf((float)Thi, my_sc, my_q);
+                float vlo = lds_f32(hrow + 4 * rb * kRowsPerBlock) * fmaf((float)Tlo, my_sc, my_q);
+                float vhi = lds_f32(hrow + 4 * (rb * kRowsPerBlock + 8)) * fmaf((float)Thi, my_sc, my_q);
                 vlo += __shfl_xor_sync(0xffffffffu, vlo, 1);
                 vhi += __shfl_xor_sync(0xffffffffu, vhi, 1);
                 const int nlo = rg * kRowsPerGroup + rb * kRowsPerBlock + g;
