@@ -125,12 +125,46 @@ __global__ void __launch_bounds__(kDecodeThreads)
     uint32_t issued = 0, consumed = 0;
     unsigned char *my_ring = ring + warp * kP1Stages * kStage;
 
+    // Fill cursor: this warp's stages (item, row group, part) in the order the
+    // warp consumes them; it runs kP1Stages ahead, across item boundaries.
+    int f_it = blockIdx.x, f_q = 0, f_nseq = 0, f_hp = 1, f_kb0 = 0, f_nkb = 0, f_KB1 = 0;
+    const uint2 *f_vt = nullptr;
+    auto f_load = [&]() {
+        if (f_it >= nitems) return;
+        const P1Item fi = items[f_it];
+        const LayerDev *fd = layers + fi.layer;
+        f_KB1 = fd->KB1;
+        f_kb0 = fi.kc * kP1ChunkKB;
+        f_nkb = min(kP1ChunkKB, f_KB1 - f_kb0);
+        f_hp = (f_nkb + kHalf - 1) / kHalf;
+        f_nseq = max(0, (fd->RG1 - warp + NW - 1) / NW) * f_hp;
+        f_q = 0;
+        f_vt = fd->vt;
+    };
+    auto fill_next = [&]() {
+        while (f_it < nitems && f_q >= f_nseq) {
+            f_it += gridDim.x;
+            f_load();
+        }
+        if (f_it >= nitems) return;
+        const int rg = warp + NW * (f_q / f_hp), h = f_q % f_hp;
+        const int n = min(kHalf, f_nkb - h * kHalf);
+        if (lane == 0) {
+            const int st = issued % kP1Stages;
+            ring_fill(my_ring + st * kStage, f_vt + ((size_t)rg * f_KB1 + f_kb0 + h * kHalf) * 32, (unsigned)n * 256u,
+                      &bars[warp][st]);
+        }
+        ++issued;
+        ++f_q;
+    };
+    f_load();
+    for (int s = 0; s < kP1Stages; ++s) fill_next();
+
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
         const P1Item item = items[it];
         const LayerDev *dp = layers + item.layer;
         const int K = dp->K, K32 = dp->K32, KB1 = dp->KB1, RG1 = dp->RG1, r16 = dp->r16, npaths = dp->npaths;
         const int R1 = dp->R1;
-        const uint2 *__restrict__ vt = dp->vt;
         const __half *__restrict__ gsc = dp->g;
         double *__restrict__ acc = dp->acc;
         const uint16_t *__restrict__ x = io.x[item.layer - base];
@@ -140,17 +174,6 @@ __global__ void __launch_bounds__(kDecodeThreads)
         const int klen = nkb * kKPerBlock;
         const int hp = (nkb + kHalf - 1) / kHalf;
         const int nmine = (RG1 - warp + NW - 1) / NW;
-        const int nseq = max(0, nmine) * hp;
-        auto fill = [&](int q) {
-            const int rg = warp + NW * (q / hp), h = q % hp;
-            const int n = min(kHalf, nkb - h * kHalf);
-            const int st = issued % kP1Stages;
-            ring_fill(my_ring + st * kStage, vt + ((size_t)rg * KB1 + kb0 + h * kHalf) * 32, (unsigned)n * 256u,
-                      &bars[warp][st]);
-            ++issued;
-        };
-        if (lane == 0)
-            for (int q = 0; q < min(kP1Stages, nseq); ++q) fill(q);
 
         {
             uint4 *z4 = (uint4 *)sB;
@@ -308,13 +331,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
                     }
                 }
                 __syncwarp();
-                if (lane == 0) {
-                    const int q = rgi * hp + h + kP1Stages;
-                    if (q < nseq) {
-                        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-                        fill(q);
-                    }
-                }
+                if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                fill_next();
             }
             // keep the columns of each row block's own path
 #pragma unroll
@@ -370,24 +388,43 @@ __global__ void __launch_bounds__(kDecodeThreads)
     uint32_t issued = 0, consumed = 0;
     unsigned char *my_ring = ring + (size_t)warp * kP2Stages * kStage;
 
+    // Fill cursor over this warp's (item, row group) sequence, kP2Stages ahead
+    // of the consumer and across item boundaries.
+    int f_it = blockIdx.x, f_rg = 0, f_end = 0, f_kb2 = 0;
+    const uint2 *f_ut = nullptr;
+    auto f_load = [&]() {
+        if (f_it >= nitems) return;
+        const P2Item fi = items[f_it];
+        const LayerDev *fd = layers + fi.layer;
+        f_rg = fi.rg0 + warp;
+        f_end = fi.rg1;
+        f_ut = fd->ut;
+        f_kb2 = fd->KB2;
+    };
+    auto fill_next = [&]() {
+        while (f_it < nitems && f_rg >= f_end) {
+            f_it += gridDim.x;
+            f_load();
+        }
+        if (f_it >= nitems) return;
+        if (lane == 0) {
+            const int st = issued % kP2Stages;
+            ring_fill(my_ring + (size_t)st * kStage, f_ut + (size_t)f_rg * f_kb2 * 32, (unsigned)f_kb2 * 256u,
+                      &bars[warp][st]);
+        }
+        ++issued;
+        f_rg += NW;
+    };
+    f_load();
+    for (int s = 0; s < kP2Stages; ++s) fill_next();
+
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
         const P2Item item = items[it];
         const LayerDev *dp = layers + item.layer;
         const int N = dp->N, N64 = dp->N64, KB2 = dp->KB2, npaths = dp->npaths;
-        const uint2 *__restrict__ ut = dp->ut;
         const __half *__restrict__ hsc = dp->h;
         float *__restrict__ y = io.y[item.layer - base];
-        const unsigned stage_bytes = (unsigned)KB2 * 256u;
 
-        if (lane == 0)
-            for (int s = 0; s < kP2Stages; ++s) {
-                const int rg = item.rg0 + warp + NW * s;
-                if (rg < item.rg1) {
-                    const int st = issued % kP2Stages;
-                    ring_fill(my_ring + (size_t)st * kStage, ut + (size_t)rg * KB2 * 32, stage_bytes, &bars[warp][st]);
-                    ++issued;
-                }
-            }
         {
             const uint4 *src = reinterpret_cast<const uint4 *>(dp->zfrag);
             uint4 *dst = reinterpret_cast<uint4 *>(sB);
@@ -451,15 +488,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 }
             }
             __syncwarp();
-            if (lane == 0) {
-                const int rgn = rg + NW * kP2Stages;
-                if (rgn < item.rg1) {
-                    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-                    const int sn = issued % kP2Stages;
-                    ring_fill(my_ring + (size_t)sn * kStage, ut + (size_t)rgn * KB2 * 32, stage_bytes, &bars[warp][sn]);
-                    ++issued;
-                }
-            }
+            if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+            fill_next();
             // lane (m, path): its path's share of rows g and g + 8, then the pair sum
             const uint32_t hrow = sm_addr(sH + lane_p * kRows + (rg * kRowsPerGroup - n0) + g);
 #pragma unroll

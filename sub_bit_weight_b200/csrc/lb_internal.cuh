@@ -35,7 +35,7 @@ constexpr int kRowsPerBlock = 16;
 constexpr int kRowsPerGroup = 64;
 constexpr int kKPerBlock = 32;
 constexpr int kP1ChunkKB = 32;          // k-blocks per contraction-1 work item (1024 inputs)
-constexpr int kP2ItemGroups = 8;        // row groups per contraction-2 work item (512 outputs)
+constexpr int kP2ItemGroups = 16;       // row groups per contraction-2 work item (1024 outputs)
 constexpr int kDecodeThreads = 128;     // 4 warps
 constexpr int kMaxDecodeM = LB_DECODE_MAX_M;
 constexpr int kMaxNT = (kMaxDecodeM + 3) / 4;   // n-tiles of 4 activation rows

@@ -311,6 +311,26 @@ __device__ __forceinline__ uint32_t idesc_f16(int n)
     return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kPfBM >> 4) << 24);
 }
 
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v)
+{
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(addr));
+    return v;
+}
+
 // Byte offset of 16-byte chunk c of row `row` in a 128-byte-swizzled tile.
 __device__ __forceinline__ uint32_t sw128(int row, int c)
 {
@@ -348,7 +368,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                    int *err)
 {
     extern __shared__ __align__(1024) unsigned char pf_raw[];
-    PfSmem &S = *reinterpret_cast<PfSmem *>((reinterpret_cast<uintptr_t>(pf_raw) + 1023) & ~(uintptr_t)1023);
+    // align inside the shared window by an offset, keeping the pointer a shared-memory pointer
+    const uint32_t raw_addr = smem_u32(pf_raw);
+    PfSmem &S = *reinterpret_cast<PfSmem *>(pf_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     volatile int *abort = &S.abort;
 
@@ -474,15 +496,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         ok = false;
                         break;
                     }
-                    uint4 *A4 = reinterpret_cast<uint4 *>(S.A[s]);
+                    const uint32_t A4 = smem_u32(S.A[s]) + 16u * ct;
 #pragma unroll 4
                     for (int i = 0; i < kPfBM * kPfBK * 2 / 16 / 64; ++i) {
-                        uint4 v = A4[ct + 64 * i];
+                        uint4 v = lds128(A4 + 1024u * i);
                         v.x = bf16x2_to_f16x2(v.x);
                         v.y = bf16x2_to_f16x2(v.y);
                         v.z = bf16x2_to_f16x2(v.z);
                         v.w = bf16x2_to_f16x2(v.w);
-                        A4[ct + 64 * i] = v;
+                        sts128(A4 + 1024u * i, v);
                     }
                     fence_proxy_async();
                     __syncwarp();
@@ -525,8 +547,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int c = c0 + 2 * i;
-                            const float a = __uint_as_float(v[2 * i]) * S.lsc[ch + 2 * i];
-                            const float b = __uint_as_float(v[2 * i + 1]) * S.lsc[ch + 2 * i + 1];
+                            const uint32_t la = smem_u32(&S.lsc[ch + 2 * i]);
+                            const float a = __uint_as_float(v[2 * i]) * __uint_as_float(lds32(la));
+                            const float b = __uint_as_float(v[2 * i + 1]) * __uint_as_float(lds32(la + 4));
                             (void)c;
                             const __half2 hh = __floats2half2_rn(a, b);
                             hw[i] = *reinterpret_cast<const uint32_t *>(&hh);
@@ -549,9 +572,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         __syncwarp();
                     }
                     unsigned char *st = S.ST[q];
+                    const uint32_t sta = smem_u32(st);
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
-                        *reinterpret_cast<uint4 *>(st + sw128(lane, i)) = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                        sts128(sta + sw128(lane, i), make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
                     fence_proxy_async();
                     __syncwarp();
                     if (lane == 0 && mt * kPfBM + q * 32 < M) {
@@ -597,17 +621,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     ok = false;
                     break;
                 }
-                unsigned char *Bt = S.B[s];
-                const uint32_t *bits = reinterpret_cast<const uint32_t *>(Bt);   // [256 rows][4 words]
+                const uint32_t Bt = smem_u32(S.B[s]);   // sign bits first: [256 rows][4 words]
                 if (MODE == 0) {
                     // thread -> chunk c (8 inputs), rows gt/8 + 32 i
                     const int c = gt & 7;
                     uint32_t R[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) R[i] = bits[((gt >> 3) + 32 * i) * 4 + (c >> 1)];
+                    for (int i = 0; i < 8; ++i) R[i] = lds32(Bt + 4u * (((gt >> 3) + 32 * i) * 4 + (c >> 1)));
                     uint4 gb[2];
 #pragma unroll
-                    for (int p = 0; p < 2; ++p) gb[p] = *reinterpret_cast<const uint4 *>(S.gst[s] + p * 64 + 8 * c);
+                    for (int p = 0; p < 2; ++p) gb[p] = lds128(smem_u32(S.gst[s] + p * 64 + 8 * c));
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.bread[s]);
                     if (!mbar_wait(&S.bread[s], ph, abort, err, 8)) {   // every generator has its bits
@@ -626,13 +649,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                             o.y = ((R[i] << (sh0 + 1)) & 0x80008000u) ^ base.y;
                             o.z = ((R[i] << (sh0 + 2)) & 0x80008000u) ^ base.z;
                             o.w = ((R[i] << (sh0 + 3)) & 0x80008000u) ^ base.w;
-                            *reinterpret_cast<uint4 *>(Bt + sw128(row, c)) = o;
+                            sts128(Bt + sw128(row, c), o);
                         }
                     }
                 } else {
                     // thread -> row gt, all 8 chunks
                     const int row = gt;
-                    const uint4 Rw = *reinterpret_cast<const uint4 *>(bits + row * 4);
+                    const uint4 Rw = lds128(Bt + 16u * row);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.bread[s]);
                     if (!mbar_wait(&S.bread[s], ph, abort, err, 8)) {   // every generator has its bits
@@ -652,7 +675,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                             o.y = ((R << (sh0 + 1)) & 0x80008000u) ^ base;
                             o.z = ((R << (sh0 + 2)) & 0x80008000u) ^ base;
                             o.w = ((R << (sh0 + 3)) & 0x80008000u) ^ base;
-                            *reinterpret_cast<uint4 *>(Bt + sw128(row, c)) = o;
+                            sts128(Bt + sw128(row, c), o);
                         }
                     }
                 }
