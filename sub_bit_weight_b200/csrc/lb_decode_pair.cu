@@ -295,11 +295,11 @@ __global__ void __launch_bounds__(kDecodeThreads)
         // ---- main stream
         for (int rgi = 0; rgi < nmine; ++rgi) {
             const int rg = warp + NW * rgi;
-            int a4[4][4];
+            int a4[4][4], a4o[4][4];   // even / odd k-blocks: eight independent MMA chains
 #pragma unroll
             for (int rb = 0; rb < 4; ++rb)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) a4[rb][c] = 0;
+                for (int c = 0; c < 4; ++c) a4[rb][c] = a4o[rb][c] = 0;
             for (int h = 0; h < hp; ++h) {
                 const int st = consumed % kP1Stages;
                 const uint32_t ph = (consumed / kP1Stages) & 1;
@@ -316,7 +316,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
 #pragma unroll
                         for (int rb = 0; rb < 4; ++rb) {
                             const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                            mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+                            if (u & 1) mma_u8s8(a4o[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+                            else mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
                         }
                     }
                 } else {
@@ -334,6 +335,10 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
                 fill_next();
             }
+#pragma unroll
+            for (int rb = 0; rb < 4; ++rb)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) a4[rb][c] += a4o[rb][c];
             // keep the columns of each row block's own path
 #pragma unroll
             for (int rb = 0; rb < 4; ++rb) {
@@ -460,11 +465,12 @@ __global__ void __launch_bounds__(kDecodeThreads)
             ++consumed;
             const uint32_t src = sm_addr(my_ring + (size_t)st * kStage) + lane * 8;
             const uint32_t bsrc = sm_addr(sB) + lane * 8;
-            int a4[4][4];
+            // two accumulator sets (even / odd k-blocks): eight independent MMA chains per warp
+            int a4[4][4], a4o[4][4];
 #pragma unroll
             for (int rb = 0; rb < 4; ++rb)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) a4[rb][c] = 0;
+                for (int c = 0; c < 4; ++c) a4[rb][c] = a4o[rb][c] = 0;
             int kb = 0;
             for (; kb + 4 <= KB2; kb += 4) {
 #pragma unroll
@@ -474,7 +480,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
 #pragma unroll
                     for (int rb = 0; rb < 4; ++rb) {
                         const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                        mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+                        if (u & 1) mma_u8s8(a4o[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+                        else mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
                     }
                 }
             }
@@ -487,6 +494,10 @@ __global__ void __launch_bounds__(kDecodeThreads)
                     mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
                 }
             }
+#pragma unroll
+            for (int rb = 0; rb < 4; ++rb)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) a4[rb][c] += a4o[rb][c];
             __syncwarp();
             if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
             fill_next();
