@@ -137,8 +137,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
         f_kb0 = fi.kc * kP1ChunkKB;
         f_nkb = min(kP1ChunkKB, f_KB1 - f_kb0);
         f_hp = (f_nkb + kHalf - 1) / kHalf;
-        f_nseq = max(0, (fd->RG1 - warp + NW - 1) / NW) * f_hp;
-        f_q = 0;
+        const int S = fd->RG1 * f_hp;   // stages of the item, split into equal contiguous ranges per warp
+        f_q = (int)((long long)S * warp / NW);
+        f_nseq = (int)((long long)S * (warp + 1) / NW);
         f_vt = fd->vt;
     };
     auto fill_next = [&]() {
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
             f_load();
         }
         if (f_it >= nitems) return;
-        const int rg = warp + NW * (f_q / f_hp), h = f_q % f_hp;
+        const int rg = f_q / f_hp, h = f_q % f_hp;
         const int n = min(kHalf, f_nkb - h * kHalf);
         if (lane == 0) {
             const int st = issued % kP1Stages;
@@ -173,7 +174,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
         const int k0 = kb0 * kKPerBlock;
         const int klen = nkb * kKPerBlock;
         const int hp = (nkb + kHalf - 1) / kHalf;
-        const int nmine = (RG1 - warp + NW - 1) / NW;
+        const int S = RG1 * hp;
+        const int qa = (int)((long long)S * warp / NW), qb = (int)((long long)S * (warp + 1) / NW);
 
         {
             uint4 *z4 = (uint4 *)sB;
@@ -292,63 +294,60 @@ __global__ void __launch_bounds__(kDecodeThreads)
         const int lane_E = (lane_m < M && lane_p < npaths) ? sE[lane_p * 16 + lane_m] : kNanExp;
         const double lane_sc = (lane_E == kNanExp) ? 0.0 : pow2d(-lane_E);
 
-        // ---- main stream
-        for (int rgi = 0; rgi < nmine; ++rgi) {
-            const int rg = warp + NW * rgi;
-            int a4[4][4], a4o[4][4];   // even / odd k-blocks: eight independent MMA chains
+        // ---- main stream: an equal contiguous range of the item's (row group, part) stages per warp
+        int a4[4][4];
+        for (int q = qa; q < qb; ++q) {
+            const int rg = q / hp, h = q - rg * hp;
+            if (q == qa || h == 0) {
 #pragma unroll
-            for (int rb = 0; rb < 4; ++rb)
+                for (int rb = 0; rb < 4; ++rb)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) a4[rb][c] = a4o[rb][c] = 0;
-            for (int h = 0; h < hp; ++h) {
-                const int st = consumed % kP1Stages;
-                const uint32_t ph = (consumed / kP1Stages) & 1;
-                if (!ring_wait(&bars[warp][st], ph, err)) return;
-                ++consumed;
-                const uint32_t src = sm_addr(my_ring + st * kStage) + lane * 8;
-                const uint32_t bsrc = sm_addr(sB + (size_t)(h * kHalf) * 32) + lane * 8;
-                const int n = min(kHalf, nkb - h * kHalf);
-                if (n == kHalf) {
+                    for (int c = 0; c < 4; ++c) a4[rb][c] = 0;
+            }
+            const int st = consumed % kP1Stages;
+            const uint32_t ph = (consumed / kP1Stages) & 1;
+            if (!ring_wait(&bars[warp][st], ph, err)) return;
+            ++consumed;
+            const uint32_t src = sm_addr(my_ring + st * kStage) + lane * 8;
+            const uint32_t bsrc = sm_addr(sB + (size_t)(h * kHalf) * 32) + lane * 8;
+            const int n = min(kHalf, nkb - h * kHalf);
+            if (n == kHalf) {
 #pragma unroll
-                    for (int u = 0; u < kHalf; ++u) {
-                        const uint2 w = lds64(src + u * 256);
-                        const uint2 b = lds64(bsrc + u * 256);
+                for (int u = 0; u < kHalf; ++u) {
+                    const uint2 w = lds64(src + u * 256);
+                    const uint2 b = lds64(bsrc + u * 256);
 #pragma unroll
-                        for (int rb = 0; rb < 4; ++rb) {
-                            const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                            if (u & 1) mma_u8s8(a4o[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
-                            else mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
-                        }
-                    }
-                } else {
-                    for (int u = 0; u < n; ++u) {
-                        const uint2 w = lds64(src + u * 256);
-                        const uint2 b = lds64(bsrc + u * 256);
-#pragma unroll
-                        for (int rb = 0; rb < 4; ++rb) {
-                            const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                            mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
-                        }
+                    for (int rb = 0; rb < 4; ++rb) {
+                        const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                        mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
                     }
                 }
-                __syncwarp();
-                if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-                fill_next();
+            } else {
+                for (int u = 0; u < n; ++u) {
+                    const uint2 w = lds64(src + u * 256);
+                    const uint2 b = lds64(bsrc + u * 256);
+#pragma unroll
+                    for (int rb = 0; rb < 4; ++rb) {
+                        const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                        mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+                    }
+                }
             }
+            __syncwarp();
+            if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+            fill_next();
+            if (h == hp - 1 || q == qb - 1) {
+                // keep the columns of each row block's own path; partial row groups add up exactly
 #pragma unroll
-            for (int rb = 0; rb < 4; ++rb)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) a4[rb][c] += a4o[rb][c];
-            // keep the columns of each row block's own path
-#pragma unroll
-            for (int rb = 0; rb < 4; ++rb) {
-                const int row0 = rg * kRowsPerGroup + rb * kRowsPerBlock;
-                const int prb = min(row0 / r16, npaths - 1);
-                if (prb != lane_p || lane_E == kNanExp) continue;
-                const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
-                const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
-                if (Tlo) atomicAdd(acc + (size_t)(row0 + g) * 16 + lane_m, (double)Tlo * lane_sc);
-                if (Thi) atomicAdd(acc + (size_t)(row0 + g + 8) * 16 + lane_m, (double)Thi * lane_sc);
+                for (int rb = 0; rb < 4; ++rb) {
+                    const int row0 = rg * kRowsPerGroup + rb * kRowsPerBlock;
+                    const int prb = min(row0 / r16, npaths - 1);
+                    if (prb != lane_p || lane_E == kNanExp) continue;
+                    const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
+                    const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
+                    if (Tlo) atomicAdd(acc + (size_t)(row0 + g) * 16 + lane_m, (double)Tlo * lane_sc);
+                    if (Thi) atomicAdd(acc + (size_t)(row0 + g + 8) * 16 + lane_m, (double)Thi * lane_sc);
+                }
             }
         }
 
@@ -375,27 +374,27 @@ __global__ void __launch_bounds__(kDecodeThreads)
 {
     constexpr int NW = kDecodeThreads / 32;
     constexpr int kRows = kP2ItemGroups * kRowsPerGroup;   // outputs per item
+    constexpr int kStage = kP2StageKB * 256;               // one ring stage: 8 k-blocks of one row group
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    const int kStage = kb2max * 256;
-    unsigned char *ring = smem_raw;                                         // [NW][kP2Stages][kStage]
-    uint2 *sB = (uint2 *)(smem_raw + (size_t)NW * kP2Stages * kStage);     // [KB2][32]
+    unsigned char *ring = smem_raw;                                         // [NW][kP2PairStages][kStage]
+    uint2 *sB = (uint2 *)(smem_raw + (size_t)NW * kP2PairStages * kStage);     // [KB2][32] (kb2max slots)
     float *sH = (float *)(sB + (size_t)kb2max * 32);                       // [2][kRows]
-    __shared__ uint64_t bars[NW][kP2Stages];
+    __shared__ uint64_t bars[NW][kP2PairStages];
     __shared__ float sScale[4], sQsc[4];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;
     const int lane_m = t4 >> 1, lane_p = t4 & 1;
     if (lane == 0)
-        for (int s = 0; s < kP2Stages; ++s) bar_init(&bars[warp][s]);
+        for (int s = 0; s < kP2PairStages; ++s) bar_init(&bars[warp][s]);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     __syncwarp();
     uint32_t issued = 0, consumed = 0;
-    unsigned char *my_ring = ring + (size_t)warp * kP2Stages * kStage;
+    unsigned char *my_ring = ring + (size_t)warp * kP2PairStages * kStage;
 
-    // Fill cursor over this warp's (item, row group) sequence, kP2Stages ahead
+    // Fill cursor over this warp's (item, row group) sequence, kP2PairStages ahead
     // of the consumer and across item boundaries.
-    int f_it = blockIdx.x, f_rg = 0, f_end = 0, f_kb2 = 0;
+    int f_it = blockIdx.x, f_rg = 0, f_end = 0, f_kb2 = 0, f_h = 0, f_hp = 1;
     const uint2 *f_ut = nullptr;
     auto f_load = [&]() {
         if (f_it >= nitems) return;
@@ -405,6 +404,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
         f_end = fi.rg1;
         f_ut = fd->ut;
         f_kb2 = fd->KB2;
+        f_hp = (f_kb2 + kP2StageKB - 1) / kP2StageKB;
+        f_h = 0;
     };
     auto fill_next = [&]() {
         while (f_it < nitems && f_rg >= f_end) {
@@ -412,16 +413,20 @@ __global__ void __launch_bounds__(kDecodeThreads)
             f_load();
         }
         if (f_it >= nitems) return;
+        const int n = min(kP2StageKB, f_kb2 - f_h * kP2StageKB);
         if (lane == 0) {
-            const int st = issued % kP2Stages;
-            ring_fill(my_ring + (size_t)st * kStage, f_ut + (size_t)f_rg * f_kb2 * 32, (unsigned)f_kb2 * 256u,
-                      &bars[warp][st]);
+            const int st = issued % kP2PairStages;
+            ring_fill(my_ring + (size_t)st * kStage, f_ut + ((size_t)f_rg * f_kb2 + f_h * kP2StageKB) * 32,
+                      (unsigned)n * 256u, &bars[warp][st]);
         }
         ++issued;
-        f_rg += NW;
+        if (++f_h == f_hp) {
+            f_h = 0;
+            f_rg += NW;
+        }
     };
     f_load();
-    for (int s = 0; s < kP2Stages; ++s) fill_next();
+    for (int s = 0; s < kP2PairStages; ++s) fill_next();
 
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
         const P2Item item = items[it];
@@ -458,49 +463,48 @@ __global__ void __launch_bounds__(kDecodeThreads)
         __syncthreads();
         const float my_sc = sScale[t4], my_q = sQsc[t4];
 
+        const int hp2 = (KB2 + kP2StageKB - 1) / kP2StageKB;
+        const uint32_t bsrc0 = sm_addr(sB) + lane * 8;
         for (int rg = item.rg0 + warp; rg < item.rg1; rg += NW) {
-            const int st = consumed % kP2Stages;
-            const uint32_t ph = (consumed / kP2Stages) & 1;
-            if (!ring_wait(&bars[warp][st], ph, err)) return;
-            ++consumed;
-            const uint32_t src = sm_addr(my_ring + (size_t)st * kStage) + lane * 8;
-            const uint32_t bsrc = sm_addr(sB) + lane * 8;
-            // two accumulator sets (even / odd k-blocks): eight independent MMA chains per warp
-            int a4[4][4], a4o[4][4];
+            int a4[4][4];
 #pragma unroll
             for (int rb = 0; rb < 4; ++rb)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) a4[rb][c] = a4o[rb][c] = 0;
-            int kb = 0;
-            for (; kb + 4 <= KB2; kb += 4) {
+                for (int c = 0; c < 4; ++c) a4[rb][c] = 0;
+            for (int h = 0; h < hp2; ++h) {
+                const int st = consumed % kP2PairStages;
+                const uint32_t ph = (consumed / kP2PairStages) & 1;
+                if (!ring_wait(&bars[warp][st], ph, err)) return;
+                ++consumed;
+                const uint32_t src = sm_addr(my_ring + (size_t)st * kStage) + lane * 8;
+                const uint32_t bsrc = bsrc0 + h * kP2StageKB * 256;
+                const int n = min(kP2StageKB, KB2 - h * kP2StageKB);
+                if (n == kP2StageKB) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const uint2 w = lds64(src + (kb + u) * 256);
-                    const uint2 b = lds64(bsrc + (kb + u) * 256);
+                    for (int u = 0; u < kP2StageKB; ++u) {
+                        const uint2 w = lds64(src + u * 256);
+                        const uint2 b = lds64(bsrc + u * 256);
 #pragma unroll
-                    for (int rb = 0; rb < 4; ++rb) {
-                        const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                        if (u & 1) mma_u8s8(a4o[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
-                        else mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+                        for (int rb = 0; rb < 4; ++rb) {
+                            const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                            mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+                        }
+                    }
+                } else {
+                    for (int u = 0; u < n; ++u) {
+                        const uint2 w = lds64(src + u * 256);
+                        const uint2 b = lds64(bsrc + u * 256);
+#pragma unroll
+                        for (int rb = 0; rb < 4; ++rb) {
+                            const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                            mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+                        }
                     }
                 }
+                __syncwarp();
+                if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                fill_next();
             }
-            for (; kb < KB2; ++kb) {
-                const uint2 w = lds64(src + kb * 256);
-                const uint2 b = lds64(bsrc + kb * 256);
-#pragma unroll
-                for (int rb = 0; rb < 4; ++rb) {
-                    const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                    mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
-                }
-            }
-#pragma unroll
-            for (int rb = 0; rb < 4; ++rb)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) a4[rb][c] += a4o[rb][c];
-            __syncwarp();
-            if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-            fill_next();
             // lane (m, path): its path's share of rows g and g + 8, then the pair sum
             const uint32_t hrow = sm_addr(sH + lane_p * kRows + (rg * kRowsPerGroup - n0) + g);
 #pragma unroll
@@ -538,7 +542,7 @@ lb_status decode_pair_launch(const LayerDev *dev_layers, const P1Item *p1, int n
     }
     const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * kP1StageKB * 256 +
                          (size_t)kP1ChunkKB * 32 * sizeof(uint2);
-    const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * kb2max * 256 + (size_t)kb2max * 32 * sizeof(uint2) +
+    const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2PairStages * kP2StageKB * 256 + (size_t)kb2max * 32 * sizeof(uint2) +
                          (size_t)2 * kP2ItemGroups * kRowsPerGroup * sizeof(float);
     if (smem2 > 227 * 1024) return LB_ERR_UNSUPPORTED;
     if ((int)smem1 > set1) {

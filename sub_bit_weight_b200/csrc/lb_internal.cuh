@@ -43,6 +43,8 @@ constexpr int kIoBatch = 1024;          // layers per launch (pointer tables rid
 constexpr int kP1StageKB = 8;           // k-blocks per ring stage, contraction 1 (2 KB)
 constexpr int kP1Stages = 3;            // per-warp bulk-copy ring depth, contraction 1
 constexpr int kP2Stages = 2;            // per-warp bulk-copy ring depth, contraction 2 (one row group per stage)
+constexpr int kP2StageKB = 8;           // path-merged contraction 2: k-blocks per ring stage (2 KB)
+constexpr int kP2PairStages = 3;        // path-merged contraction 2: per-warp ring depth
 
 // doubles in the accumulator block of a layer's scratch
 __host__ __device__ inline size_t acc_doubles(int R1) { return (size_t)R1 * 16 + 32 + 16; }
