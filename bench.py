@@ -53,6 +53,8 @@ def peaks():
 
 CSRC = os.path.join(ROOT, "sub_bit_weight_b200", "csrc")
 KERNEL_SOURCES = {
+    "quantize_pair_kernel": ["lb_decode_pair.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
+    "finish_pair_kernel": ["lb_decode_pair.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
     "contraction1_pair_kernel": ["lb_decode_pair.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
     "contraction2_pair_kernel": ["lb_decode_pair.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
     "contraction1_kernel": ["lb_decode.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
@@ -213,9 +215,10 @@ def run_gpu(w: synth.Workload, M: int, steps: int, warmup: int, dist, dev, want_
     for _ in range(warmup):
         lib.lb_stack_forward(S, io=io)
     torch.cuda.synchronize()
+    nl = lib.lb_last_launch_count()
 
     nlaunch_per_step = None
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)] for _ in range(steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for trio in ev:          # torch creates the CUDA event on first record
         for e in trio:
@@ -237,10 +240,8 @@ def run_gpu(w: synth.Workload, M: int, steps: int, warmup: int, dist, dev, want_
         dist.barrier()
     total_ms = start.elapsed_time(stop)
     per_launch = None
-    if nlaunch_per_step == 2:
-        k1 = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
-        k2 = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
-        per_launch = (k1, k2)
+    if nlaunch_per_step == nl and nl in (2, 4):
+        per_launch = tuple(sum(e[i].elapsed_time(e[i + 1]) for e in ev) / steps for i in range(nl))
 
     e2e = None
     if want_e2e:
@@ -334,9 +335,9 @@ def main():
 
     roof = None
     if res["per_launch"]:
-        k1ms, k2ms = res["per_launch"]
-        dom = 1 if k2ms >= k1ms else 0
         if prefill_main:
+            k1ms, k2ms = res["per_launch"][:2]
+            dom = 1 if k2ms >= k1ms else 0
             f1 = sum(2.0 * M * 2 * s.r * s.K for s in shapes)
             f2 = sum(2.0 * M * 2 * s.r * s.N for s in shapes)
             dom_w, dom_ms = (f2, k2ms) if dom else (f1, k1ms)
@@ -350,16 +351,25 @@ def main():
                     "per_kernel_ms": {"latent": round(k1ms, 4), "output": round(k2ms, 4)},
                     "per_kernel_flops": {"latent": f1, "output": f2}}
         else:
-            dom_bytes, dom_ms = (k2b, k2ms) if dom else (k1b, k1ms)
-            ach = dom_bytes / (dom_ms * 1e-3) / 1e9
             suffix = "_pair_kernel" if M <= 2 else "_kernel"
-            kname = ("contraction2" if dom else "contraction1") + suffix
+            names = ["contraction1" + suffix, "contraction2" + suffix]
+            kbytes = [k1b, k2b]
+            if len(res["per_launch"]) == 4:
+                # activation quantisation and the contraction-1 finish run as their own launches:
+                # x and g are the bytes of the first, the finish moves no algorithmic bytes
+                qb = sum(2.0 * M * s.K + 2 * 2.0 * s.K for s in shapes)
+                names = ["quantize" + suffix, names[0], "finish" + suffix, names[1]]
+                kbytes = [qb, k1b - qb, 0.0, k2b]
+            kms = list(res["per_launch"])
+            di = max(range(len(kms)), key=lambda i: kms[i])
+            dom_bytes, dom_ms, kname = kbytes[di], kms[di], names[di]
+            ach = dom_bytes / (dom_ms * 1e-3) / 1e9
             roof = {"bound": "hbm", "kernel": kname,
                     "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                     "frac": round(ach / pk["hbm_gbs"], 4), "peak_src": pk["src"],
                     "traffic": measured_traffic(kname, w.key), "algorithmic_bytes_per_launch": dom_bytes,
-                    "per_kernel_ms": {"contraction1_kernel": round(k1ms, 5), "contraction2_kernel": round(k2ms, 5)},
-                    "per_kernel_bytes": {"contraction1_kernel": k1b, "contraction2_kernel": k2b}}
+                    "per_kernel_ms": {n: round(t, 5) for n, t in zip(names, kms)},
+                    "per_kernel_bytes": {n: b for n, b in zip(names, kbytes)}}
     e2e = None
     if res["e2e"]:
         e_ms = max_over_ranks(res["e2e"]["ms"], dist)

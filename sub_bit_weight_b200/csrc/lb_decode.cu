@@ -600,11 +600,14 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
         }
         const int n1 = P.p1_start[b + 1] - P.p1_start[b];
         const int n2 = P.p2_start[b + 1] - P.p2_start[b];
-        if (M <= 2) {
-            lb_status st = decode_pair_launch(P.dev, P.p1 + P.p1_start[b], n1, P.p2 + P.p2_start[b], n2, io, base, M,
-                                              kb2max, P.err, s, launches, true);
-            if (st != LB_OK) return st;
-            continue;
+        if (M <= 2 && kb2max <= kPairMaxKB2) {
+            const int W = P.pair_warps[M - 1];
+            lb_status st = decode_pair_launch(P.dev, cnt, P.p1 + P.p1_start[b], n1, P.u1, P.wr1[M - 1] + (size_t)b * (W + 1),
+                                              P.u2, P.wr2[M - 1] + (size_t)b * (W + 1), W, io, base, M, kb2max, P.err,
+                                              s, launches, true);
+            if (st == LB_OK) continue;
+            if (st != LB_ERR_UNSUPPORTED) return st;
+            // shapes the streaming kernels cannot hold in shared memory take the general kernels
         }
         const int grid1 = std::max(1, std::min(n1, g_sms * occ1));
         const int grid2 = std::max(1, std::min(n2, g_sms * occ2));
@@ -618,17 +621,20 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
 }
 
 // One layer whose descriptor (and scratch) the caller placed in device
-// memory: the two decode kernels over the given work items.  Used by the
-// entry point that must not allocate.
-lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc, const P1Item *p1, int n1,
-                            const P2Item *p2, int n2, const uint16_t *x, float *y, int M, int *err, cudaStream_t s,
-                            int *launches)
+// memory: the decode kernels over the work items of the layer's own plan.
+// Used by the entry point that must not allocate.
+lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc, const Plan &P, const uint16_t *x,
+                            float *y, int M, int *err, cudaStream_t s, int *launches)
 {
-    if (M <= 2) {
+    const P1Item *p1 = P.p1;
+    const P2Item *p2 = P.p2;
+    const int n1 = P.n_p1, n2 = P.n_p2;
+    if (M <= 2 && host_desc.KB2 <= kPairMaxKB2) {
         static thread_local IoPtrs io1;
         io1.x[0] = x;
         io1.y[0] = y;
-        return decode_pair_launch(dev_desc, p1, n1, p2, n2, io1, 0, M, host_desc.KB2, err, s, launches, false);
+        return decode_pair_launch(dev_desc, 1, p1, n1, P.u1, P.wr1[M - 1], P.u2, P.wr2[M - 1], P.pair_warps[M - 1], io1, 0,
+                                  M, host_desc.KB2, err, s, launches, false);
     }
     const int NT = (M + 3) / 4;
     cudaError_t e = cudaSuccess;

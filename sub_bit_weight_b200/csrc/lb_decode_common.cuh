@@ -84,6 +84,13 @@ static __device__ __forceinline__ uint2 lds64(uint32_t addr)
     return v;
 }
 
+static __device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(addr));
+    return v;
+}
+
 static __device__ __forceinline__ float lds_f32(uint32_t addr)
 {
     float v;
@@ -109,6 +116,15 @@ static __device__ __forceinline__ void ring_fill(void *dst, const void *src, uns
     asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(sm_addr(bar)),
                  "r"(bytes)
                  : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                     sm_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(sm_addr(bar))
+                 : "memory");
+}
+
+// Bulk copy completing on `bar` (the caller has announced the bytes with expect_tx).
+static __device__ __forceinline__ void bulk_copy(void *dst, const void *src, unsigned bytes, uint64_t *bar)
+{
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
                      sm_addr(dst)),
                  "l"(src), "r"(bytes), "r"(sm_addr(bar))

@@ -8,571 +8,690 @@
 //
 //     column = 4 * m + 2 * path + digit        (m < 2, path < 2, digit < 2)
 //
-// so one MMA per (row block, k-block) serves both paths.  In contraction 1
-// (rows = latent indices of one path) the accumulator columns of the row
-// block's own path are kept; in contraction 2 (k = latent indices, the other
-// path's columns of a k-block are zero) lane pairs (path 0, path 1) hold the
-// two path results of one output and add them with one shuffle.  No
-// per-path loop, no operand selects, one fold per row group.
+// so one MMA per (row block, k-block) serves both paths.  For M = 1 only the
+// first 16 lanes of a B fragment carry data; those fragments are stored
+// compactly (16 * M lanes per k-block) and the other lanes read zeros.
+//
+// Four launches:
+//   quantize_pair_kernel      x (.) g_p as 16-bit fixed point per 1024-input
+//                             chunk -> contraction-1 B fragments + exponents
+//   contraction1_pair_kernel  z = sum_k b * t over V tiles, float64 atomics
+//   finish_pair_kernel        zl = z (.) l_p as 16-bit fixed point -> the
+//                             contraction-2 B fragments (one CTA per layer)
+//   contraction2_pair_kernel  y = sum_p h_p (.) (U_p zl_p) over U tiles
+// In both contractions every warp streams its own contiguous, equal share of
+// the weight bytes (a static partition made at plan build) through a private
+// ring of bulk copies; warps never synchronise with each other.
 
 #include "lb_decode_common.cuh"
 
 namespace lb {
 
-// Lane of column (m, path, digit) holding activation index kk of a k-block,
-// and which of its two fragment words.
+// Lane of column (m, path, digit) holding activation index kk of a k-block.
 static __device__ __forceinline__ int pair_lane(int m, int p, int d, int kk)
 {
     return ((4 * m + 2 * p + d) << 2) + ((kk & 15) >> 2);
 }
 
 // ---------------------------------------------------------------------------
-// Finish of contraction 1 (last item of a layer): zl fragments, merged layout
+// Activation quantisation (one CTA per 1024-input chunk of a layer)
 // ---------------------------------------------------------------------------
-static __device__ void finish_pair(const LayerDev *dp, int M, float *sMax, int *sBad, int *sE, int *sQs)
+template <int MM>
+__global__ void __launch_bounds__(kDecodeThreads)
+    quantize_pair_kernel(const LayerDev *__restrict__ layers, const P1Item *__restrict__ items,
+                         const __grid_constant__ IoPtrs io, int base, int M)
 {
+    constexpr int kLanes = 16 * MM;     // stored lanes per k-block
+    __shared__ float sMax[4];
+    __shared__ int sBad[4], sE[4], sQs[4];
+    const int tid = threadIdx.x, lane = tid & 31;
+    const P1Item item = items[blockIdx.x];
+    const LayerDev *dp = layers + item.layer;
+    const int K = dp->K, K32 = dp->K32, KB1 = dp->KB1, npaths = dp->npaths, R1 = dp->R1;
+    const __half *__restrict__ gsc = dp->g;
+    const uint16_t *__restrict__ x = io.x[item.layer - base];
+    const int kb0 = item.kc * kP1ChunkKB;
+    const int nkb = min(kP1ChunkKB, KB1 - kb0);
+    const int k0 = kb0 * kKPerBlock;
+    const int klen = nkb * kKPerBlock;
+    if (tid < 4) {
+        sMax[tid] = 0.0f;
+        sBad[tid] = 0;
+        sQs[tid] = 0;
+    }
+    __syncthreads();
+
+    // t = x (.) g_p for 8 consecutive inputs per thread
+    const int kk0 = 8 * tid;
+    const bool act = kk0 < klen;
+    const int kg = k0 + kk0;
+    float gv[2][8];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+        if (act && p < npaths) {
+            const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(gsc + (size_t)p * K32 + kg));
+            const __half *hv = reinterpret_cast<const __half *>(&raw);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) gv[p][e] = __half2float(hv[e]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) gv[p][e] = 0.0f;
+        }
+    }
+    float xv[MM][8];
+    const bool vec = ((K & 7) == 0) && (kg + 8 <= K);
+#pragma unroll
+    for (int m = 0; m < MM; ++m) {
+        if (!act || m >= M) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xv[m][e] = 0.0f;
+        } else if (vec) {
+            const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + kg));
+            const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                xv[m][2 * e] = __uint_as_float(w4[e] << 16);
+                xv[m][2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                xv[m][e] = (kg + e < K) ? bf16_bits_to_float(__ldg(x + (size_t)m * K + kg + e)) : 0.0f;
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < MM; ++m)
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            float amax = 0.0f;
+            int bad = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float tv = fabsf(xv[m][e] * gv[p][e]);
+                if (!(tv <= FLT_MAX)) bad = 1;
+                else amax = fmaxf(amax, tv);
+            }
+            amax = warp_max(amax);
+            bad = warp_or(bad);
+            if (lane == 0 && p < npaths && m < M) {
+                smem_max(&sMax[2 * p + m], amax);
+                if (bad) atomicOr(&sBad[2 * p + m], 1);
+            }
+        }
+    __syncthreads();
+    if (tid < 4) {
+        const int p = tid >> 1, m = tid & 1;
+        sE[tid] = (p < npaths && m < M) ? exponent_for(sMax[tid], sBad[tid] != 0) : kNanExp;
+    }
+    __syncthreads();
+    uint32_t *xw = reinterpret_cast<uint32_t *>(dp->xfrag + (size_t)kb0 * kLanes);
+#pragma unroll
+    for (int m = 0; m < MM; ++m)
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const bool live = m < M && p < npaths;
+            const int E = sE[2 * p + m];
+            const float sc = (!live || E == kNanExp) ? 0.0f : pow2f(E);
+            int qs = 0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t wlo = 0, whi = 0;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int q = quantize_s(xv[m][4 * h + e] * gv[p][4 * h + e], sc);
+                    int lo, hi;
+                    digits(q, lo, hi);
+                    wlo |= (uint32_t)(lo & 255) << (8 * e);
+                    whi |= (uint32_t)(hi & 255) << (8 * e);
+                    qs += q;
+                }
+                if (act) {
+                    // every word of the chunk's fragments is written (zeros for absent rows and paths)
+                    const int kk = kk0 + 4 * h;
+                    uint32_t *fb = xw + (size_t)(kk >> 5) * kLanes * 2;
+                    const int word = (kk & 31) >> 4;
+                    fb[2 * pair_lane(m, p, 0, kk & 31) + word] = wlo;
+                    fb[2 * pair_lane(m, p, 1, kk & 31) + word] = whi;
+                }
+            }
+            qs = warp_sum(qs);
+            if (lane == 0 && qs) atomicAdd(&sQs[2 * p + m], qs);
+        }
+    __syncthreads();
+    if (tid < 4) {
+        const int p = tid >> 1, m = tid & 1;
+        const int E = sE[tid];
+        dp->xmeta[item.kc * 4 + tid] = E;
+        if (p < npaths && m < M) {
+            double *acc = dp->acc;
+            if (E == kNanExp) atomicOr(reinterpret_cast<int *>(acc + (size_t)R1 * 16 + 32) + p * 16 + m, 1);
+            else if (sQs[tid]) atomicAdd(acc + (size_t)R1 * 16 + p * 16 + m, (double)sQs[tid] * pow2d(-E));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Finish of contraction 1 (one CTA per layer): zl = (S_p - 2 acc) * l_p as
+// 16-bit fixed point per (path, row), written as contraction-2 B fragments
+// (16 * M lanes per k-block) plus (exponent, digit sum) in zmeta; clears the
+// accumulators for the next call.
+// ---------------------------------------------------------------------------
+constexpr int kFinishThreads = 256;
+
+template <int MM>
+__global__ void __launch_bounds__(kFinishThreads)
+    finish_pair_kernel(const LayerDev *__restrict__ layers, int base, int M)
+{
+    __shared__ float sMax[4];
+    __shared__ int sBad[4], sE[4], sQs[4];
     const int tid = threadIdx.x;
+    const LayerDev *dp = layers + base + blockIdx.x;
     const int R1 = dp->R1, r = dp->r, r16 = dp->r16, r32 = dp->r32, npaths = dp->npaths, KB2 = dp->KB2;
     double *acc = dp->acc;
     const __half *lsc = dp->l;
     const double *S = acc + (size_t)R1 * 16;
     const int *badf = reinterpret_cast<const int *>(acc + (size_t)R1 * 16 + 32);
-    if (tid < 32) {
+    if (tid < 4) {
         sMax[tid] = 0.0f;
         sBad[tid] = 0;
         sQs[tid] = 0;
-    }
-    {
-        uint4 *z = reinterpret_cast<uint4 *>(dp->zfrag);
-        for (int i = tid; i < KB2 * 32 * (int)sizeof(uint2) / 16; i += kDecodeThreads) z[i] = make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
     auto zl_at = [&](int p, int j, int m) -> float {
         const double z = __ldcg(S + p * 16 + m) - 2.0 * __ldcg(acc + (size_t)(p * r16 + j) * 16 + m);
         return (float)z * __half2float(lsc[p * r16 + j]);
     };
-    for (int e = tid; e < npaths * r * M; e += kDecodeThreads) {
+    for (int e = tid; e < npaths * r * M; e += kFinishThreads) {
         const int m = e % M, pj = e / M;
         const int p = pj / r, j = pj - p * r;
         const float zl = zl_at(p, j, m);
-        if (!(fabsf(zl) <= FLT_MAX)) atomicOr(&sBad[p * 16 + m], 1);
-        else smem_max(&sMax[p * 16 + m], fabsf(zl));
+        if (!(fabsf(zl) <= FLT_MAX)) atomicOr(&sBad[2 * p + m], 1);
+        else smem_max(&sMax[2 * p + m], fabsf(zl));
     }
     __syncthreads();
-    if (tid < npaths * M) {
-        const int p = tid / M, m = tid - p * M;
-        sE[p * 16 + m] = exponent_for(sMax[p * 16 + m], sBad[p * 16 + m] != 0 || __ldcg(badf + p * 16 + m) != 0);
+    if (tid < 4) {
+        const int p = tid >> 1, m = tid & 1;
+        sE[tid] = (p < npaths && m < M) ? exponent_for(sMax[tid], sBad[tid] != 0 || __ldcg(badf + p * 16 + m) != 0)
+                                        : kNanExp;
     }
     __syncthreads();
-    const int ngrp = r32 / 4;
-    for (int e = tid; e < npaths * M * ngrp; e += kDecodeThreads) {
-        const int c = e % ngrp, pm = e / ngrp;
-        const int p = pm / M, m = pm - p * M;
-        const int E = sE[p * 16 + m];
-        const float sc = (E == kNanExp) ? 0.0f : pow2f(E);
-        uint32_t wlo = 0, whi = 0;
+    // fragment word pairs: lane L < 16 * MM of k-block kb holds column L / 4 = 4 m + 2 p + d
+    for (int idx = tid; idx < KB2 * 16 * MM; idx += kFinishThreads) {
+        const int kb = idx / (16 * MM), lane = idx - kb * 16 * MM;
+        const int col = lane >> 2, t = lane & 3;
+        const int fm = col >> 2, fp = (col >> 1) & 1, fd = col & 1;
+        uint32_t w[2] = {0u, 0u};
         int qs = 0;
+        if (fm < M && fp < npaths && kb * kKPerBlock / r32 == fp) {
+            const int E = sE[2 * fp + fm];
+            const float sc = (E == kNanExp) ? 0.0f : pow2f(E);
+            const int j0 = kb * kKPerBlock - fp * r32 + 4 * t;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int j = 4 * c + u;
-            const int q = (j < r) ? quantize_s(zl_at(p, j, m), sc) : 0;
-            int lo, hi;
-            digits(q, lo, hi);
-            wlo |= (uint32_t)(lo & 255) << (8 * u);
-            whi |= (uint32_t)(hi & 255) << (8 * u);
-            qs += q;
-        }
-        if (qs) atomicAdd(&sQs[p * 16 + m], qs);
-        const int jj = p * r32 + 4 * c;
-        uint2 *fb = dp->zfrag + (size_t)(jj >> 5) * 32;
-        const int word = (jj & 31) >> 4;
-        set_word(fb[pair_lane(m, p, 0, jj & 31)], word, wlo);
-        set_word(fb[pair_lane(m, p, 1, jj & 31)], word, whi);
-    }
-    __syncthreads();
-    if (tid < npaths * M) {
-        const int p = tid / M, m = tid - p * M;
-        dp->zmeta[p * 16 + m] = make_int2(sE[p * 16 + m], sQs[p * 16 + m]);
-    }
-    for (int i = tid; i < (int)acc_doubles(R1); i += kDecodeThreads) acc[i] = 0.0;
-}
-
-// ---------------------------------------------------------------------------
-// Contraction 1, M <= 2
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kDecodeThreads)
-    contraction1_pair_kernel(const LayerDev *__restrict__ layers, const P1Item *__restrict__ items, int nitems,
-                             const __grid_constant__ IoPtrs io, int base, int M, int *err)
-{
-    constexpr int NW = kDecodeThreads / 32;
-    constexpr int kHalf = kP1StageKB;
-    constexpr int kStage = kHalf * 256;
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    unsigned char *ring = smem_raw;                                      // [NW][kP1Stages][kStage]
-    uint2 *sB = (uint2 *)(smem_raw + NW * kP1Stages * kStage);          // [kP1ChunkKB][32]
-    __shared__ uint64_t bars[NW][kP1Stages];
-    __shared__ float sMax[32];
-    __shared__ int sBad[32], sE[32], sQs[32];
-    __shared__ int sLast;
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = lane >> 2, t4 = lane & 3;
-    const int lane_m = t4 >> 1, lane_p = t4 & 1;       // accumulator columns of this lane
-    if (lane == 0)
-        for (int s = 0; s < kP1Stages; ++s) bar_init(&bars[warp][s]);
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    __syncwarp();
-    uint32_t issued = 0, consumed = 0;
-    unsigned char *my_ring = ring + warp * kP1Stages * kStage;
-
-    // Fill cursor: this warp's stages (item, row group, part) in the order the
-    // warp consumes them; it runs kP1Stages ahead, across item boundaries.
-    int f_it = blockIdx.x, f_q = 0, f_nseq = 0, f_hp = 1, f_kb0 = 0, f_nkb = 0, f_KB1 = 0;
-    const uint2 *f_vt = nullptr;
-    auto f_load = [&]() {
-        if (f_it >= nitems) return;
-        const P1Item fi = items[f_it];
-        const LayerDev *fd = layers + fi.layer;
-        f_KB1 = fd->KB1;
-        f_kb0 = fi.kc * kP1ChunkKB;
-        f_nkb = min(kP1ChunkKB, f_KB1 - f_kb0);
-        f_hp = (f_nkb + kHalf - 1) / kHalf;
-        const int S = fd->RG1 * f_hp;   // stages of the item, split into equal contiguous ranges per warp
-        f_q = (int)((long long)S * warp / NW);
-        f_nseq = (int)((long long)S * (warp + 1) / NW);
-        f_vt = fd->vt;
-    };
-    auto fill_next = [&]() {
-        while (f_it < nitems && f_q >= f_nseq) {
-            f_it += gridDim.x;
-            f_load();
-        }
-        if (f_it >= nitems) return;
-        const int rg = f_q / f_hp, h = f_q % f_hp;
-        const int n = min(kHalf, f_nkb - h * kHalf);
-        if (lane == 0) {
-            const int st = issued % kP1Stages;
-            ring_fill(my_ring + st * kStage, f_vt + ((size_t)rg * f_KB1 + f_kb0 + h * kHalf) * 32, (unsigned)n * 256u,
-                      &bars[warp][st]);
-        }
-        ++issued;
-        ++f_q;
-    };
-    f_load();
-    for (int s = 0; s < kP1Stages; ++s) fill_next();
-
-    for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
-        const P1Item item = items[it];
-        const LayerDev *dp = layers + item.layer;
-        const int K = dp->K, K32 = dp->K32, KB1 = dp->KB1, RG1 = dp->RG1, r16 = dp->r16, npaths = dp->npaths;
-        const int R1 = dp->R1;
-        const __half *__restrict__ gsc = dp->g;
-        double *__restrict__ acc = dp->acc;
-        const uint16_t *__restrict__ x = io.x[item.layer - base];
-        const int kb0 = item.kc * kP1ChunkKB;
-        const int nkb = min(kP1ChunkKB, KB1 - kb0);
-        const int k0 = kb0 * kKPerBlock;
-        const int klen = nkb * kKPerBlock;
-        const int hp = (nkb + kHalf - 1) / kHalf;
-        const int S = RG1 * hp;
-        const int qa = (int)((long long)S * warp / NW), qb = (int)((long long)S * (warp + 1) / NW);
-
-        {
-            uint4 *z4 = (uint4 *)sB;
-            for (int i = tid; i < kP1ChunkKB * 32 * (int)sizeof(uint2) / 16; i += kDecodeThreads)
-                z4[i] = make_uint4(0, 0, 0, 0);
-        }
-        if (tid < 32) {
-            sMax[tid] = 0.0f;
-            sBad[tid] = 0;
-            sQs[tid] = 0;
-        }
-        __syncthreads();
-
-        // ---- t = x (.) g_p for 8 consecutive inputs per thread
-        const int kk0 = 8 * tid;
-        const bool act = kk0 < klen;
-        const int kg = k0 + kk0;
-        float gv[2][8];
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            if (act && p < npaths) {
-                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(gsc + (size_t)p * K32 + kg));
-                const __half *hv = reinterpret_cast<const __half *>(&raw);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) gv[p][e] = __half2float(hv[e]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) gv[p][e] = 0.0f;
-            }
-        }
-        float xv[2][8];
-        const bool vec = ((K & 7) == 0) && (kg + 8 <= K);
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-            if (!act || m >= M) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) xv[m][e] = 0.0f;
-            } else if (vec) {
-                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + kg));
-                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+            for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    xv[m][2 * e] = __uint_as_float(w4[e] << 16);
-                    xv[m][2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
+                    const int j = j0 + 16 * hh + e;
+                    const int q = (j < r) ? quantize_s(zl_at(fp, j, fm), sc) : 0;
+                    int lo, hi;
+                    digits(q, lo, hi);
+                    w[hh] |= (uint32_t)((fd ? hi : lo) & 255) << (8 * e);
+                    qs += q;
                 }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    xv[m][e] = (kg + e < K) ? bf16_bits_to_float(__ldg(x + (size_t)m * K + kg + e)) : 0.0f;
-            }
+            if (fd == 0 && qs) atomicAdd(&sQs[2 * fp + fm], qs);
         }
-#pragma unroll
-        for (int m = 0; m < 2; ++m)
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                float amax = 0.0f;
-                int bad = 0;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float tv = fabsf(xv[m][e] * gv[p][e]);
-                    if (!(tv <= FLT_MAX)) bad = 1;
-                    else amax = fmaxf(amax, tv);
-                }
-                amax = warp_max(amax);
-                bad = warp_or(bad);
-                if (lane == 0 && p < npaths && m < M) {
-                    smem_max(&sMax[p * 16 + m], amax);
-                    if (bad) atomicOr(&sBad[p * 16 + m], 1);
-                }
-            }
-        __syncthreads();
-        if (tid < npaths * M) {
-            const int p = tid / M, m = tid - p * M;
-            sE[p * 16 + m] = exponent_for(sMax[p * 16 + m], sBad[p * 16 + m] != 0);
-        }
-        __syncthreads();
-#pragma unroll
-        for (int m = 0; m < 2; ++m)
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                if (m >= M || p >= npaths) continue;
-                const int E = sE[p * 16 + m];
-                const float sc = (E == kNanExp) ? 0.0f : pow2f(E);
-                int qs = 0;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t wlo = 0, whi = 0;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int q = quantize_s(xv[m][4 * h + e] * gv[p][4 * h + e], sc);
-                        int lo, hi;
-                        digits(q, lo, hi);
-                        wlo |= (uint32_t)(lo & 255) << (8 * e);
-                        whi |= (uint32_t)(hi & 255) << (8 * e);
-                        qs += q;
-                    }
-                    if (act) {
-                        const int kk = kk0 + 4 * h;
-                        uint2 *fb = sB + (size_t)(kk >> 5) * 32;
-                        const int word = (kk & 31) >> 4;
-                        set_word(fb[pair_lane(m, p, 0, kk & 31)], word, wlo);
-                        set_word(fb[pair_lane(m, p, 1, kk & 31)], word, whi);
-                    }
-                }
-                qs = warp_sum(qs);
-                if (lane == 0 && qs) atomicAdd(&sQs[p * 16 + m], qs);
-            }
-        __syncthreads();
-        if (tid < npaths * M) {
-            const int p = tid / M, m = tid - p * M;
-            const int E = sE[p * 16 + m];
-            if (E == kNanExp) atomicOr(reinterpret_cast<int *>(acc + (size_t)R1 * 16 + 32) + p * 16 + m, 1);
-            else if (sQs[p * 16 + m]) atomicAdd(acc + (size_t)R1 * 16 + p * 16 + m, (double)sQs[p * 16 + m] * pow2d(-E));
-        }
-        // this lane's dequantisation scale for its (m, path) columns
-        const int lane_E = (lane_m < M && lane_p < npaths) ? sE[lane_p * 16 + lane_m] : kNanExp;
-        const double lane_sc = (lane_E == kNanExp) ? 0.0 : pow2d(-lane_E);
+        dp->zfrag[idx] = make_uint2(w[0], w[1]);
+    }
+    __syncthreads();
+    if (tid < 4) {
+        const int p = tid >> 1, m = tid & 1;
+        dp->zmeta[p * 16 + m] = make_int2(sE[tid], sQs[tid]);
+    }
+    // clear for the next call: rows' columns m < MM, the k sums and the flags
+    for (int i = tid; i < R1 * MM; i += kFinishThreads) acc[(size_t)(i / MM) * 16 + (i % MM)] = 0.0;
+    for (int i = tid; i < 48; i += kFinishThreads) acc[(size_t)R1 * 16 + i] = 0.0;
+}
 
-        // ---- main stream: an equal contiguous range of the item's (row group, part) stages per warp
-        int a4[4][4];
-        for (int q = qa; q < qb; ++q) {
-            const int rg = q / hp, h = q - rg * hp;
-            if (q == qa || h == 0) {
+// ---------------------------------------------------------------------------
+// Per-warp streaming: a ring of kPairStages bulk-copy stages (kPairStageKB
+// k-blocks each) and two B slots (fragments + their metadata), one mbarrier
+// each.  Unit records are read one unit ahead so no global load sits on the
+// path from one unit to the next.
+// ---------------------------------------------------------------------------
+
+template <int MM>
+static __device__ __forceinline__ void mma_stage(int (&a4)[4][4], uint32_t src, uint32_t bsrc, uint32_t bstride, int n)
+{
+    if (n == kPairStageKB) {
 #pragma unroll
-                for (int rb = 0; rb < 4; ++rb)
+        for (int v = 0; v < kPairStageKB; ++v) {
+            const uint2 w = lds64(src + v * 256);
+            const uint2 b = lds64(bsrc + v * bstride);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) a4[rb][c] = 0;
+            for (int rb = 0; rb < 4; ++rb) {
+                const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
             }
-            const int st = consumed % kP1Stages;
-            const uint32_t ph = (consumed / kP1Stages) & 1;
-            if (!ring_wait(&bars[warp][st], ph, err)) return;
-            ++consumed;
-            const uint32_t src = sm_addr(my_ring + st * kStage) + lane * 8;
-            const uint32_t bsrc = sm_addr(sB + (size_t)(h * kHalf) * 32) + lane * 8;
-            const int n = min(kHalf, nkb - h * kHalf);
-            if (n == kHalf) {
+        }
+    } else {
+        int v = 0;
+        for (; v + 4 <= n; v += 4) {
 #pragma unroll
-                for (int u = 0; u < kHalf; ++u) {
-                    const uint2 w = lds64(src + u * 256);
-                    const uint2 b = lds64(bsrc + u * 256);
-#pragma unroll
-                    for (int rb = 0; rb < 4; ++rb) {
-                        const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                        mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
-                    }
-                }
-            } else {
-                for (int u = 0; u < n; ++u) {
-                    const uint2 w = lds64(src + u * 256);
-                    const uint2 b = lds64(bsrc + u * 256);
-#pragma unroll
-                    for (int rb = 0; rb < 4; ++rb) {
-                        const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                        mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-            fill_next();
-            if (h == hp - 1 || q == qb - 1) {
-                // keep the columns of each row block's own path; partial row groups add up exactly
+            for (int vv = 0; vv < 4; ++vv) {
+                const uint2 w = lds64(src + (v + vv) * 256);
+                const uint2 b = lds64(bsrc + (v + vv) * bstride);
 #pragma unroll
                 for (int rb = 0; rb < 4; ++rb) {
-                    const int row0 = rg * kRowsPerGroup + rb * kRowsPerBlock;
-                    const int prb = min(row0 / r16, npaths - 1);
-                    if (prb != lane_p || lane_E == kNanExp) continue;
-                    const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
-                    const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
-                    if (Tlo) atomicAdd(acc + (size_t)(row0 + g) * 16 + lane_m, (double)Tlo * lane_sc);
-                    if (Thi) atomicAdd(acc + (size_t)(row0 + g + 8) * 16 + lane_m, (double)Thi * lane_sc);
+                    const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                    mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
                 }
             }
         }
-
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) sLast = (atomicAdd(dp->counter, 1u) == (unsigned)(dp->nkc - 1));
-        __syncthreads();
-        if (sLast) {
-            __threadfence();
-            finish_pair(dp, M, sMax, sBad, sE, sQs);
-            __syncthreads();
-            if (tid == 0) atomicExch(dp->counter, 0u);
+        for (; v < n; ++v) {
+            const uint2 w = lds64(src + v * 256);
+            const uint2 b = lds64(bsrc + v * bstride);
+#pragma unroll
+            for (int rb = 0; rb < 4; ++rb) {
+                const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+                mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+            }
         }
-        __syncthreads();
     }
 }
 
 // ---------------------------------------------------------------------------
-// Contraction 2 (+ h, + path sum), M <= 2
+// Contraction 1 (one warp per contiguous run of units)
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kDecodeThreads)
-    contraction2_pair_kernel(const LayerDev *__restrict__ layers, const P2Item *__restrict__ items, int nitems,
-                             const __grid_constant__ IoPtrs io, int base, int M, int kb2max, int *err)
+template <int MM>
+__global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
+    contraction1_pair_kernel(const LayerDev *__restrict__ layers, const PairUnit1 *__restrict__ units,
+                             const int *__restrict__ wrange, int M, int *err)
 {
-    constexpr int NW = kDecodeThreads / 32;
-    constexpr int kRows = kP2ItemGroups * kRowsPerGroup;   // outputs per item
-    constexpr int kStage = kP2StageKB * 256;               // one ring stage: 8 k-blocks of one row group
+    constexpr int kStage = kPairStageKB * 256;
+    constexpr int kBStride = 16 * MM * 8;                   // bytes of B fragments per k-block
+    constexpr int kBFrag = kP1ChunkKB * kBStride;
+    constexpr int kBSlot = kBFrag + 128;                    // fragments, then the chunk's exponents
+    constexpr int kWarpBytes = kPairStages * kStage + 2 * kBSlot;
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    unsigned char *ring = smem_raw;                                         // [NW][kP2PairStages][kStage]
-    uint2 *sB = (uint2 *)(smem_raw + (size_t)NW * kP2PairStages * kStage);     // [KB2][32] (kb2max slots)
-    float *sH = (float *)(sB + (size_t)kb2max * 32);                       // [2][kRows]
-    __shared__ uint64_t bars[NW][kP2PairStages];
-    __shared__ float sScale[4], sQsc[4];
+    constexpr int kPairWarps = pair_warps_per_cta(MM);
+    __shared__ uint64_t rbar[kPairWarps][kPairStages];
+    __shared__ uint64_t bbar[kPairWarps][2];
+    __shared__ __align__(16) uint2 zero8[2];
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int lane_m = t4 >> 1, lane_p = t4 & 1;       // accumulator columns of this lane
+    unsigned char *ring = smem_raw + warp * kWarpBytes;
+    unsigned char *bslot = ring + kPairStages * kStage;
+    if (threadIdx.x == 0) zero8[0] = zero8[1] = make_uint2(0u, 0u);
+    if (lane == 0) {
+        for (int s = 0; s < kPairStages; ++s) bar_init(&rbar[warp][s]);
+        bar_init(&bbar[warp][0]);
+        bar_init(&bbar[warp][1]);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    __syncthreads();    // the only CTA-wide barrier: zero8 and the barriers are ready
+
+    const int gw = warp * gridDim.x + blockIdx.x;     // an SM's warps take ranges spread over the whole batch
+    const int u0 = wrange[gw], u1 = wrange[gw + 1];
+    if (u0 >= u1) return;
+
+    // ---- fill cursor: stages of units [f_u, u1) in consumption order, at most
+    // kPairStages ahead; B fragments of at most two chunks resident at a time.
+    int f_u = u0, f_h = 0, f_cs = -1, f_layer = -1, f_kc = -1, issued = 0, consumed = 0, c_cs = -1;
+    const uint2 *f_xfrag = nullptr;
+    const int *f_xmeta = nullptr;
+    PairUnit1 f_cur = units[u0], f_nxt = f_cur;
+    if (u0 + 1 < u1) f_nxt = units[u0 + 1];
+    auto fill = [&]() {
+        while (f_u < u1 && issued - consumed < kPairStages) {
+            if (f_h == 0 && (f_cur.layer != f_layer || f_cur.kc != f_kc)) {
+                if (f_cs >= c_cs + 1) return;           // both B slots still in use
+                if (f_cur.layer != f_layer) {
+                    f_layer = f_cur.layer;
+                    f_xfrag = layers[f_layer].xfrag;
+                    f_xmeta = layers[f_layer].xmeta;
+                }
+                f_kc = f_cur.kc;
+                ++f_cs;
+                if (lane == 0) {
+                    unsigned char *dst = bslot + (f_cs & 1) * kBSlot;
+                    uint64_t *bar = &bbar[warp][f_cs & 1];
+                    const unsigned fb = (unsigned)f_cur.nkb * kBStride;
+                    asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(
+                                     sm_addr(bar)),
+                                 "r"(fb + 16u)
+                                 : "memory");
+                    bulk_copy(dst, f_xfrag + (size_t)f_kc * kP1ChunkKB * 16 * MM, fb, bar);
+                    bulk_copy(dst + kBFrag, f_xmeta + f_kc * 4, 16u, bar);
+                }
+            }
+            const int n = min(kPairStageKB, f_cur.nkb - f_h * kPairStageKB);
+            if (lane == 0) {
+                const int st = issued % kPairStages;
+                ring_fill(ring + st * kStage, f_cur.a + (size_t)f_h * kPairStageKB * 32, (unsigned)n * 256u,
+                          &rbar[warp][st]);
+            }
+            ++issued;
+            if (++f_h * kPairStageKB >= f_cur.nkb) {
+                f_h = 0;
+                ++f_u;
+                f_cur = f_nxt;
+                if (f_u + 1 < u1) f_nxt = units[f_u + 1];
+            }
+        }
+    };
+    fill();
+
+    // ---- consumer
+    int c_layer = -1, c_kc = -1, c_r16 = 1, c_npaths = 1;
+    double *c_acc = nullptr;
+    double lane_sc = 0.0;
+    bool lane_live = false;
+    uint32_t bbase = 0, bstride = 0;
+    const uint32_t zaddr = sm_addr(zero8);
+
+    PairUnit1 c_nxt = units[u0];
+    for (int u = u0; u < u1; ++u) {
+        const PairUnit1 cu = c_nxt;
+        if (u + 1 < u1) c_nxt = units[u + 1];
+        if (cu.layer != c_layer) {
+            const LayerDev *dp = layers + cu.layer;
+            c_layer = cu.layer;
+            c_acc = dp->acc;
+            c_r16 = dp->r16;
+            c_npaths = dp->npaths;
+            c_kc = -1;
+        }
+        if (cu.kc != c_kc) {
+            c_kc = cu.kc;
+            ++c_cs;
+            fill();                                        // the next chunk's B may start now
+            if (!ring_wait(&bbar[warp][c_cs & 1], (c_cs >> 1) & 1, err)) return;
+            const unsigned char *slot = bslot + (c_cs & 1) * kBSlot;
+            const int E = (lane_m < M && lane_p < c_npaths)
+                              ? (int)lds_u32(sm_addr(slot + kBFrag + 4 * (2 * lane_p + lane_m)))
+                              : kNanExp;
+            lane_live = E != kNanExp;
+            lane_sc = lane_live ? pow2d(-E) : 0.0;
+            const bool real = lane < 16 * MM;
+            bbase = real ? sm_addr(slot) + lane * 8 : zaddr;
+            bstride = real ? (uint32_t)kBStride : 0u;
+        }
+
+        int a4[4][4];
+#pragma unroll
+        for (int rb = 0; rb < 4; ++rb)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) a4[rb][c] = 0;
+        for (int h = 0; h * kPairStageKB < cu.nkb; ++h) {
+            const int st = consumed % kPairStages;
+            if (!ring_wait(&rbar[warp][st], (consumed / kPairStages) & 1, err)) return;
+            mma_stage<MM>(a4, sm_addr(ring + st * kStage) + lane * 8, bbase + (uint32_t)(h * kPairStageKB) * bstride,
+                          bstride, min(kPairStageKB, cu.nkb - h * kPairStageKB));
+            __syncwarp();
+            if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+            ++consumed;
+            fill();
+        }
+        // keep the columns of each row block's own path; partial sums over chunks add up exactly
+#pragma unroll
+        for (int rb = 0; rb < 4; ++rb) {
+            const int row0 = cu.rg * kRowsPerGroup + rb * kRowsPerBlock;
+            const int prb = min(row0 / c_r16, c_npaths - 1);
+            if (prb != lane_p || !lane_live) continue;
+            const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
+            const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
+            if (Tlo) atomicAdd(c_acc + (size_t)(row0 + g) * 16 + lane_m, (double)Tlo * lane_sc);
+            if (Thi) atomicAdd(c_acc + (size_t)(row0 + g + 8) * 16 + lane_m, (double)Thi * lane_sc);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Contraction 2 (+ h, + path sum): one warp per contiguous run of row groups.
+// A layer's U tiles are contiguous over its row groups, so a ring stage takes
+// up to kPairStageKB consecutive k-blocks across row-group boundaries (never
+// across layers); the consumer folds a row group when its KB2 k-blocks are in.
+// ---------------------------------------------------------------------------
+template <int MM>
+__global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
+    contraction2_pair_kernel(const LayerDev *__restrict__ layers, const PairUnit2 *__restrict__ units,
+                             const int *__restrict__ wrange, const __grid_constant__ IoPtrs io, int base, int M,
+                             int kb2max, int *err)
+{
+    constexpr int kStage = kPairStageKB * 256;
+    constexpr int kBStride = 16 * MM * 8;
+    constexpr int kPairWarps = pair_warps_per_cta(MM);
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ uint64_t rbar[kPairWarps][kPairStages];
+    __shared__ uint64_t bbar[kPairWarps][2];
+    __shared__ int snb[kPairWarps][kPairStages];       // k-blocks in each ring stage
+    __shared__ __align__(16) uint2 zero8[2];
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t4 = lane & 3;
     const int lane_m = t4 >> 1, lane_p = t4 & 1;
-    if (lane == 0)
-        for (int s = 0; s < kP2PairStages; ++s) bar_init(&bars[warp][s]);
+    const int kBFrag = kb2max * kBStride, kBSlot = kBFrag + kPairMeta2;
+    unsigned char *ring = smem_raw + (size_t)warp * (kPairStages * kStage + 2 * kBSlot);
+    unsigned char *bslot = ring + kPairStages * kStage;
+    if (threadIdx.x == 0) zero8[0] = zero8[1] = make_uint2(0u, 0u);
+    if (lane == 0) {
+        for (int s = 0; s < kPairStages; ++s) bar_init(&rbar[warp][s]);
+        bar_init(&bbar[warp][0]);
+        bar_init(&bbar[warp][1]);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    __syncwarp();
-    uint32_t issued = 0, consumed = 0;
-    unsigned char *my_ring = ring + (size_t)warp * kP2PairStages * kStage;
+    __syncthreads();
 
-    // Fill cursor over this warp's (item, row group) sequence, kP2PairStages ahead
-    // of the consumer and across item boundaries.
-    int f_it = blockIdx.x, f_rg = 0, f_end = 0, f_kb2 = 0, f_h = 0, f_hp = 1;
-    const uint2 *f_ut = nullptr;
-    auto f_load = [&]() {
-        if (f_it >= nitems) return;
-        const P2Item fi = items[f_it];
-        const LayerDev *fd = layers + fi.layer;
-        f_rg = fi.rg0 + warp;
-        f_end = fi.rg1;
-        f_ut = fd->ut;
-        f_kb2 = fd->KB2;
-        f_hp = (f_kb2 + kP2StageKB - 1) / kP2StageKB;
-        f_h = 0;
-    };
-    auto fill_next = [&]() {
-        while (f_it < nitems && f_rg >= f_end) {
-            f_it += gridDim.x;
-            f_load();
-        }
-        if (f_it >= nitems) return;
-        const int n = min(kP2StageKB, f_kb2 - f_h * kP2StageKB);
-        if (lane == 0) {
-            const int st = issued % kP2PairStages;
-            ring_fill(my_ring + (size_t)st * kStage, f_ut + ((size_t)f_rg * f_kb2 + f_h * kP2StageKB) * 32,
-                      (unsigned)n * 256u, &bars[warp][st]);
-        }
-        ++issued;
-        if (++f_h == f_hp) {
-            f_h = 0;
-            f_rg += NW;
-        }
-    };
-    f_load();
-    for (int s = 0; s < kP2PairStages; ++s) fill_next();
+    const int gw = warp * gridDim.x + blockIdx.x;     // an SM's warps take ranges spread over the whole batch
+    const int u0 = wrange[gw], u1 = wrange[gw + 1];
+    if (u0 >= u1) return;
 
-    for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
-        const P2Item item = items[it];
-        const LayerDev *dp = layers + item.layer;
-        const int N = dp->N, N64 = dp->N64, KB2 = dp->KB2, npaths = dp->npaths;
-        const __half *__restrict__ hsc = dp->h;
-        float *__restrict__ y = io.y[item.layer - base];
-
-        {
-            const uint4 *src = reinterpret_cast<const uint4 *>(dp->zfrag);
-            uint4 *dst = reinterpret_cast<uint4 *>(sB);
-            for (int i = tid; i < KB2 * 32 * (int)sizeof(uint2) / 16; i += kDecodeThreads) dst[i] = __ldcg(src + i);
-        }
-        const int n0 = item.rg0 * kRowsPerGroup;
-        for (int i = tid; i < 2 * kRows; i += kDecodeThreads) {
-            const int p = i / kRows, n = n0 + (i - p * kRows);
-            sH[i] = (p < npaths && n < N64) ? __half2float(hsc[p * N64 + n]) : 0.0f;
-        }
-        if (tid < 4) {
-            const int m = tid >> 1, p = tid & 1;
-            float sc = 0.0f, qsc = 0.0f;
-            if (m < M && p < npaths) {
-                const int2 mt = __ldcg(&dp->zmeta[p * 16 + m]);
-                if (mt.x == kNanExp) {
-                    sc = qsc = __int_as_float(0x7fc00000);
-                } else {
-                    sc = -2.0f * pow2f(-mt.x);                  // s = Q 2^-E - 2 T 2^-E
-                    qsc = (float)mt.y * pow2f(-mt.x);
+    // ---- fill cursor (position: unit f_u, k-block f_kb within it)
+    int f_u = u0, f_kb = 0, f_layer = -1, f_cs = -1, issued = 0, consumed = 0, c_cs = -1;
+    PairUnit2 f_cur = units[u0], f_nxt = f_cur;
+    if (u0 + 1 < u1) f_nxt = units[u0 + 1];
+    auto fill = [&]() {
+        while (f_u < u1 && issued - consumed < kPairStages) {
+            if (f_cur.layer != f_layer) {
+                if (f_cs >= c_cs + 1) return;           // both B slots still in use
+                ++f_cs;
+                f_layer = f_cur.layer;
+                if (lane == 0) {
+                    const LayerDev *fd = layers + f_layer;
+                    unsigned char *dst = bslot + (f_cs & 1) * kBSlot;
+                    uint64_t *bar = &bbar[warp][f_cs & 1];
+                    const unsigned fb = (unsigned)f_cur.kb2 * kBStride;
+                    asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(
+                                     sm_addr(bar)),
+                                 "r"(fb + (unsigned)kPairMeta2)
+                                 : "memory");
+                    bulk_copy(dst, fd->zfrag, fb, bar);
+                    bulk_copy(dst + kBFrag, fd->zmeta, (unsigned)kPairMeta2, bar);
                 }
             }
-            sScale[tid] = sc;
-            sQsc[tid] = qsc;
+            const uint2 *src = f_cur.a + (size_t)f_kb * 32;
+            int n = 0;
+            while (true) {
+                const int t = min(kPairStageKB - n, f_cur.kb2 - f_kb);
+                n += t;
+                f_kb += t;
+                if (f_kb < f_cur.kb2) break;            // the stage is full inside this row group
+                f_kb = 0;
+                ++f_u;
+                f_cur = f_nxt;
+                if (f_u + 1 < u1) f_nxt = units[f_u + 1];
+                if (n == kPairStageKB || f_u >= u1 || f_cur.layer != f_layer) break;
+            }
+            const int st = issued % kPairStages;
+            snb[warp][st] = n;
+            if (lane == 0) ring_fill(ring + st * kStage, src, (unsigned)n * 256u, &rbar[warp][st]);
+            ++issued;
         }
-        __syncthreads();
-        const float my_sc = sScale[t4], my_q = sQsc[t4];
+    };
+    fill();
 
-        const int hp2 = (KB2 + kP2StageKB - 1) / kP2StageKB;
-        const uint32_t bsrc0 = sm_addr(sB) + lane * 8;
-        for (int rg = item.rg0 + warp; rg < item.rg1; rg += NW) {
-            int a4[4][4];
+    int c_layer = -1, N = 0, npaths = 1;
+    float *y = nullptr;
+    float my_sc = 0.0f, my_q = 0.0f;
+    uint32_t bbase = 0, bstride = 0;
+    const uint32_t zaddr = sm_addr(zero8);
+    int s_left = 0;             // k-blocks of the current stage not yet used
+    uint32_t s_addr = 0;        // this lane's word pair of the stage's next k-block
+
+    // h of this lane's path for rows g and g + 8 of each row block of a unit,
+    // read one unit ahead
+    int h_layer = -1;
+    const __half *h_base = nullptr;      // this lane's path row of h in layer h_layer, or null
+    auto load_h = [&](const PairUnit2 &un, __half (&hq)[8]) {
+        if (un.layer != h_layer) {
+            const LayerDev *dp = layers + un.layer;
+            h_layer = un.layer;
+            h_base = (lane_p < dp->npaths) ? dp->h + (size_t)lane_p * dp->N64 : nullptr;
+        }
+        const __half *hp = h_base + un.rg * kRowsPerGroup + g;
 #pragma unroll
-            for (int rb = 0; rb < 4; ++rb)
+        for (int i = 0; i < 8; ++i) hq[i] = h_base ? hp[(i >> 1) * kRowsPerBlock + 8 * (i & 1)] : __half(0.0f);
+    };
+    PairUnit2 c_nxt = units[u0];
+    __half h_nxt[8];
+    load_h(c_nxt, h_nxt);
+    for (int u = u0; u < u1; ++u) {
+        const PairUnit2 cu = c_nxt;
+        float hv[4][2];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) a4[rb][c] = 0;
-            for (int h = 0; h < hp2; ++h) {
-                const int st = consumed % kP2PairStages;
-                const uint32_t ph = (consumed / kP2PairStages) & 1;
-                if (!ring_wait(&bars[warp][st], ph, err)) return;
-                ++consumed;
-                const uint32_t src = sm_addr(my_ring + (size_t)st * kStage) + lane * 8;
-                const uint32_t bsrc = bsrc0 + h * kP2StageKB * 256;
-                const int n = min(kP2StageKB, KB2 - h * kP2StageKB);
-                if (n == kP2StageKB) {
-#pragma unroll
-                    for (int u = 0; u < kP2StageKB; ++u) {
-                        const uint2 w = lds64(src + u * 256);
-                        const uint2 b = lds64(bsrc + u * 256);
-#pragma unroll
-                        for (int rb = 0; rb < 4; ++rb) {
-                            const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                            mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
-                        }
-                    }
+        for (int i = 0; i < 8; ++i) hv[i >> 1][i & 1] = __half2float(h_nxt[i]);
+        if (u + 1 < u1) {
+            c_nxt = units[u + 1];
+            load_h(c_nxt, h_nxt);
+        }
+        if (cu.layer != c_layer) {
+            const LayerDev *dp = layers + cu.layer;
+            c_layer = cu.layer;
+            N = dp->N;
+            npaths = dp->npaths;
+            y = io.y[cu.layer - base];
+            ++c_cs;
+            fill();
+            if (!ring_wait(&bbar[warp][c_cs & 1], (c_cs >> 1) & 1, err)) return;
+            const unsigned char *slot = bslot + (c_cs & 1) * kBSlot;
+            my_sc = my_q = 0.0f;
+            if (lane_m < M && lane_p < npaths) {
+                const uint32_t ma = sm_addr(slot + kBFrag + 8 * (lane_p * 16 + lane_m));
+                const int ex = (int)lds_u32(ma), qsum = (int)lds_u32(ma + 4);
+                if (ex == kNanExp) {
+                    my_sc = my_q = __int_as_float(0x7fc00000);
                 } else {
-                    for (int u = 0; u < n; ++u) {
-                        const uint2 w = lds64(src + u * 256);
-                        const uint2 b = lds64(bsrc + u * 256);
-#pragma unroll
-                        for (int rb = 0; rb < 4; ++rb) {
-                            const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                            mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
-                        }
-                    }
+                    my_sc = -2.0f * pow2f(-ex);                  // s = Q 2^-E - 2 T 2^-E
+                    my_q = (float)qsum * pow2f(-ex);
                 }
+            }
+            const bool real = lane < 16 * MM;
+            bbase = real ? sm_addr(slot) + lane * 8 : zaddr;
+            bstride = real ? (uint32_t)kBStride : 0u;
+        }
+        const int n0 = cu.rg * kRowsPerGroup + g;
+
+        int a4[4][4];
+#pragma unroll
+        for (int rb = 0; rb < 4; ++rb)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) a4[rb][c] = 0;
+        for (int kb = 0; kb < cu.kb2;) {
+            if (s_left == 0) {
+                const int st = consumed % kPairStages;
+                if (!ring_wait(&rbar[warp][st], (consumed / kPairStages) & 1, err)) return;
+                s_left = snb[warp][st];
+                s_addr = sm_addr(ring + st * kStage) + lane * 8;
+            }
+            const int seg = min(s_left, cu.kb2 - kb);
+            mma_stage<MM>(a4, s_addr, bbase + (uint32_t)kb * bstride, bstride, seg);
+            kb += seg;
+            s_left -= seg;
+            s_addr += (uint32_t)seg * 256u;
+            if (s_left == 0) {
                 __syncwarp();
                 if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-                fill_next();
-            }
-            // lane (m, path): its path's share of rows g and g + 8, then the pair sum
-            const uint32_t hrow = sm_addr(sH + lane_p * kRows + (rg * kRowsPerGroup - n0) + g);
-#pragma unroll
-            for (int rb = 0; rb < 4; ++rb) {
-                const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
-                const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
-                float vlo = lds_f32(hrow + 4 * rb * kRowsPerBlock) * fmaf((float)Tlo, my_sc, my_q);
-                float vhi = lds_f32(hrow + 4 * (rb * kRowsPerBlock + 8)) * fmaf((float)Thi, my_sc, my_q);
-                vlo += __shfl_xor_sync(0xffffffffu, vlo, 1);
-                vhi += __shfl_xor_sync(0xffffffffu, vhi, 1);
-                const int nlo = rg * kRowsPerGroup + rb * kRowsPerBlock + g;
-                if (lane_p == 0 && lane_m < M) {
-                    if (nlo < N) y[(size_t)lane_m * N + nlo] = vlo;
-                    if (nlo + 8 < N) y[(size_t)lane_m * N + nlo + 8] = vhi;
-                }
+                ++consumed;
+                fill();
             }
         }
-        __syncthreads();
+
+        // lane (m, path): its path's share of rows g and g + 8, then the pair sum
+#pragma unroll
+        for (int rb = 0; rb < 4; ++rb) {
+            const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
+            const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
+            float vlo = hv[rb][0] * fmaf((float)Tlo, my_sc, my_q);
+            float vhi = hv[rb][1] * fmaf((float)Thi, my_sc, my_q);
+            vlo += __shfl_xor_sync(0xffffffffu, vlo, 1);
+            vhi += __shfl_xor_sync(0xffffffffu, vhi, 1);
+            const int nlo = n0 + rb * kRowsPerBlock;
+            if (lane_p == 0 && lane_m < M) {
+                if (nlo < N) y[(size_t)lane_m * N + nlo] = vlo;
+                if (nlo + 8 < N) y[(size_t)lane_m * N + nlo + 8] = vhi;
+            }
+        }
     }
 }
 
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-lb_status decode_pair_launch(const LayerDev *dev_layers, const P1Item *p1, int n1, const P2Item *p2, int n2,
-                             const IoPtrs &io, int base, int M, int kb2max, int *err, cudaStream_t s, int *launches,
-                             bool mark)
+static int g_pair_smem[2][2];     // dynamic shared memory attribute set so far, per kernel and MM
+
+template <int MM>
+static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1,
+                                const PairUnit1 *u1, const int *wr1, const PairUnit2 *u2, const int *wr2,
+                                int pair_warps, const IoPtrs &io, int base, int M, int kb2max, int *err, cudaStream_t s,
+                                int *launches, bool mark)
 {
-    static int sms = 0, set1 = 0, set2 = 0;
     cudaError_t e;
-    if (!sms) {
-        int dev = 0;
-        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return status_from(e);
-        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return status_from(e);
-    }
-    const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * kP1StageKB * 256 +
-                         (size_t)kP1ChunkKB * 32 * sizeof(uint2);
-    const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2PairStages * kP2StageKB * 256 + (size_t)kb2max * 32 * sizeof(uint2) +
-                         (size_t)2 * kP2ItemGroups * kRowsPerGroup * sizeof(float);
-    if (smem2 > 227 * 1024) return LB_ERR_UNSUPPORTED;
-    if ((int)smem1 > set1) {
-        if ((e = cudaFuncSetAttribute(contraction1_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) !=
-            cudaSuccess)
+    constexpr int kPairWarps = pair_warps_per_cta(MM);
+    const size_t smem1 =
+        (size_t)kPairWarps * (kPairStages * kPairStageKB * 256 + 2 * (kP1ChunkKB * 16 * MM * 8 + 128));
+    const size_t smem2 =
+        (size_t)kPairWarps * (kPairStages * kPairStageKB * 256 + 2 * ((size_t)kb2max * 16 * MM * 8 + kPairMeta2));
+    if (smem1 > 227 * 1024 || smem2 > 227 * 1024 || kb2max > kPairMaxKB2) return LB_ERR_UNSUPPORTED;
+    if ((int)smem1 > g_pair_smem[0][MM - 1]) {
+        if ((e = cudaFuncSetAttribute(contraction1_pair_kernel<MM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem1)) != cudaSuccess)
             return status_from(e);
-        set1 = (int)smem1;
+        g_pair_smem[0][MM - 1] = (int)smem1;
     }
-    if ((int)smem2 > set2) {
-        if ((e = cudaFuncSetAttribute(contraction2_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)) !=
-            cudaSuccess)
+    if ((int)smem2 > g_pair_smem[1][MM - 1]) {
+        if ((e = cudaFuncSetAttribute(contraction2_pair_kernel<MM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem2)) != cudaSuccess)
             return status_from(e);
-        set2 = (int)smem2;
+        g_pair_smem[1][MM - 1] = (int)smem2;
     }
-    int occ1 = 0, occ2 = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, contraction1_pair_kernel, kDecodeThreads, smem1)) !=
-        cudaSuccess)
-        return status_from(e);
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ2, contraction2_pair_kernel, kDecodeThreads, smem2)) !=
-        cudaSuccess)
-        return status_from(e);
-    const int grid1 = std::max(1, std::min(n1, sms * std::max(1, occ1)));
-    const int grid2 = std::max(1, std::min(n2, sms * std::max(1, occ2)));
-    contraction1_pair_kernel<<<grid1, kDecodeThreads, smem1, s>>>(dev_layers, p1, n1, io, base, M, err);
+    const int grid = pair_warps / kPairWarps;
+    if (n1 > 0) {
+        quantize_pair_kernel<MM><<<n1, kDecodeThreads, 0, s>>>(dev_layers, p1, io, base, M);
+        ++*launches;
+        if (mark) profile_mark(*launches, s);
+    }
+    contraction1_pair_kernel<MM><<<grid, kPairWarps * 32, smem1, s>>>(dev_layers, u1, wr1, M, err);
     ++*launches;
     if (mark) profile_mark(*launches, s);
-    contraction2_pair_kernel<<<grid2, kDecodeThreads, smem2, s>>>(dev_layers, p2, n2, io, base, M, kb2max, err);
+    finish_pair_kernel<MM><<<nlayers, kFinishThreads, 0, s>>>(dev_layers, base, M);
+    ++*launches;
+    if (mark) profile_mark(*launches, s);
+    contraction2_pair_kernel<MM><<<grid, kPairWarps * 32, smem2, s>>>(dev_layers, u2, wr2, io, base, M, kb2max, err);
     ++*launches;
     if (mark) profile_mark(*launches, s);
     return status_from(cudaGetLastError());
+}
+
+lb_status decode_pair_launch(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1, const PairUnit1 *u1,
+                             const int *wr1, const PairUnit2 *u2, const int *wr2, int pair_warps, const IoPtrs &io,
+                             int base, int M, int kb2max, int *err, cudaStream_t s, int *launches, bool mark)
+{
+    if (M == 1)
+        return pair_launch_mm<1>(dev_layers, nlayers, p1, n1, u1, wr1, u2, wr2, pair_warps, io, base, M, kb2max, err, s,
+                                 launches, mark);
+    return pair_launch_mm<2>(dev_layers, nlayers, p1, n1, u1, wr1, u2, wr2, pair_warps, io, base, M, kb2max, err, s,
+                             launches, mark);
 }
 
 }  // namespace lb

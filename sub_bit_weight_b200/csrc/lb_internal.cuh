@@ -46,6 +46,20 @@ constexpr int kP2Stages = 2;            // per-warp bulk-copy ring depth, contra
 constexpr int kP2StageKB = 8;           // path-merged contraction 2: k-blocks per ring stage (2 KB)
 constexpr int kP2PairStages = 3;        // path-merged contraction 2: per-warp ring depth
 
+// Warp-streaming kernels for one or two activation rows.  Every warp owns an
+// equal contiguous share of the bytes a contraction streams (fixed at plan
+// build for one CTA per SM), so no work is handed out at run
+// time and no warp waits for another.
+// warps per CTA (independent of each other), one CTA per SM: 12 for one row,
+// 8 for two rows (their larger B slots)
+__host__ __device__ constexpr int pair_warps_per_cta(int MM) { return MM == 1 ? 12 : 8; }
+constexpr int kPairMaxWarps = 12;
+constexpr int kPairStages = 3;          // ring stages per warp
+constexpr int kPairStageKB = 8;         // k-blocks per ring stage (2 KB)
+constexpr int kPairMaxKB2 = 40;         // largest contraction-2 depth (k-blocks) these kernels take
+constexpr int kPairMeta1 = 16;          // bytes of exponents copied with a contraction-1 B slot
+constexpr int kPairMeta2 = 144;         // bytes of zmeta copied with a contraction-2 B slot (p * 16 + m, m < 2)
+
 // doubles in the accumulator block of a layer's scratch
 __host__ __device__ inline size_t acc_doubles(int R1) { return (size_t)R1 * 16 + 32 + 16; }
 
@@ -72,14 +86,23 @@ struct LayerDev {
     //         [2][16]  int     non-finite flags (per path x activation row)
     //   zfrag [kMaxNT][KB2][32] B fragments of contraction 2, zmeta [2][16] (exponent, digit sum)
     //   counter: contraction-1 items finished (the last one builds zfrag and clears acc)
+    //   xfrag [KB1][32] B fragments of contraction 1 (one or two rows: 16 * M lanes per k-block)
+    //   xmeta [nkc][2][2] exponent of each (k chunk, path, row)
     double *acc;
     uint2 *zfrag;
     int2 *zmeta;
     unsigned *counter;
+    uint2 *xfrag;
+    int *xmeta;
 };
 
 struct P1Item { int layer, kc; };
 struct P2Item { int layer, rg0, rg1, pad; };
+
+// Streaming units of the one/two-row kernels.  Contraction 1: row group rg of
+// k chunk kc (nkb k-blocks at a); contraction 2: row group rg (KB2 k-blocks at a).
+struct PairUnit1 { const uint2 *a; int layer, kc, rg, nkb; };
+struct PairUnit2 { const uint2 *a; int layer, rg, kb2, pad; };
 
 struct IoPtrs {
     const uint16_t *x[kIoBatch];
@@ -116,6 +139,12 @@ struct Plan {
     P1Item *p1 = nullptr;           // device work items
     P2Item *p2 = nullptr;
     std::vector<int> p1_start, p2_start;   // per IO batch: first item index
+    PairUnit1 *u1 = nullptr;        // one/two-row streaming units, all batches
+    PairUnit2 *u2 = nullptr;
+    // per row count MM (index MM - 1) and batch: pair_warps[MM - 1] + 1 unit boundaries (absolute)
+    int *wr1[2] = {nullptr, nullptr}, *wr2[2] = {nullptr, nullptr};
+    int pair_warps[2] = {0, 0};     // warps the streaming units are partitioned over, per MM
+    int kb2max = 0;                 // largest KB2 of the plan
     int *err = nullptr;             // device error code (bounded waits that gave up)
     int n_p1 = 0, n_p2 = 0;
     void *scratch = nullptr;
@@ -128,12 +157,11 @@ void plan_free(Plan &P);
 lb_status decode_forward(const Plan &P, const uint16_t *const *xs, float *const *ys, int M,
                          cudaStream_t s, int *launches);
 
-lb_status decode_pair_launch(const LayerDev *dev_layers, const P1Item *p1, int n1, const P2Item *p2, int n2,
-                             const IoPtrs &io, int base, int M, int kb2max, int *err, cudaStream_t s, int *launches,
-                             bool mark);
-lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc, const P1Item *p1, int n1,
-                            const P2Item *p2, int n2, const uint16_t *x, float *y, int M, int *err, cudaStream_t s,
-                            int *launches);
+lb_status decode_pair_launch(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1, const PairUnit1 *u1,
+                             const int *wr1, const PairUnit2 *u2, const int *wr2, int pair_warps, const IoPtrs &io,
+                             int base, int M, int kb2max, int *err, cudaStream_t s, int *launches, bool mark);
+lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc, const struct Plan &P,
+                            const uint16_t *x, float *y, int M, int *err, cudaStream_t s, int *launches);
 
 lb_status status_from(cudaError_t e);
 void set_launch_count(int n);

@@ -114,6 +114,12 @@ void plan_free(Plan &P)
     if (P.dev) cudaFree(P.dev);
     if (P.p1) cudaFree(P.p1);
     if (P.p2) cudaFree(P.p2);
+    if (P.u1) cudaFree(P.u1);
+    if (P.u2) cudaFree(P.u2);
+    for (int mm = 0; mm < 2; ++mm) {
+        if (P.wr1[mm]) cudaFree(P.wr1[mm]);
+        if (P.wr2[mm]) cudaFree(P.wr2[mm]);
+    }
     if (P.scratch) cudaFree(P.scratch);
     P = Plan();
 }
@@ -133,6 +139,8 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
         total += align256((size_t)kMaxNT * d.KB2 * 32 * sizeof(uint2));
         total += align256((size_t)2 * 16 * sizeof(int2));
         total += align256(sizeof(unsigned));
+        total += align256((size_t)d.KB1 * 32 * sizeof(uint2));
+        total += align256((size_t)d.nkc * 4 * sizeof(int));
     }
     total += 256;   // error code
     cudaError_t e = cudaMalloc(&P.scratch, std::max<size_t>(total, 256));
@@ -147,7 +155,9 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
         d.acc = (double *)c;       c += align256(acc_doubles(d.R1) * sizeof(double));
         d.zfrag = (uint2 *)c;      c += align256((size_t)kMaxNT * d.KB2 * 32 * sizeof(uint2));
         d.zmeta = (int2 *)c;       c += align256((size_t)2 * 16 * sizeof(int2));
-        d.counter = (unsigned *)c;
+        d.counter = (unsigned *)c; c += align256(sizeof(unsigned));
+        d.xfrag = (uint2 *)c;      c += align256((size_t)d.KB1 * 32 * sizeof(uint2));
+        d.xmeta = (int *)c;
         P.host[i] = d;
     }
     P.err = (int *)(base + total - 256);
@@ -181,6 +191,71 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
     }
     P.n_p1 = (int)p1.size();
     P.n_p2 = (int)p2.size();
+
+    // One/two-row streaming units in layer order, and per batch an equal split
+    // of their estimated cost over pair_warps warps (warp w streams units
+    // [wr[w], wr[w + 1]) of its batch).
+    int sms = 148, dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    P.kb2max = 0;
+    for (int i = 0; i < n; ++i) P.kb2max = std::max(P.kb2max, P.host[i].KB2);
+    std::vector<PairUnit1> u1;
+    std::vector<PairUnit2> u2;
+    std::vector<int> wr1[2], wr2[2];
+    const int nb = (int)P.p1_start.size() - 1;
+    // cost in issued instructions per warp (MMA k-blocks, ring stages, per-unit epilogue)
+    auto stages = [](int nkb) { return (double)((nkb + kPairStageKB - 1) / kPairStageKB); };
+    auto cost1 = [&](const PairUnit1 &u) { return 22.0 * u.nkb + 40.0 * stages(u.nkb) + 60.0; };
+    auto cost2 = [&](const PairUnit2 &u) { return 22.0 * u.kb2 + 40.0 * stages(u.kb2) + 110.0; };
+    for (int b = 0; b < nb; ++b) {
+        const int l0 = b * kIoBatch, l1 = std::min(n, l0 + kIoBatch);
+        const size_t s1 = u1.size(), s2 = u2.size();
+        for (int i = l0; i < l1; ++i) {
+            const LayerDev &d = P.host[i];
+            for (int kc = 0; kc < d.nkc; ++kc) {
+                const int nkb = std::min(kP1ChunkKB, d.KB1 - kc * kP1ChunkKB);
+                for (int rg = 0; rg < d.RG1; ++rg)
+                    u1.push_back({d.vt + ((size_t)rg * d.KB1 + (size_t)kc * kP1ChunkKB) * 32, i, kc, rg, nkb});
+            }
+            for (int rg = 0; rg < d.RG2; ++rg) u2.push_back({d.ut + (size_t)rg * d.KB2 * 32, i, rg, d.KB2, 0});
+        }
+        // per row count: an equal split of the estimated cost over all warps of one CTA per SM
+        for (int mm = 0; mm < 2; ++mm) {
+            const int W = sms * pair_warps_per_cta(mm + 1);
+            P.pair_warps[mm] = W;
+            auto split = [&](std::vector<int> &wr, size_t first, size_t last, auto cost_of) {
+                double total_c = 0.0;
+                for (size_t u = first; u < last; ++u) total_c += cost_of(u);
+                size_t u = first;
+                double acc = 0.0;
+                for (int w = 0; w <= W; ++w) {
+                    const double target = total_c * w / W;
+                    while (u < last && acc + 0.5 * cost_of(u) < target) acc += cost_of(u++);
+                    wr.push_back((int)(w == W ? last : u));
+                }
+            };
+            split(wr1[mm], s1, u1.size(), [&](size_t u) { return cost1(u1[u]); });
+            split(wr2[mm], s2, u2.size(), [&](size_t u) { return cost2(u2[u]); });
+        }
+    }
+    if ((e = cudaMalloc(&P.u1, sizeof(PairUnit1) * std::max<size_t>(1, u1.size()))) != cudaSuccess) return e;
+    if ((e = cudaMalloc(&P.u2, sizeof(PairUnit2) * std::max<size_t>(1, u2.size()))) != cudaSuccess) return e;
+    if (!u1.empty() && (e = cudaMemcpy(P.u1, u1.data(), sizeof(PairUnit1) * u1.size(), cudaMemcpyHostToDevice)) != cudaSuccess)
+        return e;
+    if (!u2.empty() && (e = cudaMemcpy(P.u2, u2.data(), sizeof(PairUnit2) * u2.size(), cudaMemcpyHostToDevice)) != cudaSuccess)
+        return e;
+    for (int mm = 0; mm < 2; ++mm) {
+        if ((e = cudaMalloc(&P.wr1[mm], sizeof(int) * std::max<size_t>(1, wr1[mm].size()))) != cudaSuccess) return e;
+        if ((e = cudaMalloc(&P.wr2[mm], sizeof(int) * std::max<size_t>(1, wr2[mm].size()))) != cudaSuccess) return e;
+        if ((e = cudaMemcpy(P.wr1[mm], wr1[mm].data(), sizeof(int) * wr1[mm].size(), cudaMemcpyHostToDevice)) !=
+            cudaSuccess)
+            return e;
+        if ((e = cudaMemcpy(P.wr2[mm], wr2[mm].data(), sizeof(int) * wr2[mm].size(), cudaMemcpyHostToDevice)) !=
+            cudaSuccess)
+            return e;
+    }
+
     if ((e = cudaMalloc(&P.dev, sizeof(LayerDev) * n)) != cudaSuccess) return e;
     if ((e = cudaMalloc(&P.p1, sizeof(P1Item) * std::max(1, P.n_p1))) != cudaSuccess) return e;
     if ((e = cudaMalloc(&P.p2, sizeof(P2Item) * std::max(1, P.n_p2))) != cudaSuccess) return e;

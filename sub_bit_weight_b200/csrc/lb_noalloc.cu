@@ -56,7 +56,9 @@ extern "C" lb_status lb_linear_forward_noalloc(const uint16_t *x, int M, const l
     const LayerDev &src = L->d;
     const size_t acc_n = acc_doubles(src.R1);
     const size_t off_frag = kOffAcc + al256(acc_n * sizeof(double));
-    const size_t need = off_frag + (size_t)kMaxNT * src.KB2 * 32 * sizeof(uint2);
+    const size_t off_xfrag = off_frag + al256((size_t)kMaxNT * src.KB2 * 32 * sizeof(uint2));
+    const size_t off_xmeta = off_xfrag + al256((size_t)src.KB1 * 32 * sizeof(uint2));
+    const size_t need = off_xmeta + (size_t)src.nkc * 4 * sizeof(int);
     if (need > LB_NOALLOC_SCRATCH_BYTES) return LB_ERR_UNSUPPORTED;
 
     int dev = 0;
@@ -79,13 +81,15 @@ extern "C" lb_status lb_linear_forward_noalloc(const uint16_t *x, int M, const l
     d.zfrag = reinterpret_cast<uint2 *>(base + off_frag);
     d.zmeta = reinterpret_cast<int2 *>(base + kOffMeta);
     d.counter = reinterpret_cast<unsigned *>(base + kOffCounter);
+    d.xfrag = reinterpret_cast<uint2 *>(base + off_xfrag);
+    d.xmeta = reinterpret_cast<int *>(base + off_xmeta);
     cudaStream_t s = (cudaStream_t)stream;
     noalloc_setup_kernel<<<64, 256, 0, s>>>(d, acc_n);
     if ((e = cudaGetLastError()) != cudaSuccess) return status_from(e);
     const Plan &P = L->self->plan;   // the layer's own work items (read only)
     int launches = 1;
-    lb_status st = decode_launch_one(reinterpret_cast<const LayerDev *>(base + kOffDesc), d, P.p1, P.n_p1, P.p2, P.n_p2,
-                                     x, y, M, reinterpret_cast<int *>(base + kOffErr), s, &launches);
+    lb_status st = decode_launch_one(reinterpret_cast<const LayerDev *>(base + kOffDesc), d, P, x, y, M,
+                                     reinterpret_cast<int *>(base + kOffErr), s, &launches);
     set_launch_count(launches);
     return st;
 }

@@ -71,11 +71,12 @@ def test_rows_above_decode_limit(env):
         assert rel_err(y, ref) <= TOL
 
 
-def test_repeatable(env):
+@pytest.mark.parametrize("M", [1, 4])
+def test_repeatable(env, M):
     torch, lib, stacks = env
     shape = synth.LayerShape("t", 512, 2048, 128)
     layer = stacks.build_layer(5, 0, shape)
-    x = stacks.bf16_on_device(synth.activations(5, 0, 4, shape.K), "cuda")
+    x = stacks.bf16_on_device(synth.activations(5, 0, M, shape.K), "cuda")
     y1 = lib.lb_linear_forward(x, layer).clone()
     y2 = lib.lb_linear_forward(x, layer)
     torch.cuda.synchronize()
@@ -122,32 +123,39 @@ def test_zero_and_negative_scales(env):
     assert torch.count_nonzero(y2).item() == 0
 
 
-def test_nonfinite_activation_row(env):
+@pytest.mark.parametrize("M", [1, 2, 3])
+def test_nonfinite_activation_row(env, M):
     torch, lib, stacks = env
     shape = synth.LayerShape("t", 128, 256, 32)
     layer = stacks.build_layer(10, 0, shape)
-    xb = synth.activations(10, 0, 3, shape.K).copy()
-    xb[1, 17] = 0x7FC0            # bfloat16 NaN in row 1
+    xb = synth.activations(10, 0, M, shape.K).copy()
+    bad = min(1, M - 1)
+    xb[bad, 17] = 0x7FC0          # bfloat16 NaN in one row
     y = lib.lb_linear_forward(stacks.bf16_on_device(xb, "cuda"), layer).cpu().numpy()
-    assert np.all(np.isnan(y[1]))
+    assert np.all(np.isnan(y[bad]))
     ref = oracle.forward(xb, oracle_layer(10, 0, shape))
-    assert np.all(np.isnan(ref[1]))
-    keep = [0, 2]
-    assert rel_err(y[keep], ref[keep]) <= TOL
+    assert np.all(np.isnan(ref[bad]))
+    keep = [m for m in range(M) if m != bad]
+    if keep:
+        assert rel_err(y[keep], ref[keep]) <= TOL
+    # the next call on the same layer is unaffected by the non-finite row
+    xg = synth.activations(11, 0, M, shape.K)
+    y2 = lib.lb_linear_forward(stacks.bf16_on_device(xg, "cuda"), layer).cpu().numpy()
+    assert rel_err(y2, oracle.forward(xg, oracle_layer(10, 0, shape))) <= TOL
 
 
-def test_stack_matches_single_layer_calls(env):
+@pytest.mark.parametrize("M", [1, 5])
+def test_stack_matches_single_layer_calls(env, M):
     torch, lib, stacks = env
     shapes = [synth.LayerShape("a", 192, 320, 40), synth.LayerShape("b", 64, 1024, 16),
               synth.LayerShape("c", 1000, 96, 200), synth.LayerShape("a", 192, 320, 40)]
     layers = [stacks.build_layer(20 + i, i, s) for i, s in enumerate(shapes)]
     layers[3] = layers[0]                       # a layer may repeat in a stack
     S = lib.lb_stack_create(layers)
-    M = 5
     xs = [stacks.bf16_on_device(synth.activations(30 + i, i, M, s.K), "cuda") for i, s in enumerate(shapes)]
     ys = [torch.empty((M, s.N), dtype=torch.float32, device="cuda") for s in shapes]
     lib.lb_stack_forward(S, xs, ys)
-    assert lib.lb_last_launch_count() == 2
+    assert lib.lb_last_launch_count() == (4 if M <= 2 else 2)
     for i, s in enumerate(shapes):
         single = lib.lb_linear_forward(xs[i], layers[i])
         torch.cuda.synchronize()
