@@ -34,71 +34,80 @@ static __device__ __forceinline__ int pair_lane(int m, int p, int d, int kk)
 }
 
 // ---------------------------------------------------------------------------
-// Activation quantisation (one CTA per 1024-input chunk of a layer)
+// Activation quantisation: one warp per 1024-input chunk, lane L takes k-block
+// L of the chunk (32 inputs) and writes that k-block's whole B fragment.
 // ---------------------------------------------------------------------------
+constexpr int kQuantWarps = 4;
+
+// The four bytes of 32-bit values a..d, low byte first.
+static __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
+{
+    return (uint32_t)(a & 255) | ((uint32_t)(b & 255) << 8) | ((uint32_t)(c & 255) << 16) | ((uint32_t)(d & 255) << 24);
+}
+
 template <int MM>
-__global__ void __launch_bounds__(kDecodeThreads)
-    quantize_pair_kernel(const LayerDev *__restrict__ layers, const P1Item *__restrict__ items,
+__global__ void __launch_bounds__(kQuantWarps * 32, MM == 1 ? 5 : 3)
+    quantize_pair_kernel(const LayerDev *__restrict__ layers, const P1Item *__restrict__ items, int nitems,
                          const __grid_constant__ IoPtrs io, int base, int M)
 {
-    constexpr int kLanes = 16 * MM;     // stored lanes per k-block
-    __shared__ float sMax[4];
-    __shared__ int sBad[4], sE[4], sQs[4];
-    const int tid = threadIdx.x, lane = tid & 31;
-    const P1Item item = items[blockIdx.x];
+    const int lane = threadIdx.x & 31;
+    const int it = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+    if (it >= nitems) return;
+    const P1Item item = items[it];
     const LayerDev *dp = layers + item.layer;
     const int K = dp->K, K32 = dp->K32, KB1 = dp->KB1, npaths = dp->npaths, R1 = dp->R1;
-    const __half *__restrict__ gsc = dp->g;
     const uint16_t *__restrict__ x = io.x[item.layer - base];
-    const int kb0 = item.kc * kP1ChunkKB;
-    const int nkb = min(kP1ChunkKB, KB1 - kb0);
-    const int k0 = kb0 * kKPerBlock;
-    const int klen = nkb * kKPerBlock;
-    if (tid < 4) {
-        sMax[tid] = 0.0f;
-        sBad[tid] = 0;
-        sQs[tid] = 0;
-    }
-    __syncthreads();
+    const int kb = item.kc * kP1ChunkKB + lane;
+    const bool act = kb < KB1;
+    const int k0 = kb * kKPerBlock;
 
-    // t = x (.) g_p for 8 consecutive inputs per thread
-    const int kk0 = 8 * tid;
-    const bool act = kk0 < klen;
-    const int kg = k0 + kk0;
-    float gv[2][8];
+    // raw bf16 activations and binary16 g of this lane's 32 inputs (two per word)
+    uint32_t xr[MM][16], gr[2][16];
 #pragma unroll
     for (int p = 0; p < 2; ++p) {
         if (act && p < npaths) {
-            const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(gsc + (size_t)p * K32 + kg));
-            const __half *hv = reinterpret_cast<const __half *>(&raw);
+            const uint4 *src = reinterpret_cast<const uint4 *>(dp->g + (size_t)p * K32 + k0);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) gv[p][e] = __half2float(hv[e]);
+            for (int i = 0; i < 4; ++i) {
+                const uint4 v = __ldg(src + i);
+                gr[p][4 * i] = v.x; gr[p][4 * i + 1] = v.y; gr[p][4 * i + 2] = v.z; gr[p][4 * i + 3] = v.w;
+            }
         } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) gv[p][e] = 0.0f;
+            for (int i = 0; i < 16; ++i) gr[p][i] = 0u;
         }
     }
-    float xv[MM][8];
-    const bool vec = ((K & 7) == 0) && (kg + 8 <= K);
+    const bool vec = ((K & 7) == 0) && (k0 + kKPerBlock <= K);
 #pragma unroll
     for (int m = 0; m < MM; ++m) {
         if (!act || m >= M) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) xv[m][e] = 0.0f;
+            for (int i = 0; i < 16; ++i) xr[m][i] = 0u;
         } else if (vec) {
-            const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + kg));
-            const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)m * K + k0);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                xv[m][2 * e] = __uint_as_float(w4[e] << 16);
-                xv[m][2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
+            for (int i = 0; i < 4; ++i) {
+                const uint4 v = __ldg(src + i);
+                xr[m][4 * i] = v.x; xr[m][4 * i + 1] = v.y; xr[m][4 * i + 2] = v.z; xr[m][4 * i + 3] = v.w;
             }
         } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                xv[m][e] = (kg + e < K) ? bf16_bits_to_float(__ldg(x + (size_t)m * K + kg + e)) : 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                const int k = k0 + 2 * i;
+                const uint32_t lo = (k < K) ? __ldg(x + (size_t)m * K + k) : 0u;
+                const uint32_t hi = (k + 1 < K) ? __ldg(x + (size_t)m * K + k + 1) : 0u;
+                xr[m][i] = lo | (hi << 16);
+            }
         }
     }
+    auto tval = [&](int m, int p, int e) -> float {      // x_e * g_{p,e} (exact in fp32)
+        const uint32_t xw = xr[m][e >> 1], gw = gr[p][e >> 1];
+        const float xv = __uint_as_float((e & 1) ? (xw & 0xffff0000u) : (xw << 16));
+        const float gv = __half2float(__ushort_as_half((unsigned short)((e & 1) ? (gw >> 16) : (gw & 0xffffu))));
+        return xv * gv;
+    };
+
+    uint4 *dst = reinterpret_cast<uint4 *>(dp->xfrag + (size_t)kb * 16 * MM);
 #pragma unroll
     for (int m = 0; m < MM; ++m)
 #pragma unroll
@@ -106,67 +115,54 @@ __global__ void __launch_bounds__(kDecodeThreads)
             float amax = 0.0f;
             int bad = 0;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float tv = fabsf(xv[m][e] * gv[p][e]);
+            for (int e = 0; e < 32; ++e) {
+                const float tv = fabsf(tval(m, p, e));
                 if (!(tv <= FLT_MAX)) bad = 1;
                 else amax = fmaxf(amax, tv);
             }
             amax = warp_max(amax);
             bad = warp_or(bad);
-            if (lane == 0 && p < npaths && m < M) {
-                smem_max(&sMax[2 * p + m], amax);
-                if (bad) atomicOr(&sBad[2 * p + m], 1);
-            }
-        }
-    __syncthreads();
-    if (tid < 4) {
-        const int p = tid >> 1, m = tid & 1;
-        sE[tid] = (p < npaths && m < M) ? exponent_for(sMax[tid], sBad[tid] != 0) : kNanExp;
-    }
-    __syncthreads();
-    uint32_t *xw = reinterpret_cast<uint32_t *>(dp->xfrag + (size_t)kb0 * kLanes);
-#pragma unroll
-    for (int m = 0; m < MM; ++m)
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
             const bool live = m < M && p < npaths;
-            const int E = sE[2 * p + m];
-            const float sc = (!live || E == kNanExp) ? 0.0f : pow2f(E);
+            const int E = live ? exponent_for(amax, bad != 0) : kNanExp;
+            const float sc = (E == kNanExp) ? 0.0f : pow2f(E);
+            // column 4 m + 2 p + d: lanes t = 0..3 hold k 4t..4t+3 (first word) and 16+4t.. (second);
+            // one 16-byte store covers lanes 2 tp and 2 tp + 1 of a column
             int qs = 0;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t wlo = 0, whi = 0;
+            for (int tp = 0; tp < 2; ++tp) {
+                uint32_t wlo[4], whi[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int q = quantize_s(xv[m][4 * h + e] * gv[p][4 * h + e], sc);
-                    int lo, hi;
-                    digits(q, lo, hi);
-                    wlo |= (uint32_t)(lo & 255) << (8 * e);
-                    whi |= (uint32_t)(hi & 255) << (8 * e);
-                    qs += q;
+                for (int i = 0; i < 4; ++i) {
+                    const int t = 2 * tp + (i >> 1), k = 16 * (i & 1) + 4 * t;
+                    int q[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        q[e] = quantize_s(tval(m, p, k + e), sc);
+                        qs += q[e];
+                    }
+                    wlo[i] = pack4(q[0], q[1], q[2], q[3]);
+                    whi[i] = pack4((q[0] + 128) >> 8, (q[1] + 128) >> 8, (q[2] + 128) >> 8, (q[3] + 128) >> 8);
                 }
                 if (act) {
-                    // every word of the chunk's fragments is written (zeros for absent rows and paths)
-                    const int kk = kk0 + 4 * h;
-                    uint32_t *fb = xw + (size_t)(kk >> 5) * kLanes * 2;
-                    const int word = (kk & 31) >> 4;
-                    fb[2 * pair_lane(m, p, 0, kk & 31) + word] = wlo;
-                    fb[2 * pair_lane(m, p, 1, kk & 31) + word] = whi;
+                    const int col = 4 * m + 2 * p;
+                    dst[2 * col + tp] = make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
+                    dst[2 * (col + 1) + tp] = make_uint4(whi[0], whi[1], whi[2], whi[3]);
                 }
             }
             qs = warp_sum(qs);
-            if (lane == 0 && qs) atomicAdd(&sQs[2 * p + m], qs);
+            if (lane == 0) {
+                dp->xmeta[item.kc * 4 + 2 * p + m] = E;
+                if (live) {
+                    double *acc = dp->acc;
+                    if (E == kNanExp) atomicOr(reinterpret_cast<int *>(acc + (size_t)R1 * 16 + 32) + p * 16 + m, 1);
+                    else if (qs) atomicAdd(acc + (size_t)R1 * 16 + p * 16 + m, (double)qs * pow2d(-E));
+                }
+            }
         }
-    __syncthreads();
-    if (tid < 4) {
-        const int p = tid >> 1, m = tid & 1;
-        const int E = sE[tid];
-        dp->xmeta[item.kc * 4 + tid] = E;
-        if (p < npaths && m < M) {
-            double *acc = dp->acc;
-            if (E == kNanExp) atomicOr(reinterpret_cast<int *>(acc + (size_t)R1 * 16 + 32) + p * 16 + m, 1);
-            else if (sQs[tid]) atomicAdd(acc + (size_t)R1 * 16 + p * 16 + m, (double)sQs[tid] * pow2d(-E));
-        }
+    if (MM == 1 && lane == 0) {
+        // m = 1 slots of the chunk's exponents stay absent
+        dp->xmeta[item.kc * 4 + 1] = kNanExp;
+        dp->xmeta[item.kc * 4 + 3] = kNanExp;
     }
 }
 
@@ -174,7 +170,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
 // Finish of contraction 1 (one CTA per layer): zl = (S_p - 2 acc) * l_p as
 // 16-bit fixed point per (path, row), written as contraction-2 B fragments
 // (16 * M lanes per k-block) plus (exponent, digit sum) in zmeta; clears the
-// accumulators for the next call.
+// accumulators for the next call.  zl is staged in shared memory.
 // ---------------------------------------------------------------------------
 constexpr int kFinishThreads = 256;
 
@@ -182,6 +178,7 @@ template <int MM>
 __global__ void __launch_bounds__(kFinishThreads)
     finish_pair_kernel(const LayerDev *__restrict__ layers, int base, int M)
 {
+    extern __shared__ float szl[];      // [npaths][r][MM]
     __shared__ float sMax[4];
     __shared__ int sBad[4], sE[4], sQs[4];
     const int tid = threadIdx.x;
@@ -197,16 +194,17 @@ __global__ void __launch_bounds__(kFinishThreads)
         sQs[tid] = 0;
     }
     __syncthreads();
-    auto zl_at = [&](int p, int j, int m) -> float {
-        const double z = __ldcg(S + p * 16 + m) - 2.0 * __ldcg(acc + (size_t)(p * r16 + j) * 16 + m);
-        return (float)z * __half2float(lsc[p * r16 + j]);
-    };
-    for (int e = tid; e < npaths * r * M; e += kFinishThreads) {
-        const int m = e % M, pj = e / M;
+    for (int e = tid; e < npaths * r * MM; e += kFinishThreads) {
+        const int m = e % MM, pj = e / MM;
         const int p = pj / r, j = pj - p * r;
-        const float zl = zl_at(p, j, m);
-        if (!(fabsf(zl) <= FLT_MAX)) atomicOr(&sBad[2 * p + m], 1);
-        else smem_max(&sMax[2 * p + m], fabsf(zl));
+        float zl = 0.0f;
+        if (m < M) {
+            const double z = __ldcg(S + p * 16 + m) - 2.0 * __ldcg(acc + (size_t)(p * r16 + j) * 16 + m);
+            zl = (float)z * __half2float(lsc[p * r16 + j]);
+            if (!(fabsf(zl) <= FLT_MAX)) atomicOr(&sBad[2 * p + m], 1);
+            else smem_max(&sMax[2 * p + m], fabsf(zl));
+        }
+        szl[e] = zl;
     }
     __syncthreads();
     if (tid < 4) {
@@ -231,7 +229,7 @@ __global__ void __launch_bounds__(kFinishThreads)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = j0 + 16 * hh + e;
-                    const int q = (j < r) ? quantize_s(zl_at(fp, j, fm), sc) : 0;
+                    const int q = (j < r) ? quantize_s(szl[(fp * r + j) * MM + fm], sc) : 0;
                     int lo, hi;
                     digits(q, lo, hi);
                     w[hh] |= (uint32_t)((fd ? hi : lo) & 255) << (8 * e);
@@ -643,8 +641,8 @@ static int g_pair_smem[2][2];     // dynamic shared memory attribute set so far,
 template <int MM>
 static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1,
                                 const PairUnit1 *u1, const int *wr1, const PairUnit2 *u2, const int *wr2,
-                                int pair_warps, const IoPtrs &io, int base, int M, int kb2max, int *err, cudaStream_t s,
-                                int *launches, bool mark)
+                                int pair_warps, const IoPtrs &io, int base, int M, int kb2max, int rmax, int *err,
+                                cudaStream_t s, int *launches, bool mark)
 {
     cudaError_t e;
     constexpr int kPairWarps = pair_warps_per_cta(MM);
@@ -652,7 +650,8 @@ static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P
         (size_t)kPairWarps * (kPairStages * kPairStageKB * 256 + 2 * (kP1ChunkKB * 16 * MM * 8 + 128));
     const size_t smem2 =
         (size_t)kPairWarps * (kPairStages * kPairStageKB * 256 + 2 * ((size_t)kb2max * 16 * MM * 8 + kPairMeta2));
-    if (smem1 > 227 * 1024 || smem2 > 227 * 1024 || kb2max > kPairMaxKB2) return LB_ERR_UNSUPPORTED;
+    if (smem1 > 227 * 1024 || smem2 > 227 * 1024 || kb2max > kPairMaxKB2 || (size_t)2 * rmax * MM * sizeof(float) > 48 * 1024)
+        return LB_ERR_UNSUPPORTED;
     if ((int)smem1 > g_pair_smem[0][MM - 1]) {
         if ((e = cudaFuncSetAttribute(contraction1_pair_kernel<MM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem1)) != cudaSuccess)
@@ -667,14 +666,15 @@ static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P
     }
     const int grid = pair_warps / kPairWarps;
     if (n1 > 0) {
-        quantize_pair_kernel<MM><<<n1, kDecodeThreads, 0, s>>>(dev_layers, p1, io, base, M);
+        quantize_pair_kernel<MM><<<(n1 + kQuantWarps - 1) / kQuantWarps, kQuantWarps * 32, 0, s>>>(dev_layers, p1, n1, io,
+                                                                                                  base, M);
         ++*launches;
         if (mark) profile_mark(*launches, s);
     }
     contraction1_pair_kernel<MM><<<grid, kPairWarps * 32, smem1, s>>>(dev_layers, u1, wr1, M, err);
     ++*launches;
     if (mark) profile_mark(*launches, s);
-    finish_pair_kernel<MM><<<nlayers, kFinishThreads, 0, s>>>(dev_layers, base, M);
+    finish_pair_kernel<MM><<<nlayers, kFinishThreads, (size_t)2 * rmax * MM * sizeof(float), s>>>(dev_layers, base, M);
     ++*launches;
     if (mark) profile_mark(*launches, s);
     contraction2_pair_kernel<MM><<<grid, kPairWarps * 32, smem2, s>>>(dev_layers, u2, wr2, io, base, M, kb2max, err);
@@ -685,13 +685,13 @@ static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P
 
 lb_status decode_pair_launch(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1, const PairUnit1 *u1,
                              const int *wr1, const PairUnit2 *u2, const int *wr2, int pair_warps, const IoPtrs &io,
-                             int base, int M, int kb2max, int *err, cudaStream_t s, int *launches, bool mark)
+                             int base, int M, int kb2max, int rmax, int *err, cudaStream_t s, int *launches, bool mark)
 {
     if (M == 1)
-        return pair_launch_mm<1>(dev_layers, nlayers, p1, n1, u1, wr1, u2, wr2, pair_warps, io, base, M, kb2max, err, s,
-                                 launches, mark);
-    return pair_launch_mm<2>(dev_layers, nlayers, p1, n1, u1, wr1, u2, wr2, pair_warps, io, base, M, kb2max, err, s,
-                             launches, mark);
+        return pair_launch_mm<1>(dev_layers, nlayers, p1, n1, u1, wr1, u2, wr2, pair_warps, io, base, M, kb2max, rmax,
+                                 err, s, launches, mark);
+    return pair_launch_mm<2>(dev_layers, nlayers, p1, n1, u1, wr1, u2, wr2, pair_warps, io, base, M, kb2max, rmax, err,
+                             s, launches, mark);
 }
 
 }  // namespace lb

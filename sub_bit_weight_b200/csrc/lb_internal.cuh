@@ -145,6 +145,7 @@ struct Plan {
     int *wr1[2] = {nullptr, nullptr}, *wr2[2] = {nullptr, nullptr};
     int pair_warps[2] = {0, 0};     // warps the streaming units are partitioned over, per MM
     int kb2max = 0;                 // largest KB2 of the plan
+    int rmax = 0;                   // largest rank of the plan
     int *err = nullptr;             // device error code (bounded waits that gave up)
     int n_p1 = 0, n_p2 = 0;
     void *scratch = nullptr;
@@ -159,7 +160,7 @@ lb_status decode_forward(const Plan &P, const uint16_t *const *xs, float *const 
 
 lb_status decode_pair_launch(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1, const PairUnit1 *u1,
                              const int *wr1, const PairUnit2 *u2, const int *wr2, int pair_warps, const IoPtrs &io,
-                             int base, int M, int kb2max, int *err, cudaStream_t s, int *launches, bool mark);
+                             int base, int M, int kb2max, int rmax, int *err, cudaStream_t s, int *launches, bool mark);
 lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc, const struct Plan &P,
                             const uint16_t *x, float *y, int M, int *err, cudaStream_t s, int *launches);
 

@@ -199,7 +199,11 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     P.kb2max = 0;
-    for (int i = 0; i < n; ++i) P.kb2max = std::max(P.kb2max, P.host[i].KB2);
+    P.rmax = 0;
+    for (int i = 0; i < n; ++i) {
+        P.kb2max = std::max(P.kb2max, P.host[i].KB2);
+        P.rmax = std::max(P.rmax, P.host[i].r);
+    }
     std::vector<PairUnit1> u1;
     std::vector<PairUnit2> u2;
     std::vector<int> wr1[2], wr2[2];
