@@ -603,8 +603,9 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
         if (M <= 2 && kb2max <= kPairMaxKB2) {
             const int W = P.pair_warps[M - 1];
             lb_status st = decode_pair_launch(P.dev, cnt, P.p1 + P.p1_start[b], n1, P.u1, P.wr1[M - 1] + (size_t)b * (W + 1),
-                                              P.u2, P.wr2[M - 1] + (size_t)b * (W + 1), W, io, base, M, kb2max, P.rmax,
-                                              P.err, s, launches, true);
+                                              P.u2, P.wr2[M - 1] + (size_t)b * (P.pair_warps2[M - 1] + 1), W,
+                                              P.pair_warps2[M - 1], io, base, M, kb2max, P.rmax, P.err, s, launches,
+                                              true);
             if (st == LB_OK) continue;
             if (st != LB_ERR_UNSUPPORTED) return st;
             // shapes the streaming kernels cannot hold in shared memory take the general kernels
@@ -633,8 +634,8 @@ lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc,
         static thread_local IoPtrs io1;
         io1.x[0] = x;
         io1.y[0] = y;
-        return decode_pair_launch(dev_desc, 1, p1, n1, P.u1, P.wr1[M - 1], P.u2, P.wr2[M - 1], P.pair_warps[M - 1], io1, 0,
-                                  M, host_desc.KB2, host_desc.r, err, s, launches, false);
+        return decode_pair_launch(dev_desc, 1, p1, n1, P.u1, P.wr1[M - 1], P.u2, P.wr2[M - 1], P.pair_warps[M - 1],
+                                  P.pair_warps2[M - 1], io1, 0, M, host_desc.KB2, host_desc.r, err, s, launches, false);
     }
     const int NT = (M + 3) / 4;
     cudaError_t e = cudaSuccess;

@@ -84,6 +84,13 @@ static __device__ __forceinline__ uint2 lds64(uint32_t addr)
     return v;
 }
 
+static __device__ __forceinline__ unsigned short lds_u16(uint32_t addr)
+{
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];\n" : "=h"(v) : "r"(addr));
+    return v;
+}
+
 static __device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
 {
     uint32_t v;
@@ -128,6 +135,32 @@ static __device__ __forceinline__ void bulk_copy(void *dst, const void *src, uns
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
                      sm_addr(dst)),
                  "l"(src), "r"(bytes), "r"(sm_addr(bar))
+                 : "memory");
+}
+
+// L2 policy for data read exactly once per call (the weight streams): evict first,
+// so that what is re-read (fragments, scales) stays in L2.
+static __device__ __forceinline__ uint64_t l2_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+    return pol;
+}
+
+static __device__ __forceinline__ void bulk_copy_hint(void *dst, const void *src, unsigned bytes, uint64_t *bar,
+                                                      uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;\n" ::"r"(
+            sm_addr(dst)),
+        "l"(src), "r"(bytes), "r"(sm_addr(bar)), "l"(pol)
+        : "memory");
+}
+
+static __device__ __forceinline__ void expect_tx(uint64_t *bar, unsigned bytes)
+{
+    asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(sm_addr(bar)),
+                 "r"(bytes)
                  : "memory");
 }
 

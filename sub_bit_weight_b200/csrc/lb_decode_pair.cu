@@ -297,77 +297,62 @@ static __device__ __forceinline__ void mma_stage(int (&a4)[4][4], uint32_t src, 
 }
 
 // ---------------------------------------------------------------------------
-// Contraction 1 (one warp per contiguous run of units)
+// Contraction 1 (one warp per contiguous run of units).  A ring stage holds up
+// to kPairStageKB k-blocks of one unit's V tiles, the B fragments of the same
+// k-blocks and the chunk's four exponents (three bulk copies on one mbarrier);
+// nothing else is shared between units, so the warp needs no B slots.
 // ---------------------------------------------------------------------------
 template <int MM>
 __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
     contraction1_pair_kernel(const LayerDev *__restrict__ layers, const PairUnit1 *__restrict__ units,
                              const int *__restrict__ wrange, int M, int *err)
 {
-    constexpr int kStage = kPairStageKB * 256;
     constexpr int kBStride = 16 * MM * 8;                   // bytes of B fragments per k-block
-    constexpr int kBFrag = kP1ChunkKB * kBStride;
-    constexpr int kBSlot = kBFrag + 128;                    // fragments, then the chunk's exponents
-    constexpr int kWarpBytes = kPairStages * kStage + 2 * kBSlot;
-    extern __shared__ __align__(128) unsigned char smem_raw[];
+    constexpr int kA = kPairStageKB * 256, kB = kPairStageKB * kBStride;
+    constexpr int kStageAll = kA + kB + 16;                 // V tiles, B fragments, exponents
     constexpr int kPairWarps = pair_warps_per_cta(MM);
+    extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ uint64_t rbar[kPairWarps][kPairStages];
-    __shared__ uint64_t bbar[kPairWarps][2];
     __shared__ __align__(16) uint2 zero8[2];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t4 = lane & 3;
     const int lane_m = t4 >> 1, lane_p = t4 & 1;       // accumulator columns of this lane
-    unsigned char *ring = smem_raw + warp * kWarpBytes;
-    unsigned char *bslot = ring + kPairStages * kStage;
+    unsigned char *ring = smem_raw + warp * (kPairStages * kStageAll);
     if (threadIdx.x == 0) zero8[0] = zero8[1] = make_uint2(0u, 0u);
-    if (lane == 0) {
+    if (lane == 0)
         for (int s = 0; s < kPairStages; ++s) bar_init(&rbar[warp][s]);
-        bar_init(&bbar[warp][0]);
-        bar_init(&bbar[warp][1]);
-    }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     __syncthreads();    // the only CTA-wide barrier: zero8 and the barriers are ready
 
     const int gw = warp * gridDim.x + blockIdx.x;     // an SM's warps take ranges spread over the whole batch
     const int u0 = wrange[gw], u1 = wrange[gw + 1];
     if (u0 >= u1) return;
+    const uint64_t pol = l2_evict_first();
 
-    // ---- fill cursor: stages of units [f_u, u1) in consumption order, at most
-    // kPairStages ahead; B fragments of at most two chunks resident at a time.
-    int f_u = u0, f_h = 0, f_cs = -1, f_layer = -1, f_kc = -1, issued = 0, consumed = 0, c_cs = -1;
+    // ---- fill cursor: stages of units [f_u, u1) in consumption order, at most kPairStages ahead
+    int f_u = u0, f_h = 0, f_layer = -1, issued = 0, consumed = 0;
     const uint2 *f_xfrag = nullptr;
     const int *f_xmeta = nullptr;
     PairUnit1 f_cur = units[u0], f_nxt = f_cur;
     if (u0 + 1 < u1) f_nxt = units[u0 + 1];
     auto fill = [&]() {
         while (f_u < u1 && issued - consumed < kPairStages) {
-            if (f_h == 0 && (f_cur.layer != f_layer || f_cur.kc != f_kc)) {
-                if (f_cs >= c_cs + 1) return;           // both B slots still in use
-                if (f_cur.layer != f_layer) {
-                    f_layer = f_cur.layer;
-                    f_xfrag = layers[f_layer].xfrag;
-                    f_xmeta = layers[f_layer].xmeta;
-                }
-                f_kc = f_cur.kc;
-                ++f_cs;
-                if (lane == 0) {
-                    unsigned char *dst = bslot + (f_cs & 1) * kBSlot;
-                    uint64_t *bar = &bbar[warp][f_cs & 1];
-                    const unsigned fb = (unsigned)f_cur.nkb * kBStride;
-                    asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(
-                                     sm_addr(bar)),
-                                 "r"(fb + 16u)
-                                 : "memory");
-                    bulk_copy(dst, f_xfrag + (size_t)f_kc * kP1ChunkKB * 16 * MM, fb, bar);
-                    bulk_copy(dst + kBFrag, f_xmeta + f_kc * 4, 16u, bar);
-                }
+            if (f_cur.layer != f_layer) {
+                f_layer = f_cur.layer;
+                f_xfrag = layers[f_layer].xfrag;
+                f_xmeta = layers[f_layer].xmeta;
             }
             const int n = min(kPairStageKB, f_cur.nkb - f_h * kPairStageKB);
             if (lane == 0) {
                 const int st = issued % kPairStages;
-                ring_fill(ring + st * kStage, f_cur.a + (size_t)f_h * kPairStageKB * 32, (unsigned)n * 256u,
-                          &rbar[warp][st]);
+                unsigned char *dst = ring + st * kStageAll;
+                uint64_t *bar = &rbar[warp][st];
+                const int kb0 = f_cur.kc * kP1ChunkKB + f_h * kPairStageKB;
+                expect_tx(bar, (unsigned)n * (256u + kBStride) + 16u);
+                bulk_copy_hint(dst, f_cur.a + (size_t)f_h * kPairStageKB * 32, (unsigned)n * 256u, bar, pol);
+                bulk_copy(dst + kA, f_xfrag + (size_t)kb0 * 16 * MM, (unsigned)n * kBStride, bar);
+                bulk_copy(dst + kA + kB, f_xmeta + f_cur.kc * 4, 16u, bar);
             }
             ++issued;
             if (++f_h * kPairStageKB >= f_cur.nkb) {
@@ -381,13 +366,11 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
     fill();
 
     // ---- consumer
-    int c_layer = -1, c_kc = -1, c_r16 = 1, c_npaths = 1;
+    int c_layer = -1, c_r16 = 1, c_npaths = 1;
     double *c_acc = nullptr;
-    double lane_sc = 0.0;
-    bool lane_live = false;
-    uint32_t bbase = 0, bstride = 0;
+    const bool real = lane < 16 * MM;
+    const uint32_t bstride = real ? (uint32_t)kBStride : 0u;
     const uint32_t zaddr = sm_addr(zero8);
-
     PairUnit1 c_nxt = units[u0];
     for (int u = u0; u < u1; ++u) {
         const PairUnit1 cu = c_nxt;
@@ -398,34 +381,26 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
             c_acc = dp->acc;
             c_r16 = dp->r16;
             c_npaths = dp->npaths;
-            c_kc = -1;
         }
-        if (cu.kc != c_kc) {
-            c_kc = cu.kc;
-            ++c_cs;
-            fill();                                        // the next chunk's B may start now
-            if (!ring_wait(&bbar[warp][c_cs & 1], (c_cs >> 1) & 1, err)) return;
-            const unsigned char *slot = bslot + (c_cs & 1) * kBSlot;
-            const int E = (lane_m < M && lane_p < c_npaths)
-                              ? (int)lds_u32(sm_addr(slot + kBFrag + 4 * (2 * lane_p + lane_m)))
-                              : kNanExp;
-            lane_live = E != kNanExp;
-            lane_sc = lane_live ? pow2d(-E) : 0.0;
-            const bool real = lane < 16 * MM;
-            bbase = real ? sm_addr(slot) + lane * 8 : zaddr;
-            bstride = real ? (uint32_t)kBStride : 0u;
-        }
-
         int a4[4][4];
 #pragma unroll
         for (int rb = 0; rb < 4; ++rb)
 #pragma unroll
             for (int c = 0; c < 4; ++c) a4[rb][c] = 0;
+        double lane_sc = 0.0;
+        bool lane_live = false;
         for (int h = 0; h * kPairStageKB < cu.nkb; ++h) {
             const int st = consumed % kPairStages;
             if (!ring_wait(&rbar[warp][st], (consumed / kPairStages) & 1, err)) return;
-            mma_stage<MM>(a4, sm_addr(ring + st * kStage) + lane * 8, bbase + (uint32_t)(h * kPairStageKB) * bstride,
-                          bstride, min(kPairStageKB, cu.nkb - h * kPairStageKB));
+            const uint32_t sbase = sm_addr(ring + st * kStageAll);
+            if (h == 0) {
+                const int E = (lane_m < M && lane_p < c_npaths) ? (int)lds_u32(sbase + kA + kB + 4 * (2 * lane_p + lane_m))
+                                                                 : kNanExp;
+                lane_live = E != kNanExp;
+                lane_sc = lane_live ? pow2d(-E) : 0.0;
+            }
+            mma_stage<MM>(a4, sbase + lane * 8, real ? sbase + kA + lane * 8 : zaddr, bstride,
+                          min(kPairStageKB, cu.nkb - h * kPairStageKB));
             __syncwarp();
             if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
             ++consumed;
@@ -435,7 +410,7 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
 #pragma unroll
         for (int rb = 0; rb < 4; ++rb) {
             const int row0 = cu.rg * kRowsPerGroup + rb * kRowsPerBlock;
-            const int prb = min(row0 / c_r16, c_npaths - 1);
+            const int prb = (c_npaths > 1 && row0 >= c_r16) ? 1 : 0;     // path 1 owns rows r16..
             if (prb != lane_p || !lane_live) continue;
             const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
             const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
@@ -451,19 +426,18 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
 // up to kPairStageKB consecutive k-blocks across row-group boundaries (never
 // across layers); the consumer folds a row group when its KB2 k-blocks are in.
 // ---------------------------------------------------------------------------
-template <int MM>
-__global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
+template <int MM, int NW>
+__global__ void __launch_bounds__(NW * 32, 1)
     contraction2_pair_kernel(const LayerDev *__restrict__ layers, const PairUnit2 *__restrict__ units,
                              const int *__restrict__ wrange, const __grid_constant__ IoPtrs io, int base, int M,
                              int kb2max, int *err)
 {
     constexpr int kStage = kPairStageKB * 256;
     constexpr int kBStride = 16 * MM * 8;
-    constexpr int kPairWarps = pair_warps_per_cta(MM);
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    __shared__ uint64_t rbar[kPairWarps][kPairStages];
-    __shared__ uint64_t bbar[kPairWarps][2];
-    __shared__ int snb[kPairWarps][kPairStages];       // k-blocks in each ring stage
+    __shared__ uint64_t rbar[NW][kPairStages];
+    __shared__ uint64_t bbar[NW][2];
+    __shared__ int snb[NW][kPairStages];       // k-blocks in each ring stage
     __shared__ __align__(16) uint2 zero8[2];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -484,6 +458,7 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
     const int gw = warp * gridDim.x + blockIdx.x;     // an SM's warps take ranges spread over the whole batch
     const int u0 = wrange[gw], u1 = wrange[gw + 1];
     if (u0 >= u1) return;
+    const uint64_t pol = l2_evict_first();
 
     // ---- fill cursor (position: unit f_u, k-block f_kb within it)
     int f_u = u0, f_kb = 0, f_layer = -1, f_cs = -1, issued = 0, consumed = 0, c_cs = -1;
@@ -523,7 +498,10 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
             }
             const int st = issued % kPairStages;
             snb[warp][st] = n;
-            if (lane == 0) ring_fill(ring + st * kStage, src, (unsigned)n * 256u, &rbar[warp][st]);
+            if (lane == 0) {
+                expect_tx(&rbar[warp][st], (unsigned)n * 256u);
+                bulk_copy_hint(ring + st * kStage, src, (unsigned)n * 256u, &rbar[warp][st], pol);
+            }
             ++issued;
         }
     };
@@ -636,62 +614,80 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-static int g_pair_smem[2][2];     // dynamic shared memory attribute set so far, per kernel and MM
+static int g_pair_smem1[2];          // dynamic shared memory attribute set so far, per MM
+static int g_pair_smem2[2][5];       // per MM and contraction-2 warp count (16, 12, 8, 6, 4)
+
+template <int MM, int NW>
+static cudaError_t launch_c2(int grid, size_t smem, cudaStream_t s, int slot, const LayerDev *dev_layers,
+                             const PairUnit2 *u2, const int *wr2, const IoPtrs &io, int base, int M, int kb2max, int *err)
+{
+    cudaError_t e;
+    if ((int)smem > g_pair_smem2[MM - 1][slot]) {
+        if ((e = cudaFuncSetAttribute(contraction2_pair_kernel<MM, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess)
+            return e;
+        g_pair_smem2[MM - 1][slot] = (int)smem;
+    }
+    contraction2_pair_kernel<MM, NW><<<grid, NW * 32, smem, s>>>(dev_layers, u2, wr2, io, base, M, kb2max, err);
+    return cudaGetLastError();
+}
 
 template <int MM>
 static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1,
                                 const PairUnit1 *u1, const int *wr1, const PairUnit2 *u2, const int *wr2,
-                                int pair_warps, const IoPtrs &io, int base, int M, int kb2max, int rmax, int *err,
-                                cudaStream_t s, int *launches, bool mark)
+                                int pair_warps, int pair_warps2, const IoPtrs &io, int base, int M, int kb2max, int rmax,
+                                int *err, cudaStream_t s, int *launches, bool mark)
 {
     cudaError_t e;
     constexpr int kPairWarps = pair_warps_per_cta(MM);
-    const size_t smem1 =
-        (size_t)kPairWarps * (kPairStages * kPairStageKB * 256 + 2 * (kP1ChunkKB * 16 * MM * 8 + 128));
-    const size_t smem2 =
-        (size_t)kPairWarps * (kPairStages * kPairStageKB * 256 + 2 * ((size_t)kb2max * 16 * MM * 8 + kPairMeta2));
-    if (smem1 > 227 * 1024 || smem2 > 227 * 1024 || kb2max > kPairMaxKB2 || (size_t)2 * rmax * MM * sizeof(float) > 48 * 1024)
+    const int nw2 = pair2_warps_per_cta(MM, kb2max);
+    const size_t smem1 = (size_t)kPairWarps * kPairStages * (kPairStageKB * (256 + 16 * MM * 8) + 16);
+    const size_t smem2 = (size_t)nw2 * pair2_smem_per_warp(MM, kb2max);
+    if (smem1 > 227 * 1024 || smem2 > 227 * 1024 || kb2max > kPairMaxKB2 || pair_warps2 % nw2 != 0 ||
+        (size_t)2 * rmax * MM * sizeof(float) > 48 * 1024)
         return LB_ERR_UNSUPPORTED;
-    if ((int)smem1 > g_pair_smem[0][MM - 1]) {
+    if ((int)smem1 > g_pair_smem1[MM - 1]) {
         if ((e = cudaFuncSetAttribute(contraction1_pair_kernel<MM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem1)) != cudaSuccess)
             return status_from(e);
-        g_pair_smem[0][MM - 1] = (int)smem1;
+        g_pair_smem1[MM - 1] = (int)smem1;
     }
-    if ((int)smem2 > g_pair_smem[1][MM - 1]) {
-        if ((e = cudaFuncSetAttribute(contraction2_pair_kernel<MM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)smem2)) != cudaSuccess)
-            return status_from(e);
-        g_pair_smem[1][MM - 1] = (int)smem2;
-    }
-    const int grid = pair_warps / kPairWarps;
     if (n1 > 0) {
         quantize_pair_kernel<MM><<<(n1 + kQuantWarps - 1) / kQuantWarps, kQuantWarps * 32, 0, s>>>(dev_layers, p1, n1, io,
                                                                                                   base, M);
         ++*launches;
         if (mark) profile_mark(*launches, s);
     }
-    contraction1_pair_kernel<MM><<<grid, kPairWarps * 32, smem1, s>>>(dev_layers, u1, wr1, M, err);
+    contraction1_pair_kernel<MM><<<pair_warps / kPairWarps, kPairWarps * 32, smem1, s>>>(dev_layers, u1, wr1, M, err);
     ++*launches;
     if (mark) profile_mark(*launches, s);
     finish_pair_kernel<MM><<<nlayers, kFinishThreads, (size_t)2 * rmax * MM * sizeof(float), s>>>(dev_layers, base, M);
     ++*launches;
     if (mark) profile_mark(*launches, s);
-    contraction2_pair_kernel<MM><<<grid, kPairWarps * 32, smem2, s>>>(dev_layers, u2, wr2, io, base, M, kb2max, err);
+    const int grid2 = pair_warps2 / nw2;
+    switch (nw2) {
+    case 16: e = launch_c2<MM, 16>(grid2, smem2, s, 0, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
+    case 12: e = launch_c2<MM, 12>(grid2, smem2, s, 1, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
+    case 8: e = launch_c2<MM, 8>(grid2, smem2, s, 2, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
+    case 6: e = launch_c2<MM, 6>(grid2, smem2, s, 3, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
+    default: e = launch_c2<MM, 4>(grid2, smem2, s, 4, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
+    }
+    if (e != cudaSuccess) return status_from(e);
     ++*launches;
     if (mark) profile_mark(*launches, s);
     return status_from(cudaGetLastError());
 }
 
 lb_status decode_pair_launch(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1, const PairUnit1 *u1,
-                             const int *wr1, const PairUnit2 *u2, const int *wr2, int pair_warps, const IoPtrs &io,
-                             int base, int M, int kb2max, int rmax, int *err, cudaStream_t s, int *launches, bool mark)
+                             const int *wr1, const PairUnit2 *u2, const int *wr2, int pair_warps, int pair_warps2,
+                             const IoPtrs &io, int base, int M, int kb2max, int rmax, int *err, cudaStream_t s,
+                             int *launches, bool mark)
 {
     if (M == 1)
-        return pair_launch_mm<1>(dev_layers, nlayers, p1, n1, u1, wr1, u2, wr2, pair_warps, io, base, M, kb2max, rmax,
-                                 err, s, launches, mark);
-    return pair_launch_mm<2>(dev_layers, nlayers, p1, n1, u1, wr1, u2, wr2, pair_warps, io, base, M, kb2max, rmax, err,
-                             s, launches, mark);
+        return pair_launch_mm<1>(dev_layers, nlayers, p1, n1, u1, wr1, u2, wr2, pair_warps, pair_warps2, io, base, M,
+                                 kb2max, rmax, err, s, launches, mark);
+    return pair_launch_mm<2>(dev_layers, nlayers, p1, n1, u1, wr1, u2, wr2, pair_warps, pair_warps2, io, base, M,
+                             kb2max, rmax, err, s, launches, mark);
 }
 
 }  // namespace lb

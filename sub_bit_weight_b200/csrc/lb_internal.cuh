@@ -50,14 +50,26 @@ constexpr int kP2PairStages = 3;        // path-merged contraction 2: per-warp r
 // equal contiguous share of the bytes a contraction streams (fixed at plan
 // build for one CTA per SM), so no work is handed out at run
 // time and no warp waits for another.
-// warps per CTA (independent of each other), one CTA per SM: 12 for one row,
-// 8 for two rows (their larger B slots)
-__host__ __device__ constexpr int pair_warps_per_cta(int MM) { return MM == 1 ? 12 : 8; }
-constexpr int kPairMaxWarps = 12;
-constexpr int kPairStages = 3;          // ring stages per warp
-constexpr int kPairStageKB = 8;         // k-blocks per ring stage (2 KB)
+// contraction-1 warps per CTA (independent of each other), one CTA per SM: 16
+// for one row, 12 for two rows (their larger B fragments)
+__host__ __device__ constexpr int pair_warps_per_cta(int MM) { return MM == 1 ? 16 : 12; }
+constexpr int kPairStages = 2;          // ring stages per warp
+constexpr int kPairStageKB = 16;        // k-blocks per ring stage (4 KB)
 constexpr int kPairMaxKB2 = 40;         // largest contraction-2 depth (k-blocks) these kernels take
-constexpr int kPairMeta1 = 16;          // bytes of exponents copied with a contraction-1 B slot
+// Shared memory per warp of the contraction-2 kernel, and its warps per CTA: the
+// most of {16, 12, 8, 6, 4} whose CTA fits in 227 KB.
+__host__ __device__ constexpr int pair2_smem_per_warp(int MM, int kb2max)
+{
+    return kPairStages * kPairStageKB * 256 + 2 * (kb2max * 16 * MM * 8 + 144);
+}
+__host__ __device__ constexpr int pair2_warps_per_cta(int MM, int kb2max)
+{
+    return (16 * pair2_smem_per_warp(MM, kb2max) <= 227 * 1024)   ? 16
+           : (12 * pair2_smem_per_warp(MM, kb2max) <= 227 * 1024) ? 12
+           : (8 * pair2_smem_per_warp(MM, kb2max) <= 227 * 1024)  ? 8
+           : (6 * pair2_smem_per_warp(MM, kb2max) <= 227 * 1024)  ? 6
+                                                                   : 4;
+}
 constexpr int kPairMeta2 = 144;         // bytes of zmeta copied with a contraction-2 B slot (p * 16 + m, m < 2)
 
 // doubles in the accumulator block of a layer's scratch
@@ -143,7 +155,8 @@ struct Plan {
     PairUnit2 *u2 = nullptr;
     // per row count MM (index MM - 1) and batch: pair_warps[MM - 1] + 1 unit boundaries (absolute)
     int *wr1[2] = {nullptr, nullptr}, *wr2[2] = {nullptr, nullptr};
-    int pair_warps[2] = {0, 0};     // warps the streaming units are partitioned over, per MM
+    int pair_warps[2] = {0, 0};     // contraction-1 warps the streaming units are partitioned over, per MM
+    int pair_warps2[2] = {0, 0};    // the same for contraction 2
     int kb2max = 0;                 // largest KB2 of the plan
     int rmax = 0;                   // largest rank of the plan
     int *err = nullptr;             // device error code (bounded waits that gave up)
@@ -159,8 +172,9 @@ lb_status decode_forward(const Plan &P, const uint16_t *const *xs, float *const 
                          cudaStream_t s, int *launches);
 
 lb_status decode_pair_launch(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1, const PairUnit1 *u1,
-                             const int *wr1, const PairUnit2 *u2, const int *wr2, int pair_warps, const IoPtrs &io,
-                             int base, int M, int kb2max, int rmax, int *err, cudaStream_t s, int *launches, bool mark);
+                             const int *wr1, const PairUnit2 *u2, const int *wr2, int pair_warps, int pair_warps2,
+                             const IoPtrs &io, int base, int M, int kb2max, int rmax, int *err, cudaStream_t s,
+                             int *launches, bool mark);
 lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc, const struct Plan &P,
                             const uint16_t *x, float *y, int M, int *err, cudaStream_t s, int *launches);
 

@@ -211,7 +211,7 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
     // cost in issued instructions per warp (MMA k-blocks, ring stages, per-unit epilogue)
     auto stages = [](int nkb) { return (double)((nkb + kPairStageKB - 1) / kPairStageKB); };
     auto cost1 = [&](const PairUnit1 &u) { return 22.0 * u.nkb + 40.0 * stages(u.nkb) + 60.0; };
-    auto cost2 = [&](const PairUnit2 &u) { return 22.0 * u.kb2 + 40.0 * stages(u.kb2) + 110.0; };
+    auto cost2 = [&](const PairUnit2 &u) { return 22.0 * u.kb2 + 40.0 * u.kb2 / kPairStageKB + 110.0; };
     for (int b = 0; b < nb; ++b) {
         const int l0 = b * kIoBatch, l1 = std::min(n, l0 + kIoBatch);
         const size_t s1 = u1.size(), s2 = u2.size();
@@ -226,9 +226,11 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
         }
         // per row count: an equal split of the estimated cost over all warps of one CTA per SM
         for (int mm = 0; mm < 2; ++mm) {
-            const int W = sms * pair_warps_per_cta(mm + 1);
-            P.pair_warps[mm] = W;
-            auto split = [&](std::vector<int> &wr, size_t first, size_t last, auto cost_of) {
+            const int W1 = sms * pair_warps_per_cta(mm + 1);
+            const int W2 = sms * pair2_warps_per_cta(mm + 1, std::min(P.kb2max, kPairMaxKB2));
+            P.pair_warps[mm] = W1;
+            P.pair_warps2[mm] = W2;
+            auto split = [&](std::vector<int> &wr, size_t first, size_t last, int W, auto cost_of) {
                 double total_c = 0.0;
                 for (size_t u = first; u < last; ++u) total_c += cost_of(u);
                 size_t u = first;
@@ -239,8 +241,8 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
                     wr.push_back((int)(w == W ? last : u));
                 }
             };
-            split(wr1[mm], s1, u1.size(), [&](size_t u) { return cost1(u1[u]); });
-            split(wr2[mm], s2, u2.size(), [&](size_t u) { return cost2(u2[u]); });
+            split(wr1[mm], s1, u1.size(), W1, [&](size_t u) { return cost1(u1[u]); });
+            split(wr2[mm], s2, u2.size(), W2, [&](size_t u) { return cost2(u2[u]); });
         }
     }
     if ((e = cudaMalloc(&P.u1, sizeof(PairUnit1) * std::max<size_t>(1, u1.size()))) != cudaSuccess) return e;
