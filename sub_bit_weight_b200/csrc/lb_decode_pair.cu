@@ -256,43 +256,46 @@ __global__ void __launch_bounds__(kFinishThreads)
 // path from one unit to the next.
 // ---------------------------------------------------------------------------
 
-template <int MM>
-static __device__ __forceinline__ void mma_stage(int (&a4)[4][4], uint32_t src, uint32_t bsrc, uint32_t bstride, int n)
+// N k-blocks of MMAs, fully unrolled: A word pairs 256 bytes apart, B fragments
+// 16 * MM * 8 bytes apart (lanes without B data read a zero buffer of the same
+// shape), so every shared-memory address is a register plus an immediate.
+template <int MM, int N>
+static __device__ __forceinline__ void mma_run(int (&a4)[4][4], uint32_t src, uint32_t bsrc)
 {
-    if (n == kPairStageKB) {
 #pragma unroll
-        for (int v = 0; v < kPairStageKB; ++v) {
-            const uint2 w = lds64(src + v * 256);
-            const uint2 b = lds64(bsrc + v * bstride);
+    for (int v = 0; v < N; ++v) {
+        const uint2 w = lds64(src + v * 256);
+        const uint2 b = lds64(bsrc + v * (16 * MM * 8));
 #pragma unroll
-            for (int rb = 0; rb < 4; ++rb) {
-                const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
-            }
+        for (int rb = 0; rb < 4; ++rb) {
+            const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+            mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
         }
-    } else {
-        int v = 0;
-        for (; v + 4 <= n; v += 4) {
-#pragma unroll
-            for (int vv = 0; vv < 4; ++vv) {
-                const uint2 w = lds64(src + (v + vv) * 256);
-                const uint2 b = lds64(bsrc + (v + vv) * bstride);
-#pragma unroll
-                for (int rb = 0; rb < 4; ++rb) {
-                    const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                    mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
-                }
-            }
-        }
-        for (; v < n; ++v) {
-            const uint2 w = lds64(src + v * 256);
-            const uint2 b = lds64(bsrc + v * bstride);
-#pragma unroll
-            for (int rb = 0; rb < 4; ++rb) {
-                const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-                mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
-            }
-        }
+    }
+}
+
+template <int MM>
+static __device__ __forceinline__ void mma_stage(int (&a4)[4][4], uint32_t src, uint32_t bsrc, int n)
+{
+    static_assert(kPairStageKB == 16, "one case per segment length");
+    switch (n) {
+    case 16: mma_run<MM, 16>(a4, src, bsrc); break;
+    case 15: mma_run<MM, 15>(a4, src, bsrc); break;
+    case 14: mma_run<MM, 14>(a4, src, bsrc); break;
+    case 13: mma_run<MM, 13>(a4, src, bsrc); break;
+    case 12: mma_run<MM, 12>(a4, src, bsrc); break;
+    case 11: mma_run<MM, 11>(a4, src, bsrc); break;
+    case 10: mma_run<MM, 10>(a4, src, bsrc); break;
+    case 9: mma_run<MM, 9>(a4, src, bsrc); break;
+    case 8: mma_run<MM, 8>(a4, src, bsrc); break;
+    case 7: mma_run<MM, 7>(a4, src, bsrc); break;
+    case 6: mma_run<MM, 6>(a4, src, bsrc); break;
+    case 5: mma_run<MM, 5>(a4, src, bsrc); break;
+    case 4: mma_run<MM, 4>(a4, src, bsrc); break;
+    case 3: mma_run<MM, 3>(a4, src, bsrc); break;
+    case 2: mma_run<MM, 2>(a4, src, bsrc); break;
+    case 1: mma_run<MM, 1>(a4, src, bsrc); break;
+    default: break;
     }
 }
 
@@ -313,17 +316,17 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
     constexpr int kPairWarps = pair_warps_per_cta(MM);
     extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ uint64_t rbar[kPairWarps][kPairStages];
-    __shared__ __align__(16) uint2 zero8[2];
+    __shared__ __align__(16) uint4 zbuf[MM == 1 ? kPairStageKB * 128 / 16 : 1];   // B of the lanes past 16 * MM
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t4 = lane & 3;
     const int lane_m = t4 >> 1, lane_p = t4 & 1;       // accumulator columns of this lane
     unsigned char *ring = smem_raw + warp * (kPairStages * kStageAll);
-    if (threadIdx.x == 0) zero8[0] = zero8[1] = make_uint2(0u, 0u);
+    for (int i = threadIdx.x; i < (int)(sizeof(zbuf) / 16); i += blockDim.x) zbuf[i] = make_uint4(0u, 0u, 0u, 0u);
     if (lane == 0)
         for (int s = 0; s < kPairStages; ++s) bar_init(&rbar[warp][s]);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    __syncthreads();    // the only CTA-wide barrier: zero8 and the barriers are ready
+    __syncthreads();    // the only CTA-wide barrier: the zero buffer and the barriers are ready
 
     const int gw = warp * gridDim.x + blockIdx.x;     // an SM's warps take ranges spread over the whole batch
     const int u0 = wrange[gw], u1 = wrange[gw + 1];
@@ -369,8 +372,7 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
     int c_layer = -1, c_r16 = 1, c_npaths = 1;
     double *c_acc = nullptr;
     const bool real = lane < 16 * MM;
-    const uint32_t bstride = real ? (uint32_t)kBStride : 0u;
-    const uint32_t zaddr = sm_addr(zero8);
+    const uint32_t zaddr = sm_addr(zbuf) + (lane & 15) * 8;
     PairUnit1 c_nxt = units[u0];
     for (int u = u0; u < u1; ++u) {
         const PairUnit1 cu = c_nxt;
@@ -399,7 +401,7 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
                 lane_live = E != kNanExp;
                 lane_sc = lane_live ? pow2d(-E) : 0.0;
             }
-            mma_stage<MM>(a4, sbase + lane * 8, real ? sbase + kA + lane * 8 : zaddr, bstride,
+            mma_stage<MM>(a4, sbase + lane * 8, real ? sbase + kA + lane * 8 : zaddr,
                           min(kPairStageKB, cu.nkb - h * kPairStageKB));
             __syncwarp();
             if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
@@ -438,7 +440,6 @@ __global__ void __launch_bounds__(NW * 32, 1)
     __shared__ uint64_t rbar[NW][kPairStages];
     __shared__ uint64_t bbar[NW][2];
     __shared__ int snb[NW][kPairStages];       // k-blocks in each ring stage
-    __shared__ __align__(16) uint2 zero8[2];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t4 = lane & 3;
@@ -446,7 +447,10 @@ __global__ void __launch_bounds__(NW * 32, 1)
     const int kBFrag = kb2max * kBStride, kBSlot = kBFrag + kPairMeta2;
     unsigned char *ring = smem_raw + (size_t)warp * (kPairStages * kStage + 2 * kBSlot);
     unsigned char *bslot = ring + kPairStages * kStage;
-    if (threadIdx.x == 0) zero8[0] = zero8[1] = make_uint2(0u, 0u);
+    // after the warps' regions: zeros shaped like a B slot, read by the lanes past 16 * MM
+    uint4 *zbuf = reinterpret_cast<uint4 *>(smem_raw + (size_t)NW * (kPairStages * kStage + 2 * kBSlot));
+    if (MM == 1)
+        for (int i = threadIdx.x; i < kb2max * kBStride / 16; i += blockDim.x) zbuf[i] = make_uint4(0u, 0u, 0u, 0u);
     if (lane == 0) {
         for (int s = 0; s < kPairStages; ++s) bar_init(&rbar[warp][s]);
         bar_init(&bbar[warp][0]);
@@ -510,8 +514,8 @@ __global__ void __launch_bounds__(NW * 32, 1)
     int c_layer = -1, N = 0, npaths = 1;
     float *y = nullptr;
     float my_sc = 0.0f, my_q = 0.0f;
-    uint32_t bbase = 0, bstride = 0;
-    const uint32_t zaddr = sm_addr(zero8);
+    uint32_t bbase = 0;
+    const uint32_t zaddr = sm_addr(zbuf) + (lane & 15) * 8;
     int s_left = 0;             // k-blocks of the current stage not yet used
     uint32_t s_addr = 0;        // this lane's word pair of the stage's next k-block
 
@@ -527,7 +531,7 @@ __global__ void __launch_bounds__(NW * 32, 1)
         }
         const __half *hp = h_base + un.rg * kRowsPerGroup + g;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) hq[i] = h_base ? hp[(i >> 1) * kRowsPerBlock + 8 * (i & 1)] : __half(0.0f);
+        for (int i = 0; i < 8; ++i) hq[i] = h_base ? __ldg(hp + (i >> 1) * kRowsPerBlock + 8 * (i & 1)) : __half(0.0f);
     };
     PairUnit2 c_nxt = units[u0];
     __half h_nxt[8];
@@ -564,7 +568,6 @@ __global__ void __launch_bounds__(NW * 32, 1)
             }
             const bool real = lane < 16 * MM;
             bbase = real ? sm_addr(slot) + lane * 8 : zaddr;
-            bstride = real ? (uint32_t)kBStride : 0u;
         }
         const int n0 = cu.rg * kRowsPerGroup + g;
 
@@ -581,7 +584,7 @@ __global__ void __launch_bounds__(NW * 32, 1)
                 s_addr = sm_addr(ring + st * kStage) + lane * 8;
             }
             const int seg = min(s_left, cu.kb2 - kb);
-            mma_stage<MM>(a4, s_addr, bbase + (uint32_t)kb * bstride, bstride, seg);
+            mma_stage<MM>(a4, s_addr, bbase + (uint32_t)kb * kBStride, seg);
             kb += seg;
             s_left -= seg;
             s_addr += (uint32_t)seg * 256u;
@@ -642,7 +645,7 @@ static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P
     constexpr int kPairWarps = pair_warps_per_cta(MM);
     const int nw2 = pair2_warps_per_cta(MM, kb2max);
     const size_t smem1 = (size_t)kPairWarps * kPairStages * (kPairStageKB * (256 + 16 * MM * 8) + 16);
-    const size_t smem2 = (size_t)nw2 * pair2_smem_per_warp(MM, kb2max);
+    const size_t smem2 = pair2_cta_smem(MM, kb2max, nw2);
     if (smem1 > 227 * 1024 || smem2 > 227 * 1024 || kb2max > kPairMaxKB2 || pair_warps2 % nw2 != 0 ||
         (size_t)2 * rmax * MM * sizeof(float) > 48 * 1024)
         return LB_ERR_UNSUPPORTED;

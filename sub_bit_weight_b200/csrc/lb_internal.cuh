@@ -56,19 +56,24 @@ __host__ __device__ constexpr int pair_warps_per_cta(int MM) { return MM == 1 ? 
 constexpr int kPairStages = 2;          // ring stages per warp
 constexpr int kPairStageKB = 16;        // k-blocks per ring stage (4 KB)
 constexpr int kPairMaxKB2 = 40;         // largest contraction-2 depth (k-blocks) these kernels take
-// Shared memory per warp of the contraction-2 kernel, and its warps per CTA: the
-// most of {16, 12, 8, 6, 4} whose CTA fits in 227 KB.
+// Shared memory of the contraction-2 kernel (per warp; per CTA with the zero
+// buffer of one-row batches), and its warps per CTA: the most of
+// {16, 12, 8, 6, 4} whose CTA fits in 227 KB.
 __host__ __device__ constexpr int pair2_smem_per_warp(int MM, int kb2max)
 {
     return kPairStages * kPairStageKB * 256 + 2 * (kb2max * 16 * MM * 8 + 144);
 }
+__host__ __device__ constexpr int pair2_cta_smem(int MM, int kb2max, int nw)
+{
+    return nw * pair2_smem_per_warp(MM, kb2max) + (MM == 1 ? kb2max * 128 : 0);
+}
 __host__ __device__ constexpr int pair2_warps_per_cta(int MM, int kb2max)
 {
-    return (16 * pair2_smem_per_warp(MM, kb2max) <= 227 * 1024)   ? 16
-           : (12 * pair2_smem_per_warp(MM, kb2max) <= 227 * 1024) ? 12
-           : (8 * pair2_smem_per_warp(MM, kb2max) <= 227 * 1024)  ? 8
-           : (6 * pair2_smem_per_warp(MM, kb2max) <= 227 * 1024)  ? 6
-                                                                   : 4;
+    return (pair2_cta_smem(MM, kb2max, 16) <= 227 * 1024)   ? 16
+           : (pair2_cta_smem(MM, kb2max, 12) <= 227 * 1024) ? 12
+           : (pair2_cta_smem(MM, kb2max, 8) <= 227 * 1024)  ? 8
+           : (pair2_cta_smem(MM, kb2max, 6) <= 227 * 1024)  ? 6
+                                                             : 4;
 }
 constexpr int kPairMeta2 = 144;         // bytes of zmeta copied with a contraction-2 B slot (p * 16 + m, m < 2)
 
