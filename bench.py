@@ -87,6 +87,12 @@ def measured_traffic(kernel: str, workload: str):
     return None
 
 
+def prefill_traffic(workload: str):
+    """DRAM bytes of one prefill step (both tensor-core launches), while their sources are unchanged."""
+    t = [measured_traffic(k, workload) for k in ("prefill_kernel<0>", "prefill_kernel<1>")]
+    return None if any(v is None for v in t) else sum(t)
+
+
 # ----------------------------------------------------------------- algorithmic work
 
 def layer_bytes(s: synth.LayerShape, M: int, npaths: int = 2):
@@ -227,6 +233,7 @@ def run_gpu(w: synth.Workload, M: int, steps: int, warmup: int, dist, dev, want_
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
+        torch.cuda.nvtx.range_push("bench_timed")       # lets a profiler select the timed launches
         start.record(stream)
         for k in range(steps):
             lib.lb_profile_events(ev[k])
@@ -235,6 +242,7 @@ def run_gpu(w: synth.Workload, M: int, steps: int, warmup: int, dist, dev, want_
                 nlaunch_per_step = lib.lb_last_launch_count()
         stop.record(stream)
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
     lib.lb_profile_events([])
     if dist:
         dist.barrier()
@@ -405,7 +413,7 @@ def main():
                                         "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                                         "frac": round(tf / pk["bf16_tflops_sustained"], 4),
                                         "peak_src": pk["src"] + " bf16 sustained (dense 16-bit tensor peak)",
-                                        "traffic": None},
+                                        "traffic": prefill_traffic(pw.key)},
                            "clocks": pres["clocks"]}
 
     if rank == 0 and args.cpu_seconds > 0:
