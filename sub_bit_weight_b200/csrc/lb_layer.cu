@@ -208,10 +208,12 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
     std::vector<PairUnit2> u2;
     std::vector<int> wr1[2], wr2[2];
     const int nb = (int)P.p1_start.size() - 1;
-    // cost in issued instructions per warp (MMA k-blocks, ring stages, per-unit epilogue)
+    // contraction 1: cost in issued instructions per warp (MMA k-blocks, ring stages, per-unit epilogue)
     auto stages = [](int nkb) { return (double)((nkb + kPairStageKB - 1) / kPairStageKB); };
     auto cost1 = [&](const PairUnit1 &u) { return 22.0 * u.nkb + 40.0 * stages(u.nkb) + 60.0; };
-    auto cost2 = [&](const PairUnit2 &u) { return 22.0 * u.kb2 + 40.0 * u.kb2 / kPairStageKB + 110.0; };
+    // contraction 2, in k-block equivalents (fitted to per-warp times on B200): a k-block, 8.5 per row group
+    // (fold, h, stores), 15 where a layer starts (its zl fragments are waited for)
+    auto cost2 = [&](const PairUnit2 &u) { return (double)u.kb2 + 8.5 + (u.rg == 0 ? 15.0 : 0.0); };
     for (int b = 0; b < nb; ++b) {
         const int l0 = b * kIoBatch, l1 = std::min(n, l0 + kIoBatch);
         const size_t s1 = u1.size(), s2 = u2.size();
