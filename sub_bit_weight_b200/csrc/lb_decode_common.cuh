@@ -109,6 +109,16 @@ static __device__ __forceinline__ float lds_f32(uint32_t addr)
 static __device__ __forceinline__ void smem_max(float *a, float v) { atomicMax((int *)a, __float_as_int(v)); }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while the previous kernel of the stream still runs;
+// dep_wait() returns once that kernel has completed and its writes are visible
+// (immediately when the launch had no such dependency).  dep_release() lets the
+// next kernel of the stream start launching.
+// ---------------------------------------------------------------------------
+static __device__ __forceinline__ void dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+static __device__ __forceinline__ void dep_release() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // mbarrier + bulk copy (one ring of buffers per warp)
 // ---------------------------------------------------------------------------
 static __device__ __forceinline__ uint32_t sm_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }

@@ -19,9 +19,14 @@
 //   finish_pair_kernel        zl = z (.) l_p as 16-bit fixed point -> the
 //                             contraction-2 B fragments (one CTA per layer)
 //   contraction2_pair_kernel  y = sum_p h_p (.) (U_p zl_p) over U tiles
+// The float64 row sums of contraction 1 use the first R1 * M doubles of the
+// layer's accumulator block as a compact [R1][M] array (the general decode
+// kernels use [R1][16]); both leave the block zero for the next call.
 // In both contractions every warp streams its own contiguous, equal share of
 // the weight bytes (a static partition made at plan build) through a private
 // ring of bulk copies; warps never synchronise with each other.
+
+#include <utility>
 
 #include "lb_decode_common.cuh"
 
@@ -50,6 +55,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32, MM == 1 ? 5 : 3)
     quantize_pair_kernel(const LayerDev *__restrict__ layers, const P1Item *__restrict__ items, int nitems,
                          const __grid_constant__ IoPtrs io, int base, int M)
 {
+    dep_release();
     const int lane = threadIdx.x & 31;
     const int it = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
     if (it >= nitems) return;
@@ -182,10 +188,12 @@ __global__ void __launch_bounds__(kFinishThreads)
     __shared__ float sMax[4];
     __shared__ int sBad[4], sE[4], sQs[4];
     const int tid = threadIdx.x;
+    dep_release();
     const LayerDev *dp = layers + base + blockIdx.x;
     const int R1 = dp->R1, r = dp->r, r16 = dp->r16, r32 = dp->r32, npaths = dp->npaths, KB2 = dp->KB2;
     double *acc = dp->acc;
     const __half *lsc = dp->l;
+    dep_wait();                          // the row sums of contraction 1
     const double *S = acc + (size_t)R1 * 16;
     const int *badf = reinterpret_cast<const int *>(acc + (size_t)R1 * 16 + 32);
     if (tid < 4) {
@@ -199,7 +207,7 @@ __global__ void __launch_bounds__(kFinishThreads)
         const int p = pj / r, j = pj - p * r;
         float zl = 0.0f;
         if (m < M) {
-            const double z = __ldcg(S + p * 16 + m) - 2.0 * __ldcg(acc + (size_t)(p * r16 + j) * 16 + m);
+            const double z = __ldcg(S + p * 16 + m) - 2.0 * __ldcg(acc + (size_t)(p * r16 + j) * MM + m);
             zl = (float)z * __half2float(lsc[p * r16 + j]);
             if (!(fabsf(zl) <= FLT_MAX)) atomicOr(&sBad[2 * p + m], 1);
             else smem_max(&sMax[2 * p + m], fabsf(zl));
@@ -244,8 +252,8 @@ __global__ void __launch_bounds__(kFinishThreads)
         const int p = tid >> 1, m = tid & 1;
         dp->zmeta[p * 16 + m] = make_int2(sE[tid], sQs[tid]);
     }
-    // clear for the next call: rows' columns m < MM, the k sums and the flags
-    for (int i = tid; i < R1 * MM; i += kFinishThreads) acc[(size_t)(i / MM) * 16 + (i % MM)] = 0.0;
+    // clear for the next call: the rows (compact [R1][MM] here), the k sums and the flags
+    for (int i = tid; i < R1 * MM; i += kFinishThreads) acc[i] = 0.0;
     for (int i = tid; i < 48; i += kFinishThreads) acc[(size_t)R1 * 16 + i] = 0.0;
 }
 
@@ -327,11 +335,19 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
         for (int s = 0; s < kPairStages; ++s) bar_init(&rbar[warp][s]);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     __syncthreads();    // the only CTA-wide barrier: the zero buffer and the barriers are ready
+    dep_release();
 
     const int gw = warp * gridDim.x + blockIdx.x;     // an SM's warps take ranges spread over the whole batch
     const int u0 = wrange[gw], u1 = wrange[gw + 1];
     if (u0 >= u1) return;
     const uint64_t pol = l2_evict_first();
+    // V tiles do not depend on the previous kernel; B fragments and exponents do: stages
+    // filled before dep_wait() get theirs afterwards (at most kPairStages of them)
+    bool dep_ok = false;
+    int npend = 0;
+    const uint2 *pend_b[kPairStages];
+    const int *pend_e[kPairStages];
+    unsigned pend_nb[kPairStages];
 
     // ---- fill cursor: stages of units [f_u, u1) in consumption order, at most kPairStages ahead
     int f_u = u0, f_h = 0, f_layer = -1, issued = 0, consumed = 0;
@@ -354,9 +370,20 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
                 const int kb0 = f_cur.kc * kP1ChunkKB + f_h * kPairStageKB;
                 expect_tx(bar, (unsigned)n * (256u + kBStride) + 16u);
                 bulk_copy_hint(dst, f_cur.a + (size_t)f_h * kPairStageKB * 32, (unsigned)n * 256u, bar, pol);
-                bulk_copy(dst + kA, f_xfrag + (size_t)kb0 * 16 * MM, (unsigned)n * kBStride, bar);
-                bulk_copy(dst + kA + kB, f_xmeta + f_cur.kc * 4, 16u, bar);
+                if (dep_ok) {
+                    bulk_copy(dst + kA, f_xfrag + (size_t)kb0 * 16 * MM, (unsigned)n * kBStride, bar);
+                    bulk_copy(dst + kA + kB, f_xmeta + f_cur.kc * 4, 16u, bar);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kPairStages; ++i)
+                        if (i == npend) {
+                            pend_b[i] = f_xfrag + (size_t)kb0 * 16 * MM;
+                            pend_e[i] = f_xmeta + f_cur.kc * 4;
+                            pend_nb[i] = (unsigned)n * kBStride;
+                        }
+                }
             }
+            if (!dep_ok) ++npend;
             ++issued;
             if (++f_h * kPairStageKB >= f_cur.nkb) {
                 f_h = 0;
@@ -367,6 +394,16 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
         }
     };
     fill();
+    dep_wait();
+    dep_ok = true;
+    if (lane == 0)
+#pragma unroll
+        for (int i = 0; i < kPairStages; ++i)
+            if (i < npend) {
+                unsigned char *dst = ring + i * kStageAll;
+                bulk_copy(dst + kA, pend_b[i], pend_nb[i], &rbar[warp][i]);
+                bulk_copy(dst + kA + kB, pend_e[i], 16u, &rbar[warp][i]);
+            }
 
     // ---- consumer
     int c_layer = -1, c_r16 = 1, c_npaths = 1;
@@ -416,8 +453,8 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
             if (prb != lane_p || !lane_live) continue;
             const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
             const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
-            if (Tlo) atomicAdd(c_acc + (size_t)(row0 + g) * 16 + lane_m, (double)Tlo * lane_sc);
-            if (Thi) atomicAdd(c_acc + (size_t)(row0 + g + 8) * 16 + lane_m, (double)Thi * lane_sc);
+            if (Tlo) atomicAdd(c_acc + (size_t)(row0 + g) * MM + lane_m, (double)Tlo * lane_sc);
+            if (Thi) atomicAdd(c_acc + (size_t)(row0 + g + 8) * MM + lane_m, (double)Thi * lane_sc);
         }
     }
 }
@@ -458,11 +495,16 @@ __global__ void __launch_bounds__(NW * 32, 1)
     }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     __syncthreads();
+    dep_release();
 
     const int gw = warp * gridDim.x + blockIdx.x;     // an SM's warps take ranges spread over the whole batch
     const int u0 = wrange[gw], u1 = wrange[gw + 1];
     if (u0 >= u1) return;
     const uint64_t pol = l2_evict_first();
+    // U tiles and h do not depend on the previous kernel; the zl fragments do: a layer's B
+    // slot wanted before dep_wait() is filled afterwards (at most one: the first layer)
+    bool dep_ok = false;
+    int pend_layer = -1;
 
     // ---- fill cursor (position: unit f_u, k-block f_kb within it)
     int f_u = u0, f_kb = 0, f_layer = -1, f_cs = -1, issued = 0, consumed = 0, c_cs = -1;
@@ -474,7 +516,8 @@ __global__ void __launch_bounds__(NW * 32, 1)
                 if (f_cs >= c_cs + 1) return;           // both B slots still in use
                 ++f_cs;
                 f_layer = f_cur.layer;
-                if (lane == 0) {
+                if (!dep_ok) pend_layer = f_layer;
+                else if (lane == 0) {
                     const LayerDev *fd = layers + f_layer;
                     unsigned char *dst = bslot + (f_cs & 1) * kBSlot;
                     uint64_t *bar = &bbar[warp][f_cs & 1];
@@ -510,6 +553,16 @@ __global__ void __launch_bounds__(NW * 32, 1)
         }
     };
     fill();
+    dep_wait();
+    dep_ok = true;
+    if (pend_layer >= 0 && lane == 0) {
+        const LayerDev *fd = layers + pend_layer;
+        uint64_t *bar = &bbar[warp][0];
+        const unsigned fb = (unsigned)fd->KB2 * kBStride;
+        expect_tx(bar, fb + (unsigned)kPairMeta2);
+        bulk_copy(bslot, fd->zfrag, fb, bar);
+        bulk_copy(bslot + kBFrag, fd->zmeta, (unsigned)kPairMeta2, bar);
+    }
 
     int c_layer = -1, N = 0, npaths = 1;
     float *y = nullptr;
@@ -618,10 +671,29 @@ __global__ void __launch_bounds__(NW * 32, 1)
 // Host side
 // ---------------------------------------------------------------------------
 static int g_pair_smem1[2];          // dynamic shared memory attribute set so far, per MM
+
+// Launch that may overlap the previous kernel of the stream (programmatic stream
+// serialisation; the kernel waits with dep_wait() before using its results).
+template <typename... P, typename... A>
+static cudaError_t launch_dependent(bool pdl, void (*kernel)(P...), dim3 grid, dim3 block, size_t smem,
+                                   cudaStream_t s, A &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
 static int g_pair_smem2[2][5];       // per MM and contraction-2 warp count (16, 12, 8, 6, 4)
 
 template <int MM, int NW>
-static cudaError_t launch_c2(int grid, size_t smem, cudaStream_t s, int slot, const LayerDev *dev_layers,
+static cudaError_t launch_c2(bool pdl, int grid, size_t smem, cudaStream_t s, int slot, const LayerDev *dev_layers,
                              const PairUnit2 *u2, const int *wr2, const IoPtrs &io, int base, int M, int kb2max, int *err)
 {
     cudaError_t e;
@@ -631,8 +703,8 @@ static cudaError_t launch_c2(int grid, size_t smem, cudaStream_t s, int slot, co
             return e;
         g_pair_smem2[MM - 1][slot] = (int)smem;
     }
-    contraction2_pair_kernel<MM, NW><<<grid, NW * 32, smem, s>>>(dev_layers, u2, wr2, io, base, M, kb2max, err);
-    return cudaGetLastError();
+    return launch_dependent(pdl, contraction2_pair_kernel<MM, NW>, dim3(grid), dim3(NW * 32), smem, s, dev_layers, u2,
+                            wr2, io, base, M, kb2max, err);
 }
 
 template <int MM>
@@ -661,19 +733,26 @@ static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P
         ++*launches;
         if (mark) profile_mark(*launches, s);
     }
-    contraction1_pair_kernel<MM><<<pair_warps / kPairWarps, kPairWarps * 32, smem1, s>>>(dev_layers, u1, wr1, M, err);
+    // the three kernels after the quantisation may each start while the previous one drains,
+    // unless timing events separate the launches
+    const bool pdl = !profiling_active();
+    if ((e = launch_dependent(pdl, contraction1_pair_kernel<MM>, dim3(pair_warps / kPairWarps), dim3(kPairWarps * 32),
+                              smem1, s, dev_layers, u1, wr1, M, err)) != cudaSuccess)
+        return status_from(e);
     ++*launches;
     if (mark) profile_mark(*launches, s);
-    finish_pair_kernel<MM><<<nlayers, kFinishThreads, (size_t)2 * rmax * MM * sizeof(float), s>>>(dev_layers, base, M);
+    if ((e = launch_dependent(pdl, finish_pair_kernel<MM>, dim3(nlayers), dim3(kFinishThreads),
+                              (size_t)2 * rmax * MM * sizeof(float), s, dev_layers, base, M)) != cudaSuccess)
+        return status_from(e);
     ++*launches;
     if (mark) profile_mark(*launches, s);
     const int grid2 = pair_warps2 / nw2;
     switch (nw2) {
-    case 16: e = launch_c2<MM, 16>(grid2, smem2, s, 0, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
-    case 12: e = launch_c2<MM, 12>(grid2, smem2, s, 1, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
-    case 8: e = launch_c2<MM, 8>(grid2, smem2, s, 2, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
-    case 6: e = launch_c2<MM, 6>(grid2, smem2, s, 3, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
-    default: e = launch_c2<MM, 4>(grid2, smem2, s, 4, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
+    case 16: e = launch_c2<MM, 16>(pdl, grid2, smem2, s, 0, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
+    case 12: e = launch_c2<MM, 12>(pdl, grid2, smem2, s, 1, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
+    case 8: e = launch_c2<MM, 8>(pdl, grid2, smem2, s, 2, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
+    case 6: e = launch_c2<MM, 6>(pdl, grid2, smem2, s, 3, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
+    default: e = launch_c2<MM, 4>(pdl, grid2, smem2, s, 4, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
     }
     if (e != cudaSuccess) return status_from(e);
     ++*launches;

@@ -98,7 +98,8 @@ struct LayerDev {
     const __half *h;    // [npaths][N64], zero padded
     const __half *l;    // [npaths][r16], zero padded
     // scratch (owned by the plan that holds this descriptor):
-    //   acc:  [R1][16] double  sum over k of b * t (contraction-1 rows x activation rows)
+    //   acc:  [R1][16] double  sum over k of b * t (contraction-1 rows x activation rows; the
+    //                           one/two-row kernels use the first R1 * M doubles as [R1][M])
     //         [2][16]  double  sum over k of t (per path x activation row)
     //         [2][16]  int     non-finite flags (per path x activation row)
     //   zfrag [kMaxNT][KB2][32] B fragments of contraction 2, zmeta [2][16] (exponent, digit sum)
@@ -187,6 +188,8 @@ lb_status status_from(cudaError_t e);
 void set_launch_count(int n);
 // Timing hook: record the registered event `i` (if any) on stream s.
 void profile_mark(int i, cudaStream_t s);
+// Whether timing events are registered (launches then stay strictly serialised).
+bool profiling_active();
 
 }  // namespace lb
 

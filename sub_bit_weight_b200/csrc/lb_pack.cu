@@ -21,6 +21,8 @@ void profile_mark(int i, cudaStream_t s)
     if (i >= 0 && i < g_prof_n && g_prof_events[i]) cudaEventRecord(g_prof_events[i], s);
 }
 
+bool profiling_active() { return g_prof_n > 0; }
+
 lb_status status_from(cudaError_t e)
 {
     if (e == cudaSuccess) return LB_OK;
