@@ -282,29 +282,32 @@ static __device__ __forceinline__ void mma_run(int (&a4)[4][4], uint32_t src, ui
     }
 }
 
+// n (1..kPairStageKB) k-blocks: a full stage in one unrolled body, otherwise the
+// binary decomposition of n (at most four unrolled bodies, no jump table).
 template <int MM>
 static __device__ __forceinline__ void mma_stage(int (&a4)[4][4], uint32_t src, uint32_t bsrc, int n)
 {
-    static_assert(kPairStageKB == 16, "one case per segment length");
-    switch (n) {
-    case 16: mma_run<MM, 16>(a4, src, bsrc); break;
-    case 15: mma_run<MM, 15>(a4, src, bsrc); break;
-    case 14: mma_run<MM, 14>(a4, src, bsrc); break;
-    case 13: mma_run<MM, 13>(a4, src, bsrc); break;
-    case 12: mma_run<MM, 12>(a4, src, bsrc); break;
-    case 11: mma_run<MM, 11>(a4, src, bsrc); break;
-    case 10: mma_run<MM, 10>(a4, src, bsrc); break;
-    case 9: mma_run<MM, 9>(a4, src, bsrc); break;
-    case 8: mma_run<MM, 8>(a4, src, bsrc); break;
-    case 7: mma_run<MM, 7>(a4, src, bsrc); break;
-    case 6: mma_run<MM, 6>(a4, src, bsrc); break;
-    case 5: mma_run<MM, 5>(a4, src, bsrc); break;
-    case 4: mma_run<MM, 4>(a4, src, bsrc); break;
-    case 3: mma_run<MM, 3>(a4, src, bsrc); break;
-    case 2: mma_run<MM, 2>(a4, src, bsrc); break;
-    case 1: mma_run<MM, 1>(a4, src, bsrc); break;
-    default: break;
+    static_assert(kPairStageKB == 16, "stage of 16 k-blocks");
+    if (n == 16) {
+        mma_run<MM, 16>(a4, src, bsrc);
+        return;
     }
+    if (n & 8) {
+        mma_run<MM, 8>(a4, src, bsrc);
+        src += 8 * 256;
+        bsrc += 8 * (16 * MM * 8);
+    }
+    if (n & 4) {
+        mma_run<MM, 4>(a4, src, bsrc);
+        src += 4 * 256;
+        bsrc += 4 * (16 * MM * 8);
+    }
+    if (n & 2) {
+        mma_run<MM, 2>(a4, src, bsrc);
+        src += 2 * 256;
+        bsrc += 2 * (16 * MM * 8);
+    }
+    if (n & 1) mma_run<MM, 1>(a4, src, bsrc);
 }
 
 // ---------------------------------------------------------------------------
