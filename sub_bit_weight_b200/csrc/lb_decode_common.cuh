@@ -167,6 +167,34 @@ static __device__ __forceinline__ void bulk_copy_hint(void *dst, const void *src
         : "memory");
 }
 
+// One thread's bookkeeping without a divergent branch: `lead` (non-zero in one
+// lane) announces `tx` bytes on `bar` and starts a bulk copy of `bytes` into it
+// (evict-first L2 policy), all as predicated instructions.
+static __device__ __forceinline__ void lead_fill_hint(uint32_t lead, uint64_t *bar, unsigned tx, void *dst,
+                                                      const void *src, unsigned bytes, uint64_t pol)
+{
+    asm volatile("{\n.reg .pred p;\n.reg .b64 st;\nsetp.ne.u32 p, %0, 0;\n"
+                 "@p mbarrier.arrive.expect_tx.shared::cta.b64 st, [%1], %2;\n"
+                 "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%3], [%4], %5, [%1], %6;\n"
+                 "}\n" ::"r"(lead),
+                 "r"(sm_addr(bar)), "r"(tx), "r"(sm_addr(dst)), "l"(src), "r"(bytes), "l"(pol)
+                 : "memory");
+}
+
+// A further bulk copy on `bar` by the leading lane (bytes already announced).
+static __device__ __forceinline__ void lead_copy(uint32_t lead, uint64_t *bar, void *dst, const void *src,
+                                                 unsigned bytes)
+{
+    asm volatile("{\n.reg .pred p;\nsetp.ne.u32 p, %0, 0;\n"
+                 "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%1], [%2], %3, [%4];\n"
+                 "}\n" ::"r"(lead),
+                 "r"(sm_addr(dst)), "l"(src), "r"(bytes), "r"(sm_addr(bar))
+                 : "memory");
+}
+
+// Generic-proxy reads of a ring stage are ordered before the async-proxy copy that refills it.
+static __device__ __forceinline__ void proxy_fence() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
 static __device__ __forceinline__ void expect_tx(uint64_t *bar, unsigned bytes)
 {
     asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(sm_addr(bar)),

@@ -366,16 +366,17 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
                 f_xmeta = layers[f_layer].xmeta;
             }
             const int n = min(kPairStageKB, f_cur.nkb - f_h * kPairStageKB);
-            if (lane == 0) {
+            {
                 const int st = issued % kPairStages;
                 unsigned char *dst = ring + st * kStageAll;
                 uint64_t *bar = &rbar[warp][st];
                 const int kb0 = f_cur.kc * kP1ChunkKB + f_h * kPairStageKB;
-                expect_tx(bar, (unsigned)n * (256u + kBStride) + 16u);
-                bulk_copy_hint(dst, f_cur.a + (size_t)f_h * kPairStageKB * 32, (unsigned)n * 256u, bar, pol);
+                const uint32_t lead = lane == 0;
+                lead_fill_hint(lead, bar, (unsigned)n * (256u + kBStride) + 16u, dst,
+                               f_cur.a + (size_t)f_h * kPairStageKB * 32, (unsigned)n * 256u, pol);
                 if (dep_ok) {
-                    bulk_copy(dst + kA, f_xfrag + (size_t)kb0 * 16 * MM, (unsigned)n * kBStride, bar);
-                    bulk_copy(dst + kA + kB, f_xmeta + f_cur.kc * 4, 16u, bar);
+                    lead_copy(lead, bar, dst + kA, f_xfrag + (size_t)kb0 * 16 * MM, (unsigned)n * kBStride);
+                    lead_copy(lead, bar, dst + kA + kB, f_xmeta + f_cur.kc * 4, 16u);
                 } else {
 #pragma unroll
                     for (int i = 0; i < kPairStages; ++i)
@@ -444,7 +445,7 @@ __global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
             mma_stage<MM>(a4, sbase + lane * 8, real ? sbase + kA + lane * 8 : zaddr,
                           min(kPairStageKB, cu.nkb - h * kPairStageKB));
             __syncwarp();
-            if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+            proxy_fence();
             ++consumed;
             fill();
         }
@@ -646,7 +647,7 @@ __global__ void __launch_bounds__(NW * 32, 1)
             s_addr += (uint32_t)seg * 256u;
             if (s_left == 0) {
                 __syncwarp();
-                if (lane == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                if (lane == 0) proxy_fence();
                 ++consumed;
                 fill();
             }
