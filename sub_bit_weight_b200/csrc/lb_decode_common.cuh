@@ -84,24 +84,10 @@ static __device__ __forceinline__ uint2 lds64(uint32_t addr)
     return v;
 }
 
-static __device__ __forceinline__ unsigned short lds_u16(uint32_t addr)
-{
-    unsigned short v;
-    asm volatile("ld.shared.u16 %0, [%1];\n" : "=h"(v) : "r"(addr));
-    return v;
-}
-
 static __device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
 {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(addr));
-    return v;
-}
-
-static __device__ __forceinline__ float lds_f32(uint32_t addr)
-{
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(v) : "r"(addr));
     return v;
 }
 

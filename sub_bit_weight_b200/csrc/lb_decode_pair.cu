@@ -32,12 +32,6 @@
 
 namespace lb {
 
-// Lane of column (m, path, digit) holding activation index kk of a k-block.
-static __device__ __forceinline__ int pair_lane(int m, int p, int d, int kk)
-{
-    return ((4 * m + 2 * p + d) << 2) + ((kk & 15) >> 2);
-}
-
 // ---------------------------------------------------------------------------
 // Activation quantisation: one warp per 1024-input chunk, lane L takes k-block
 // L of the chunk (32 inputs) and writes that k-block's whole B fragment.

@@ -43,8 +43,6 @@ constexpr int kIoBatch = 1024;          // layers per launch (pointer tables rid
 constexpr int kP1StageKB = 8;           // k-blocks per ring stage, contraction 1 (2 KB)
 constexpr int kP1Stages = 3;            // per-warp bulk-copy ring depth, contraction 1
 constexpr int kP2Stages = 2;            // per-warp bulk-copy ring depth, contraction 2 (one row group per stage)
-constexpr int kP2StageKB = 8;           // path-merged contraction 2: k-blocks per ring stage (2 KB)
-constexpr int kP2PairStages = 3;        // path-merged contraction 2: per-warp ring depth
 
 // Warp-streaming kernels for one or two activation rows.  Every warp owns an
 // equal contiguous share of the bytes a contraction streams (fixed at plan
@@ -210,16 +208,6 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Streamed once: read-only path, no L1 allocation.
-__device__ __forceinline__ uint2 ld_stream_u2(const uint2 *p)
-{
-    uint2 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];\n"
-                 : "=r"(v.x), "=r"(v.y)
-                 : "l"(p));
-    return v;
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b)
