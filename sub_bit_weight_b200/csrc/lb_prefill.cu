@@ -363,7 +363,7 @@ struct PfSmem {
 };
 
 template <int MODE>
-__global__ void __launch_bounds__(kPfThreads, 1)
+__global__ void __launch_bounds__(pf_threads(MODE), 1)
     prefill_kernel(const PfLayer *__restrict__ layers, const int *__restrict__ tile_start, int nlayers, int M,
                    int *err)
 {
@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < kPfStages; ++s) {
             mbar_init(&S.full[s], 1);
-            mbar_init(&S.ready[s], MODE == 0 ? 10 : 8);   // generator warps (+ converter warps)
+            mbar_init(&S.ready[s], MODE == 0 ? 10 + kPfExtraConv : 8);   // generator warps (+ converter warps)
             mbar_init(&S.bread[s], 8);                    // generator warps have read the stage's sign bits
             mbar_init(&S.empty[s], 1);
         }
@@ -479,10 +479,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 tc_commit(&S.accf[ab]);
             }
         }
-    } else if (warp == 2 || warp == 3) {
+    } else if (warp == 2 || warp == 3 || warp >= 16) {
         // ---------------- converters (latent GEMM): bf16 -> fp16 A tile in place
         if (MODE == 0) {
-            const int ct = tid - 64;   // 0..63
+            constexpr int kConv = 32 * (2 + kPfExtraConv);
+            const int ct = warp < 16 ? tid - 64 : tid - 512 + 64;   // 0 .. kConv - 1
             uint32_t it = 0;
             for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
                 int L, mt, nt;
@@ -496,15 +497,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         ok = false;
                         break;
                     }
-                    const uint32_t A4 = smem_u32(S.A[s]) + 16u * ct;
-#pragma unroll 4
-                    for (int i = 0; i < kPfBM * kPfBK * 2 / 16 / 64; ++i) {
-                        uint4 v = lds128(A4 + 1024u * i);
+                    const uint32_t A0 = smem_u32(S.A[s]);
+#pragma unroll 2
+                    for (int i = ct; i < kPfBM * kPfBK * 2 / 16; i += kConv) {
+                        uint4 v = lds128(A0 + 16u * i);
                         v.x = bf16x2_to_f16x2(v.x);
                         v.y = bf16x2_to_f16x2(v.y);
                         v.z = bf16x2_to_f16x2(v.z);
                         v.w = bf16x2_to_f16x2(v.w);
-                        sts128(A4 + 1024u * i, v);
+                        sts128(A0 + 16u * i, v);
                     }
                     fence_proxy_async();
                     __syncwarp();
@@ -884,9 +885,10 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
     }
     const int g0 = std::max(1, std::min(st.tiles[0], sms));
     const int g1 = std::max(1, std::min(st.tiles[1], sms));
-    prefill_kernel<0><<<g0, kPfThreads, smem, s>>>(st.rec, st.starts, n, M, st.err);
+    profile_mark(0, s);
+    prefill_kernel<0><<<g0, pf_threads(0), smem, s>>>(st.rec, st.starts, n, M, st.err);
     profile_mark(++*launches, s);
-    prefill_kernel<1><<<g1, kPfThreads, smem, s>>>(st.rec + n, st.starts + n + 1, n, M, st.err);
+    prefill_kernel<1><<<g1, pf_threads(1), smem, s>>>(st.rec + n, st.starts + n + 1, n, M, st.err);
     profile_mark(++*launches, s);
     return status_from(cudaGetLastError());
 }

@@ -11,7 +11,9 @@ constexpr int kPfBM = 128;          // activation rows per tile (UMMA M)
 constexpr int kPfBN = 256;          // output columns per tile (UMMA N, at most)
 constexpr int kPfBK = 64;           // contraction depth per pipeline stage (one 128-byte swizzle atom of fp16)
 constexpr int kPfStages = 4;
-constexpr int kPfThreads = 512;     // 16 warps: producer, MMA, 4 epilogue, 8 generator warps
+constexpr int kPfThreads = 512;     // 16 warps: producer, MMA, 2 converters, 4 epilogue, 8 generator warps
+constexpr int kPfExtraConv = 4;     // latent GEMM: converter warps 16.. beyond the 16
+__host__ __device__ constexpr int pf_threads(int mode) { return kPfThreads + (mode == 0 ? 32 * kPfExtraConv : 0); }
 
 cudaError_t prefill_build_weights(PfWeights &W, const LayerDev &d, const uint32_t *const *U,
                                   const uint32_t *const *V, const uint16_t *const *h,
