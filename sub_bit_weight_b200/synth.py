@@ -215,3 +215,24 @@ def layer_inputs(seed: int, layer: int, shape: LayerShape, npaths: int = 2) -> d
         out["g"].append(scale_vector(seed, layer, p, "g", K))
         out["l"].append(scale_vector(seed, layer, p, "l", r))
     return out
+
+
+def dense_weight(seed: int, N: int, K: int, alpha: float = 1.0, rms: float = 0.02) -> np.ndarray:
+    """Synthetic dense weight W [N, K] (float32 holding bfloat16 values) with a power-law spectrum.
+
+    ``W = A diag(s) B`` with A [N, R], B [R, K] i.i.d. N(0, 1) in float32
+    (``R = min(N, K)``, from ``default_rng([seed, N, K, 0x5D])``, A drawn
+    first) and ``s_i = (i + 1) ** -alpha``; scaled so that the RMS entry is
+    ``rms`` (the magnitude of LLM projection weights) and rounded to bfloat16
+    (nearest even), the storage type of such weights.  The decaying spectrum
+    stands for the low-rank structure of LLM weight matrices that the
+    factorisation relies on.
+    """
+    rng = np.random.default_rng([seed, N, K, 0x5D])
+    R = min(N, K)
+    A = rng.standard_normal((N, R), dtype=np.float32)
+    B = rng.standard_normal((R, K), dtype=np.float32)
+    s = (np.arange(1, R + 1, dtype=np.float64) ** -float(alpha)).astype(np.float32)
+    W = (A * s[None, :]) @ B
+    W *= np.float32(rms / np.sqrt(np.mean(np.square(W, dtype=np.float64))))
+    return bf16_bits_to_f32(f32_to_bf16_bits(W))
