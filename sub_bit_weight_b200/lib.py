@@ -57,6 +57,8 @@ _sig("lb_profile_events", _st, [ctypes.POINTER(_vp), _i])
 _sig("lb_stack_status", _st, [_vp, _vp])
 _sig("lb_layer_status", _st, [_vp, _vp])
 _sig("lb_selftest_wait_timeout", _st, [ctypes.c_longlong, _vp])
+_sig("lb_dual_svid_workspace_bytes", ctypes.c_size_t, [_i, _i, _i])
+_sig("lb_dual_svid_init", _st, [_vp, _i, _i, _i, _i, _i] + [ctypes.POINTER(_vp)] * 5 + [_vp, _vp, ctypes.c_size_t, _vp])
 
 
 class LittleBitError(RuntimeError):
@@ -262,3 +264,57 @@ def lb_stack_forward(stack: Stack, xs=None, ys=None, stream=None, io: StackIO | 
         io = StackIO(stack, xs, ys)
     _check(_lib.lb_stack_forward(stack.handle, io.xp, io.yp, io.M, _stream(stream)), "lb_stack_forward")
     return io
+
+
+# ---------------------------------------------------------------------------
+# Initialisation: Dual-SVID + residual compensation (include/littlebit_init.h)
+# ---------------------------------------------------------------------------
+
+def lb_dual_svid_workspace_bytes(N: int, K: int, r: int) -> int:
+    return int(_lib.lb_dual_svid_workspace_bytes(N, K, r))
+
+
+class DualSvidResult:
+    """Per-path outputs of ``lb_dual_svid_init``: packed signs (int32 bit patterns) and float32 scales."""
+
+    def __init__(self, U, V, h, g, l, sigma):
+        self.U, self.V, self.h, self.g, self.l, self.sigma = U, V, h, g, l, sigma
+
+    def layer_args(self):
+        """(U, V, h, g, l) lists for lb_layer_create, the scales rounded to binary16."""
+        return self.U, self.V, [x.half() for x in self.h], [x.half() for x in self.g], [x.half() for x in self.l]
+
+
+def lb_dual_svid_init(W: torch.Tensor, r: int, npaths: int = 2, iters: int = 24, workspace: torch.Tensor | None = None,
+                      stream=None) -> DualSvidResult:
+    """Dual-SVID (+ residual) initialisation of a LittleBit layer from a dense float32 W [N, K] (CUDA).
+
+    Allocates the outputs (and the workspace unless one is passed: a uint8 CUDA tensor of at least
+    ``lb_dual_svid_workspace_bytes(N, K, r)`` bytes).  The call waits for its stream.
+    """
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D [N, K]")
+    N, K = W.shape
+    need = lb_dual_svid_workspace_bytes(N, K, r)
+    if need == 0:
+        raise ValueError(f"invalid shape N={N} K={K} r={r}")
+    dev = W.device
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    wpr = (r + 31) // 32
+    U = [torch.empty((N, wpr), dtype=torch.int32, device=dev) for _ in range(npaths)]
+    V = [torch.empty((K, wpr), dtype=torch.int32, device=dev) for _ in range(npaths)]
+    h = [torch.empty(N, dtype=torch.float32, device=dev) for _ in range(npaths)]
+    g = [torch.empty(K, dtype=torch.float32, device=dev) for _ in range(npaths)]
+    l = [torch.empty(r, dtype=torch.float32, device=dev) for _ in range(npaths)]
+    sigma = torch.empty((npaths, r), dtype=torch.float32, device=dev)
+
+    def arr(lst, dtype, name):
+        return (_vp * max(1, len(lst)))(*[_dev(t, dtype, f"{name}[{p}]") for p, t in enumerate(lst)])
+
+    _check(_lib.lb_dual_svid_init(_dev(W, torch.float32, "W"), N, K, r, npaths, iters,
+                                  arr(U, torch.int32, "U"), arr(V, torch.int32, "V"), arr(h, torch.float32, "h"),
+                                  arr(g, torch.float32, "g"), arr(l, torch.float32, "l"),
+                                  _dev(sigma, torch.float32, "sigma"), _dev(workspace, torch.uint8, "workspace"),
+                                  workspace.numel(), _stream(stream)), "lb_dual_svid_init")
+    return DualSvidResult(U, V, h, g, l, sigma)

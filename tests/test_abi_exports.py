@@ -11,7 +11,8 @@ import re
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "littlebit.h")
+INCLUDE = os.path.join(ROOT, "include")
+HEADERS = sorted(os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h"))
 
 
 @pytest.fixture(scope="module")
@@ -22,15 +23,18 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(lb_[a-z0-9_]+)\s*\(", text)))
+    names = set()
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names.update(re.findall(r"\b(lb_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("lb_pack_signs", "lb_layer_create", "lb_linear_forward", "lb_layer_destroy",
-                     "lb_stack_create", "lb_stack_forward", "lb_stack_destroy", "lb_layer_bpw"):
+                     "lb_stack_create", "lb_stack_forward", "lb_stack_destroy", "lb_layer_bpw",
+                     "lb_dual_svid_workspace_bytes", "lb_dual_svid_init"):
         assert required in names
 
 
@@ -74,3 +78,24 @@ def test_host_side_argument_checks(lib):
     lib.lb_layer_destroy(None)
     lib.lb_stack_destroy.argtypes = [vp]
     lib.lb_stack_destroy(None)
+
+
+def test_initialisation_argument_checks(lib):
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.lb_dual_svid_workspace_bytes.restype = ctypes.c_size_t
+    lib.lb_dual_svid_workspace_bytes.argtypes = [i, i, i]
+    assert lib.lb_dual_svid_workspace_bytes(8, 8, 9) == 0          # r above min(N, K)
+    assert lib.lb_dual_svid_workspace_bytes(0, 8, 1) == 0
+    ws = lib.lb_dual_svid_workspace_bytes(96, 40, 6)
+    assert ws > 96 * 40 * 8
+    lib.lb_dual_svid_init.argtypes = [vp, i, i, i, i, i] + [ctypes.POINTER(vp)] * 5 + [vp, vp, ctypes.c_size_t, vp]
+    one = (vp * 1)(vp(256))
+    args = [one] * 5
+    assert lib.lb_dual_svid_init(vp(256), 96, 40, 6, 3, 24, *args, None, vp(256), ws, None) == 2   # npaths
+    assert lib.lb_dual_svid_init(None, 96, 40, 6, 1, 24, *args, None, vp(256), ws, None) == 1      # W
+    assert lib.lb_dual_svid_init(vp(256), 96, 40, 41, 1, 24, *args, None, vp(256), ws, None) == 1  # rank
+    assert lib.lb_dual_svid_init(vp(256), 96, 40, 6, 1, -1, *args, None, vp(256), ws, None) == 1   # iters
+    assert lib.lb_dual_svid_init(vp(256), 96, 40, 6, 1, 24, *args, None, vp(256), ws - 8, None) == 1   # small
+    assert lib.lb_dual_svid_init(vp(256), 96, 40, 6, 1, 24, *args, None, vp(264), ws, None) == 1   # misaligned
+    nulls = (vp * 1)(None)
+    assert lib.lb_dual_svid_init(vp(256), 96, 40, 6, 1, 24, nulls, *args[1:], None, vp(256), ws, None) == 1
