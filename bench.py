@@ -37,6 +37,10 @@ from sub_bit_weight_b200 import synth  # noqa: E402
 METRIC = "LittleBit linear decode GB/s & prefill TFLOP/s, % of B200 roofline"
 DECODE_DEFAULT = "llama2_70b_0.1"
 PREFILL_DEFAULT = "llama2_13b_0.3_prefill"
+INIT_DEFAULT = "llama2_7b_0.1"
+INIT_ITERS = 24
+# binary64 FMA rate of B200: 148 SMs x 64 FP64 FMA per clock x 2 FLOP at the 1965 MHz maximum SM clock
+FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
 
 
 def peaks():
@@ -310,6 +314,9 @@ def main():
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--blocks", type=int, default=None, help="only the first N blocks of the stack (profiling)")
+    ap.add_argument("--init", default=INIT_DEFAULT,
+                    help="workload whose first block gets the Dual-SVID + residual initialisation ('' = skip)")
+    ap.add_argument("--init-steps", type=int, default=2)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -424,6 +431,9 @@ def main():
                                         "traffic": prefill_traffic(pw.key)},
                            "clocks": pres["clocks"]}
 
+    if args.init and world == 1:
+        line["init"] = run_init(args.init, args.init_steps, 3, dev, args.cpu_seconds > 0)
+
     if rank == 0 and args.cpu_seconds > 0:
         cs = oracle_sample(w, M, args.cpu_seconds)
         cv = (cs["flops"] / cs["seconds"] / 1e12) if prefill_main else (cs["bytes"] / cs["seconds"] / 1e9)
@@ -436,6 +446,93 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line))
+
+
+def subspace_width(s: synth.LayerShape) -> int:
+    """Columns of the subspace the initialisation iterates (include/littlebit_init.h)."""
+    return min(min(s.N, s.K), max(64, -(-2 * s.r // 64) * 64))
+
+
+def run_init(wkey: str, steps: int, warmup: int, dev, with_cpu: bool):
+    """Dual-SVID + residual initialisation of every layer of one block of a workload, from synthetic dense W.
+
+    One step = both paths of all layers of the block (lb_dual_svid_init, binary64, INIT_ITERS iterations).  The
+    dominant kernel is the binary64 GEMM of the subspace iteration; its launches are timed with the library's
+    event hook on the largest layer.
+    """
+    import torch
+    from sub_bit_weight_b200 import lib
+    w = synth.WORKLOADS[wkey]
+    shapes = list(w.block)
+    Ws = {}
+    for s in shapes:        # one synthetic W per distinct shape (the work per layer does not depend on the values)
+        if (s.N, s.K) not in Ws:
+            Ws[(s.N, s.K)] = torch.from_numpy(synth.dense_weight(w.seed, s.N, s.K)).to(dev)
+    ws = torch.empty(max(lib.lb_dual_svid_workspace_bytes(s.N, s.K, s.r) for s in shapes), dtype=torch.uint8,
+                     device=dev)
+
+    def block():
+        for s in shapes:
+            lib.lb_dual_svid_init(Ws[(s.N, s.K)], s.r, 2, INIT_ITERS, workspace=ws)
+
+    for _ in range(warmup):
+        block()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record()
+        for _ in range(steps):
+            block()
+        e1.record()
+        torch.cuda.synchronize()
+    ms_block = e0.elapsed_time(e1) / steps
+    # the dominant kernel: the two products of the first subspace iteration of the largest layer
+    big = max(shapes, key=lambda s: s.N * s.K * subspace_width(s))
+    Lb = subspace_width(big)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for e in ev:             # torch creates the CUDA event on first record
+        e.record()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(3):
+        lib.lb_profile_events(ev)
+        lib.lb_dual_svid_init(Ws[(big.N, big.K)], big.r, 2, INIT_ITERS, workspace=ws)
+        lib.lb_profile_events([])
+        times += [ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2])]
+    gemm_ms = statistics.median(times)
+    gemm_flops = 2.0 * big.N * big.K * Lb
+    ach = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    # iteration products per layer and path: iters x 2 + the Rayleigh-Ritz product, each 2 N K L
+    it_flops = sum(2 * (2 * INIT_ITERS + 1) * 2.0 * s.N * s.K * subspace_width(s) for s in shapes)
+    out = {"workload": f"{w.key} first block: " + ", ".join(f"{s.name} {s.N}x{s.K} r={s.r}" for s in shapes)
+                       + f"; dense W synthetic (power-law spectrum s_i ~ 1/i, bf16 values); two paths, "
+                         f"{INIT_ITERS} subspace iterations, binary64",
+           "value": round(len(shapes) / (ms_block * 1e-3), 3), "unit": "layers/s", "higher_is_better": True,
+           "ms_per_block": round(ms_block, 2), "steps": steps, "warmup": warmup,
+           "iteration_gemm_tflops": round(it_flops / (ms_block * 1e-3) / 1e12, 2),
+           "roofline": {"bound": "alu", "kernel": f"dgemm_kernel (W^T (W Q) products, {big.name} {big.N}x{big.K}, "
+                                                  f"L={Lb})",
+                        "achieved": round(ach, 2), "peak": round(FP64_PEAK_TFLOPS, 1), "unit": "TFLOP/s",
+                        "frac": round(ach / FP64_PEAK_TFLOPS, 4),
+                        "peak_src": "derived: 148 SMs x 64 FP64 FMA/clk x 2 x 1965 MHz (binary64 CUDA-core rate)",
+                        "flops_per_launch": gemm_flops, "ms_per_launch": round(gemm_ms, 4), "traffic": None},
+           "clocks": clk.summary()}
+    if with_cpu:
+        from oracle import dual_svid as ods
+        s = shapes[0]
+        W = Ws[(s.N, s.K)].cpu().numpy().astype(np.float64)
+        t = time.perf_counter()
+        ods.littlebit_init(W, s.r, 2)
+        dt = time.perf_counter() - t
+        try:
+            from threadpoolctl import threadpool_info
+            cores = max((i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"), default=1)
+        except Exception:
+            cores = os.cpu_count()
+        out["cpu_baseline"] = {"value": round(1.0 / dt, 4), "unit": "layers/s", "cores": cores, "kind": "oracle",
+                               "sample": f"one {s.name} layer {s.N}x{s.K} r={s.r}, two paths, numpy/LAPACK "
+                                         f"float64 ({dt:.1f} s)"}
+    return out
 
 
 def reference_arm(args, w, M, world, rank, pk):

@@ -24,8 +24,11 @@
  *     gives zero vectors.
  *
  * All arithmetic is IEEE binary64 on the device.  The truncated SVD is found
- * by randomised subspace iteration (orthonormalised after every product with
- * W or W^T) followed by a Rayleigh-Ritz step with a Jacobi eigensolver, so
+ * by randomised subspace iteration (orthonormalised by Cholesky QR after
+ * every product with W^T W; a column whose part orthogonal to the others
+ * falls below ~3e-7 of its norm is dropped, which only happens when
+ * s_1 / s_L exceeds ~1e3 or W has rank below L) followed by a Rayleigh-Ritz
+ * step with a Jacobi eigensolver, so
  * its accuracy depends on the number of iterations and on the spectrum: the
  * error of the rank-r subspace shrinks like (s_{L+1} / s_r)^(2 iters), with
  * L = min(min(N, K), max(64, 64 * ceil(2r / 64))) columns in the subspace.
@@ -75,7 +78,13 @@ LB_API size_t lb_dual_svid_workspace_bytes(int N, int K, int r);
  * outside {1, 2}.  The work is enqueued on `stream`, and the call then waits
  * for the stream (it is not a hot-path call): LB_ERR_TIMEOUT if a bounded
  * device-side wait of the eigensolver gave up, LB_ERR_CUDA for a CUDA error
- * (including an earlier asynchronous one); the outputs are then undefined. */
+ * (including an earlier asynchronous one); the outputs are then undefined.
+ *
+ * With the timing hook of littlebit.h (lb_profile_events) holding at least 3
+ * events, the primary path's first subspace iteration records events[0]
+ * before the product Z = A Q, events[1] after it and events[2] after the
+ * product A^T Z (A = W if K <= N, else W^T); nothing is recorded when the
+ * subspace is the whole space. */
 LB_API lb_status lb_dual_svid_init(const float *W, int N, int K, int r, int npaths, int iters,
                                    uint32_t *const *U, uint32_t *const *V,
                                    float *const *h, float *const *g, float *const *l, float *sigma,

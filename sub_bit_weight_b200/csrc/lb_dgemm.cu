@@ -5,12 +5,15 @@
 // kernel is the binary64 contraction here.  CTA tile 128 x 64, k-step 16,
 // 256 threads with an 8 x 4 block of C each; operands staged through
 // registers into double-buffered shared memory (one __syncthreads per
-// k-step).  A warp is 4 rows x 8 columns of threads, so every LDS.128 of an
-// operand is one shared-memory wavefront.  Small output grids split k over
-// CTAs and add the partial sums in a fixed order.
+// k-step), fragments double-buffered in registers.  A warp is 4 rows x 8
+// columns of threads, so every LDS.128 of an operand is one shared-memory
+// wavefront, and the staging stores are conflict-free.  Small output grids
+// split k over CTAs (the split that fills whole waves) and add the partial
+// sums in a fixed order.
 #include "lb_linalg.cuh"
 
 #include <algorithm>
+#include <math.h>
 
 namespace lb {
 namespace {
@@ -48,30 +51,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) ra[e] = (gi < m && gk + e < kend) ? A[(long)gi * lda + gk + e] : 0.0;
             }
-        } else {                                     // A is k x m: 8 consecutive rows of one k
-            const int kk = tid >> 4, ms = (tid & 15) * 8, gk = k0 + kk, gi = m0 + ms;
-            if (gk < kend && vec && gi + 8 <= m) {
-                const double2 *src = reinterpret_cast<const double2 *>(A + (long)gk * lda + gi);
+        } else {                                     // A is k x m: rows 2t, 2t+1 (+32e) of one k
+            const int kk = tid >> 4, mo = 2 * (tid & 15), gk = k0 + kk;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const double2 v = src[e];
+            for (int e = 0; e < 4; ++e) {
+                const int gi = m0 + mo + 32 * e;
+                if (gk < kend && vec && gi + 2 <= m) {
+                    const double2 v = *reinterpret_cast<const double2 *>(A + (long)gk * lda + gi);
                     ra[2 * e] = v.x;
                     ra[2 * e + 1] = v.y;
+                } else {
+                    ra[2 * e] = (gk < kend && gi < m) ? A[(long)gk * lda + gi] : 0.0;
+                    ra[2 * e + 1] = (gk < kend && gi + 1 < m) ? A[(long)gk * lda + gi + 1] : 0.0;
                 }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ra[e] = (gk < kend && gi + e < m) ? A[(long)gk * lda + gi + e] : 0.0;
             }
         }
-        if (!TB) {                                   // B is k x n: 4 consecutive columns of one k
-            const int kk = tid >> 4, ns = (tid & 15) * 4, gk = k0 + kk, gj = n0 + ns;
-            if (gk < kend && vec && gj + 4 <= n) {
-                const double2 *src = reinterpret_cast<const double2 *>(B + (long)gk * ldb + gj);
-                const double2 v0 = src[0], v1 = src[1];
-                rb[0] = v0.x; rb[1] = v0.y; rb[2] = v1.x; rb[3] = v1.y;
-            } else {
+        if (!TB) {                                   // B is k x n: columns 2t, 2t+1 (+32e) of one k
+            const int kk = tid >> 4, no = 2 * (tid & 15), gk = k0 + kk;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) rb[e] = (gk < kend && gj + e < n) ? B[(long)gk * ldb + gj + e] : 0.0;
+            for (int e = 0; e < 2; ++e) {
+                const int gj = n0 + no + 32 * e;
+                if (gk < kend && vec && gj + 2 <= n) {
+                    const double2 v = *reinterpret_cast<const double2 *>(B + (long)gk * ldb + gj);
+                    rb[2 * e] = v.x;
+                    rb[2 * e + 1] = v.y;
+                } else {
+                    rb[2 * e] = (gk < kend && gj < n) ? B[(long)gk * ldb + gj] : 0.0;
+                    rb[2 * e + 1] = (gk < kend && gj + 1 < n) ? B[(long)gk * ldb + gj + 1] : 0.0;
+                }
             }
         } else {                                     // B is n x k: 4 consecutive k of one column
             const int col = tid & (BN - 1), ks = (tid >> 6) * 4, gj = n0 + col, gk = k0 + ks;
@@ -92,16 +99,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) As[b][ks + e][row] = ra[e];
         } else {
-            const int kk = tid >> 4, ms = (tid & 15) * 8;
-            double2 *dst = reinterpret_cast<double2 *>(&As[b][kk][ms]);
+            const int kk = tid >> 4, mo = 2 * (tid & 15);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = make_double2(ra[2 * e], ra[2 * e + 1]);
+            for (int e = 0; e < 4; ++e)
+                *reinterpret_cast<double2 *>(&As[b][kk][mo + 32 * e]) = make_double2(ra[2 * e], ra[2 * e + 1]);
         }
         if (!TB) {
-            const int kk = tid >> 4, ns = (tid & 15) * 4;
-            double2 *dst = reinterpret_cast<double2 *>(&Bs[b][kk][ns]);
-            dst[0] = make_double2(rb[0], rb[1]);
-            dst[1] = make_double2(rb[2], rb[3]);
+            const int kk = tid >> 4, no = 2 * (tid & 15);
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                *reinterpret_cast<double2 *>(&Bs[b][kk][no + 32 * e]) = make_double2(rb[2 * e], rb[2 * e + 1]);
         } else {
             const int col = tid & (BN - 1), ks = (tid >> 6) * 4;
 #pragma unroll
@@ -124,16 +131,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int st = 0; st < nsteps; ++st) {
         const int b = st & 1;
         if (st + 1 < nsteps) load(kbeg + (st + 1) * BK);
+        // operand fragments of step kk + 1 are read while step kk's FMAs issue
+        double2 fa[2][4], fb[2][2];
+        auto frag = [&](int s, int kk) {
+            fa[s][0] = *reinterpret_cast<const double2 *>(&As[b][kk][ty * 4]);
+            fa[s][1] = *reinterpret_cast<const double2 *>(&As[b][kk][ty * 4 + 2]);
+            fa[s][2] = *reinterpret_cast<const double2 *>(&As[b][kk][64 + ty * 4]);
+            fa[s][3] = *reinterpret_cast<const double2 *>(&As[b][kk][64 + ty * 4 + 2]);
+            fb[s][0] = *reinterpret_cast<const double2 *>(&Bs[b][kk][tx * 2]);
+            fb[s][1] = *reinterpret_cast<const double2 *>(&Bs[b][kk][32 + tx * 2]);
+        };
+        frag(0, 0);
 #pragma unroll
         for (int kk = 0; kk < BK; ++kk) {
-            const double2 a0 = *reinterpret_cast<const double2 *>(&As[b][kk][ty * 4]);
-            const double2 a1 = *reinterpret_cast<const double2 *>(&As[b][kk][ty * 4 + 2]);
-            const double2 a2 = *reinterpret_cast<const double2 *>(&As[b][kk][64 + ty * 4]);
-            const double2 a3 = *reinterpret_cast<const double2 *>(&As[b][kk][64 + ty * 4 + 2]);
-            const double2 b0 = *reinterpret_cast<const double2 *>(&Bs[b][kk][tx * 2]);
-            const double2 b1 = *reinterpret_cast<const double2 *>(&Bs[b][kk][32 + tx * 2]);
-            const double av[8] = {a0.x, a0.y, a1.x, a1.y, a2.x, a2.y, a3.x, a3.y};
-            const double bv[4] = {b0.x, b0.y, b1.x, b1.y};
+            const int s = kk & 1;
+            if (kk + 1 < BK) frag(s ^ 1, kk + 1);
+            const double av[8] = {fa[s][0].x, fa[s][0].y, fa[s][1].x, fa[s][1].y,
+                                  fa[s][2].x, fa[s][2].y, fa[s][3].x, fa[s][3].y};
+            const double bv[4] = {fb[s][0].x, fb[s][0].y, fb[s][1].x, fb[s][1].y};
 #pragma unroll
             for (int i = 0; i < 8; ++i)
 #pragma unroll
@@ -208,12 +223,21 @@ void dgemm(bool ta, bool tb, int m, int n, int k, double alpha, const double *A,
         return;
     }
     const long tiles = (long)((m + BM - 1) / BM) * ((n + BN - 1) / BN);
+    // split k so that the grid fills whole waves of one CTA per SM (and at most 16 slices of >= 256)
     int S = 1;
-    const long target = 2L * sms;
-    if (part && tiles < target) {
-        S = (int)std::min<long>((target + tiles - 1) / tiles, std::max(1, k / 256));
-        S = std::min(S, 16);
-        while (S > 1 && (size_t)S * m * n > part_elems) --S;
+    if (part && tiles < 4L * sms) {
+        double best = -1.0;
+        const int smax = (int)std::min<long>(16, std::max(1, k / 256));
+        for (int c = 1; c <= smax; ++c) {
+            if ((size_t)c * m * n > part_elems) break;
+            const long ctas = tiles * c;
+            const double waves = (double)ctas / sms;
+            const double eff = waves / std::ceil(waves);     // busy fraction of the SMs over the launch
+            if (eff > best + 0.02) {
+                best = eff;
+                S = c;
+            }
+        }
     }
     int kchunk = ((k + S - 1) / S + BK - 1) / BK * BK;
     S = (k + kchunk - 1) / kchunk;

@@ -8,7 +8,9 @@
 // with J = [[c, s], [-s, c]] on (p, q), (J^T A J)_pq = 0, a_pp -= t a_pq,
 // a_qq += t a_pq.  A rotation is skipped when |a_pq| <= tol sqrt(|a_pp a_qq|)
 // (the threshold that gives eigenvalues to high relative accuracy); the
-// iteration stops after a sweep with no rotation.
+// iteration stops after a sweep whose rotations all had |a_pq| <= 1e-12
+// sqrt(|a_pp a_qq|) (convergence is quadratic, so the next sweep would leave
+// off-diagonal entries of order 1e-24 of the diagonal over the eigenvalue gaps).
 //
 // Parallel ordering: the round-robin ("circle") tournament, n/2 disjoint
 // pairs per round, n-1 rounds per sweep.  Position 0 is fixed, positions
@@ -22,6 +24,7 @@
 // a round needs a single grid-wide barrier; the barrier waits are bounded and
 // report through `err`.
 #include "lb_linalg.cuh"
+#include "lb_coop.cuh"
 
 #include <algorithm>
 #include <math.h>
@@ -31,47 +34,7 @@ namespace {
 
 constexpr int kJThreads = 512;
 constexpr double kJTol = 1e-15;
-constexpr long long kBarrierCycles = 2000000000LL;   // ~1 s at the boost clock
-
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p)
-{
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Grid-wide barrier (all CTAs are co-resident: cooperative launch).  bar[0]
-// counts arrivals, bar[1] is the generation.  False if the wait gave up.
-__device__ bool grid_barrier(unsigned *bar, unsigned &gen, int *err)
-{
-    __shared__ int ok;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int good = 1;
-        const unsigned want = gen + 1;
-        __threadfence();
-        if (atomicAdd(&bar[0], 1u) == gridDim.x - 1) {
-            atomicExch(&bar[0], 0u);
-            __threadfence();
-            atomicExch(&bar[1], want);
-        } else {
-            const long long t0 = clock64();
-            while (ld_acquire_u32(&bar[1]) != want) {
-                if (*(volatile int *)err != 0 || clock64() - t0 > kBarrierCycles) {
-                    atomicCAS(err, 0, 32);
-                    good = 0;
-                    break;
-                }
-                __nanosleep(32);
-            }
-        }
-        gen = want;
-        __threadfence();
-        ok = good;
-    }
-    __syncthreads();
-    return ok != 0;
-}
+constexpr double kJStop = 1e-12;
 
 __device__ __forceinline__ int circle_index(int pos, int t, int np)
 {
@@ -110,10 +73,11 @@ __global__ void __launch_bounds__(kJThreads, 1)
     }
     if (!grid_barrier(bar, gen, err)) return;
 
-    const long blocks = (long)H * H, items = blocks + (long)H * n;
+    const int nblocks = H * H, nvt = H * n;     // 2x2 blocks of A, row-pair entries of Vt (< 2^31 for n <= 4096)
+    const int gt = (int)gtid, gs = (int)gstride;
     int b = 0;
     for (int sweep = 0; sweep < max_sweeps; ++sweep) {
-        int rotated = 0;
+        double worst = 0.0;      // largest |a_pq| / sqrt(|a_pp a_qq|) rotated in this sweep
         for (int t = 0; t < np - 1; ++t) {
             const int tn = (t + 1) % (np - 1);
             const double *dgc = dgs[b], *odc = ods[b];
@@ -129,7 +93,8 @@ __global__ void __launch_bounds__(kJThreads, 1)
                         tt = fabs(tau) > 1e150 ? 0.5 / tau : sg / (fabs(tau) + sqrt(1.0 + tau * tau));
                         c = 1.0 / sqrt(1.0 + tt * tt);
                         s = tt * c;
-                        rotated = 1;
+                        const double den = sqrt(fabs(app) * fabs(aqq));
+                        worst = fmax(worst, den > 0.0 ? fabs(apq) / den : INFINITY);
                     }
                 }
                 cs[k] = c;
@@ -151,61 +116,60 @@ __global__ void __launch_bounds__(kJThreads, 1)
                 if (x == y) dgn[x] = v;
                 else if (nq[x] == y) odn[nk[x]] = v;
             };
-            for (long e = gtid; e < items; e += gstride) {
-                if (e < blocks) {
-                    const int i = (int)(e / H), j = (int)(e % H);
-                    const double ci = cs[i], si = sn[i], cj = cs[j], sj = sn[j];
-                    const int pi = P[i], qi = Q[i], pj = P[j], qj = Q[j];
-                    const bool vp = pi < n, vq = qi < n, wp = pj < n, wq = qj < n;
-                    if (si == 0.0 && sj == 0.0) {      // unchanged: copy what the next round pivots on
-                        if (vp && wp && (pi == pj || nq[pi] == pj)) note(pi, pj, __ldcg(A + pi * lda + pj));
-                        if (vp && wq && (pi == qj || nq[pi] == qj)) note(pi, qj, __ldcg(A + pi * lda + qj));
-                        if (vq && wp && (qi == pj || nq[qi] == pj)) note(qi, pj, __ldcg(A + qi * lda + pj));
-                        if (vq && wq && (qi == qj || nq[qi] == qj)) note(qi, qj, __ldcg(A + qi * lda + qj));
-                        continue;
-                    }
-                    if (i == j) {
-                        // diagonal block: the closed form keeps the off-diagonal exactly zero
-                        const double t = tv[i], apq = __ldcg(odc + i);
-                        const double npp = __ldcg(dgc + pi) - t * apq, nqq = __ldcg(dgc + qi) + t * apq;
-                        A[pi * lda + pi] = npp;
-                        A[qi * lda + qi] = nqq;
-                        A[pi * lda + qi] = 0.0;
-                        A[qi * lda + pi] = 0.0;
-                        note(pi, pi, npp);
-                        note(qi, qi, nqq);
-                        note(pi, qi, 0.0);
-                        note(qi, pi, 0.0);
-                        continue;
-                    }
-                    const double b00 = vp && wp ? __ldcg(A + pi * lda + pj) : 0.0;
-                    const double b01 = vp && wq ? __ldcg(A + pi * lda + qj) : 0.0;
-                    const double b10 = vq && wp ? __ldcg(A + qi * lda + pj) : 0.0;
-                    const double b11 = vq && wq ? __ldcg(A + qi * lda + qj) : 0.0;
-                    const double r00 = ci * b00 - si * b10, r01 = ci * b01 - si * b11;
-                    const double r10 = si * b00 + ci * b10, r11 = si * b01 + ci * b11;
-                    const double n00 = cj * r00 - sj * r01, n01 = sj * r00 + cj * r01;
-                    const double n10 = cj * r10 - sj * r11, n11 = sj * r10 + cj * r11;
-                    if (vp && wp) { A[pi * lda + pj] = n00; note(pi, pj, n00); }
-                    if (vp && wq) { A[pi * lda + qj] = n01; note(pi, qj, n01); }
-                    if (vq && wp) { A[qi * lda + pj] = n10; note(qi, pj, n10); }
-                    if (vq && wq) { A[qi * lda + qj] = n11; note(qi, qj, n11); }
-                } else {
-                    const long f = e - blocks;
-                    const int i = (int)(f / n), col = (int)(f % n);
-                    const double ci = cs[i], si = sn[i];
-                    if (si == 0.0) continue;
-                    double *rp = Vt + P[i] * ldv + col, *rq = Vt + Q[i] * ldv + col;
-                    const double vpv = __ldcg(rp), vqv = __ldcg(rq);
-                    *rp = ci * vpv - si * vqv;
-                    *rq = si * vpv + ci * vqv;
+            for (int e = gt; e < nblocks; e += gs) {
+                const int i = e / H, j = e - (e / H) * H;
+                const double ci = cs[i], si = sn[i], cj = cs[j], sj = sn[j];
+                const int pi = P[i], qi = Q[i], pj = P[j], qj = Q[j];
+                const bool vp = pi < n, vq = qi < n, wp = pj < n, wq = qj < n;
+                if (si == 0.0 && sj == 0.0) {          // unchanged: copy what the next round pivots on
+                    if (vp && wp && (pi == pj || nq[pi] == pj)) note(pi, pj, __ldcg(A + pi * lda + pj));
+                    if (vp && wq && (pi == qj || nq[pi] == qj)) note(pi, qj, __ldcg(A + pi * lda + qj));
+                    if (vq && wp && (qi == pj || nq[qi] == pj)) note(qi, pj, __ldcg(A + qi * lda + pj));
+                    if (vq && wq && (qi == qj || nq[qi] == qj)) note(qi, qj, __ldcg(A + qi * lda + qj));
+                    continue;
                 }
+                if (i == j) {
+                    // diagonal block: the closed form keeps the off-diagonal exactly zero
+                    const double t = tv[i], apq = __ldcg(odc + i);
+                    const double npp = __ldcg(dgc + pi) - t * apq, nqq = __ldcg(dgc + qi) + t * apq;
+                    A[pi * lda + pi] = npp;
+                    A[qi * lda + qi] = nqq;
+                    A[pi * lda + qi] = 0.0;
+                    A[qi * lda + pi] = 0.0;
+                    note(pi, pi, npp);
+                    note(qi, qi, nqq);
+                    note(pi, qi, 0.0);
+                    note(qi, pi, 0.0);
+                    continue;
+                }
+                const double b00 = vp && wp ? __ldcg(A + pi * lda + pj) : 0.0;
+                const double b01 = vp && wq ? __ldcg(A + pi * lda + qj) : 0.0;
+                const double b10 = vq && wp ? __ldcg(A + qi * lda + pj) : 0.0;
+                const double b11 = vq && wq ? __ldcg(A + qi * lda + qj) : 0.0;
+                const double r00 = ci * b00 - si * b10, r01 = ci * b01 - si * b11;
+                const double r10 = si * b00 + ci * b10, r11 = si * b01 + ci * b11;
+                const double n00 = cj * r00 - sj * r01, n01 = sj * r00 + cj * r01;
+                const double n10 = cj * r10 - sj * r11, n11 = sj * r10 + cj * r11;
+                if (vp && wp) { A[pi * lda + pj] = n00; note(pi, pj, n00); }
+                if (vp && wq) { A[pi * lda + qj] = n01; note(pi, qj, n01); }
+                if (vq && wp) { A[qi * lda + pj] = n10; note(qi, pj, n10); }
+                if (vq && wq) { A[qi * lda + qj] = n11; note(qi, qj, n11); }
+            }
+            for (int f = gt; f < nvt; f += gs) {
+                const int i = f / n, col = f - (f / n) * n;
+                const double ci = cs[i], si = sn[i];
+                if (si == 0.0) continue;
+                double *rp = Vt + P[i] * ldv + col, *rq = Vt + Q[i] * ldv + col;
+                const double vpv = __ldcg(rp), vqv = __ldcg(rq);
+                *rp = ci * vpv - si * vqv;
+                *rq = si * vpv + ci * vqv;
             }
             if (!grid_barrier(bar, gen, err)) return;
             b ^= 1;
         }
-        // every CTA saw the same rotations, so all CTAs take the same decision
-        if (!__syncthreads_or(rotated)) break;
+        // every CTA saw the same rotations, so all CTAs take the same decision.  Convergence is quadratic: once
+        // every rotation of a sweep was below kJStop, what is left off the diagonal is of order kJStop^2
+        if (!__syncthreads_or(worst > kJStop)) break;
     }
 }
 
@@ -240,8 +204,8 @@ cudaError_t jacobi_eig(double *A, int n, long lda, double *Vt, long ldv, double 
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, jacobi_kernel, kJThreads, smem);
     if (e != cudaSuccess) return e;
     if (occ < 1) return cudaErrorInvalidConfiguration;
-    const long items = (long)H * H + (long)H * n;
-    const int grid = (int)std::max<long>(1, std::min<long>((long)sm_count_j(), (items + kJThreads * 8 - 1) / (kJThreads * 8)));
+    const long items = std::max((long)H * H, (long)H * n);
+    const int grid = (int)std::max<long>(1, std::min<long>((long)sm_count_j(), (items + kJThreads - 1) / kJThreads));
     e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned), s);
     if (e != cudaSuccess) return e;
     void *args[] = {&A, &n, &lda, &Vt, &ldv, &side, &bar, &err, &max_sweeps};

@@ -36,4 +36,13 @@ constexpr int kJacobiMaxN = 4096;
 cudaError_t jacobi_eig(double *A, int n, long lda, double *Vt, long ldv, double *side, unsigned *bar, int *err,
                        int max_sweeps, cudaStream_t s);
 
+// Cholesky factor of the Gram matrix S (n x n, lower triangle read and
+// overwritten) and its inverse, in one cooperative launch: Linv (n x n, ld
+// ldI, lower triangular) = L^{-1} with S = L L^T, so X Linv^T has orthonormal
+// columns when S = X^T X.  A column whose pivot falls to 1e-13 times its
+// original squared norm or below counts as dependent and is dropped (its row
+// of Linv is zero).  Lf (n x n, ld ldI) and dg (n) are scratch.
+cudaError_t chol_inverse(double *S, int n, long ldS, double *Lf, double *Linv, long ldI, double *dg, unsigned *bar,
+                         int *err, cudaStream_t s);
+
 }  // namespace lb
