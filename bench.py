@@ -317,6 +317,8 @@ def main():
     ap.add_argument("--init", default=INIT_DEFAULT,
                     help="workload whose first block gets the Dual-SVID + residual initialisation ('' = skip)")
     ap.add_argument("--init-steps", type=int, default=2)
+    ap.add_argument("--init-warmup", type=int, default=3)
+    ap.add_argument("--init-layers", default="", help="comma-separated layer names of the block (default: all)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -432,7 +434,8 @@ def main():
                            "clocks": pres["clocks"]}
 
     if args.init and world == 1:
-        line["init"] = run_init(args.init, args.init_steps, 3, dev, args.cpu_seconds > 0)
+        line["init"] = run_init(args.init, args.init_steps, args.init_warmup, dev, args.cpu_seconds > 0,
+                                args.init_layers)
 
     if rank == 0 and args.cpu_seconds > 0:
         cs = oracle_sample(w, M, args.cpu_seconds)
@@ -453,7 +456,7 @@ def subspace_width(s: synth.LayerShape) -> int:
     return min(min(s.N, s.K), max(64, -(-2 * s.r // 64) * 64))
 
 
-def run_init(wkey: str, steps: int, warmup: int, dev, with_cpu: bool):
+def run_init(wkey: str, steps: int, warmup: int, dev, with_cpu: bool, only: str = ""):
     """Dual-SVID + residual initialisation of every layer of one block of a workload, from synthetic dense W.
 
     One step = both paths of all layers of the block (lb_dual_svid_init, binary64, INIT_ITERS iterations).  The
@@ -463,7 +466,7 @@ def run_init(wkey: str, steps: int, warmup: int, dev, with_cpu: bool):
     import torch
     from sub_bit_weight_b200 import lib
     w = synth.WORKLOADS[wkey]
-    shapes = list(w.block)
+    shapes = [s for s in w.block if not only or s.name in only.split(",")]
     Ws = {}
     for s in shapes:        # one synthetic W per distinct shape (the work per layer does not depend on the values)
         if (s.N, s.K) not in Ws:
@@ -480,11 +483,13 @@ def run_init(wkey: str, steps: int, warmup: int, dev, with_cpu: bool):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clk:
+        torch.cuda.nvtx.range_push("init_timed")
         e0.record()
         for _ in range(steps):
             block()
         e1.record()
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
     ms_block = e0.elapsed_time(e1) / steps
     # the dominant kernel: the two products of the first subspace iteration of the largest layer
     big = max(shapes, key=lambda s: s.N * s.K * subspace_width(s))
