@@ -1,0 +1,366 @@
+// Backward pass of a LittleBit layer for quantisation-aware training
+// (LittleBit paper notes page, "Multi-scale compensation" and "Loss /
+// training strategy": SmoothSign, forward sign and backward tanh(100 u)).
+//
+// Per path, with ds = dy (.) h:
+//   dzl = ds U_s            = latent contraction of the transposed layer (U <-> V, h <-> g) applied to dy
+//   dx  = sum_p g (.) (dz V_s^T), dz = dzl (.) l
+//                           = output contraction of the transposed layer applied to dz
+//   z   = (x (.) g) V_s     = latent contraction of the forward layer with l = 1
+//   dl  = sum_m dzl (.) z,  zl = z (.) l
+//   G_U = dy^T zl, dh = sum_j U_s (.) G_U, dU = h (.) G_U (.) 100 (1 - tanh^2(100 U))
+//   G_V = x^T dz,  dg = sum_j V_s (.) G_V, dV = g (.) G_V (.) 100 (1 - tanh^2(100 V))
+// The contractions run on the tcgen05 kernels of the forward pass (two helper
+// layers with l = 1); G_U and G_V are plain fp16 GEMMs (cuBLAS).  dy is
+// multiplied by one power of two 2^E, chosen on the device so that dy 2^E and
+// dzl 2^E (and dz 2^E) stay below 2^14, and divided out exactly at the end.
+#include "littlebit_backward.h"
+#include "lb_internal.cuh"
+#include "lb_prefill.cuh"
+
+#include <cublas_v2.h>
+#include <cuda_fp16.h>
+#include <algorithm>
+#include <math.h>
+#include <new>
+
+struct lb_backward {
+    int N = 0, K = 0, r = 0, npaths = 0, r8 = 0, K2 = 0;
+    lb_layer *Lf = nullptr;        // forward layer with l = 1: its latent contraction gives z
+    lb_layer *Lt = nullptr;        // transposed layer with l = 1: latent gives dzl, output gives dx from dz
+    float *lcat = nullptr;         // [K2] l per latent column j' = p*r8 + j (0 on padding)
+    float *h32 = nullptr;          // [npaths][N]
+    float *g32 = nullptr;          // [npaths][K]
+    float *hmax = nullptr;         // [N] max_p |h_p|
+    uint32_t *Uw = nullptr;        // [npaths][N][wpr] canonical packed signs
+    uint32_t *Vw = nullptr;        // [npaths][K][wpr]
+    float *dl_acc = nullptr;       // [K2]
+    float *stat = nullptr;         // [0] bound (float bits, atomic max), [1] 2^E, [2] 2^-E, [3] max l, [4] 0
+    int M = 0;                     // rows the scratch below holds
+    __half *dy16 = nullptr;        // [M][N]
+    __half *x16 = nullptr;         // [M][K]
+    float *GU = nullptr;           // [N][K2]
+    float *GV = nullptr;           // [K][K2]
+    cublasHandle_t blas = nullptr;
+};
+
+namespace lb {
+namespace {
+
+constexpr int kT = 256;
+
+int grid_for(long n) { return (int)std::max<long>(1, std::min<long>((n + kT - 1) / kT, 148L * 16)); }
+
+__global__ void half_ones_kernel(uint16_t *o, int n)
+{
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) o[i] = 0x3C00;
+}
+
+// float32 copies of binary16 scales; l laid out per latent column; max_p |h_p| per row
+__global__ void scales_kernel(const uint16_t *h0, const uint16_t *h1, const uint16_t *g0, const uint16_t *g1,
+                              const uint16_t *l0, const uint16_t *l1, int npaths, int N, int K, int r, int r8,
+                              int K2, float *h32, float *g32, float *hmax, float *lcat, float *stat)
+{
+    const int n = max(max(N, K), K2);
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        if (i < N) {
+            const float a = __half2float(__ushort_as_half(h0[i]));
+            const float b = npaths > 1 ? __half2float(__ushort_as_half(h1[i])) : 0.0f;
+            h32[i] = a;
+            if (npaths > 1) h32[N + i] = b;
+            hmax[i] = fmaxf(fabsf(a), fabsf(b));
+        }
+        if (i < K) {
+            g32[i] = __half2float(__ushort_as_half(g0[i]));
+            if (npaths > 1) g32[K + i] = __half2float(__ushort_as_half(g1[i]));
+        }
+        if (i < K2) {
+            const int p = i / r8, j = i - p * r8;
+            float v = 0.0f;
+            if (p < npaths && j < r) v = __half2float(__ushort_as_half(p ? l1[j] : l0[j]));
+            lcat[i] = v;
+            if (v != 0.0f) atomicMax(reinterpret_cast<int *>(stat + 3), __float_as_int(fabsf(v)));
+        }
+    }
+}
+
+// bound = max over rows of max(max_n |dy|, sum_n |dy| hmax[n]) (atomic max on the float's bits: non-negative)
+__global__ void dy_bound_kernel(const float *__restrict__ dy, int M, int N, const float *__restrict__ hmax, float *stat)
+{
+    const int lane = threadIdx.x & 31;
+    for (int m = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; m < M; m += (gridDim.x * blockDim.x) >> 5) {
+        const float *row = dy + (size_t)m * N;
+        float mx = 0.0f, l1 = 0.0f;
+        for (int n = lane; n < N; n += 32) {
+            const float a = fabsf(row[n]);
+            mx = fmaxf(mx, a);
+            l1 += a * hmax[n];
+        }
+        for (int o = 16; o; o >>= 1) {
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+        }
+        if (lane == 0) atomicMax(reinterpret_cast<int *>(stat), __float_as_int(fmaxf(mx, l1)));
+    }
+}
+
+// 2^E with bound * max(1, max l) * 2^E < 2^14 (E = 0 for a zero or non-finite bound)
+__global__ void exponent_kernel(float *stat)
+{
+    const float b = stat[0] * fmaxf(1.0f, stat[3]);
+    int e = 0;
+    if (b > 0.0f && isfinite(b)) {
+        frexpf(b, &e);                  // b < 2^e
+        e = 14 - e;
+        e = max(-120, min(120, e));
+    } else {
+        e = 0;
+    }
+    stat[1] = ldexpf(1.0f, e);
+    stat[2] = ldexpf(1.0f, -e);
+}
+
+__global__ void convert_kernel(const float *__restrict__ dy, long ndy, const uint16_t *__restrict__ x, long nx,
+                               const float *__restrict__ stat, __half *dy16, __half *x16)
+{
+    const float sc = stat[1];
+    const long n = max(ndy, nx);
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+        if (i < ndy) dy16[i] = __float2half_rn(dy[i] * sc);
+        if (i < nx) x16[i] = __float2half_rn(__uint_as_float((uint32_t)x[i] << 16));
+    }
+}
+
+// dl_acc[j'] += sum_m dzl[m][j'] z[m][j']; dzl <- fp16(dzl l) (= dz), z <- fp16(z l) (= zl).  One column per
+// thread, a slice of rows per CTA (blockIdx.y).
+__global__ void latent_mix_kernel(__half *dzl, __half *z, int M, int ncols, int ld, const float *__restrict__ lcat,
+                                  float *dl_acc, int rows_per)
+{
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= ncols) return;
+    const int m0 = blockIdx.y * rows_per, m1 = min(M, m0 + rows_per);
+    const float lj = lcat[j];
+    float acc = 0.0f;
+    for (int m = m0; m < m1; ++m) {
+        const size_t o = (size_t)m * ld + j;
+        const float a = __half2float(dzl[o]), b = __half2float(z[o]);
+        acc = fmaf(a, b, acc);
+        dzl[o] = __float2half_rn(a * lj);
+        z[o] = __float2half_rn(b * lj);
+    }
+    atomicAdd(dl_acc + j, acc);
+}
+
+__global__ void scale_kernel(float *x, long n, const float *__restrict__ stat)
+{
+    const float sc = stat[2];
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) x[i] *= sc;
+}
+
+__global__ void dl_out_kernel(const float *__restrict__ dl_acc, int r, int r8, const float *__restrict__ stat,
+                              float *dl0, float *dl1)
+{
+    const float sc = stat[2];
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < r; j += gridDim.x * blockDim.x) {
+        dl0[j] = dl_acc[j] * sc;
+        if (dl1) dl1[j] = dl_acc[r8 + j] * sc;
+    }
+}
+
+// factor gradients of one path: one warp per row i of G (rows x K2, the path's columns at off .. off + r):
+// dF[i][j] = s[i] G[i][off + j] 100 (1 - tanh^2(100 F[i][j])),  dsc[i] = sum_j sign_ij G[i][off + j]
+__global__ void factor_grad_kernel(const float *__restrict__ G, int rows, int K2, int off, int r,
+                                   const float *__restrict__ s, const uint32_t *__restrict__ words,
+                                   const float *__restrict__ F, float *dF, float *dsc)
+{
+    const int lane = threadIdx.x & 31, wpr = (r + 31) / 32;
+    for (int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < rows; i += (gridDim.x * blockDim.x) >> 5) {
+        const float si = s[i];
+        float acc = 0.0f;
+        for (int j = lane; j < r; j += 32) {
+            const float gv = G[(size_t)i * K2 + off + j];
+            const bool neg = (words[(size_t)i * wpr + j / 32] >> (j % 32)) & 1u;
+            acc += neg ? -gv : gv;
+            // 100 (1 - tanh^2(100 u)) = 400 e^{-2a} / (1 + e^{-2a})^2, a = |100 u| (no cancellation for large a)
+            const float ea = expf(-2.0f * fabsf(100.0f * F[(size_t)i * r + j]));
+            const float d1 = 1.0f + ea;
+            dF[(size_t)i * r + j] = si * gv * (400.0f * ea / (d1 * d1));
+        }
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) dsc[i] = acc;
+    }
+}
+
+lb_status grow(lb_backward *B, int M, cudaStream_t s)
+{
+    if (M <= B->M) return LB_OK;
+    if (B->M) cudaStreamSynchronize(s);
+    cudaFree(B->dy16);
+    cudaFree(B->x16);
+    B->dy16 = nullptr;
+    B->x16 = nullptr;
+    B->M = 0;
+    if (cudaMalloc(&B->dy16, (size_t)M * B->N * sizeof(__half)) != cudaSuccess ||
+        cudaMalloc(&B->x16, (size_t)M * B->K * sizeof(__half)) != cudaSuccess)
+        return LB_ERR_OOM;
+    B->M = M;
+    return LB_OK;
+}
+
+}  // namespace
+}  // namespace lb
+
+using namespace lb;
+
+extern "C" {
+
+void lb_backward_destroy(lb_backward *B)
+{
+    if (!B) return;
+    lb_layer_destroy(B->Lf);
+    lb_layer_destroy(B->Lt);
+    for (void *p : {(void *)B->lcat, (void *)B->h32, (void *)B->g32, (void *)B->hmax, (void *)B->Uw, (void *)B->Vw,
+                    (void *)B->dl_acc, (void *)B->stat, (void *)B->dy16, (void *)B->x16, (void *)B->GU,
+                    (void *)B->GV})
+        cudaFree(p);
+    if (B->blas) cublasDestroy(B->blas);
+    delete B;
+}
+
+lb_status lb_backward_create(lb_backward **out, int N, int K, int r, int npaths, const uint32_t *const *U,
+                             const uint32_t *const *V, const uint16_t *const *h, const uint16_t *const *g,
+                             const uint16_t *const *l, void *stream)
+{
+    if (!out) return LB_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (N < 1 || K < 1 || r < 1 || r > LB_MAX_RANK) return LB_ERR_INVALID_ARG;
+    if (npaths != 1 && npaths != 2) return LB_ERR_UNSUPPORTED;
+    if (!U || !V || !h || !g || !l) return LB_ERR_INVALID_ARG;
+    for (int p = 0; p < npaths; ++p)
+        if (!U[p] || !V[p] || !h[p] || !g[p] || !l[p]) return LB_ERR_INVALID_ARG;
+    if (N % 8 || K % 8) return LB_ERR_UNSUPPORTED;
+    cudaStream_t s = (cudaStream_t)stream;
+    lb_backward *B = new (std::nothrow) lb_backward();
+    if (!B) return LB_ERR_OOM;
+    B->N = N;
+    B->K = K;
+    B->r = r;
+    B->npaths = npaths;
+    B->r8 = (r + 7) / 8 * 8;
+    const int N1p = (npaths * B->r8 + 15) / 16 * 16;
+    B->K2 = (N1p + 63) / 64 * 64;
+    const int wpr = (r + 31) / 32;
+    lb_status st = LB_OK;
+    uint16_t *ones = nullptr;
+    auto fail = [&](lb_status e) {
+        cudaFree(ones);
+        lb_backward_destroy(B);
+        return e;
+    };
+    if (cudaMalloc(&ones, (size_t)r * sizeof(uint16_t)) != cudaSuccess) return fail(LB_ERR_OOM);
+    half_ones_kernel<<<grid_for(r), kT, 0, s>>>(ones, r);
+    const uint16_t *ones2[2] = {ones, ones};
+    const uint32_t *Ut[2] = {V[0], npaths > 1 ? V[1] : V[0]};
+    const uint32_t *Vt[2] = {U[0], npaths > 1 ? U[1] : U[0]};
+    if ((st = lb_layer_create(&B->Lf, N, K, r, npaths, U, V, h, g, ones2, stream)) != LB_OK) return fail(st);
+    if ((st = lb_layer_create(&B->Lt, K, N, r, npaths, Ut, Vt, g, h, ones2, stream)) != LB_OK) return fail(st);
+    auto alloc = [&](void **p, size_t bytes) { return cudaMalloc(p, bytes) == cudaSuccess; };
+    if (!alloc((void **)&B->lcat, (size_t)B->K2 * 4) || !alloc((void **)&B->h32, (size_t)npaths * N * 4) ||
+        !alloc((void **)&B->g32, (size_t)npaths * K * 4) || !alloc((void **)&B->hmax, (size_t)N * 4) ||
+        !alloc((void **)&B->Uw, (size_t)npaths * N * wpr * 4) || !alloc((void **)&B->Vw, (size_t)npaths * K * wpr * 4) ||
+        !alloc((void **)&B->dl_acc, (size_t)B->K2 * 4) || !alloc((void **)&B->stat, 8 * 4) ||
+        !alloc((void **)&B->GU, (size_t)N * B->K2 * 4) || !alloc((void **)&B->GV, (size_t)K * B->K2 * 4))
+        return fail(LB_ERR_OOM);
+    cudaMemsetAsync(B->stat, 0, 8 * 4, s);
+    scales_kernel<<<grid_for(std::max(std::max(N, K), B->K2)), kT, 0, s>>>(
+        h[0], npaths > 1 ? h[1] : h[0], g[0], npaths > 1 ? g[1] : g[0], l[0], npaths > 1 ? l[1] : l[0], npaths, N, K, r,
+        B->r8, B->K2, B->h32, B->g32, B->hmax, B->lcat, B->stat);
+    for (int p = 0; p < npaths; ++p) {
+        cudaMemcpyAsync(B->Uw + (size_t)p * N * wpr, U[p], (size_t)N * wpr * 4, cudaMemcpyDeviceToDevice, s);
+        cudaMemcpyAsync(B->Vw + (size_t)p * K * wpr, V[p], (size_t)K * wpr * 4, cudaMemcpyDeviceToDevice, s);
+    }
+    if (cublasCreate(&B->blas) != CUBLAS_STATUS_SUCCESS) return fail(LB_ERR_CUDA);
+    cublasSetPointerMode(B->blas, CUBLAS_POINTER_MODE_DEVICE);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return fail(LB_ERR_CUDA);
+    cudaFree(ones);
+    ones = nullptr;
+    if (cudaGetLastError() != cudaSuccess) return fail(LB_ERR_CUDA);
+    *out = B;
+    return LB_OK;
+}
+
+lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, int M, const float *const *U_lat,
+                            const float *const *V_lat, float *dx, float *const *dh, float *const *dg,
+                            float *const *dl, float *const *dU, float *const *dV, void *stream)
+{
+    set_launch_count(0);
+    if (!B || M < 1 || !x || !dy || !dx || !U_lat || !V_lat || !dh || !dg || !dl || !dU || !dV)
+        return LB_ERR_INVALID_ARG;
+    if (((uintptr_t)x | (uintptr_t)dy | (uintptr_t)dx) & 15) return LB_ERR_INVALID_ARG;
+    for (int p = 0; p < B->npaths; ++p)
+        if (!U_lat[p] || !V_lat[p] || !dh[p] || !dg[p] || !dl[p] || !dU[p] || !dV[p]) return LB_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaGetLastError() != cudaSuccess) return LB_ERR_CUDA;
+    lb_status st = grow(B, M, s);
+    if (st != LB_OK) return st;
+    const int N = B->N, K = B->K, r = B->r, K2 = B->K2;
+    int launches = 0;
+
+    // dy scale (device-side exponent), fp16 copies of dy 2^E and x
+    cudaMemsetAsync(B->stat, 0, sizeof(float), s);
+    cudaMemsetAsync(B->dl_acc, 0, (size_t)K2 * 4, s);
+    dy_bound_kernel<<<grid_for(32L * M), kT, 0, s>>>(dy, M, N, B->hmax, B->stat);
+    exponent_kernel<<<1, 1, 0, s>>>(B->stat);
+    convert_kernel<<<grid_for((long)M * std::max(N, K)), kT, 0, s>>>(dy, (long)M * N, x, (long)M * K, B->stat, B->dy16,
+                                                                      B->x16);
+    launches += 3;
+
+    // z (forward latent, l = 1) and dzl 2^E (transposed latent, l = 1); the y map of the forward helper is never
+    // used (its output contraction is not run), dx only stands in for a well-aligned pointer there
+    const uint16_t *xs[1] = {x};
+    const uint16_t *dys[1] = {reinterpret_cast<const uint16_t *>(B->dy16)};
+    float *ys[1] = {dx};
+    if ((st = prefill_forward(B->Lf->self->plan, &B->Lf, xs, ys, M, s, &launches, 1, false)) != LB_OK) return st;
+    if ((st = prefill_forward(B->Lt->self->plan, &B->Lt, dys, ys, M, s, &launches, 1, true)) != LB_OK) return st;
+    __half *zf = prefill_zl(B->Lf->self->plan, 0), *dz = prefill_zl(B->Lt->self->plan, 0);
+    if (!zf || !dz) return LB_ERR_CUDA;
+
+    // dl, dz = dzl l, zl = z l
+    const int ncols = B->npaths * B->r8, rows_per = 64;
+    latent_mix_kernel<<<dim3((ncols + kT - 1) / kT, (M + rows_per - 1) / rows_per), kT, 0, s>>>(
+        dz, zf, M, ncols, K2, B->lcat, B->dl_acc, rows_per);
+    // dx 2^E = sum_p g (.) (dz 2^E V_s^T)
+    if ((st = prefill_forward(B->Lt->self->plan, &B->Lt, dys, ys, M, s, &launches, 2, true)) != LB_OK) return st;
+    scale_kernel<<<grid_for((long)M * K), kT, 0, s>>>(dx, (long)M * K, B->stat);
+    dl_out_kernel<<<grid_for(r), kT, 0, s>>>(B->dl_acc, r, B->r8, B->stat, dl[0], B->npaths > 1 ? dl[1] : nullptr);
+    launches += 3;
+
+    // G_U = dy^T zl, G_V = x^T dz (row-major; cuBLAS sees the column-major transposes), alpha = 2^-E
+    const float *alpha = B->stat + 2, *zero_d = B->stat + 4;
+    cublasSetStream(B->blas, s);
+    if (cublasGemmEx(B->blas, CUBLAS_OP_N, CUBLAS_OP_T, K2, N, M, alpha, zf, CUDA_R_16F, K2, B->dy16, CUDA_R_16F, N,
+                     zero_d, B->GU, CUDA_R_32F, K2, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+        return LB_ERR_CUDA;
+    if (cublasGemmEx(B->blas, CUBLAS_OP_N, CUBLAS_OP_T, K2, K, M, alpha, dz, CUDA_R_16F, K2, B->x16, CUDA_R_16F, K,
+                     zero_d, B->GV, CUDA_R_32F, K2, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+        return LB_ERR_CUDA;
+    const int wpr = (r + 31) / 32;
+    for (int p = 0; p < B->npaths; ++p) {
+        factor_grad_kernel<<<grid_for(32L * N), kT, 0, s>>>(B->GU, N, K2, p * B->r8, r, B->h32 + (size_t)p * N,
+                                                           B->Uw + (size_t)p * N * wpr, U_lat[p], dU[p], dh[p]);
+        factor_grad_kernel<<<grid_for(32L * K), kT, 0, s>>>(B->GV, K, K2, p * B->r8, r, B->g32 + (size_t)p * K,
+                                                           B->Vw + (size_t)p * K * wpr, V_lat[p], dV[p], dg[p]);
+        launches += 2;
+    }
+    set_launch_count(launches);
+    return cudaGetLastError() == cudaSuccess ? LB_OK : LB_ERR_CUDA;
+}
+
+lb_status lb_backward_status(lb_backward *B, void *stream)
+{
+    if (!B) return LB_ERR_INVALID_ARG;
+    lb_status a = lb_layer_status(B->Lf, stream), b = lb_layer_status(B->Lt, stream);
+    return a != LB_OK ? a : b;
+}
+
+}  // extern "C"

@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
             for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
                 int L, mt, nt;
                 locate(t, L, mt, nt);
-                const int nk = layers[L].nk;
+                const int nk = layers[L].nk, a_f16 = layers[L].a_f16;
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % kPfStages;
@@ -498,14 +498,16 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
                         break;
                     }
                     const uint32_t A0 = smem_u32(S.A[s]);
+                    if (!a_f16) {
 #pragma unroll 2
-                    for (int i = ct; i < kPfBM * kPfBK * 2 / 16; i += kConv) {
-                        uint4 v = lds128(A0 + 16u * i);
-                        v.x = bf16x2_to_f16x2(v.x);
-                        v.y = bf16x2_to_f16x2(v.y);
-                        v.z = bf16x2_to_f16x2(v.z);
-                        v.w = bf16x2_to_f16x2(v.w);
-                        sts128(A0 + 16u * i, v);
+                        for (int i = ct; i < kPfBM * kPfBK * 2 / 16; i += kConv) {
+                            uint4 v = lds128(A0 + 16u * i);
+                            v.x = bf16x2_to_f16x2(v.x);
+                            v.y = bf16x2_to_f16x2(v.y);
+                            v.z = bf16x2_to_f16x2(v.z);
+                            v.w = bf16x2_to_f16x2(v.w);
+                            sts128(A0 + 16u * i, v);
+                        }
                     }
                     fence_proxy_async();
                     __syncwarp();
@@ -731,6 +733,7 @@ static bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base
 struct PrefillState {
     int M = 0;                       // rows the scratch was sized for
     int lastM = -1;
+    bool lastF16 = false;            // the activations of the last encoded maps are fp16
     std::vector<const void *> lastX, lastY;
     void *zl = nullptr;              // latent activations of every layer, fp16 [M][K2]
     std::vector<size_t> zl_off;
@@ -757,7 +760,7 @@ void prefill_free(PrefillState *st)
 static size_t smem_bytes(int nlayers) { return sizeof(PfSmem) + 1024 + sizeof(int) * (size_t)(nlayers + 1); }
 
 lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const uint16_t *const *xs,
-                          float *const *ys, int M, cudaStream_t s, int *launches)
+                          float *const *ys, int M, cudaStream_t s, int *launches, int parts, bool a_f16)
 {
     Plan &P = const_cast<Plan &>(Pc);
     const int n = P.n;
@@ -797,7 +800,7 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
         st.M = M;
         dirty = true;
     }
-    if (M != st.lastM) dirty = true;
+    if (M != st.lastM || a_f16 != st.lastF16) dirty = true;
     if ((int)st.lastX.size() != n) {
         st.lastX.assign(n, nullptr);
         st.lastY.assign(n, nullptr);
@@ -814,7 +817,8 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
             const LayerDev &d = layers[i]->d;
             const PfWeights &W = layers[i]->pf;
             __half *zl = (__half *)((char *)st.zl + st.zl_off[i]);
-            if (!encode_2d(&maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xs[i], d.K, M) ||
+            if (!encode_2d(&maps[i], a_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xs[i],
+                           d.K, M) ||
                 !encode_2d(&maps[n + i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, zl, W.K2, M) ||
                 !encode_2d(&maps[2 * n + i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ys[i], d.N, M, 4, 32, 32))
                 return LB_ERR_UNSUPPORTED;
@@ -833,6 +837,7 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
             a.r8 = W.r8;
             a.base_ld = W.K64;
             a.npaths = d.npaths;
+            a.a_f16 = a_f16;
             PfLayer &b = rec[n + i];
             b.tmA = st.maps + n + i;
             b.tmY = st.maps + 2 * n + i;
@@ -847,6 +852,7 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
             b.r8 = W.r8;
             b.base_ld = W.N256;
             b.npaths = d.npaths;
+            b.a_f16 = 0;
             starts[i + 1] = starts[i] + mtiles * a.ntn;
             starts[n + 1 + i + 1] = starts[n + 1 + i] + mtiles * b.ntn;
             st.lastX[i] = xs[i];
@@ -855,6 +861,7 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
         st.tiles[0] = starts[n];
         st.tiles[1] = starts[2 * n + 1];
         st.lastM = M;
+        st.lastF16 = a_f16;
         // pageable sources: the copies are staged before these calls return
         if ((e = cudaMemcpyAsync(st.maps, maps.data(), sizeof(CUtensorMap) * 3 * n, cudaMemcpyHostToDevice, s)) !=
             cudaSuccess)
@@ -886,11 +893,21 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
     const int g0 = std::max(1, std::min(st.tiles[0], sms));
     const int g1 = std::max(1, std::min(st.tiles[1], sms));
     profile_mark(0, s);
-    prefill_kernel<0><<<g0, pf_threads(0), smem, s>>>(st.rec, st.starts, n, M, st.err);
-    profile_mark(++*launches, s);
-    prefill_kernel<1><<<g1, pf_threads(1), smem, s>>>(st.rec + n, st.starts + n + 1, n, M, st.err);
-    profile_mark(++*launches, s);
+    if (parts & 1) {
+        prefill_kernel<0><<<g0, pf_threads(0), smem, s>>>(st.rec, st.starts, n, M, st.err);
+        profile_mark(++*launches, s);
+    }
+    if (parts & 2) {
+        prefill_kernel<1><<<g1, pf_threads(1), smem, s>>>(st.rec + n, st.starts + n + 1, n, M, st.err);
+        profile_mark(++*launches, s);
+    }
     return status_from(cudaGetLastError());
+}
+
+__half *prefill_zl(const Plan &P, int i)
+{
+    if (!P.pf || !P.pf->zl || i < 0 || i >= (int)P.pf->zl_off.size()) return nullptr;
+    return (__half *)((char *)P.pf->zl + P.pf->zl_off[i]);
 }
 
 }  // namespace lb

@@ -39,6 +39,7 @@ struct PfLayer {
     int r8;                   // columns per path
     int base_ld;              // row stride of base (K64 or N256)
     int npaths;
+    int a_f16;                // latent contraction: A is already fp16 (no bf16 conversion)
 };
 
 }  // namespace lb

@@ -58,6 +58,10 @@ _sig("lb_stack_status", _st, [_vp, _vp])
 _sig("lb_layer_status", _st, [_vp, _vp])
 _sig("lb_selftest_wait_timeout", _st, [ctypes.c_longlong, _vp])
 _sig("lb_dual_svid_workspace_bytes", ctypes.c_size_t, [_i, _i, _i])
+_sig("lb_backward_create", _st, [ctypes.POINTER(_vp), _i, _i, _i, _i] + [ctypes.POINTER(_vp)] * 5 + [_vp])
+_sig("lb_backward_destroy", None, [_vp])
+_sig("lb_layer_backward", _st, [_vp, _vp, _vp, _i] + [ctypes.POINTER(_vp)] * 2 + [_vp] + [ctypes.POINTER(_vp)] * 5 + [_vp])
+_sig("lb_backward_status", _st, [_vp, _vp])
 _sig("lb_dual_svid_init", _st, [_vp, _i, _i, _i, _i, _i] + [ctypes.POINTER(_vp)] * 5 + [_vp, _vp, ctypes.c_size_t, _vp])
 
 
@@ -318,3 +322,69 @@ def lb_dual_svid_init(W: torch.Tensor, r: int, npaths: int = 2, iters: int = 24,
                                   _dev(sigma, torch.float32, "sigma"), _dev(workspace, torch.uint8, "workspace"),
                                   workspace.numel(), _stream(stream)), "lb_dual_svid_init")
     return DualSvidResult(U, V, h, g, l, sigma)
+
+
+# ---------------------------------------------------------------------------
+# QAT backward (include/littlebit_backward.h)
+# ---------------------------------------------------------------------------
+
+class Backward:
+    """Owns an ``lb_backward`` handle (see ``lb_backward_create``)."""
+
+    def __init__(self, handle: int, N: int, K: int, r: int, npaths: int):
+        self.handle = handle
+        self.N, self.K, self.r, self.npaths = N, K, r, npaths
+
+    def close(self):
+        if self.handle:
+            _lib.lb_backward_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def lb_backward_create(N: int, K: int, r: int, U, V, h, g, l, stream=None) -> Backward:
+    """Per-path lists as lb_layer_create: canonical packed U, V (int32) and binary16 h, g, l (CUDA)."""
+    npaths = len(U)
+    arrs = []
+    for name, lst in (("U", U), ("V", V), ("h", h), ("g", g), ("l", l)):
+        if len(lst) != npaths:
+            raise ValueError(f"{name} must have one entry per path")
+        ptrs = [_dev(t, torch.int32, f"{name}[{p}]") if name in ("U", "V") else _u16(t, f"{name}[{p}]")
+                for p, t in enumerate(lst)]
+        arrs.append((_vp * max(1, npaths))(*ptrs))
+    out = _vp()
+    _check(_lib.lb_backward_create(ctypes.byref(out), N, K, r, npaths, *arrs, _stream(stream)), "lb_backward_create")
+    return Backward(out.value, N, K, r, npaths)
+
+
+def lb_layer_backward(B: Backward, x: torch.Tensor, dy: torch.Tensor, U_lat, V_lat, stream=None) -> dict:
+    """Gradients for x [M, K] (bfloat16) and dy [M, N] (float32): dx [M, K] and per-path lists dh, dg, dl, dU, dV."""
+    M = x.shape[0]
+    if tuple(x.shape) != (M, B.K) or tuple(dy.shape) != (M, B.N):
+        raise ValueError("x must be [M, K] and dy [M, N]")
+    dev = x.device
+    P = B.npaths
+    out = {"dx": torch.empty((M, B.K), dtype=torch.float32, device=dev),
+           "dh": [torch.empty(B.N, dtype=torch.float32, device=dev) for _ in range(P)],
+           "dg": [torch.empty(B.K, dtype=torch.float32, device=dev) for _ in range(P)],
+           "dl": [torch.empty(B.r, dtype=torch.float32, device=dev) for _ in range(P)],
+           "dU": [torch.empty((B.N, B.r), dtype=torch.float32, device=dev) for _ in range(P)],
+           "dV": [torch.empty((B.K, B.r), dtype=torch.float32, device=dev) for _ in range(P)]}
+
+    def arr(lst, name):
+        return (_vp * max(1, len(lst)))(*[_dev(t, torch.float32, f"{name}[{p}]") for p, t in enumerate(lst)])
+
+    _check(_lib.lb_layer_backward(B.handle, _dev(x, torch.bfloat16, "x"), _dev(dy, torch.float32, "dy"), M,
+                                  arr(U_lat, "U_lat"), arr(V_lat, "V_lat"), _dev(out["dx"], torch.float32, "dx"),
+                                  arr(out["dh"], "dh"), arr(out["dg"], "dg"), arr(out["dl"], "dl"),
+                                  arr(out["dU"], "dU"), arr(out["dV"], "dV"), _stream(stream)), "lb_layer_backward")
+    return out
+
+
+def lb_backward_status(B: Backward, stream=None) -> int:
+    return int(_lib.lb_backward_status(B.handle, _stream(stream)))

@@ -99,3 +99,25 @@ def test_initialisation_argument_checks(lib):
     assert lib.lb_dual_svid_init(vp(256), 96, 40, 6, 1, 24, *args, None, vp(264), ws, None) == 1   # misaligned
     nulls = (vp * 1)(None)
     assert lib.lb_dual_svid_init(vp(256), 96, 40, 6, 1, 24, nulls, *args[1:], None, vp(256), ws, None) == 1
+
+
+def test_backward_argument_checks(lib):
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    P = ctypes.POINTER(vp)
+    one = (vp * 1)(vp(256))
+    lib.lb_backward_create.argtypes = [P, i, i, i, i] + [P] * 5 + [vp]
+    out = vp()
+    assert lib.lb_backward_create(None, 64, 64, 8, 1, one, one, one, one, one, None) == 1
+    assert lib.lb_backward_create(ctypes.byref(out), 64, 64, 8, 3, one, one, one, one, one, None) == 2
+    assert lib.lb_backward_create(ctypes.byref(out), 64, 60, 8, 1, one, one, one, one, one, None) == 2   # K % 8
+    assert lib.lb_backward_create(ctypes.byref(out), 0, 64, 8, 1, one, one, one, one, one, None) == 1
+    nulls = (vp * 1)(None)
+    assert lib.lb_backward_create(ctypes.byref(out), 64, 64, 8, 1, nulls, one, one, one, one, None) == 1
+    lib.lb_layer_backward.argtypes = [vp, vp, vp, i] + [P] * 2 + [vp] + [P] * 5 + [vp]
+    assert lib.lb_layer_backward(None, vp(256), vp(256), 4, one, one, vp(256), one, one, one, one, one, None) == 1
+    lib.lb_backward_destroy.argtypes = [vp]
+    lib.lb_backward_destroy(None)
+    from sub_bit_weight_b200 import lib as binding     # the binding declares the same argument counts
+    assert len(binding._lib.lb_layer_backward.argtypes) == 13
+    assert len(binding._lib.lb_backward_create.argtypes) == 11
+    assert len(binding._lib.lb_dual_svid_init.argtypes) == 15
