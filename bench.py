@@ -38,6 +38,7 @@ METRIC = "LittleBit linear decode GB/s & prefill TFLOP/s, % of B200 roofline"
 DECODE_DEFAULT = "llama2_70b_0.1"
 PREFILL_DEFAULT = "llama2_13b_0.3_prefill"
 INIT_DEFAULT = "llama2_7b_0.1"
+BACKWARD_DEFAULT = "llama2_13b_0.3_prefill"
 INIT_ITERS = 24
 # binary64 FMA rate of B200: 148 SMs x 64 FP64 FMA per clock x 2 FLOP at the 1965 MHz maximum SM clock
 FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
@@ -319,6 +320,9 @@ def main():
     ap.add_argument("--init-steps", type=int, default=2)
     ap.add_argument("--init-warmup", type=int, default=3)
     ap.add_argument("--init-layers", default="", help="comma-separated layer names of the block (default: all)")
+    ap.add_argument("--backward", default=BACKWARD_DEFAULT,
+                    help="workload whose first block gets the QAT backward pass ('' = skip)")
+    ap.add_argument("--backward-steps", type=int, default=5)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -433,6 +437,9 @@ def main():
                                         "traffic": prefill_traffic(pw.key)},
                            "clocks": pres["clocks"]}
 
+    if args.backward and world == 1:
+        line["backward"] = run_backward(args.backward, args.backward_steps, 3, dev, args.cpu_seconds > 0, pk)
+
     if args.init and world == 1:
         line["init"] = run_init(args.init, args.init_steps, args.init_warmup, dev, args.cpu_seconds > 0,
                                 args.init_layers)
@@ -537,6 +544,117 @@ def run_init(wkey: str, steps: int, warmup: int, dev, with_cpu: bool, only: str 
         out["cpu_baseline"] = {"value": round(1.0 / dt, 4), "unit": "layers/s", "cores": cores, "kind": "oracle",
                                "sample": f"one {s.name} layer {s.N}x{s.K} r={s.r}, two paths, numpy/LAPACK "
                                          f"float64 ({dt:.1f} s)"}
+    return out
+
+
+def backward_stage_flops(s: synth.LayerShape, M: int, npaths: int = 2):
+    """Algorithmic FLOPs of the backward stages of one layer (2 FLOPs per multiply-add, no padding)."""
+    R = npaths * s.r
+    return {"z = (x.g) V_s": 2.0 * M * s.K * R, "(dy.h) U_s": 2.0 * M * s.N * R, "dx": 2.0 * M * R * s.K,
+            "dy^T zl": 2.0 * M * s.N * R, "x^T dz": 2.0 * M * s.K * R}
+
+
+def run_backward(wkey: str, steps: int, warmup: int, dev, with_cpu: bool, pk):
+    """QAT backward pass of every layer of one block of a workload (lb_layer_backward), M rows of the workload.
+
+    One step = the backward of all layers of the block.  Inputs: latent factors N(0, 0.02) (their signs are the
+    layer's), the workload's scales and activations, dy ~ N(0, 1) * 1e-4.  The dominant stage is timed with the
+    library's event hook on the largest layer.
+    """
+    import torch
+    from sub_bit_weight_b200 import lib
+    w = synth.WORKLOADS[wkey]
+    shapes = list(w.block)
+    M = w.Ms[0]
+    rng = np.random.default_rng(w.seed + 77)
+    objs = {}
+    for s in shapes:
+        if (s.N, s.K) in objs:
+            continue
+        U = [torch.from_numpy(rng.normal(0, 0.02, (s.N, s.r)).astype(np.float32)).to(dev) for _ in range(2)]
+        V = [torch.from_numpy(rng.normal(0, 0.02, (s.K, s.r)).astype(np.float32)).to(dev) for _ in range(2)]
+        sc = {k: [torch.from_numpy(synth.scale_vector(w.seed, 0, p, k, n).view(np.int16)).to(dev) for p in range(2)]
+              for k, n in (("h", s.N), ("g", s.K), ("l", s.r))}
+        B = lib.lb_backward_create(s.N, s.K, s.r, [lib.lb_pack_signs(u) for u in U], [lib.lb_pack_signs(v) for v in V],
+                                   sc["h"], sc["g"], sc["l"])
+        x = torch.from_numpy(synth.activations(w.seed, 0, M, s.K).view(np.int16)).to(dev).view(torch.bfloat16)
+        dy = torch.from_numpy((rng.standard_normal((M, s.N)) * 1e-4).astype(np.float32)).to(dev)
+        objs[(s.N, s.K)] = (B, x, dy, U, V, sc)
+
+    def block():
+        for s in shapes:
+            B, x, dy, U, V, _ = objs[(s.N, s.K)]
+            lib.lb_layer_backward(B, x, dy, U, V)
+
+    for _ in range(warmup):
+        block()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        torch.cuda.nvtx.range_push("backward_timed")
+        e0.record()
+        for _ in range(steps):
+            block()
+        e1.record()
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
+    ms_block = e0.elapsed_time(e1) / steps
+    flops = sum(sum(backward_stage_flops(s, M).values()) for s in shapes)
+    tf = flops / (ms_block * 1e-3) / 1e12
+    # stages of the largest layer, timed with the event hook (one event at every stage boundary)
+    big = max(shapes, key=lambda s: s.N * s.K)
+    B, x, dy, U, V, _ = objs[(big.N, big.K)]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(9)]
+    for e in ev:
+        e.record()
+    torch.cuda.synchronize()
+    names = ["dy scaling", "z = (x.g) V_s", "(dy.h) U_s", "dl, dz, zl", "dx", "dy^T zl", "x^T dz", "dh, dg, dU, dV"]
+    stage = {n: 0.0 for n in names}
+    reps = 5
+    for _ in range(reps):
+        lib.lb_profile_events(ev)
+        lib.lb_layer_backward(B, x, dy, U, V)
+        lib.lb_profile_events([])
+        torch.cuda.synchronize()
+        for i, n in enumerate(names):
+            stage[n] += ev[i].elapsed_time(ev[i + 1]) / reps
+    sf = backward_stage_flops(big, M)
+    dom = max(sf, key=lambda n: stage[n])
+    ach = sf[dom] / (stage[dom] * 1e-3) / 1e12
+    kern = {"z = (x.g) V_s": "prefill_kernel<0> (latent contraction of the forward helper)",
+            "(dy.h) U_s": "prefill_kernel<0> (latent contraction of the transposed helper, fp16 input)",
+            "dx": "prefill_kernel<1> (output contraction of the transposed helper)",
+            "dy^T zl": "cuBLAS fp16 GEMM", "x^T dz": "cuBLAS fp16 GEMM"}[dom]
+    out = {"workload": f"{w.key} first block: " + ", ".join(f"{s.name} {s.N}x{s.K} r={s.r}" for s in shapes)
+                       + f"; M = {M}, two paths; latent factors N(0, 0.02), dy N(0, 1) x 1e-4",
+           "value": round(tf, 2), "unit": "TFLOP/s", "higher_is_better": True, "ms_per_block": round(ms_block, 3),
+           "steps": steps, "warmup": warmup, "flops_per_block": flops,
+           "stages_ms_largest_layer": {n: round(v, 4) for n, v in stage.items()},
+           "roofline": {"bound": "tensor", "kernel": f"{dom}: {kern}, {big.name} {big.N}x{big.K}",
+                        "achieved": round(ach, 1), "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                        "frac": round(ach / pk["bf16_tflops_sustained"], 4),
+                        "peak_src": pk["src"] + " bf16 sustained (fp16 has the same dense rate)", "traffic": None},
+           "clocks": clk.summary()}
+    if with_cpu:
+        from oracle import qat_backward as qb
+        s = shapes[0]
+        Bq, x, dy, U, V, sc = objs[(s.N, s.K)]
+        f16 = lambda t: t.cpu().numpy().view(np.float16).astype(np.float64)
+        xn = synth.bf16_bits_to_f32(x.view(torch.int16).cpu().numpy().view(np.uint16))
+        t0 = time.perf_counter()
+        qb.backward(xn, dy.cpu().numpy(), [u.cpu().numpy() for u in U], [v.cpu().numpy() for v in V],
+                    [f16(v) for v in sc["h"]], [f16(v) for v in sc["g"]], [f16(v) for v in sc["l"]])
+        dt = time.perf_counter() - t0
+        try:
+            from threadpoolctl import threadpool_info
+            cores = max((i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"), default=1)
+        except Exception:
+            cores = os.cpu_count()
+        of = sum(backward_stage_flops(s, M).values())
+        out["cpu_baseline"] = {"value": round(of / dt / 1e12, 5), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                               "sample": f"one {s.name} layer {s.N}x{s.K} r={s.r}, M = {M}, numpy float64 ({dt:.1f} s)"}
+    for v in objs.values():
+        v[0].close()
     return out
 
 

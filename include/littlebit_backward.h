@@ -65,7 +65,12 @@ LB_API void lb_backward_destroy(lb_backward *B);
  * work is enqueued on `stream` (no host synchronisation); scratch grows with M
  * and is owned by B, so calls on one B must not overlap.  Errors:
  * LB_ERR_INVALID_ARG, LB_ERR_OOM, LB_ERR_CUDA; a bounded wait that gave up in
- * a contraction kernel surfaces through lb_backward_status. */
+ * a contraction kernel surfaces through lb_backward_status.
+ *
+ * With the timing hook of littlebit.h (lb_profile_events) holding 9 events,
+ * events[i] is recorded at the i-th stage boundary: 0 | dy scaling | 1 |
+ * z = (x (.) g) V_s | 2 | (dy (.) h) U_s | 3 | dl, dz, zl | 4 | dx | 5 |
+ * dy^T zl | 6 | x^T dz | 7 | dh, dg, dU, dV | 8. */
 LB_API lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, int M,
                                    const float *const *U_lat, const float *const *V_lat, float *dx,
                                    float *const *dh, float *const *dg, float *const *dl,

@@ -84,23 +84,40 @@ __global__ void scales_kernel(const uint16_t *h0, const uint16_t *h1, const uint
     }
 }
 
-// bound = max over rows of max(max_n |dy|, sum_n |dy| hmax[n]) (atomic max on the float's bits: non-negative)
-__global__ void dy_bound_kernel(const float *__restrict__ dy, int M, int N, const float *__restrict__ hmax, float *stat)
+// bound = max over rows of max(max_n |dy|, sum_n |dy| hmax[n]) (atomic max on the float's bits: non-negative);
+// one CTA per row, float4 loads (N is a multiple of 8)
+__global__ void __launch_bounds__(kT) dy_bound_kernel(const float *__restrict__ dy, int M, int N,
+                                                      const float *__restrict__ hmax, float *stat)
 {
-    const int lane = threadIdx.x & 31;
-    for (int m = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; m < M; m += (gridDim.x * blockDim.x) >> 5) {
-        const float *row = dy + (size_t)m * N;
+    __shared__ float smx[kT / 32], sl1[kT / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n4 = N / 4;
+    const float4 *hm = reinterpret_cast<const float4 *>(hmax);
+    for (int m = blockIdx.x; m < M; m += gridDim.x) {
+        const float4 *row = reinterpret_cast<const float4 *>(dy + (size_t)m * N);
         float mx = 0.0f, l1 = 0.0f;
-        for (int n = lane; n < N; n += 32) {
-            const float a = fabsf(row[n]);
-            mx = fmaxf(mx, a);
-            l1 += a * hmax[n];
+#pragma unroll 4
+        for (int q = threadIdx.x; q < n4; q += kT) {
+            const float4 a = __ldg(row + q), h = __ldg(hm + q);
+            mx = fmaxf(fmaxf(fmaxf(mx, fabsf(a.x)), fmaxf(fabsf(a.y), fabsf(a.z))), fabsf(a.w));
+            l1 += fabsf(a.x) * h.x + fabsf(a.y) * h.y + fabsf(a.z) * h.z + fabsf(a.w) * h.w;
         }
         for (int o = 16; o; o >>= 1) {
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             l1 += __shfl_xor_sync(0xffffffffu, l1, o);
         }
-        if (lane == 0) atomicMax(reinterpret_cast<int *>(stat), __float_as_int(fmaxf(mx, l1)));
+        if (lane == 0) {
+            smx[warp] = mx;
+            sl1[warp] = l1;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            for (int w = 1; w < kT / 32; ++w) {
+                mx = fmaxf(mx, smx[w]);
+                l1 += sl1[w];
+            }
+            atomicMax(reinterpret_cast<int *>(stat), __float_as_int(fmaxf(mx, l1)));
+        }
+        __syncthreads();
     }
 }
 
@@ -120,14 +137,25 @@ __global__ void exponent_kernel(float *stat)
     stat[2] = ldexpf(1.0f, -e);
 }
 
+// dy16 = fp16(dy 2^E), x16 = fp16(x); four elements per thread (N and K are multiples of 8)
 __global__ void convert_kernel(const float *__restrict__ dy, long ndy, const uint16_t *__restrict__ x, long nx,
                                const float *__restrict__ stat, __half *dy16, __half *x16)
 {
     const float sc = stat[1];
-    const long n = max(ndy, nx);
+    const long n = max(ndy, nx) / 4;
     for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
-        if (i < ndy) dy16[i] = __float2half_rn(dy[i] * sc);
-        if (i < nx) x16[i] = __float2half_rn(__uint_as_float((uint32_t)x[i] << 16));
+        if (4 * i < ndy) {
+            const float4 a = reinterpret_cast<const float4 *>(dy)[i];
+            __half2 *o = reinterpret_cast<__half2 *>(dy16) + 2 * i;
+            o[0] = __floats2half2_rn(a.x * sc, a.y * sc);
+            o[1] = __floats2half2_rn(a.z * sc, a.w * sc);
+        }
+        if (4 * i < nx) {
+            const uint2 b = reinterpret_cast<const uint2 *>(x)[i];
+            __half2 *o = reinterpret_cast<__half2 *>(x16) + 2 * i;
+            o[0] = __floats2half2_rn(__uint_as_float(b.x << 16), __uint_as_float(b.x & 0xFFFF0000u));
+            o[1] = __floats2half2_rn(__uint_as_float(b.y << 16), __uint_as_float(b.y & 0xFFFF0000u));
+        }
     }
 }
 
@@ -167,27 +195,42 @@ __global__ void dl_out_kernel(const float *__restrict__ dl_acc, int r, int r8, c
     }
 }
 
-// factor gradients of one path: one warp per row i of G (rows x K2, the path's columns at off .. off + r):
-// dF[i][j] = s[i] G[i][off + j] 100 (1 - tanh^2(100 F[i][j])),  dsc[i] = sum_j sign_ij G[i][off + j]
-__global__ void factor_grad_kernel(const float *__restrict__ G, int rows, int K2, int off, int r,
-                                   const float *__restrict__ s, const uint32_t *__restrict__ words,
-                                   const float *__restrict__ F, float *dF, float *dsc)
+// factor gradients of all paths: one warp per row i of G (rows x K2; path p's columns at p r8 .. p r8 + r):
+// dF_p[i][j] = s_p[i] G[i][p r8 + j] 100 (1 - tanh^2(100 F_p[i][j])),  dsc_p[i] = sum_j sign_pij G[i][p r8 + j].
+// 100 (1 - tanh^2(a)) is evaluated as 400 e^{-2|a|} / (1 + e^{-2|a|})^2 (no cancellation for large |a|).
+struct FactorArgs {
+    const float *s[2];
+    const uint32_t *words[2];
+    const float *F[2];
+    float *dF[2];
+    float *dsc[2];
+};
+
+template <int P>
+__global__ void __launch_bounds__(kT) factor_grad_kernel(const float *__restrict__ G, int rows, int K2, int r, int r8,
+                                                         const FactorArgs a)
 {
     const int lane = threadIdx.x & 31, wpr = (r + 31) / 32;
     for (int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < rows; i += (gridDim.x * blockDim.x) >> 5) {
-        const float si = s[i];
-        float acc = 0.0f;
-        for (int j = lane; j < r; j += 32) {
-            const float gv = G[(size_t)i * K2 + off + j];
-            const bool neg = (words[(size_t)i * wpr + j / 32] >> (j % 32)) & 1u;
-            acc += neg ? -gv : gv;
-            // 100 (1 - tanh^2(100 u)) = 400 e^{-2a} / (1 + e^{-2a})^2, a = |100 u| (no cancellation for large a)
-            const float ea = expf(-2.0f * fabsf(100.0f * F[(size_t)i * r + j]));
-            const float d1 = 1.0f + ea;
-            dF[(size_t)i * r + j] = si * gv * (400.0f * ea / (d1 * d1));
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+            const float si = a.s[p][i];
+            const float *__restrict__ g = G + (size_t)i * K2 + p * r8;
+            const uint32_t *__restrict__ w = a.words[p] + (size_t)i * wpr;
+            const float *__restrict__ f = a.F[p] + (size_t)i * r;
+            float *__restrict__ df = a.dF[p] + (size_t)i * r;
+            float acc = 0.0f;
+#pragma unroll 4
+            for (int j = lane; j < r; j += 32) {
+                const float gv = __ldg(g + j);
+                acc += ((__ldg(w + (j >> 5)) >> (j & 31)) & 1u) ? -gv : gv;
+                const float ea = __expf(-200.0f * fabsf(__ldg(f + j)));
+                const float d1 = 1.0f + ea;
+                df[j] = si * gv * (400.0f * ea / (d1 * d1));
+            }
+            for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == 0) a.dsc[p][i] = acc;
         }
-        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) dsc[i] = acc;
     }
 }
 
@@ -306,22 +349,28 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
     const int N = B->N, K = B->K, r = B->r, K2 = B->K2;
     int launches = 0;
 
+    // timing hook (littlebit.h): events 0 | scaling | 1 | z | 2 | dzl | 3 | dl, dz, zl | 4 | dx | 5 | G_U | 6 | G_V | 7
+    // | factor gradients | 8
+    profile_mark(0, s);
     // dy scale (device-side exponent), fp16 copies of dy 2^E and x
     cudaMemsetAsync(B->stat, 0, sizeof(float), s);
     cudaMemsetAsync(B->dl_acc, 0, (size_t)K2 * 4, s);
-    dy_bound_kernel<<<grid_for(32L * M), kT, 0, s>>>(dy, M, N, B->hmax, B->stat);
+    dy_bound_kernel<<<std::min(M, 148 * 8), kT, 0, s>>>(dy, M, N, B->hmax, B->stat);
     exponent_kernel<<<1, 1, 0, s>>>(B->stat);
     convert_kernel<<<grid_for((long)M * std::max(N, K)), kT, 0, s>>>(dy, (long)M * N, x, (long)M * K, B->stat, B->dy16,
                                                                       B->x16);
     launches += 3;
+    profile_mark(1, s);
 
     // z (forward latent, l = 1) and dzl 2^E (transposed latent, l = 1); the y map of the forward helper is never
     // used (its output contraction is not run), dx only stands in for a well-aligned pointer there
     const uint16_t *xs[1] = {x};
     const uint16_t *dys[1] = {reinterpret_cast<const uint16_t *>(B->dy16)};
     float *ys[1] = {dx};
-    if ((st = prefill_forward(B->Lf->self->plan, &B->Lf, xs, ys, M, s, &launches, 1, false)) != LB_OK) return st;
-    if ((st = prefill_forward(B->Lt->self->plan, &B->Lt, dys, ys, M, s, &launches, 1, true)) != LB_OK) return st;
+    if ((st = prefill_forward(B->Lf->self->plan, &B->Lf, xs, ys, M, s, &launches, 1, false, false)) != LB_OK) return st;
+    profile_mark(2, s);
+    if ((st = prefill_forward(B->Lt->self->plan, &B->Lt, dys, ys, M, s, &launches, 1, true, false)) != LB_OK) return st;
+    profile_mark(3, s);
     __half *zf = prefill_zl(B->Lf->self->plan, 0), *dz = prefill_zl(B->Lt->self->plan, 0);
     if (!zf || !dz) return LB_ERR_CUDA;
 
@@ -329,11 +378,13 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
     const int ncols = B->npaths * B->r8, rows_per = 64;
     latent_mix_kernel<<<dim3((ncols + kT - 1) / kT, (M + rows_per - 1) / rows_per), kT, 0, s>>>(
         dz, zf, M, ncols, K2, B->lcat, B->dl_acc, rows_per);
-    // dx 2^E = sum_p g (.) (dz 2^E V_s^T)
-    if ((st = prefill_forward(B->Lt->self->plan, &B->Lt, dys, ys, M, s, &launches, 2, true)) != LB_OK) return st;
-    scale_kernel<<<grid_for((long)M * K), kT, 0, s>>>(dx, (long)M * K, B->stat);
     dl_out_kernel<<<grid_for(r), kT, 0, s>>>(B->dl_acc, r, B->r8, B->stat, dl[0], B->npaths > 1 ? dl[1] : nullptr);
+    profile_mark(4, s);
+    // dx 2^E = sum_p g (.) (dz 2^E V_s^T)
+    if ((st = prefill_forward(B->Lt->self->plan, &B->Lt, dys, ys, M, s, &launches, 2, true, false)) != LB_OK) return st;
+    scale_kernel<<<grid_for((long)M * K), kT, 0, s>>>(dx, (long)M * K, B->stat);
     launches += 3;
+    profile_mark(5, s);
 
     // G_U = dy^T zl, G_V = x^T dz (row-major; cuBLAS sees the column-major transposes), alpha = 2^-E
     const float *alpha = B->stat + 2, *zero_d = B->stat + 4;
@@ -341,17 +392,34 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
     if (cublasGemmEx(B->blas, CUBLAS_OP_N, CUBLAS_OP_T, K2, N, M, alpha, zf, CUDA_R_16F, K2, B->dy16, CUDA_R_16F, N,
                      zero_d, B->GU, CUDA_R_32F, K2, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
         return LB_ERR_CUDA;
+    profile_mark(6, s);
     if (cublasGemmEx(B->blas, CUBLAS_OP_N, CUBLAS_OP_T, K2, K, M, alpha, dz, CUDA_R_16F, K2, B->x16, CUDA_R_16F, K,
                      zero_d, B->GV, CUDA_R_32F, K2, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
         return LB_ERR_CUDA;
+    profile_mark(7, s);
     const int wpr = (r + 31) / 32;
+    FactorArgs fu{}, fv{};
     for (int p = 0; p < B->npaths; ++p) {
-        factor_grad_kernel<<<grid_for(32L * N), kT, 0, s>>>(B->GU, N, K2, p * B->r8, r, B->h32 + (size_t)p * N,
-                                                           B->Uw + (size_t)p * N * wpr, U_lat[p], dU[p], dh[p]);
-        factor_grad_kernel<<<grid_for(32L * K), kT, 0, s>>>(B->GV, K, K2, p * B->r8, r, B->g32 + (size_t)p * K,
-                                                           B->Vw + (size_t)p * K * wpr, V_lat[p], dV[p], dg[p]);
-        launches += 2;
+        fu.s[p] = B->h32 + (size_t)p * N;
+        fu.words[p] = B->Uw + (size_t)p * N * wpr;
+        fu.F[p] = U_lat[p];
+        fu.dF[p] = dU[p];
+        fu.dsc[p] = dh[p];
+        fv.s[p] = B->g32 + (size_t)p * K;
+        fv.words[p] = B->Vw + (size_t)p * K * wpr;
+        fv.F[p] = V_lat[p];
+        fv.dF[p] = dV[p];
+        fv.dsc[p] = dg[p];
     }
+    if (B->npaths == 2) {
+        factor_grad_kernel<2><<<grid_for(32L * N), kT, 0, s>>>(B->GU, N, K2, r, B->r8, fu);
+        factor_grad_kernel<2><<<grid_for(32L * K), kT, 0, s>>>(B->GV, K, K2, r, B->r8, fv);
+    } else {
+        factor_grad_kernel<1><<<grid_for(32L * N), kT, 0, s>>>(B->GU, N, K2, r, B->r8, fu);
+        factor_grad_kernel<1><<<grid_for(32L * K), kT, 0, s>>>(B->GV, K, K2, r, B->r8, fv);
+    }
+    launches += 2;
+    profile_mark(8, s);
     set_launch_count(launches);
     return cudaGetLastError() == cudaSuccess ? LB_OK : LB_ERR_CUDA;
 }

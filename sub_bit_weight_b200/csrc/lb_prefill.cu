@@ -760,7 +760,8 @@ void prefill_free(PrefillState *st)
 static size_t smem_bytes(int nlayers) { return sizeof(PfSmem) + 1024 + sizeof(int) * (size_t)(nlayers + 1); }
 
 lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const uint16_t *const *xs,
-                          float *const *ys, int M, cudaStream_t s, int *launches, int parts, bool a_f16)
+                          float *const *ys, int M, cudaStream_t s, int *launches, int parts, bool a_f16,
+                          bool marks)
 {
     Plan &P = const_cast<Plan &>(Pc);
     const int n = P.n;
@@ -892,14 +893,16 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
     }
     const int g0 = std::max(1, std::min(st.tiles[0], sms));
     const int g1 = std::max(1, std::min(st.tiles[1], sms));
-    profile_mark(0, s);
+    if (marks) profile_mark(0, s);
     if (parts & 1) {
         prefill_kernel<0><<<g0, pf_threads(0), smem, s>>>(st.rec, st.starts, n, M, st.err);
-        profile_mark(++*launches, s);
+        ++*launches;
+        if (marks) profile_mark(*launches, s);
     }
     if (parts & 2) {
         prefill_kernel<1><<<g1, pf_threads(1), smem, s>>>(st.rec + n, st.starts + n + 1, n, M, st.err);
-        profile_mark(++*launches, s);
+        ++*launches;
+        if (marks) profile_mark(*launches, s);
     }
     return status_from(cudaGetLastError());
 }

@@ -22,9 +22,10 @@ size_t prefill_weight_bytes(const LayerDev &d);
 
 struct PrefillState;   // per plan (owned by Plan)
 // parts: 1 = latent contraction only (writes the plan's zl), 2 = output contraction only (reads it), 3 = both.
-// a_f16: the activations xs are fp16 (bit patterns) rather than bf16.
+// a_f16: the activations xs are fp16 (bit patterns) rather than bf16.  marks: record the timing hook's events.
 lb_status prefill_forward(const Plan &P, const lb_layer *const *layers, const uint16_t *const *xs,
-                          float *const *ys, int M, cudaStream_t s, int *launches, int parts = 3, bool a_f16 = false);
+                          float *const *ys, int M, cudaStream_t s, int *launches, int parts = 3, bool a_f16 = false,
+                          bool marks = true);
 // latent activations of layer i of the plan, fp16 [M][pf.K2] (null before the first prefill call)
 __half *prefill_zl(const Plan &P, int i);
 void prefill_free(PrefillState *st);
