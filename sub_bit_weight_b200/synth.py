@@ -236,3 +236,16 @@ def dense_weight(seed: int, N: int, K: int, alpha: float = 1.0, rms: float = 0.0
     W = (A * s[None, :]) @ B
     W *= np.float32(rms / np.sqrt(np.mean(np.square(W, dtype=np.float64))))
     return bf16_bits_to_f32(f32_to_bf16_bits(W))
+
+
+def random_rotation(seed: int, r: int, path: int = 0) -> np.ndarray:
+    """A seeded random orthogonal r x r matrix (float64), the random start of an iterative-quantisation rotation.
+
+    The Q factor of a QR decomposition of an i.i.d. N(0, 1) matrix from
+    ``default_rng([seed, r, path, 0x17])``, its columns signed so that R's
+    diagonal is positive (Haar-distributed).  A random draw of the method, made
+    here and handed to both sides as an input.
+    """
+    rng = np.random.default_rng([seed, r, path, 0x17])
+    Q, Rq = np.linalg.qr(rng.standard_normal((r, r)))
+    return np.ascontiguousarray(Q * np.where(np.diag(Rq) < 0, -1.0, 1.0)[None, :])
