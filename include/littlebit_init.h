@@ -90,6 +90,52 @@ LB_API lb_status lb_dual_svid_init(const float *W, int N, int K, int r, int npat
                                    float *const *h, float *const *g, float *const *l, float *sigma,
                                    void *workspace, size_t workspace_bytes, void *stream);
 
+/* ------------------------------------------------------------------------
+ * LittleBit-2 initialisation: latent rotation by Joint-ITQ.
+ *
+ * Wiki page on LittleBit and LittleBit-2, section 1 ("What happened"): the
+ * second paper rotates the latent space and runs a joint iterative
+ * quantisation (Joint-ITQ) before QAT so that the factors line up with the
+ * binary hypercube; only the initialisation changes.  For an orthogonal
+ * r x r matrix R, (U' R)(V' R)^T = U' V'^T, so the rotation is free; it only
+ * changes the sign patterns.  Definitions this library fixes (the page gives
+ * no formulas):
+ *   - X = [U' / rho_u ; V' / rho_v] ((N + K) x r), each factor divided by the
+ *     root mean square of its entries (a zero factor is left as is);
+ *   - ITQ (Gong and Lazebnik's iterative quantisation): from R0, itq_iters
+ *     alternations of B = sign(X R) (sign(0) = +1) and R = the orthogonal
+ *     Procrustes solution for X^T B (its polar factor; computed here by
+ *     Newton-Schulz iteration on binary64 GEMMs);
+ *   - then U' <- U' R, V' <- V' R, canonical column signs as above, and the
+ *     Dual-SVID steps (signs, rank-1 SVDs of the magnitudes) and the residual
+ *     path as in lb_dual_svid_init, each path with its own rotation.
+ * The loss ||sign(X R_t) - X R_t||_F^2 / ((N + K) r) never increases.
+ * itq_iters = 0 with R0 = NULL is exactly lb_dual_svid_init.
+ * ------------------------------------------------------------------------ */
+
+/* Workspace bytes of lb_littlebit2_init (0 for an invalid shape). */
+LB_API size_t lb_littlebit2_workspace_bytes(int N, int K, int r);
+
+/* As lb_dual_svid_init, plus:
+ *   itq_iters  ITQ alternations per path (0 .. 1000; ITQ's customary 50).
+ *   R0         NULL (every path starts from the identity) or a host array of
+ *              npaths pointers, each NULL (identity) or a device binary64
+ *              r x r row-major orthogonal matrix, 8-byte aligned (ITQ's usual
+ *              start is a random rotation).  With itq_iters = 0 it is applied
+ *              as given, so it must then be orthogonal.
+ *   itq_loss   NULL or device binary64 [npaths][itq_iters + 1]: the loss
+ *              after t alternations, t = 0 .. itq_iters.
+ *   R_out      NULL or a host array of npaths pointers, each NULL or device
+ *              binary64 r x r row-major: the final rotation of the path.
+ *   workspace  at least lb_littlebit2_workspace_bytes(N, K, r) bytes.
+ * Errors and waiting as lb_dual_svid_init (LB_ERR_INVALID_ARG also for
+ * itq_iters out of range or a misaligned R0, R_out or itq_loss). */
+LB_API lb_status lb_littlebit2_init(const float *W, int N, int K, int r, int npaths, int iters, int itq_iters,
+                                    const double *const *R0, uint32_t *const *U, uint32_t *const *V,
+                                    float *const *h, float *const *g, float *const *l, float *sigma,
+                                    double *itq_loss, double *const *R_out,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

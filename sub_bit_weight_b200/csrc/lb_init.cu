@@ -23,6 +23,14 @@
 //      >= 0), a = |U'| b / s_A;
 //      h = a_u, g = a_v, l = s_u s_v (b_u (.) b_v);
 //   4. the residual path repeats 1-3 on W - diag(h) U_sign diag(l) V_sign^T diag(g).
+//
+// LittleBit-2 (wiki page on LittleBit and LittleBit-2, section 1: latent
+// rotation by joint iterative quantisation before QAT, initialisation only)
+// inserts between 1 and 2 a rotation R of the latent space, which leaves
+// U' V'^T unchanged: X = [U' / rho_u ; V' / rho_v] (each factor scaled to
+// unit RMS entry), then `itq_iters` alternations of B = sign(X R) and
+// R = polar(X^T B) (orthogonal Procrustes; the polar factor by Newton-Schulz
+// iteration, GEMMs only), and U' <- U' R, V' <- V' R before the signs.
 #include "littlebit_init.h"
 #include "lb_internal.cuh"
 #include "lb_linalg.cuh"
@@ -47,13 +55,19 @@ struct InitPlan {
     long ldK, ldL, ldr;
     size_t o_Wd, o_Q, o_Q2, o_Z, o_Z2, o_S, o_dg, o_Lf, o_Li, o_T, o_Vt, o_G, o_E, o_F, o_Up, o_Vp, o_M, o_vec, o_side,
         o_part;
+    size_t o_X, o_Y, o_R, o_C, o_P0, o_P1, o_NS, o_red;   // Joint-ITQ (LittleBit-2) only
+    bool itq;
     size_t o_int;             // int region (in doubles from the base)
     size_t total;             // doubles
 };
 
-InitPlan make_plan(int N, int K, int r)
+constexpr int kRedBlocks = 296;        // CTAs of the fixed-order reductions (two per SM)
+constexpr int kPolarIters = 40;        // Newton-Schulz steps: enough for sigma_min / ||C||_F down to ~1e-6
+
+InitPlan make_plan(int N, int K, int r, bool itq = false)
 {
     InitPlan P{};
+    P.itq = itq;
     P.N = N;
     P.K = K;
     P.r = r;
@@ -87,6 +101,16 @@ InitPlan make_plan(int N, int K, int r)
     P.o_vec = take((size_t)5 * r + 2 * (size_t)N + 2 * (size_t)K + 8);   // s, bu, bv, ls, misc | au, hs | av, gs
     P.o_side = take((size_t)3 * (P.L + 1));
     P.o_part = take(kDgemmPartElems);
+    if (itq) {
+        P.o_X = take((size_t)(N + K) * P.ldr);
+        P.o_Y = take((size_t)(N + K) * P.ldr);
+        P.o_R = take((size_t)r * P.ldr);
+        P.o_C = take((size_t)r * P.ldr);
+        P.o_P0 = take((size_t)r * P.ldr);
+        P.o_P1 = take((size_t)r * P.ldr);
+        P.o_NS = take((size_t)r * P.ldr);
+        P.o_red = take((size_t)kRedBlocks + 8);
+    }
     P.o_int = take((size_t)(2 * r + 16) / 2 + 1);                          // ints: bar[2], err, ord[r], flip[r]
     P.total = o;
     return P;
@@ -340,6 +364,123 @@ __global__ void signed_factor_kernel(const uint32_t *__restrict__ words, int row
 }
 
 // ---------------------------------------------------------------------------
+// Joint-ITQ kernels (LittleBit-2)
+// ---------------------------------------------------------------------------
+// block-wide sum of one value per thread (kT threads); the result is valid in thread 0
+__device__ double block_sum(double v)
+{
+    __shared__ double red[kT / 32];
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    if (threadIdx.x == 0)
+        for (int w = 1; w < kT / 32; ++w) v += red[w];
+    return v;
+}
+
+// part[b] = sum of X[i, j]^2 over this CTA's strided share of the entries (grid kRedBlocks x kT)
+__global__ void __launch_bounds__(kT) sumsq_kernel(const double *X, int rows, int r, long ld, double *part)
+{
+    double acc = 0.0;
+    const long total = (long)rows * r;
+    for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < total; e += (long)gridDim.x * blockDim.x) {
+        const double v = X[(e / r) * ld + e % r];
+        acc += v * v;
+    }
+    acc = block_sum(acc);
+    if (threadIdx.x == 0) part[blockIdx.x] = acc;
+}
+
+// out = scale * (part[0] + ... + part[n - 1]), summed in index order (one thread: deterministic)
+__global__ void finalize_sum_kernel(const double *part, int n, double scale, double *out)
+{
+    double a = 0.0;
+    for (int i = 0; i < n; ++i) a += part[i];
+    *out = a * scale;
+}
+
+// 1 / RMS entry of a rows x r factor from its sum of squares (1 for a zero factor)
+__device__ __forceinline__ double inv_rms(double ss, long n) { return ss > 0.0 ? 1.0 / sqrt(ss / (double)n) : 1.0; }
+
+// X = [U' / rho_u ; V' / rho_v] ((N + K) x r, ld); ss = the two sums of squares
+__global__ void itq_stack_kernel(const double *Up, int N, const double *Vp, int K, int r, long ld,
+                                 const double *__restrict__ ss, double *X)
+{
+    const double fu = inv_rms(ss[0], (long)N * r), fv = inv_rms(ss[1], (long)K * r);
+    const long total = (long)(N + K) * r;
+    for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < total; e += (long)gridDim.x * blockDim.x) {
+        const long i = e / r;
+        const int j = (int)(e % r);
+        X[i * ld + j] = i < N ? Up[i * ld + j] * fu : Vp[(i - N) * ld + j] * fv;
+    }
+}
+
+// U' = rho_u Y[0 .. N), V' = rho_v Y[N .. N + K): the rotated factors at their own scale
+__global__ void itq_unstack_kernel(const double *Y, int N, int K, int r, long ld, const double *__restrict__ ss,
+                                   double *Up, double *Vp)
+{
+    const double fu = 1.0 / inv_rms(ss[0], (long)N * r), fv = 1.0 / inv_rms(ss[1], (long)K * r);
+    const long total = (long)(N + K) * r;
+    for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < total; e += (long)gridDim.x * blockDim.x) {
+        const long i = e / r;
+        const int j = (int)(e % r);
+        if (i < N) Up[i * ld + j] = Y[i * ld + j] * fu;
+        else Vp[(i - N) * ld + j] = Y[i * ld + j] * fv;
+    }
+}
+
+// part[b] = this CTA's share of sum (sign(Y) - Y)^2 (sign(0) = +1); with `write`, Y <- sign(Y)
+__global__ void __launch_bounds__(kT) itq_sign_kernel(double *Y, int rows, int r, long ld, int write, double *part)
+{
+    double acc = 0.0;
+    const long total = (long)rows * r;
+    for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < total; e += (long)gridDim.x * blockDim.x) {
+        double *y = Y + (e / r) * ld + e % r;
+        const double v = *y, b = v < 0.0 ? -1.0 : 1.0;
+        acc += (b - v) * (b - v);
+        if (write) *y = b;
+    }
+    acc = block_sum(acc);
+    if (threadIdx.x == 0) part[blockIdx.x] = acc;
+}
+
+// X0 = C / ||C||_F, the start of the Newton-Schulz iteration (all singular values in (0, 1]); C = 0 gives the
+// identity.  One CTA of kT threads.
+__global__ void __launch_bounds__(kT) polar_start_kernel(const double *C, int r, long ld, double *X0)
+{
+    __shared__ double bc;
+    double acc = 0.0;
+    for (int e = threadIdx.x; e < r * r; e += blockDim.x) {
+        const double v = C[(long)(e / r) * ld + e % r];
+        acc += v * v;
+    }
+    acc = block_sum(acc);
+    if (threadIdx.x == 0) bc = acc;
+    __syncthreads();
+    const double nrm = sqrt(bc);
+    for (int e = threadIdx.x; e < r * r; e += blockDim.x) {
+        const int i = e / r, j = e % r;
+        X0[(long)i * ld + j] = nrm > 0.0 ? C[(long)i * ld + j] / nrm : (i == j ? 1.0 : 0.0);
+    }
+}
+
+// T = 1.5 I - 0.5 T (the Newton-Schulz factor X_{k+1} = X_k (3 I - X_k^T X_k) / 2)
+__global__ void ns_affine_kernel(double *T, int r, long ld)
+{
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < r * r; e += gridDim.x * blockDim.x) {
+        const int i = e / r, j = e % r;
+        double *t = T + (long)i * ld + j;
+        *t = (i == j ? 1.5 : 0.0) - 0.5 * *t;
+    }
+}
+
+__global__ void copy_square_kernel(const double *src, int r, long lds, double *dst, long ldd)
+{
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < r * r; e += gridDim.x * blockDim.x)
+        dst[(long)(e / r) * ldd + e % r] = src[(long)(e / r) * lds + e % r];
+}
+
+// ---------------------------------------------------------------------------
 // host steps
 // ---------------------------------------------------------------------------
 struct Ctx {
@@ -395,8 +536,56 @@ void rank1(const Ctx &c, const double *X, int rows, double *a, double *b, double
     vec_div_kernel<<<grid_for(rows), kT, 0, c.s>>>(a, rows, s);
 }
 
+// Joint-ITQ options of lb_littlebit2_init (none for lb_dual_svid_init)
+struct ItqArgs {
+    int iters = 0;
+    const double *const *R0 = nullptr;   // host array of device r x r (ld r) starts, or null (identity)
+    double *loss = nullptr;              // device [npaths][iters + 1], or null
+    double *const *Rout = nullptr;       // host array of device r x r (ld r) outputs, or null
+};
+
+// Rotate U', V' (N x r and K x r, ld ldr) by the Joint-ITQ rotation of path p (LittleBit-2).
+void joint_itq(const Ctx &c, const ItqArgs &a, int p, double *Up, double *Vp)
+{
+    const InitPlan &P = c.P;
+    const int N = P.N, K = P.K, r = P.r, rows = N + K;
+    const long ld = P.ldr;
+    double *X = c.at(P.o_X), *Y = c.at(P.o_Y), *R = c.at(P.o_R), *C = c.at(P.o_C), *T = c.at(P.o_NS);
+    double *Pa = c.at(P.o_P0), *Pb = c.at(P.o_P1);
+    double *red = c.at(P.o_red), *ss = red + kRedBlocks, *scratch = ss + 2;
+    sumsq_kernel<<<kRedBlocks, kT, 0, c.s>>>(Up, N, r, ld, red);
+    finalize_sum_kernel<<<1, 1, 0, c.s>>>(red, kRedBlocks, 1.0, ss);
+    sumsq_kernel<<<kRedBlocks, kT, 0, c.s>>>(Vp, K, r, ld, red);
+    finalize_sum_kernel<<<1, 1, 0, c.s>>>(red, kRedBlocks, 1.0, ss + 1);
+    itq_stack_kernel<<<grid_for((long)rows * r), kT, 0, c.s>>>(Up, N, Vp, K, r, ld, ss, X);
+    if (a.R0 && a.R0[p]) copy_square_kernel<<<grid_for((long)r * r), kT, 0, c.s>>>(a.R0[p], r, r, R, ld);
+    else identity_kernel<<<grid_for((long)r * r), kT, 0, c.s>>>(R, r, ld);
+    const double inv_n = 1.0 / ((double)rows * r);
+    for (int t = 0;; ++t) {
+        const bool last = t == a.iters;
+        c.gemm(false, false, rows, r, r, 1.0, X, ld, R, ld, 0.0, Y, ld);          // Y = X R
+        itq_sign_kernel<<<kRedBlocks, kT, 0, c.s>>>(Y, rows, r, ld, last ? 0 : 1, red);
+        finalize_sum_kernel<<<1, 1, 0, c.s>>>(red, kRedBlocks, inv_n,
+                                              a.loss ? a.loss + (size_t)p * (a.iters + 1) + t : scratch);
+        if (last) break;
+        c.gemm(true, false, r, r, rows, 1.0, X, ld, Y, ld, 0.0, C, ld);           // C = X^T B
+        polar_start_kernel<<<1, kT, 0, c.s>>>(C, r, ld, Pa);
+        for (int k = 0; k < kPolarIters; ++k) {
+            c.gemm(true, false, r, r, r, 1.0, Pa, ld, Pa, ld, 0.0, T, ld);        // T = X_k^T X_k
+            ns_affine_kernel<<<grid_for((long)r * r), kT, 0, c.s>>>(T, r, ld);
+            c.gemm(false, false, r, r, r, 1.0, Pa, ld, T, ld, 0.0, Pb, ld);       // X_{k+1} = X_k T
+            std::swap(Pa, Pb);
+        }
+        copy_square_kernel<<<grid_for((long)r * r), kT, 0, c.s>>>(Pa, r, ld, R, ld);
+    }
+    // Y = X R with the final R: back to each factor's own scale
+    itq_unstack_kernel<<<grid_for((long)rows * r), kT, 0, c.s>>>(Y, N, K, r, ld, ss, Up, Vp);
+    if (a.Rout && a.Rout[p]) copy_square_kernel<<<grid_for((long)r * r), kT, 0, c.s>>>(R, r, ld, a.Rout[p], r);
+}
+
 cudaError_t one_path(const Ctx &c, int iters, uint64_t seed, uint32_t *Uw, uint32_t *Vw, float *h, float *g, float *l,
-                     float *sigma, bool residual_next, unsigned *bar, int *err, int *ord, int *flip)
+                     float *sigma, bool residual_next, unsigned *bar, int *err, int *ord, int *flip,
+                     const ItqArgs *itq = nullptr, int path = 0)
 {
     const InitPlan &P = c.P;
     const int N = P.N, K = P.K, r = P.r, L = P.L;
@@ -446,6 +635,13 @@ cudaError_t one_path(const Ctx &c, int iters, uint64_t seed, uint32_t *Uw, uint3
         col_scale_kernel<<<grid_for((long)N * r), kT, 0, c.s>>>(E, N, r, P.ldr, sig, 1, Up, P.ldr);
         col_scale_kernel<<<grid_for((long)K * r), kT, 0, c.s>>>(F, K, r, P.ldr, sig, 0, Vp, P.ldr);
     }
+    if (itq) {
+        // LittleBit-2 latent rotation, started from the canonically signed factors
+        col_sign_kernel<<<grid_for(32L * r), kT, 0, c.s>>>(Up, N, r, P.ldr, flip);
+        col_flip_kernel<<<grid_for((long)N * r), kT, 0, c.s>>>(Up, N, r, P.ldr, flip);
+        col_flip_kernel<<<grid_for((long)K * r), kT, 0, c.s>>>(Vp, K, r, P.ldr, flip);
+        joint_itq(c, *itq, path, Up, Vp);
+    }
     col_sign_kernel<<<grid_for(32L * r), kT, 0, c.s>>>(Up, N, r, P.ldr, flip);
     col_flip_kernel<<<grid_for((long)N * r), kT, 0, c.s>>>(Up, N, r, P.ldr, flip);
     col_flip_kernel<<<grid_for((long)K * r), kT, 0, c.s>>>(Vp, K, r, P.ldr, flip);
@@ -477,19 +673,20 @@ extern "C" LB_API size_t lb_dual_svid_workspace_bytes(int N, int K, int r)
     return lb::make_plan(N, K, r).total * sizeof(double);
 }
 
-extern "C" LB_API lb_status lb_dual_svid_init(const float *W, int N, int K, int r, int npaths, int iters,
-                                              uint32_t *const *U, uint32_t *const *V, float *const *h,
-                                              float *const *g, float *const *l, float *sigma, void *workspace,
-                                              size_t workspace_bytes, void *stream)
+namespace lb {
+namespace {
+
+lb_status run_init(const float *W, int N, int K, int r, int npaths, int iters, uint32_t *const *U, uint32_t *const *V,
+                   float *const *h, float *const *g, float *const *l, float *sigma, void *workspace,
+                   size_t workspace_bytes, void *stream, const ItqArgs *itq)
 {
-    using namespace lb;
     if (N < 1 || K < 1 || r < 1 || r > std::min(N, K) || r > LB_MAX_RANK) return LB_ERR_INVALID_ARG;
     if (npaths != 1 && npaths != 2) return LB_ERR_UNSUPPORTED;
     if (!W || ((uintptr_t)W & 3) || iters < 0 || iters > 1000) return LB_ERR_INVALID_ARG;
     if (!U || !V || !h || !g || !l) return LB_ERR_INVALID_ARG;
     for (int p = 0; p < npaths; ++p)
         if (!U[p] || !V[p] || !h[p] || !g[p] || !l[p]) return LB_ERR_INVALID_ARG;
-    const InitPlan P = make_plan(N, K, r);
+    const InitPlan P = make_plan(N, K, r, itq != nullptr);
     if (!workspace || ((uintptr_t)workspace & 255) || workspace_bytes < P.total * sizeof(double))
         return LB_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
@@ -505,11 +702,50 @@ extern "C" LB_API lb_status lb_dual_svid_init(const float *W, int N, int K, int 
     f32_to_f64_kernel<<<grid_for((long)N * K), kT, 0, s>>>(W, N, K, c.at(P.o_Wd), P.ldK);
     for (int p = 0; p < npaths && e == cudaSuccess; ++p)
         e = one_path(c, iters, kSeed + (uint64_t)p, U[p], V[p], h[p], g[p], l[p],
-                     sigma ? sigma + (size_t)p * r : nullptr, p + 1 < npaths, bar, err, ord, flip);
+                     sigma ? sigma + (size_t)p * r : nullptr, p + 1 < npaths, bar, err, ord, flip, itq, p);
     if (e != cudaSuccess) return LB_ERR_CUDA;
     int herr = 0;
     if (cudaMemcpyAsync(&herr, err, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return LB_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return LB_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return LB_ERR_CUDA;
     return herr ? LB_ERR_TIMEOUT : LB_OK;
+}
+
+}  // namespace
+}  // namespace lb
+
+extern "C" LB_API lb_status lb_dual_svid_init(const float *W, int N, int K, int r, int npaths, int iters,
+                                              uint32_t *const *U, uint32_t *const *V, float *const *h,
+                                              float *const *g, float *const *l, float *sigma, void *workspace,
+                                              size_t workspace_bytes, void *stream)
+{
+    return lb::run_init(W, N, K, r, npaths, iters, U, V, h, g, l, sigma, workspace, workspace_bytes, stream, nullptr);
+}
+
+extern "C" LB_API size_t lb_littlebit2_workspace_bytes(int N, int K, int r)
+{
+    if (N < 1 || K < 1 || r < 1 || r > std::min(N, K) || r > LB_MAX_RANK) return 0;
+    return lb::make_plan(N, K, r, true).total * sizeof(double);
+}
+
+extern "C" LB_API lb_status lb_littlebit2_init(const float *W, int N, int K, int r, int npaths, int iters,
+                                               int itq_iters, const double *const *R0, uint32_t *const *U,
+                                               uint32_t *const *V, float *const *h, float *const *g,
+                                               float *const *l, float *sigma, double *itq_loss, double *const *R_out,
+                                               void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (itq_iters < 0 || itq_iters > 1000) return LB_ERR_INVALID_ARG;
+    if (npaths == 1 || npaths == 2) {
+        for (int p = 0; p < npaths; ++p) {
+            if (R0 && R0[p] && ((uintptr_t)R0[p] & 7)) return LB_ERR_INVALID_ARG;
+            if (R_out && R_out[p] && ((uintptr_t)R_out[p] & 7)) return LB_ERR_INVALID_ARG;
+        }
+    }
+    if ((uintptr_t)itq_loss & 7) return LB_ERR_INVALID_ARG;
+    lb::ItqArgs a;
+    a.iters = itq_iters;
+    a.R0 = R0;
+    a.loss = itq_loss;
+    a.Rout = R_out;
+    return lb::run_init(W, N, K, r, npaths, iters, U, V, h, g, l, sigma, workspace, workspace_bytes, stream, &a);
 }

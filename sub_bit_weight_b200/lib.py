@@ -63,6 +63,9 @@ _sig("lb_backward_destroy", None, [_vp])
 _sig("lb_layer_backward", _st, [_vp, _vp, _vp, _i] + [ctypes.POINTER(_vp)] * 2 + [_vp] + [ctypes.POINTER(_vp)] * 5 + [_vp])
 _sig("lb_backward_status", _st, [_vp, _vp])
 _sig("lb_dual_svid_init", _st, [_vp, _i, _i, _i, _i, _i] + [ctypes.POINTER(_vp)] * 5 + [_vp, _vp, ctypes.c_size_t, _vp])
+_sig("lb_littlebit2_workspace_bytes", ctypes.c_size_t, [_i, _i, _i])
+_sig("lb_littlebit2_init", _st, [_vp, _i, _i, _i, _i, _i, _i] + [ctypes.POINTER(_vp)] * 6 +
+     [_vp, _vp, ctypes.POINTER(_vp), _vp, ctypes.c_size_t, _vp])
 
 
 class LittleBitError(RuntimeError):
@@ -322,6 +325,62 @@ def lb_dual_svid_init(W: torch.Tensor, r: int, npaths: int = 2, iters: int = 24,
                                   _dev(sigma, torch.float32, "sigma"), _dev(workspace, torch.uint8, "workspace"),
                                   workspace.numel(), _stream(stream)), "lb_dual_svid_init")
     return DualSvidResult(U, V, h, g, l, sigma)
+
+
+def lb_littlebit2_workspace_bytes(N: int, K: int, r: int) -> int:
+    return int(_lib.lb_littlebit2_workspace_bytes(N, K, r))
+
+
+class LittleBit2Result(DualSvidResult):
+    """Outputs of ``lb_littlebit2_init``: those of Dual-SVID plus the ITQ loss [npaths, itq_iters + 1] and R."""
+
+    def __init__(self, U, V, h, g, l, sigma, itq_loss, R):
+        super().__init__(U, V, h, g, l, sigma)
+        self.itq_loss, self.R = itq_loss, R
+
+
+def lb_littlebit2_init(W: torch.Tensor, r: int, npaths: int = 2, iters: int = 24, itq_iters: int = 50,
+                       R0: list | None = None, workspace: torch.Tensor | None = None, stream=None) -> LittleBit2Result:
+    """LittleBit-2 initialisation (Joint-ITQ latent rotation, then Dual-SVID + residual) of a dense float32 W (CUDA).
+
+    ``R0``: None (identity starts) or a list of npaths float64 CUDA [r, r] orthogonal matrices (or None entries).
+    Allocates the outputs (and the workspace unless one is passed).  The call waits for its stream.
+    """
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D [N, K]")
+    N, K = W.shape
+    need = lb_littlebit2_workspace_bytes(N, K, r)
+    if need == 0:
+        raise ValueError(f"invalid shape N={N} K={K} r={r}")
+    dev = W.device
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    wpr = (r + 31) // 32
+    U = [torch.empty((N, wpr), dtype=torch.int32, device=dev) for _ in range(npaths)]
+    V = [torch.empty((K, wpr), dtype=torch.int32, device=dev) for _ in range(npaths)]
+    h = [torch.empty(N, dtype=torch.float32, device=dev) for _ in range(npaths)]
+    g = [torch.empty(K, dtype=torch.float32, device=dev) for _ in range(npaths)]
+    l = [torch.empty(r, dtype=torch.float32, device=dev) for _ in range(npaths)]
+    sigma = torch.empty((npaths, r), dtype=torch.float32, device=dev)
+    loss = torch.empty((npaths, itq_iters + 1), dtype=torch.float64, device=dev)
+    R = [torch.empty((r, r), dtype=torch.float64, device=dev) for _ in range(npaths)]
+
+    def arr(lst, dtype, name):
+        return (_vp * max(1, len(lst)))(*[None if t is None else _dev(t, dtype, f"{name}[{p}]")
+                                          for p, t in enumerate(lst)])
+
+    r0 = None
+    if R0 is not None:
+        if len(R0) != npaths or any(t is not None and tuple(t.shape) != (r, r) for t in R0):
+            raise ValueError("R0 must hold npaths [r, r] matrices (or None entries)")
+        r0 = arr(list(R0), torch.float64, "R0")
+    _check(_lib.lb_littlebit2_init(_dev(W, torch.float32, "W"), N, K, r, npaths, iters, itq_iters, r0,
+                                   arr(U, torch.int32, "U"), arr(V, torch.int32, "V"), arr(h, torch.float32, "h"),
+                                   arr(g, torch.float32, "g"), arr(l, torch.float32, "l"),
+                                   _dev(sigma, torch.float32, "sigma"), _dev(loss, torch.float64, "itq_loss"),
+                                   arr(R, torch.float64, "R"), _dev(workspace, torch.uint8, "workspace"),
+                                   workspace.numel(), _stream(stream)), "lb_littlebit2_init")
+    return LittleBit2Result(U, V, h, g, l, sigma, loss, R)
 
 
 # ---------------------------------------------------------------------------

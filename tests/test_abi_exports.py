@@ -34,7 +34,8 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("lb_pack_signs", "lb_layer_create", "lb_linear_forward", "lb_layer_destroy",
                      "lb_stack_create", "lb_stack_forward", "lb_stack_destroy", "lb_layer_bpw",
-                     "lb_dual_svid_workspace_bytes", "lb_dual_svid_init"):
+                     "lb_dual_svid_workspace_bytes", "lb_dual_svid_init", "lb_littlebit2_workspace_bytes",
+                     "lb_littlebit2_init"):
         assert required in names
 
 
@@ -99,6 +100,22 @@ def test_initialisation_argument_checks(lib):
     assert lib.lb_dual_svid_init(vp(256), 96, 40, 6, 1, 24, *args, None, vp(264), ws, None) == 1   # misaligned
     nulls = (vp * 1)(None)
     assert lib.lb_dual_svid_init(vp(256), 96, 40, 6, 1, 24, nulls, *args[1:], None, vp(256), ws, None) == 1
+    # LittleBit-2 (Joint-ITQ) variant: its own workspace size, the same checks plus its own arguments
+    lib.lb_littlebit2_workspace_bytes.restype = ctypes.c_size_t
+    lib.lb_littlebit2_workspace_bytes.argtypes = [i, i, i]
+    assert lib.lb_littlebit2_workspace_bytes(8, 8, 9) == 0
+    ws2 = lib.lb_littlebit2_workspace_bytes(96, 40, 6)
+    assert ws2 > ws
+    P = ctypes.POINTER(vp)
+    lib.lb_littlebit2_init.argtypes = [vp, i, i, i, i, i, i] + [P] * 6 + [vp, vp, P, vp, ctypes.c_size_t, vp]
+    call = lambda it, R0=None, loss=None, w=ws2, npaths=1: lib.lb_littlebit2_init(
+        vp(256), 96, 40, 6, npaths, 24, it, R0, *args, None, loss, None, vp(256), w, None)
+    assert call(-1) == 1                                         # itq_iters
+    assert call(1001) == 1
+    assert call(50, npaths=3) == 2
+    assert call(50, w=ws) == 1                                   # the Dual-SVID workspace is too small
+    assert call(50, R0=(vp * 1)(vp(260))) == 1                   # misaligned R0
+    assert call(50, loss=vp(260)) == 1                           # misaligned loss
 
 
 def test_backward_argument_checks(lib):
@@ -121,3 +138,4 @@ def test_backward_argument_checks(lib):
     assert len(binding._lib.lb_layer_backward.argtypes) == 13
     assert len(binding._lib.lb_backward_create.argtypes) == 11
     assert len(binding._lib.lb_dual_svid_init.argtypes) == 15
+    assert len(binding._lib.lb_littlebit2_init.argtypes) == 19
