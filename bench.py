@@ -40,6 +40,7 @@ PREFILL_DEFAULT = "llama2_13b_0.3_prefill"
 INIT_DEFAULT = "llama2_7b_0.1"
 BACKWARD_DEFAULT = "llama2_13b_0.3_prefill"
 INIT_ITERS = 24
+ITQ_ITERS = 50          # Joint-ITQ alternations of the LittleBit-2 initialisation (iterative quantisation's usual 50)
 # binary64 FMA rate of B200: 148 SMs x 64 FP64 FMA per clock x 2 FLOP at the 1965 MHz maximum SM clock
 FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
 
@@ -544,6 +545,45 @@ def run_init(wkey: str, steps: int, warmup: int, dev, with_cpu: bool, only: str 
         out["cpu_baseline"] = {"value": round(1.0 / dt, 4), "unit": "layers/s", "cores": cores, "kind": "oracle",
                                "sample": f"one {s.name} layer {s.N}x{s.K} r={s.r}, two paths, numpy/LAPACK "
                                          f"float64 ({dt:.1f} s)"}
+
+    # LittleBit-2: the same block with the Joint-ITQ latent rotation before the binarisation (lb_littlebit2_init)
+    ws2 = torch.empty(max(lib.lb_littlebit2_workspace_bytes(s.N, s.K, s.r) for s in shapes), dtype=torch.uint8,
+                      device=dev)
+    last = []
+
+    def block2():
+        last[:] = [lib.lb_littlebit2_init(Ws[(s.N, s.K)], s.r, 2, INIT_ITERS, ITQ_ITERS, workspace=ws2)
+                   for s in shapes]
+
+    for _ in range(warmup):
+        block2()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk2:
+        e0.record()
+        for _ in range(steps):
+            block2()
+        e1.record()
+        torch.cuda.synchronize()
+    ms2 = e0.elapsed_time(e1) / steps
+    loss = np.array([r_.itq_loss.cpu().numpy() for r_ in last])       # [layer, path, ITQ_ITERS + 1]
+    lb2 = {"value": round(len(shapes) / (ms2 * 1e-3), 3), "unit": "layers/s", "higher_is_better": True,
+           "ms_per_block": round(ms2, 2), "itq_iters": ITQ_ITERS,
+           "itq_ms_per_layer": round((ms2 - ms_block) / len(shapes), 2),
+           "itq_loss_mean": {"start": round(float(loss[:, :, 0].mean()), 4),
+                             "end": round(float(loss[:, :, -1].mean()), 4)},
+           "clocks": clk2.summary()}
+    if with_cpu:
+        from oracle import littlebit2 as olb2
+        s = shapes[0]
+        W = Ws[(s.N, s.K)].cpu().numpy().astype(np.float64)
+        t = time.perf_counter()
+        olb2.littlebit2_init(W, s.r, 2, ITQ_ITERS)
+        dt = time.perf_counter() - t
+        lb2["cpu_baseline"] = {"value": round(1.0 / dt, 4), "unit": "layers/s", "cores": out["cpu_baseline"]["cores"],
+                               "kind": "oracle", "sample": f"one {s.name} layer {s.N}x{s.K} r={s.r}, two paths, "
+                                                           f"{ITQ_ITERS} ITQ alternations, numpy/LAPACK float64 "
+                                                           f"({dt:.1f} s)"}
+    out["littlebit2"] = lb2
     return out
 
 
