@@ -590,7 +590,7 @@ def run_init(wkey: str, steps: int, warmup: int, dev, with_cpu: bool, only: str 
 def backward_stage_flops(s: synth.LayerShape, M: int, npaths: int = 2):
     """Algorithmic FLOPs of the backward stages of one layer (2 FLOPs per multiply-add, no padding)."""
     R = npaths * s.r
-    return {"z = (x.g) V_s": 2.0 * M * s.K * R, "(dy.h) U_s": 2.0 * M * s.N * R, "dx": 2.0 * M * R * s.K,
+    return {"z = (x.g) V_s, (dy.h) U_s": 2.0 * M * (s.K + s.N) * R, "dx": 2.0 * M * R * s.K,
             "dy^T zl": 2.0 * M * s.N * R, "x^T dz": 2.0 * M * s.K * R}
 
 
@@ -648,7 +648,9 @@ def run_backward(wkey: str, steps: int, warmup: int, dev, with_cpu: bool, pk):
     for e in ev:
         e.record()
     torch.cuda.synchronize()
-    names = ["dy scaling", "z = (x.g) V_s", "(dy.h) U_s", "dl, dz, zl", "dx", "dy^T zl", "x^T dz", "dh, dg, dU, dV"]
+    # events 2 and 3 mark the same point: z and dzl run in one launch
+    names = ["dy scaling", "z = (x.g) V_s, (dy.h) U_s", "-", "dl, dz, zl", "dx", "dy^T zl", "x^T dz",
+             "dh, dg, dU, dV"]
     stage = {n: 0.0 for n in names}
     reps = 5
     for _ in range(reps):
@@ -661,8 +663,9 @@ def run_backward(wkey: str, steps: int, warmup: int, dev, with_cpu: bool, pk):
     sf = backward_stage_flops(big, M)
     dom = max(sf, key=lambda n: stage[n])
     ach = sf[dom] / (stage[dom] * 1e-3) / 1e12
-    kern = {"z = (x.g) V_s": "prefill_kernel<0> (latent contraction of the forward helper)",
-            "(dy.h) U_s": "prefill_kernel<0> (latent contraction of the transposed helper, fp16 input)",
+    stage.pop("-")
+    kern = {"z = (x.g) V_s, (dy.h) U_s": "prefill_kernel<0> (latent contractions of the forward and transposed "
+                                         "helpers in one launch, k-split units)",
             "dx": "prefill_kernel<1> (output contraction of the transposed helper)",
             "dy^T zl": "cuBLAS fp16 GEMM", "x^T dz": "cuBLAS fp16 GEMM"}[dom]
     out = {"workload": f"{w.key} first block: " + ", ".join(f"{s.name} {s.N}x{s.K} r={s.r}" for s in shapes)

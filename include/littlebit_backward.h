@@ -16,14 +16,16 @@
  *
  * The two binary contractions of the backward are those of the forward pass
  * of the transposed layer (U <-> V, h <-> g) and run on the same tcgen05
- * kernels; the two dense products dy^T zl (N x 2r) and x^T dz (K x 2r) are
- * plain fp16 GEMMs (cuBLAS) with float32 accumulation.
+ * kernels (z and (dy (.) h) U_s in one launch whose output tiles are split
+ * over k, partial sums added in float32); the two dense products dy^T zl
+ * (N x 2r) and x^T dz (K x 2r) are plain fp16 GEMMs (cuBLAS) with float32
+ * accumulation.
  *
  * Arithmetic: x enters as bfloat16 (converted to fp16 exactly in fp16's normal
  * range, as in the forward pass); dy is multiplied by one power of two chosen
  * on the device so that dy and (dy (.) h) U_s cannot overflow fp16, and
- * rounded to fp16; z, zl, (dy (.) h) U_s and dz are rounded to fp16 between
- * the contractions; every product accumulates in float32 and the power of two
+ * rounded to fp16; zl and dz are rounded to fp16 between the contractions (z
+ * and (dy (.) h) U_s are kept in float32); every product accumulates in float32 and the power of two
  * is divided out exactly.  Scales are the layer's binary16 values (the ones
  * its forward pass uses).
  *
@@ -69,8 +71,9 @@ LB_API void lb_backward_destroy(lb_backward *B);
  *
  * With the timing hook of littlebit.h (lb_profile_events) holding 9 events,
  * events[i] is recorded at the i-th stage boundary: 0 | dy scaling | 1 |
- * z = (x (.) g) V_s | 2 | (dy (.) h) U_s | 3 | dl, dz, zl | 4 | dx | 5 |
- * dy^T zl | 6 | x^T dz | 7 | dh, dg, dU, dV | 8. */
+ * z = (x (.) g) V_s and (dy (.) h) U_s, one launch | 2, 3 | dl, dz, zl | 4 |
+ * dx | 5 | dy^T zl | 6 | x^T dz | 7 | dh, dg, dU, dV | 8 (events 2 and 3
+ * mark the same point). */
 LB_API lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, int M,
                                    const float *const *U_lat, const float *const *V_lat, float *dx,
                                    float *const *dh, float *const *dg, float *const *dl,

@@ -11,7 +11,10 @@
 //   G_U = dy^T zl, dh = sum_j U_s (.) G_U, dU = h (.) G_U (.) 100 (1 - tanh^2(100 U))
 //   G_V = x^T dz,  dg = sum_j V_s (.) G_V, dV = g (.) G_V (.) 100 (1 - tanh^2(100 V))
 // The contractions run on the tcgen05 kernels of the forward pass (two helper
-// layers with l = 1); G_U and G_V are plain fp16 GEMMs (cuBLAS).  dy is
+// layers with l = 1): z and dzl, which are independent, in one launch whose
+// output tiles are split over k into units of even length (their fp32 partial
+// sums are added in place), dx on the output kernel.  G_U and G_V are plain
+// fp16 GEMMs (cuBLAS).  dy is
 // multiplied by one power of two 2^E, chosen on the device so that dy 2^E and
 // dzl 2^E (and dz 2^E) stay below 2^14, and divided out exactly at the end.
 #include "littlebit_backward.h"
@@ -39,6 +42,9 @@ struct lb_backward {
     int M = 0;                     // rows the scratch below holds
     __half *dy16 = nullptr;        // [M][N]
     __half *x16 = nullptr;         // [M][K]
+    float *zpart = nullptr;        // [M][K2] z from the k-split latent contraction (fp32)
+    float *dzpart = nullptr;       // [M][K2] dzl 2^E, likewise
+    lb::PfJobState *jobs = nullptr;   // the one-launch latent contractions (tensor maps, unit records)
     float *GU = nullptr;           // [N][K2]
     float *GV = nullptr;           // [K][K2]
     cublasHandle_t blas = nullptr;
@@ -159,24 +165,36 @@ __global__ void convert_kernel(const float *__restrict__ dy, long ndy, const uin
     }
 }
 
-// dl_acc[j'] += sum_m dzl[m][j'] z[m][j']; dzl <- fp16(dzl l) (= dz), z <- fp16(z l) (= zl).  One column per
-// thread, a slice of rows per CTA (blockIdx.y).
-__global__ void latent_mix_kernel(__half *dzl, __half *z, int M, int ncols, int ld, const float *__restrict__ lcat,
-                                  float *dl_acc, int rows_per)
+// dl_acc[j'] += sum_m dzl[m][j'] z[m][j'] over this CTA's rows; dz = fp16(dzl l), zl = fp16(z l).  dzl and z are
+// the fp32 sums of the k-split latent contraction.  Four columns per thread (ncols and ld are multiples of 4), a
+// slice of rows per CTA (blockIdx.y).
+__global__ void latent_mix_kernel(const float *__restrict__ dzl, const float *__restrict__ z, int M, int ncols, int ld,
+                                  const float *__restrict__ lcat, float *dl_acc, __half *dz, __half *zl, int rows_per)
 {
-    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    const int j = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
     if (j >= ncols) return;
     const int m0 = blockIdx.y * rows_per, m1 = min(M, m0 + rows_per);
-    const float lj = lcat[j];
-    float acc = 0.0f;
+    const float4 l = *reinterpret_cast<const float4 *>(lcat + j);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
     for (int m = m0; m < m1; ++m) {
         const size_t o = (size_t)m * ld + j;
-        const float a = __half2float(dzl[o]), b = __half2float(z[o]);
-        acc = fmaf(a, b, acc);
-        dzl[o] = __float2half_rn(a * lj);
-        z[o] = __float2half_rn(b * lj);
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(dzl + o));
+        const float4 b = __ldg(reinterpret_cast<const float4 *>(z + o));
+        acc.x = fmaf(a.x, b.x, acc.x);
+        acc.y = fmaf(a.y, b.y, acc.y);
+        acc.z = fmaf(a.z, b.z, acc.z);
+        acc.w = fmaf(a.w, b.w, acc.w);
+        __half2 *pd = reinterpret_cast<__half2 *>(dz + o), *pz = reinterpret_cast<__half2 *>(zl + o);
+        pd[0] = __floats2half2_rn(a.x * l.x, a.y * l.y);
+        pd[1] = __floats2half2_rn(a.z * l.z, a.w * l.w);
+        pz[0] = __floats2half2_rn(b.x * l.x, b.y * l.y);
+        pz[1] = __floats2half2_rn(b.z * l.z, b.w * l.w);
     }
-    atomicAdd(dl_acc + j, acc);
+    atomicAdd(dl_acc + j, acc.x);
+    atomicAdd(dl_acc + j + 1, acc.y);
+    atomicAdd(dl_acc + j + 2, acc.z);
+    atomicAdd(dl_acc + j + 3, acc.w);
 }
 
 __global__ void scale_kernel(float *x, long n, const float *__restrict__ stat)
@@ -205,6 +223,48 @@ struct FactorArgs {
     float *dF[2];
     float *dsc[2];
 };
+
+// 100 (1 - tanh^2(100 f))
+__device__ __forceinline__ float smooth_sign_grad(float f)
+{
+    const float ea = __expf(-200.0f * fabsf(f));
+    const float d1 = 1.0f + ea;
+    return 400.0f * ea / (d1 * d1);
+}
+
+// as factor_grad_kernel, four latent columns per lane (r a multiple of 4: rows of F, dF and G 16-byte aligned)
+template <int P>
+__global__ void __launch_bounds__(kT) factor_grad4_kernel(const float *__restrict__ G, int rows, int K2, int r, int r8,
+                                                          const FactorArgs a)
+{
+    const int lane = threadIdx.x & 31, wpr = (r + 31) / 32, r4 = r / 4;
+    for (int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < rows; i += (gridDim.x * blockDim.x) >> 5) {
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+            const float si = a.s[p][i];
+            const float4 *__restrict__ g = reinterpret_cast<const float4 *>(G + (size_t)i * K2 + p * r8);
+            const uint32_t *__restrict__ w = a.words[p] + (size_t)i * wpr;
+            const float4 *__restrict__ f = reinterpret_cast<const float4 *>(a.F[p] + (size_t)i * r);
+            float4 *__restrict__ df = reinterpret_cast<float4 *>(a.dF[p] + (size_t)i * r);
+            float acc = 0.0f;
+#pragma unroll 2
+            for (int q = lane; q < r4; q += 32) {
+                const float4 gv = __ldg(g + q), fv = __ldg(f + q);
+                const uint32_t bits = __ldg(w + (q >> 3)) >> ((4 * q) & 31);
+                acc += (bits & 1u ? -gv.x : gv.x) + (bits & 2u ? -gv.y : gv.y) + (bits & 4u ? -gv.z : gv.z) +
+                       (bits & 8u ? -gv.w : gv.w);
+                float4 o;
+                o.x = si * gv.x * smooth_sign_grad(fv.x);
+                o.y = si * gv.y * smooth_sign_grad(fv.y);
+                o.z = si * gv.z * smooth_sign_grad(fv.z);
+                o.w = si * gv.w * smooth_sign_grad(fv.w);
+                __stcs(df + q, o);
+            }
+            for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == 0) a.dsc[p][i] = acc;
+        }
+    }
+}
 
 template <int P>
 __global__ void __launch_bounds__(kT) factor_grad_kernel(const float *__restrict__ G, int rows, int K2, int r, int r8,
@@ -240,11 +300,16 @@ lb_status grow(lb_backward *B, int M, cudaStream_t s)
     if (B->M) cudaStreamSynchronize(s);
     cudaFree(B->dy16);
     cudaFree(B->x16);
+    cudaFree(B->zpart);
+    cudaFree(B->dzpart);
     B->dy16 = nullptr;
     B->x16 = nullptr;
+    B->zpart = B->dzpart = nullptr;
     B->M = 0;
     if (cudaMalloc(&B->dy16, (size_t)M * B->N * sizeof(__half)) != cudaSuccess ||
-        cudaMalloc(&B->x16, (size_t)M * B->K * sizeof(__half)) != cudaSuccess)
+        cudaMalloc(&B->x16, (size_t)M * B->K * sizeof(__half)) != cudaSuccess ||
+        cudaMalloc(&B->zpart, (size_t)M * B->K2 * sizeof(float)) != cudaSuccess ||
+        cudaMalloc(&B->dzpart, (size_t)M * B->K2 * sizeof(float)) != cudaSuccess)
         return LB_ERR_OOM;
     B->M = M;
     return LB_OK;
@@ -262,8 +327,10 @@ void lb_backward_destroy(lb_backward *B)
     if (!B) return;
     lb_layer_destroy(B->Lf);
     lb_layer_destroy(B->Lt);
+    prefill_jobs_free(B->jobs);
     for (void *p : {(void *)B->lcat, (void *)B->h32, (void *)B->g32, (void *)B->hmax, (void *)B->Uw, (void *)B->Vw,
-                    (void *)B->dl_acc, (void *)B->stat, (void *)B->dy16, (void *)B->x16, (void *)B->GU,
+                    (void *)B->dl_acc, (void *)B->stat, (void *)B->dy16, (void *)B->x16, (void *)B->zpart,
+                    (void *)B->dzpart, (void *)B->GU,
                     (void *)B->GV})
         cudaFree(p);
     if (B->blas) cublasDestroy(B->blas);
@@ -349,8 +416,8 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
     const int N = B->N, K = B->K, r = B->r, K2 = B->K2;
     int launches = 0;
 
-    // timing hook (littlebit.h): events 0 | scaling | 1 | z | 2 | dzl | 3 | dl, dz, zl | 4 | dx | 5 | G_U | 6 | G_V | 7
-    // | factor gradients | 8
+    // timing hook (littlebit.h): events 0 | scaling | 1 | z and dzl (one launch) | 2, 3 | dl, dz, zl | 4 | dx | 5 |
+    // G_U | 6 | G_V | 7 | factor gradients | 8
     profile_mark(0, s);
     // dy scale (device-side exponent), fp16 copies of dy 2^E and x
     cudaMemsetAsync(B->stat, 0, sizeof(float), s);
@@ -362,22 +429,28 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
     launches += 3;
     profile_mark(1, s);
 
-    // z (forward latent, l = 1) and dzl 2^E (transposed latent, l = 1); the y map of the forward helper is never
-    // used (its output contraction is not run), dx only stands in for a well-aligned pointer there
+    // z (forward latent, l = 1) and dzl 2^E (transposed latent, l = 1), both in one launch with k-split units
+    // adding into zeroed fp32 buffers.  The two helpers' plans are set up first (no launch): they own the fp16
+    // buffers of zl and dz and the maps of the dx contraction.  The y map of the forward helper is never used (its
+    // output contraction is not run); dx only stands in for a well-aligned pointer there.
     const uint16_t *xs[1] = {x};
     const uint16_t *dys[1] = {reinterpret_cast<const uint16_t *>(B->dy16)};
     float *ys[1] = {dx};
-    if ((st = prefill_forward(B->Lf->self->plan, &B->Lf, xs, ys, M, s, &launches, 1, false, false)) != LB_OK) return st;
-    profile_mark(2, s);
-    if ((st = prefill_forward(B->Lt->self->plan, &B->Lt, dys, ys, M, s, &launches, 1, true, false)) != LB_OK) return st;
-    profile_mark(3, s);
+    if ((st = prefill_forward(B->Lf->self->plan, &B->Lf, xs, ys, M, s, &launches, 0, false, false)) != LB_OK) return st;
+    if ((st = prefill_forward(B->Lt->self->plan, &B->Lt, dys, ys, M, s, &launches, 0, true, false)) != LB_OK) return st;
     __half *zf = prefill_zl(B->Lf->self->plan, 0), *dz = prefill_zl(B->Lt->self->plan, 0);
     if (!zf || !dz) return LB_ERR_CUDA;
+    cudaMemsetAsync(B->zpart, 0, (size_t)M * K2 * sizeof(float), s);
+    cudaMemsetAsync(B->dzpart, 0, (size_t)M * K2 * sizeof(float), s);
+    const PfLatentJob jobs[2] = {{B->Lf, x, false, B->zpart, K2}, {B->Lt, B->dy16, true, B->dzpart, K2}};
+    if ((st = prefill_latent_jobs(&B->jobs, jobs, 2, M, s, &launches)) != LB_OK) return st;
+    profile_mark(2, s);
+    profile_mark(3, s);
 
     // dl, dz = dzl l, zl = z l
-    const int ncols = B->npaths * B->r8, rows_per = 64;
-    latent_mix_kernel<<<dim3((ncols + kT - 1) / kT, (M + rows_per - 1) / rows_per), kT, 0, s>>>(
-        dz, zf, M, ncols, K2, B->lcat, B->dl_acc, rows_per);
+    const int ncols = B->npaths * B->r8, rows_per = 16, mix_t = 128;
+    latent_mix_kernel<<<dim3((ncols / 4 + mix_t - 1) / mix_t, (M + rows_per - 1) / rows_per), mix_t, 0, s>>>(
+        B->dzpart, B->zpart, M, ncols, K2, B->lcat, B->dl_acc, dz, zf, rows_per);
     dl_out_kernel<<<grid_for(r), kT, 0, s>>>(B->dl_acc, r, B->r8, B->stat, dl[0], B->npaths > 1 ? dl[1] : nullptr);
     profile_mark(4, s);
     // dx 2^E = sum_p g (.) (dz 2^E V_s^T)
@@ -411,7 +484,18 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
         fv.dF[p] = dV[p];
         fv.dsc[p] = dg[p];
     }
-    if (B->npaths == 2) {
+    bool vec4 = r % 4 == 0;
+    for (int p = 0; p < B->npaths; ++p)
+        vec4 = vec4 && !(((uintptr_t)U_lat[p] | (uintptr_t)V_lat[p] | (uintptr_t)dU[p] | (uintptr_t)dV[p]) & 15);
+    if (vec4) {
+        if (B->npaths == 2) {
+            factor_grad4_kernel<2><<<grid_for(32L * N), kT, 0, s>>>(B->GU, N, K2, r, B->r8, fu);
+            factor_grad4_kernel<2><<<grid_for(32L * K), kT, 0, s>>>(B->GV, K, K2, r, B->r8, fv);
+        } else {
+            factor_grad4_kernel<1><<<grid_for(32L * N), kT, 0, s>>>(B->GU, N, K2, r, B->r8, fu);
+            factor_grad4_kernel<1><<<grid_for(32L * K), kT, 0, s>>>(B->GV, K, K2, r, B->r8, fv);
+        }
+    } else if (B->npaths == 2) {
         factor_grad_kernel<2><<<grid_for(32L * N), kT, 0, s>>>(B->GU, N, K2, r, B->r8, fu);
         factor_grad_kernel<2><<<grid_for(32L * K), kT, 0, s>>>(B->GV, K, K2, r, B->r8, fv);
     } else {
@@ -428,7 +512,20 @@ lb_status lb_backward_status(lb_backward *B, void *stream)
 {
     if (!B) return LB_ERR_INVALID_ARG;
     lb_status a = lb_layer_status(B->Lf, stream), b = lb_layer_status(B->Lt, stream);
-    return a != LB_OK ? a : b;
+    lb_status c = LB_OK;
+    if (int *e = prefill_jobs_err(B->jobs)) {
+        cudaStream_t s = (cudaStream_t)stream;
+        int h = 0;
+        if (cudaMemcpyAsync(&h, e, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return LB_ERR_CUDA;
+        if (h) {
+            cudaMemsetAsync(e, 0, sizeof(int), s);
+            cudaStreamSynchronize(s);
+            c = LB_ERR_TIMEOUT;
+        }
+    }
+    return a != LB_OK ? a : b != LB_OK ? b : c;
 }
 
 }  // extern "C"

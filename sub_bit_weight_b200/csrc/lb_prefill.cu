@@ -399,17 +399,24 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
     const uint32_t tmem = S.tmem_base;
     const int total = S.tile_start[nlayers];
 
-    auto locate = [&](int t, int &L, int &mt, int &nt) {
+    // unit t -> layer L, tile (mt, nt) and k-blocks [kb0, kb1); the k-range index is the slowest, so the units of
+    // one tile fall in different waves
+    const int mtiles = (M + kPfBM - 1) / kPfBM;
+    auto locate = [&](int t, int &L, int &mt, int &nt, int &kb0, int &kb1) {
         int lo = 0, hi = nlayers - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
             if (S.tile_start[mid] <= t) lo = mid; else hi = mid - 1;
         }
         L = lo;
-        const int local = t - S.tile_start[lo];
-        const int ntn = layers[lo].ntn;
+        int local = t - S.tile_start[lo];
+        const int ntn = layers[lo].ntn, nsp = layers[lo].ksplit, nk = layers[lo].nk;
+        const int ks = local / (mtiles * ntn);
+        local -= ks * mtiles * ntn;
         mt = local / ntn;
         nt = local - mt * ntn;
+        kb0 = ks * nk / nsp;
+        kb1 = (ks + 1) * nk / nsp;
     };
 
     if (warp == 0) {
@@ -418,11 +425,11 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
             uint32_t it = 0;
             uint32_t pend = 0, pend_ph = 0;   // stages with a copy issued, and its phase parity
             for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-                int L, mt, nt;
-                locate(t, L, mt, nt);
+                int L, mt, nt, kb0, kb1;
+                locate(t, L, mt, nt, kb0, kb1);
                 const PfLayer ly = layers[L];   // register copy: waits below clobber memory
                 const uint32_t *bits = ly.bits + (size_t)nt * ly.nk * 1024;
-                for (int kb = 0; kb < ly.nk; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % kPfStages;
                     const uint32_t ph = (it / kPfStages) & 1;
                     if (!mbar_wait(&S.empty[s], ph ^ 1, abort, err, 1)) break;
@@ -449,8 +456,8 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
         if (lane == 0) {
             uint32_t it = 0, tcount = 0;
             for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x, ++tcount) {
-                int L, mt, nt;
-                locate(t, L, mt, nt);
+                int L, mt, nt, kb0, kb1;
+                locate(t, L, mt, nt, kb0, kb1);
                 const PfLayer ly = layers[L];   // register copy: waits below clobber memory
                 const int nw = min(kPfBN, ly.ncols - nt * kPfBN);
                 const int ab = tcount & 1;
@@ -460,7 +467,7 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
                 const uint32_t idesc = idesc_f16((nw + 15) & ~15);
                 const uint32_t dacc = tmem + (uint32_t)(ab * kPfBN);
                 bool ok = true;
-                for (int kb = 0; kb < ly.nk; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % kPfStages;
                     const uint32_t ph = (it / kPfStages) & 1;
                     if (!mbar_wait(&S.full[s], ph, abort, err, 3) || !mbar_wait(&S.ready[s], ph, abort, err, 4)) {
@@ -472,7 +479,7 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
                     const uint64_t bd = smem_desc_sw128(S.B[s]);
 #pragma unroll
                     for (int kk = 0; kk < kPfBK / 16; ++kk)
-                        tc_mma_f16(dacc, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+                        tc_mma_f16(dacc, ad + 2 * kk, bd + 2 * kk, idesc, (kb > kb0 || kk) ? 1u : 0u);
                     tc_commit(&S.empty[s]);
                 }
                 if (!ok) break;
@@ -486,11 +493,11 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
             const int ct = warp < 16 ? tid - 64 : tid - 512 + 64;   // 0 .. kConv - 1
             uint32_t it = 0;
             for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-                int L, mt, nt;
-                locate(t, L, mt, nt);
-                const int nk = layers[L].nk, a_f16 = layers[L].a_f16;
+                int L, mt, nt, kb0, kb1;
+                locate(t, L, mt, nt, kb0, kb1);
+                const int a_f16 = layers[L].a_f16;
                 bool ok = true;
-                for (int kb = 0; kb < nk; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % kPfStages;
                     const uint32_t ph = (it / kPfStages) & 1;
                     if (!mbar_wait(&S.full[s], ph, abort, err, 7)) {
@@ -521,15 +528,15 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
         const int q = warp - 4;
         uint32_t tcount = 0;
         for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x, ++tcount) {
-            int L, mt, nt;
-            locate(t, L, mt, nt);
+            int L, mt, nt, kb0, kb1;
+            locate(t, L, mt, nt, kb0, kb1);
             const PfLayer ly = layers[L];   // register copy: waits below clobber memory
             const int nw = min(kPfBN, ly.ncols - nt * kPfBN);
             const int ab = tcount & 1;
             const uint32_t aph = (tcount >> 1) & 1;
             if (!mbar_wait(&S.accf[ab], aph, abort, err, 5)) break;
             tc_fence_after();
-            if (MODE == 0) {
+            if (MODE == 0 && !ly.part) {
                 // l of this tile's columns into shared memory (the 4 epilogue warps, named barrier 1)
                 asm volatile("bar.sync 1, 128;\n" ::: "memory");   // previous tile done with S.lsc
                 for (int i = tid - 128; i < kPfBN; i += 128) {
@@ -543,7 +550,19 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
                 uint32_t v[32];
                 tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * kPfBN + ch), v);
                 const int c0 = nt * kPfBN + ch;
-                if (MODE == 0) {
+                if (MODE == 0 && ly.part) {
+                    // k-split unit: add the raw partial sums (fp32) to the caller's zeroed buffer
+                    if (m < M) {
+                        float *o = ly.part + (size_t)m * ly.ld_part + c0;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            if (c0 + 4 * i < ly.ncols)
+                                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(o + 4 * i),
+                                             "f"(__uint_as_float(v[4 * i])), "f"(__uint_as_float(v[4 * i + 1])),
+                                             "f"(__uint_as_float(v[4 * i + 2])), "f"(__uint_as_float(v[4 * i + 3]))
+                                             : "memory");
+                    }
+                } else if (MODE == 0) {
                     if (m < M) {
                         __half *out = reinterpret_cast<__half *>(ly.out) + (size_t)m * ly.ld_out + c0;
                         uint32_t hw[16];
@@ -600,8 +619,8 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
         const int gw = warp - 8;
         uint32_t it = 0;
         for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-            int L, mt, nt;
-            locate(t, L, mt, nt);
+            int L, mt, nt, kb0, kb1;
+            locate(t, L, mt, nt, kb0, kb1);
             const PfLayer ly = layers[L];   // register copy: waits below clobber memory
             const int nw = min(kPfBN, ly.ncols - nt * kPfBN);
             // output contraction: this thread's row n and its two path scales
@@ -617,7 +636,7 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
                 }
             }
             bool ok = true;
-            for (int kb = 0; kb < ly.nk; ++kb, ++it) {
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 const int s = it % kPfStages;
                 const uint32_t ph = (it / kPfStages) & 1;
                 if (!mbar_wait(&S.full[s], ph, abort, err, 6)) {
@@ -759,6 +778,34 @@ void prefill_free(PrefillState *st)
 
 static size_t smem_bytes(int nlayers) { return sizeof(PfSmem) + 1024 + sizeof(int) * (size_t)(nlayers + 1); }
 
+static int sm_count()
+{
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    return sms;
+}
+
+// raise the kernels' dynamic shared-memory limit to at least `smem` (grow-only, shared by every launch path)
+static cudaError_t ensure_smem(size_t smem)
+{
+    static size_t smem_set = 0;
+    if (smem > 232448) return cudaErrorInvalidValue;
+    if (smem <= smem_set) return cudaSuccess;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(prefill_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+        cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(prefill_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+        cudaSuccess)
+        return e;
+    smem_set = smem;
+    return cudaSuccess;
+}
+
 lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const uint16_t *const *xs,
                           float *const *ys, int M, cudaStream_t s, int *launches, int parts, bool a_f16,
                           bool marks)
@@ -839,6 +886,9 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
             a.base_ld = W.K64;
             a.npaths = d.npaths;
             a.a_f16 = a_f16;
+            a.ksplit = 1;
+            a.part = nullptr;
+            a.ld_part = 0;
             PfLayer &b = rec[n + i];
             b.tmA = st.maps + n + i;
             b.tmY = st.maps + 2 * n + i;
@@ -854,6 +904,9 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
             b.base_ld = W.N256;
             b.npaths = d.npaths;
             b.a_f16 = 0;
+            b.ksplit = 1;
+            b.part = nullptr;
+            b.ld_part = 0;
             starts[i + 1] = starts[i] + mtiles * a.ntn;
             starts[n + 1 + i + 1] = starts[n + 1 + i] + mtiles * b.ntn;
             st.lastX[i] = xs[i];
@@ -875,22 +928,9 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
         if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return status_from(e);
     }
 
-    static int sms = 0;
-    static size_t smem_set = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    }
+    const int sms = sm_count();
     const size_t smem = smem_bytes(n);
-    if (smem > 232448) return LB_ERR_UNSUPPORTED;
-    if (smem > smem_set) {
-        if ((e = cudaFuncSetAttribute(prefill_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
-            return status_from(e);
-        if ((e = cudaFuncSetAttribute(prefill_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
-            return status_from(e);
-        smem_set = smem;
-    }
+    if ((e = ensure_smem(smem)) != cudaSuccess) return smem > 232448 ? LB_ERR_UNSUPPORTED : status_from(e);
     const int g0 = std::max(1, std::min(st.tiles[0], sms));
     const int g1 = std::max(1, std::min(st.tiles[1], sms));
     if (marks) profile_mark(0, s);
@@ -913,4 +953,168 @@ __half *prefill_zl(const Plan &P, int i)
     return (__half *)((char *)P.pf->zl + P.pf->zl_off[i]);
 }
 
+// ---------------------------------------------------------------------------
+// Latent contractions of several layers with k-split units (one launch)
+// ---------------------------------------------------------------------------
+struct PfJobState {
+    int n = 0, lastM = -1;
+    std::vector<const void *> lastX;
+    std::vector<float *> lastPart;
+    std::vector<int> lastF16;
+    CUtensorMap *maps = nullptr;   // device [n]
+    PfLayer *rec = nullptr;        // device [n]
+    int *starts = nullptr;         // device [n + 1]
+    int *err = nullptr;
+    int total = 0;
+};
+
+void prefill_jobs_free(PfJobState *st)
+{
+    if (!st) return;
+    cudaFree(st->maps);
+    cudaFree(st->rec);
+    cudaFree(st->starts);
+    cudaFree(st->err);
+    delete st;
+}
+
+int *prefill_jobs_err(PfJobState *st) { return st ? st->err : nullptr; }
+
+// k-ranges per tile for each job so that the kernel's round-robin assignment of units to `grid` CTAs finishes
+// evenly: every target unit length u is tried, job i gets round(nk_i / u) ranges, and the unit costs (k-blocks +
+// a fixed per-unit overhead) are dealt out in the kernel's order; the smallest makespan wins.
+static std::vector<int> choose_splits(const std::vector<int> &tiles, const std::vector<int> &nk, int sms)
+{
+    const int n = (int)tiles.size();
+    const double overhead = 3.0;      // pipeline fill and epilogue of a unit, in k-blocks
+    int maxnk = 1;
+    for (int v : nk) maxnk = std::max(maxnk, v);
+    std::vector<int> best(n, 1), cur(n);
+    double best_t = 1e300;
+    std::vector<double> load;
+    for (int u = 1; u <= maxnk; ++u) {
+        long units = 0;
+        for (int i = 0; i < n; ++i) {
+            cur[i] = std::max(1, std::min(nk[i], (nk[i] + u / 2) / u));
+            units += (long)tiles[i] * cur[i];
+        }
+        const int grid = (int)std::min<long>(units, sms);
+        load.assign(grid, 0.0);
+        long t = 0;
+        for (int i = 0; i < n; ++i)
+            for (int ks = 0; ks < cur[i]; ++ks) {
+                const double c = (ks + 1) * nk[i] / cur[i] - ks * nk[i] / cur[i] + overhead;
+                for (int k = 0; k < tiles[i]; ++k, ++t) load[t % grid] += c;
+            }
+        double mk = 0.0;
+        for (double v : load) mk = std::max(mk, v);
+        if (mk < best_t - 1e-9) {
+            best_t = mk;
+            best = cur;
+        }
+    }
+    return best;
+}
+
+lb_status prefill_latent_jobs(PfJobState **state, const PfLatentJob *jobs, int n, int M, cudaStream_t s,
+                              int *launches)
+{
+    if (!state || !jobs || n < 1 || M < 1) return LB_ERR_INVALID_ARG;
+    cudaError_t e = get_encoder();
+    if (e != cudaSuccess) return LB_ERR_UNSUPPORTED;
+    for (int i = 0; i < n; ++i) {
+        if (!jobs[i].layer || !jobs[i].x || !jobs[i].part || jobs[i].ld_part < jobs[i].layer->pf.N1p ||
+            (jobs[i].ld_part & 3) || ((uintptr_t)jobs[i].part & 15))
+            return LB_ERR_INVALID_ARG;
+        if (jobs[i].layer->d.K % 8) return LB_ERR_UNSUPPORTED;
+    }
+    if (!*state) {
+        PfJobState *st = new (std::nothrow) PfJobState();
+        if (!st) return LB_ERR_OOM;
+        st->n = n;
+        if (cudaMalloc(&st->maps, sizeof(CUtensorMap) * n) != cudaSuccess ||
+            cudaMalloc(&st->rec, sizeof(PfLayer) * n) != cudaSuccess ||
+            cudaMalloc(&st->starts, sizeof(int) * (n + 1)) != cudaSuccess ||
+            cudaMalloc(&st->err, sizeof(int)) != cudaSuccess || cudaMemsetAsync(st->err, 0, sizeof(int), s) != cudaSuccess) {
+            prefill_jobs_free(st);
+            return LB_ERR_OOM;
+        }
+        *state = st;
+    }
+    PfJobState &st = **state;
+    if (st.n != n) return LB_ERR_INVALID_ARG;
+    bool dirty = st.lastM != M || (int)st.lastX.size() != n;
+    for (int i = 0; i < n && !dirty; ++i)
+        dirty = st.lastX[i] != jobs[i].x || st.lastPart[i] != jobs[i].part || st.lastF16[i] != (int)jobs[i].a_f16;
+    const int sms = sm_count();
+    if (dirty) {
+        // longest contraction first: the round-robin deal then starts with the long units
+        std::vector<int> ord(n);
+        for (int i = 0; i < n; ++i) ord[i] = i;
+        std::stable_sort(ord.begin(), ord.end(),
+                         [&](int a, int b) { return jobs[a].layer->pf.KB1 > jobs[b].layer->pf.KB1; });
+        const int mtiles = ceil_div(M, kPfBM);
+        std::vector<int> tiles(n), nk(n);
+        for (int q = 0; q < n; ++q) {
+            const PfWeights &W = jobs[ord[q]].layer->pf;
+            tiles[q] = mtiles * ceil_div(W.N1p, kPfBN);
+            nk[q] = W.KB1;
+        }
+        const std::vector<int> split = choose_splits(tiles, nk, sms);
+        std::vector<CUtensorMap> maps(n);
+        std::vector<PfLayer> rec(n);
+        std::vector<int> starts(n + 1, 0);
+        for (int q = 0; q < n; ++q) {
+            const PfLatentJob &j = jobs[ord[q]];
+            const LayerDev &d = j.layer->d;
+            const PfWeights &W = j.layer->pf;
+            if (!encode_2d(&maps[q], j.a_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, j.x,
+                           d.K, M))
+                return LB_ERR_UNSUPPORTED;
+            PfLayer &a = rec[q];
+            a.tmA = st.maps + q;
+            a.tmY = nullptr;
+            a.bits = W.b1;
+            a.base = W.g64;
+            a.lcat = W.lcat;
+            a.out = nullptr;
+            a.nk = W.KB1;
+            a.ncols = W.N1p;
+            a.ld_out = W.K2;
+            a.ntn = ceil_div(W.N1p, kPfBN);
+            a.r8 = W.r8;
+            a.base_ld = W.K64;
+            a.npaths = d.npaths;
+            a.a_f16 = j.a_f16;
+            a.ksplit = split[q];
+            a.part = j.part;
+            a.ld_part = j.ld_part;
+            starts[q + 1] = starts[q] + tiles[q] * split[q];
+        }
+        if ((e = cudaMemcpyAsync(st.maps, maps.data(), sizeof(CUtensorMap) * n, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(st.rec, rec.data(), sizeof(PfLayer) * n, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(st.starts, starts.data(), sizeof(int) * (n + 1), cudaMemcpyHostToDevice, s)) !=
+                cudaSuccess ||
+            (e = cudaStreamSynchronize(s)) != cudaSuccess)
+            return status_from(e);
+        st.total = starts[n];
+        st.lastM = M;
+        st.lastX.assign(n, nullptr);
+        st.lastPart.assign(n, nullptr);
+        st.lastF16.assign(n, 0);
+        for (int i = 0; i < n; ++i) {
+            st.lastX[i] = jobs[i].x;
+            st.lastPart[i] = jobs[i].part;
+            st.lastF16[i] = jobs[i].a_f16;
+        }
+    }
+    const size_t smem = smem_bytes(n);
+    if ((e = ensure_smem(smem)) != cudaSuccess) return smem > 232448 ? LB_ERR_UNSUPPORTED : status_from(e);
+    const int grid = std::max(1, std::min(st.total, sms));
+    prefill_kernel<0><<<grid, pf_threads(0), smem, s>>>(st.rec, st.starts, n, M, st.err);
+    ++*launches;
+    return status_from(cudaGetLastError());
+}
+
 }  // namespace lb
+

@@ -31,4 +31,21 @@ __half *prefill_zl(const Plan &P, int i);
 void prefill_free(PrefillState *st);
 int *prefill_err_ptr(PrefillState *st);
 
+// Latent contractions of several layers in one launch, each output tile split over k into units whose raw fp32
+// partial sums are added (red.global.add) into the job's zeroed `part` [M][ld_part] (no l, no fp16 rounding).  The
+// split is chosen so that the units spread evenly over the SMs.  `state` caches tensor maps and records between
+// calls (create on first use, free with prefill_jobs_free).
+struct PfLatentJob {
+    const lb_layer *layer;
+    const void *x;        // activations [M][K], bf16 or (a_f16) fp16, 16-byte aligned
+    bool a_f16;
+    float *part;          // fp32 [M][ld_part], ld_part >= the layer's padded latent width, 16-byte aligned
+    int ld_part;
+};
+struct PfJobState;
+lb_status prefill_latent_jobs(PfJobState **state, const PfLatentJob *jobs, int n, int M, cudaStream_t s,
+                              int *launches);
+void prefill_jobs_free(PfJobState *st);
+int *prefill_jobs_err(PfJobState *st);
+
 }  // namespace lb

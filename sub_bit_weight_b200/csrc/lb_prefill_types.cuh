@@ -40,6 +40,10 @@ struct PfLayer {
     int base_ld;              // row stride of base (K64 or N256)
     int npaths;
     int a_f16;                // latent contraction: A is already fp16 (no bf16 conversion)
+    int ksplit;               // k-ranges per output tile (units of work); 1 = whole contraction per tile
+    float *part;              // latent contraction with ksplit: fp32 [M][ld_part] that each unit adds its raw
+                              // partial sums to (no l; zeroed by the caller); null = the fp16 zl epilogue
+    int ld_part;
 };
 
 }  // namespace lb
