@@ -105,7 +105,8 @@ LB_API lb_status lb_dual_svid_init(const float *W, int N, int K, int r, int npat
  *   - ITQ (Gong and Lazebnik's iterative quantisation): from R0, itq_iters
  *     alternations of B = sign(X R) (sign(0) = +1) and R = the orthogonal
  *     Procrustes solution for X^T B (its polar factor; computed here by
- *     Newton-Schulz iteration on binary64 GEMMs);
+ *     Newton-Schulz iteration in binary64, run until an update moves no
+ *     entry by more than 1e-9, at most 60 steps);
  *   - then U' <- U' R, V' <- V' R, canonical column signs as above, and the
  *     Dual-SVID steps (signs, rank-1 SVDs of the magnitudes) and the residual
  *     path as in lb_dual_svid_init, each path with its own rotation.

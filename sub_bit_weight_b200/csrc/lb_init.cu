@@ -30,8 +30,10 @@
 // U' V'^T unchanged: X = [U' / rho_u ; V' / rho_v] (each factor scaled to
 // unit RMS entry), then `itq_iters` alternations of B = sign(X R) and
 // R = polar(X^T B) (orthogonal Procrustes; the polar factor by Newton-Schulz
-// iteration, GEMMs only), and U' <- U' R, V' <- V' R before the signs.
+// iteration in one cooperative launch), and U' <- U' R, V' <- V' R before
+// the signs.
 #include "littlebit_init.h"
+#include "lb_coop.cuh"
 #include "lb_internal.cuh"
 #include "lb_linalg.cuh"
 
@@ -62,7 +64,8 @@ struct InitPlan {
 };
 
 constexpr int kRedBlocks = 296;        // CTAs of the fixed-order reductions (two per SM)
-constexpr int kPolarIters = 40;        // Newton-Schulz steps: enough for sigma_min / ||C||_F down to ~1e-6
+constexpr int kPolarMaxSteps = 60;     // Newton-Schulz steps at most: enough for sigma_min / ||C||_F down to ~1e-9
+constexpr double kPolarStop = 1e-9;    // an update below this makes the new iterate exact to rounding (error squares)
 
 InitPlan make_plan(int N, int K, int r, bool itq = false)
 {
@@ -444,34 +447,84 @@ __global__ void __launch_bounds__(kT) itq_sign_kernel(double *Y, int rows, int r
     if (threadIdx.x == 0) part[blockIdx.x] = acc;
 }
 
-// X0 = C / ||C||_F, the start of the Newton-Schulz iteration (all singular values in (0, 1]); C = 0 gives the
-// identity.  One CTA of kT threads.
-__global__ void __launch_bounds__(kT) polar_start_kernel(const double *C, int r, long ld, double *X0)
+// block-wide max of one value per thread (kT threads); the result is valid in thread 0
+__device__ double block_max(double v)
 {
-    __shared__ double bc;
+    __shared__ double red[kT / 32];
+    for (int o = 16; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    if (threadIdx.x == 0)
+        for (int w = 1; w < kT / 32; ++w) v = fmax(v, red[w]);
+    return v;
+}
+
+// Polar factor of C (r x r, ld) by Newton-Schulz iteration in one cooperative launch: X_0 = C / ||C||_F (all
+// singular values in (0, 1]; C = 0 gives the identity), X_{k+1} = X_k (3 I - X_k^T X_k) / 2, until an update moves no
+// entry by more than kPolarStop (the error of the new iterate is then ~the square of that: exact to rounding) or
+// kPolarMaxSteps.  X, Xn, T: r x r scratch (ld); side: gridDim.x doubles; the result goes to R (ld).  Every CTA
+// takes the same decisions from the same fixed-order sums, so all pass the same grid barriers.
+__global__ void __launch_bounds__(kT) polar_ns_kernel(const double *C, int r, long ld, double *X, double *Xn,
+                                                      double *T, double *side, double *R, unsigned *bar, int *err)
+{
+    __shared__ double sh;
+    unsigned gen = 0;
+    const long n2 = (long)r * r;
+    const long tid = blockIdx.x * (long)blockDim.x + threadIdx.x, nth = (long)gridDim.x * blockDim.x;
     double acc = 0.0;
-    for (int e = threadIdx.x; e < r * r; e += blockDim.x) {
-        const double v = C[(long)(e / r) * ld + e % r];
+    for (long e = tid; e < n2; e += nth) {
+        const double v = C[(e / r) * ld + e % r];
         acc += v * v;
     }
     acc = block_sum(acc);
-    if (threadIdx.x == 0) bc = acc;
+    if (threadIdx.x == 0) side[blockIdx.x] = acc;
+    if (!grid_barrier(bar, gen, err)) return;
+    if (threadIdx.x == 0) {
+        double a = 0.0;
+        for (int b = 0; b < (int)gridDim.x; ++b) a += side[b];
+        sh = sqrt(a);
+    }
     __syncthreads();
-    const double nrm = sqrt(bc);
-    for (int e = threadIdx.x; e < r * r; e += blockDim.x) {
-        const int i = e / r, j = e % r;
-        X0[(long)i * ld + j] = nrm > 0.0 ? C[(long)i * ld + j] / nrm : (i == j ? 1.0 : 0.0);
+    const double nrm = sh;
+    for (long e = tid; e < n2; e += nth) {
+        const long i = e / r, j = e % r;
+        X[i * ld + j] = nrm > 0.0 ? C[i * ld + j] / nrm : (i == j ? 1.0 : 0.0);
     }
-}
-
-// T = 1.5 I - 0.5 T (the Newton-Schulz factor X_{k+1} = X_k (3 I - X_k^T X_k) / 2)
-__global__ void ns_affine_kernel(double *T, int r, long ld)
-{
-    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < r * r; e += gridDim.x * blockDim.x) {
-        const int i = e / r, j = e % r;
-        double *t = T + (long)i * ld + j;
-        *t = (i == j ? 1.5 : 0.0) - 0.5 * *t;
+    if (!grid_barrier(bar, gen, err)) return;
+    for (int k = 0; k < kPolarMaxSteps; ++k) {
+        // T = (3 I - X^T X) / 2
+        for (long e = tid; e < n2; e += nth) {
+            const long i = e / r, j = e % r;
+            double a = 0.0;
+            for (int l = 0; l < r; ++l) a = fma(X[l * ld + i], X[l * ld + j], a);
+            T[i * ld + j] = (i == j ? 1.5 : 0.0) - 0.5 * a;
+        }
+        if (!grid_barrier(bar, gen, err)) return;
+        // X_{k+1} = X T and the largest change of an entry
+        double dmax = 0.0;
+        for (long e = tid; e < n2; e += nth) {
+            const long i = e / r, j = e % r;
+            double a = 0.0;
+            for (int l = 0; l < r; ++l) a = fma(X[i * ld + l], T[l * ld + j], a);
+            Xn[i * ld + j] = a;
+            dmax = fmax(dmax, fabs(a - X[i * ld + j]));
+        }
+        dmax = block_max(dmax);
+        if (threadIdx.x == 0) side[blockIdx.x] = dmax;
+        if (!grid_barrier(bar, gen, err)) return;
+        if (threadIdx.x == 0) {
+            double m = 0.0;
+            for (int b = 0; b < (int)gridDim.x; ++b) m = fmax(m, side[b]);
+            sh = m;
+        }
+        __syncthreads();
+        const double d = sh;
+        double *t = X;
+        X = Xn;
+        Xn = t;
+        if (d <= kPolarStop) break;
     }
+    for (long e = tid; e < n2; e += nth) R[(e / r) * ld + e % r] = X[(e / r) * ld + e % r];
 }
 
 __global__ void copy_square_kernel(const double *src, int r, long lds, double *dst, long ldd)
@@ -544,8 +597,36 @@ struct ItqArgs {
     double *const *Rout = nullptr;       // host array of device r x r (ld r) outputs, or null
 };
 
+int sm_count_init()
+{
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+// R = polar factor of C (r x r, ld): one cooperative launch of polar_ns_kernel
+cudaError_t polar(const Ctx &c, const double *C, double *R, double *X, double *Xn, double *T, double *side,
+                  unsigned *bar, int *err)
+{
+    const InitPlan &P = c.P;
+    const int r = P.r;
+    long ld = P.ldr;
+    const int grid = (int)std::max<long>(1, std::min<long>(std::min(sm_count_init(), kRedBlocks),
+                                                           ((long)r * r + kT - 1) / kT));
+    cudaError_t e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned), c.s);
+    if (e != cudaSuccess) return e;
+    int rr = r;
+    void *args[] = {(void *)&C, &rr, &ld, &X, &Xn, &T, &side, &R, &bar, &err};
+    return cudaLaunchCooperativeKernel((const void *)polar_ns_kernel, dim3(grid), dim3(kT), args, 0, c.s);
+}
+
 // Rotate U', V' (N x r and K x r, ld ldr) by the Joint-ITQ rotation of path p (LittleBit-2).
-void joint_itq(const Ctx &c, const ItqArgs &a, int p, double *Up, double *Vp)
+cudaError_t joint_itq(const Ctx &c, const ItqArgs &a, int p, double *Up, double *Vp, unsigned *bar, int *err)
 {
     const InitPlan &P = c.P;
     const int N = P.N, K = P.K, r = P.r, rows = N + K;
@@ -569,18 +650,13 @@ void joint_itq(const Ctx &c, const ItqArgs &a, int p, double *Up, double *Vp)
                                               a.loss ? a.loss + (size_t)p * (a.iters + 1) + t : scratch);
         if (last) break;
         c.gemm(true, false, r, r, rows, 1.0, X, ld, Y, ld, 0.0, C, ld);           // C = X^T B
-        polar_start_kernel<<<1, kT, 0, c.s>>>(C, r, ld, Pa);
-        for (int k = 0; k < kPolarIters; ++k) {
-            c.gemm(true, false, r, r, r, 1.0, Pa, ld, Pa, ld, 0.0, T, ld);        // T = X_k^T X_k
-            ns_affine_kernel<<<grid_for((long)r * r), kT, 0, c.s>>>(T, r, ld);
-            c.gemm(false, false, r, r, r, 1.0, Pa, ld, T, ld, 0.0, Pb, ld);       // X_{k+1} = X_k T
-            std::swap(Pa, Pb);
-        }
-        copy_square_kernel<<<grid_for((long)r * r), kT, 0, c.s>>>(Pa, r, ld, R, ld);
+        cudaError_t e = polar(c, C, R, Pa, Pb, T, red, bar, err);                 // R = polar factor of C
+        if (e != cudaSuccess) return e;
     }
     // Y = X R with the final R: back to each factor's own scale
     itq_unstack_kernel<<<grid_for((long)rows * r), kT, 0, c.s>>>(Y, N, K, r, ld, ss, Up, Vp);
     if (a.Rout && a.Rout[p]) copy_square_kernel<<<grid_for((long)r * r), kT, 0, c.s>>>(R, r, ld, a.Rout[p], r);
+    return cudaGetLastError();
 }
 
 cudaError_t one_path(const Ctx &c, int iters, uint64_t seed, uint32_t *Uw, uint32_t *Vw, float *h, float *g, float *l,
@@ -640,7 +716,7 @@ cudaError_t one_path(const Ctx &c, int iters, uint64_t seed, uint32_t *Uw, uint3
         col_sign_kernel<<<grid_for(32L * r), kT, 0, c.s>>>(Up, N, r, P.ldr, flip);
         col_flip_kernel<<<grid_for((long)N * r), kT, 0, c.s>>>(Up, N, r, P.ldr, flip);
         col_flip_kernel<<<grid_for((long)K * r), kT, 0, c.s>>>(Vp, K, r, P.ldr, flip);
-        joint_itq(c, *itq, path, Up, Vp);
+        if ((e = joint_itq(c, *itq, path, Up, Vp, bar, err)) != cudaSuccess) return e;
     }
     col_sign_kernel<<<grid_for(32L * r), kT, 0, c.s>>>(Up, N, r, P.ldr, flip);
     col_flip_kernel<<<grid_for((long)N * r), kT, 0, c.s>>>(Up, N, r, P.ldr, flip);
