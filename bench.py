@@ -559,11 +559,13 @@ def run_init(wkey: str, steps: int, warmup: int, dev, with_cpu: bool, only: str 
         block2()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk2:
+        torch.cuda.nvtx.range_push("littlebit2_timed")
         e0.record()
         for _ in range(steps):
             block2()
         e1.record()
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
     ms2 = e0.elapsed_time(e1) / steps
     loss = np.array([r_.itq_loss.cpu().numpy() for r_ in last])       # [layer, path, ITQ_ITERS + 1]
     lb2 = {"value": round(len(shapes) / (ms2 * 1e-3), 3), "unit": "layers/s", "higher_is_better": True,
