@@ -37,6 +37,8 @@
 #include "lb_internal.cuh"
 #include "lb_linalg.cuh"
 
+#include <cooperative_groups.h>
+
 #include <algorithm>
 #include <math.h>
 
@@ -527,6 +529,95 @@ __global__ void __launch_bounds__(kT) polar_ns_kernel(const double *C, int r, lo
     for (long e = tid; e < n2; e += nth) R[(e / r) * ld + e % r] = X[(e / r) * ld + e % r];
 }
 
+// The same iteration for small r in one thread-block cluster: kPolarCtas CTAs of kPolarThreads threads, the
+// hardware cluster barrier in place of the grid barrier (all CTAs of a cluster are scheduled together).
+constexpr int kPolarCtas = 8;           // portable cluster size
+constexpr int kPolarThreads = 1024;
+constexpr int kPolarClusterMaxR = 96;   // above this the grid-wide kernel (more SMs for the r^3 steps) is faster
+
+// block-wide sum / max of one value per thread (any multiple of 32 threads up to 1024); valid in thread 0
+__device__ double block_reduce_any(double v, bool is_max)
+{
+    __shared__ double red[32];
+    for (int o = 16; o; o >>= 1) {
+        const double w = __shfl_xor_sync(0xffffffffu, v, o);
+        v = is_max ? fmax(v, w) : v + w;
+    }
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    if (threadIdx.x == 0)
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) v = is_max ? fmax(v, red[w]) : v + red[w];
+    return v;
+}
+
+__global__ void __cluster_dims__(kPolarCtas, 1, 1) __launch_bounds__(kPolarThreads)
+    polar_ns_cluster_kernel(const double *C, int r, long ld, double *X, double *Xn, double *T, double *side, double *R)
+{
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    __shared__ double sh;
+    const long n2 = (long)r * r;
+    const int rank = (int)cl.block_rank();
+    const long tid = rank * (long)blockDim.x + threadIdx.x, nth = (long)kPolarCtas * blockDim.x;
+    auto sync = [&]() {
+        __threadfence();
+        cl.sync();
+    };
+    double acc = 0.0;
+    for (long e = tid; e < n2; e += nth) {
+        const double v = C[(e / r) * ld + e % r];
+        acc += v * v;
+    }
+    acc = block_reduce_any(acc, false);
+    if (threadIdx.x == 0) side[rank] = acc;
+    sync();
+    if (threadIdx.x == 0) {
+        double a = 0.0;
+        for (int b = 0; b < kPolarCtas; ++b) a += side[b];
+        sh = sqrt(a);
+    }
+    __syncthreads();
+    const double nrm = sh;
+    for (long e = tid; e < n2; e += nth) {
+        const long i = e / r, j = e % r;
+        X[i * ld + j] = nrm > 0.0 ? C[i * ld + j] / nrm : (i == j ? 1.0 : 0.0);
+    }
+    sync();
+    for (int k = 0; k < kPolarMaxSteps; ++k) {
+        for (long e = tid; e < n2; e += nth) {
+            const long i = e / r, j = e % r;
+            double a = 0.0;
+            for (int l = 0; l < r; ++l) a = fma(X[l * ld + i], X[l * ld + j], a);
+            T[i * ld + j] = (i == j ? 1.5 : 0.0) - 0.5 * a;
+        }
+        sync();
+        double dmax = 0.0;
+        for (long e = tid; e < n2; e += nth) {
+            const long i = e / r, j = e % r;
+            double a = 0.0;
+            for (int l = 0; l < r; ++l) a = fma(X[i * ld + l], T[l * ld + j], a);
+            Xn[i * ld + j] = a;
+            dmax = fmax(dmax, fabs(a - X[i * ld + j]));
+        }
+        dmax = block_reduce_any(dmax, true);
+        if (threadIdx.x == 0) side[rank] = dmax;
+        sync();
+        if (threadIdx.x == 0) {
+            double m = 0.0;
+            for (int b = 0; b < kPolarCtas; ++b) m = fmax(m, side[b]);
+            sh = m;
+        }
+        __syncthreads();
+        const double d = sh;
+        double *t = X;
+        X = Xn;
+        Xn = t;
+        if (d <= kPolarStop) break;
+    }
+    for (long e = tid; e < n2; e += nth) R[(e / r) * ld + e % r] = X[(e / r) * ld + e % r];
+}
+
 __global__ void copy_square_kernel(const double *src, int r, long lds, double *dst, long ldd)
 {
     for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < r * r; e += gridDim.x * blockDim.x)
@@ -616,6 +707,10 @@ cudaError_t polar(const Ctx &c, const double *C, double *R, double *X, double *X
     const InitPlan &P = c.P;
     const int r = P.r;
     long ld = P.ldr;
+    if (r <= kPolarClusterMaxR) {
+        polar_ns_cluster_kernel<<<kPolarCtas, kPolarThreads, 0, c.s>>>(C, r, ld, X, Xn, T, side, R);
+        return cudaGetLastError();
+    }
     const int grid = (int)std::max<long>(1, std::min<long>(std::min(sm_count_init(), kRedBlocks),
                                                            ((long)r * r + kT - 1) / kT));
     cudaError_t e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned), c.s);

@@ -79,6 +79,7 @@ def _parity(lib, W, r, npaths, itq_iters, R0s=None, iters=24):
     (512, 384, 16, 2, 50),
     (1000, 513, 100, 2, 50),  # odd K, r not a multiple of 32
     (2048, 1024, 128, 1, 50),
+    (600, 400, 200, 2, 12),   # r above the one-cluster polar kernel's limit: the grid-wide kernel
 ])
 def test_parity_on_power_law_weights(lib, shape):
     N, K, r, npaths, it = shape
