@@ -19,7 +19,7 @@
  * kernels (z and (dy (.) h) U_s in one launch whose output tiles are split
  * over k, partial sums added in float32); the two dense products dy^T zl
  * (N x 2r) and x^T dz (K x 2r) are plain fp16 GEMMs (cuBLAS) with float32
- * accumulation.
+ * accumulation, run with the factor gradients on a second stream beside dx.
  *
  * Arithmetic: x enters as bfloat16 (converted to fp16 exactly in fp16's normal
  * range, as in the forward pass); dy is multiplied by one power of two chosen
@@ -71,9 +71,10 @@ LB_API void lb_backward_destroy(lb_backward *B);
  *
  * With the timing hook of littlebit.h (lb_profile_events) holding 9 events,
  * events[i] is recorded at the i-th stage boundary: 0 | dy scaling | 1 |
- * z = (x (.) g) V_s and (dy (.) h) U_s, one launch | 2, 3 | dl, dz, zl | 4 |
- * dx | 5 | dy^T zl | 6 | x^T dz | 7 | dh, dg, dU, dV | 8 (events 2 and 3
- * mark the same point). */
+ * z = (x (.) g) V_s and (dy (.) h) U_s, one launch | 2, 3 | dl, dz, zl | 4;
+ * after 4 the work forks: dx | 5 on `stream`, and on a second stream of the
+ * library (joined back into `stream` before the call returns) dy^T zl | 6 |
+ * x^T dz | 7 | dh, dg, dU, dV | 8 (events 2 and 3 mark the same point). */
 LB_API lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, int M,
                                    const float *const *U_lat, const float *const *V_lat, float *dx,
                                    float *const *dh, float *const *dg, float *const *dl,

@@ -48,6 +48,8 @@ struct lb_backward {
     float *GU = nullptr;           // [N][K2]
     float *GV = nullptr;           // [K][K2]
     cublasHandle_t blas = nullptr;
+    cudaStream_t side = nullptr;   // G_U, G_V and the factor gradients run here, beside dx
+    cudaEvent_t fork = nullptr, join = nullptr;
 };
 
 namespace lb {
@@ -197,12 +199,6 @@ __global__ void latent_mix_kernel(const float *__restrict__ dzl, const float *__
     atomicAdd(dl_acc + j + 3, acc.w);
 }
 
-__global__ void scale_kernel(float *x, long n, const float *__restrict__ stat)
-{
-    const float sc = stat[2];
-    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) x[i] *= sc;
-}
-
 __global__ void dl_out_kernel(const float *__restrict__ dl_acc, int r, int r8, const float *__restrict__ stat,
                               float *dl0, float *dl1)
 {
@@ -334,6 +330,9 @@ void lb_backward_destroy(lb_backward *B)
                     (void *)B->GV})
         cudaFree(p);
     if (B->blas) cublasDestroy(B->blas);
+    if (B->fork) cudaEventDestroy(B->fork);
+    if (B->join) cudaEventDestroy(B->join);
+    if (B->side) cudaStreamDestroy(B->side);
     delete B;
 }
 
@@ -390,6 +389,10 @@ lb_status lb_backward_create(lb_backward **out, int N, int K, int r, int npaths,
         cudaMemcpyAsync(B->Vw + (size_t)p * K * wpr, V[p], (size_t)K * wpr * 4, cudaMemcpyDeviceToDevice, s);
     }
     if (cublasCreate(&B->blas) != CUBLAS_STATUS_SUCCESS) return fail(LB_ERR_CUDA);
+    if (cudaStreamCreateWithFlags(&B->side, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&B->fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&B->join, cudaEventDisableTiming) != cudaSuccess)
+        return fail(LB_ERR_CUDA);
     cublasSetPointerMode(B->blas, CUBLAS_POINTER_MODE_DEVICE);
     if (cudaStreamSynchronize(s) != cudaSuccess) return fail(LB_ERR_CUDA);
     cudaFree(ones);
@@ -416,8 +419,8 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
     const int N = B->N, K = B->K, r = B->r, K2 = B->K2;
     int launches = 0;
 
-    // timing hook (littlebit.h): events 0 | scaling | 1 | z and dzl (one launch) | 2, 3 | dl, dz, zl | 4 | dx | 5 |
-    // G_U | 6 | G_V | 7 | factor gradients | 8
+    // timing hook (littlebit.h): events 0 | scaling | 1 | z and dzl (one launch) | 2, 3 | dl, dz, zl | 4, then
+    // dx | 5 on this stream and, from 4 on the side stream, G_U | 6 | G_V | 7 | factor gradients | 8
     profile_mark(0, s);
     // dy scale (device-side exponent), fp16 copies of dy 2^E and x
     cudaMemsetAsync(B->stat, 0, sizeof(float), s);
@@ -437,7 +440,9 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
     const uint16_t *dys[1] = {reinterpret_cast<const uint16_t *>(B->dy16)};
     float *ys[1] = {dx};
     if ((st = prefill_forward(B->Lf->self->plan, &B->Lf, xs, ys, M, s, &launches, 0, false, false)) != LB_OK) return st;
-    if ((st = prefill_forward(B->Lt->self->plan, &B->Lt, dys, ys, M, s, &launches, 0, true, false)) != LB_OK) return st;
+    if ((st = prefill_forward(B->Lt->self->plan, &B->Lt, dys, ys, M, s, &launches, 0, true, false, B->stat + 2)) !=
+        LB_OK)
+        return st;
     __half *zf = prefill_zl(B->Lf->self->plan, 0), *dz = prefill_zl(B->Lt->self->plan, 0);
     if (!zf || !dz) return LB_ERR_CUDA;
     cudaMemsetAsync(B->zpart, 0, (size_t)M * K2 * sizeof(float), s);
@@ -453,23 +458,29 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
         B->dzpart, B->zpart, M, ncols, K2, B->lcat, B->dl_acc, dz, zf, rows_per);
     dl_out_kernel<<<grid_for(r), kT, 0, s>>>(B->dl_acc, r, B->r8, B->stat, dl[0], B->npaths > 1 ? dl[1] : nullptr);
     profile_mark(4, s);
-    // dx 2^E = sum_p g (.) (dz 2^E V_s^T)
-    if ((st = prefill_forward(B->Lt->self->plan, &B->Lt, dys, ys, M, s, &launches, 2, true, false)) != LB_OK) return st;
-    scale_kernel<<<grid_for((long)M * K), kT, 0, s>>>(dx, (long)M * K, B->stat);
-    launches += 3;
+    // from here two streams: dx here; G_U, G_V and the factor gradients on the side stream (they read dz, zl, dy16
+    // and x16, which are complete), so the side work fills the SMs that the tail of the dx tiles leaves idle
+    if (cudaEventRecord(B->fork, s) != cudaSuccess || cudaStreamWaitEvent(B->side, B->fork, 0) != cudaSuccess)
+        return LB_ERR_CUDA;
+    cudaStream_t s2 = B->side;
+    // dx = 2^-E sum_p g (.) (dz 2^E V_s^T): the output contraction's epilogue multiplies by 2^-E (stat[2])
+    if ((st = prefill_forward(B->Lt->self->plan, &B->Lt, dys, ys, M, s, &launches, 2, true, false, B->stat + 2)) !=
+        LB_OK)
+        return st;
+    launches += 2;
     profile_mark(5, s);
 
     // G_U = dy^T zl, G_V = x^T dz (row-major; cuBLAS sees the column-major transposes), alpha = 2^-E
     const float *alpha = B->stat + 2, *zero_d = B->stat + 4;
-    cublasSetStream(B->blas, s);
+    cublasSetStream(B->blas, s2);
     if (cublasGemmEx(B->blas, CUBLAS_OP_N, CUBLAS_OP_T, K2, N, M, alpha, zf, CUDA_R_16F, K2, B->dy16, CUDA_R_16F, N,
                      zero_d, B->GU, CUDA_R_32F, K2, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
         return LB_ERR_CUDA;
-    profile_mark(6, s);
+    profile_mark(6, s2);
     if (cublasGemmEx(B->blas, CUBLAS_OP_N, CUBLAS_OP_T, K2, K, M, alpha, dz, CUDA_R_16F, K2, B->x16, CUDA_R_16F, K,
                      zero_d, B->GV, CUDA_R_32F, K2, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
         return LB_ERR_CUDA;
-    profile_mark(7, s);
+    profile_mark(7, s2);
     const int wpr = (r + 31) / 32;
     FactorArgs fu{}, fv{};
     for (int p = 0; p < B->npaths; ++p) {
@@ -489,21 +500,23 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
         vec4 = vec4 && !(((uintptr_t)U_lat[p] | (uintptr_t)V_lat[p] | (uintptr_t)dU[p] | (uintptr_t)dV[p]) & 15);
     if (vec4) {
         if (B->npaths == 2) {
-            factor_grad4_kernel<2><<<grid_for(32L * N), kT, 0, s>>>(B->GU, N, K2, r, B->r8, fu);
-            factor_grad4_kernel<2><<<grid_for(32L * K), kT, 0, s>>>(B->GV, K, K2, r, B->r8, fv);
+            factor_grad4_kernel<2><<<grid_for(32L * N), kT, 0, s2>>>(B->GU, N, K2, r, B->r8, fu);
+            factor_grad4_kernel<2><<<grid_for(32L * K), kT, 0, s2>>>(B->GV, K, K2, r, B->r8, fv);
         } else {
-            factor_grad4_kernel<1><<<grid_for(32L * N), kT, 0, s>>>(B->GU, N, K2, r, B->r8, fu);
-            factor_grad4_kernel<1><<<grid_for(32L * K), kT, 0, s>>>(B->GV, K, K2, r, B->r8, fv);
+            factor_grad4_kernel<1><<<grid_for(32L * N), kT, 0, s2>>>(B->GU, N, K2, r, B->r8, fu);
+            factor_grad4_kernel<1><<<grid_for(32L * K), kT, 0, s2>>>(B->GV, K, K2, r, B->r8, fv);
         }
     } else if (B->npaths == 2) {
-        factor_grad_kernel<2><<<grid_for(32L * N), kT, 0, s>>>(B->GU, N, K2, r, B->r8, fu);
-        factor_grad_kernel<2><<<grid_for(32L * K), kT, 0, s>>>(B->GV, K, K2, r, B->r8, fv);
+        factor_grad_kernel<2><<<grid_for(32L * N), kT, 0, s2>>>(B->GU, N, K2, r, B->r8, fu);
+        factor_grad_kernel<2><<<grid_for(32L * K), kT, 0, s2>>>(B->GV, K, K2, r, B->r8, fv);
     } else {
-        factor_grad_kernel<1><<<grid_for(32L * N), kT, 0, s>>>(B->GU, N, K2, r, B->r8, fu);
-        factor_grad_kernel<1><<<grid_for(32L * K), kT, 0, s>>>(B->GV, K, K2, r, B->r8, fv);
+        factor_grad_kernel<1><<<grid_for(32L * N), kT, 0, s2>>>(B->GU, N, K2, r, B->r8, fu);
+        factor_grad_kernel<1><<<grid_for(32L * K), kT, 0, s2>>>(B->GV, K, K2, r, B->r8, fv);
     }
     launches += 2;
-    profile_mark(8, s);
+    profile_mark(8, s2);
+    if (cudaEventRecord(B->join, s2) != cudaSuccess || cudaStreamWaitEvent(s, B->join, 0) != cudaSuccess)
+        return LB_ERR_CUDA;
     set_launch_count(launches);
     return cudaGetLastError() == cudaSuccess ? LB_OK : LB_ERR_CUDA;
 }

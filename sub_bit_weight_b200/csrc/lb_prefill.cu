@@ -588,6 +588,11 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
                     }
                 }
                 if (MODE == 1) {
+                    if (ly.oscale) {
+                        const float f = __ldg(ly.oscale);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+                    }
                     // 32 rows x 32 columns of y through a 128B-swizzled block and one TMA store
                     if (ch > 0 || tcount > 0) {
                         if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
@@ -753,6 +758,7 @@ struct PrefillState {
     int M = 0;                       // rows the scratch was sized for
     int lastM = -1;
     bool lastF16 = false;            // the activations of the last encoded maps are fp16
+    const float *lastScale = nullptr;   // the output scale of the last encoded records
     std::vector<const void *> lastX, lastY;
     void *zl = nullptr;              // latent activations of every layer, fp16 [M][K2]
     std::vector<size_t> zl_off;
@@ -808,7 +814,7 @@ static cudaError_t ensure_smem(size_t smem)
 
 lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const uint16_t *const *xs,
                           float *const *ys, int M, cudaStream_t s, int *launches, int parts, bool a_f16,
-                          bool marks)
+                          bool marks, const float *out_scale)
 {
     Plan &P = const_cast<Plan &>(Pc);
     const int n = P.n;
@@ -848,7 +854,7 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
         st.M = M;
         dirty = true;
     }
-    if (M != st.lastM || a_f16 != st.lastF16) dirty = true;
+    if (M != st.lastM || a_f16 != st.lastF16 || out_scale != st.lastScale) dirty = true;
     if ((int)st.lastX.size() != n) {
         st.lastX.assign(n, nullptr);
         st.lastY.assign(n, nullptr);
@@ -889,6 +895,7 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
             a.ksplit = 1;
             a.part = nullptr;
             a.ld_part = 0;
+            a.oscale = nullptr;
             PfLayer &b = rec[n + i];
             b.tmA = st.maps + n + i;
             b.tmY = st.maps + 2 * n + i;
@@ -907,6 +914,7 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
             b.ksplit = 1;
             b.part = nullptr;
             b.ld_part = 0;
+            b.oscale = out_scale;
             starts[i + 1] = starts[i] + mtiles * a.ntn;
             starts[n + 1 + i + 1] = starts[n + 1 + i] + mtiles * b.ntn;
             st.lastX[i] = xs[i];
@@ -916,6 +924,7 @@ lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const u
         st.tiles[1] = starts[2 * n + 1];
         st.lastM = M;
         st.lastF16 = a_f16;
+        st.lastScale = out_scale;
         // pageable sources: the copies are staged before these calls return
         if ((e = cudaMemcpyAsync(st.maps, maps.data(), sizeof(CUtensorMap) * 3 * n, cudaMemcpyHostToDevice, s)) !=
             cudaSuccess)
@@ -1089,6 +1098,7 @@ lb_status prefill_latent_jobs(PfJobState **state, const PfLatentJob *jobs, int n
             a.ksplit = split[q];
             a.part = j.part;
             a.ld_part = j.ld_part;
+            a.oscale = nullptr;
             starts[q + 1] = starts[q] + tiles[q] * split[q];
         }
         if ((e = cudaMemcpyAsync(st.maps, maps.data(), sizeof(CUtensorMap) * n, cudaMemcpyHostToDevice, s)) != cudaSuccess ||

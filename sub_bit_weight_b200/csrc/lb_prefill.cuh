@@ -21,11 +21,13 @@ cudaError_t prefill_build_weights(PfWeights &W, const LayerDev &d, const uint32_
 size_t prefill_weight_bytes(const LayerDev &d);
 
 struct PrefillState;   // per plan (owned by Plan)
-// parts: 1 = latent contraction only (writes the plan's zl), 2 = output contraction only (reads it), 3 = both.
-// a_f16: the activations xs are fp16 (bit patterns) rather than bf16.  marks: record the timing hook's events.
+// parts: 1 = latent contraction only (writes the plan's zl), 2 = output contraction only (reads it), 3 = both,
+// 0 = set up the plan's maps and buffers only.  a_f16: the activations xs are fp16 (bit patterns) rather than
+// bf16.  marks: record the timing hook's events.  out_scale: null, or a device scalar the output contraction
+// multiplies every y by.
 lb_status prefill_forward(const Plan &P, const lb_layer *const *layers, const uint16_t *const *xs,
                           float *const *ys, int M, cudaStream_t s, int *launches, int parts = 3, bool a_f16 = false,
-                          bool marks = true);
+                          bool marks = true, const float *out_scale = nullptr);
 // latent activations of layer i of the plan, fp16 [M][pf.K2] (null before the first prefill call)
 __half *prefill_zl(const Plan &P, int i);
 void prefill_free(PrefillState *st);

@@ -44,6 +44,7 @@ struct PfLayer {
     float *part;              // latent contraction with ksplit: fp32 [M][ld_part] that each unit adds its raw
                               // partial sums to (no l; zeroed by the caller); null = the fp16 zl epilogue
     int ld_part;
+    const float *oscale;      // output contraction: null, or a device scalar every output is multiplied by
 };
 
 }  // namespace lb
