@@ -200,7 +200,8 @@ def oracle_sample(w: synth.Workload, M: int, budget_s: float, max_layers: int | 
 
 # ----------------------------------------------------------------- GPU runs
 
-def run_gpu(w: synth.Workload, M: int, steps: int, warmup: int, dist, dev, want_e2e=True, nblocks=None):
+def run_gpu(w: synth.Workload, M: int, steps: int, warmup: int, dist, dev, want_e2e=True, nblocks=None,
+            flush_l2=False):
     import torch
     from sub_bit_weight_b200 import lib, stacks
 
@@ -237,17 +238,32 @@ def run_gpu(w: synth.Workload, M: int, steps: int, warmup: int, dist, dev, want_
     # whole steps: no events between a step's launches (consecutive kernels may overlap)
     with ClockSampler(torch.cuda.current_device()) as clk:
         torch.cuda.nvtx.range_push("bench_timed")       # lets a profiler select the timed launches
-        start.record(stream)
-        for k in range(steps):
-            lib.lb_stack_forward(S, io=io)
-            if nlaunch_per_step is None:
-                nlaunch_per_step = lib.lb_last_launch_count()
-        stop.record(stream)
-        torch.cuda.synchronize()
+        if flush_l2:
+            # a 256 MB write (twice the L2) before every step; only the steps are timed, each with its own events
+            flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+            se = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            for k in range(steps):
+                flush.zero_()
+                se[k][0].record(stream)
+                lib.lb_stack_forward(S, io=io)
+                se[k][1].record(stream)
+                if nlaunch_per_step is None:
+                    nlaunch_per_step = lib.lb_last_launch_count()
+            torch.cuda.synchronize()
+            total_ms = sum(a.elapsed_time(b) for a, b in se)
+            del flush
+        else:
+            start.record(stream)
+            for k in range(steps):
+                lib.lb_stack_forward(S, io=io)
+                if nlaunch_per_step is None:
+                    nlaunch_per_step = lib.lb_last_launch_count()
+            stop.record(stream)
+            torch.cuda.synchronize()
+            total_ms = start.elapsed_time(stop)
         torch.cuda.nvtx.range_pop()
     if dist:
         dist.barrier()
-    total_ms = start.elapsed_time(stop)
 
     # each kernel alone: a CUDA event after every launch (launches then run strictly one after another)
     pk_steps = max(3, min(steps, 100))
@@ -364,6 +380,8 @@ def main():
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--blocks", type=int, default=None, help="only the first N blocks of the stack (profiling)")
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="write 256 MB before every timed step and time the steps alone (stacks that fit in L2)")
     ap.add_argument("--init", default=INIT_DEFAULT,
                     help="workload whose first block gets the Dual-SVID + residual initialisation ('' = skip)")
     ap.add_argument("--init-steps", type=int, default=2)
@@ -395,7 +413,8 @@ def main():
         dist = tdist
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    res = run_gpu(w, M, args.steps, args.warmup, dist, dev, nblocks=args.blocks, want_e2e=not w.pool_rows)
+    res = run_gpu(w, M, args.steps, args.warmup, dist, dev, nblocks=args.blocks, want_e2e=not w.pool_rows,
+                  flush_l2=args.flush_l2)
     total_ms = max_over_ranks(res["total_ms"], dist)
     shapes = res["shapes"]
     ms_step = total_ms / args.steps
@@ -467,9 +486,11 @@ def main():
                       "bf16 in, int8 tensor-core MMA (u8 signs x s8 fixed-point digits, s32 acc), fp32 out"),
             "data": "synthetic (seeded; signs Bernoulli(0.5), scales lognormal(-3,0.5) fp16, x N(0,1) bf16)",
             "config": {"workload": f"{w.key}: {w.title}", "layers": len(shapes), "M": M,
-                       "l2": ("inputs larger than L2 (stack streams from HBM every step)"
-                              if prefill_main or step_bytes > 126e6 else "stack fits in L2 (effective GB/s)"),
+                       "l2": ("L2 flushed (256 MB write) before every step; steps timed alone" if args.flush_l2 else
+                              "inputs larger than L2 (stack streams from HBM every step)"
+                              if prefill_main or step_bytes > 126e6 else "stack fits in L2 (effective GB/s, warm)"),
                        "parallelism": f"replicas x{world}"},
+            "tokens_per_s": round(world * M * args.steps / (total_ms * 1e-3), 1),
             "roofline": roof, "gpu_launches": res["launches"], "clocks": res["clocks"], "e2e": e2e}
     if not prefill_main:
         line["config"]["bytes_per_step"] = step_bytes
@@ -483,6 +504,7 @@ def main():
         tf = pflops / (pms * 1e-3) / 1e12
         line["prefill"] = {"workload": f"{pw.key}: {pw.title}", "M": pM, "layers": len(pres["shapes"]),
                            "value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(pms, 3),
+                           "tokens_per_s": round(pM / (pms * 1e-3), 1),
                            "steps": args.prefill_steps, "gpu_launches": pres["launches"],
                            "roofline": {"bound": "tensor", "achieved": round(tf, 2),
                                         "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
