@@ -53,7 +53,7 @@ constexpr int kP2Stages = 2;            // per-warp bulk-copy ring depth, contra
 __host__ __device__ constexpr int pair_warps_per_cta(int MM) { return MM == 1 ? 16 : 12; }
 constexpr int kPairStages = 2;          // ring stages per warp
 constexpr int kPairStageKB = 16;        // k-blocks per ring stage (4 KB)
-constexpr int kPairMaxKB2 = 40;         // largest contraction-2 depth (k-blocks) these kernels take
+constexpr int kPairMaxKB2 = 64;         // largest contraction-2 depth (k-blocks) these kernels take (r = 1024, 2 paths)
 // Shared memory of the contraction-2 kernel (per warp; per CTA with the zero
 // buffer of one-row batches), and its warps per CTA: the most of
 // {16, 12, 8, 6, 4} whose CTA fits in 227 KB.

@@ -45,11 +45,13 @@ def test_single_512_workload(env, M):
 SHAPES = [
     (100, 70, 5, 2), (64, 64, 16, 1), (1, 1, 1, 2), (257, 1000, 33, 2), (130, 2050, 80, 2),
     (1024, 8192, 32, 2), (65, 33, 800, 2), (700, 3000, 184, 2), (96, 4100, 304, 1),
+    (100, 300, 1024, 2),   # contraction-2 depth 64 k-blocks: the deepest the one/two-row kernels take
+    (80, 200, 1030, 2),    # one k-block deeper: the general kernels
 ]
 
 
 @pytest.mark.parametrize("N,K,r,P", SHAPES)
-@pytest.mark.parametrize("M", [1, 3, 4, 5, 16])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 16])
 def test_ragged_shapes(env, N, K, r, P, M):
     shape = synth.LayerShape("t", N, K, r)
     y, ref, _, _ = _run(env, 1000 + N + K + r, shape, M, npaths=P)
