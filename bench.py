@@ -360,12 +360,19 @@ def run_gpu(w: synth.Workload, M: int, steps: int, warmup: int, dist, dev, want_
 
 
 def max_over_ranks(v: float, dist):
+    """The largest of every rank's v (a device time): one all-reduce, taken by every rank in the same order."""
     if not dist:
         return v
     import torch
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(world: int, work_per_rank: float, steps: int, max_ms: float) -> float:
+    """Whole-job throughput of independent replicas: every rank's work over the slowest rank's time."""
+    return world * work_per_rank * steps / (max_ms * 1e-3)
 
 
 def main():
@@ -421,13 +428,13 @@ def main():
     prefill_main = bool(w.pool_rows)
     if prefill_main:
         flops = sum(layer_flops(s, M) for s in shapes)
-        value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+        value = replica_throughput(world, flops, args.steps, total_ms) / 1e12
         unit = "TFLOP/s"
     else:
         k1b = sum(layer_bytes(s, M)[0] for s in shapes)
         k2b = sum(layer_bytes(s, M)[1] for s in shapes)
         step_bytes = k1b + k2b
-        value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
+        value = replica_throughput(world, step_bytes, args.steps, total_ms) / 1e9
         unit = "GB/s"
 
     roof = None
@@ -782,7 +789,8 @@ def reference_arm(args, w, M, world, rank, pk):
     """The CPU oracle timed as it stands, on the same workload/metric (rank 0 only)."""
     if rank != 0:
         return
-    per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    # each step a bounded sample of the workload: at most --cpu-seconds of oracle time, the whole run a few minutes
+    per_step = max(0.2, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample(w, M, per_step / 4, max_layers=1)
     t_work = t_sec = 0.0
