@@ -278,7 +278,7 @@ def run_gpu(w: synth.Workload, M: int, steps: int, warmup: int, dist, dev, want_
     torch.cuda.synchronize()
     lib.lb_profile_events([])
     per_launch = None
-    if nlaunch_per_step == nl and nl in (2, 4):
+    if nlaunch_per_step == nl and nl in (2, 3, 4):
         per_launch = tuple(sum(e[i].elapsed_time(e[i + 1]) for e in ev) / pk_steps for i in range(nl))
 
     e2e = None
@@ -458,6 +458,10 @@ def main():
             suffix = "_pair_kernel" if M <= 2 else "_kernel"
             names = ["contraction1" + suffix, "contraction2" + suffix]
             kbytes = [k1b, k2b]
+            if len(res["per_launch"]) == 3:
+                # general kernels (3..16 rows): the per-layer finish between the contractions moves no algorithmic bytes
+                names = [names[0], "finish_general_kernel", names[1]]
+                kbytes = [k1b, 0.0, k2b]
             if len(res["per_launch"]) == 4:
                 # activation quantisation and the contraction-1 finish run as their own launches:
                 # x and g are the bytes of the first, the finish moves no algorithmic bytes

@@ -13,11 +13,11 @@
 //     results into float64 accumulators: sum_k b*t per latent row and sum_k t
 //     per path.  Those terms are integers below 2^26 times powers of two, so
 //     the float64 sums are exact (hence independent of arrival order) as long
-//     as the chunks' exponents lie within ~26 of each other.  The last item of
-//     a layer to finish (a completion counter; nothing waits) forms
-//     z = sum_k t - 2 * sum_k b*t (a sign is s = 1 - 2b), zl = z (.) l, writes
-//     zl as 16-bit fixed-point B fragments for contraction 2 and clears the
-//     accumulators for the next call.
+//     as the chunks' exponents lie within ~26 of each other.
+//   finish (one CTA per layer, its own launch): z = sum_k t - 2 * sum_k b*t
+//     (a sign is s = 1 - 2b), zl = z (.) l, written as 16-bit fixed-point B
+//     fragments for contraction 2; the accumulators are cleared for the next
+//     call.
 //   contraction 2 (work item = one layer x 512 outputs):
 //     s = zl . U_sign^T on integer tensor cores, y = sum_p h_p (.) s_p.
 //
@@ -51,7 +51,7 @@ __device__ void finish_latent(const LayerDev *dp, int M, float *sMax, int *sBad,
         const double z = __ldcg(S + p * 16 + m) - 2.0 * __ldcg(acc + (size_t)(p * r16 + j) * 16 + m);
         return (float)z * __half2float(lsc[p * r16 + j]);
     };
-    for (int e = tid; e < npaths * r * M; e += kDecodeThreads) {
+    for (int e = tid; e < npaths * r * M; e += (int)blockDim.x) {
         const int m = e % M, pj = e / M;
         const int p = pj / r, j = pj - p * r;
         const float zl = zl_at(p, j, m);
@@ -66,7 +66,7 @@ __device__ void finish_latent(const LayerDev *dp, int M, float *sMax, int *sBad,
     __syncthreads();
     // digits into the fragments of this call's n-tiles (rows m in [M, 4*NT) get zeros)
     const int MT = 4 * NT, ngrp = r32 / 4;
-    for (int e = tid; e < npaths * MT * ngrp; e += kDecodeThreads) {
+    for (int e = tid; e < npaths * MT * ngrp; e += (int)blockDim.x) {
         const int c = e % ngrp, pm = e / ngrp;
         const int p = pm / MT, m = pm - p * MT;
         uint32_t wlo = 0, whi = 0;
@@ -99,7 +99,18 @@ __device__ void finish_latent(const LayerDev *dp, int M, float *sMax, int *sBad,
         dp->zmeta[p * 16 + m] = make_int2(sE[p * 16 + m], sQs[p * 16 + m]);
     }
     // accumulators back to zero for the next call
-    for (int i = tid; i < (int)acc_doubles(R1); i += kDecodeThreads) acc[i] = 0.0;
+    for (int i = tid; i < (int)acc_doubles(R1); i += (int)blockDim.x) acc[i] = 0.0;
+}
+
+// One CTA per layer of the batch (layer base + blockIdx.x), after contraction 1.
+constexpr int kFinishGeneralThreads = 1024;
+template <int NT>
+__global__ void __launch_bounds__(kFinishGeneralThreads) finish_general_kernel(const LayerDev *__restrict__ layers,
+                                                                               int base, int M)
+{
+    __shared__ float sMax[32];
+    __shared__ int sBad[32], sE[32], sQs[32];
+    finish_latent<NT>(layers + base + blockIdx.x, M, sMax, sBad, sE, sQs);
 }
 
 // ---------------------------------------------------------------------------
@@ -119,7 +130,6 @@ __global__ void __launch_bounds__(kDecodeThreads)
     __shared__ uint64_t bars[NW][kP1Stages];
     __shared__ float sMax[32];
     __shared__ int sBad[32], sE[32], sQs[32];
-    __shared__ int sLast;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;
@@ -189,12 +199,18 @@ __global__ void __launch_bounds__(kDecodeThreads)
             }
         }
         const bool vec = ((K & 7) == 0) && (kg + 8 <= K);
+        // the rows' 8 activations each, all loads in flight together (the loops over m below are unrolled)
+        uint4 xr[kMaxDecodeM];
+#pragma unroll
+        for (int m = 0; m < kMaxDecodeM; ++m)
+            xr[m] = (m < M && act && vec) ? __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + kg))
+                                          : make_uint4(0u, 0u, 0u, 0u);
         auto load_x = [&](int m, float (&xv)[8]) {
             if (!act) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) xv[e] = 0.0f;
             } else if (vec) {
-                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + kg));
+                const uint4 raw = xr[m];
                 const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -207,7 +223,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
                     xv[e] = (kg + e < K) ? bf16_bits_to_float(__ldg(x + (size_t)m * K + kg + e)) : 0.0f;
             }
         };
-        for (int m = 0; m < M; ++m) {
+#pragma unroll
+        for (int m = 0; m < kMaxDecodeM; ++m) {
+            if (m >= M) break;
             float xv[8];
             load_x(m, xv);
 #pragma unroll
@@ -235,7 +253,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
         }
         __syncthreads();
         // ---- digits into B fragments, digit sums per (path, m)
-        for (int m = 0; m < M; ++m) {
+#pragma unroll
+        for (int m = 0; m < kMaxDecodeM; ++m) {
+            if (m >= M) break;
             float xv[8];
             load_x(m, xv);
 #pragma unroll
@@ -350,17 +370,6 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 }
         }
 
-        // ---- completion count; the last item of the layer finishes the latent vector
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) sLast = (atomicAdd(dp->counter, 1u) == (unsigned)(dp->nkc - 1));
-        __syncthreads();
-        if (sLast) {
-            __threadfence();
-            finish_latent<NT>(dp, M, sMax, sBad, sE, sQs);
-            __syncthreads();
-            if (tid == 0) atomicExch(dp->counter, 0u);
-        }
         __syncthreads();   // shared state is rebuilt by the next item
     }
 }
@@ -515,12 +524,14 @@ __global__ void __launch_bounds__(kDecodeThreads)
 // Host side
 // ---------------------------------------------------------------------------
 typedef void (*K1Fn)(const LayerDev *, const P1Item *, int, const IoPtrs, int, int, int *);
+typedef void (*KFFn)(const LayerDev *, int, int);
 typedef void (*K2Fn)(const LayerDev *, const P2Item *, int, const IoPtrs, int, int, int, int *);
 
 template <int NT>
-static void kernels_for(K1Fn &k1, K2Fn &k2)
+static void kernels_for(K1Fn &k1, KFFn &kf, K2Fn &k2)
 {
     k1 = contraction1_kernel<NT>;
+    kf = finish_general_kernel<NT>;
     k2 = contraction2_kernel<NT>;
 }
 
@@ -564,12 +575,13 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
             return status_from(e);
     }
     K1Fn k1;
+    KFFn kf;
     K2Fn k2;
     switch (NT) {
-    case 1: kernels_for<1>(k1, k2); break;
-    case 2: kernels_for<2>(k1, k2); break;
-    case 3: kernels_for<3>(k1, k2); break;
-    default: kernels_for<4>(k1, k2); break;
+    case 1: kernels_for<1>(k1, kf, k2); break;
+    case 2: kernels_for<2>(k1, kf, k2); break;
+    case 3: kernels_for<3>(k1, kf, k2); break;
+    default: kernels_for<4>(k1, kf, k2); break;
     }
     int kb2max = 0;
     for (const LayerDev &d : P.host) kb2max = std::max(kb2max, d.KB2);
@@ -614,6 +626,8 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
         const int grid2 = std::max(1, std::min(n2, g_sms * occ2));
         k1<<<grid1, kDecodeThreads, smem1, s>>>(P.dev, P.p1 + P.p1_start[b], n1, io, base, M, P.err);
         profile_mark(++*launches, s);
+        kf<<<cnt, kFinishGeneralThreads, 0, s>>>(P.dev, base, M);
+        profile_mark(++*launches, s);
         k2<<<grid2, kDecodeThreads, smem2, s>>>(P.dev, P.p2 + P.p2_start[b], n2, io, base, M, kb2max, P.err);
         profile_mark(++*launches, s);
     }
@@ -643,12 +657,13 @@ lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc,
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return status_from(e);
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return status_from(e);
     K1Fn k1;
+    KFFn kf;
     K2Fn k2;
     switch (NT) {
-    case 1: kernels_for<1>(k1, k2); break;
-    case 2: kernels_for<2>(k1, k2); break;
-    case 3: kernels_for<3>(k1, k2); break;
-    default: kernels_for<4>(k1, k2); break;
+    case 1: kernels_for<1>(k1, kf, k2); break;
+    case 2: kernels_for<2>(k1, kf, k2); break;
+    case 3: kernels_for<3>(k1, kf, k2); break;
+    default: kernels_for<4>(k1, kf, k2); break;
     }
     const int kb2max = host_desc.KB2;
     const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * kP1StageKB * 256 +
@@ -669,6 +684,8 @@ lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc,
     const int grid1 = std::max(1, std::min(n1, sms * std::max(1, occ1)));
     const int grid2 = std::max(1, std::min(n2, sms * std::max(1, occ2)));
     k1<<<grid1, kDecodeThreads, smem1, s>>>(dev_desc, p1, n1, io, 0, M, err);
+    ++*launches;
+    kf<<<1, kFinishGeneralThreads, 0, s>>>(dev_desc, 0, M);
     ++*launches;
     k2<<<grid2, kDecodeThreads, smem2, s>>>(dev_desc, p2, n2, io, 0, M, kb2max, err);
     ++*launches;

@@ -101,13 +101,11 @@ struct LayerDev {
     //         [2][16]  double  sum over k of t (per path x activation row)
     //         [2][16]  int     non-finite flags (per path x activation row)
     //   zfrag [kMaxNT][KB2][32] B fragments of contraction 2, zmeta [2][16] (exponent, digit sum)
-    //   counter: contraction-1 items finished (the last one builds zfrag and clears acc)
     //   xfrag [KB1][32] B fragments of contraction 1 (one or two rows: 16 * M lanes per k-block)
     //   xmeta [nkc][2][2] exponent of each (k chunk, path, row)
     double *acc;
     uint2 *zfrag;
     int2 *zmeta;
-    unsigned *counter;
     uint2 *xfrag;
     int *xmeta;
 };

@@ -155,7 +155,6 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
         d.acc = (double *)c;       c += align256(acc_doubles(d.R1) * sizeof(double));
         d.zfrag = (uint2 *)c;      c += align256((size_t)kMaxNT * d.KB2 * 32 * sizeof(uint2));
         d.zmeta = (int2 *)c;       c += align256((size_t)2 * 16 * sizeof(int2));
-        d.counter = (unsigned *)c; c += align256(sizeof(unsigned));
         d.xfrag = (uint2 *)c;      c += align256((size_t)d.KB1 * 32 * sizeof(uint2));
         d.xmeta = (int *)c;
         P.host[i] = d;

@@ -18,7 +18,6 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[LB_NOALLOC_SCRA
 // Offsets inside the array.
 constexpr size_t kOffDesc = 0;        // LayerDev (the kernels read descriptors from device memory)
 constexpr size_t kOffErr = 256;       // int error code
-constexpr size_t kOffCounter = 512;   // unsigned completion counter
 constexpr size_t kOffMeta = 768;      // int2 [2][16]
 constexpr size_t kOffAcc = 1024;      // double accumulators, then the fragments
 
@@ -33,7 +32,6 @@ __global__ void noalloc_setup_kernel(LayerDev d, size_t acc_n)
 {
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         *reinterpret_cast<LayerDev *>(g_noalloc_scratch + kOffDesc) = d;
-        *reinterpret_cast<unsigned *>(g_noalloc_scratch + kOffCounter) = 0u;
     }
     double *acc = reinterpret_cast<double *>(g_noalloc_scratch + kOffAcc);
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < acc_n; i += (size_t)gridDim.x * blockDim.x)
@@ -80,7 +78,6 @@ extern "C" lb_status lb_linear_forward_noalloc(const uint16_t *x, int M, const l
     d.acc = reinterpret_cast<double *>(base + kOffAcc);
     d.zfrag = reinterpret_cast<uint2 *>(base + off_frag);
     d.zmeta = reinterpret_cast<int2 *>(base + kOffMeta);
-    d.counter = reinterpret_cast<unsigned *>(base + kOffCounter);
     d.xfrag = reinterpret_cast<uint2 *>(base + off_xfrag);
     d.xmeta = reinterpret_cast<int *>(base + off_xmeta);
     cudaStream_t s = (cudaStream_t)stream;
