@@ -171,13 +171,13 @@ LB_API lb_status lb_stack_forward(lb_stack *S, const uint16_t *const *xs, float 
  * allocates); this call does not.
  *
  * Same arguments, layouts and result as lb_linear_forward for M <= 16.  The
- * scratch of the two decode kernels (float64 accumulators, latent fragments,
- * completion counter, error code) lives in one fixed array of
+ * scratch of the decode kernels (float64 accumulators, latent fragments,
+ * error code) lives in one fixed array of
  * LB_NOALLOC_SCRATCH_BYTES bytes of static device memory inside this library,
  * which every GPU that loads the library holds until the process exits.  The
  * call issues no cudaMalloc, cudaFree or allocating library routine: it
  * launches one small kernel that writes the layer descriptor into that array
- * and clears the accumulators and counter, then the two decode kernels.
+ * and clears the accumulators, then the decode kernels.
  * The first call on each device looks the array's device address up once
  * (cudaGetSymbolAddress, with that device current); make that first call
  * before any stream capture begins.

@@ -2,8 +2,8 @@
 //
 // The notes page of LittleBit (section "Multi-scale compensation") evaluates
 // a path as  x (.) g -> . V_sign -> (.) l -> . U_sign^T -> (.) h  and
-// "Residual compensation" sums the primary and residual paths.  Two kernels
-// cover every layer of a plan (a stack) in one launch each:
+// "Residual compensation" sums the primary and residual paths.  Three kernels
+// cover every layer of a plan (a stack), one launch each:
 //
 //   contraction 1 (work item = one layer x 1024 inputs):
 //     t = x (.) g_p for both paths in 16-bit fixed point (one power-of-two
