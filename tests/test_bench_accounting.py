@@ -1,0 +1,71 @@
+"""The algorithmic work bench.py divides by, pinned to the method's own accounting (CPU).
+
+Bytes per layer are the packed signs and binary16 scales of both paths — the
+bits-per-weight formula of the wiki page on LittleBit and LittleBit-2 ("How to
+judge an ultra-low-bit scheme", point 1: factors and scales both count),
+BPW = sum over paths of (r (N + K) + 16 (N + K + r)) / (N K) — plus the bf16
+activations in and the float32 outputs out.  FLOPs per layer are those of the
+two binary contractions, 2 M r (K + N) per path (LittleBit paper notes page,
+"Multi-scale compensation": x (.) g -> . V_sign -> (.) l -> . U_sign^T -> (.) h);
+the dense 2 M N K the method avoids is never counted.
+"""
+
+from fractions import Fraction
+
+import pytest
+
+import bench
+from sub_bit_weight_b200 import synth
+
+
+def bpw(N, K, r, npaths=2):
+    return Fraction(npaths * (r * (N + K) + 16 * (N + K + r)), N * K)
+
+
+@pytest.mark.parametrize("wkey", ["single_512", "llama2_7b_0.1", "llama2_7b_0.55", "llama2_13b_0.3_prefill",
+                                  "llama2_70b_0.1"])
+def test_weight_bytes_follow_the_bits_per_weight_formula(wkey):
+    for s in synth.WORKLOADS[wkey].block:
+        k1, k2 = bench.layer_bytes(s, 0)          # M = 0: weights and scales only
+        assert Fraction(int(8 * (k1 + k2)), s.N * s.K) == bpw(s.N, s.K, s.r)
+
+
+@pytest.mark.parametrize("wkey,per_layer", [
+    # packed signs + scales of both paths per layer, worked out by hand from the formula
+    ("single_512", {"t": 8256}),
+    ("llama2_7b_0.1", {"q": 196928, "gate": 544256}),
+    ("llama2_7b_0.55", {"q": 1149056, "gate": 3084416}),
+    ("llama2_13b_0.3_prefill", {"q": 984512, "gate": 2654336}),
+    ("llama2_70b_0.1", {"q": 819936, "k": 110720, "gate": 2950336}),
+])
+def test_weight_bytes_of_the_workload_layers(wkey, per_layer):
+    shapes = {s.name: s for s in synth.WORKLOADS[wkey].block}
+    for name, want in per_layer.items():
+        s = shapes.get(name) or next(iter(shapes.values()))
+        assert sum(bench.layer_bytes(s, 0)) == want
+
+
+def test_stack_totals():
+    w = synth.WORKLOADS["llama2_70b_0.1"]
+    weights = sum(sum(bench.layer_bytes(s, 0)) for s in w.block) * w.nblocks
+    assert weights == pytest.approx(857.0e6, rel=1e-3)          # > L2: the stack streams from HBM
+    p = synth.WORKLOADS["llama2_13b_0.3_prefill"]
+    flops = sum(bench.layer_flops(s, 2048) for s in p.block) * p.nblocks
+    assert flops == pytest.approx(15.07e12, rel=1e-3)
+
+
+def test_activation_and_output_bytes():
+    s = synth.LayerShape("t", 300, 200, 7)
+    for M in (1, 5, 16):
+        k1, k2 = bench.layer_bytes(s, M)
+        k10, k20 = bench.layer_bytes(s, 0)
+        assert k1 - k10 == 2 * M * s.K            # x in, bfloat16
+        assert k2 - k20 == 4 * M * s.N            # y out, float32
+
+
+def test_flops_are_the_two_binary_contractions():
+    s = synth.LayerShape("t", 300, 200, 7)
+    assert bench.layer_flops(s, 3) == 2 * 3 * 2 * 7 * (200 + 300)
+    assert bench.layer_flops(s, 3, npaths=1) == 2 * 3 * 7 * (200 + 300)
+    st = bench.backward_stage_flops(s, 3)
+    assert sum(st.values()) == 2 * 3 * 2 * 7 * (3 * 200 + 2 * 300)
