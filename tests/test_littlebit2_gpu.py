@@ -80,6 +80,8 @@ def _parity(lib, W, r, npaths, itq_iters, R0s=None, iters=24):
     (1000, 513, 100, 2, 50),  # odd K, r not a multiple of 32
     (2048, 1024, 128, 1, 50),
     (600, 400, 200, 2, 12),   # r above the one-cluster polar kernel's limit: the grid-wide kernel
+    (130, 70, 1, 2, 5),       # r = 1: the rotation is +-1
+    (256, 512, 24, 1, 20),    # one path, K > N
 ])
 def test_parity_on_power_law_weights(lib, shape):
     N, K, r, npaths, it = shape
