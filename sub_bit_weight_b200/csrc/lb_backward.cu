@@ -463,10 +463,16 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
     if (cudaEventRecord(B->fork, s) != cudaSuccess || cudaStreamWaitEvent(B->side, B->fork, 0) != cudaSuccess)
         return LB_ERR_CUDA;
     cudaStream_t s2 = B->side;
+    // a failure from here on joins the side stream back into the caller's before returning
+    auto joined = [&](lb_status e) {
+        cudaEventRecord(B->join, s2);
+        cudaStreamWaitEvent(s, B->join, 0);
+        return e;
+    };
     // dx = 2^-E sum_p g (.) (dz 2^E V_s^T): the output contraction's epilogue multiplies by 2^-E (stat[2])
     if ((st = prefill_forward(B->Lt->self->plan, &B->Lt, dys, ys, M, s, &launches, 2, true, false, B->stat + 2)) !=
         LB_OK)
-        return st;
+        return joined(st);
     launches += 2;
     profile_mark(5, s);
 
@@ -475,11 +481,11 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
     cublasSetStream(B->blas, s2);
     if (cublasGemmEx(B->blas, CUBLAS_OP_N, CUBLAS_OP_T, K2, N, M, alpha, zf, CUDA_R_16F, K2, B->dy16, CUDA_R_16F, N,
                      zero_d, B->GU, CUDA_R_32F, K2, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-        return LB_ERR_CUDA;
+        return joined(LB_ERR_CUDA);
     profile_mark(6, s2);
     if (cublasGemmEx(B->blas, CUBLAS_OP_N, CUBLAS_OP_T, K2, K, M, alpha, dz, CUDA_R_16F, K2, B->x16, CUDA_R_16F, K,
                      zero_d, B->GV, CUDA_R_32F, K2, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-        return LB_ERR_CUDA;
+        return joined(LB_ERR_CUDA);
     profile_mark(7, s2);
     const int wpr = (r + 31) / 32;
     FactorArgs fu{}, fv{};
