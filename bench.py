@@ -11,6 +11,16 @@ prefill stack (M = 2048, tensor-core bound) as "prefill".
 Metric: algorithmic bytes (packed signs + binary16 scales + x + y) per second
 for decode, algorithmic FLOPs (2*M*2r*(K+N) per layer) per second for prefill.
 
+The JSON line also carries: "roofline" (the dominant kernel against the
+measured peak, with its full-size DRAM traffic while the kernel sources match
+the capture in profiles/traffic.txt), "e2e" (the same step through the C ABI
+from pinned host x to pinned host y, steps pipelined over two device buffer
+sets; the serial figure beside it), "cpu_baseline" (the float64 oracle on a
+bounded sample), "backward" (QAT backward of one Llama-2-13B-shaped block),
+"init" (Dual-SVID + residual initialisation of one Llama-2-7B-shaped block, and
+its LittleBit-2 variant with Joint-ITQ as "init.littlebit2"), clocks and
+tokens/s.
+
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
         python bench.py --impl reference ...   (the CPU oracle, timed as is)
 Multi-GPU: one process per GPU (torchrun); every rank runs the whole stack
