@@ -119,7 +119,8 @@ LB_API lb_status lb_layer_shape(const lb_layer *L, int *N, int *K, int *r, int *
 
 /* Bits per weight by the pages' accounting,
  *   sum_paths [r(N+K) * 1 + 16 (N+K+r)] / (N K),
- * padding excluded (aibk.xyz wiki, "How to judge", item 1).  0 for NULL. */
+ * padding excluded (wiki page on LittleBit and LittleBit-2, "How to judge an
+ * ultra-low-bit scheme", point 1).  0 for NULL. */
 LB_API double lb_layer_bpw(const lb_layer *L);
 
 /* Device bytes the layer owns (weights in all layouts, scales and scratch). */
