@@ -388,15 +388,17 @@ __global__ void __launch_bounds__(kDecodeThreads)
     unsigned char *ring = smem_raw;                                          // [NW][kP2Stages][kStage]
     uint2 *sB = (uint2 *)(smem_raw + (size_t)NW * kP2Stages * kStage);      // [NT][KB2][32]
     __shared__ uint64_t bars[NW][kP2Stages];
+    __shared__ uint64_t fbar;                    // the layer's zl fragments, one bulk copy per item
     __shared__ int sE[32], sQs[32];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;
     if (lane == 0)
         for (int s = 0; s < kP2Stages; ++s) bar_init(&bars[warp][s]);
+    if (tid == 0) bar_init(&fbar);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    __syncwarp();
-    uint32_t issued = 0, consumed = 0;
+    __syncthreads();
+    uint32_t issued = 0, consumed = 0, nitem = 0;
     unsigned char *my_ring = ring + (size_t)warp * kP2Stages * kStage;
 
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
@@ -418,17 +420,18 @@ __global__ void __launch_bounds__(kDecodeThreads)
                     ++issued;
                 }
             }
-        {
-            const uint4 *src = reinterpret_cast<const uint4 *>(dp->zfrag);
-            uint4 *dst = reinterpret_cast<uint4 *>(sB);
-            const int n16 = NT * KB2 * 32 * (int)sizeof(uint2) / 16;
-            for (int i = tid; i < n16; i += kDecodeThreads) dst[i] = __ldcg(src + i);
+        // the previous item's reads of sB are done (barrier at its end): one bulk copy brings this layer's fragments
+        if (tid == 0) {
+            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+            ring_fill(sB, dp->zfrag, (unsigned)(NT * KB2 * 32 * sizeof(uint2)), &fbar);
         }
         if (tid < 32) {
             const int2 mt = __ldcg(&dp->zmeta[tid]);
             sE[tid] = mt.x;
             sQs[tid] = mt.y;
         }
+        if (!ring_wait(&fbar, nitem & 1, err)) return;
+        ++nitem;
         __syncthreads();
 
         // ---- main stream: this warp's row groups of 64 outputs
