@@ -69,3 +69,12 @@ def test_flops_are_the_two_binary_contractions():
     assert bench.layer_flops(s, 3, npaths=1) == 2 * 3 * 7 * (200 + 300)
     st = bench.backward_stage_flops(s, 3)
     assert sum(st.values()) == 2 * 3 * 2 * 7 * (3 * 200 + 2 * 300)
+
+
+def test_peaks_fall_back_without_the_measured_file(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    pk = bench.peaks()
+    assert pk["src"] == "fallback" and pk["hbm_gbs"] == 6650.0 and pk["bf16_tflops"] == 1590.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 6500.0, "bf16_tflops": 1600.0}')
+    pk = bench.peaks()
+    assert pk["src"] == "measured" and pk["hbm_gbs"] == 6500.0 and pk["bf16_tflops_sustained"] == 1600.0

@@ -164,3 +164,12 @@ def test_rotation_aligns_the_factors_with_the_hypercube():
     X1 = lb2.itq_data(p1["U_prime"], p1["V_prime"])
     assert _loss(X1, np.eye(32)) == pytest.approx(p1["itq_loss"][-1], abs=1e-12)
     assert _loss(X1, np.eye(32)) < _loss(X0, np.eye(32))
+
+
+def test_random_rotation_generator():
+    # the seeded start rotations handed to both sides: orthogonal, reproducible, distinct per path
+    for r in (1, 5, 64):
+        Q = synth.random_rotation(3, r)
+        np.testing.assert_allclose(Q.T @ Q, np.eye(r), rtol=0, atol=1e-13)
+        np.testing.assert_array_equal(Q, synth.random_rotation(3, r))
+    assert not np.allclose(synth.random_rotation(3, 8, 0), synth.random_rotation(3, 8, 1))
