@@ -30,7 +30,8 @@
 // U' V'^T unchanged: X = [U' / rho_u ; V' / rho_v] (each factor scaled to
 // unit RMS entry), then `itq_iters` alternations of B = sign(X R) and
 // R = polar(X^T B) (orthogonal Procrustes; the polar factor by Newton-Schulz
-// iteration in one cooperative launch), and U' <- U' R, V' <- V' R before
+// iteration in one launch: one thread-block cluster for r <= 96, else a
+// cooperative grid), and U' <- U' R, V' <- V' R before
 // the signs.
 #include "littlebit_init.h"
 #include "lb_coop.cuh"
