@@ -136,17 +136,51 @@ def lb_pack_signs(F: torch.Tensor, packed: torch.Tensor | None = None, stream=No
     rows, r = F.shape
     if packed is None:
         packed = torch.empty((rows, (r + 31) // 32), dtype=torch.int32, device=F.device)
+    else:
+        _numel(packed, rows * ((r + 31) // 32), "packed")
     _check(_lib.lb_pack_signs(_dev(F, torch.float32, "F"), rows, r, _dev(packed, torch.int32, "packed"),
                               _stream(stream)), "lb_pack_signs")
     return packed
 
 
 def _u16(t: torch.Tensor, name: str) -> int:
-    if t.dtype in (torch.float16, torch.bfloat16, torch.int16, torch.uint16):
+    # binary16 values, or their bit patterns; bfloat16 is refused since its bits read as binary16 are other numbers
+    if t.dtype in (torch.float16, torch.int16, torch.uint16):
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA tensor")
         return t.data_ptr()
-    raise TypeError(f"{name} must be a 16-bit tensor, got {t.dtype}")
+    raise TypeError(f"{name} must be binary16 (float16, or its bit patterns as int16/uint16), got {t.dtype}")
+
+
+def _numel(t, n: int, name: str):
+    """The library takes bare pointers: a tensor shorter than the layout it stands for would be read or
+    written past its end on the device, so every size is checked here, before any call."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if t.numel() != n:
+        raise ValueError(f"{name} must hold {n} elements, got {t.numel()} (shape {tuple(t.shape)})")
+
+
+def _layer_arrays(N: int, K: int, r: int, U, V, h, g, l):
+    """Per-path pointer arrays of lb_layer_create / lb_backward_create: U[p] [N, ceil(r/32)] and
+    V[p] [K, ceil(r/32)] int32, h[p] [N], g[p] [K], l[p] [r] binary16, each size checked (invalid shapes
+    themselves are left to the library, which rejects them)."""
+    npaths = len(U)
+    wpr = (r + 31) // 32
+    sizes = {"U": N * wpr, "V": K * wpr, "h": N, "g": K, "l": r}
+    lists = (("U", U), ("V", V), ("h", h), ("g", g), ("l", l))
+    for name, lst in lists:
+        if len(lst) != npaths:
+            raise ValueError(f"{name} must have one entry per path")
+        if min(N, K, r) > 0:
+            for p, t in enumerate(lst):
+                _numel(t, sizes[name], f"{name}[{p}]")
+    arrs = []
+    for name, lst in lists:
+        ptrs = [_dev(t, torch.int32, f"{name}[{p}]") if name in ("U", "V") else _u16(t, f"{name}[{p}]")
+                for p, t in enumerate(lst)]
+        arrs.append((_vp * max(1, npaths))(*ptrs))
+    return npaths, arrs
 
 
 class Layer:
@@ -179,16 +213,7 @@ class Layer:
 def lb_layer_create(N: int, K: int, r: int, U, V, h, g, l, stream=None) -> Layer:
     """Per-path lists: U[p] int32 [N, ceil(r/32)], V[p] int32 [K, ceil(r/32)] (canonical packed),
     h[p] [N], g[p] [K], l[p] [r] binary16 (float16 or int16/uint16 bit patterns), all CUDA."""
-    npaths = len(U)
-    arrs = []
-    for name, lst in (("U", U), ("V", V), ("h", h), ("g", g), ("l", l)):
-        if len(lst) != npaths:
-            raise ValueError(f"{name} must have one entry per path")
-        if name in ("U", "V"):
-            ptrs = [_dev(t, torch.int32, f"{name}[{p}]") for p, t in enumerate(lst)]
-        else:
-            ptrs = [_u16(t, f"{name}[{p}]") for p, t in enumerate(lst)]
-        arrs.append((_vp * max(1, npaths))(*ptrs))
+    npaths, arrs = _layer_arrays(N, K, r, U, V, h, g, l)
     out = _vp()
     _check(_lib.lb_layer_create(ctypes.byref(out), N, K, r, npaths, *arrs, _stream(stream)), "lb_layer_create")
     return Layer(out.value, N, K, r, npaths)
@@ -408,14 +433,7 @@ class Backward:
 
 def lb_backward_create(N: int, K: int, r: int, U, V, h, g, l, stream=None) -> Backward:
     """Per-path lists as lb_layer_create: canonical packed U, V (int32) and binary16 h, g, l (CUDA)."""
-    npaths = len(U)
-    arrs = []
-    for name, lst in (("U", U), ("V", V), ("h", h), ("g", g), ("l", l)):
-        if len(lst) != npaths:
-            raise ValueError(f"{name} must have one entry per path")
-        ptrs = [_dev(t, torch.int32, f"{name}[{p}]") if name in ("U", "V") else _u16(t, f"{name}[{p}]")
-                for p, t in enumerate(lst)]
-        arrs.append((_vp * max(1, npaths))(*ptrs))
+    npaths, arrs = _layer_arrays(N, K, r, U, V, h, g, l)
     out = _vp()
     _check(_lib.lb_backward_create(ctypes.byref(out), N, K, r, npaths, *arrs, _stream(stream)), "lb_backward_create")
     return Backward(out.value, N, K, r, npaths)
@@ -423,9 +441,14 @@ def lb_backward_create(N: int, K: int, r: int, U, V, h, g, l, stream=None) -> Ba
 
 def lb_layer_backward(B: Backward, x: torch.Tensor, dy: torch.Tensor, U_lat, V_lat, stream=None) -> dict:
     """Gradients for x [M, K] (bfloat16) and dy [M, N] (float32): dx [M, K] and per-path lists dh, dg, dl, dU, dV."""
+    if x.dim() != 2 or x.shape[1] != B.K or tuple(dy.shape) != (x.shape[0], B.N):
+        raise ValueError(f"x must be [M, {B.K}] and dy [M, {B.N}]")
     M = x.shape[0]
-    if tuple(x.shape) != (M, B.K) or tuple(dy.shape) != (M, B.N):
-        raise ValueError("x must be [M, K] and dy [M, N]")
+    for name, lst, rows in (("U_lat", U_lat, B.N), ("V_lat", V_lat, B.K)):
+        if len(lst) != B.npaths:
+            raise ValueError(f"{name} must have one entry per path")
+        for p, t in enumerate(lst):
+            _numel(t, rows * B.r, f"{name}[{p}]")
     dev = x.device
     P = B.npaths
     out = {"dx": torch.empty((M, B.K), dtype=torch.float32, device=dev),
