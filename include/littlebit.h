@@ -137,7 +137,15 @@ LB_API size_t lb_layer_device_bytes(const lb_layer *L);
  * stream, or explicit events); concurrent calls on one layer race.
  * Non-finite values in a row of x give NaN in that row of y.
  * Errors: LB_ERR_INVALID_ARG (NULL, M < 0, misalignment), LB_ERR_OOM
- * (scratch growth for a larger M than before), LB_ERR_CUDA.
+ * (scratch growth for a larger M than before), LB_ERR_CUDA, and
+ * LB_ERR_UNSUPPORTED when the decode kernels cannot hold the layer's
+ * contraction-2 depth in shared memory.  Decode (M <= 16, and larger M when
+ * K is not a multiple of 8 or N not a multiple of 4, which then run as 16-row
+ * blocks) needs (8 + ceil(min(M,16)/4)) * KB2 * 256 bytes <= 227 KB, with
+ * KB2 = npaths * ceil(r/32) k-blocks of 32 latent indices: one path takes any
+ * r <= LB_MAX_RANK; two paths take r <= 1184 at every M, r <= 1600 at M <= 4.
+ * (For one or two rows and KB2 <= 64 a streaming design without this limit
+ * runs instead.)
  */
 LB_API lb_status lb_linear_forward(const uint16_t *x, int M, const lb_layer *L, float *y, void *stream);
 
@@ -186,8 +194,9 @@ LB_API lb_status lb_stack_forward(lb_stack *S, const uint16_t *const *xs, float 
  * that overlap on the GPU (different streams, or other host threads) race:
  * order them on one stream.
  * Errors: LB_ERR_INVALID_ARG (NULL, M < 0, misalignment), LB_ERR_UNSUPPORTED
- * (M > LB_DECODE_MAX_M, or the layer needs more than LB_NOALLOC_SCRATCH_BYTES
- * of scratch), LB_ERR_CUDA.  M = 0 is a valid empty call.
+ * (M > LB_DECODE_MAX_M, the layer needs more than LB_NOALLOC_SCRATCH_BYTES
+ * of scratch, or its contraction-2 depth exceeds the decode kernels' shared
+ * memory as for lb_linear_forward), LB_ERR_CUDA.  M = 0 is a valid empty call.
  */
 #define LB_NOALLOC_SCRATCH_BYTES (1u << 20)
 LB_API lb_status lb_linear_forward_noalloc(const uint16_t *x, int M, const lb_layer *L, float *y, void *stream);
