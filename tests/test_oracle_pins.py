@@ -312,3 +312,35 @@ def test_generator_sign_blocks_are_consistent():
     part = synth.sign_factor(1, 2, 0, synth.MAT_U, 50, 70, row0=13, row1=29)
     assert np.array_equal(full[13:29], part)
     assert 0.4 < np.mean(full < 0) < 0.6
+
+
+def _golden_splitmix64():
+    rows = []
+    with open(os.path.join(GOLDEN, "splitmix64.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                seed, n, out = (int(v) for v in line.split())
+                rows.append((seed, n, out))
+    return rows
+
+
+def test_generator_matches_splitmix64_reference_outputs():
+    # the shared input generator is SplitMix64 as published: output n of the stream keyed s is
+    # mix(s + (n + 1) * golden), the same value as the n-th call of the sequential generator seeded with s
+    rows = _golden_splitmix64()
+    assert len(rows) == 10
+    for seed, n, out in rows:
+        assert int(synth.splitmix64(seed, np.array([n]))[0]) == out, (seed, n)
+        assert synth._mix64_int(seed + (n + 1) * synth._GOLDEN) == out
+
+
+def test_generator_sign_layout_follows_its_definition():
+    # word n of row i covers columns 64 * (n % W64) .. +63, bit b is column 64 * (n % W64) + b, set bit = -1
+    seed, layer, path, mat, rows, r = 3, 1, 1, synth.MAT_V, 5, 150
+    w64 = (r + 63) // 64
+    key = synth.stream_key(seed, layer, path, mat)
+    F = synth.sign_factor(seed, layer, path, mat, rows, r)
+    for i in range(rows):
+        for j in range(r):
+            word = int(synth.splitmix64(key, np.array([i * w64 + j // 64]))[0])
+            assert F[i, j] == (-1.0 if (word >> (j % 64)) & 1 else 1.0), (i, j)
