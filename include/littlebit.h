@@ -51,7 +51,7 @@ extern "C" {
 typedef enum lb_status {
     LB_OK = 0,
     LB_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, misaligned buffer      */
-    LB_ERR_UNSUPPORTED = 2,  /* a valid request this build does not implement           */
+    LB_ERR_UNSUPPORTED = 2,  /* a valid request this library does not implement         */
     LB_ERR_OOM = 3,          /* a device allocation of the library failed               */
     LB_ERR_CUDA = 4,         /* the CUDA runtime returned an error                      */
     LB_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (state was reset)    */
