@@ -31,6 +31,12 @@
  *     (including an asynchronous error of earlier work on the device).
  *   - The caller keeps ownership of every buffer it passes; the library owns
  *     the objects it creates (lb_layer, lb_stack) and their device memory.
+ *   - Use one process per GPU, with one host thread making the calls.  The
+ *     library raises each kernel's shared-memory limit once per process and
+ *     remembers that it did, in an unlocked cache, while CUDA keeps the limit
+ *     per device.  A second GPU in the same process, or two threads whose
+ *     first calls overlap, can therefore see a launch fail with LB_ERR_CUDA.
+ *     Nothing faults.
  */
 #ifndef LITTLEBIT_H
 #define LITTLEBIT_H
