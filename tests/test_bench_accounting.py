@@ -10,6 +10,7 @@ two binary contractions, 2 M r (K + N) per path (LittleBit paper notes page,
 the dense 2 M N K the method avoids is never counted.
 """
 
+import os
 from fractions import Fraction
 
 import pytest
@@ -78,3 +79,32 @@ def test_peaks_fall_back_without_the_measured_file(tmp_path, monkeypatch):
     (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 6500.0, "bf16_tflops": 1600.0}')
     pk = bench.peaks()
     assert pk["src"] == "measured" and pk["hbm_gbs"] == 6500.0 and pk["bf16_tflops_sustained"] == 1600.0
+
+
+def test_dram_traffic_is_reported_only_for_the_sources_it_was_captured_with(tmp_path, monkeypatch):
+    # profiles/traffic.txt records, per kernel and workload, the DRAM bytes of one launch and a hash of the
+    # sources they were captured with; a changed source makes the figure null rather than stale
+    for kernel in bench.KERNEL_SOURCES:
+        assert all(os.path.exists(os.path.join(bench.CSRC, f)) for f in bench.KERNEL_SOURCES[kernel])
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    k = "contraction2_pair_kernel"
+    good = bench.source_hash(k)
+    (prof / "traffic.txt").write_text("# kernel workload source_sha16 dram_bytes_per_launch note\n"
+                                      f"{k} wl_a {good} 123456 x\n"
+                                      f"{k} wl_b {'0' * 16} 999 x\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic(k, "wl_a") == 123456.0
+    assert bench.measured_traffic(k, "wl_b") is None          # captured with other sources
+    assert bench.measured_traffic(k, "wl_c") is None          # never captured
+    assert bench.measured_traffic("prefill_kernel<0>", "wl_a") is None
+    # the hash covers every listed source: any edit changes it
+    src = tmp_path / "csrc"
+    src.mkdir()
+    for f in bench.KERNEL_SOURCES[k]:
+        (src / f).write_bytes(open(os.path.join(bench.CSRC, f), "rb").read())
+    monkeypatch.setattr(bench, "CSRC", str(src))
+    assert bench.source_hash(k) == good
+    last = src / bench.KERNEL_SOURCES[k][-1]
+    last.write_bytes(last.read_bytes() + b"\n")
+    assert bench.source_hash(k) != good
