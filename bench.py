@@ -136,15 +136,34 @@ class ClockSampler:
         self.period = period
         self._stop = threading.Event()
         self.max_mhz = None
+        self.nvml_index = None
         try:
             import pynvml
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.nvml_index = self.nvml_index_of(pynvml, index)
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self.nvml_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
         except Exception as e:  # NVML missing: report that
             self.nv = None
             self.err = str(e)
+
+    @staticmethod
+    def nvml_index_of(nv, torch_index: int) -> int:
+        """NVML index of CUDA device ``torch_index``: the NVML device with the same PCI domain, bus and device
+        numbers (CUDA_VISIBLE_DEVICES renumbers the devices CUDA sees, not those NVML sees); the same index
+        when no device matches or the lookup fails."""
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(torch_index)
+            want = (int(p.pci_domain_id), int(p.pci_bus_id), int(p.pci_device_id))
+            for i in range(nv.nvmlDeviceGetCount()):
+                info = nv.nvmlDeviceGetPciInfo(nv.nvmlDeviceGetHandleByIndex(i))
+                if (int(info.domain), int(info.bus), int(info.device)) == want:
+                    return i
+        except Exception:
+            pass
+        return torch_index
 
     def _run(self):
         while not self._stop.is_set():
@@ -173,7 +192,8 @@ class ClockSampler:
         if not self.nv:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "nvml_index": self.nvml_index}
 
 
 # ----------------------------------------------------------------- CPU oracle baseline
