@@ -71,8 +71,8 @@ CSRC = os.path.join(ROOT, "sub_bit_weight_b200", "csrc")
 KERNEL_SOURCES = {
     "quantize_pair_kernel": ["lb_decode_pair.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
     "finish_pair_kernel": ["lb_decode_pair.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
-    "contraction1_pair_kernel": ["lb_decode_pair.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
-    "contraction2_pair_kernel": ["lb_decode_pair.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
+    "contraction1_ldg_kernel": ["lb_decode_pair.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
+    "contraction2_ldg_kernel": ["lb_decode_pair.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
     "contraction1_kernel": ["lb_decode.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
     "contraction2_kernel": ["lb_decode.cu", "lb_decode_common.cuh", "lb_internal.cuh"],
     "prefill_kernel<0>": ["lb_prefill.cu", "lb_prefill.cuh", "lb_prefill_types.cuh", "lb_internal.cuh"],
@@ -485,7 +485,7 @@ def main():
                     "per_kernel_ms": {"latent": round(k1ms, 4), "output": round(k2ms, 4)},
                     "per_kernel_flops": {"latent": f1, "output": f2}}
         else:
-            suffix = "_pair_kernel" if M <= 2 else "_kernel"
+            suffix = "_ldg_kernel" if M <= 2 else "_kernel"
             names = ["contraction1" + suffix, "contraction2" + suffix]
             kbytes = [k1b, k2b]
             if len(res["per_launch"]) == 3:
@@ -496,7 +496,7 @@ def main():
                 # activation quantisation and the contraction-1 finish run as their own launches:
                 # x and g are the bytes of the first, the finish moves no algorithmic bytes
                 qb = sum(2.0 * M * s.K + 2 * 2.0 * s.K for s in shapes)
-                names = ["quantize" + suffix, names[0], "finish" + suffix, names[1]]
+                names = ["quantize_pair_kernel", names[0], "finish_pair_kernel", names[1]]
                 kbytes = [qb, k1b - qb, 0.0, k2b]
             kms = list(res["per_launch"])
             di = max(range(len(kms)), key=lambda i: kms[i])

@@ -196,9 +196,15 @@ LB_API lb_status lb_stack_forward(lb_stack *S, const uint16_t *const *xs, float 
  * The first call on each device looks the array's device address up once
  * (cudaGetSymbolAddress, with that device current); make that first call
  * before any stream capture begins.
- * Every call shares the one array and leaves its contents behind, so calls
- * that overlap on the GPU (different streams, or other host threads) race:
- * order them on one stream.
+ * Every call writes the descriptor and clears the accumulators at its start;
+ * the other parts of the array (fragments, exponents) are overwritten before
+ * they are read, and otherwise keep the last call's contents.  Calls share the
+ * one array, so calls that overlap on the GPU (different streams, or other
+ * host threads) race: order them on one stream.
+ * A bounded device-side wait that gives up during this call records its code
+ * in the layer's own error slot (device memory allocated with the layer, the
+ * slot lb_linear_forward reports to as well); lb_layer_status reads and
+ * clears it.
  * Errors: LB_ERR_INVALID_ARG (NULL, M < 0, misalignment), LB_ERR_UNSUPPORTED
  * (M > LB_DECODE_MAX_M, the layer needs more than LB_NOALLOC_SCRATCH_BYTES
  * of scratch, or its contraction-2 depth exceeds the decode kernels' shared
@@ -227,6 +233,16 @@ LB_API lb_status lb_layer_status(const lb_layer *L, void *stream);
  * LB_OK if it did not.  No GPU fault or hang is involved.
  */
 LB_API lb_status lb_selftest_wait_timeout(long long cycles, void *stream);
+
+/*
+ * The same self-test aimed at a layer's error slot, the slot the layer's
+ * decode kernels report to (lb_linear_forward and lb_linear_forward_noalloc):
+ * launches the waiting thread on `stream` and returns without synchronising;
+ * a following lb_layer_status(L, stream) returns LB_ERR_TIMEOUT once (and
+ * clears the slot).  Errors: L NULL or cycles < 0 -> LB_ERR_INVALID_ARG,
+ * LB_ERR_CUDA.
+ */
+LB_API lb_status lb_layer_selftest_wait_timeout(const lb_layer *L, long long cycles, void *stream);
 
 /* Timing hook.  Registers n CUDA events (cudaEvent_t passed as void*) for the
  * calling thread: the following forward calls record events[0] on their

@@ -143,7 +143,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
         const P1Item item = items[it];
         const LayerDev *dp = layers + item.layer;
-        const int K = dp->K, K32 = dp->K32, KB1 = dp->KB1, RG1 = dp->RG1, r16 = dp->r16, npaths = dp->npaths;
+        const int K = dp->K, K32 = dp->K32, KB1 = dp->KB1, KB1e = dp->KB1e, RG1 = dp->RG1, r16 = dp->r16,
+                  npaths = dp->npaths;
         const uint2 *__restrict__ vt = dp->vt;
         const __half *__restrict__ gsc = dp->g;
         double *__restrict__ acc = dp->acc;
@@ -160,8 +161,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
             const int rg = warp + NW * (q / hp), h = q % hp;
             const int n = min(kHalf, nkb - h * kHalf);
             const int st = issued % kP1Stages;
-            ring_fill(my_ring + st * kStage, vt + ((size_t)rg * KB1 + kb0 + h * kHalf) * 32, (unsigned)n * 256u,
-                      &bars[warp][st]);
+            // k-blocks come in pairs: an odd last stage also brings the (empty) padding k-block
+            ring_fill(my_ring + st * kStage, vt + ((size_t)rg * KB1e + kb0 + h * kHalf) * 32,
+                      (unsigned)((n + 1) & ~1) * 256u, &bars[warp][st]);
             ++issued;
         };
 
@@ -317,13 +319,13 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 const uint32_t ph = (consumed / kP1Stages) & 1;
                 if (!ring_wait(&bars[warp][st], ph, err)) return;
                 ++consumed;
-                const uint32_t src = sm_addr(my_ring + st * kStage) + lane * 8;
+                const uint32_t src = sm_addr(my_ring + st * kStage) + lane * 16;   // pairs of k-blocks
                 const uint32_t bbase = sm_addr(sB) + lane * 8;
                 const int kbA = h * kHalf, n = min(kHalf, nkb - kbA);
 #pragma unroll 4
                 for (int u = 0; u < n; ++u) {
                     const int kb = kbA + u;
-                    const uint2 w = lds64(src + u * 256);
+                    const uint2 w = lds64(src + (u >> 1) * 512 + (u & 1) * 8);
                     uint2 bp[2][NT];
 #pragma unroll
                     for (int p = 0; p < 2; ++p)
@@ -384,7 +386,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
 {
     constexpr int NW = kDecodeThreads / 32;
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    const int kStage = kb2max * 256;
+    const int kStage = ((kb2max + 1) & ~1) * 256;                           // a row group's KB2e k-blocks
     unsigned char *ring = smem_raw;                                          // [NW][kP2Stages][kStage]
     uint2 *sB = (uint2 *)(smem_raw + (size_t)NW * kP2Stages * kStage);      // [NT][KB2][32]
     __shared__ uint64_t bars[NW][kP2Stages];
@@ -404,19 +406,19 @@ __global__ void __launch_bounds__(kDecodeThreads)
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
         const P2Item item = items[it];
         const LayerDev *dp = layers + item.layer;
-        const int N = dp->N, N64 = dp->N64, KB2 = dp->KB2, r32 = dp->r32;
+        const int N = dp->N, N64 = dp->N64, KB2 = dp->KB2, KB2e = dp->KB2e, r32 = dp->r32;
         const int npaths = dp->npaths;
         const uint2 *__restrict__ ut = dp->ut;
         const __half *__restrict__ hsc = dp->h;
         float *__restrict__ y = io.y[item.layer - base];
-        const unsigned stage_bytes = (unsigned)KB2 * 256u;
+        const unsigned stage_bytes = (unsigned)KB2e * 256u;
 
         if (lane == 0)
             for (int s = 0; s < kP2Stages; ++s) {
                 const int rg = item.rg0 + warp + NW * s;
                 if (rg < item.rg1) {
                     const int st = issued % kP2Stages;
-                    ring_fill(my_ring + (size_t)st * kStage, ut + (size_t)rg * KB2 * 32, stage_bytes, &bars[warp][st]);
+                    ring_fill(my_ring + (size_t)st * kStage, ut + (size_t)rg * KB2e * 32, stage_bytes, &bars[warp][st]);
                     ++issued;
                 }
             }
@@ -450,7 +452,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 }
             if (!ring_wait(&bars[warp][st], ph, err)) return;
             ++consumed;
-            const uint32_t src = sm_addr(my_ring + (size_t)st * kStage) + lane * 8;
+            const uint32_t src = sm_addr(my_ring + (size_t)st * kStage) + lane * 16;   // pairs of k-blocks
             const uint32_t bbase = sm_addr(sB) + lane * 8;
             float yv[4][NT][2];
 #pragma unroll
@@ -467,7 +469,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
                         for (int c = 0; c < 4; ++c) a4[rb][n][c] = 0;
 #pragma unroll 4
                 for (int kb = p * kbp; kb < (p + 1) * kbp; ++kb) {
-                    const uint2 w = lds64(src + kb * 256);
+                    const uint2 w = lds64(src + (kb >> 1) * 512 + (kb & 1) * 8);
                     uint2 b[NT];
 #pragma unroll
                     for (int n = 0; n < NT; ++n) b[n] = lds64(bbase + (uint32_t)((n * KB2 + kb) * 256));
@@ -502,7 +504,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 if (rgn < item.rg1) {
                     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
                     const int sn = issued % kP2Stages;
-                    ring_fill(my_ring + (size_t)sn * kStage, ut + (size_t)rgn * KB2 * 32, stage_bytes, &bars[warp][sn]);
+                    ring_fill(my_ring + (size_t)sn * kStage, ut + (size_t)rgn * KB2e * 32, stage_bytes, &bars[warp][sn]);
                     ++issued;
                 }
             }
@@ -590,7 +592,7 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
     for (const LayerDev &d : P.host) kb2max = std::max(kb2max, d.KB2);
     const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * kP1StageKB * 256 +
                          (size_t)2 * kP1ChunkKB * NT * 32 * sizeof(uint2);
-    const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * kb2max * 256 +
+    const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * ((kb2max + 1) & ~1) * 256 +
                          (size_t)NT * kb2max * 32 * sizeof(uint2);
     if (smem2 > 227 * 1024) return LB_ERR_UNSUPPORTED;
     if ((e = ensure_smem((const void *)k1, smem1, g_smem_set1[NT])) != cudaSuccess) return status_from(e);
@@ -616,11 +618,8 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
         const int n1 = P.p1_start[b + 1] - P.p1_start[b];
         const int n2 = P.p2_start[b + 1] - P.p2_start[b];
         if (M <= 2 && kb2max <= kPairMaxKB2) {
-            const int W = P.pair_warps[M - 1];
-            lb_status st = decode_pair_launch(P.dev, cnt, P.p1 + P.p1_start[b], n1, P.u1, P.wr1[M - 1] + (size_t)b * (W + 1),
-                                              P.u2, P.wr2[M - 1] + (size_t)b * (P.pair_warps2[M - 1] + 1), W,
-                                              P.pair_warps2[M - 1], io, base, M, kb2max, P.rmax, P.err, s, launches,
-                                              true);
+            lb_status st = decode_pair_launch(P.dev, cnt, P.p1 + P.p1_start[b], n1, P, b, io, base, M, kb2max, P.rmax,
+                                              P.err, s, launches, true);
             if (st == LB_OK) continue;
             if (st != LB_ERR_UNSUPPORTED) return st;
             // shapes the streaming kernels cannot hold in shared memory take the general kernels
@@ -651,8 +650,10 @@ lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc,
         static thread_local IoPtrs io1;
         io1.x[0] = x;
         io1.y[0] = y;
-        return decode_pair_launch(dev_desc, 1, p1, n1, P.u1, P.wr1[M - 1], P.u2, P.wr2[M - 1], P.pair_warps[M - 1],
-                                  P.pair_warps2[M - 1], io1, 0, M, host_desc.KB2, host_desc.r, err, s, launches, false);
+        lb_status st = decode_pair_launch(dev_desc, 1, p1, n1, P, 0, io1, 0, M, host_desc.KB2, host_desc.r, err, s,
+                                          launches, false);
+        if (st != LB_ERR_UNSUPPORTED) return st;
+        // as in decode_forward: a shape the streaming kernels cannot hold takes the general kernels
     }
     const int NT = (M + 3) / 4;
     cudaError_t e = cudaSuccess;
@@ -671,7 +672,7 @@ lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc,
     const int kb2max = host_desc.KB2;
     const size_t smem1 = (size_t)(kDecodeThreads / 32) * kP1Stages * kP1StageKB * 256 +
                          (size_t)2 * kP1ChunkKB * NT * 32 * sizeof(uint2);
-    const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * kb2max * 256 +
+    const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * ((kb2max + 1) & ~1) * 256 +
                          (size_t)NT * kb2max * 32 * sizeof(uint2);
     if (smem2 > 227 * 1024) return LB_ERR_UNSUPPORTED;
     if ((e = ensure_smem((const void *)k1, smem1, g_smem_set1[NT])) != cudaSuccess) return status_from(e);

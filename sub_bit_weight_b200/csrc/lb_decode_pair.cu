@@ -10,22 +10,23 @@
 //
 // so one MMA per (row block, k-block) serves both paths.  For M = 1 only the
 // first 16 lanes of a B fragment carry data; those fragments are stored
-// compactly (16 * M lanes per k-block) and the other lanes read zeros.
+// compactly (16 * M lanes per k-block).
 //
 // Four launches:
 //   quantize_pair_kernel      x (.) g_p as 16-bit fixed point per 1024-input
 //                             chunk -> contraction-1 B fragments + exponents
-//   contraction1_pair_kernel  z = sum_k b * t over V tiles, float64 atomics
+//   contraction1_ldg_kernel   z = sum_k b * t over V tiles, float64 atomics
 //   finish_pair_kernel        zl = z (.) l_p as 16-bit fixed point -> the
 //                             contraction-2 B fragments (one CTA per layer)
-//   contraction2_pair_kernel  y = sum_p h_p (.) (U_p zl_p) over U tiles
+//   contraction2_ldg_kernel   y = sum_p h_p (.) (U_p zl_p) over U tiles
 // The float64 row sums of contraction 1 use the first R1 * M doubles of the
 // layer's accumulator block as a compact [R1][M] array (the general decode
 // kernels use [R1][16]); both leave the block zero for the next call.
-// In both contractions every warp streams its own contiguous, equal share of
-// the weight bytes (a static partition made at plan build) through a private
-// ring of bulk copies; warps never synchronise with each other.
+// In both contractions every warp streams its own range of units (a
+// cost-balanced partition made at plan build) straight into registers;
+// warps never synchronise with each other.
 
+#include <algorithm>
 #include <utility>
 
 #include "lb_decode_common.cuh"
@@ -37,12 +38,6 @@ namespace lb {
 // L of the chunk (32 inputs) and writes that k-block's whole B fragment.
 // ---------------------------------------------------------------------------
 constexpr int kQuantWarps = 4;
-
-// The four bytes of 32-bit values a..d, low byte first.
-static __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
-{
-    return (uint32_t)(a & 255) | ((uint32_t)(b & 255) << 8) | ((uint32_t)(c & 255) << 16) | ((uint32_t)(d & 255) << 24);
-}
 
 template <int MM>
 __global__ void __launch_bounds__(kQuantWarps * 32, MM == 1 ? 5 : 3)
@@ -107,16 +102,20 @@ __global__ void __launch_bounds__(kQuantWarps * 32, MM == 1 ? 5 : 3)
         return xv * gv;
     };
 
-    uint4 *dst = reinterpret_cast<uint4 *>(dp->xfrag + (size_t)kb * 16 * MM);
+    // k-block kb's fragment: lane L at uint2 (pair * 16 MM + L) * 2 + (kb & 1), pair = kb / 2
+    uint2 *dst = dp->xfrag + (size_t)(kb >> 1) * 32 * MM + (kb & 1);
 #pragma unroll
     for (int m = 0; m < MM; ++m)
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
+            // every product once: the chunk maximum and the digits both read t[]
+            float t[32];
             float amax = 0.0f;
             int bad = 0;
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-                const float tv = fabsf(tval(m, p, e));
+                t[e] = tval(m, p, e);
+                const float tv = fabsf(t[e]);
                 if (!(tv <= FLT_MAX)) bad = 1;
                 else amax = fmaxf(amax, tv);
             }
@@ -124,29 +123,34 @@ __global__ void __launch_bounds__(kQuantWarps * 32, MM == 1 ? 5 : 3)
             bad = warp_or(bad);
             const bool live = m < M && p < npaths;
             const int E = live ? exponent_for(amax, bad != 0) : kNanExp;
-            const float sc = (E == kNanExp) ? 0.0f : pow2f(E);
-            // column 4 m + 2 p + d: lanes t = 0..3 hold k 4t..4t+3 (first word) and 16+4t.. (second);
-            // one 16-byte store covers lanes 2 tp and 2 tp + 1 of a column
+            // q = rint(t 2^E).  t 2^E is exact and |t 2^E| <= 32639 < 2^22, so one FMA that adds 1.5 * 2^23
+            // rounds it to the nearest integer (ties to even) in the low mantissa bits, and subtracting the
+            // bit pattern of 1.5 * 2^23 leaves q.  An absent or non-finite block gives q = 0.
+            const bool none = E == kNanExp;
+            const float sc = none ? 0.0f : pow2f(E);
             int qs = 0;
 #pragma unroll
             for (int tp = 0; tp < 2; ++tp) {
                 uint32_t wlo[4], whi[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int t = 2 * tp + (i >> 1), k = 16 * (i & 1) + 4 * t;
-                    int q[4];
+                    const int tt = 2 * tp + (i >> 1), k = 16 * (i & 1) + 4 * tt;
+                    int q[4], hq[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        q[e] = quantize_s(tval(m, p, k + e), sc);
+                        q[e] = __float_as_int(fmaf(none ? 0.0f : t[k + e], sc, 12582912.0f)) - 0x4B400000;
+                        hq[e] = q[e] + 128;         // the high digit (q + 128) >> 8 is byte 1 of q + 128
                         qs += q[e];
                     }
-                    wlo[i] = pack4(q[0], q[1], q[2], q[3]);
-                    whi[i] = pack4((q[0] + 128) >> 8, (q[1] + 128) >> 8, (q[2] + 128) >> 8, (q[3] + 128) >> 8);
+                    wlo[i] = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+                    whi[i] = __byte_perm(__byte_perm(hq[0], hq[1], 0x0051), __byte_perm(hq[2], hq[3], 0x0051), 0x5410);
                 }
                 if (act) {
-                    const int col = 4 * m + 2 * p;
-                    dst[2 * col + tp] = make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
-                    dst[2 * (col + 1) + tp] = make_uint4(whi[0], whi[1], whi[2], whi[3]);
+                    const int l0 = 4 * (4 * m + 2 * p) + 2 * tp;      // column 4 m + 2 p, lanes 2 tp and 2 tp + 1
+                    dst[2 * l0] = make_uint2(wlo[0], wlo[1]);
+                    dst[2 * (l0 + 1)] = make_uint2(wlo[2], wlo[3]);
+                    dst[2 * (l0 + 4)] = make_uint2(whi[0], whi[1]);
+                    dst[2 * (l0 + 5)] = make_uint2(whi[2], whi[3]);
                 }
             }
             qs = warp_sum(qs);
@@ -184,7 +188,7 @@ __global__ void __launch_bounds__(kFinishThreads)
     const int tid = threadIdx.x;
     dep_release();
     const LayerDev *dp = layers + base + blockIdx.x;
-    const int R1 = dp->R1, r = dp->r, r16 = dp->r16, r32 = dp->r32, npaths = dp->npaths, KB2 = dp->KB2;
+    const int R1 = dp->R1, r = dp->r, r16 = dp->r16, r32 = dp->r32, npaths = dp->npaths;
     double *acc = dp->acc;
     const __half *lsc = dp->l;
     dep_wait();                          // the row sums of contraction 1
@@ -216,7 +220,7 @@ __global__ void __launch_bounds__(kFinishThreads)
     }
     __syncthreads();
     // fragment word pairs: lane L < 16 * MM of k-block kb holds column L / 4 = 4 m + 2 p + d
-    for (int idx = tid; idx < KB2 * 16 * MM; idx += kFinishThreads) {
+    for (int idx = tid; idx < dp->KB2e * 16 * MM; idx += kFinishThreads) {
         const int kb = idx / (16 * MM), lane = idx - kb * 16 * MM;
         const int col = lane >> 2, t = lane & 3;
         const int fm = col >> 2, fp = (col >> 1) & 1, fd = col & 1;
@@ -239,7 +243,7 @@ __global__ void __launch_bounds__(kFinishThreads)
                 }
             if (fd == 0 && qs) atomicAdd(&sQs[2 * fp + fm], qs);
         }
-        dp->zfrag[idx] = make_uint2(w[0], w[1]);
+        dp->zfrag[((size_t)(kb >> 1) * 16 * MM + lane) * 2 + (kb & 1)] = make_uint2(w[0], w[1]);
     }
     __syncthreads();
     if (tid < 4) {
@@ -252,423 +256,660 @@ __global__ void __launch_bounds__(kFinishThreads)
 }
 
 // ---------------------------------------------------------------------------
-// Per-warp streaming: a ring of kPairStages bulk-copy stages (kPairStageKB
-// k-blocks each) and two B slots (fragments + their metadata), one mbarrier
-// each.  Unit records are read one unit ahead so no global load sits on the
-// path from one unit to the next.
+// The two contractions, streamed warp by warp into registers.
+//
+// One CTA of kLdgWarps warps per SM; every warp owns a contiguous range of
+// units (64-row groups; the plan splits each batch's units into equal-cost
+// ranges, one per warp, cut into segments of one layer).  A warp runs two
+// streams at once, the two halves of each unit's k-range (stream 0 the first
+// ceil(P/2) pairs of k-blocks, stream 1 the rest), each with its own
+// accumulators, and keeps kLdgRing pairs of k-blocks per stream in flight in
+// registers: every step consumes the oldest pair of each stream and loads the
+// pair kLdgRing steps ahead, across unit and segment boundaries.  The weights
+// are read once (no L1 allocation, evict-first in L2); the B fragments of a
+// layer or chunk are reused by many units and stay in L1, loaded one step
+// ahead.  No shared memory, no barrier, no warp waits for another.
 // ---------------------------------------------------------------------------
 
-// N k-blocks of MMAs, fully unrolled: A word pairs 256 bytes apart, B fragments
-// 16 * MM * 8 bytes apart (lanes without B data read a zero buffer of the same
-// shape), so every shared-memory address is a register plus an immediate.
-template <int MM, int N>
-static __device__ __forceinline__ void mma_run(int (&a4)[4][4], uint32_t src, uint32_t bsrc)
+static __device__ __forceinline__ uint4 ldg_weights(const uint4 *p, uint64_t pol)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;\n"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
+// B fragments and exponents come from the previous kernel, which may still be finishing while this one starts
+// (programmatic dependent launch): they are read through L2 (.cg), never through the read-only path, whose
+// contents are only defined for data that stays unchanged for the kernel's whole lifetime.
+static __device__ __forceinline__ uint4 ldg_frag(const uint4 *p)
+{
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+// One k-block of MMAs: the lane's sign words (w0, w1) against its B fragment words (b0, b1).
+static __device__ __forceinline__ void kblock(int (&a4)[4][4], uint32_t w0, uint32_t w1, uint32_t b0, uint32_t b1)
 {
 #pragma unroll
-    for (int v = 0; v < N; ++v) {
-        const uint2 w = lds64(src + v * 256);
-        const uint2 b = lds64(bsrc + v * (16 * MM * 8));
+    for (int rb = 0; rb < 4; ++rb) {
+        const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
+        mma_u8s8(a4[rb], w0 & mlo, w0 & mhi, w1 & mlo, w1 & mhi, b0, b1);
+    }
+}
+
+// One step: a pair of k-blocks of each stream (the two halves of the unit's k-range), one accumulator set.
+static __device__ __forceinline__ void step_mma(int (&a4)[4][4], const uint4 &w0, const uint4 &w1, const uint4 &b0,
+                                                const uint4 &b1)
+{
+    kblock(a4, w0.x, w0.y, b0.x, b0.y);
+    kblock(a4, w1.x, w1.y, b1.x, b1.y);
+    kblock(a4, w0.z, w0.w, b0.z, b0.w);
+    kblock(a4, w1.z, w1.w, b1.z, b1.w);
+}
+
+static __device__ __forceinline__ void zero_acc(int (&a)[4][4])
+{
 #pragma unroll
-        for (int rb = 0; rb < 4; ++rb) {
-            const uint32_t mlo = 0x01010101u << rb, mhi = 0x01010101u << (rb + 4);
-            mma_u8s8(a4[rb], w.x & mlo, w.x & mhi, w.y & mlo, w.y & mhi, b.x, b.y);
+    for (int rb = 0; rb < 4; ++rb)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) a[rb][c] = 0;
+}
+
+// The weight stream of a warp: the address of the next pair of k-blocks of stream 0 (stream 1 reads h pairs
+// further, when the unit has that pair), walking steps, units and segments; runs kLdgRing steps ahead of the
+// MMAs.  Lanes 16..31 of one-row batches read the B data of lanes 0..15: their columns (activation row 1)
+// are computed and never used.
+template <typename Seg>
+struct Prefetch {
+    const uint4 *a;         // this lane's 16 bytes of the current unit's first pair
+    int t, h, P, rem, stride, s;
+    bool live;
+    __device__ __forceinline__ void seg(const Seg &sg, int lane, int rstride)
+    {
+        a = sg_base(sg) + lane;
+        P = sg.P;
+        h = (P + 1) >> 1;
+        rem = sg.n;
+        stride = rstride;
+        t = 0;
+    }
+    static __device__ __forceinline__ const uint4 *sg_base(const Seg1 &sg) { return sg.v; }
+    static __device__ __forceinline__ const uint4 *sg_base(const Seg2 &sg) { return sg.u; }
+};
+
+static __device__ __forceinline__ int seg_stride(const Seg1 &sg) { return sg.rstride; }
+static __device__ __forceinline__ int seg_stride(const Seg2 &sg) { return sg.P * 32; }
+
+// 512 bytes of zeros: the pair a stream reads where its unit has none (stream 1 of an odd number of pairs) or
+// past the warp's last unit, so that every ring load is unconditional and nothing waits on a load it issued
+static __device__ __align__(16) uint4 g_zero_pair[32];
+
+template <typename Seg>
+static __device__ __forceinline__ void fetch_step(Prefetch<Seg> &pf, const Seg *segs, int s1, int lane, uint64_t pol,
+                                                  uint4 &w0, uint4 &w1)
+{
+    const uint4 *zero = g_zero_pair + lane;
+    const uint4 *a0 = pf.live ? pf.a + pf.t * 32 : zero;
+    const uint4 *a1 = (pf.live && pf.h + pf.t < pf.P) ? a0 + pf.h * 32 : zero;
+    w0 = ldg_weights(a0, pol);
+    w1 = ldg_weights(a1, pol);
+    if (!pf.live) return;
+    if (++pf.t == pf.h) {
+        pf.t = 0;
+        if (--pf.rem > 0) {
+            pf.a += pf.stride;
+        } else if (++pf.s < s1) {
+            const Seg sg = segs[pf.s];
+            pf.seg(sg, lane, seg_stride(sg));
+        } else {
+            pf.live = false;
         }
     }
 }
 
-// n (1..kPairStageKB) k-blocks: a full stage in one unrolled body, otherwise the
-// binary decomposition of n (at most four unrolled bodies, no jump table).
-template <int MM>
-static __device__ __forceinline__ void mma_stage(int (&a4)[4][4], uint32_t src, uint32_t bsrc, int n)
-{
-    static_assert(kPairStageKB == 16, "stage of 16 k-blocks");
-    if (n == 16) {
-        mma_run<MM, 16>(a4, src, bsrc);
-        return;
-    }
-    if (n & 8) {
-        mma_run<MM, 8>(a4, src, bsrc);
-        src += 8 * 256;
-        bsrc += 8 * (16 * MM * 8);
-    }
-    if (n & 4) {
-        mma_run<MM, 4>(a4, src, bsrc);
-        src += 4 * 256;
-        bsrc += 4 * (16 * MM * 8);
-    }
-    if (n & 2) {
-        mma_run<MM, 2>(a4, src, bsrc);
-        src += 2 * 256;
-        bsrc += 2 * (16 * MM * 8);
-    }
-    if (n & 1) mma_run<MM, 1>(a4, src, bsrc);
-}
-
 // ---------------------------------------------------------------------------
-// Contraction 1 (one warp per contiguous run of units).  A ring stage holds up
-// to kPairStageKB k-blocks of one unit's V tiles, the B fragments of the same
-// k-blocks and the chunk's four exponents (three bulk copies on one mbarrier);
-// nothing else is shared between units, so the warp needs no B slots.
+// Contraction 1: z_p = sum_k t_p[k] V_sign,p[k][.] for every latent row.  A
+// unit is a row group over one 1024-input chunk (P = ceil(nkb / 2) pairs);
+// its exact integer sums per (path, row) times 2^-E of the chunk go to
+// float64 accumulators.  A segment lies in one chunk, so its exponents and B
+// fragments serve all its units.
 // ---------------------------------------------------------------------------
 template <int MM>
-__global__ void __launch_bounds__(pair_warps_per_cta(MM) * 32, 1)
-    contraction1_pair_kernel(const LayerDev *__restrict__ layers, const PairUnit1 *__restrict__ units,
-                             const int *__restrict__ wrange, int M, int *err)
+static __device__ __noinline__ void c1_generic(const LayerDev *__restrict__ layers, const Seg1 *__restrict__ segs,
+                                                  int s0, int s1, int M, int lane, uint64_t pol)
 {
-    constexpr int kBStride = 16 * MM * 8;                   // bytes of B fragments per k-block
-    constexpr int kA = kPairStageKB * 256, kB = kPairStageKB * kBStride;
-    constexpr int kStageAll = kA + kB + 16;                 // V tiles, B fragments, exponents
-    constexpr int kPairWarps = pair_warps_per_cta(MM);
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    __shared__ uint64_t rbar[kPairWarps][kPairStages];
-    __shared__ __align__(16) uint4 zbuf[MM == 1 ? kPairStageKB * 128 / 16 : 1];   // B of the lanes past 16 * MM
-
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t4 = lane & 3;
-    const int lane_m = t4 >> 1, lane_p = t4 & 1;       // accumulator columns of this lane
-    unsigned char *ring = smem_raw + warp * (kPairStages * kStageAll);
-    for (int i = threadIdx.x; i < (int)(sizeof(zbuf) / 16); i += blockDim.x) zbuf[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (lane == 0)
-        for (int s = 0; s < kPairStages; ++s) bar_init(&rbar[warp][s]);
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    __syncthreads();    // the only CTA-wide barrier: the zero buffer and the barriers are ready
-    dep_release();
+    const int lane_m = t4 >> 1, lane_p = t4 & 1;        // accumulator columns of this lane
+    const int blane = lane & (16 * MM - 1);
 
-    const int gw = warp * gridDim.x + blockIdx.x;     // an SM's warps take ranges spread over the whole batch
-    const int u0 = wrange[gw], u1 = wrange[gw + 1];
-    if (u0 >= u1) return;
-    const uint64_t pol = l2_evict_first();
-    // V tiles do not depend on the previous kernel; B fragments and exponents do: stages
-    // filled before dep_wait() get theirs afterwards (at most kPairStages of them)
-    bool dep_ok = false;
-    int npend = 0;
-    const uint2 *pend_b[kPairStages];
-    const int *pend_e[kPairStages];
-    unsigned pend_nb[kPairStages];
-
-    // ---- fill cursor: stages of units [f_u, u1) in consumption order, at most kPairStages ahead
-    int f_u = u0, f_h = 0, f_layer = -1, issued = 0, consumed = 0;
-    const uint2 *f_xfrag = nullptr;
-    const int *f_xmeta = nullptr;
-    PairUnit1 f_cur = units[u0], f_nxt = f_cur;
-    if (u0 + 1 < u1) f_nxt = units[u0 + 1];
-    auto fill = [&]() {
-        while (f_u < u1 && issued - consumed < kPairStages) {
-            if (f_cur.layer != f_layer) {
-                f_layer = f_cur.layer;
-                f_xfrag = layers[f_layer].xfrag;
-                f_xmeta = layers[f_layer].xmeta;
-            }
-            const int n = min(kPairStageKB, f_cur.nkb - f_h * kPairStageKB);
-            {
-                const int st = issued % kPairStages;
-                unsigned char *dst = ring + st * kStageAll;
-                uint64_t *bar = &rbar[warp][st];
-                const int kb0 = f_cur.kc * kP1ChunkKB + f_h * kPairStageKB;
-                const uint32_t lead = lane == 0;
-                lead_fill_hint(lead, bar, (unsigned)n * (256u + kBStride) + 16u, dst,
-                               f_cur.a + (size_t)f_h * kPairStageKB * 32, (unsigned)n * 256u, pol);
-                if (dep_ok) {
-                    lead_copy(lead, bar, dst + kA, f_xfrag + (size_t)kb0 * 16 * MM, (unsigned)n * kBStride);
-                    lead_copy(lead, bar, dst + kA + kB, f_xmeta + f_cur.kc * 4, 16u);
-                } else {
+    Prefetch<Seg1> pf;
+    pf.s = s0;
+    pf.live = true;
+    {
+        const Seg1 sg = segs[s0];
+        pf.seg(sg, lane, sg.rstride);
+    }
+    uint4 r0[kLdgRing], r1[kLdgRing];
 #pragma unroll
-                    for (int i = 0; i < kPairStages; ++i)
-                        if (i == npend) {
-                            pend_b[i] = f_xfrag + (size_t)kb0 * 16 * MM;
-                            pend_e[i] = f_xmeta + f_cur.kc * 4;
-                            pend_nb[i] = (unsigned)n * kBStride;
+    for (int d = 0; d < kLdgRing; ++d) fetch_step(pf, segs, s1, lane, pol, r0[d], r1[d]);
+
+    dep_wait();     // B fragments, exponents and cleared accumulators come from the previous kernels
+
+    // consumer: segment cs, row group crg, step ct of the unit
+    int cs = s0, crg = 0, ct = 0, ch = 1, cP = 1, crem = 0, npaths = 1, r16 = 0;
+    const uint4 *xb = nullptr;
+    double *acc = nullptr;
+    double lsc = 0.0;
+    bool elive = false;
+    auto seg_in = [&]() {
+        const Seg1 sg = segs[cs];
+        const LayerDev *dp = layers + sg.layer;
+        crg = sg.rg0;
+        crem = sg.n;
+        cP = sg.P;
+        ch = (cP + 1) >> 1;
+        xb = reinterpret_cast<const uint4 *>(dp->xfrag) + (size_t)sg.kc * (kP1ChunkKB / 2) * 16 * MM + blane;
+        acc = dp->acc;
+        npaths = dp->npaths;
+        r16 = dp->r16;
+        const int E = (lane_m < M && lane_p < npaths) ? __ldcg(dp->xmeta + sg.kc * 4 + 2 * lane_p + lane_m) : kNanExp;
+        elive = E != kNanExp;
+        lsc = elive ? pow2d(-E) : 0.0;
+    };
+    seg_in();
+    auto bload = [&](int t, uint4 &b0, uint4 &b1) {       // B pairs of step t (stream 1 clamped: its A is zero)
+        b0 = ldg_frag(xb + (size_t)t * 16 * MM);
+        b1 = ldg_frag(xb + (size_t)min(ch + t, cP - 1) * 16 * MM);
+    };
+    uint4 bn0, bn1;
+    bload(0, bn0, bn1);
+    int a4[4][4];
+    zero_acc(a4);
+    bool live = true;
+    while (live) {
+#pragma unroll
+        for (int d = 0; d < kLdgRing; ++d) {
+            if (live) {
+                const uint4 w0 = r0[d], w1 = r1[d], b0 = bn0, b1 = bn1;
+                fetch_step(pf, segs, s1, lane, pol, r0[d], r1[d]);
+                const bool unit_end = ct + 1 == ch;
+                bload(unit_end ? 0 : ct + 1, bn0, bn1);     // the next unit of the segment starts at step 0
+                step_mma(a4, w0, w1, b0, b1);
+                if (unit_end) {
+                    // keep the columns of each row block's own path; partial sums over chunks add up exactly
+                    if (elive) {
+#pragma unroll
+                        for (int rb = 0; rb < 4; ++rb) {
+                            const int row0 = crg * kRowsPerGroup + rb * kRowsPerBlock;
+                            const int prb = (npaths > 1 && row0 >= r16) ? 1 : 0;     // path 1 owns rows r16..
+                            if (prb != lane_p) continue;
+                            const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
+                            const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
+                            if (Tlo) atomicAdd(acc + (size_t)(row0 + g) * MM + lane_m, (double)Tlo * lsc);
+                            if (Thi) atomicAdd(acc + (size_t)(row0 + g + 8) * MM + lane_m, (double)Thi * lsc);
                         }
+                    }
+                    zero_acc(a4);
+                    ct = 0;
+                    if (--crem > 0) {
+                        ++crg;
+                    } else if (++cs < s1) {
+                        seg_in();
+                        bload(0, bn0, bn1);
+                    } else {
+                        live = false;
+                    }
+                } else {
+                    ++ct;
                 }
             }
-            if (!dep_ok) ++npend;
-            ++issued;
-            if (++f_h * kPairStageKB >= f_cur.nkb) {
-                f_h = 0;
-                ++f_u;
-                f_cur = f_nxt;
-                if (f_u + 1 < u1) f_nxt = units[f_u + 1];
-            }
-        }
-    };
-    fill();
-    dep_wait();
-    dep_ok = true;
-    if (lane == 0)
-#pragma unroll
-        for (int i = 0; i < kPairStages; ++i)
-            if (i < npend) {
-                unsigned char *dst = ring + i * kStageAll;
-                bulk_copy(dst + kA, pend_b[i], pend_nb[i], &rbar[warp][i]);
-                bulk_copy(dst + kA + kB, pend_e[i], 16u, &rbar[warp][i]);
-            }
-
-    // ---- consumer
-    int c_layer = -1, c_r16 = 1, c_npaths = 1;
-    double *c_acc = nullptr;
-    const bool real = lane < 16 * MM;
-    const uint32_t zaddr = sm_addr(zbuf) + (lane & 15) * 8;
-    PairUnit1 c_nxt = units[u0];
-    for (int u = u0; u < u1; ++u) {
-        const PairUnit1 cu = c_nxt;
-        if (u + 1 < u1) c_nxt = units[u + 1];
-        if (cu.layer != c_layer) {
-            const LayerDev *dp = layers + cu.layer;
-            c_layer = cu.layer;
-            c_acc = dp->acc;
-            c_r16 = dp->r16;
-            c_npaths = dp->npaths;
-        }
-        int a4[4][4];
-#pragma unroll
-        for (int rb = 0; rb < 4; ++rb)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) a4[rb][c] = 0;
-        double lane_sc = 0.0;
-        bool lane_live = false;
-        for (int h = 0; h * kPairStageKB < cu.nkb; ++h) {
-            const int st = consumed % kPairStages;
-            if (!ring_wait(&rbar[warp][st], (consumed / kPairStages) & 1, err)) return;
-            const uint32_t sbase = sm_addr(ring + st * kStageAll);
-            if (h == 0) {
-                const int E = (lane_m < M && lane_p < c_npaths) ? (int)lds_u32(sbase + kA + kB + 4 * (2 * lane_p + lane_m))
-                                                                 : kNanExp;
-                lane_live = E != kNanExp;
-                lane_sc = lane_live ? pow2d(-E) : 0.0;
-            }
-            mma_stage<MM>(a4, sbase + lane * 8, real ? sbase + kA + lane * 8 : zaddr,
-                          min(kPairStageKB, cu.nkb - h * kPairStageKB));
-            __syncwarp();
-            proxy_fence();
-            ++consumed;
-            fill();
-        }
-        // keep the columns of each row block's own path; partial sums over chunks add up exactly
-#pragma unroll
-        for (int rb = 0; rb < 4; ++rb) {
-            const int row0 = cu.rg * kRowsPerGroup + rb * kRowsPerBlock;
-            const int prb = (c_npaths > 1 && row0 >= c_r16) ? 1 : 0;     // path 1 owns rows r16..
-            if (prb != lane_p || !lane_live) continue;
-            const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
-            const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
-            if (Tlo) atomicAdd(c_acc + (size_t)(row0 + g) * MM + lane_m, (double)Tlo * lane_sc);
-            if (Thi) atomicAdd(c_acc + (size_t)(row0 + g + 8) * MM + lane_m, (double)Thi * lane_sc);
         }
     }
 }
 
 // ---------------------------------------------------------------------------
-// Contraction 2 (+ h, + path sum): one warp per contiguous run of row groups.
-// A layer's U tiles are contiguous over its row groups, so a ring stage takes
-// up to kPairStageKB consecutive k-blocks across row-group boundaries (never
-// across layers); the consumer folds a row group when its KB2 k-blocks are in.
+// Contraction 2 (+ h, + path sum): y[m][n] = sum_p h_p[n] * sum_j U_sign,p[n][j] zl_p[m][j].
+// Its epilogue keeps more state than contraction 1's, so its ring is one step shallower.
+constexpr int kRing2 = kLdgRing - 1;
+// A unit is a row group (P = KB2e / 2 pairs); the layer's B fragments serve every unit.
 // ---------------------------------------------------------------------------
-template <int MM, int NW>
-__global__ void __launch_bounds__(NW * 32, 1)
-    contraction2_pair_kernel(const LayerDev *__restrict__ layers, const PairUnit2 *__restrict__ units,
-                             const int *__restrict__ wrange, const __grid_constant__ IoPtrs io, int base, int M,
-                             int kb2max, int *err)
+template <int MM>
+static __device__ __noinline__ void c2_generic(const LayerDev *__restrict__ layers, const Seg2 *__restrict__ segs,
+                                                  int s0, int s1, const IoPtrs &io, int base, int M, int lane,
+                                                  uint64_t pol)
 {
-    constexpr int kStage = kPairStageKB * 256;
-    constexpr int kBStride = 16 * MM * 8;
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    __shared__ uint64_t rbar[NW][kPairStages];
-    __shared__ uint64_t bbar[NW][2];
-    __shared__ int snb[NW][kPairStages];       // k-blocks in each ring stage
-
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t4 = lane & 3;
     const int lane_m = t4 >> 1, lane_p = t4 & 1;
-    const int kBFrag = kb2max * kBStride, kBSlot = kBFrag + kPairMeta2;
-    unsigned char *ring = smem_raw + (size_t)warp * (kPairStages * kStage + 2 * kBSlot);
-    unsigned char *bslot = ring + kPairStages * kStage;
-    // after the warps' regions: zeros shaped like a B slot, read by the lanes past 16 * MM
-    uint4 *zbuf = reinterpret_cast<uint4 *>(smem_raw + (size_t)NW * (kPairStages * kStage + 2 * kBSlot));
-    if (MM == 1)
-        for (int i = threadIdx.x; i < kb2max * kBStride / 16; i += blockDim.x) zbuf[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (lane == 0) {
-        for (int s = 0; s < kPairStages; ++s) bar_init(&rbar[warp][s]);
-        bar_init(&bbar[warp][0]);
-        bar_init(&bbar[warp][1]);
+    const int blane = lane & (16 * MM - 1);
+    const bool store = lane_p == 0 && lane_m < M;
+
+    Prefetch<Seg2> pf;
+    pf.s = s0;
+    pf.live = true;
+    {
+        const Seg2 sg = segs[s0];
+        pf.seg(sg, lane, sg.P * 32);
     }
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    __syncthreads();
-    dep_release();
+    uint4 r0[kRing2], r1[kRing2];
+#pragma unroll
+    for (int d = 0; d < kRing2; ++d) fetch_step(pf, segs, s1, lane, pol, r0[d], r1[d]);
 
-    const int gw = warp * gridDim.x + blockIdx.x;     // an SM's warps take ranges spread over the whole batch
-    const int u0 = wrange[gw], u1 = wrange[gw + 1];
-    if (u0 >= u1) return;
-    const uint64_t pol = l2_evict_first();
-    // U tiles and h do not depend on the previous kernel; the zl fragments do: a layer's B
-    // slot wanted before dep_wait() is filled afterwards (at most one: the first layer)
-    bool dep_ok = false;
-    int pend_layer = -1;
-
-    // ---- fill cursor (position: unit f_u, k-block f_kb within it)
-    int f_u = u0, f_kb = 0, f_layer = -1, f_cs = -1, issued = 0, consumed = 0, c_cs = -1;
-    PairUnit2 f_cur = units[u0], f_nxt = f_cur;
-    if (u0 + 1 < u1) f_nxt = units[u0 + 1];
-    auto fill = [&]() {
-        while (f_u < u1 && issued - consumed < kPairStages) {
-            if (f_cur.layer != f_layer) {
-                if (f_cs >= c_cs + 1) return;           // both B slots still in use
-                ++f_cs;
-                f_layer = f_cur.layer;
-                if (!dep_ok) pend_layer = f_layer;
-                else if (lane == 0) {
-                    const LayerDev *fd = layers + f_layer;
-                    unsigned char *dst = bslot + (f_cs & 1) * kBSlot;
-                    uint64_t *bar = &bbar[warp][f_cs & 1];
-                    const unsigned fb = (unsigned)f_cur.kb2 * kBStride;
-                    asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(
-                                     sm_addr(bar)),
-                                 "r"(fb + (unsigned)kPairMeta2)
-                                 : "memory");
-                    bulk_copy(dst, fd->zfrag, fb, bar);
-                    bulk_copy(dst + kBFrag, fd->zmeta, (unsigned)kPairMeta2, bar);
-                }
-            }
-            const uint2 *src = f_cur.a + (size_t)f_kb * 32;
-            int n = 0;
-            while (true) {
-                const int t = min(kPairStageKB - n, f_cur.kb2 - f_kb);
-                n += t;
-                f_kb += t;
-                if (f_kb < f_cur.kb2) break;            // the stage is full inside this row group
-                f_kb = 0;
-                ++f_u;
-                f_cur = f_nxt;
-                if (f_u + 1 < u1) f_nxt = units[f_u + 1];
-                if (n == kPairStageKB || f_u >= u1 || f_cur.layer != f_layer) break;
-            }
-            const int st = issued % kPairStages;
-            snb[warp][st] = n;
-            if (lane == 0) {
-                expect_tx(&rbar[warp][st], (unsigned)n * 256u);
-                bulk_copy_hint(ring + st * kStage, src, (unsigned)n * 256u, &rbar[warp][st], pol);
-            }
-            ++issued;
-        }
-    };
-    fill();
-    dep_wait();
-    dep_ok = true;
-    if (pend_layer >= 0 && lane == 0) {
-        const LayerDev *fd = layers + pend_layer;
-        uint64_t *bar = &bbar[warp][0];
-        const unsigned fb = (unsigned)fd->KB2 * kBStride;
-        expect_tx(bar, fb + (unsigned)kPairMeta2);
-        bulk_copy(bslot, fd->zfrag, fb, bar);
-        bulk_copy(bslot + kBFrag, fd->zmeta, (unsigned)kPairMeta2, bar);
-    }
-
-    int c_layer = -1, N = 0, npaths = 1;
-    float *y = nullptr;
+    // consumer: segment cs, row group crg, step ct of the unit
+    int cs = s0, crg = 0, ct = 0, ch = 1, cP = 1, crem = 0, N = 0;
+    const uint4 *hq = nullptr, *zb = nullptr;
+    float *ym = nullptr;
     float my_sc = 0.0f, my_q = 0.0f;
-    uint32_t bbase = 0;
-    const uint32_t zaddr = sm_addr(zbuf) + (lane & 15) * 8;
-    int s_left = 0;             // k-blocks of the current stage not yet used
-    uint32_t s_addr = 0;        // this lane's word pair of the stage's next k-block
-
-    // h of this lane's path for rows g and g + 8 of each row block of a unit,
-    // read one unit ahead
-    int h_layer = -1;
-    const __half *h_base = nullptr;      // this lane's path row of h in layer h_layer, or null
-    auto load_h = [&](const PairUnit2 &un, __half (&hq)[8]) {
-        if (un.layer != h_layer) {
-            const LayerDev *dp = layers + un.layer;
-            h_layer = un.layer;
-            h_base = (lane_p < dp->npaths) ? dp->h + (size_t)lane_p * dp->N64 : nullptr;
-        }
-        const __half *hp = h_base + un.rg * kRowsPerGroup + g;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) hq[i] = h_base ? __ldg(hp + (i >> 1) * kRowsPerBlock + 8 * (i & 1)) : __half(0.0f);
+    auto seg_w = [&]() {        // the weights side of a segment: no dependency on the previous kernel
+        const Seg2 sg = segs[cs];
+        crg = sg.rg0;
+        crem = sg.n;
+        cP = sg.P;
+        ch = (cP + 1) >> 1;
+        hq = sg.hq + lane_p * 8 + g;
+        return sg.layer;
     };
-    PairUnit2 c_nxt = units[u0];
-    __half h_nxt[8];
-    load_h(c_nxt, h_nxt);
-    for (int u = u0; u < u1; ++u) {
-        const PairUnit2 cu = c_nxt;
-        float hv[4][2];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) hv[i >> 1][i & 1] = __half2float(h_nxt[i]);
-        if (u + 1 < u1) {
-            c_nxt = units[u + 1];
-            load_h(c_nxt, h_nxt);
+    auto seg_b = [&](int layer) {   // the activation side: zl fragments and exponents of the finish kernel
+        const LayerDev *dp = layers + layer;
+        zb = reinterpret_cast<const uint4 *>(dp->zfrag) + blane;
+        N = dp->N;
+        ym = io.y[layer - base] + (size_t)lane_m * N;
+        my_sc = my_q = 0.0f;
+        if (lane_m < M && lane_p < dp->npaths) {
+            const int2 mt = __ldcg(dp->zmeta + lane_p * 16 + lane_m);
+            if (mt.x == kNanExp) {
+                my_sc = my_q = __int_as_float(0x7fc00000);
+            } else {
+                my_sc = -2.0f * pow2f(-mt.x);                 // s = Q 2^-E - 2 T 2^-E
+                my_q = (float)mt.y * pow2f(-mt.x);
+            }
         }
-        if (cu.layer != c_layer) {
-            const LayerDev *dp = layers + cu.layer;
-            c_layer = cu.layer;
-            N = dp->N;
-            npaths = dp->npaths;
-            y = io.y[cu.layer - base];
-            ++c_cs;
-            fill();
-            if (!ring_wait(&bbar[warp][c_cs & 1], (c_cs >> 1) & 1, err)) return;
-            const unsigned char *slot = bslot + (c_cs & 1) * kBSlot;
-            my_sc = my_q = 0.0f;
-            if (lane_m < M && lane_p < npaths) {
-                const uint32_t ma = sm_addr(slot + kBFrag + 8 * (lane_p * 16 + lane_m));
-                const int ex = (int)lds_u32(ma), qsum = (int)lds_u32(ma + 4);
-                if (ex == kNanExp) {
-                    my_sc = my_q = __int_as_float(0x7fc00000);
+    };
+    const int layer0 = seg_w();
+    uint4 hn = __ldg(hq);                   // the current unit's row scales
+
+    dep_wait();     // the zl fragments and their exponents come from the finish kernel
+
+    seg_b(layer0);
+    auto bload = [&](int t, uint4 &b0, uint4 &b1) {       // B pairs of step t (stream 1 clamped: its A is zero)
+        b0 = ldg_frag(zb + (size_t)t * 16 * MM);
+        b1 = ldg_frag(zb + (size_t)min(ch + t, cP - 1) * 16 * MM);
+    };
+    uint4 bn0, bn1;
+    bload(0, bn0, bn1);
+    int a4[4][4];
+    zero_acc(a4);
+    bool live = true;
+    while (live) {
+#pragma unroll
+        for (int d = 0; d < kRing2; ++d) {
+            if (live) {
+                const uint4 w0 = r0[d], w1 = r1[d], b0 = bn0, b1 = bn1;
+                fetch_step(pf, segs, s1, lane, pol, r0[d], r1[d]);
+                const bool unit_end = ct + 1 == ch;
+                bload(unit_end ? 0 : ct + 1, bn0, bn1);     // the layer's fragments repeat for every unit
+                step_mma(a4, w0, w1, b0, b1);
+                if (unit_end) {
+                    // lane (m, path): its path's share of rows g and g + 8, then the pair sum
+                    const uint32_t hwv[4] = {hn.x, hn.y, hn.z, hn.w};
+                    const int n0 = crg * kRowsPerGroup + g;
+#pragma unroll
+                    for (int rb = 0; rb < 4; ++rb) {
+                        const float2 hv = __half22float2(*reinterpret_cast<const __half2 *>(&hwv[rb]));
+                        const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
+                        const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
+                        float vlo = hv.x * fmaf((float)Tlo, my_sc, my_q);
+                        float vhi = hv.y * fmaf((float)Thi, my_sc, my_q);
+                        vlo += __shfl_xor_sync(0xffffffffu, vlo, 1);
+                        vhi += __shfl_xor_sync(0xffffffffu, vhi, 1);
+                        const int nlo = n0 + rb * kRowsPerBlock;
+                        if (store) {
+                            if (nlo < N) ym[nlo] = vlo;
+                            if (nlo + 8 < N) ym[nlo + 8] = vhi;
+                        }
+                    }
+                    zero_acc(a4);
+                    ct = 0;
+                    if (--crem > 0) {
+                        ++crg;
+                        hq += 16;
+                        hn = __ldg(hq);
+                    } else if (++cs < s1) {
+                        seg_b(seg_w());
+                        hn = __ldg(hq);
+                        bload(0, bn0, bn1);
+                    } else {
+                        live = false;
+                    }
                 } else {
-                    my_sc = -2.0f * pow2f(-ex);                  // s = Q 2^-E - 2 T 2^-E
-                    my_q = (float)qsum * pow2f(-ex);
+                    ++ct;
                 }
             }
-            const bool real = lane < 16 * MM;
-            bbase = real ? sm_addr(slot) + lane * 8 : zaddr;
         }
-        const int n0 = cu.rg * kRowsPerGroup + g;
+    }
+}
 
-        int a4[4][4];
-#pragma unroll
-        for (int rb = 0; rb < 4; ++rb)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) a4[rb][c] = 0;
-        for (int kb = 0; kb < cu.kb2;) {
-            if (s_left == 0) {
-                const int st = consumed % kPairStages;
-                if (!ring_wait(&rbar[warp][st], (consumed / kPairStages) & 1, err)) return;
-                s_left = snb[warp][st];
-                s_addr = sm_addr(ring + st * kStage) + lane * 8;
-            }
-            const int seg = min(s_left, cu.kb2 - kb);
-            mma_stage<MM>(a4, s_addr, bbase + (uint32_t)kb * kBStride, seg);
-            kb += seg;
-            s_left -= seg;
-            s_addr += (uint32_t)seg * 256u;
-            if (s_left == 0) {
-                __syncwarp();
-                if (lane == 0) proxy_fence();
-                ++consumed;
-                fill();
-            }
-        }
+// ---------------------------------------------------------------------------
+// Static unit structure.  When every unit of a warp takes the same number H
+// of steps, the warp runs blocks of U units (L = U H steps, fully unrolled):
+// the ring holds one block, the prefetcher loads the next block at the same
+// positions, and every unit boundary, B index and epilogue sits at a
+// compile-time position, so the only branches are at block ends.  The last
+// block of a segment may hold fewer than U units: the rest read zeros and
+// store nothing.  The plan gives each warp units of one step count; counts
+// without a static path take the generic loops above.
+// ---------------------------------------------------------------------------
 
-        // lane (m, path): its path's share of rows g and g + 8, then the pair sum
+// 16 pairs of zeros: the weights of a unit past a segment's end or the warp's range (a unit has at most 16
+// pairs), so that each ring load is one address plus an immediate offset.
+static __device__ __align__(16) uint4 g_zero_unit[16 * 32];
+
+// A cursor over a warp's segments in blocks of U units, with this lane's address of each unit's first pair.
+template <typename Seg, int U>
+struct BlockCur {
+    int s, k;           // segment index, first unit of the block within it
+    bool live;
+    Seg sg;
+    const uint4 *ub[U];
+    __device__ __forceinline__ void bases(int lane)
+    {
 #pragma unroll
-        for (int rb = 0; rb < 4; ++rb) {
-            const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
-            const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
-            float vlo = hv[rb][0] * fmaf((float)Tlo, my_sc, my_q);
-            float vhi = hv[rb][1] * fmaf((float)Thi, my_sc, my_q);
-            vlo += __shfl_xor_sync(0xffffffffu, vlo, 1);
-            vhi += __shfl_xor_sync(0xffffffffu, vhi, 1);
-            const int nlo = n0 + rb * kRowsPerBlock;
-            if (lane_p == 0 && lane_m < M) {
-                if (nlo < N) y[(size_t)lane_m * N + nlo] = vlo;
-                if (nlo + 8 < N) y[(size_t)lane_m * N + nlo + 8] = vhi;
+        for (int j = 0; j < U; ++j)
+            ub[j] = (live && k + j < sg.n) ? seg_a(sg) + (size_t)(k + j) * seg_stride(sg) + lane : g_zero_unit + lane;
+    }
+    __device__ __forceinline__ void start(const Seg *segs, int s0, int lane)
+    {
+        s = s0;
+        k = 0;
+        live = true;
+        sg = segs[s0];
+        bases(lane);
+    }
+    // returns true when the block moved to another segment
+    __device__ __forceinline__ bool next(const Seg *segs, int s1, int lane)
+    {
+        k += U;
+        bool moved = false;
+        if (k >= sg.n) {
+            k = 0;
+            moved = true;
+            if (++s < s1) sg = segs[s];
+            else live = false;
+        }
+        bases(lane);
+        return moved;
+    }
+    static __device__ __forceinline__ const uint4 *seg_a(const Seg1 &x) { return x.v; }
+    static __device__ __forceinline__ const uint4 *seg_a(const Seg2 &x) { return x.u; }
+};
+
+// Step t of a unit whose first pair this lane reads at ub: pair t (stream 0) and H + t (stream 1).  Where a
+// unit has only 2H - 1 pairs, stream 1's last load reads the 512 bytes after the unit (the tile arrays are padded
+// by one pair); its B fragment is zero there, so nothing of it counts.
+template <int H>
+static __device__ __forceinline__ void fetch_unit_step(const uint4 *ub, int t, uint64_t pol, uint4 &w0, uint4 &w1)
+{
+    w0 = ldg_weights(ub + t * 32, pol);
+    w1 = ldg_weights(ub + (H + t) * 32, pol);
+}
+
+// The ring load at block position i: step i + D of the stream, in this block (cur) or the next one (nxt).
+template <int H, int U, int D, typename Seg>
+static __device__ __forceinline__ void fetch_ahead(const BlockCur<Seg, U> &cur, const BlockCur<Seg, U> &nxt, int i,
+                                                   uint64_t pol, uint4 &w0, uint4 &w1)
+{
+    constexpr int L = H * U;
+    const int j = i + D;
+    if (j < L) fetch_unit_step<H>(cur.ub[j / H], j % H, pol, w0, w1);
+    else fetch_unit_step<H>(nxt.ub[(j - L) / H], (j - L) % H, pol, w0, w1);
+}
+
+// B fragments of the static paths live in the warp's shared-memory slot: 2H pairs of 16 MM lanes, copied from
+// global memory (through L2: the previous kernel wrote them) whenever the warp enters a segment; where the units
+// have only 2H - 1 pairs, the last pair of the slot is zero, so stream 1's extra load counts for nothing.
+constexpr int kSlotPairs = 16;      // the largest 2H of a static path
+
+static __device__ __forceinline__ uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+static __device__ __forceinline__ void sts128(uint32_t addr, uint4 v)
+{
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+template <int MM>
+static __device__ __forceinline__ uint32_t b_slot(int warp)
+{
+    extern __shared__ __align__(16) unsigned char sm_raw[];
+    return sm_addr(sm_raw) + (uint32_t)warp * (kSlotPairs * 16 * MM * 16);
+}
+template <int MM, int H>
+static __device__ __forceinline__ void b_fill(uint32_t slot, const uint4 *src, int P, int lane)
+{
+    __syncwarp();      // every lane is done with the slot's previous contents
+#pragma unroll
+    for (int i = lane; i < 2 * H * 16 * MM; i += 32) {
+        const uint4 v = (i < P * 16 * MM) ? __ldcg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+        sts128(slot + (uint32_t)i * 16, v);
+    }
+    __syncwarp();
+}
+template <int MM, int H>
+static __device__ __forceinline__ void b_read(uint32_t bsl, int t, uint4 &b0, uint4 &b1)
+{
+    b0 = lds128(bsl + (uint32_t)t * 16 * MM * 16);
+    b1 = lds128(bsl + (uint32_t)(H + t) * 16 * MM * 16);
+}
+
+// Blocks of U units (L = U H steps, unrolled), a ring of D steps (D divides L): the ring slot of block position
+// i is i % D, refilled with step i + D once consumed.
+template <int MM, int H, int U, int D>
+static __device__ __noinline__ void c1_static(const LayerDev *__restrict__ layers, const Seg1 *__restrict__ segs,
+                                              int s0, int s1, int M, int lane, int warp, uint64_t pol)
+{
+    constexpr int L = H * U;
+    static_assert(L % D == 0 && D <= L, "ring");
+    const int g = lane >> 2, t4 = lane & 3;
+    const int lane_m = t4 >> 1, lane_p = t4 & 1;
+    const int blane = lane & (16 * MM - 1);
+
+    BlockCur<Seg1, U> cc, nb;       // the block being computed and the one after it
+    cc.start(segs, s0, lane);
+    nb = cc;
+    nb.next(segs, s1, lane);
+    uint4 r0[D], r1[D];
+#pragma unroll
+    for (int i = 0; i < D; ++i) fetch_unit_step<H>(cc.ub[i / H], i % H, pol, r0[i], r1[i]);
+
+    dep_wait();     // B fragments, exponents and cleared accumulators come from the previous kernels
+
+    const uint32_t slot = b_slot<MM>(warp), bsl = slot + blane * 16;
+    double *acc = nullptr;
+    int npaths = 1, r16 = 0;
+    double lsc = 0.0;
+    bool elive = false;
+    auto seg_in = [&]() {
+        const LayerDev *dp = layers + cc.sg.layer;
+        b_fill<MM, H>(slot, reinterpret_cast<const uint4 *>(dp->xfrag) + (size_t)cc.sg.kc * (kP1ChunkKB / 2) * 16 * MM,
+                      cc.sg.P, lane);
+        acc = dp->acc;
+        npaths = dp->npaths;
+        r16 = dp->r16;
+        const int E = (lane_m < M && lane_p < npaths) ? __ldcg(dp->xmeta + cc.sg.kc * 4 + 2 * lane_p + lane_m)
+                                                     : kNanExp;
+        elive = E != kNanExp;
+        lsc = elive ? pow2d(-E) : 0.0;
+    };
+    seg_in();
+    int a4[4][4];
+    zero_acc(a4);
+    while (cc.live) {
+#pragma unroll
+        for (int i = 0; i < L; ++i) {
+            const int k = i / H, t = i % H;
+            const uint4 w0 = r0[i % D], w1 = r1[i % D];
+            uint4 b0, b1;
+            b_read<MM, H>(bsl, t, b0, b1);
+            fetch_ahead<H, U, D>(cc, nb, i, pol, r0[i % D], r1[i % D]);
+            step_mma(a4, w0, w1, b0, b1);
+            if (t == H - 1) {
+                // unit k: keep the columns of each row block's own path; partial sums over chunks add up exactly
+                if (elive && cc.k + k < cc.sg.n) {
+                    const int rowg = (cc.sg.rg0 + cc.k + k) * kRowsPerGroup;
+#pragma unroll
+                    for (int rb = 0; rb < 4; ++rb) {
+                        const int row0 = rowg + rb * kRowsPerBlock;
+                        const int prb = (npaths > 1 && row0 >= r16) ? 1 : 0;     // path 1 owns rows r16..
+                        if (prb != lane_p) continue;
+                        const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
+                        const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
+                        if (Tlo) atomicAdd(acc + (size_t)(row0 + g) * MM + lane_m, (double)Tlo * lsc);
+                        if (Thi) atomicAdd(acc + (size_t)(row0 + g + 8) * MM + lane_m, (double)Thi * lsc);
+                    }
+                }
+                zero_acc(a4);
             }
         }
+        const bool moved = cc.next(segs, s1, lane);
+        nb.next(segs, s1, lane);
+        if (moved && cc.live) seg_in();
+    }
+}
+
+template <int MM, int H, int U, int D>
+static __device__ __noinline__ void c2_static(const LayerDev *__restrict__ layers, const Seg2 *__restrict__ segs,
+                                              int s0, int s1, const IoPtrs &io, int base, int M, int lane, int warp,
+                                              uint64_t pol)
+{
+    constexpr int L = H * U;
+    static_assert(L % D == 0 && D <= L, "ring");
+    const int g = lane >> 2, t4 = lane & 3;
+    const int lane_m = t4 >> 1, lane_p = t4 & 1;
+    const int blane = lane & (16 * MM - 1);
+    const bool store = lane_p == 0 && lane_m < M;
+
+    BlockCur<Seg2, U> cc, nb;
+    cc.start(segs, s0, lane);
+    nb = cc;
+    nb.next(segs, s1, lane);
+    uint4 r0[D], r1[D];
+#pragma unroll
+    for (int i = 0; i < D; ++i) fetch_unit_step<H>(cc.ub[i / H], i % H, pol, r0[i], r1[i]);
+
+    dep_wait();     // the zl fragments and their exponents come from the finish kernel
+
+    const uint32_t slot = b_slot<MM>(warp), bsl = slot + blane * 16;
+    int N = 0;
+    float *ym = nullptr;
+    float my_sc = 0.0f, my_q = 0.0f;
+    auto seg_in = [&]() {
+        const LayerDev *dp = layers + cc.sg.layer;
+        b_fill<MM, H>(slot, reinterpret_cast<const uint4 *>(dp->zfrag), cc.sg.P, lane);
+        N = dp->N;
+        ym = io.y[cc.sg.layer - base] + (size_t)lane_m * N;
+        my_sc = my_q = 0.0f;
+        if (lane_m < M && lane_p < dp->npaths) {
+            const int2 mt = __ldcg(dp->zmeta + lane_p * 16 + lane_m);
+            if (mt.x == kNanExp) {
+                my_sc = my_q = __int_as_float(0x7fc00000);
+            } else {
+                my_sc = -2.0f * pow2f(-mt.x);                 // s = Q 2^-E - 2 T 2^-E
+                my_q = (float)mt.y * pow2f(-mt.x);
+            }
+        }
+    };
+    seg_in();
+    uint4 hn = make_uint4(0u, 0u, 0u, 0u);
+    int a4[4][4];
+    zero_acc(a4);
+    while (cc.live) {
+#pragma unroll
+        for (int i = 0; i < L; ++i) {
+            const int k = i / H, t = i % H;
+            const uint4 w0 = r0[i % D], w1 = r1[i % D];
+            uint4 b0, b1;
+            b_read<MM, H>(bsl, t, b0, b1);
+            fetch_ahead<H, U, D>(cc, nb, i, pol, r0[i % D], r1[i % D]);
+            if (t == 0)     // the unit's row scales (a unit past the segment's end reads the block's first unit's)
+                hn = __ldg(cc.sg.hq + (size_t)(cc.k + (cc.k + k < cc.sg.n ? k : 0)) * 16 + lane_p * 8 + g);
+            step_mma(a4, w0, w1, b0, b1);
+            if (t == H - 1) {
+                // unit k, lane (m, path): its path's share of rows g and g + 8, then the pair sum
+                const bool st = store && cc.k + k < cc.sg.n;
+                const uint32_t hwv[4] = {hn.x, hn.y, hn.z, hn.w};
+                const int n0 = (cc.sg.rg0 + cc.k + k) * kRowsPerGroup + g;
+#pragma unroll
+                for (int rb = 0; rb < 4; ++rb) {
+                    const float2 hv = __half22float2(*reinterpret_cast<const __half2 *>(&hwv[rb]));
+                    const int Tlo = (a4[rb][0] >> rb) + 256 * (a4[rb][1] >> rb);
+                    const int Thi = (a4[rb][2] >> (rb + 4)) + 256 * (a4[rb][3] >> (rb + 4));
+                    float vlo = hv.x * fmaf((float)Tlo, my_sc, my_q);
+                    float vhi = hv.y * fmaf((float)Thi, my_sc, my_q);
+                    vlo += __shfl_xor_sync(0xffffffffu, vlo, 1);
+                    vhi += __shfl_xor_sync(0xffffffffu, vhi, 1);
+                    const int nlo = n0 + rb * kRowsPerBlock;
+                    if (st && nlo < N) ym[nlo] = vlo;
+                    if (st && nlo + 8 < N) ym[nlo + 8] = vhi;
+                }
+                zero_acc(a4);
+            }
+        }
+        const bool moved = cc.next(segs, s1, lane);
+        nb.next(segs, s1, lane);
+        if (moved && cc.live) seg_in();
+    }
+}
+
+// Per warp: its units' step count (a static path) or 0 (the generic loop).
+template <int MM>
+__global__ void __launch_bounds__(kLdgWarps * 32, 1)
+    contraction1_ldg_kernel(const LayerDev *__restrict__ layers, const Seg1 *__restrict__ segs,
+                            const int *__restrict__ bnd, const int *__restrict__ cls, int M)
+{
+    dep_release();
+    const int lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * kLdgWarps + (threadIdx.x >> 5);
+    const int s0 = bnd[gw], s1 = bnd[gw + 1];
+    if (s0 >= s1) return;
+    const uint64_t pol = l2_evict_first();
+    switch (cls[gw]) {
+    case 8: c1_static<MM, 8, 1, 4>(layers, segs, s0, s1, M, lane, threadIdx.x >> 5, pol); break;
+    default: c1_generic<MM>(layers, segs, s0, s1, M, lane, pol); break;
+    }
+}
+
+template <int MM>
+__global__ void __launch_bounds__(kLdgWarps * 32, 1)
+    contraction2_ldg_kernel(const LayerDev *__restrict__ layers, const Seg2 *__restrict__ segs,
+                            const int *__restrict__ bnd, const int *__restrict__ cls, const __grid_constant__ IoPtrs io,
+                            int base, int M)
+{
+    dep_release();
+    const int lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * kLdgWarps + (threadIdx.x >> 5);
+    const int s0 = bnd[gw], s1 = bnd[gw + 1];
+    if (s0 >= s1) return;
+    const uint64_t pol = l2_evict_first();
+    switch (cls[gw]) {
+    case 1: c2_static<MM, 1, 6, 6>(layers, segs, s0, s1, io, base, M, lane, threadIdx.x >> 5, pol); break;
+    case 2: c2_static<MM, 2, 3, 6>(layers, segs, s0, s1, io, base, M, lane, threadIdx.x >> 5, pol); break;
+    case 3: c2_static<MM, 3, 2, 6>(layers, segs, s0, s1, io, base, M, lane, threadIdx.x >> 5, pol); break;
+    case 4: c2_static<MM, 4, 3, 6>(layers, segs, s0, s1, io, base, M, lane, threadIdx.x >> 5, pol); break;
+    case 5: c2_static<MM, 5, 1, 5>(layers, segs, s0, s1, io, base, M, lane, threadIdx.x >> 5, pol); break;
+    case 6: c2_static<MM, 6, 1, 6>(layers, segs, s0, s1, io, base, M, lane, threadIdx.x >> 5, pol); break;
+    default: c2_generic<MM>(layers, segs, s0, s1, io, base, M, lane, pol); break;
     }
 }
 
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-static int g_pair_smem1[2];          // dynamic shared memory attribute set so far, per MM
 
 // Launch that may overlap the previous kernel of the stream (programmatic stream
 // serialisation; the kernel waits with dep_wait() before using its results).
@@ -688,43 +929,21 @@ static cudaError_t launch_dependent(bool pdl, void (*kernel)(P...), dim3 grid, d
     cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
 }
-static int g_pair_smem2[2][5];       // per MM and contraction-2 warp count (16, 12, 8, 6, 4)
 
-template <int MM, int NW>
-static cudaError_t launch_c2(bool pdl, int grid, size_t smem, cudaStream_t s, int slot, const LayerDev *dev_layers,
-                             const PairUnit2 *u2, const int *wr2, const IoPtrs &io, int base, int M, int kb2max, int *err)
-{
-    cudaError_t e;
-    if ((int)smem > g_pair_smem2[MM - 1][slot]) {
-        if ((e = cudaFuncSetAttribute(contraction2_pair_kernel<MM, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)smem)) != cudaSuccess)
-            return e;
-        g_pair_smem2[MM - 1][slot] = (int)smem;
-    }
-    return launch_dependent(pdl, contraction2_pair_kernel<MM, NW>, dim3(grid), dim3(NW * 32), smem, s, dev_layers, u2,
-                            wr2, io, base, M, kb2max, err);
-}
+static int g_ldg_smem[2];           // dynamic shared-memory limit raised so far, per MM
 
 template <int MM>
-static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1,
-                                const PairUnit1 *u1, const int *wr1, const PairUnit2 *u2, const int *wr2,
-                                int pair_warps, int pair_warps2, const IoPtrs &io, int base, int M, int kb2max, int rmax,
-                                int *err, cudaStream_t s, int *launches, bool mark)
+static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1, const Plan &P,
+                                int batch, const IoPtrs &io, int base, int M, int kb2max, int rmax, cudaStream_t s,
+                                int *launches, bool mark)
 {
     cudaError_t e;
-    constexpr int kPairWarps = pair_warps_per_cta(MM);
-    const int nw2 = pair2_warps_per_cta(MM, kb2max);
-    const size_t smem1 = (size_t)kPairWarps * kPairStages * (kPairStageKB * (256 + 16 * MM * 8) + 16);
-    const size_t smem2 = pair2_cta_smem(MM, kb2max, nw2);
-    if (smem1 > 227 * 1024 || smem2 > 227 * 1024 || kb2max > kPairMaxKB2 || pair_warps2 % nw2 != 0 ||
-        (size_t)2 * rmax * MM * sizeof(float) > 48 * 1024)
-        return LB_ERR_UNSUPPORTED;
-    if ((int)smem1 > g_pair_smem1[MM - 1]) {
-        if ((e = cudaFuncSetAttribute(contraction1_pair_kernel<MM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)smem1)) != cudaSuccess)
-            return status_from(e);
-        g_pair_smem1[MM - 1] = (int)smem1;
-    }
+    const int G = P.stream_grid;
+    if (G < 1 || kb2max > kPairMaxKB2 || (size_t)2 * rmax * MM * sizeof(float) > 48 * 1024) return LB_ERR_UNSUPPORTED;
+    const int nw = G * kLdgWarps;
+    const int *bnd1 = P.bnd1 + (size_t)batch * (nw + 1);
+    const int *bnd2 = P.bnd2 + (size_t)batch * (nw + 1);
+    const int *cls1 = P.cls1 + (size_t)batch * nw, *cls2 = P.cls2 + (size_t)batch * nw;
     if (n1 > 0) {
         quantize_pair_kernel<MM><<<(n1 + kQuantWarps - 1) / kQuantWarps, kQuantWarps * 32, 0, s>>>(dev_layers, p1, n1, io,
                                                                                                   base, M);
@@ -734,8 +953,17 @@ static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P
     // the three kernels after the quantisation may each start while the previous one drains,
     // unless timing events separate the launches
     const bool pdl = !profiling_active();
-    if ((e = launch_dependent(pdl, contraction1_pair_kernel<MM>, dim3(pair_warps / kPairWarps), dim3(kPairWarps * 32),
-                              smem1, s, dev_layers, u1, wr1, M, err)) != cudaSuccess)
+    const size_t slots = (size_t)kLdgWarps * kSlotPairs * 16 * MM * 16;    // one B slot per warp
+    if ((int)slots > g_ldg_smem[MM - 1]) {
+        if ((e = cudaFuncSetAttribute(contraction1_ldg_kernel<MM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)slots)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(contraction2_ldg_kernel<MM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)slots)) != cudaSuccess)
+            return status_from(e);
+        g_ldg_smem[MM - 1] = (int)slots;
+    }
+    if ((e = launch_dependent(pdl, contraction1_ldg_kernel<MM>, dim3(G), dim3(kLdgWarps * 32), slots, s, dev_layers,
+                              (const Seg1 *)P.sg1, bnd1, cls1, M)) != cudaSuccess)
         return status_from(e);
     ++*launches;
     if (mark) profile_mark(*launches, s);
@@ -744,30 +972,22 @@ static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P
         return status_from(e);
     ++*launches;
     if (mark) profile_mark(*launches, s);
-    const int grid2 = pair_warps2 / nw2;
-    switch (nw2) {
-    case 16: e = launch_c2<MM, 16>(pdl, grid2, smem2, s, 0, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
-    case 12: e = launch_c2<MM, 12>(pdl, grid2, smem2, s, 1, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
-    case 8: e = launch_c2<MM, 8>(pdl, grid2, smem2, s, 2, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
-    case 6: e = launch_c2<MM, 6>(pdl, grid2, smem2, s, 3, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
-    default: e = launch_c2<MM, 4>(pdl, grid2, smem2, s, 4, dev_layers, u2, wr2, io, base, M, kb2max, err); break;
-    }
-    if (e != cudaSuccess) return status_from(e);
+    if ((e = launch_dependent(pdl, contraction2_ldg_kernel<MM>, dim3(G), dim3(kLdgWarps * 32), slots, s, dev_layers,
+                              (const Seg2 *)P.sg2, bnd2, cls2, io, base, M)) != cudaSuccess)
+        return status_from(e);
     ++*launches;
     if (mark) profile_mark(*launches, s);
     return status_from(cudaGetLastError());
 }
 
-lb_status decode_pair_launch(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1, const PairUnit1 *u1,
-                             const int *wr1, const PairUnit2 *u2, const int *wr2, int pair_warps, int pair_warps2,
-                             const IoPtrs &io, int base, int M, int kb2max, int rmax, int *err, cudaStream_t s,
-                             int *launches, bool mark)
+lb_status decode_pair_launch(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1, const Plan &P,
+                             int batch, const IoPtrs &io, int base, int M, int kb2max, int rmax, int *err,
+                             cudaStream_t s, int *launches, bool mark)
 {
+    (void)err;     // these kernels wait on nothing but their predecessors' completion
     if (M == 1)
-        return pair_launch_mm<1>(dev_layers, nlayers, p1, n1, u1, wr1, u2, wr2, pair_warps, pair_warps2, io, base, M,
-                                 kb2max, rmax, err, s, launches, mark);
-    return pair_launch_mm<2>(dev_layers, nlayers, p1, n1, u1, wr1, u2, wr2, pair_warps, pair_warps2, io, base, M,
-                             kb2max, rmax, err, s, launches, mark);
+        return pair_launch_mm<1>(dev_layers, nlayers, p1, n1, P, batch, io, base, M, kb2max, rmax, s, launches, mark);
+    return pair_launch_mm<2>(dev_layers, nlayers, p1, n1, P, batch, io, base, M, kb2max, rmax, s, launches, mark);
 }
 
 }  // namespace lb

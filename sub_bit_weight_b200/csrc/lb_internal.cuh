@@ -19,10 +19,15 @@ namespace lb {
 // the activations are the B operand as two balanced base-256 digits of a
 // 16-bit fixed-point value (column = 2*m + digit).
 //
-// A "unit" is 64 rows x 32 k of one weight matrix, stored as 256 contiguous
-// bytes: lane L (g = L >> 2, t = L & 3) owns the uint2 {w0, w1}.  Bit i of
-// byte b of word q is the sign bit (1 = -1) of
+// A "k-block" is 64 rows x 32 k of one weight matrix, 256 bytes: lane L
+// (g = L >> 2, t = L & 3) owns the uint2 {w0, w1}.  Bit i of byte b of word q
+// is the sign bit (1 = -1) of
 //     row = 16 * (i & 3) + g + 8 * (i >> 2),   k = 4 * t + b + 16 * q.
+// The k-blocks of a 64-row group are stored in pairs: k-blocks 2j and 2j + 1
+// take 512 contiguous bytes in which lane L owns the 16 bytes at 16 L (its
+// uint2 of k-block 2j, then its uint2 of k-block 2j + 1), so one 16-byte load
+// per lane fetches two k-blocks.  A row group's k-block count is rounded up to
+// even (KB1e, KB2e); the padding k-block has no bit set and adds nothing.
 // Masking a word with (0x01010101 << i) gives four u8 A elements equal to
 // 2^i times the bit, in exactly the register slots mma.sync expects, so a
 // row-block's MMA costs four LOP3s and no shifts:
@@ -44,36 +49,15 @@ constexpr int kP1StageKB = 8;           // k-blocks per ring stage, contraction 
 constexpr int kP1Stages = 3;            // per-warp bulk-copy ring depth, contraction 1
 constexpr int kP2Stages = 2;            // per-warp bulk-copy ring depth, contraction 2 (one row group per stage)
 
-// Warp-streaming kernels for one or two activation rows.  Every warp owns an
-// equal contiguous share of the bytes a contraction streams (fixed at plan
-// build for one CTA per SM), so no work is handed out at run
-// time and no warp waits for another.
-// contraction-1 warps per CTA (independent of each other), one CTA per SM: 16
-// for one row, 12 for two rows (their larger B fragments)
-__host__ __device__ constexpr int pair_warps_per_cta(int MM) { return MM == 1 ? 16 : 12; }
-constexpr int kPairStages = 2;          // ring stages per warp
-constexpr int kPairStageKB = 16;        // k-blocks per ring stage (4 KB)
+// Streaming kernels for one or two activation rows (M <= 2): one CTA of
+// kLdgWarps warps per SM, every warp streaming its own contiguous range of
+// row-group units straight into registers (a ring of kLdgRing pairs of
+// k-blocks per stream, two streams per warp: the two halves of each unit's
+// k-range).  The ranges are built with the plan, cost-balanced over all warps.
+constexpr int kLdgWarps = 16;           // warps per CTA (one CTA per SM)
+constexpr int kLdgRing = 6;             // k-block pairs in flight per stream
 constexpr int kPairMaxKB2 = 64;         // largest contraction-2 depth (k-blocks) these kernels take (r = 1024, 2 paths)
-// Shared memory of the contraction-2 kernel (per warp; per CTA with the zero
-// buffer of one-row batches), and its warps per CTA: the most of
-// {16, 12, 8, 6, 4} whose CTA fits in 227 KB.
-__host__ __device__ constexpr int pair2_smem_per_warp(int MM, int kb2max)
-{
-    return kPairStages * kPairStageKB * 256 + 2 * (kb2max * 16 * MM * 8 + 144);
-}
-__host__ __device__ constexpr int pair2_cta_smem(int MM, int kb2max, int nw)
-{
-    return nw * pair2_smem_per_warp(MM, kb2max) + (MM == 1 ? kb2max * 128 : 0);
-}
-__host__ __device__ constexpr int pair2_warps_per_cta(int MM, int kb2max)
-{
-    return (pair2_cta_smem(MM, kb2max, 16) <= 227 * 1024)   ? 16
-           : (pair2_cta_smem(MM, kb2max, 12) <= 227 * 1024) ? 12
-           : (pair2_cta_smem(MM, kb2max, 8) <= 227 * 1024)  ? 8
-           : (pair2_cta_smem(MM, kb2max, 6) <= 227 * 1024)  ? 6
-                                                             : 4;
-}
-constexpr int kPairMeta2 = 144;         // bytes of zmeta copied with a contraction-2 B slot (p * 16 + m, m < 2)
+constexpr int kPairMeta2 = 144;         // bytes of zmeta a contraction-2 stage carries (p * 16 + m, m < 2)
 
 // doubles in the accumulator block of a layer's scratch
 __host__ __device__ inline size_t acc_doubles(int R1) { return (size_t)R1 * 16 + 32 + 16; }
@@ -90,18 +74,22 @@ struct LayerDev {
     int N64, RG2;       // outputs rounded to 64, contraction-2 row groups
     int KB2;            // contraction-2 k-blocks (npaths * r32 / 32)
     int nkc;            // contraction-1 work items (k chunks)
-    const uint2 *vt;    // V tiles  [RG1][KB1][32]
-    const uint2 *ut;    // U tiles  [RG2][KB2][32]
+    int KB1e, KB2e;     // KB1, KB2 rounded up to even (k-blocks are stored in pairs)
+    const uint2 *vt;    // V tiles  [RG1][KB1e / 2 pairs][32 lanes][2]
+    const uint2 *ut;    // U tiles  [RG2][KB2e / 2 pairs][32 lanes][2]
     const __half *g;    // [npaths][K32], zero padded
     const __half *h;    // [npaths][N64], zero padded
     const __half *l;    // [npaths][r16], zero padded
+    const uint4 *hq;    // [RG2][2][8][4][2] binary16: h of path p, rows 16 rb + g + 8 hf of each row
+                        //   group, ordered so that lane (g, p) of a warp reads its eight with one 16-byte load
     // scratch (owned by the plan that holds this descriptor):
     //   acc:  [R1][16] double  sum over k of b * t (contraction-1 rows x activation rows; the
     //                           one/two-row kernels use the first R1 * M doubles as [R1][M])
     //         [2][16]  double  sum over k of t (per path x activation row)
     //         [2][16]  int     non-finite flags (per path x activation row)
-    //   zfrag [kMaxNT][KB2][32] B fragments of contraction 2, zmeta [2][16] (exponent, digit sum)
-    //   xfrag [KB1][32] B fragments of contraction 1 (one or two rows: 16 * M lanes per k-block)
+    //   zfrag [kMaxNT][KB2][32] B fragments of contraction 2 (one or two rows: [KB2e / 2][16 * M][2],
+    //         pairs of k-blocks as in the tiles), zmeta [2][16] (exponent, digit sum)
+    //   xfrag [KB1e / 2][16 * M][2] B fragments of contraction 1 (one or two rows, pairs of k-blocks)
     //   xmeta [nkc][2][2] exponent of each (k chunk, path, row)
     double *acc;
     uint2 *zfrag;
@@ -113,10 +101,14 @@ struct LayerDev {
 struct P1Item { int layer, kc; };
 struct P2Item { int layer, rg0, rg1, pad; };
 
-// Streaming units of the one/two-row kernels.  Contraction 1: row group rg of
-// k chunk kc (nkb k-blocks at a); contraction 2: row group rg (KB2 k-blocks at a).
-struct PairUnit1 { const uint2 *a; int layer, kc, rg, nkb; };
-struct PairUnit2 { const uint2 *a; int layer, rg, kb2, pad; };
+// Segments of the one/two-row streaming kernels (32 bytes each): n
+// consecutive units of one layer in a warp's range, each P pairs of k-blocks.
+// Contraction 1: row groups rg0 .. rg0 + n - 1 of one 1024-input chunk kc
+// (v: the tiles of (rg0, kc); consecutive row groups are rstride uint4
+// apart); contraction 2: row groups rg0 .. rg0 + n - 1 (u: the tiles of rg0;
+// consecutive row groups are contiguous; hq: the row scales of rg0).
+struct Seg1 { const uint4 *v; int layer, kc, rg0, n, P, rstride; };
+struct Seg2 { const uint4 *u; const uint4 *hq; int layer, rg0, n, P; };
 
 struct IoPtrs {
     const uint16_t *x[kIoBatch];
@@ -153,12 +145,13 @@ struct Plan {
     P1Item *p1 = nullptr;           // device work items
     P2Item *p2 = nullptr;
     std::vector<int> p1_start, p2_start;   // per IO batch: first item index
-    PairUnit1 *u1 = nullptr;        // one/two-row streaming units, all batches
-    PairUnit2 *u2 = nullptr;
-    // per row count MM (index MM - 1) and batch: pair_warps[MM - 1] + 1 unit boundaries (absolute)
-    int *wr1[2] = {nullptr, nullptr}, *wr2[2] = {nullptr, nullptr};
-    int pair_warps[2] = {0, 0};     // contraction-1 warps the streaming units are partitioned over, per MM
-    int pair_warps2[2] = {0, 0};    // the same for contraction 2
+    // one/two-row streaming segments, all batches; per batch #SM * kLdgWarps + 1 segment boundaries
+    // (absolute indices into the segment arrays), warp w of the launch taking [bnd[w], bnd[w + 1])
+    Seg1 *sg1 = nullptr;
+    Seg2 *sg2 = nullptr;
+    int *bnd1 = nullptr, *bnd2 = nullptr;
+    int *cls1 = nullptr, *cls2 = nullptr;   // per batch and warp: the step count of its units (0: mixed counts)
+    int stream_grid = 0;            // CTAs of the streaming launches (the SM count)
     int kb2max = 0;                 // largest KB2 of the plan
     int rmax = 0;                   // largest rank of the plan
     int *err = nullptr;             // device error code (bounded waits that gave up)
@@ -173,10 +166,9 @@ void plan_free(Plan &P);
 lb_status decode_forward(const Plan &P, const uint16_t *const *xs, float *const *ys, int M,
                          cudaStream_t s, int *launches);
 
-lb_status decode_pair_launch(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1, const PairUnit1 *u1,
-                             const int *wr1, const PairUnit2 *u2, const int *wr2, int pair_warps, int pair_warps2,
-                             const IoPtrs &io, int base, int M, int kb2max, int rmax, int *err, cudaStream_t s,
-                             int *launches, bool mark);
+lb_status decode_pair_launch(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1, const Plan &P,
+                             int batch, const IoPtrs &io, int base, int M, int kb2max, int rmax, int *err,
+                             cudaStream_t s, int *launches, bool mark);
 lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc, const struct Plan &P,
                             const uint16_t *x, float *y, int M, int *err, cudaStream_t s, int *launches);
 

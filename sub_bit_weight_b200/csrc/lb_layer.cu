@@ -7,6 +7,7 @@
 // the scales zero-padded, so padded rank slots and rows contribute nothing.
 
 #include <algorithm>
+#include <array>
 #include <cstring>
 #include <new>
 
@@ -21,18 +22,18 @@ __device__ __forceinline__ uint32_t canon_bit(const uint32_t *P, int wpr, int64_
 
 // Contraction-1 tiles: rows are latent indices of both paths (path p owns
 // rows [p*r16, p*r16 + r16)), k runs over the K inputs.  Bit = V_sign[k][j] < 0.
-__global__ void build_vtiles_kernel(uint2 *__restrict__ vt, int RG1, int KB1, int r, int r16, int K,
+__global__ void build_vtiles_kernel(uint2 *__restrict__ vt, int RG1, int KB1e, int r, int r16, int K,
                                     int npaths, const uint32_t *__restrict__ V0,
                                     const uint32_t *__restrict__ V1)
 {
     const int wpr = (r + 31) / 32;
-    const int64_t total = (int64_t)RG1 * KB1 * 32;
+    const int64_t total = (int64_t)RG1 * KB1e * 32;
     for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
          idx += (int64_t)gridDim.x * blockDim.x) {
         const int lane = (int)(idx & 31);
         const int64_t u = idx >> 5;
-        const int kb = (int)(u % KB1);
-        const int rg = (int)(u / KB1);
+        const int kb = (int)(u % KB1e);
+        const int rg = (int)(u / KB1e);
         const int g = lane >> 2, t = lane & 3;
         uint32_t w[2] = {0u, 0u};
 #pragma unroll
@@ -48,24 +49,25 @@ __global__ void build_vtiles_kernel(uint2 *__restrict__ vt, int RG1, int KB1, in
                     if (p < npaths && j < r && k < K)
                         w[q] |= canon_bit(p ? V1 : V0, wpr, k, j) << (8 * b + i);
                 }
-        vt[idx] = make_uint2(w[0], w[1]);
+        // pairs of k-blocks: lane L's uint2 of k-blocks 2j and 2j + 1 side by side
+        vt[(((int64_t)rg * (KB1e >> 1) + (kb >> 1)) * 32 + lane) * 2 + (kb & 1)] = make_uint2(w[0], w[1]);
     }
 }
 
 // Contraction-2 tiles: rows are the N outputs, k runs over the latent indices
 // of both paths (path p owns k in [p*r32, p*r32 + r32)).  Bit = U_sign[n][j] < 0.
-__global__ void build_utiles_kernel(uint2 *__restrict__ ut, int RG2, int KB2, int r, int r32, int N,
+__global__ void build_utiles_kernel(uint2 *__restrict__ ut, int RG2, int KB2e, int r, int r32, int N,
                                     int npaths, const uint32_t *__restrict__ U0,
                                     const uint32_t *__restrict__ U1)
 {
     const int wpr = (r + 31) / 32;
-    const int64_t total = (int64_t)RG2 * KB2 * 32;
+    const int64_t total = (int64_t)RG2 * KB2e * 32;
     for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
          idx += (int64_t)gridDim.x * blockDim.x) {
         const int lane = (int)(idx & 31);
         const int64_t u = idx >> 5;
-        const int kb = (int)(u % KB2);
-        const int rg = (int)(u / KB2);
+        const int kb = (int)(u % KB2e);
+        const int rg = (int)(u / KB2e);
         const int g = lane >> 2, t = lane & 3;
         uint32_t w[2] = {0u, 0u};
 #pragma unroll
@@ -81,7 +83,7 @@ __global__ void build_utiles_kernel(uint2 *__restrict__ ut, int RG2, int KB2, in
                     if (p < npaths && j < r && n < N)
                         w[q] |= canon_bit(p ? U1 : U0, wpr, n, j) << (8 * b + i);
                 }
-        ut[idx] = make_uint2(w[0], w[1]);
+        ut[(((int64_t)rg * (KB2e >> 1) + (kb >> 1)) * 32 + lane) * 2 + (kb & 1)] = make_uint2(w[0], w[1]);
     }
 }
 
@@ -95,6 +97,23 @@ __global__ void pad_copy_kernel(uint16_t *__restrict__ dst, const uint16_t *__re
         const int p = (int)(idx / npad);
         const int i = (int)(idx - (int64_t)p * npad);
         dst[idx] = (i < n) ? (p ? s1 : s0)[i] : (uint16_t)0;
+    }
+}
+
+// Row scales of contraction 2 in fragment order: for row group rg, path p and
+// lane row g, the eight values h_p[64 rg + 16 rb + g + 8 hf] (rb < 4, hf < 2)
+// are contiguous, [rg][p][g][rb][hf]; zero for an absent path or row >= N.
+__global__ void build_hq_kernel(uint16_t *__restrict__ hq, int RG2, int N, int npaths,
+                                const uint16_t *__restrict__ h0, const uint16_t *__restrict__ h1)
+{
+    const int64_t total = (int64_t)RG2 * 128;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int w = (int)(idx & 127);
+        const int rg = (int)(idx >> 7);
+        const int p = w >> 6, g = (w >> 3) & 7, rb = (w >> 1) & 3, hf = w & 1;
+        const int row = rg * kRowsPerGroup + 16 * rb + g + 8 * hf;
+        hq[idx] = (p < npaths && row < N) ? (p ? h1 : h0)[row] : (uint16_t)0;
     }
 }
 
@@ -114,12 +133,12 @@ void plan_free(Plan &P)
     if (P.dev) cudaFree(P.dev);
     if (P.p1) cudaFree(P.p1);
     if (P.p2) cudaFree(P.p2);
-    if (P.u1) cudaFree(P.u1);
-    if (P.u2) cudaFree(P.u2);
-    for (int mm = 0; mm < 2; ++mm) {
-        if (P.wr1[mm]) cudaFree(P.wr1[mm]);
-        if (P.wr2[mm]) cudaFree(P.wr2[mm]);
-    }
+    if (P.sg1) cudaFree(P.sg1);
+    if (P.sg2) cudaFree(P.sg2);
+    if (P.bnd1) cudaFree(P.bnd1);
+    if (P.bnd2) cudaFree(P.bnd2);
+    if (P.cls1) cudaFree(P.cls1);
+    if (P.cls2) cudaFree(P.cls2);
     if (P.scratch) cudaFree(P.scratch);
     P = Plan();
 }
@@ -139,7 +158,7 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
         total += align256((size_t)kMaxNT * d.KB2 * 32 * sizeof(uint2));
         total += align256((size_t)2 * 16 * sizeof(int2));
         total += align256(sizeof(unsigned));
-        total += align256((size_t)d.KB1 * 32 * sizeof(uint2));
+        total += align256((size_t)d.KB1e * 32 * sizeof(uint2));
         total += align256((size_t)d.nkc * 4 * sizeof(int));
     }
     total += 256;   // error code
@@ -155,7 +174,7 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
         d.acc = (double *)c;       c += align256(acc_doubles(d.R1) * sizeof(double));
         d.zfrag = (uint2 *)c;      c += align256((size_t)kMaxNT * d.KB2 * 32 * sizeof(uint2));
         d.zmeta = (int2 *)c;       c += align256((size_t)2 * 16 * sizeof(int2));
-        d.xfrag = (uint2 *)c;      c += align256((size_t)d.KB1 * 32 * sizeof(uint2));
+        d.xfrag = (uint2 *)c;      c += align256((size_t)d.KB1e * 32 * sizeof(uint2));
         d.xmeta = (int *)c;
         P.host[i] = d;
     }
@@ -191,9 +210,12 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
     P.n_p1 = (int)p1.size();
     P.n_p2 = (int)p2.size();
 
-    // One/two-row streaming units in layer order, and per batch an equal split
-    // of their estimated cost over pair_warps warps (warp w streams units
-    // [wr[w], wr[w + 1]) of its batch).
+    // Segments of the one/two-row streaming kernels, per IO batch.  A unit takes H = ceil(P / 2) steps (P pairs
+    // of k-blocks, two per step); the kernels have unrolled paths for some H (the static classes) and a generic
+    // loop for the rest.  The batch's units are grouped by class (layer order within a class), every class gets
+    // a share of the #SM * kLdgWarps warps in proportion to its estimated cost, and each class's units are split
+    // into contiguous ranges of equal cost, one per warp, cut into segments (runs of one layer; in contraction 1
+    // of one chunk).  Range r goes to warp r / #SM of CTA r % #SM, so each SM holds ranges of every class.
     int sms = 148, dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
@@ -203,65 +225,156 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
         P.kb2max = std::max(P.kb2max, P.host[i].KB2);
         P.rmax = std::max(P.rmax, P.host[i].r);
     }
-    std::vector<PairUnit1> u1;
-    std::vector<PairUnit2> u2;
-    std::vector<int> wr1[2], wr2[2];
+    P.stream_grid = sms;
+    const int nwarps = sms * kLdgWarps;
+    std::vector<Seg1> sg1;
+    std::vector<Seg2> sg2;
+    std::vector<int> bnd1, bnd2, cls1, cls2;
     const int nb = (int)P.p1_start.size() - 1;
-    // contraction 1: cost in issued instructions per warp (MMA k-blocks, ring stages, per-unit epilogue)
-    auto stages = [](int nkb) { return (double)((nkb + kPairStageKB - 1) / kPairStageKB); };
-    auto cost1 = [&](const PairUnit1 &u) { return 22.0 * u.nkb + 40.0 * stages(u.nkb) + 60.0; };
-    // contraction 2, in k-block equivalents (fitted to per-warp times on B200): a k-block, 8.5 per row group
-    // (fold, h, stores), 15 where a layer starts (its zl fragments are waited for)
-    auto cost2 = [&](const PairUnit2 &u) { return (double)u.kb2 + 8.5 + (u.rg == 0 ? 15.0 : 0.0); };
+    // a unit: layer, linear index within the layer, pairs, cost (k-blocks plus the epilogue; the generic loop
+    // runs slower per k-block)
+    struct Unit { int layer, ul, P; double cost; };
+    auto class1 = [](int pairs) { const int H = (pairs + 1) / 2; return H == 8 ? H : 0; };
+    auto class2 = [](int pairs) { const int H = (pairs + 1) / 2; return (H >= 1 && H <= 6) ? H : 0; };
+    // a unit's k-blocks plus its epilogue and block bookkeeping, in k-block equivalents (fitted to per-warp times
+    // on B200); the generic loop runs about a third slower
+    auto unit_cost = [](int pairs, int cls) { return (2.0 * pairs + 16.0) * (cls ? 1.0 : 1.35); };
+    // ranges[r] = (class, first unit, end unit) over `order` (unit indices grouped by class)
+    auto partition = [&](const std::vector<Unit> &us, auto class_of, std::vector<int> &order,
+                         std::vector<std::array<int, 3>> &ranges) {
+        std::vector<int> classes;
+        for (const Unit &x : us) {
+            const int c = class_of(x.P);
+            if (std::find(classes.begin(), classes.end(), c) == classes.end()) classes.push_back(c);
+        }
+        std::sort(classes.begin(), classes.end());
+        std::vector<double> cost(classes.size(), 0.0);
+        order.clear();
+        std::vector<size_t> cstart;
+        for (size_t ci = 0; ci < classes.size(); ++ci) {
+            cstart.push_back(order.size());
+            for (size_t u = 0; u < us.size(); ++u)
+                if (class_of(us[u].P) == classes[ci]) {
+                    order.push_back((int)u);
+                    cost[ci] += us[u].cost;
+                }
+        }
+        cstart.push_back(order.size());
+        double total = 0.0;
+        for (double c : cost) total += c;
+        // warps per class: at least one each, the rest by largest remainder
+        std::vector<int> nw(classes.size(), 1);
+        int left = nwarps - (int)classes.size();
+        std::vector<double> want(classes.size());
+        for (size_t ci = 0; ci < classes.size(); ++ci) want[ci] = total > 0 ? cost[ci] / total * left : 0.0;
+        for (size_t ci = 0; ci < classes.size(); ++ci) {
+            nw[ci] += (int)want[ci];
+            left -= (int)want[ci];
+        }
+        while (left > 0) {
+            size_t best = 0;
+            for (size_t ci = 1; ci < classes.size(); ++ci)
+                if (want[ci] - (int)want[ci] > want[best] - (int)want[best]) best = ci;
+            ++nw[best];
+            want[best] = (int)want[best];     // its remainder is used up
+            --left;
+        }
+        ranges.clear();
+        for (size_t ci = 0; ci < classes.size(); ++ci) {
+            const size_t a0 = cstart[ci], a1 = cstart[ci + 1];
+            size_t u = a0;
+            double acc = 0.0;
+            for (int w = 0; w < nw[ci]; ++w) {
+                const double target = cost[ci] * (w + 1) / nw[ci];
+                const size_t first = u;
+                while (u < a1 && (w + 1 == nw[ci] || acc + 0.5 * us[order[u]].cost < target)) acc += us[order[u++]].cost;
+                ranges.push_back({classes[ci], (int)first, (int)u});
+            }
+        }
+    };
     for (int b = 0; b < nb; ++b) {
         const int l0 = b * kIoBatch, l1 = std::min(n, l0 + kIoBatch);
-        const size_t s1 = u1.size(), s2 = u2.size();
+        std::vector<Unit> us1, us2;
         for (int i = l0; i < l1; ++i) {
             const LayerDev &d = P.host[i];
             for (int kc = 0; kc < d.nkc; ++kc) {
-                const int nkb = std::min(kP1ChunkKB, d.KB1 - kc * kP1ChunkKB);
+                const int pairs = (std::min(kP1ChunkKB, d.KB1 - kc * kP1ChunkKB) + 1) / 2;
                 for (int rg = 0; rg < d.RG1; ++rg)
-                    u1.push_back({d.vt + ((size_t)rg * d.KB1 + (size_t)kc * kP1ChunkKB) * 32, i, kc, rg, nkb});
+                    us1.push_back({i, kc * d.RG1 + rg, pairs, unit_cost(pairs, class1(pairs))});
             }
-            for (int rg = 0; rg < d.RG2; ++rg) u2.push_back({d.ut + (size_t)rg * d.KB2 * 32, i, rg, d.KB2, 0});
+            for (int rg = 0; rg < d.RG2; ++rg) us2.push_back({i, rg, d.KB2e / 2, unit_cost(d.KB2e / 2, class2(d.KB2e / 2))});
         }
-        // per row count: an equal split of the estimated cost over all warps of one CTA per SM
-        for (int mm = 0; mm < 2; ++mm) {
-            const int W1 = sms * pair_warps_per_cta(mm + 1);
-            const int W2 = sms * pair2_warps_per_cta(mm + 1, std::min(P.kb2max, kPairMaxKB2));
-            P.pair_warps[mm] = W1;
-            P.pair_warps2[mm] = W2;
-            auto split = [&](std::vector<int> &wr, size_t first, size_t last, int W, auto cost_of) {
-                double total_c = 0.0;
-                for (size_t u = first; u < last; ++u) total_c += cost_of(u);
-                size_t u = first;
-                double acc = 0.0;
-                for (int w = 0; w <= W; ++w) {
-                    const double target = total_c * w / W;
-                    while (u < last && acc + 0.5 * cost_of(u) < target) acc += cost_of(u++);
-                    wr.push_back((int)(w == W ? last : u));
-                }
-            };
-            split(wr1[mm], s1, u1.size(), W1, [&](size_t u) { return cost1(u1[u]); });
-            split(wr2[mm], s2, u2.size(), W2, [&](size_t u) { return cost2(u2[u]); });
+        std::vector<int> o1, o2;
+        std::vector<std::array<int, 3>> r1, r2;
+        partition(us1, class1, o1, r1);
+        partition(us2, class2, o2, r2);
+        const size_t first1 = bnd1.size(), first2 = bnd2.size();
+        bnd1.resize(first1 + nwarps + 1);
+        bnd2.resize(first2 + nwarps + 1);
+        const size_t fc1 = cls1.size(), fc2 = cls2.size();
+        cls1.resize(fc1 + nwarps, 0);
+        cls2.resize(fc2 + nwarps, 0);
+        std::vector<std::vector<Seg1>> per1(nwarps);
+        std::vector<std::vector<Seg2>> per2(nwarps);
+        for (int r = 0; r < nwarps; ++r) {
+            const int w = (r % sms) * kLdgWarps + r / sms;
+            cls1[fc1 + w] = r1[r][0];
+            for (int a = r1[r][1]; a < r1[r][2];) {
+                // units of one layer and one chunk: ul = kc * RG1 + rg (consecutive in `order` within a class)
+                const Unit &f = us1[o1[a]];
+                const LayerDev &d = P.host[f.layer];
+                const int kc = f.ul / d.RG1, rg0 = f.ul - kc * d.RG1;
+                int e2 = a + 1;
+                while (e2 < r1[r][2] && us1[o1[e2]].layer == f.layer && us1[o1[e2]].ul == f.ul + (e2 - a) &&
+                       us1[o1[e2]].ul / d.RG1 == kc)
+                    ++e2;
+                per1[w].push_back({reinterpret_cast<const uint4 *>(d.vt) +
+                                       ((size_t)rg0 * (d.KB1e / 2) + (size_t)kc * (kP1ChunkKB / 2)) * 32,
+                                   f.layer, kc, rg0, e2 - a, f.P, d.KB1e / 2 * 32});
+                a = e2;
+            }
+            cls2[fc2 + w] = r2[r][0];
+            for (int a = r2[r][1]; a < r2[r][2];) {
+                const Unit &f = us2[o2[a]];
+                const LayerDev &d = P.host[f.layer];
+                int e2 = a + 1;
+                while (e2 < r2[r][2] && us2[o2[e2]].layer == f.layer && us2[o2[e2]].ul == f.ul + (e2 - a)) ++e2;
+                per2[w].push_back({reinterpret_cast<const uint4 *>(d.ut) + (size_t)f.ul * (d.KB2e / 2) * 32,
+                                   d.hq + (size_t)f.ul * 16, f.layer, f.ul, e2 - a, d.KB2e / 2});
+                a = e2;
+            }
         }
+        for (int w = 0; w < nwarps; ++w) {
+            bnd1[first1 + w] = (int)sg1.size();
+            sg1.insert(sg1.end(), per1[w].begin(), per1[w].end());
+            bnd2[first2 + w] = (int)sg2.size();
+            sg2.insert(sg2.end(), per2[w].begin(), per2[w].end());
+        }
+        bnd1[first1 + nwarps] = (int)sg1.size();
+        bnd2[first2 + nwarps] = (int)sg2.size();
     }
-    if ((e = cudaMalloc(&P.u1, sizeof(PairUnit1) * std::max<size_t>(1, u1.size()))) != cudaSuccess) return e;
-    if ((e = cudaMalloc(&P.u2, sizeof(PairUnit2) * std::max<size_t>(1, u2.size()))) != cudaSuccess) return e;
-    if (!u1.empty() && (e = cudaMemcpy(P.u1, u1.data(), sizeof(PairUnit1) * u1.size(), cudaMemcpyHostToDevice)) != cudaSuccess)
+    if ((e = cudaMalloc(&P.sg1, sizeof(Seg1) * std::max<size_t>(1, sg1.size()))) != cudaSuccess) return e;
+    if ((e = cudaMalloc(&P.sg2, sizeof(Seg2) * std::max<size_t>(1, sg2.size()))) != cudaSuccess) return e;
+    if ((e = cudaMalloc(&P.bnd1, sizeof(int) * bnd1.size())) != cudaSuccess) return e;
+    if ((e = cudaMalloc(&P.bnd2, sizeof(int) * bnd2.size())) != cudaSuccess) return e;
+    if ((e = cudaMalloc(&P.cls1, sizeof(int) * std::max<size_t>(1, cls1.size()))) != cudaSuccess) return e;
+    if ((e = cudaMalloc(&P.cls2, sizeof(int) * std::max<size_t>(1, cls2.size()))) != cudaSuccess) return e;
+    if (!sg1.empty() && (e = cudaMemcpy(P.sg1, sg1.data(), sizeof(Seg1) * sg1.size(), cudaMemcpyHostToDevice)) !=
+                            cudaSuccess)
         return e;
-    if (!u2.empty() && (e = cudaMemcpy(P.u2, u2.data(), sizeof(PairUnit2) * u2.size(), cudaMemcpyHostToDevice)) != cudaSuccess)
+    if (!sg2.empty() && (e = cudaMemcpy(P.sg2, sg2.data(), sizeof(Seg2) * sg2.size(), cudaMemcpyHostToDevice)) !=
+                            cudaSuccess)
         return e;
-    for (int mm = 0; mm < 2; ++mm) {
-        if ((e = cudaMalloc(&P.wr1[mm], sizeof(int) * std::max<size_t>(1, wr1[mm].size()))) != cudaSuccess) return e;
-        if ((e = cudaMalloc(&P.wr2[mm], sizeof(int) * std::max<size_t>(1, wr2[mm].size()))) != cudaSuccess) return e;
-        if ((e = cudaMemcpy(P.wr1[mm], wr1[mm].data(), sizeof(int) * wr1[mm].size(), cudaMemcpyHostToDevice)) !=
-            cudaSuccess)
-            return e;
-        if ((e = cudaMemcpy(P.wr2[mm], wr2[mm].data(), sizeof(int) * wr2[mm].size(), cudaMemcpyHostToDevice)) !=
-            cudaSuccess)
-            return e;
-    }
+    if ((e = cudaMemcpy(P.bnd1, bnd1.data(), sizeof(int) * bnd1.size(), cudaMemcpyHostToDevice)) != cudaSuccess)
+        return e;
+    if ((e = cudaMemcpy(P.bnd2, bnd2.data(), sizeof(int) * bnd2.size(), cudaMemcpyHostToDevice)) != cudaSuccess)
+        return e;
+    if (!cls1.empty() && (e = cudaMemcpy(P.cls1, cls1.data(), sizeof(int) * cls1.size(), cudaMemcpyHostToDevice)) !=
+                             cudaSuccess)
+        return e;
+    if (!cls2.empty() && (e = cudaMemcpy(P.cls2, cls2.data(), sizeof(int) * cls2.size(), cudaMemcpyHostToDevice)) !=
+                             cudaSuccess)
+        return e;
 
     if ((e = cudaMalloc(&P.dev, sizeof(LayerDev) * n)) != cudaSuccess) return e;
     if ((e = cudaMalloc(&P.p1, sizeof(P1Item) * std::max(1, P.n_p1))) != cudaSuccess) return e;
@@ -323,14 +436,19 @@ lb_status lb_layer_create(lb_layer **out, int N, int K, int r, int npaths, const
     d.RG2 = d.N64 / kRowsPerGroup;
     d.KB2 = npaths * d.r32 / kKPerBlock;
     d.nkc = ceil_div(d.KB1, kP1ChunkKB);
+    d.KB1e = round_up(d.KB1, 2);
+    d.KB2e = round_up(d.KB2, 2);
 
-    const size_t b_vt = align256((size_t)d.RG1 * d.KB1 * 32 * sizeof(uint2));
-    const size_t b_ut = align256((size_t)d.RG2 * d.KB2 * 32 * sizeof(uint2));
+    // one pair of k-blocks (512 bytes) of padding after each tile array: the streaming kernels may read the pair
+    // after a unit whose pair count is odd (with a zero B fragment)
+    const size_t b_vt = align256((size_t)d.RG1 * d.KB1e * 32 * sizeof(uint2) + 512);
+    const size_t b_ut = align256((size_t)d.RG2 * d.KB2e * 32 * sizeof(uint2) + 512);
     const size_t b_g = align256((size_t)npaths * d.K32 * 2);
     const size_t b_h = align256((size_t)npaths * d.N64 * 2);
     const size_t b_l = align256((size_t)npaths * d.r16 * 2);
+    const size_t b_hq = align256((size_t)d.RG2 * 256);
     const size_t b_pf = prefill_weight_bytes(d);
-    L->weight_bytes = b_vt + b_ut + b_g + b_h + b_l + b_pf;
+    L->weight_bytes = b_vt + b_ut + b_g + b_h + b_l + b_hq + b_pf;
     cudaError_t e = cudaMalloc(&L->weights, L->weight_bytes);
     if (e != cudaSuccess) {
         delete L;
@@ -342,23 +460,26 @@ lb_status lb_layer_create(lb_layer **out, int N, int K, int r, int npaths, const
     d.g = (const __half *)c;   c += b_g;
     d.h = (const __half *)c;   c += b_h;
     d.l = (const __half *)c;   c += b_l;
+    d.hq = (const uint4 *)c;   c += b_hq;
     L->pf.b1 = (uint32_t *)c;  // prefill layouts are carved from here
 
     const int T = 256;
     const uint32_t *V1 = npaths > 1 ? V[1] : V[0];
     const uint32_t *U1 = npaths > 1 ? U[1] : U[0];
     int launches = 0;
-    build_vtiles_kernel<<<grid_for((int64_t)d.RG1 * d.KB1 * 32, T), T, 0, s>>>(
-        (uint2 *)d.vt, d.RG1, d.KB1, r, d.r16, K, npaths, V[0], V1);
-    build_utiles_kernel<<<grid_for((int64_t)d.RG2 * d.KB2 * 32, T), T, 0, s>>>(
-        (uint2 *)d.ut, d.RG2, d.KB2, r, d.r32, N, npaths, U[0], U1);
+    build_vtiles_kernel<<<grid_for((int64_t)d.RG1 * d.KB1e * 32, T), T, 0, s>>>(
+        (uint2 *)d.vt, d.RG1, d.KB1e, r, d.r16, K, npaths, V[0], V1);
+    build_utiles_kernel<<<grid_for((int64_t)d.RG2 * d.KB2e * 32, T), T, 0, s>>>(
+        (uint2 *)d.ut, d.RG2, d.KB2e, r, d.r32, N, npaths, U[0], U1);
     pad_copy_kernel<<<grid_for((int64_t)npaths * d.K32, T), T, 0, s>>>(
         (uint16_t *)d.g, g[0], npaths > 1 ? g[1] : g[0], npaths, K, d.K32);
     pad_copy_kernel<<<grid_for((int64_t)npaths * d.N64, T), T, 0, s>>>(
         (uint16_t *)d.h, h[0], npaths > 1 ? h[1] : h[0], npaths, N, d.N64);
     pad_copy_kernel<<<grid_for((int64_t)npaths * d.r16, T), T, 0, s>>>(
         (uint16_t *)d.l, l[0], npaths > 1 ? l[1] : l[0], npaths, r, d.r16);
-    launches = 5;
+    build_hq_kernel<<<grid_for((int64_t)d.RG2 * 128, T), T, 0, s>>>((uint16_t *)d.hq, d.RG2, N, npaths, h[0],
+                                                                     npaths > 1 ? h[1] : h[0]);
+    launches = 6;
     e = cudaGetLastError();
     if (e == cudaSuccess) {
         e = prefill_build_weights(L->pf, d, U, V, h, g, l, s);

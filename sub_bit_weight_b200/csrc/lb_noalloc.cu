@@ -17,7 +17,6 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[LB_NOALLOC_SCRA
 
 // Offsets inside the array.
 constexpr size_t kOffDesc = 0;        // LayerDev (the kernels read descriptors from device memory)
-constexpr size_t kOffErr = 256;       // int error code
 constexpr size_t kOffMeta = 768;      // int2 [2][16]
 constexpr size_t kOffAcc = 1024;      // double accumulators, then the fragments
 
@@ -55,7 +54,7 @@ extern "C" lb_status lb_linear_forward_noalloc(const uint16_t *x, int M, const l
     const size_t acc_n = acc_doubles(src.R1);
     const size_t off_frag = kOffAcc + al256(acc_n * sizeof(double));
     const size_t off_xfrag = off_frag + al256((size_t)kMaxNT * src.KB2 * 32 * sizeof(uint2));
-    const size_t off_xmeta = off_xfrag + al256((size_t)src.KB1 * 32 * sizeof(uint2));
+    const size_t off_xmeta = off_xfrag + al256((size_t)src.KB1e * 32 * sizeof(uint2));
     const size_t need = off_xmeta + (size_t)src.nkc * 4 * sizeof(int);
     if (need > LB_NOALLOC_SCRATCH_BYTES) return LB_ERR_UNSUPPORTED;
 
@@ -85,8 +84,10 @@ extern "C" lb_status lb_linear_forward_noalloc(const uint16_t *x, int M, const l
     if ((e = cudaGetLastError()) != cudaSuccess) return status_from(e);
     const Plan &P = L->self->plan;   // the layer's own work items (read only)
     int launches = 1;
-    lb_status st = decode_launch_one(reinterpret_cast<const LayerDev *>(base + kOffDesc), d, P, x, y, M,
-                                     reinterpret_cast<int *>(base + kOffErr), s, &launches);
+    // a bounded wait that gives up reports to the layer's own error slot (allocated with the layer),
+    // which lb_layer_status reads and clears
+    lb_status st = decode_launch_one(reinterpret_cast<const LayerDev *>(base + kOffDesc), d, P, x, y, M, P.err, s,
+                                     &launches);
     set_launch_count(launches);
     return st;
 }

@@ -130,6 +130,13 @@ lb_status lb_selftest_wait_timeout(long long cycles, void *stream)
     return read_and_clear(lb::g_selftest_err, s);
 }
 
+lb_status lb_layer_selftest_wait_timeout(const lb_layer *L, long long cycles, void *stream)
+{
+    if (!L || cycles < 0) return LB_ERR_INVALID_ARG;
+    lb::wait_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(L->self->plan.err, cycles);
+    return lb::status_from(cudaGetLastError());
+}
+
 lb_status lb_profile_events(void *const *events, int n)
 {
     if (n < 0 || n > LB_MAX_PROFILE_EVENTS) return LB_ERR_INVALID_ARG;

@@ -57,6 +57,7 @@ _sig("lb_profile_events", _st, [ctypes.POINTER(_vp), _i])
 _sig("lb_stack_status", _st, [_vp, _vp])
 _sig("lb_layer_status", _st, [_vp, _vp])
 _sig("lb_selftest_wait_timeout", _st, [ctypes.c_longlong, _vp])
+_sig("lb_layer_selftest_wait_timeout", _st, [_vp, ctypes.c_longlong, _vp])
 _sig("lb_dual_svid_workspace_bytes", ctypes.c_size_t, [_i, _i, _i])
 _sig("lb_backward_create", _st, [ctypes.POINTER(_vp), _i, _i, _i, _i] + [ctypes.POINTER(_vp)] * 5 + [_vp])
 _sig("lb_backward_destroy", None, [_vp])
@@ -112,6 +113,11 @@ def lb_stack_status(stack, stream=None) -> int:
 
 def lb_selftest_wait_timeout(cycles: int, stream=None) -> int:
     return int(_lib.lb_selftest_wait_timeout(int(cycles), _stream(stream)))
+
+
+def lb_layer_selftest_wait_timeout(layer, cycles: int, stream=None) -> int:
+    """Run the bounded-wait self-test against the layer's error slot (no synchronisation)."""
+    return int(_lib.lb_layer_selftest_wait_timeout(layer.handle, int(cycles), _stream(stream)))
 
 
 def lb_packed_words(rows: int, r: int) -> int:

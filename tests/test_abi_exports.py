@@ -75,6 +75,8 @@ def test_host_side_argument_checks(lib):
     lib.lb_layer_bpw.restype = ctypes.c_double
     lib.lb_layer_bpw.argtypes = [vp]
     assert lib.lb_layer_bpw(None) == 0.0
+    lib.lb_layer_selftest_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
+    assert lib.lb_layer_selftest_wait_timeout(None, 10, None) == 1
     lib.lb_layer_destroy.argtypes = [vp]
     lib.lb_layer_destroy(None)
     lib.lb_stack_destroy.argtypes = [vp]

@@ -88,7 +88,7 @@ def test_dram_traffic_is_reported_only_for_the_sources_it_was_captured_with(tmp_
         assert all(os.path.exists(os.path.join(bench.CSRC, f)) for f in bench.KERNEL_SOURCES[kernel])
     prof = tmp_path / "profiles"
     prof.mkdir()
-    k = "contraction2_pair_kernel"
+    k = "contraction2_ldg_kernel"
     good = bench.source_hash(k)
     (prof / "traffic.txt").write_text("# kernel workload source_sha16 dram_bytes_per_launch note\n"
                                       f"{k} wl_a {good} 123456 x\n"
