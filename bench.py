@@ -432,6 +432,11 @@ def main():
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.gpus != world:
+        # one process per GPU: N > 1 ranks come from the launcher, never from this flag alone
+        sys.stderr.write(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; run N ranks as "
+                         f"python -m torch.distributed.run --nproc-per-node N bench.py --gpus N\n")
+        sys.exit(2)
     w = synth.WORKLOADS[args.workload]
     M = args.M if args.M is not None else w.Ms[0]
     pk = peaks()

@@ -304,13 +304,8 @@ __global__ void __launch_bounds__(kCT, 1)
 
 int sm_count_c()
 {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
+    int n = 0;
+    if (sm_count_of_current(&n) != cudaSuccess || n <= 0) n = 148;
     return n;
 }
 
@@ -320,11 +315,9 @@ cudaError_t chol_inverse(double *S, int n, long ldS, double *Lf, double *Linv, l
                          int *err, cudaStream_t s)
 {
     if (n < 1) return cudaErrorInvalidValue;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCholSmem);
+    {
+        const cudaError_t e = ensure_dyn_smem((const void *)chol_inv_kernel, kCholSmem);
         if (e != cudaSuccess) return e;
-        attr = true;
     }
     const int npan = (n + kB - 1) / kB;
     const int tiles = std::max(1, npan - 1);

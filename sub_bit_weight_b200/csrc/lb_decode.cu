@@ -540,19 +540,6 @@ static void kernels_for(K1Fn &k1, KFFn &kf, K2Fn &k2)
     k2 = contraction2_kernel<NT>;
 }
 
-static int g_sms = 0;
-static int g_smem_set1[kMaxNT + 1] = {0}, g_smem_set2[kMaxNT + 1] = {0};
-
-// Raise a kernel's dynamic shared-memory limit to at least `bytes`, never lower it:
-// every launch path of that kernel shares the cached value.
-static cudaError_t ensure_smem(const void *fn, size_t bytes, int &cached)
-{
-    if ((int)bytes <= cached) return cudaSuccess;
-    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e == cudaSuccess) cached = (int)bytes;
-    return e;
-}
-
 lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const *ys, int M, cudaStream_t s,
                          int *launches)
 {
@@ -573,12 +560,8 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
     }
     const int NT = (M + 3) / 4;
     cudaError_t e = cudaSuccess;
-    if (!g_sms) {
-        int dev = 0;
-        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return status_from(e);
-        if ((e = cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-            return status_from(e);
-    }
+    int sms = 0;
+    if ((e = sm_count_of_current(&sms)) != cudaSuccess) return status_from(e);
     K1Fn k1;
     KFFn kf;
     K2Fn k2;
@@ -595,8 +578,8 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
     const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * ((kb2max + 1) & ~1) * 256 +
                          (size_t)NT * kb2max * 32 * sizeof(uint2);
     if (smem2 > 227 * 1024) return LB_ERR_UNSUPPORTED;
-    if ((e = ensure_smem((const void *)k1, smem1, g_smem_set1[NT])) != cudaSuccess) return status_from(e);
-    if ((e = ensure_smem((const void *)k2, smem2, g_smem_set2[NT])) != cudaSuccess) return status_from(e);
+    if ((e = ensure_dyn_smem((const void *)k1, smem1)) != cudaSuccess) return status_from(e);
+    if ((e = ensure_dyn_smem((const void *)k2, smem2)) != cudaSuccess) return status_from(e);
     int occ1 = 0, occ2 = 0;
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, k1, kDecodeThreads, smem1)) != cudaSuccess)
         return status_from(e);
@@ -624,8 +607,8 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
             if (st != LB_ERR_UNSUPPORTED) return st;
             // shapes the streaming kernels cannot hold in shared memory take the general kernels
         }
-        const int grid1 = std::max(1, std::min(n1, g_sms * occ1));
-        const int grid2 = std::max(1, std::min(n2, g_sms * occ2));
+        const int grid1 = std::max(1, std::min(n1, sms * occ1));
+        const int grid2 = std::max(1, std::min(n2, sms * occ2));
         k1<<<grid1, kDecodeThreads, smem1, s>>>(P.dev, P.p1 + P.p1_start[b], n1, io, base, M, P.err);
         profile_mark(++*launches, s);
         kf<<<cnt, kFinishGeneralThreads, 0, s>>>(P.dev, base, M);
@@ -657,9 +640,8 @@ lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc,
     }
     const int NT = (M + 3) / 4;
     cudaError_t e = cudaSuccess;
-    int sms = 0, dev = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return status_from(e);
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return status_from(e);
+    int sms = 0;
+    if ((e = sm_count_of_current(&sms)) != cudaSuccess) return status_from(e);
     K1Fn k1;
     KFFn kf;
     K2Fn k2;
@@ -675,8 +657,8 @@ lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc,
     const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * ((kb2max + 1) & ~1) * 256 +
                          (size_t)NT * kb2max * 32 * sizeof(uint2);
     if (smem2 > 227 * 1024) return LB_ERR_UNSUPPORTED;
-    if ((e = ensure_smem((const void *)k1, smem1, g_smem_set1[NT])) != cudaSuccess) return status_from(e);
-    if ((e = ensure_smem((const void *)k2, smem2, g_smem_set2[NT])) != cudaSuccess) return status_from(e);
+    if ((e = ensure_dyn_smem((const void *)k1, smem1)) != cudaSuccess) return status_from(e);
+    if ((e = ensure_dyn_smem((const void *)k2, smem2)) != cudaSuccess) return status_from(e);
     int occ1 = 0, occ2 = 0;
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, k1, kDecodeThreads, smem1)) != cudaSuccess)
         return status_from(e);

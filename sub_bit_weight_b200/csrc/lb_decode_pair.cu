@@ -607,24 +607,34 @@ static __device__ __noinline__ void c2_generic(const LayerDev *__restrict__ laye
 static __device__ __align__(16) uint4 g_zero_unit[16 * 32];
 
 // A cursor over a warp's segments in blocks of U units, with this lane's address of each unit's first pair.
+static __device__ __forceinline__ const uint4 *seg_a(const Seg1 &x) { return x.v; }
+static __device__ __forceinline__ const uint4 *seg_a(const Seg2 &x) { return x.u; }
+
 template <typename Seg, int U>
 struct BlockCur {
-    int s, k;           // segment index, first unit of the block within it
+    int s, k, n, stride;    // segment index, first unit of the block, units in the segment, uint4 between units
     bool live;
-    Seg sg;
+    const uint4 *base;      // this lane's address of the segment's first unit's first pair
     const uint4 *ub[U];
+    __device__ __forceinline__ void seg_load(const Seg *segs, int lane)
+    {
+        const Seg sg = segs[s];
+        base = seg_a(sg) + lane;
+        n = sg.n;
+        stride = seg_stride(sg);
+    }
     __device__ __forceinline__ void bases(int lane)
     {
 #pragma unroll
         for (int j = 0; j < U; ++j)
-            ub[j] = (live && k + j < sg.n) ? seg_a(sg) + (size_t)(k + j) * seg_stride(sg) + lane : g_zero_unit + lane;
+            ub[j] = (live && k + j < n) ? base + (size_t)(k + j) * stride : g_zero_unit + lane;
     }
     __device__ __forceinline__ void start(const Seg *segs, int s0, int lane)
     {
         s = s0;
         k = 0;
         live = true;
-        sg = segs[s0];
+        seg_load(segs, lane);
         bases(lane);
     }
     // returns true when the block moved to another segment
@@ -632,17 +642,15 @@ struct BlockCur {
     {
         k += U;
         bool moved = false;
-        if (k >= sg.n) {
+        if (k >= n) {
             k = 0;
             moved = true;
-            if (++s < s1) sg = segs[s];
+            if (++s < s1) seg_load(segs, lane);
             else live = false;
         }
         bases(lane);
         return moved;
     }
-    static __device__ __forceinline__ const uint4 *seg_a(const Seg1 &x) { return x.v; }
-    static __device__ __forceinline__ const uint4 *seg_a(const Seg2 &x) { return x.u; }
 };
 
 // Step t of a unit whose first pair this lane reads at ub: pair t (stream 0) and H + t (stream 1).  Where a
@@ -734,14 +742,17 @@ static __device__ __noinline__ void c1_static(const LayerDev *__restrict__ layer
     int npaths = 1, r16 = 0;
     double lsc = 0.0;
     bool elive = false;
+    int rg0 = 0;
     auto seg_in = [&]() {
-        const LayerDev *dp = layers + cc.sg.layer;
-        b_fill<MM, H>(slot, reinterpret_cast<const uint4 *>(dp->xfrag) + (size_t)cc.sg.kc * (kP1ChunkKB / 2) * 16 * MM,
-                      cc.sg.P, lane);
+        const Seg1 sg = segs[cc.s];
+        const LayerDev *dp = layers + sg.layer;
+        b_fill<MM, H>(slot, reinterpret_cast<const uint4 *>(dp->xfrag) + (size_t)sg.kc * (kP1ChunkKB / 2) * 16 * MM,
+                      sg.P, lane);
+        rg0 = sg.rg0;
         acc = dp->acc;
         npaths = dp->npaths;
         r16 = dp->r16;
-        const int E = (lane_m < M && lane_p < npaths) ? __ldcg(dp->xmeta + cc.sg.kc * 4 + 2 * lane_p + lane_m)
+        const int E = (lane_m < M && lane_p < npaths) ? __ldcg(dp->xmeta + sg.kc * 4 + 2 * lane_p + lane_m)
                                                      : kNanExp;
         elive = E != kNanExp;
         lsc = elive ? pow2d(-E) : 0.0;
@@ -760,8 +771,8 @@ static __device__ __noinline__ void c1_static(const LayerDev *__restrict__ layer
             step_mma(a4, w0, w1, b0, b1);
             if (t == H - 1) {
                 // unit k: keep the columns of each row block's own path; partial sums over chunks add up exactly
-                if (elive && cc.k + k < cc.sg.n) {
-                    const int rowg = (cc.sg.rg0 + cc.k + k) * kRowsPerGroup;
+                if (elive && cc.k + k < cc.n) {
+                    const int rowg = (rg0 + cc.k + k) * kRowsPerGroup;
 #pragma unroll
                     for (int rb = 0; rb < 4; ++rb) {
                         const int row0 = rowg + rb * kRowsPerBlock;
@@ -808,11 +819,16 @@ static __device__ __noinline__ void c2_static(const LayerDev *__restrict__ layer
     int N = 0;
     float *ym = nullptr;
     float my_sc = 0.0f, my_q = 0.0f;
+    int rg0 = 0;
+    const uint4 *hq = nullptr;
     auto seg_in = [&]() {
-        const LayerDev *dp = layers + cc.sg.layer;
-        b_fill<MM, H>(slot, reinterpret_cast<const uint4 *>(dp->zfrag), cc.sg.P, lane);
+        const Seg2 sg = segs[cc.s];
+        const LayerDev *dp = layers + sg.layer;
+        b_fill<MM, H>(slot, reinterpret_cast<const uint4 *>(dp->zfrag), sg.P, lane);
+        rg0 = sg.rg0;
+        hq = sg.hq + lane_p * 8 + g;
         N = dp->N;
-        ym = io.y[cc.sg.layer - base] + (size_t)lane_m * N;
+        ym = io.y[sg.layer - base] + (size_t)lane_m * N;
         my_sc = my_q = 0.0f;
         if (lane_m < M && lane_p < dp->npaths) {
             const int2 mt = __ldcg(dp->zmeta + lane_p * 16 + lane_m);
@@ -837,13 +853,13 @@ static __device__ __noinline__ void c2_static(const LayerDev *__restrict__ layer
             b_read<MM, H>(bsl, t, b0, b1);
             fetch_ahead<H, U, D>(cc, nb, i, pol, r0[i % D], r1[i % D]);
             if (t == 0)     // the unit's row scales (a unit past the segment's end reads the block's first unit's)
-                hn = __ldg(cc.sg.hq + (size_t)(cc.k + (cc.k + k < cc.sg.n ? k : 0)) * 16 + lane_p * 8 + g);
+                hn = __ldg(hq + (size_t)(cc.k + (cc.k + k < cc.n ? k : 0)) * 16);
             step_mma(a4, w0, w1, b0, b1);
             if (t == H - 1) {
                 // unit k, lane (m, path): its path's share of rows g and g + 8, then the pair sum
-                const bool st = store && cc.k + k < cc.sg.n;
+                const bool st = store && cc.k + k < cc.n;
                 const uint32_t hwv[4] = {hn.x, hn.y, hn.z, hn.w};
-                const int n0 = (cc.sg.rg0 + cc.k + k) * kRowsPerGroup + g;
+                const int n0 = (rg0 + cc.k + k) * kRowsPerGroup + g;
 #pragma unroll
                 for (int rb = 0; rb < 4; ++rb) {
                     const float2 hv = __half22float2(*reinterpret_cast<const __half2 *>(&hwv[rb]));
@@ -930,8 +946,6 @@ static cudaError_t launch_dependent(bool pdl, void (*kernel)(P...), dim3 grid, d
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
 }
 
-static int g_ldg_smem[2];           // dynamic shared-memory limit raised so far, per MM
-
 template <int MM>
 static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P1Item *p1, int n1, const Plan &P,
                                 int batch, const IoPtrs &io, int base, int M, int kb2max, int rmax, cudaStream_t s,
@@ -954,14 +968,9 @@ static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P
     // unless timing events separate the launches
     const bool pdl = !profiling_active();
     const size_t slots = (size_t)kLdgWarps * kSlotPairs * 16 * MM * 16;    // one B slot per warp
-    if ((int)slots > g_ldg_smem[MM - 1]) {
-        if ((e = cudaFuncSetAttribute(contraction1_ldg_kernel<MM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)slots)) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(contraction2_ldg_kernel<MM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)slots)) != cudaSuccess)
-            return status_from(e);
-        g_ldg_smem[MM - 1] = (int)slots;
-    }
+    if ((e = ensure_dyn_smem((const void *)contraction1_ldg_kernel<MM>, slots)) != cudaSuccess ||
+        (e = ensure_dyn_smem((const void *)contraction2_ldg_kernel<MM>, slots)) != cudaSuccess)
+        return status_from(e);
     if ((e = launch_dependent(pdl, contraction1_ldg_kernel<MM>, dim3(G), dim3(kLdgWarps * 32), slots, s, dev_layers,
                               (const Seg1 *)P.sg1, bnd1, cls1, M)) != cudaSuccess)
         return status_from(e);

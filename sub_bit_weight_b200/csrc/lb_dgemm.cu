@@ -200,13 +200,8 @@ __global__ void dscale_kernel(int m, int n, double beta, double *C, long ldc)
 
 int sm_count()
 {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
+    int n = 0;
+    if (sm_count_of_current(&n) != cudaSuccess || n <= 0) n = 148;
     return n;
 }
 

@@ -691,13 +691,8 @@ struct ItqArgs {
 
 int sm_count_init()
 {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
+    int n = 0;
+    if (sm_count_of_current(&n) != cudaSuccess || n <= 0) n = 148;
     return n;
 }
 

@@ -173,6 +173,11 @@ lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc,
                             const uint16_t *x, float *y, int M, int *err, cudaStream_t s, int *launches);
 
 lb_status status_from(cudaError_t e);
+// Raise the dynamic shared-memory limit of kernel `fn` on the current device to at least `bytes` (never lowers
+// it; per device and kernel, thread-safe).
+cudaError_t ensure_dyn_smem(const void *fn, size_t bytes);
+// The current device's SM count (cached per device).
+cudaError_t sm_count_of_current(int *sms);
 void set_launch_count(int n);
 // Timing hook: record the registered event `i` (if any) on stream s.
 void profile_mark(int i, cudaStream_t s);

@@ -175,13 +175,8 @@ __global__ void __launch_bounds__(kJThreads, 1)
 
 int sm_count_j()
 {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
+    int n = 0;
+    if (sm_count_of_current(&n) != cudaSuccess || n <= 0) n = 148;
     return n;
 }
 
@@ -193,15 +188,12 @@ cudaError_t jacobi_eig(double *A, int n, long lda, double *Vt, long ldv, double 
     if (n < 1 || n > kJacobiMaxN) return cudaErrorInvalidValue;
     const int np = n + (n & 1), H = np / 2;
     const size_t smem = (size_t)H * (3 * sizeof(double) + 2 * sizeof(int)) + (size_t)2 * np * sizeof(int);
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)((size_t)(kJacobiMaxN / 2) * (3 * sizeof(double) + 2 * sizeof(int)) +
-                                   (size_t)2 * kJacobiMaxN * sizeof(int)));
-        attr = true;
-    }
+    cudaError_t e = ensure_dyn_smem((const void *)jacobi_kernel,
+                                    (size_t)(kJacobiMaxN / 2) * (3 * sizeof(double) + 2 * sizeof(int)) +
+                                        (size_t)2 * kJacobiMaxN * sizeof(int));
+    if (e != cudaSuccess) return e;
     int occ = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, jacobi_kernel, kJThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, jacobi_kernel, kJThreads, smem);
     if (e != cudaSuccess) return e;
     if (occ < 1) return cudaErrorInvalidConfiguration;
     const long items = std::max((long)H * H, (long)H * n);

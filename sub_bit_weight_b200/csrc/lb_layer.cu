@@ -8,9 +8,12 @@
 
 #include <algorithm>
 #include <array>
+#include <map>
+#include <mutex>
 #include <cstring>
 #include <new>
 
+#include "lb_attr_cache.h"
 #include "lb_prefill.cuh"
 
 namespace lb {
@@ -115,6 +118,37 @@ __global__ void build_hq_kernel(uint16_t *__restrict__ hq, int RG2, int N, int n
         const int row = rg * kRowsPerGroup + 16 * rb + g + 8 * hf;
         hq[idx] = (p < npaths && row < N) ? (p ? h1 : h0)[row] : (uint16_t)0;
     }
+}
+
+static AttrCache g_attr_cache;
+
+cudaError_t ensure_dyn_smem(const void *fn, size_t bytes)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int r = g_attr_cache.ensure(dev, fn, (long)bytes, [&](long b) {
+        return (int)cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b);
+    });
+    return (cudaError_t)r;
+}
+
+cudaError_t sm_count_of_current(int *sms)
+{
+    static std::mutex mu;
+    static std::map<int, int> counts;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = counts.find(dev);
+    if (it == counts.end()) {
+        int n = 0;
+        if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        it = counts.emplace(dev, n).first;
+    }
+    *sms = it->second;
+    return cudaSuccess;
 }
 
 static size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }

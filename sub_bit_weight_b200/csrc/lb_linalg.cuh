@@ -7,6 +7,11 @@
 
 namespace lb {
 
+// Shared with the rest of the library (defined with the layer code): raise a kernel's dynamic shared-memory
+// limit on the current device (per device and kernel, thread-safe), and the current device's SM count.
+cudaError_t ensure_dyn_smem(const void *fn, size_t bytes);
+cudaError_t sm_count_of_current(int *sms);
+
 // Row-major matrix view: element (i, j) at p[i * ld + j].
 struct DView {
     double *p;

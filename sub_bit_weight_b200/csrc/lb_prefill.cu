@@ -786,30 +786,18 @@ static size_t smem_bytes(int nlayers) { return sizeof(PfSmem) + 1024 + sizeof(in
 
 static int sm_count()
 {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    }
+    int sms = 0;
+    if (sm_count_of_current(&sms) != cudaSuccess || sms <= 0) sms = 148;
     return sms;
 }
 
 // raise the kernels' dynamic shared-memory limit to at least `smem` (grow-only, shared by every launch path)
 static cudaError_t ensure_smem(size_t smem)
 {
-    static size_t smem_set = 0;
     if (smem > 232448) return cudaErrorInvalidValue;
-    if (smem <= smem_set) return cudaSuccess;
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(prefill_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-        cudaSuccess)
-        return e;
-    if ((e = cudaFuncSetAttribute(prefill_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-        cudaSuccess)
-        return e;
-    smem_set = smem;
-    return cudaSuccess;
+    if ((e = ensure_dyn_smem((const void *)prefill_kernel<0>, smem)) != cudaSuccess) return e;
+    return ensure_dyn_smem((const void *)prefill_kernel<1>, smem);
 }
 
 lb_status prefill_forward(const Plan &Pc, const lb_layer *const *layers, const uint16_t *const *xs,
