@@ -49,6 +49,9 @@ DECODE_DEFAULT = "llama2_70b_0.1"
 PREFILL_DEFAULT = "llama2_13b_0.3_prefill"
 INIT_DEFAULT = "llama2_7b_0.1"
 BACKWARD_DEFAULT = "llama2_13b_0.3_prefill"
+# the other workloads, each at its batch sizes; the stack that fits in L2 both warm and with L2 flushed per step
+CONFIGS_DEFAULT = ("single_512:1,single_512:8,llama2_7b_0.1:1,llama2_7b_0.1:1:flushed,"
+                   "llama2_7b_0.55:1,llama2_7b_0.55:4,llama2_7b_0.55:16")
 INIT_ITERS = 24
 ITQ_ITERS = 50          # Joint-ITQ alternations of the LittleBit-2 initialisation (iterative quantisation's usual 50)
 # binary64 FMA rate of B200: 148 SMs x 64 FP64 FMA per clock x 2 FLOP at the 1965 MHz maximum SM clock
@@ -405,6 +408,61 @@ def replica_throughput(world: int, work_per_rank: float, steps: int, max_ms: flo
     return world * work_per_rank * steps / (max_ms * 1e-3)
 
 
+def roofline_of(res: dict, shapes, M: int, prefill: bool, pk: dict, wkey: str):
+    """Roofline object of the dominant kernel of one stack step, from the per-launch event timings of run_gpu.
+
+    Decode: algorithmic bytes of the kernel (layer_bytes) over its average launch time, against measured HBM copy
+    bandwidth.  Prefill: algorithmic FLOPs of the kernel over its launch time, against the measured bf16 tensor
+    peak; each kernel is timed alone (an event on each side), so the burst figure is the denominator, with the
+    sustained one beside it.
+    """
+    if not res["per_launch"]:
+        return None
+    if prefill:
+        k1ms, k2ms = res["per_launch"][:2]
+        dom = 1 if k2ms >= k1ms else 0
+        f1 = sum(2.0 * M * 2 * s.r * s.K for s in shapes)
+        f2 = sum(2.0 * M * 2 * s.r * s.N for s in shapes)
+        dom_w, dom_ms = (f2, k2ms) if dom else (f1, k1ms)
+        ach = dom_w / (dom_ms * 1e-3) / 1e12
+        kname = "prefill_kernel<1>" if dom else "prefill_kernel<0>"
+        return {"bound": "tensor", "kernel": kname + (" (output GEMM)" if dom else " (latent GEMM)"),
+                "achieved": round(ach, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(ach / pk["bf16_tflops"], 4),
+                "peak_src": pk["src"] + " bf16 burst (dense 16-bit tensor peak; the kernel is timed alone)",
+                "frac_of_sustained": round(ach / pk["bf16_tflops_sustained"], 4),
+                "traffic": measured_traffic(kname, wkey),
+                "per_kernel_ms": {"latent": round(k1ms, 4), "output": round(k2ms, 4)},
+                "per_kernel_flops": {"latent": f1, "output": f2},
+                "per_kernel_tflops": {"latent": round(f1 / (k1ms * 1e-3) / 1e12, 1),
+                                      "output": round(f2 / (k2ms * 1e-3) / 1e12, 1)}}
+    k1b = sum(layer_bytes(s, M)[0] for s in shapes)
+    k2b = sum(layer_bytes(s, M)[1] for s in shapes)
+    suffix = "_ldg_kernel" if M <= 2 else "_kernel"
+    names = ["contraction1" + suffix, "contraction2" + suffix]
+    kbytes = [k1b, k2b]
+    if len(res["per_launch"]) == 3:
+        # general kernels (3..16 rows): the per-layer finish between the contractions moves no algorithmic bytes
+        names = [names[0], "finish_general_kernel", names[1]]
+        kbytes = [k1b, 0.0, k2b]
+    if len(res["per_launch"]) == 4:
+        # activation quantisation and the contraction-1 finish run as their own launches:
+        # x and g are the bytes of the first, the finish moves no algorithmic bytes
+        qb = sum(2.0 * M * s.K + 2 * 2.0 * s.K for s in shapes)
+        names = ["quantize_pair_kernel", names[0], "finish_pair_kernel", names[1]]
+        kbytes = [qb, k1b - qb, 0.0, k2b]
+    kms = list(res["per_launch"])
+    di = max(range(len(kms)), key=lambda i: kms[i])
+    dom_bytes, dom_ms, kname = kbytes[di], kms[di], names[di]
+    ach = dom_bytes / (dom_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": kname,
+            "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(ach / pk["hbm_gbs"], 4), "peak_src": pk["src"],
+            "traffic": measured_traffic(kname, wkey), "algorithmic_bytes_per_launch": dom_bytes,
+            "per_kernel_ms": {n: round(t, 5) for n, t in zip(names, kms)},
+            "per_kernel_bytes": {n: b for n, b in zip(names, kbytes)}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -427,6 +485,9 @@ def main():
     ap.add_argument("--backward", default=BACKWARD_DEFAULT,
                     help="workload whose first block gets the QAT backward pass ('' = skip)")
     ap.add_argument("--backward-steps", type=int, default=5)
+    ap.add_argument("--configs", default=CONFIGS_DEFAULT,
+                    help="comma-separated workload[:M[:flushed]] runs for the 'configs' object ('' = skip)")
+    ap.add_argument("--config-steps", type=int, default=200)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -472,59 +533,9 @@ def main():
         value = replica_throughput(world, step_bytes, args.steps, total_ms) / 1e9
         unit = "GB/s"
 
-    roof = None
-    if res["per_launch"]:
-        if prefill_main:
-            k1ms, k2ms = res["per_launch"][:2]
-            dom = 1 if k2ms >= k1ms else 0
-            f1 = sum(2.0 * M * 2 * s.r * s.K for s in shapes)
-            f2 = sum(2.0 * M * 2 * s.r * s.N for s in shapes)
-            dom_w, dom_ms = (f2, k2ms) if dom else (f1, k1ms)
-            ach = dom_w / (dom_ms * 1e-3) / 1e12
-            kname = "prefill_kernel<1>" if dom else "prefill_kernel<0>"
-            roof = {"bound": "tensor", "kernel": kname + (" (output GEMM)" if dom else " (latent GEMM)"),
-                    "achieved": round(ach, 1), "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                    "frac": round(ach / pk["bf16_tflops_sustained"], 4),
-                    "peak_src": pk["src"] + " bf16 sustained (dense 16-bit tensor peak)",
-                    "traffic": measured_traffic(kname, w.key),
-                    "per_kernel_ms": {"latent": round(k1ms, 4), "output": round(k2ms, 4)},
-                    "per_kernel_flops": {"latent": f1, "output": f2}}
-        else:
-            suffix = "_ldg_kernel" if M <= 2 else "_kernel"
-            names = ["contraction1" + suffix, "contraction2" + suffix]
-            kbytes = [k1b, k2b]
-            if len(res["per_launch"]) == 3:
-                # general kernels (3..16 rows): the per-layer finish between the contractions moves no algorithmic bytes
-                names = [names[0], "finish_general_kernel", names[1]]
-                kbytes = [k1b, 0.0, k2b]
-            if len(res["per_launch"]) == 4:
-                # activation quantisation and the contraction-1 finish run as their own launches:
-                # x and g are the bytes of the first, the finish moves no algorithmic bytes
-                qb = sum(2.0 * M * s.K + 2 * 2.0 * s.K for s in shapes)
-                names = ["quantize_pair_kernel", names[0], "finish_pair_kernel", names[1]]
-                kbytes = [qb, k1b - qb, 0.0, k2b]
-            kms = list(res["per_launch"])
-            di = max(range(len(kms)), key=lambda i: kms[i])
-            dom_bytes, dom_ms, kname = kbytes[di], kms[di], names[di]
-            ach = dom_bytes / (dom_ms * 1e-3) / 1e9
-            roof = {"bound": "hbm", "kernel": kname,
-                    "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(ach / pk["hbm_gbs"], 4), "peak_src": pk["src"],
-                    "traffic": measured_traffic(kname, w.key), "algorithmic_bytes_per_launch": dom_bytes,
-                    "per_kernel_ms": {n: round(t, 5) for n, t in zip(names, kms)},
-                    "per_kernel_bytes": {n: b for n, b in zip(names, kbytes)}}
-    e2e = None
-    if res["e2e"]:
-        e_ms = max_over_ranks(res["e2e"]["ms"], dist)
-        e_ser = max_over_ranks(res["e2e"]["serial_ms"], dist)
-        e2e = {"value": round(world * step_bytes / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-               "h2d_bytes_per_step": res["e2e"]["h2d"], "d2h_bytes_per_step": res["e2e"]["d2h"],
-               "ms_per_step": round(e_ms, 4),
-               "how": "lb_stack_forward from pinned host x to pinned host y, steps pipelined: two device buffer sets, "
-                      "copies in and out on their own streams overlap the previous/next step's compute",
-               "serial": {"value": round(world * step_bytes / (e_ser * 1e-3) / 1e9, 2), "ms_per_step": round(e_ser, 4),
-                          "how": "copy in, compute, copy out, one stream, no overlap"}}
-
+    roof = roofline_of(res, shapes, M, prefill_main, pk, w.key)
+    e2e = e2e_of(res, dist, world, flops if prefill_main else step_bytes, prefill_main,
+                 "lb_stack_forward from pinned host x to pinned host y")
     line = {"metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -542,22 +553,10 @@ def main():
         line["config"]["bytes_per_step"] = step_bytes
 
     if args.prefill and world == 1 and not prefill_main:
-        pw = synth.WORKLOADS[args.prefill]
-        pM = pw.Ms[0]
-        pres = run_gpu(pw, pM, args.prefill_steps, 3, dist, dev, want_e2e=False)
-        pflops = sum(layer_flops(s, pM) for s in pres["shapes"])
-        pms = pres["total_ms"] / args.prefill_steps
-        tf = pflops / (pms * 1e-3) / 1e12
-        line["prefill"] = {"workload": f"{pw.key}: {pw.title}", "M": pM, "layers": len(pres["shapes"]),
-                           "value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(pms, 3),
-                           "tokens_per_s": round(pM / (pms * 1e-3), 1),
-                           "steps": args.prefill_steps, "gpu_launches": pres["launches"],
-                           "roofline": {"bound": "tensor", "achieved": round(tf, 2),
-                                        "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                                        "frac": round(tf / pk["bf16_tflops_sustained"], 4),
-                                        "peak_src": pk["src"] + " bf16 sustained (dense 16-bit tensor peak)",
-                                        "traffic": prefill_traffic(pw.key)},
-                           "clocks": pres["clocks"]}
+        line["prefill"] = run_prefill(args.prefill, args.prefill_steps, dev, pk, args.cpu_seconds)
+
+    if args.configs and world == 1:
+        line["configs"] = run_configs(args.configs, args.config_steps, dev, pk)
 
     if args.backward and world == 1:
         line["backward"] = run_backward(args.backward, args.backward_steps, 3, dev, args.cpu_seconds > 0, pk)
@@ -578,6 +577,75 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line))
+
+
+def e2e_of(res: dict, dist, world: int, work: float, prefill: bool, how: str):
+    """End-to-end object (host buffers, copies inside the timed region) from run_gpu's e2e timings."""
+    if not res["e2e"]:
+        return None
+    e_ms = max_over_ranks(res["e2e"]["ms"], dist)
+    e_ser = max_over_ranks(res["e2e"]["serial_ms"], dist)
+    scale, unit = (1e12, "TFLOP/s") if prefill else (1e9, "GB/s")
+    return {"value": round(world * work / (e_ms * 1e-3) / scale, 2), "unit": unit,
+            "h2d_bytes_per_step": res["e2e"]["h2d"], "d2h_bytes_per_step": res["e2e"]["d2h"],
+            "ms_per_step": round(e_ms, 4),
+            "how": how + ", steps pipelined: two device buffer sets, copies in and out on their own streams "
+                         "overlap the previous/next step's compute",
+            "serial": {"value": round(world * work / (e_ser * 1e-3) / scale, 2), "ms_per_step": round(e_ser, 4),
+                       "how": "copy in, compute, copy out, one stream, no overlap"}}
+
+
+def run_prefill(wkey: str, steps: int, dev, pk: dict, cpu_seconds: float):
+    """The tensor-core (prefill) stack: throughput, roofline of the dominant GEMM, end to end on one block, and
+    the oracle on a bounded sample."""
+    pw = synth.WORKLOADS[wkey]
+    pM = pw.Ms[0]
+    pres = run_gpu(pw, pM, steps, 3, None, dev, want_e2e=False)
+    pflops = sum(layer_flops(s, pM) for s in pres["shapes"])
+    pms = pres["total_ms"] / steps
+    tf = pflops / (pms * 1e-3) / 1e12
+    out = {"workload": f"{pw.key}: {pw.title}", "M": pM, "layers": len(pres["shapes"]),
+           "value": round(tf, 2), "unit": "TFLOP/s", "higher_is_better": True, "ms_per_step": round(pms, 3),
+           "tokens_per_s": round(pM / (pms * 1e-3), 1), "steps": steps, "gpu_launches": pres["launches"],
+           "l2": "inputs larger than L2 (every layer's x and weights are read from HBM)",
+           "roofline": roofline_of(pres, pres["shapes"], pM, True, pk, pw.key),
+           "step_traffic": prefill_traffic(pw.key), "clocks": pres["clocks"]}
+    # end to end on the first block (its 7 layers): the full stack's host inputs and outputs (about 25 GB per
+    # step) would be pinned twice over for the pipelined run
+    bres = run_gpu(pw, pM, max(3, min(steps, 5)), 3, None, dev, want_e2e=True, nblocks=1)
+    bflops = sum(layer_flops(s, pM) for s in bres["shapes"])
+    out["e2e"] = e2e_of(bres, None, 1, bflops, True,
+                        f"first block ({len(bres['shapes'])} layers) through lb_stack_forward from pinned host x "
+                        f"[{pM} rows] to pinned host y")
+    if cpu_seconds > 0:
+        cs = oracle_sample(pw, pM, cpu_seconds)
+        out["cpu_baseline"] = {"value": round(cs["flops"] / cs["seconds"] / 1e12, 9), "unit": "TFLOP/s",
+                               "cores": 1, "kind": "oracle",
+                               "sample": f"first {cs['layers']} layers of the stack, {cs['rows']} of M={pM} rows, "
+                                         f"{cs['seconds']:.1f} s single-threaded float64 C"}
+    return out
+
+
+def run_configs(spec: str, steps: int, dev, pk: dict):
+    """Decode throughput of the other workloads: one object per workload:M[:flushed] of `spec`."""
+    out = []
+    for item in [t for t in spec.split(",") if t]:
+        parts = item.split(":")
+        w = synth.WORKLOADS[parts[0]]
+        M = int(parts[1]) if len(parts) > 1 else w.Ms[0]
+        flushed = len(parts) > 2 and parts[2] == "flushed"
+        res = run_gpu(w, M, steps, 5, None, dev, want_e2e=False, flush_l2=flushed)
+        shapes = res["shapes"]
+        sb = sum(sum(layer_bytes(s, M)) for s in shapes)
+        ms = res["total_ms"] / steps
+        out.append({"workload": f"{w.key}: {w.title}", "M": M, "layers": len(shapes),
+                    "l2": ("L2 flushed (256 MB write) before every step; steps timed alone" if flushed else
+                           "inputs larger than L2" if sb > 126e6 else "stack fits in L2 (effective GB/s, warm)"),
+                    "value": round(sb / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "higher_is_better": True,
+                    "ms_per_step": round(ms, 5), "tokens_per_s": round(M / (ms * 1e-3), 1),
+                    "bytes_per_step": sb, "steps": steps, "gpu_launches": res["launches"],
+                    "roofline": roofline_of(res, shapes, M, False, pk, w.key), "clocks": res["clocks"]})
+    return out
 
 
 def subspace_width(s: synth.LayerShape) -> int:
@@ -790,7 +858,8 @@ def run_backward(wkey: str, steps: int, warmup: int, dev, with_cpu: bool, pk):
     kern = {"z = (x.g) V_s, (dy.h) U_s": "prefill_kernel<0> (latent contractions of the forward and transposed "
                                          "helpers in one launch, k-split units)",
             "dx": "prefill_kernel<1> (output contraction of the transposed helper)",
-            "dy^T zl": "cuBLAS fp16 GEMM", "x^T dz": "cuBLAS fp16 GEMM"}[dom]
+            "dy^T zl": "gemm_at_b_kernel (tcgen05 fp16 GEMM, both operands MN-major)",
+            "x^T dz": "gemm_at_b_kernel (tcgen05 fp16 GEMM, both operands MN-major)"}[dom]
     out = {"workload": f"{w.key} first block: " + ", ".join(f"{s.name} {s.N}x{s.K} r={s.r}" for s in shapes)
                        + f"; M = {M}, two paths; latent factors N(0, 0.02), dy N(0, 1) x 1e-4",
            "value": round(tf, 2), "unit": "TFLOP/s", "higher_is_better": True, "ms_per_block": round(ms_block, 3),

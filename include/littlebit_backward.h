@@ -18,8 +18,10 @@
  * of the transposed layer (U <-> V, h <-> g) and run on the same tcgen05
  * kernels (z and (dy (.) h) U_s in one launch whose output tiles are split
  * over k, partial sums added in float32); the two dense products dy^T zl
- * (N x 2r) and x^T dz (K x 2r) are plain fp16 GEMMs (cuBLAS) with float32
- * accumulation, run with the factor gradients on a second stream beside dx.
+ * (N x 2r) and x^T dz (K x 2r) are fp16 GEMMs with float32 accumulation on
+ * the library's own tcgen05 kernel (lb_gemm_at_b below: both operands are
+ * read MN-major, as stored), run with the factor gradients on a second stream
+ * beside dx.
  *
  * Arithmetic: x enters as bfloat16 (converted to fp16 exactly in fp16's normal
  * range, as in the forward pass); dy is multiplied by one power of two chosen
@@ -83,6 +85,26 @@ LB_API lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const floa
 /* Synchronises `stream`, returns and clears the device-side status of B's
  * contraction kernels: LB_OK or LB_ERR_TIMEOUT. */
 LB_API lb_status lb_backward_status(lb_backward *B, void *stream);
+
+/* D = alpha * A^T B: the dense products of the backward pass (dy^T zl and
+ * x^T dz) as one tcgen05 tensor-core GEMM, fp16 operands, float32
+ * accumulation and output.
+ *   A      binary16 [Kc][lda], columns 0 .. Mr-1 used   (row-major: A[k][i] at A + k*lda + i)
+ *   B      binary16 [Kc][ldb], columns 0 .. Nc-1 used
+ *   D      float32  [Mr][ldd], columns 0 .. Nc-1 written, overwritten (padding columns untouched)
+ *   alpha  device float32 scalar (read once per launch)
+ *   err    device int: left alone on success; a bounded wait in the kernel that gave up (about 2 s)
+ *          stores a nonzero code there (1 producer, 2 - 4 MMA / epilogue) and the launch ends early
+ * Kc is the contracted extent (the batch rows of the backward pass), Kc >= 1.
+ * A, B and D 16-byte aligned; lda and ldb multiples of 8, ldd of 4, Nc of
+ * 32, lda >= Mr, ldb >= Nc, ldd >= Nc.  Rows of A and B past Kc, and columns
+ * past Mr / Nc, are never read.  Enqueued on `stream`; nothing is allocated.
+ * Errors: LB_ERR_INVALID_ARG (null, misaligned or inconsistent sizes),
+ * LB_ERR_UNSUPPORTED (lda, ldb, ldd or Nc not a multiple as above, Kc = 0, no
+ * tensor-map encoder in the driver), LB_ERR_CUDA.  Mr = 0 or Nc = 0 is a
+ * no-op. */
+LB_API lb_status lb_gemm_at_b(const uint16_t *A, int lda, const uint16_t *B, int ldb, float *D, int ldd,
+                              int Kc, int Mr, int Nc, const float *alpha, int *err, void *stream);
 
 #ifdef __cplusplus
 }

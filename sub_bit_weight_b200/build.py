@@ -18,7 +18,6 @@ CSRC = os.path.join(HERE, "csrc")
 OUT_DIR = os.path.join(ROOT, "_build", "littlebit")
 LIB = os.path.join(HERE, "liblittlebit.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-CUDA_LIB = os.path.join(os.path.dirname(os.path.dirname(NVCC)), "lib64")    # cuBLAS (the backward's dense GEMMs)
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -58,7 +57,7 @@ def build(verbose: bool = False) -> str:
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [NVCC] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs + [
-        "-L" + CUDA_LIB, "-lcublas", "-Xlinker", "-rpath=" + CUDA_LIB, "-lrt", "-ldl", "-lpthread"]
+        "-lrt", "-ldl", "-lpthread"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

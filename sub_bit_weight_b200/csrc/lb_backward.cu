@@ -14,14 +14,14 @@
 // layers with l = 1): z and dzl, which are independent, in one launch whose
 // output tiles are split over k into units of even length (their fp32 partial
 // sums are added in place), dx on the output kernel.  G_U and G_V are plain
-// fp16 GEMMs (cuBLAS).  dy is
+// fp16 GEMMs on the library's tcgen05 kernel (lb_gemm.cu), both operands read
+// MN-major as stored.  dy is
 // multiplied by one power of two 2^E, chosen on the device so that dy 2^E and
 // dzl 2^E (and dz 2^E) stay below 2^14, and divided out exactly at the end.
 #include "littlebit_backward.h"
 #include "lb_internal.cuh"
 #include "lb_prefill.cuh"
 
-#include <cublas_v2.h>
 #include <cuda_fp16.h>
 #include <algorithm>
 #include <math.h>
@@ -47,7 +47,7 @@ struct lb_backward {
     lb::PfJobState *jobs = nullptr;   // the one-launch latent contractions (tensor maps, unit records)
     float *GU = nullptr;           // [N][K2]
     float *GV = nullptr;           // [K][K2]
-    cublasHandle_t blas = nullptr;
+    int *gerr = nullptr;           // error slot of the G_U / G_V GEMM kernel (bounded waits)
     cudaStream_t side = nullptr;   // G_U, G_V and the factor gradients run here, beside dx
     cudaEvent_t fork = nullptr, join = nullptr;
 };
@@ -326,10 +326,8 @@ void lb_backward_destroy(lb_backward *B)
     prefill_jobs_free(B->jobs);
     for (void *p : {(void *)B->lcat, (void *)B->h32, (void *)B->g32, (void *)B->hmax, (void *)B->Uw, (void *)B->Vw,
                     (void *)B->dl_acc, (void *)B->stat, (void *)B->dy16, (void *)B->x16, (void *)B->zpart,
-                    (void *)B->dzpart, (void *)B->GU,
-                    (void *)B->GV})
+                    (void *)B->dzpart, (void *)B->GU, (void *)B->GV, (void *)B->gerr})
         cudaFree(p);
-    if (B->blas) cublasDestroy(B->blas);
     if (B->fork) cudaEventDestroy(B->fork);
     if (B->join) cudaEventDestroy(B->join);
     if (B->side) cudaStreamDestroy(B->side);
@@ -388,12 +386,12 @@ lb_status lb_backward_create(lb_backward **out, int N, int K, int r, int npaths,
         cudaMemcpyAsync(B->Uw + (size_t)p * N * wpr, U[p], (size_t)N * wpr * 4, cudaMemcpyDeviceToDevice, s);
         cudaMemcpyAsync(B->Vw + (size_t)p * K * wpr, V[p], (size_t)K * wpr * 4, cudaMemcpyDeviceToDevice, s);
     }
-    if (cublasCreate(&B->blas) != CUBLAS_STATUS_SUCCESS) return fail(LB_ERR_CUDA);
+    if (!alloc((void **)&B->gerr, sizeof(int))) return fail(LB_ERR_OOM);
+    cudaMemsetAsync(B->gerr, 0, sizeof(int), s);
     if (cudaStreamCreateWithFlags(&B->side, cudaStreamNonBlocking) != cudaSuccess ||
         cudaEventCreateWithFlags(&B->fork, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&B->join, cudaEventDisableTiming) != cudaSuccess)
         return fail(LB_ERR_CUDA);
-    cublasSetPointerMode(B->blas, CUBLAS_POINTER_MODE_DEVICE);
     if (cudaStreamSynchronize(s) != cudaSuccess) return fail(LB_ERR_CUDA);
     cudaFree(ones);
     ones = nullptr;
@@ -476,17 +474,13 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
     launches += 2;
     profile_mark(5, s);
 
-    // G_U = dy^T zl, G_V = x^T dz (row-major; cuBLAS sees the column-major transposes), alpha = 2^-E
-    const float *alpha = B->stat + 2, *zero_d = B->stat + 4;
-    cublasSetStream(B->blas, s2);
-    if (cublasGemmEx(B->blas, CUBLAS_OP_N, CUBLAS_OP_T, K2, N, M, alpha, zf, CUDA_R_16F, K2, B->dy16, CUDA_R_16F, N,
-                     zero_d, B->GU, CUDA_R_32F, K2, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-        return joined(LB_ERR_CUDA);
+    // G_U = 2^-E (dy 2^E)^T zl [N][K2], G_V = 2^-E x^T (dz 2^E) [K][K2]: contracted over the M batch rows
+    const float *alpha = B->stat + 2;
+    if ((st = gemm_at_b(B->dy16, N, zf, K2, B->GU, K2, M, N, K2, alpha, B->gerr, s2)) != LB_OK) return joined(st);
     profile_mark(6, s2);
-    if (cublasGemmEx(B->blas, CUBLAS_OP_N, CUBLAS_OP_T, K2, K, M, alpha, dz, CUDA_R_16F, K2, B->x16, CUDA_R_16F, K,
-                     zero_d, B->GV, CUDA_R_32F, K2, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-        return joined(LB_ERR_CUDA);
+    if ((st = gemm_at_b(B->x16, K, dz, K2, B->GV, K2, M, K, K2, alpha, B->gerr, s2)) != LB_OK) return joined(st);
     profile_mark(7, s2);
+    launches += 2;
     const int wpr = (r + 31) / 32;
     FactorArgs fu{}, fv{};
     for (int p = 0; p < B->npaths; ++p) {
@@ -532,7 +526,9 @@ lb_status lb_backward_status(lb_backward *B, void *stream)
     if (!B) return LB_ERR_INVALID_ARG;
     lb_status a = lb_layer_status(B->Lf, stream), b = lb_layer_status(B->Lt, stream);
     lb_status c = LB_OK;
-    if (int *e = prefill_jobs_err(B->jobs)) {
+    // the error slots of the one-launch latent contractions and of the G_U / G_V GEMMs
+    for (int *e : {prefill_jobs_err(B->jobs), B->gerr}) {
+        if (!e) continue;
         cudaStream_t s = (cudaStream_t)stream;
         int h = 0;
         if (cudaMemcpyAsync(&h, e, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||

@@ -173,6 +173,9 @@ lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc,
                             const uint16_t *x, float *y, int M, int *err, cudaStream_t s, int *launches);
 
 lb_status status_from(cudaError_t e);
+// D = alpha A^T B on the tensor cores (fp16 in, fp32 out); arguments as lb_gemm_at_b in littlebit_backward.h
+lb_status gemm_at_b(const void *A, int lda, const void *B, int ldb, float *D, int ldd, int Kc, int Mr, int Nc,
+                    const float *alpha, int *err, cudaStream_t s);
 // Raise the dynamic shared-memory limit of kernel `fn` on the current device to at least `bytes` (never lowers
 // it; per device and kernel, thread-safe).
 cudaError_t ensure_dyn_smem(const void *fn, size_t bytes);

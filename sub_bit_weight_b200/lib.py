@@ -63,6 +63,7 @@ _sig("lb_backward_create", _st, [ctypes.POINTER(_vp), _i, _i, _i, _i] + [ctypes.
 _sig("lb_backward_destroy", None, [_vp])
 _sig("lb_layer_backward", _st, [_vp, _vp, _vp, _i] + [ctypes.POINTER(_vp)] * 2 + [_vp] + [ctypes.POINTER(_vp)] * 5 + [_vp])
 _sig("lb_backward_status", _st, [_vp, _vp])
+_sig("lb_gemm_at_b", _st, [_vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp])
 _sig("lb_dual_svid_init", _st, [_vp, _i, _i, _i, _i, _i] + [ctypes.POINTER(_vp)] * 5 + [_vp, _vp, ctypes.c_size_t, _vp])
 _sig("lb_littlebit2_workspace_bytes", ctypes.c_size_t, [_i, _i, _i])
 _sig("lb_littlebit2_init", _st, [_vp, _i, _i, _i, _i, _i, _i] + [ctypes.POINTER(_vp)] * 6 +
@@ -476,3 +477,19 @@ def lb_layer_backward(B: Backward, x: torch.Tensor, dy: torch.Tensor, U_lat, V_l
 
 def lb_backward_status(B: Backward, stream=None) -> int:
     return int(_lib.lb_backward_status(B.handle, _stream(stream)))
+
+
+def lb_gemm_at_b(A: torch.Tensor, B: torch.Tensor, alpha: torch.Tensor, err: torch.Tensor, stream=None) -> torch.Tensor:
+    """D = alpha * A^T B for A [Kc, Mr] and B [Kc, Nc] (float16, contiguous), alpha a one-element float32 CUDA tensor
+    and err a one-element int32 CUDA tensor (the kernel's bounded waits report there).  Returns D [Mr, Nc] float32."""
+    if A.dim() != 2 or B.dim() != 2 or A.shape[0] != B.shape[0]:
+        raise ValueError("A must be [Kc, Mr] and B [Kc, Nc]")
+    _numel(alpha, 1, "alpha")
+    _numel(err, 1, "err")
+    Kc, Mr = A.shape
+    Nc = B.shape[1]
+    D = torch.empty((Mr, Nc), dtype=torch.float32, device=A.device)
+    _check(_lib.lb_gemm_at_b(_dev(A, torch.float16, "A"), Mr, _dev(B, torch.float16, "B"), Nc,
+                             _dev(D, torch.float32, "D"), Nc, Kc, Mr, Nc, _dev(alpha, torch.float32, "alpha"),
+                             _dev(err, torch.int32, "err"), _stream(stream)), "lb_gemm_at_b")
+    return D

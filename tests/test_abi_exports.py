@@ -141,3 +141,24 @@ def test_backward_argument_checks(lib):
     assert len(binding._lib.lb_backward_create.argtypes) == 11
     assert len(binding._lib.lb_dual_svid_init.argtypes) == 15
     assert len(binding._lib.lb_littlebit2_init.argtypes) == 19
+
+
+def test_gemm_argument_checks(lib):
+    """lb_gemm_at_b rejects bad arguments before touching the device."""
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    f = lib.lb_gemm_at_b
+    f.argtypes = [vp, i, vp, i, vp, i, i, i, i, vp, vp, vp]
+    a = vp(256)
+    assert f(None, 64, a, 64, a, 64, 8, 64, 64, a, a, None) == 1            # null A
+    assert f(a, 64, a, 64, a, 64, 8, 64, 64, None, a, None) == 1            # null alpha
+    assert f(a, 64, a, 64, a, 64, 8, 64, 64, a, None, None) == 1            # null err
+    assert f(vp(264), 64, a, 64, a, 64, 8, 64, 64, a, a, None) == 1        # misaligned A
+    assert f(a, 32, a, 64, a, 64, 8, 64, 64, a, a, None) == 1               # lda < Mr
+    assert f(a, 68, a, 64, a, 64, 8, 64, 64, a, a, None) == 2               # lda not a multiple of 8
+    assert f(a, 64, a, 48, a, 48, 8, 64, 48, a, a, None) == 2               # Nc not a multiple of 32
+    assert f(a, 64, a, 64, a, 66, 8, 64, 64, a, a, None) == 2               # ldd not a multiple of 4
+    assert f(a, 64, a, 64, a, 64, 0, 64, 64, a, a, None) == 2               # Kc = 0
+    assert f(a, 64, a, 64, a, 64, 8, 0, 64, a, a, None) == 0                # Mr = 0: nothing to do
+    assert f(a, 64, a, 64, a, 64, -1, 64, 64, a, a, None) == 1
+    from sub_bit_weight_b200 import lib as binding
+    assert len(binding._lib.lb_gemm_at_b.argtypes) == 12

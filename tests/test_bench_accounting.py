@@ -108,3 +108,38 @@ def test_dram_traffic_is_reported_only_for_the_sources_it_was_captured_with(tmp_
     last = src / bench.KERNEL_SOURCES[k][-1]
     last.write_bytes(last.read_bytes() + b"\n")
     assert bench.source_hash(k) != good
+
+
+def test_roofline_denominators():
+    """Decode kernels are measured against HBM copy bandwidth; the prefill GEMMs, each timed alone, against the
+    burst tensor peak (the sustained one reported beside it)."""
+    pk = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "src": "measured"}
+    p = synth.WORKLOADS["llama2_13b_0.3_prefill"]
+    shapes = list(p.block)
+    r = bench.roofline_of({"per_launch": (1.0, 2.0)}, shapes, 2048, True, pk, p.key)
+    f2 = sum(2.0 * 2048 * 2 * s.r * s.N for s in shapes)
+    assert r["kernel"].startswith("prefill_kernel<1>")
+    assert r["achieved"] == pytest.approx(f2 / 2e-3 / 1e12, abs=0.1)
+    assert r["peak"] == 1600.0 and r["frac"] == pytest.approx(r["achieved"] / 1600.0, abs=1e-4)
+    assert r["frac_of_sustained"] == pytest.approx(r["achieved"] / 1400.0, abs=1e-4)
+    w = synth.WORKLOADS["llama2_70b_0.1"]
+    shapes = list(w.block)
+    q = sum(2.0 * s.K + 2 * 2.0 * s.K for s in shapes)
+    k1 = sum(bench.layer_bytes(s, 1)[0] for s in shapes)
+    r = bench.roofline_of({"per_launch": (0.01, 0.05, 0.005, 0.02)}, shapes, 1, False, pk, w.key)
+    assert r["kernel"] == "contraction1_ldg_kernel"
+    assert r["algorithmic_bytes_per_launch"] == pytest.approx(k1 - q)
+    assert r["frac"] == pytest.approx((k1 - q) / 0.05e-3 / 1e9 / 6000.0, abs=1e-4)
+    r = bench.roofline_of({"per_launch": (0.01, 0.001, 0.02)}, shapes, 4, False, pk, w.key)
+    assert r["kernel"] == "contraction2_kernel"
+    assert bench.roofline_of({"per_launch": None}, shapes, 4, False, pk, w.key) is None
+
+
+def test_config_runs_cover_the_other_workloads():
+    items = [t.split(":") for t in bench.CONFIGS_DEFAULT.split(",")]
+    got = {(t[0], int(t[1]), len(t) > 2) for t in items}
+    assert {("single_512", 1, False), ("single_512", 8, False)} <= got
+    assert {("llama2_7b_0.1", 1, False), ("llama2_7b_0.1", 1, True)} <= got
+    assert {("llama2_7b_0.55", m, False) for m in (1, 4, 16)} <= got
+    for name, M, _ in got:
+        assert M in synth.WORKLOADS[name].Ms
