@@ -782,7 +782,7 @@ def backward_stage_flops(s: synth.LayerShape, M: int, npaths: int = 2):
     """Algorithmic FLOPs of the backward stages of one layer (2 FLOPs per multiply-add, no padding)."""
     R = npaths * s.r
     return {"z = (x.g) V_s, (dy.h) U_s": 2.0 * M * (s.K + s.N) * R, "dx": 2.0 * M * R * s.K,
-            "dy^T zl": 2.0 * M * s.N * R, "x^T dz": 2.0 * M * s.K * R}
+            "dy^T zl, x^T dz": 2.0 * M * (s.N + s.K) * R}
 
 
 def run_backward(wkey: str, steps: int, warmup: int, dev, with_cpu: bool, pk):
@@ -839,10 +839,11 @@ def run_backward(wkey: str, steps: int, warmup: int, dev, with_cpu: bool, pk):
     for e in ev:
         e.record()
     torch.cuda.synchronize()
-    # events 2 and 3 mark the same point (z and dzl run in one launch); after event 4 dx runs on the caller's
-    # stream (4 -> 5) beside dy^T zl (4 -> 6), x^T dz (6 -> 7) and the factor gradients (7 -> 8) on a second stream
+    # events 2 and 3 mark the same point (z and dzl run in one launch), and so do 6 and 7 (dy^T zl and x^T dz);
+    # after event 4 dx runs on the caller's stream (4 -> 5) beside the two dense products (4 -> 6) and the factor
+    # gradients (7 -> 8) on a second stream
     spans = {"dy scaling": (0, 1), "z = (x.g) V_s, (dy.h) U_s": (1, 2), "dl, dz, zl": (3, 4), "dx": (4, 5),
-             "dy^T zl": (4, 6), "x^T dz": (6, 7), "dh, dg, dU, dV": (7, 8)}
+             "dy^T zl, x^T dz": (4, 6), "dh, dg, dU, dV": (7, 8)}
     stage = {n: 0.0 for n in spans}
     reps = 5
     for _ in range(reps):
@@ -858,8 +859,8 @@ def run_backward(wkey: str, steps: int, warmup: int, dev, with_cpu: bool, pk):
     kern = {"z = (x.g) V_s, (dy.h) U_s": "prefill_kernel<0> (latent contractions of the forward and transposed "
                                          "helpers in one launch, k-split units)",
             "dx": "prefill_kernel<1> (output contraction of the transposed helper)",
-            "dy^T zl": "gemm_at_b_kernel (tcgen05 fp16 GEMM, both operands MN-major)",
-            "x^T dz": "gemm_at_b_kernel (tcgen05 fp16 GEMM, both operands MN-major)"}[dom]
+            "dy^T zl, x^T dz": "gemm_at_b_kernel (tcgen05 fp16 GEMM, both operands MN-major, both products in one "
+                               "launch)"}[dom]
     out = {"workload": f"{w.key} first block: " + ", ".join(f"{s.name} {s.N}x{s.K} r={s.r}" for s in shapes)
                        + f"; M = {M}, two paths; latent factors N(0, 0.02), dy N(0, 1) x 1e-4",
            "value": round(tf, 2), "unit": "TFLOP/s", "higher_is_better": True, "ms_per_block": round(ms_block, 3),

@@ -143,15 +143,15 @@ LB_API size_t lb_layer_device_bytes(const lb_layer *L);
  * stream, or explicit events); concurrent calls on one layer race.
  * Non-finite values in a row of x give NaN in that row of y.
  * Errors: LB_ERR_INVALID_ARG (NULL, M < 0, misalignment), LB_ERR_OOM
- * (scratch growth for a larger M than before), LB_ERR_CUDA, and
- * LB_ERR_UNSUPPORTED when the decode kernels cannot hold the layer's
- * contraction-2 depth in shared memory.  Decode (M <= 16, and larger M when
- * K is not a multiple of 8 or N not a multiple of 4, which then run as 16-row
- * blocks) needs (8 + ceil(min(M,16)/4)) * KB2 * 256 bytes <= 227 KB, with
- * KB2 = npaths * ceil(r/32) k-blocks of 32 latent indices: one path takes any
- * r <= LB_MAX_RANK; two paths take r <= 1184 at every M, r <= 1600 at M <= 4.
- * (For one or two rows and KB2 <= 64 a streaming design without this limit
- * runs instead.)
+ * (scratch growth for a larger M than before), LB_ERR_CUDA.  Every r <=
+ * LB_MAX_RANK runs with one or two paths at every M: one or two rows run on
+ * streaming kernels whose depth has no shared-memory bound; 3..16 rows run on
+ * kernels that stage a row group's contraction-2 tiles in shared memory,
+ * (8 + ceil(min(M,16)/4)) * KB2 * 256 bytes <= 227 KB with KB2 = npaths *
+ * ceil(r/32) (two paths: r <= 1184 at every M, r <= 1600 at M <= 4), and a
+ * deeper layer (or stack) takes the streaming kernels once per pair of rows
+ * instead.  (Decode also serves larger M when K is not a multiple of 8 or N
+ * not a multiple of 4, as 16-row blocks.)
  */
 LB_API lb_status lb_linear_forward(const uint16_t *x, int M, const lb_layer *L, float *y, void *stream);
 

@@ -75,8 +75,9 @@ LB_API void lb_backward_destroy(lb_backward *B);
  * events[i] is recorded at the i-th stage boundary: 0 | dy scaling | 1 |
  * z = (x (.) g) V_s and (dy (.) h) U_s, one launch | 2, 3 | dl, dz, zl | 4;
  * after 4 the work forks: dx | 5 on `stream`, and on a second stream of the
- * library (joined back into `stream` before the call returns) dy^T zl | 6 |
- * x^T dz | 7 | dh, dg, dU, dV | 8 (events 2 and 3 mark the same point). */
+ * library (joined back into `stream` before the call returns) dy^T zl and
+ * x^T dz, one launch | 6, 7 | dh, dg, dU, dV | 8 (events 2 and 3 mark the same
+ * point, and so do 6 and 7). */
 LB_API lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, int M,
                                    const float *const *U_lat, const float *const *V_lat, float *dx,
                                    float *const *dh, float *const *dg, float *const *dl,

@@ -418,7 +418,7 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
     int launches = 0;
 
     // timing hook (littlebit.h): events 0 | scaling | 1 | z and dzl (one launch) | 2, 3 | dl, dz, zl | 4, then
-    // dx | 5 on this stream and, from 4 on the side stream, G_U | 6 | G_V | 7 | factor gradients | 8
+    // dx | 5 on this stream and, from 4 on the side stream, G_U and G_V (one launch) | 6, 7 | factor gradients | 8
     profile_mark(0, s);
     // dy scale (device-side exponent), fp16 copies of dy 2^E and x
     cudaMemsetAsync(B->stat, 0, sizeof(float), s);
@@ -475,12 +475,13 @@ lb_status lb_layer_backward(lb_backward *B, const uint16_t *x, const float *dy, 
     profile_mark(5, s);
 
     // G_U = 2^-E (dy 2^E)^T zl [N][K2], G_V = 2^-E x^T (dz 2^E) [K][K2]: contracted over the M batch rows
+    // (one launch: G_V's tiles fill the last wave of G_U's)
     const float *alpha = B->stat + 2;
-    if ((st = gemm_at_b(B->dy16, N, zf, K2, B->GU, K2, M, N, K2, alpha, B->gerr, s2)) != LB_OK) return joined(st);
+    const GemmDesc gd[2] = {{B->dy16, N, zf, K2, B->GU, K2, M, N, K2, alpha}, {B->x16, K, dz, K2, B->GV, K2, M, K, K2, alpha}};
+    if ((st = gemm_at_b_batch(gd, 2, B->gerr, s2)) != LB_OK) return joined(st);
     profile_mark(6, s2);
-    if ((st = gemm_at_b(B->x16, K, dz, K2, B->GV, K2, M, K, K2, alpha, B->gerr, s2)) != LB_OK) return joined(st);
     profile_mark(7, s2);
-    launches += 2;
+    launches += 1;
     const int wpr = (r + 31) / 32;
     FactorArgs fu{}, fv{};
     for (int p = 0; p < B->npaths; ++p) {

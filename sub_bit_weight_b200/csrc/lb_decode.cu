@@ -577,16 +577,20 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
                          (size_t)2 * kP1ChunkKB * NT * 32 * sizeof(uint2);
     const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * ((kb2max + 1) & ~1) * 256 +
                          (size_t)NT * kb2max * 32 * sizeof(uint2);
-    if (smem2 > 227 * 1024) return LB_ERR_UNSUPPORTED;
-    if ((e = ensure_dyn_smem((const void *)k1, smem1)) != cudaSuccess) return status_from(e);
-    if ((e = ensure_dyn_smem((const void *)k2, smem2)) != cudaSuccess) return status_from(e);
-    int occ1 = 0, occ2 = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, k1, kDecodeThreads, smem1)) != cudaSuccess)
-        return status_from(e);
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ2, k2, kDecodeThreads, smem2)) != cudaSuccess)
-        return status_from(e);
-    occ1 = std::max(1, occ1);
-    occ2 = std::max(1, occ2);
+    // a stack deeper than the general kernels' shared memory holds runs on the one/two-row streaming kernels
+    // (no shared-memory bound on the depth), once per pair of activation rows
+    const bool by_pairs = M > 2 && smem2 > 227 * 1024;
+    int occ1 = 1, occ2 = 1;
+    if (!by_pairs) {
+        if ((e = ensure_dyn_smem((const void *)k1, smem1)) != cudaSuccess) return status_from(e);
+        if ((e = ensure_dyn_smem((const void *)k2, smem2)) != cudaSuccess) return status_from(e);
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, k1, kDecodeThreads, smem1)) != cudaSuccess)
+            return status_from(e);
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ2, k2, kDecodeThreads, smem2)) != cudaSuccess)
+            return status_from(e);
+        occ1 = std::max(1, occ1);
+        occ2 = std::max(1, occ2);
+    }
 
     static thread_local IoPtrs io;
     profile_mark(0, s);
@@ -594,6 +598,20 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
     for (int b = 0; b < nb; ++b) {
         const int base = b * kIoBatch;
         const int cnt = std::min(kIoBatch, P.n - base);
+        if (by_pairs) {
+            for (int m0 = 0; m0 < M; m0 += 2) {
+                for (int i = 0; i < cnt; ++i) {
+                    const LayerDev &d = P.host[base + i];
+                    io.x[i] = xs[base + i] + (size_t)m0 * d.K;
+                    io.y[i] = ys[base + i] + (size_t)m0 * d.N;
+                }
+                const lb_status st = decode_pair_launch(P.dev, cnt, P.p1 + P.p1_start[b], P.p1_start[b + 1] - P.p1_start[b],
+                                                        P, b, io, base, std::min(2, M - m0), kb2max, P.rmax, P.err, s,
+                                                        launches, true);
+                if (st != LB_OK) return st;
+            }
+            continue;
+        }
         for (int i = 0; i < cnt; ++i) {
             io.x[i] = xs[base + i];
             io.y[i] = ys[base + i];
@@ -656,7 +674,18 @@ lb_status decode_launch_one(const LayerDev *dev_desc, const LayerDev &host_desc,
                          (size_t)2 * kP1ChunkKB * NT * 32 * sizeof(uint2);
     const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * ((kb2max + 1) & ~1) * 256 +
                          (size_t)NT * kb2max * 32 * sizeof(uint2);
-    if (smem2 > 227 * 1024) return LB_ERR_UNSUPPORTED;
+    if (smem2 > 227 * 1024) {
+        // too deep for the general kernels: the one/two-row streaming kernels, once per pair of rows
+        static thread_local IoPtrs iop;
+        for (int m0 = 0; m0 < M; m0 += 2) {
+            iop.x[0] = x + (size_t)m0 * host_desc.K;
+            iop.y[0] = y + (size_t)m0 * host_desc.N;
+            const lb_status st = decode_pair_launch(dev_desc, 1, p1, n1, P, 0, iop, 0, std::min(2, M - m0),
+                                                    host_desc.KB2, host_desc.r, err, s, launches, false);
+            if (st != LB_OK) return st;
+        }
+        return LB_OK;
+    }
     if ((e = ensure_dyn_smem((const void *)k1, smem1)) != cudaSuccess) return status_from(e);
     if ((e = ensure_dyn_smem((const void *)k2, smem2)) != cudaSuccess) return status_from(e);
     int occ1 = 0, occ2 = 0;

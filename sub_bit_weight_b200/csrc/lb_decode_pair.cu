@@ -691,12 +691,25 @@ static __device__ __forceinline__ void sts128(uint32_t addr, uint4 v)
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
 }
+// Each warp owns kSlotRegion bytes: one slot of two-row fragments, or two slots of one-row fragments (contraction
+// 1 fetches the next segment's fragments into the second while the first is read).
+constexpr uint32_t kSlotBytes1 = kSlotPairs * 16 * 16;      // one slot, one activation row
+constexpr uint32_t kSlotRegion = 2 * kSlotBytes1;
 template <int MM>
 static __device__ __forceinline__ uint32_t b_slot(int warp)
 {
+    static_assert(kSlotPairs * 16 * MM * 16 <= kSlotRegion, "slot region");
     extern __shared__ __align__(16) unsigned char sm_raw[];
-    return sm_addr(sm_raw) + (uint32_t)warp * (kSlotPairs * 16 * MM * 16);
+    return sm_addr(sm_raw) + (uint32_t)warp * kSlotRegion;
 }
+
+// 16-byte asynchronous copy global -> shared through L2 (data of the previous launch: never the read-only path)
+static __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+static __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+static __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 template <int MM, int H>
 static __device__ __forceinline__ void b_fill(uint32_t slot, const uint4 *src, int P, int lane)
 {
@@ -737,26 +750,63 @@ static __device__ __noinline__ void c1_static(const LayerDev *__restrict__ layer
 
     dep_wait();     // B fragments, exponents and cleared accumulators come from the previous kernels
 
-    const uint32_t slot = b_slot<MM>(warp), bsl = slot + blane * 16;
+    const uint32_t slot = b_slot<MM>(warp);
+    uint32_t bsl = slot + blane * 16;
     double *acc = nullptr;
     int npaths = 1, r16 = 0;
     double lsc = 0.0;
     bool elive = false;
     int rg0 = 0;
-    auto seg_in = [&]() {
-        const Seg1 sg = segs[cc.s];
+    // one row: segment s + 1's fragments (cp.async into the other slot), exponent and layer fields are fetched
+    // when segment s starts, so that entering a segment waits for nothing but copies issued a segment earlier
+    int par = 0;                     // slot of the current segment
+    double *n_acc = nullptr;
+    int n_npaths = 1, n_r16 = 0, n_rg0 = 0, n_E = kNanExp;
+    auto prefetch = [&](int s, uint32_t dst) {
+        const Seg1 sg = segs[s];
         const LayerDev *dp = layers + sg.layer;
-        b_fill<MM, H>(slot, reinterpret_cast<const uint4 *>(dp->xfrag) + (size_t)sg.kc * (kP1ChunkKB / 2) * 16 * MM,
-                      sg.P, lane);
-        rg0 = sg.rg0;
-        acc = dp->acc;
-        npaths = dp->npaths;
-        r16 = dp->r16;
-        const int E = (lane_m < M && lane_p < npaths) ? __ldcg(dp->xmeta + sg.kc * 4 + 2 * lane_p + lane_m)
-                                                     : kNanExp;
-        elive = E != kNanExp;
-        lsc = elive ? pow2d(-E) : 0.0;
+        const uint4 *src = reinterpret_cast<const uint4 *>(dp->xfrag) + (size_t)sg.kc * (kP1ChunkKB / 2) * 16 * MM;
+#pragma unroll
+        for (int i = lane; i < 2 * H * 16 * MM; i += 32) {
+            if (i < sg.P * 16 * MM) cp_async16(dst + (uint32_t)i * 16, src + i);
+            else sts128(dst + (uint32_t)i * 16, make_uint4(0u, 0u, 0u, 0u));
+        }
+        cp_async_commit();
+        n_rg0 = sg.rg0;
+        n_acc = dp->acc;
+        n_npaths = dp->npaths;
+        n_r16 = dp->r16;
+        n_E = (lane_m < M && lane_p < n_npaths) ? __ldcg(dp->xmeta + sg.kc * 4 + 2 * lane_p + lane_m) : kNanExp;
     };
+    auto seg_in = [&]() {
+        if constexpr (MM == 1) {
+            cp_async_wait_all();     // this segment's fragments (fetched a segment ago) have landed
+            __syncwarp();            // ... for every lane, and every lane is done with the other slot
+            bsl = slot + (uint32_t)par * kSlotBytes1 + blane * 16;
+            rg0 = n_rg0;
+            acc = n_acc;
+            npaths = n_npaths;
+            r16 = n_r16;
+            elive = n_E != kNanExp;
+            lsc = elive ? pow2d(-n_E) : 0.0;
+            par ^= 1;
+            if (cc.s + 1 < s1) prefetch(cc.s + 1, slot + (uint32_t)par * kSlotBytes1);
+        } else {
+            const Seg1 sg = segs[cc.s];
+            const LayerDev *dp = layers + sg.layer;
+            b_fill<MM, H>(slot, reinterpret_cast<const uint4 *>(dp->xfrag) + (size_t)sg.kc * (kP1ChunkKB / 2) * 16 * MM,
+                          sg.P, lane);
+            rg0 = sg.rg0;
+            acc = dp->acc;
+            npaths = dp->npaths;
+            r16 = dp->r16;
+            const int E = (lane_m < M && lane_p < npaths) ? __ldcg(dp->xmeta + sg.kc * 4 + 2 * lane_p + lane_m)
+                                                         : kNanExp;
+            elive = E != kNanExp;
+            lsc = elive ? pow2d(-E) : 0.0;
+        }
+    };
+    if constexpr (MM == 1) prefetch(s0, slot);
     seg_in();
     int a4[4][4];
     zero_acc(a4);
@@ -967,7 +1017,7 @@ static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P
     // the three kernels after the quantisation may each start while the previous one drains,
     // unless timing events separate the launches
     const bool pdl = !profiling_active();
-    const size_t slots = (size_t)kLdgWarps * kSlotPairs * 16 * MM * 16;    // one B slot per warp
+    const size_t slots = (size_t)kLdgWarps * kSlotRegion;    // each warp's B slots
     if ((e = ensure_dyn_smem((const void *)contraction1_ldg_kernel<MM>, slots)) != cudaSuccess ||
         (e = ensure_dyn_smem((const void *)contraction2_ldg_kernel<MM>, slots)) != cudaSuccess)
         return status_from(e);

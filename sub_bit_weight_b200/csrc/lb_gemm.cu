@@ -21,10 +21,13 @@
 //               per warp and step), times alpha, through a 128-byte-swizzled
 //               staging block, one TMA store per block (clipped at the edges)
 // Two 256-column accumulators let the epilogue of one tile overlap the main
-// loop of the next.  Every wait is bounded: on timeout the kernel records an
-// error code in *err and returns.
+// loop of the next.  One launch may carry two problems (G_U and G_V): their
+// tiles form one list dealt round-robin to the CTAs, so the smaller problem
+// fills the other's last partial wave.  Every wait is bounded: on timeout the
+// kernel records an error code in *err and returns.
 
 #include <algorithm>
+#include <cstring>
 
 #include "lb_internal.cuh"
 #include "lb_tc.cuh"
@@ -52,16 +55,26 @@ struct GemmSmem {
 
 constexpr size_t kGemmSmemBytes = sizeof(GemmSmem) + 1024;
 
+// One problem of a launch: maps of A [Kc][Mr], B [Kc][Nc] (fp16) and D [Mr][Nc] (fp32), its sizes, and the first
+// index of its tiles in the launch's tile list.
+struct GemmProb {
+    CUtensorMap mA, mB, mD;
+    const float *alpha;
+    int Kc, Mr, Nc, ntj, nkb, tile0;
+};
+constexpr int kGemmMaxProbs = 2;
+struct GemmBatch {
+    GemmProb p[kGemmMaxProbs];
+    int n, ntiles;
+};
+
 // fp16 A and B, both MN-major; fp32 accumulator; M = 128, N = n
 __device__ __forceinline__ uint32_t idesc_f16_mn(int n)
 {
     return (1u << 4) | (1u << 15) | (1u << 16) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kGBM >> 4) << 24);
 }
 
-__global__ void __launch_bounds__(kGThreads, 1)
-    gemm_at_b_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
-                     const __grid_constant__ CUtensorMap mD, int Kc, int Mr, int Nc, const float *__restrict__ alpha,
-                     int *err)
+__global__ void __launch_bounds__(kGThreads, 1) gemm_at_b_kernel(const __grid_constant__ GemmBatch G, int *err)
 {
     extern __shared__ __align__(1024) unsigned char g_raw[];
     const uint32_t raw_addr = smem_u32(g_raw);
@@ -89,27 +102,34 @@ __global__ void __launch_bounds__(kGThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
+    const int ntiles = G.ntiles;
 
-    const int nti = (Mr + kGBM - 1) / kGBM, ntj = (Nc + kGBN - 1) / kGBN;
-    const int ntiles = nti * ntj, nkb = (Kc + kGBK - 1) / kGBK;
-    // tile t -> (i tile t / ntj, j tile t % ntj): the CTAs in flight share a few i tiles of A, and B (the latent
-    // side, small) stays in L2
+    // tile t -> problem q, (i tile, j tile) = (local / ntj, local % ntj): the CTAs in flight share a few i tiles of
+    // A, and B (the latent side, small) stays in L2
+    auto locate = [&](int t, int &q, int &i0, int &j0) {
+        q = (G.n > 1 && t >= G.p[1].tile0) ? 1 : 0;
+        const int local = t - G.p[q].tile0, ntj = G.p[q].ntj;
+        i0 = (local / ntj) * kGBM;
+        j0 = (local % ntj) * kGBN;
+    };
 
     if (warp == 0) {
         // ---------------- producer
         if (lane == 0) {
             uint32_t it = 0, pend = 0, pend_ph = 0;
             for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
-                const int i0 = (t / ntj) * kGBM, j0 = (t % ntj) * kGBN;
-                const int na = min(kGBM / 64, (Mr - i0 + 63) / 64);   // slices with at least one row in range
-                const int nb = min(kGBN / 64, (Nc - j0 + 63) / 64);
-                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                int q, i0, j0;
+                locate(t, q, i0, j0);
+                const GemmProb &P = G.p[q];
+                const int na = min(kGBM / 64, (P.Mr - i0 + 63) / 64);   // slices with at least one row in range
+                const int nb = min(kGBN / 64, (P.Nc - j0 + 63) / 64);
+                for (int kb = 0; kb < P.nkb; ++kb, ++it) {
                     const int s = it % kGStages;
                     const uint32_t ph = (it / kGStages) & 1;
                     if (!mbar_wait(&S.empty[s], ph ^ 1, abort, err, 1)) break;
                     mbar_expect_tx(&S.full[s], (uint32_t)(na + nb) * kSlice);
-                    for (int b = 0; b < na; ++b) tma_load_2d(S.A[s] + b * kSlice, &mA, i0 + 64 * b, kb * kGBK, &S.full[s]);
-                    for (int b = 0; b < nb; ++b) tma_load_2d(S.B[s] + b * kSlice, &mB, j0 + 64 * b, kb * kGBK, &S.full[s]);
+                    for (int b = 0; b < na; ++b) tma_load_2d(S.A[s] + b * kSlice, &P.mA, i0 + 64 * b, kb * kGBK, &S.full[s]);
+                    for (int b = 0; b < nb; ++b) tma_load_2d(S.B[s] + b * kSlice, &P.mB, j0 + 64 * b, kb * kGBK, &S.full[s]);
                     pend |= 1u << s;
                     pend_ph = (pend_ph & ~(1u << s)) | (ph << s);
                 }
@@ -129,8 +149,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (lane == 0) {
             uint32_t it = 0, tcount = 0;
             for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tcount) {
-                const int j0 = (t % ntj) * kGBN;
-                const int nw = min(kGBN, Nc - j0);
+                int q, i0, j0;
+                locate(t, q, i0, j0);
+                const int nkb = G.p[q].nkb;
+                const int nw = min(kGBN, G.p[q].Nc - j0);
                 const int ab = tcount & 1;
                 const uint32_t aph = (tcount >> 1) & 1;
                 if (!mbar_wait(&S.acce[ab], aph ^ 1, abort, err, 2)) break;
@@ -159,21 +181,25 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
     } else {
         // ---------------- epilogue (warps 2-5: tensor-memory lanes 32 (warp % 4) ..)
-        const int q = warp & 3;
-        const float f = __ldg(alpha);
+        const int q4 = warp & 3;
+        float f[kGemmMaxProbs];
+        for (int q = 0; q < G.n; ++q) f[q] = __ldg(G.p[q].alpha);
         uint32_t tcount = 0;
         bool stored = false;
         for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tcount) {
-            const int i0 = (t / ntj) * kGBM, j0 = (t % ntj) * kGBN;
-            const int nw = min(kGBN, Nc - j0);
+            int q, i0, j0;
+            locate(t, q, i0, j0);
+            const GemmProb &P = G.p[q];
+            const float fq = q ? f[1] : f[0];
+            const int nw = min(kGBN, P.Nc - j0);
             const int ab = tcount & 1;
             const uint32_t aph = (tcount >> 1) & 1;
             if (!mbar_wait(&S.accf[ab], aph, abort, err, 4)) break;
             tc_fence_after();
-            const uint32_t sta = smem_u32(S.ST[q]);
+            const uint32_t sta = smem_u32(S.ST[q4]);
             for (int ch = 0; ch < nw; ch += 32) {
                 uint32_t v[32];
-                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * kGBN + ch), v);
+                tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(ab * kGBN + ch), v);
                 if (stored) {   // the previous store has finished reading the staging block
                     if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
                     __syncwarp();
@@ -181,16 +207,16 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     sts128(sta + sw128(lane, i),
-                           make_uint4(__float_as_uint(__uint_as_float(v[4 * i]) * f),
-                                      __float_as_uint(__uint_as_float(v[4 * i + 1]) * f),
-                                      __float_as_uint(__uint_as_float(v[4 * i + 2]) * f),
-                                      __float_as_uint(__uint_as_float(v[4 * i + 3]) * f)));
+                           make_uint4(__float_as_uint(__uint_as_float(v[4 * i]) * fq),
+                                      __float_as_uint(__uint_as_float(v[4 * i + 1]) * fq),
+                                      __float_as_uint(__uint_as_float(v[4 * i + 2]) * fq),
+                                      __float_as_uint(__uint_as_float(v[4 * i + 3]) * fq)));
                 fence_proxy_async();
                 __syncwarp();
-                if (lane == 0 && i0 + q * 32 < Mr) {
+                if (lane == 0 && i0 + q4 * 32 < P.Mr) {
                     asm volatile(
-                        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(&mD),
-                        "r"(j0 + ch), "r"(i0 + q * 32), "r"(sta)
+                        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(&P.mD),
+                        "r"(j0 + ch), "r"(i0 + q4 * 32), "r"(sta)
                         : "memory");
                     asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
                 }
@@ -213,29 +239,67 @@ __global__ void __launch_bounds__(kGThreads, 1)
 
 }  // namespace
 
-lb_status gemm_at_b(const void *A, int lda, const void *B, int ldb, float *D, int ldd, int Kc, int Mr, int Nc,
-                    const float *alpha, int *err, cudaStream_t s)
+static lb_status check_desc(const GemmDesc &d)
 {
-    if (!A || !B || !D || !alpha || !err || Kc < 0 || Mr < 0 || Nc < 0) return LB_ERR_INVALID_ARG;
-    if (Mr == 0 || Nc == 0) return LB_OK;
-    if (lda < Mr || ldb < Nc || ldd < Nc) return LB_ERR_INVALID_ARG;
-    if (((uintptr_t)A | (uintptr_t)B | (uintptr_t)D) & 15) return LB_ERR_INVALID_ARG;
-    if (lda % 8 || ldb % 8 || ldd % 4 || Nc % 32) return LB_ERR_UNSUPPORTED;
-    if (Kc == 0) return LB_ERR_UNSUPPORTED;   // an empty contraction: the caller zeroes D itself
-    if (tmap_encoder_ready() != cudaSuccess) return LB_ERR_UNSUPPORTED;
-    CUtensorMap mA, mB, mD;
-    if (!tmap_encode_2d(&mA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, A, Mr, Kc, (long)lda * 2, 64, kGBK) ||
-        !tmap_encode_2d(&mB, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, B, Nc, Kc, (long)ldb * 2, 64, kGBK) ||
-        !tmap_encode_2d(&mD, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, D, Nc, Mr, (long)ldd * 4, 32, 32))
-        return LB_ERR_INVALID_ARG;
+    if (!d.A || !d.B || !d.D || !d.alpha || d.Kc < 0 || d.Mr < 0 || d.Nc < 0) return LB_ERR_INVALID_ARG;
+    if (d.Mr == 0 || d.Nc == 0) return LB_OK;
+    if (d.lda < d.Mr || d.ldb < d.Nc || d.ldd < d.Nc) return LB_ERR_INVALID_ARG;
+    if (((uintptr_t)d.A | (uintptr_t)d.B | (uintptr_t)d.D) & 15) return LB_ERR_INVALID_ARG;
+    if (d.lda % 8 || d.ldb % 8 || d.ldd % 4 || d.Nc % 32) return LB_ERR_UNSUPPORTED;
+    if (d.Kc == 0) return LB_ERR_UNSUPPORTED;   // an empty contraction: the caller zeroes D itself
+    return LB_OK;
+}
+
+lb_status gemm_at_b_batch(const GemmDesc *descs, int n, int *err, cudaStream_t s)
+{
+    if (!descs || !err || n < 1 || n > kGemmMaxProbs) return LB_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        const lb_status st = check_desc(descs[i]);
+        if (st != LB_OK) return st;
+    }
+    GemmBatch G;
+    memset(&G, 0, sizeof(G));
+    bool encoder = false;
+    for (int i = 0; i < n; ++i) {
+        const GemmDesc &d = descs[i];
+        if (d.Mr == 0 || d.Nc == 0) continue;     // nothing to do for this one
+        if (!encoder) {
+            if (tmap_encoder_ready() != cudaSuccess) return LB_ERR_UNSUPPORTED;
+            encoder = true;
+        }
+        GemmProb &P = G.p[G.n];
+        if (!tmap_encode_2d(&P.mA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, d.A, d.Mr, d.Kc, (long)d.lda * 2, 64, kGBK) ||
+            !tmap_encode_2d(&P.mB, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, d.B, d.Nc, d.Kc, (long)d.ldb * 2, 64, kGBK) ||
+            !tmap_encode_2d(&P.mD, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d.D, d.Nc, d.Mr, (long)d.ldd * 4, 32, 32))
+            return LB_ERR_INVALID_ARG;
+        P.alpha = d.alpha;
+        P.Kc = d.Kc;
+        P.Mr = d.Mr;
+        P.Nc = d.Nc;
+        P.ntj = (d.Nc + kGBN - 1) / kGBN;
+        P.nkb = (d.Kc + kGBK - 1) / kGBK;
+        P.tile0 = G.ntiles;
+        const long tiles = (long)((d.Mr + kGBM - 1) / kGBM) * P.ntj;
+        if (G.ntiles + tiles > (1L << 30)) return LB_ERR_UNSUPPORTED;
+        G.ntiles += (int)tiles;
+        ++G.n;
+    }
+    if (G.n == 0) return LB_OK;
     cudaError_t e = ensure_dyn_smem((const void *)gemm_at_b_kernel, kGemmSmemBytes);
     if (e != cudaSuccess) return status_from(e);
     int sms = 0;
     if ((e = sm_count_of_current(&sms)) != cudaSuccess) return status_from(e);
-    const long ntiles = (long)((Mr + kGBM - 1) / kGBM) * ((Nc + kGBN - 1) / kGBN);
-    const int grid = (int)std::min<long>(ntiles, sms);
-    gemm_at_b_kernel<<<grid, kGThreads, kGemmSmemBytes, s>>>(mA, mB, mD, Kc, Mr, Nc, alpha, err);
+    const int grid = std::min(G.ntiles, sms);
+    gemm_at_b_kernel<<<grid, kGThreads, kGemmSmemBytes, s>>>(G, err);
     return status_from(cudaGetLastError());
+}
+
+lb_status gemm_at_b(const void *A, int lda, const void *B, int ldb, float *D, int ldd, int Kc, int Mr, int Nc,
+                    const float *alpha, int *err, cudaStream_t s)
+{
+    const GemmDesc d{A, lda, B, ldb, D, ldd, Kc, Mr, Nc, alpha};
+    if (!err) return LB_ERR_INVALID_ARG;
+    return gemm_at_b_batch(&d, 1, err, s);
 }
 
 }  // namespace lb

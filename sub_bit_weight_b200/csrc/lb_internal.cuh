@@ -56,8 +56,8 @@ constexpr int kP2Stages = 2;            // per-warp bulk-copy ring depth, contra
 // k-range).  The ranges are built with the plan, cost-balanced over all warps.
 constexpr int kLdgWarps = 16;           // warps per CTA (one CTA per SM)
 constexpr int kLdgRing = 6;             // k-block pairs in flight per stream
-constexpr int kPairMaxKB2 = 64;         // largest contraction-2 depth (k-blocks) these kernels take (r = 1024, 2 paths)
-constexpr int kPairMeta2 = 144;         // bytes of zmeta a contraction-2 stage carries (p * 16 + m, m < 2)
+constexpr int kPairMaxKB2 = 2 * LB_MAX_RANK / 32;   // contraction-2 depth (k-blocks) of the largest layer: every
+                                                    // depth (deep units take the generic loop, B from L2)
 
 // doubles in the accumulator block of a layer's scratch
 __host__ __device__ inline size_t acc_doubles(int R1) { return (size_t)R1 * 16 + 32 + 16; }
@@ -176,6 +176,17 @@ lb_status status_from(cudaError_t e);
 // D = alpha A^T B on the tensor cores (fp16 in, fp32 out); arguments as lb_gemm_at_b in littlebit_backward.h
 lb_status gemm_at_b(const void *A, int lda, const void *B, int ldb, float *D, int ldd, int Kc, int Mr, int Nc,
                     const float *alpha, int *err, cudaStream_t s);
+// Several such products (at most two) in one launch, their tiles dealt as one list.
+struct GemmDesc {
+    const void *A;
+    int lda;
+    const void *B;
+    int ldb;
+    float *D;
+    int ldd, Kc, Mr, Nc;
+    const float *alpha;
+};
+lb_status gemm_at_b_batch(const GemmDesc *descs, int n, int *err, cudaStream_t s);
 // Raise the dynamic shared-memory limit of kernel `fn` on the current device to at least `bytes` (never lowers
 // it; per device and kernel, thread-safe).
 cudaError_t ensure_dyn_smem(const void *fn, size_t bytes);

@@ -46,7 +46,9 @@ SHAPES = [
     (100, 70, 5, 2), (64, 64, 16, 1), (1, 1, 1, 2), (257, 1000, 33, 2), (130, 2050, 80, 2),
     (1024, 8192, 32, 2), (65, 33, 800, 2), (700, 3000, 184, 2), (96, 4100, 304, 1),
     (100, 300, 1024, 2),   # contraction-2 depth 64 k-blocks: the deepest the one/two-row kernels take
-    (80, 200, 1030, 2),    # one k-block deeper: the general kernels
+    (80, 200, 1030, 2),    # deeper than 64 k-blocks (generic streaming loop at one or two rows)
+    (72, 520, 2048, 2),    # the largest rank, both paths: 128 k-blocks; at 3..16 rows deeper than the general
+                           # kernels' shared memory, so the streaming kernels run once per pair of rows
 ]
 
 
@@ -165,3 +167,24 @@ def test_stack_matches_single_layer_calls(env, M):
         seed = 20 if i == 3 else 20 + i
         ref = oracle.forward(synth.activations(30 + i, i, M, s.K), oracle_layer(seed, 0 if i == 3 else i, s))
         assert rel_err(ys[i].cpu().numpy(), ref) <= TOL
+
+
+@pytest.mark.parametrize("M", [3, 4, 16])
+def test_stack_deeper_than_the_general_kernels(env, M):
+    """A stack holding a two-path r = 2048 layer (128 contraction-2 k-blocks) at 3..16 rows runs the streaming
+    kernels once per pair of rows (4 launches per pair); every layer, deep or shallow, still matches the oracle and
+    the single-layer call, and the row pairs' outputs land in the right rows (ragged M = 3: a last single row)."""
+    torch, lib, stacks = env
+    shapes = [synth.LayerShape("d", 136, 264, 2048), synth.LayerShape("s", 200, 96, 24)]
+    layers = [stacks.build_layer(40 + i, i, s) for i, s in enumerate(shapes)]
+    S = lib.lb_stack_create(layers)
+    xs = [stacks.bf16_on_device(synth.activations(50 + i, i, M, s.K), "cuda") for i, s in enumerate(shapes)]
+    ys = [torch.empty((M, s.N), dtype=torch.float32, device="cuda") for s in shapes]
+    lib.lb_stack_forward(S, xs, ys)
+    assert lib.lb_last_launch_count() == 4 * ((M + 1) // 2)
+    for i, s in enumerate(shapes):
+        single = lib.lb_linear_forward(xs[i], layers[i])
+        torch.cuda.synchronize()
+        ref = oracle.forward(synth.activations(50 + i, i, M, s.K), oracle_layer(40 + i, i, s))
+        assert rel_err(ys[i].cpu().numpy(), ref) <= TOL
+        assert rel_err(single.cpu().numpy(), ref) <= TOL
