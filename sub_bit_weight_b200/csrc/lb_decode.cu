@@ -578,10 +578,12 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
     const size_t smem2 = (size_t)(kDecodeThreads / 32) * kP2Stages * ((kb2max + 1) & ~1) * 256 +
                          (size_t)NT * kb2max * 32 * sizeof(uint2);
     // a stack deeper than the general kernels' shared memory holds runs on the one/two-row streaming kernels
-    // (no shared-memory bound on the depth), once per pair of activation rows
-    const bool by_pairs = M > 2 && smem2 > 227 * 1024;
+    // (no shared-memory bound on the depth), once per pair of activation rows; the general kernels are set up
+    // only where they fit
+    const bool general_fits = smem2 <= 227 * 1024;
+    const bool by_pairs = M > 2 && !general_fits;
     int occ1 = 1, occ2 = 1;
-    if (!by_pairs) {
+    if (general_fits) {
         if ((e = ensure_dyn_smem((const void *)k1, smem1)) != cudaSuccess) return status_from(e);
         if ((e = ensure_dyn_smem((const void *)k2, smem2)) != cudaSuccess) return status_from(e);
         if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, k1, kDecodeThreads, smem1)) != cudaSuccess)
@@ -622,8 +624,8 @@ lb_status decode_forward(const Plan &Pc, const uint16_t *const *xs, float *const
             lb_status st = decode_pair_launch(P.dev, cnt, P.p1 + P.p1_start[b], n1, P, b, io, base, M, kb2max, P.rmax,
                                               P.err, s, launches, true);
             if (st == LB_OK) continue;
-            if (st != LB_ERR_UNSUPPORTED) return st;
-            // shapes the streaming kernels cannot hold in shared memory take the general kernels
+            if (st != LB_ERR_UNSUPPORTED || !general_fits) return st;
+            // a shape the streaming kernels do not take runs on the general kernels
         }
         const int grid1 = std::max(1, std::min(n1, sms * occ1));
         const int grid2 = std::max(1, std::min(n2, sms * occ2));

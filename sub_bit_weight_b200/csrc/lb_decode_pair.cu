@@ -602,9 +602,11 @@ static __device__ __noinline__ void c2_generic(const LayerDev *__restrict__ laye
 // without a static path take the generic loops above.
 // ---------------------------------------------------------------------------
 
-// 16 pairs of zeros: the weights of a unit past a segment's end or the warp's range (a unit has at most 16
+// The largest unit of a static path: 2H pairs of k-blocks (contraction 2, H = 13).
+constexpr int kStaticMaxPairs = 26;
+// Zeros: the weights of a unit past a segment's end or the warp's range (a unit has at most kStaticMaxPairs
 // pairs), so that each ring load is one address plus an immediate offset.
-static __device__ __align__(16) uint4 g_zero_unit[16 * 32];
+static __device__ __align__(16) uint4 g_zero_unit[kStaticMaxPairs * 32];
 
 // A cursor over a warp's segments in blocks of U units, with this lane's address of each unit's first pair.
 static __device__ __forceinline__ const uint4 *seg_a(const Seg1 &x) { return x.v; }
@@ -677,7 +679,8 @@ static __device__ __forceinline__ void fetch_ahead(const BlockCur<Seg, U> &cur, 
 // B fragments of the static paths live in the warp's shared-memory slot: 2H pairs of 16 MM lanes, copied from
 // global memory (through L2: the previous kernel wrote them) whenever the warp enters a segment; where the units
 // have only 2H - 1 pairs, the last pair of the slot is zero, so stream 1's extra load counts for nothing.
-constexpr int kSlotPairs = 16;      // the largest 2H of a static path
+constexpr int kSlotPairs1 = kP1ChunkKB / 2;     // contraction 1: one 1024-input chunk
+constexpr int kSlotPairs2 = kStaticMaxPairs;    // contraction 2: the deepest static unit
 
 static __device__ __forceinline__ uint4 lds128(uint32_t addr)
 {
@@ -691,16 +694,18 @@ static __device__ __forceinline__ void sts128(uint32_t addr, uint4 v)
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
 }
-// Each warp owns kSlotRegion bytes: one slot of two-row fragments, or two slots of one-row fragments (contraction
-// 1 fetches the next segment's fragments into the second while the first is read).
-constexpr uint32_t kSlotBytes1 = kSlotPairs * 16 * 16;      // one slot, one activation row
-constexpr uint32_t kSlotRegion = 2 * kSlotBytes1;
+// Each warp owns a region of the CTA's shared memory.  Contraction 1: one slot of two-row fragments, or two slots
+// of one-row fragments (the next segment's fragments are fetched into the second while the first is read).
+// Contraction 2: one slot of kSlotPairs2 pairs.
+constexpr uint32_t kSlotBytes1 = kSlotPairs1 * 16 * 16;      // one contraction-1 slot, one activation row
+constexpr uint32_t kRegion1 = 2 * kSlotBytes1;
 template <int MM>
-static __device__ __forceinline__ uint32_t b_slot(int warp)
+__host__ __device__ constexpr uint32_t region2() { return kSlotPairs2 * 16 * MM * 16; }
+template <int MM>
+static __device__ __forceinline__ uint32_t b_slot(int warp, uint32_t region)
 {
-    static_assert(kSlotPairs * 16 * MM * 16 <= kSlotRegion, "slot region");
     extern __shared__ __align__(16) unsigned char sm_raw[];
-    return sm_addr(sm_raw) + (uint32_t)warp * kSlotRegion;
+    return sm_addr(sm_raw) + (uint32_t)warp * region;
 }
 
 // 16-byte asynchronous copy global -> shared through L2 (data of the previous launch: never the read-only path)
@@ -750,7 +755,8 @@ static __device__ __noinline__ void c1_static(const LayerDev *__restrict__ layer
 
     dep_wait();     // B fragments, exponents and cleared accumulators come from the previous kernels
 
-    const uint32_t slot = b_slot<MM>(warp);
+    static_assert(2 * H <= kSlotPairs1 && kSlotPairs1 * 16 * MM * 16 <= kRegion1, "contraction-1 slot");
+    const uint32_t slot = b_slot<MM>(warp, kRegion1);
     uint32_t bsl = slot + blane * 16;
     double *acc = nullptr;
     int npaths = 1, r16 = 0;
@@ -865,7 +871,8 @@ static __device__ __noinline__ void c2_static(const LayerDev *__restrict__ layer
 
     dep_wait();     // the zl fragments and their exponents come from the finish kernel
 
-    const uint32_t slot = b_slot<MM>(warp), bsl = slot + blane * 16;
+    static_assert(2 * H <= kSlotPairs2, "contraction-2 slot");
+    const uint32_t slot = b_slot<MM>(warp, region2<MM>()), bsl = slot + blane * 16;
     int N = 0;
     float *ym = nullptr;
     float my_sc = 0.0f, my_q = 0.0f;
@@ -945,6 +952,7 @@ __global__ void __launch_bounds__(kLdgWarps * 32, 1)
     if (s0 >= s1) return;
     const uint64_t pol = l2_evict_first();
     switch (cls[gw]) {
+    case 6: c1_static<MM, 6, 2, 4>(layers, segs, s0, s1, M, lane, threadIdx.x >> 5, pol); break;
     case 8: c1_static<MM, 8, 1, 4>(layers, segs, s0, s1, M, lane, threadIdx.x >> 5, pol); break;
     default: c1_generic<MM>(layers, segs, s0, s1, M, lane, pol); break;
     }
@@ -969,6 +977,8 @@ __global__ void __launch_bounds__(kLdgWarps * 32, 1)
     case 4: c2_static<MM, 4, 3, 6>(layers, segs, s0, s1, io, base, M, lane, threadIdx.x >> 5, pol); break;
     case 5: c2_static<MM, 5, 1, 5>(layers, segs, s0, s1, io, base, M, lane, threadIdx.x >> 5, pol); break;
     case 6: c2_static<MM, 6, 1, 6>(layers, segs, s0, s1, io, base, M, lane, threadIdx.x >> 5, pol); break;
+    case 9: c2_static<MM, 9, 2, 6>(layers, segs, s0, s1, io, base, M, lane, threadIdx.x >> 5, pol); break;
+    case 13: c2_static<MM, 13, 5, 5>(layers, segs, s0, s1, io, base, M, lane, threadIdx.x >> 5, pol); break;
     default: c2_generic<MM>(layers, segs, s0, s1, io, base, M, lane, pol); break;
     }
 }
@@ -1017,11 +1027,11 @@ static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P
     // the three kernels after the quantisation may each start while the previous one drains,
     // unless timing events separate the launches
     const bool pdl = !profiling_active();
-    const size_t slots = (size_t)kLdgWarps * kSlotRegion;    // each warp's B slots
-    if ((e = ensure_dyn_smem((const void *)contraction1_ldg_kernel<MM>, slots)) != cudaSuccess ||
-        (e = ensure_dyn_smem((const void *)contraction2_ldg_kernel<MM>, slots)) != cudaSuccess)
+    const size_t slots1 = (size_t)kLdgWarps * kRegion1, slots2 = (size_t)kLdgWarps * region2<MM>();   // B slots
+    if ((e = ensure_dyn_smem((const void *)contraction1_ldg_kernel<MM>, slots1)) != cudaSuccess ||
+        (e = ensure_dyn_smem((const void *)contraction2_ldg_kernel<MM>, slots2)) != cudaSuccess)
         return status_from(e);
-    if ((e = launch_dependent(pdl, contraction1_ldg_kernel<MM>, dim3(G), dim3(kLdgWarps * 32), slots, s, dev_layers,
+    if ((e = launch_dependent(pdl, contraction1_ldg_kernel<MM>, dim3(G), dim3(kLdgWarps * 32), slots1, s, dev_layers,
                               (const Seg1 *)P.sg1, bnd1, cls1, M)) != cudaSuccess)
         return status_from(e);
     ++*launches;
@@ -1031,7 +1041,7 @@ static lb_status pair_launch_mm(const LayerDev *dev_layers, int nlayers, const P
         return status_from(e);
     ++*launches;
     if (mark) profile_mark(*launches, s);
-    if ((e = launch_dependent(pdl, contraction2_ldg_kernel<MM>, dim3(G), dim3(kLdgWarps * 32), slots, s, dev_layers,
+    if ((e = launch_dependent(pdl, contraction2_ldg_kernel<MM>, dim3(G), dim3(kLdgWarps * 32), slots2, s, dev_layers,
                               (const Seg2 *)P.sg2, bnd2, cls2, io, base, M)) != cudaSuccess)
         return status_from(e);
     ++*launches;

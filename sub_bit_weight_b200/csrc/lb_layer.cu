@@ -268,8 +268,11 @@ cudaError_t plan_build(Plan &P, const lb_layer *const *layers, int n, cudaStream
     // a unit: layer, linear index within the layer, pairs, cost (k-blocks plus the epilogue; the generic loop
     // runs slower per k-block)
     struct Unit { int layer, ul, P; double cost; };
-    auto class1 = [](int pairs) { const int H = (pairs + 1) / 2; return H == 8 ? H : 0; };
-    auto class2 = [](int pairs) { const int H = (pairs + 1) / 2; return (H >= 1 && H <= 6) ? H : 0; };
+    auto class1 = [](int pairs) { const int H = (pairs + 1) / 2; return (H == 6 || H == 8) ? H : 0; };
+    auto class2 = [](int pairs) {
+        const int H = (pairs + 1) / 2;
+        return ((H >= 1 && H <= 6) || H == 9 || H == 13) ? H : 0;
+    };
     // a unit's k-blocks plus its epilogue and block bookkeeping, in k-block equivalents (fitted to per-warp times
     // on B200); the generic loop runs about a third slower
     auto unit_cost = [](int pairs, int cls) { return (2.0 * pairs + 16.0) * (cls ? 1.0 : 1.35); };
