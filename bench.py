@@ -638,11 +638,12 @@ def run_configs(spec: str, steps: int, dev, pk: dict):
         w = synth.WORKLOADS[parts[0]]
         M = int(parts[1]) if len(parts) > 1 else w.Ms[0]
         flushed = len(parts) > 2 and parts[2] == "flushed"
-        res = run_gpu(w, M, steps, 5, None, dev, want_e2e=False, flush_l2=flushed)
+        res = run_gpu(w, M, steps, 5, None, dev, want_e2e=not flushed, flush_l2=flushed)
         shapes = res["shapes"]
         sb = sum(sum(layer_bytes(s, M)) for s in shapes)
         ms = res["total_ms"] / steps
         out.append({"workload": f"{w.key}: {w.title}", "M": M, "layers": len(shapes),
+                    "e2e": e2e_of(res, None, 1, sb, False, "lb_stack_forward from pinned host x to pinned host y"),
                     "l2": ("L2 flushed (256 MB write) before every step; steps timed alone" if flushed else
                            "inputs larger than L2" if sb > 126e6 else "stack fits in L2 (effective GB/s, warm)"),
                     "value": round(sb / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "higher_is_better": True,
