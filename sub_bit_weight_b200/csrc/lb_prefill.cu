@@ -21,7 +21,11 @@
 //   warps 4-7   epilogue: tcgen05.ld of the fp32 accumulator, scaling, stores
 //   warps 8-15  generators: B tile (256 x 64 fp16, 128-byte swizzle) from
 //               signs and scales; the latent GEMM also converts the bf16 A
-//               tile to fp16 in place
+//               tile to fp16 in place.  The output GEMM's sign bits arrive in
+//               the first 4 KB of the B stage they are expanded into, so its
+//               generators meet at a barrier (all bits read) before writing;
+//               the latent GEMM's arrive in its unused epilogue staging area
+//               and need none
 // Two accumulators of 256 columns in tensor memory let the epilogue of one
 // tile overlap the main loop of the next.  Every wait is bounded: on timeout
 // the kernel records an error code and returns.
@@ -211,10 +215,12 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v)
 // ---------------------------------------------------------------------------
 // The tensor-core contraction kernel
 // ---------------------------------------------------------------------------
+static_assert(kPfStages == 4, "the latent GEMM keeps one stage's sign bits in each of the four staging blocks");
 struct PfSmem {
     alignas(1024) unsigned char A[kPfStages][kPfBM * kPfBK * 2];
     alignas(1024) unsigned char B[kPfStages][kPfBN * kPfBK * 2];   // the stage's sign bits land in its first 4 KB
-    alignas(1024) unsigned char ST[4][32 * 128];  // output GEMM epilogue: 32x32 fp32 block per warp (128B swizzle)
+    alignas(1024) unsigned char ST[4][32 * 128];  // output GEMM epilogue: 32x32 fp32 block per warp (128B swizzle);
+                                                  // latent GEMM: the sign bits of stage s (4 KB) in ST[s]
     alignas(16) __half gst[kPfStages][128];     // latent GEMM: g of both paths for the stage's k-block
     alignas(16) float lsc[kPfBN];               // latent GEMM epilogue: l of the tile's columns
     uint64_t full[kPfStages], ready[kPfStages], empty[kPfStages], bread[kPfStages];
@@ -241,7 +247,7 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
         for (int s = 0; s < kPfStages; ++s) {
             mbar_init(&S.full[s], 1);
             mbar_init(&S.ready[s], MODE == 0 ? 10 + kPfExtraConv : 8);   // generator warps (+ converter warps)
-            mbar_init(&S.bread[s], 8);                    // generator warps have read the stage's sign bits
+            mbar_init(&S.bread[s], 8);                    // output GEMM: generator warps have read the stage's bits
             mbar_init(&S.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -297,7 +303,9 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
                     if (!mbar_wait(&S.empty[s], ph ^ 1, abort, err, 1)) break;
                     mbar_expect_tx(&S.full[s], kPfBM * kPfBK * 2 + 4096 + (MODE == 0 ? 256 : 0));
                     tma_load_2d(S.A[s], ly.tmA, kb * kPfBK, mt * kPfBM, &S.full[s]);
-                    bulk_load(S.B[s], bits + (size_t)kb * 1024, 4096, &S.full[s]);
+                    // latent GEMM: the sign bits go to the (otherwise unused) staging area, so the generators
+                    // overwrite nothing they still read; output GEMM: the first 4 KB of the B stage
+                    bulk_load(MODE == 0 ? (void *)S.ST[s] : (void *)S.B[s], bits + (size_t)kb * 1024, 4096, &S.full[s]);
                     if (MODE == 0) bulk_load(S.gst[s], ly.base + (size_t)kb * 128, 256, &S.full[s]);
                     pend |= 1u << s;
                     pend_ph = (pend_ph & ~(1u << s)) | (ph << s);
@@ -510,22 +518,17 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
                     ok = false;
                     break;
                 }
-                const uint32_t Bt = smem_u32(S.B[s]);   // sign bits first: [256 rows][4 words]
+                const uint32_t Bt = smem_u32(S.B[s]);   // output GEMM: sign bits first: [256 rows][4 words]
                 if (MODE == 0) {
-                    // thread -> chunk c (8 inputs), rows gt/8 + 32 i
+                    // thread -> chunk c (8 inputs), rows gt/8 + 32 i; the bits sit apart from B (no barrier)
+                    const uint32_t Bits = smem_u32(S.ST[s]);
                     const int c = gt & 7;
                     uint32_t R[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) R[i] = lds32(Bt + 4u * (((gt >> 3) + 32 * i) * 4 + (c >> 1)));
+                    for (int i = 0; i < 8; ++i) R[i] = lds32(Bits + 4u * (((gt >> 3) + 32 * i) * 4 + (c >> 1)));
                     uint4 gb[2];
 #pragma unroll
                     for (int p = 0; p < 2; ++p) gb[p] = lds128(smem_u32(S.gst[s] + p * 64 + 8 * c));
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&S.bread[s]);
-                    if (!mbar_wait(&S.bread[s], ph, abort, err, 8)) {   // every generator has its bits
-                        ok = false;
-                        break;
-                    }
                     const int sh0 = 4 * (c & 1);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
