@@ -22,10 +22,10 @@
 //   warps 8-15  generators: B tile (256 x 64 fp16, 128-byte swizzle) from
 //               signs and scales; the latent GEMM also converts the bf16 A
 //               tile to fp16 in place.  The output GEMM's sign bits arrive in
-//               the first 4 KB of the B stage they are expanded into, so its
-//               generators meet at a barrier (all bits read) before writing;
-//               the latent GEMM's arrive in its unused epilogue staging area
-//               and need none
+//               the first 4 KB of the B stage they are expanded into, so the
+//               generator warp that writes those rows waits until every
+//               generator has read its bits; the latent GEMM's arrive in its
+//               unused epilogue staging area and need no wait
 // Two accumulators of 256 columns in tensor memory let the epilogue of one
 // tile overlap the main loop of the next.  Every wait is bounded: on timeout
 // the kernel records an error code and returns.
@@ -545,12 +545,13 @@ __global__ void __launch_bounds__(pf_threads(MODE), 1)
                         }
                     }
                 } else {
-                    // thread -> row gt, all 8 chunks
+                    // thread -> row gt, all 8 chunks.  The bits sit in B rows 0..31: only the warp that writes
+                    // those rows waits until every generator has read its bits
                     const int row = gt;
                     const uint4 Rw = lds128(Bt + 16u * row);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.bread[s]);
-                    if (!mbar_wait(&S.bread[s], ph, abort, err, 8)) {   // every generator has its bits
+                    if (gw == 0 && !mbar_wait(&S.bread[s], ph, abort, err, 8)) {
                         ok = false;
                         break;
                     }
