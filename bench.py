@@ -420,9 +420,7 @@ def roofline_of(res: dict, shapes, M: int, prefill: bool, pk: dict, wkey: str):
     if not res["per_launch"]:
         return None
     if prefill:
-        # (activation conversion,) latent GEMM, output GEMM
-        conv_ms = res["per_launch"][0] if len(res["per_launch"]) == 3 else None
-        k1ms, k2ms = res["per_launch"][-2:]
+        k1ms, k2ms = res["per_launch"][:2]
         dom = 1 if k2ms >= k1ms else 0
         f1 = sum(2.0 * M * 2 * s.r * s.K for s in shapes)
         f2 = sum(2.0 * M * 2 * s.r * s.N for s in shapes)
@@ -435,8 +433,7 @@ def roofline_of(res: dict, shapes, M: int, prefill: bool, pk: dict, wkey: str):
                 "peak_src": pk["src"] + " bf16 burst (dense 16-bit tensor peak; the kernel is timed alone)",
                 "frac_of_sustained": round(ach / pk["bf16_tflops_sustained"], 4),
                 "traffic": measured_traffic(kname, wkey),
-                "per_kernel_ms": dict(([("x_to_f16", round(conv_ms, 4))] if conv_ms is not None else []) +
-                                      [("latent", round(k1ms, 4)), ("output", round(k2ms, 4))]),
+                "per_kernel_ms": {"latent": round(k1ms, 4), "output": round(k2ms, 4)},
                 "per_kernel_flops": {"latent": f1, "output": f2},
                 "per_kernel_tflops": {"latent": round(f1 / (k1ms * 1e-3) / 1e12, 1),
                                       "output": round(f2 / (k2ms * 1e-3) / 1e12, 1)}}
