@@ -74,6 +74,14 @@ int main(void)
     CHECK(lb_backward_create(&B, 64, 64, 8, 3, cu1, cu1, ch1, ch1, ch1, NULL) == LB_ERR_UNSUPPORTED);
     CHECK(lb_backward_create(&B, 64, 60, 8, 1, cu1, cu1, ch1, ch1, ch1, NULL) == LB_ERR_UNSUPPORTED);
     lb_backward_destroy(NULL);
+    /* its dense-product GEMM: argument checks happen before any device work */
+    const uint16_t *h16 = (const uint16_t *)dev;
+    float *f32 = (float *)dev;
+    CHECK(lb_gemm_at_b(NULL, 64, h16, 64, f32, 64, 8, 64, 64, (const float *)dev, (int *)dev, NULL) ==
+          LB_ERR_INVALID_ARG);
+    CHECK(lb_gemm_at_b(h16, 64, h16, 48, f32, 48, 8, 64, 48, (const float *)dev, (int *)dev, NULL) ==
+          LB_ERR_UNSUPPORTED);
+    CHECK(lb_gemm_at_b(h16, 64, h16, 64, f32, 64, 8, 0, 64, (const float *)dev, (int *)dev, NULL) == LB_OK);
 
     printf(fails ? "FAILED (%d)\n" : "OK\n", fails);
     return fails != 0;
