@@ -143,3 +143,16 @@ def test_config_runs_cover_the_other_workloads():
     assert {("llama2_7b_0.55", m, False) for m in (1, 4, 16)} <= got
     for name, M, _ in got:
         assert M in synth.WORKLOADS[name].Ms
+
+
+def test_end_to_end_object():
+    """e2e is the same metric through the C-ABI call with host buffers: work over the pipelined step time, the serial
+    figure beside it, the bytes copied each way as measured; absent when the run measured none."""
+    res = {"e2e": {"ms": 0.5, "serial_ms": 1.0, "h2d": 1000, "d2h": 4000, "steps": 10}}
+    e = bench.e2e_of(res, None, 1, 896.0e6, False, "how")
+    assert e["unit"] == "GB/s" and e["value"] == pytest.approx(896.0e6 / 0.5e-3 / 1e9, abs=0.01)
+    assert e["serial"]["value"] == pytest.approx(896.0e6 / 1.0e-3 / 1e9, abs=0.01)
+    assert (e["h2d_bytes_per_step"], e["d2h_bytes_per_step"]) == (1000, 4000)
+    p = bench.e2e_of(res, None, 1, 0.376e12, True, "how")
+    assert p["unit"] == "TFLOP/s" and p["value"] == pytest.approx(0.376e12 / 0.5e-3 / 1e12, abs=0.01)
+    assert bench.e2e_of({"e2e": None}, None, 1, 1.0, False, "how") is None
